@@ -1,0 +1,401 @@
+"""Pins for the CPU oracle: checks against values fixed by the pages or by
+mathematics, never by the oracle itself.
+
+Each ``pin_*`` function takes the oracle module (the real one, or a variant
+built from a source with a planted mistake) and raises AssertionError when the
+oracle disagrees with the pin.  ``tests/test_oracle_pins.py`` runs them on the
+real oracle; ``tests/test_oracle_mutants.py`` checks that every planted mistake
+fails at least one of them.
+
+Independent references used here (none calls the oracle's arithmetic):
+* the E2M1 magnitudes from the format's bit fields (1 sign, 2 exponent bits
+  with bias 1, 1 mantissa bit);
+* nearest-value search over that grid in double, ties to the even code;
+* ``numpy.quantile(..., method="inverted_cdf")``, ``numpy.sort`` and a brute
+  force count for the threshold;
+* ``scipy.sparse`` for the CSR of dA and for dA * W;
+* integer matrix products (numpy int64) for the FP4 accumulator;
+* closed forms: matrices already on the scaled grid quantize to themselves;
+* invariants: A_clamped + dA == A, |A_clamped| <= T, the nnz bound, each
+  non-zero row carries a code of magnitude 6, the rounding error bound.
+"""
+from __future__ import annotations
+
+import json
+import os
+
+import numpy as np
+import scipy.sparse as sp
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden",
+                      "worked_examples.json")
+
+
+def golden():
+    with open(GOLDEN) as f:
+        return json.load(f)
+
+
+# ---------------------------------------------------------------- references
+def format_grid() -> np.ndarray:
+    """Value of each 4-bit code from the E2M1 bit fields (bias 1)."""
+    out = np.empty(16)
+    for c in range(16):
+        s, e, m = c >> 3, (c >> 1) & 3, c & 1
+        mag = 0.5 * m if e == 0 else 2.0 ** (e - 1) * (1.0 + 0.5 * m)
+        out[c] = -mag if s else mag
+    return out
+
+
+def ref_encode(x) -> np.ndarray:
+    """Nearest grid value by exhaustive distance search, ties to the even code."""
+    x = np.asarray(x, dtype=np.float32).reshape(-1)
+    grid = format_grid()[:8]
+    mag = np.abs(x.astype(np.float64))
+    d = np.abs(mag[:, None] - grid[None, :])
+    best = d.min(axis=1, keepdims=True)
+    is_best = d == best
+    # prefer even codes among equally near neighbours
+    pref = np.where(is_best, np.where(np.arange(8) % 2 == 0, 2, 1), 0)
+    code = np.argmax(pref, axis=1).astype(np.uint8)
+    # above the largest grid value the nearest one is 6 (distances of huge
+    # magnitudes all round to the same double, so decide these directly)
+    code = np.where(mag > grid[-1], np.uint8(7), code).astype(np.uint8)
+    sign = np.signbit(x).astype(np.uint8) << 3
+    return code | sign
+
+
+def pack(codes_unpacked) -> np.ndarray:
+    c = np.asarray(codes_unpacked, dtype=np.uint8)
+    return (c[..., 0::2] | (c[..., 1::2] << 4)).astype(np.uint8)
+
+
+def unpack(packed) -> np.ndarray:
+    p = np.asarray(packed, dtype=np.uint8)
+    out = np.empty(p.shape[:-1] + (2 * p.shape[-1],), dtype=np.uint8)
+    out[..., 0::2] = p & 15
+    out[..., 1::2] = p >> 4
+    return out
+
+
+def encoder_probe_inputs(rng) -> np.ndarray:
+    """Every bf16 value, dense fp32 neighbourhoods of grid points and
+    midpoints, special values and random fp32 bit patterns (no NaN)."""
+    bf = (np.arange(1 << 16, dtype=np.uint32) << 16).view(np.float32)
+    grid = format_grid()[:8]
+    mids = 0.5 * (grid[:-1] + grid[1:])
+    centres = np.concatenate([grid, mids]).astype(np.float32)
+    neigh = [centres]
+    up = centres.copy()
+    dn = centres.copy()
+    for _ in range(64):
+        up = np.nextafter(up, np.float32(np.inf))
+        dn = np.nextafter(dn, np.float32(-np.inf))
+        neigh += [up.copy(), dn.copy()]
+    neigh = np.concatenate(neigh)
+    specials = np.array([0.0, np.inf, np.finfo(np.float32).max, np.finfo(np.float32).tiny,
+                         1e-45, 6.0, 6.5, 7.0, 12.0, 1e38], dtype=np.float32)
+    rnd = rng.integers(0, 1 << 32, size=1 << 20, dtype=np.uint64).astype(np.uint32).view(
+        np.float32)
+    xs = np.concatenate([bf, neigh, -neigh, specials, -specials, rnd])
+    return xs[~np.isnan(xs)]
+
+
+# ------------------------------------------------------------------- pins
+def pin_grid(orc):
+    g = golden()["e2m1_grid"]
+    vals = orc.e2m1_values()
+    assert np.array_equal(vals, format_grid())
+    assert np.array_equal(vals, np.array(g["values"]))
+    assert np.array_equal(np.signbit(vals), np.signbit(np.array(g["values"])))
+
+
+def pin_encoder_ties(orc):
+    g = golden()["e2m1_ties"]
+    got = orc.e2m1_encode(np.array(g["inputs"], dtype=np.float32))
+    assert got.tolist() == g["codes"], (got.tolist(), g["codes"])
+
+
+def pin_encoder_nearest_search(orc, seed=1):
+    xs = encoder_probe_inputs(np.random.default_rng(seed))
+    got = orc.e2m1_encode(xs)
+    want = ref_encode(xs)
+    bad = np.nonzero(got != want)[0]
+    assert bad.size == 0, (xs[bad[:8]], got[bad[:8]], want[bad[:8]])
+
+
+def pin_row_worked_example(orc):
+    g = golden()["row_quantization"]
+    codes, s = orc.quantize_rows(np.array([g["row"]], dtype=np.float32))
+    assert codes[0].tolist() == g["codes_packed"]
+    assert unpack(codes)[0].tolist() == g["codes_unpacked"]
+    assert float(s[0]) == g["scale"]
+    dq = orc.dequant_rows(codes, s)[0]
+    assert dq.tolist() == g["dequant"]
+
+
+def pin_col_worked_example(orc):
+    g = golden()["column_quantization"]
+    W = np.array(g["W"], dtype=np.float32)
+    codesT, t = orc.quantize_cols(W)
+    assert codesT.tolist() == g["codesT_packed"]
+    assert t.tolist() == g["scales"]
+
+
+def pin_threshold_worked_example(orc):
+    g = golden()["threshold_clamp"]
+    A = np.array(g["A"], dtype=np.float32)
+    for case in g["cases"]:
+        assert orc.quantile_rank(case["alpha"], A.size) == case["k"]
+        T = orc.threshold(A, case["alpha"])
+        assert T == case["T"]
+        a_c, rp, col, val = orc.clamp_compensate(A, T)
+        assert rp.tolist() == case["row_ptr"]
+        assert col.tolist() == case["col"]
+        assert val.tolist() == case["val"]
+        assert a_c.tolist() == case["A_clamped"]
+
+
+def pin_act_worked_example(orc):
+    g = golden()["act_quantization"]
+    out = orc.quantize_act(np.array(g["A"], dtype=np.float32), g["alpha"])
+    assert out["T"] == g["T"]
+    assert out["codes"].tolist() == g["codes_packed"]
+    assert unpack(out["codes"]).tolist() == g["codes_unpacked"]
+    assert out["scales"].tolist() == g["scales"]
+    assert out["row_ptr"].tolist() == g["row_ptr"]
+    assert out["col"].tolist() == g["col"]
+    assert out["val"].tolist() == g["val"]
+
+
+def pin_gemm_worked_example(orc):
+    g = golden()["gemm"]
+    acc = orc.gemm_acc(np.array(g["codesA_packed"], np.uint8),
+                       np.array(g["codesWT_packed"], np.uint8), g["K"])
+    assert acc.tolist() == g["acc"]
+
+
+def _threshold_cases(rng):
+    cases = []
+    for n in (1, 2, 3, 7, 10, 64, 1000, 4097):
+        cases.append(rng.standard_normal(n).astype(np.float32))
+    # heavy tail with many ties (values rounded to 8 mantissa bits, like bf16)
+    t = rng.standard_t(3, size=20000).astype(np.float32)
+    cases.append((t.view(np.uint32) & np.uint32(0xFFFF0000)).view(np.float32))
+    cases.append(np.zeros(50, np.float32))
+    cases.append(np.array([3.0, -3.0, 3.0, 0.0, -0.0], np.float32))
+    return cases
+
+
+def pin_threshold_vs_sort_and_quantile(orc, seed=2):
+    rng = np.random.default_rng(seed)
+    for a in _threshold_cases(rng):
+        mag = np.sort(np.abs(a.astype(np.float64)))
+        n = a.size
+        for alpha in (1e-9, 0.1, 0.5, 0.9, 0.99, 0.999, 0.9999, 1.0):
+            T = orc.threshold(a.reshape(1, -1), alpha)
+            # brute force over the definition: the smallest |a| such that at
+            # least ceil(alpha * n) entries are <= it
+            need = int(np.ceil(alpha * n))
+            need = min(max(need, 1), n)
+            if n <= 1000:
+                cands = [v for v in np.unique(mag) if np.count_nonzero(mag <= v) >= need]
+                assert T == min(cands), (n, alpha, T, min(cands))
+            assert T == mag[need - 1]
+            q = np.quantile(np.abs(a.astype(np.float64)), alpha, method="inverted_cdf")
+            assert T == q, (n, alpha, T, q)
+
+
+def pin_clamp_invariants(orc, seed=3):
+    rng = np.random.default_rng(seed)
+    for (M, K, alpha) in ((7, 33, 0.9), (16, 64, 0.99), (40, 128, 0.999), (5, 8, 0.5)):
+        A = (rng.standard_t(3, size=(M, K)) * 2).astype(np.float32)
+        T = orc.threshold(A, alpha)
+        a_c, rp, col, val = orc.clamp_compensate(A, T)
+        # A_c + dA == A exactly (fp64)
+        dA = sp.csr_matrix((val, col, rp), shape=(M, K)).toarray()
+        assert np.array_equal(a_c.astype(np.float64) + dA, A.astype(np.float64))
+        assert np.all(np.abs(a_c) <= T)
+        # dA is non-zero exactly where |a| > T, in canonical CSR order
+        mask = np.abs(A) > T
+        ref = sp.csr_matrix(np.where(mask, A.astype(np.float64) - np.sign(A) * T, 0.0))
+        ref.sort_indices()
+        assert rp.tolist() == ref.indptr.tolist()
+        assert col.tolist() == ref.indices.tolist()
+        assert np.array_equal(val, ref.data)
+        n = A.size
+        assert col.size <= n - int(np.ceil(alpha * n))
+        assert np.count_nonzero(np.abs(A) <= T) >= int(np.ceil(alpha * n))
+
+
+def _on_grid_matrix(rng, M, K, exps):
+    """Rows that are exactly on grid * 2^e with max magnitude 6 * 2^e."""
+    grid = format_grid()[:8]
+    codes = rng.integers(0, 8, size=(M, K))
+    codes[np.arange(M), rng.integers(0, K, size=M)] = 7
+    sign = np.where(rng.random((M, K)) < 0.5, -1.0, 1.0)
+    A = sign * grid[codes] * (2.0 ** exps)[:, None]
+    return A.astype(np.float32), codes, sign, exps
+
+
+def pin_quantize_rows_identity(orc, seed=4):
+    rng = np.random.default_rng(seed)
+    M, K = 33, 64
+    exps = rng.integers(-20, 20, size=M).astype(np.float64)
+    A, codes, sign, exps = _on_grid_matrix(rng, M, K, exps)
+    q, s = orc.quantize_rows(A)
+    want = (codes | np.where(sign < 0, 8, 0)).astype(np.uint8)
+    assert np.array_equal(unpack(q), want)
+    assert np.array_equal(s.astype(np.float64), 2.0 ** exps)
+
+
+def pin_quantize_rows_properties(orc, seed=5):
+    rng = np.random.default_rng(seed)
+    grid = format_grid()[:8]
+    for (M, K, scale) in ((9, 32, 1.0), (20, 256, 1e-3), (3, 1024, 1e4)):
+        A = (rng.standard_t(3, size=(M, K)) * scale).astype(np.float32)
+        q, s = orc.quantize_rows(A)
+        u = unpack(q)
+        amax = np.abs(A).max(axis=1)
+        assert np.array_equal(s, (amax / np.float32(6)).astype(np.float32))
+        # every non-zero row has a code of magnitude 6
+        assert np.all(np.any((u & 7) == 7, axis=1))
+        # the dequantized value is the nearest grid point of a*r, so the
+        # error is at most half the local grid gap times s (gap 2 above 4)
+        r = (np.float32(6) / amax).astype(np.float32)
+        x = (A * r[:, None]).astype(np.float32).astype(np.float64)
+        dq = orc.dequant_rows(q, s) / s.astype(np.float64)[:, None]
+        err = np.abs(np.abs(x) - np.abs(dq))
+        gap = np.where(np.abs(x) > 4, 1.0, np.where(np.abs(x) > 2, 0.5, 0.25))
+        assert np.all(err <= gap + 1e-6)
+        # monotone in a within each row, odd symmetric in sign
+        for i in range(M):
+            order = np.argsort(A[i], kind="stable")
+            v = orc.dequant_rows(q[i:i + 1], s[i:i + 1])[0][order]
+            assert np.all(np.diff(v) >= 0)
+        qn, sn = orc.quantize_rows(-A)
+        assert np.array_equal(qn, q ^ np.uint8(0x88)) and np.array_equal(sn, s)
+        assert set(np.unique(np.abs(orc.dequant_rows(q, s) / s[:, None]))) <= set(grid)
+
+
+def pin_quantize_degenerate_rows(orc):
+    A = np.zeros((4, 8), np.float32)
+    A[1, :] = -0.0
+    A[2, 3] = np.float32(1e-45)     # 6 / amax overflows fp32
+    A[3, :] = np.float32(-1e-45)
+    q, s = orc.quantize_rows(A)
+    assert s.tolist() == [0.0, 0.0, 0.0, 0.0]
+    assert unpack(q)[0].tolist() == [0] * 8
+    assert unpack(q)[1].tolist() == [8] * 8
+    assert unpack(q)[2].tolist() == [0] * 8
+    assert unpack(q)[3].tolist() == [8] * 8
+
+
+def pin_quantize_cols_transpose(orc, seed=6):
+    rng = np.random.default_rng(seed)
+    K, N = 64, 24
+    exps = rng.integers(-10, 10, size=N).astype(np.float64)
+    WT, codes, sign, exps = _on_grid_matrix(rng, N, K, exps)
+    qT, t = orc.quantize_cols(np.ascontiguousarray(WT.T))
+    want = (codes | np.where(sign < 0, 8, 0)).astype(np.uint8)
+    assert np.array_equal(unpack(qT), want)
+    assert np.array_equal(t.astype(np.float64), 2.0 ** exps)
+    W = (rng.standard_normal((K, N)) * 0.02).astype(np.float32)
+    qT, t = orc.quantize_cols(W)
+    assert np.array_equal(t, (np.abs(W).max(axis=0) / np.float32(6)).astype(np.float32))
+    assert np.all(np.any((unpack(qT) & 7) == 7, axis=1))
+
+
+def pin_gemm_vs_integer_matmul(orc, seed=7):
+    rng = np.random.default_rng(seed)
+    twice = (2 * format_grid()).astype(np.int64)   # integers
+    for (M, N, K) in ((5, 7, 32), (33, 17, 256), (8, 8, 4096)):
+        cA = rng.integers(0, 256, size=(M, K // 2), dtype=np.uint8)
+        cW = rng.integers(0, 256, size=(N, K // 2), dtype=np.uint8)
+        acc = orc.gemm_acc(cA, cW, K)
+        ia = twice[unpack(cA)]
+        iw = twice[unpack(cW)]
+        ref = (ia @ iw.T).astype(np.float64) / 4.0
+        assert np.array_equal(acc, ref)
+        rows = np.array([M - 1, 0, M // 2])
+        assert np.array_equal(orc.gemm_acc(cA, cW, K, rows=rows), ref[rows])
+
+
+def pin_spmm_vs_scipy(orc, seed=8):
+    rng = np.random.default_rng(seed)
+    M, K, N = 30, 64, 40
+    A = (rng.standard_t(3, size=(M, K))).astype(np.float32)
+    W = (rng.standard_normal((K, N)) * 0.02).astype(np.float32)
+    T = orc.threshold(A, 0.9)
+    _, rp, col, val = orc.clamp_compensate(A, T)
+    C = orc.spmm(rp, col, val, W)
+    ref = sp.csr_matrix((val, col, rp), shape=(M, K)) @ W.astype(np.float64)
+    assert np.allclose(C, ref, rtol=1e-13, atol=1e-15)
+
+
+def pin_linear_no_clamp_is_dequant_matmul(orc, seed=9):
+    rng = np.random.default_rng(seed)
+    M, K, N = 17, 128, 23
+    A = rng.standard_normal((M, K)).astype(np.float32)
+    W = (rng.standard_normal((K, N)) * 0.02).astype(np.float32)
+    act = orc.quantize_act(A, 1.0)
+    assert act["col"].size == 0
+    qT, t = orc.quantize_cols(W)
+    acc = orc.gemm_acc(act["codes"], qT, K)
+    Y = orc.linear_y(acc, act["scales"], t, act["row_ptr"], act["col"], act["val"], W)
+    ref = orc.dequant_rows(act["codes"], act["scales"]) @ orc.dequant_rows(qT, t).T
+    assert np.allclose(Y, ref, rtol=1e-12, atol=1e-14)
+
+
+def pin_linear_exact_on_grid(orc, seed=10):
+    """A and W already on the scaled grid, no clamp: Y == A @ W exactly, and
+    with a clamp Y == A @ W up to rounding (the correction restores A)."""
+    rng = np.random.default_rng(seed)
+    M, K, N = 12, 64, 10
+    A, *_ = _on_grid_matrix(rng, M, K, rng.integers(-3, 3, size=M).astype(np.float64))
+    WT, *_ = _on_grid_matrix(rng, N, K, rng.integers(-6, -2, size=N).astype(np.float64))
+    W = np.ascontiguousarray(WT.T)
+    exact = A.astype(np.float64) @ W.astype(np.float64)
+    act = orc.quantize_act(A, 1.0)
+    qT, t = orc.quantize_cols(W)
+    acc = orc.gemm_acc(act["codes"], qT, K)
+    Y = orc.linear_y(acc, act["scales"], t, act["row_ptr"], act["col"], act["val"], W)
+    assert np.array_equal(Y, exact)
+    # clamp on: Y = dq(A_c) W_q + dA W with W_q == W here; dq(A_c) differs
+    # from A_c, so compare with the pieces: dA W exactly restores A - A_c
+    act = orc.quantize_act(A, 0.9)
+    assert act["col"].size > 0
+    acc = orc.gemm_acc(act["codes"], qT, K)
+    Y = orc.linear_y(acc, act["scales"], t, act["row_ptr"], act["col"], act["val"], W)
+    dA = sp.csr_matrix((act["val"], act["col"], act["row_ptr"]), shape=(M, K)).toarray()
+    ref = orc.dequant_rows(act["codes"], act["scales"]) @ W.astype(np.float64) + dA @ W
+    assert np.allclose(Y, ref, rtol=1e-12, atol=1e-12)
+
+
+def pin_quantize_act_composition(orc, seed=11):
+    rng = np.random.default_rng(seed)
+    M, K = 24, 96
+    A = (rng.standard_t(4, size=(M, K))).astype(np.float32)
+    A[:, 5] *= 30
+    out = orc.quantize_act(A, 0.99)
+    n = A.size
+    mag = np.sort(np.abs(A.astype(np.float64)).ravel())
+    assert out["T"] == mag[int(np.ceil(0.99 * n)) - 1]
+    T = np.float32(out["T"])
+    A_c = np.where(np.abs(A) > T, np.sign(A) * T, A).astype(np.float32)
+    q, s = orc.quantize_rows(A_c)
+    assert np.array_equal(out["codes"], q) and np.array_equal(out["scales"], s)
+    # amax_i = min(rowmax_i, T)
+    amax = np.minimum(np.abs(A).max(axis=1), T)
+    assert np.array_equal(out["scales"], (amax / np.float32(6)).astype(np.float32))
+
+
+ALL_PINS = [
+    pin_grid, pin_encoder_ties, pin_encoder_nearest_search, pin_row_worked_example,
+    pin_col_worked_example, pin_threshold_worked_example, pin_act_worked_example,
+    pin_gemm_worked_example, pin_threshold_vs_sort_and_quantile, pin_clamp_invariants,
+    pin_quantize_rows_identity, pin_quantize_rows_properties, pin_quantize_degenerate_rows,
+    pin_quantize_cols_transpose, pin_gemm_vs_integer_matmul, pin_spmm_vs_scipy,
+    pin_linear_no_clamp_is_dequant_matmul, pin_linear_exact_on_grid,
+    pin_quantize_act_composition,
+]
