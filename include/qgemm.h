@@ -1,0 +1,192 @@
+/*
+ * qgemm.h -- C ABI of the B200 (sm_100a) FP4 quantized linear layer.
+ *
+ * The layer is the forward pass of the FP4 training method summarised in the
+ * QbitAI write-up "微软首创FP4训练框架，训练效果媲美BF16" (news.movedaos.com/post/4103;
+ * arXiv 2501.17116, "Optimizing Large Language Model Training Using FP4
+ * Quantization"), cited below as [FP4-writeup] with the paragraph:
+ *
+ *     Y = dequant( Q(A_clamped) . Q(W) ) + dA . W
+ *
+ *   A  (M x K, row-major, tokens x in-features), fp32 or bf16
+ *   W  (K x N, row-major), fp32 or bf16
+ *   Q  E2M1 FP4 codes {0, +-0.5, +-1, +-1.5, +-2, +-3, +-4, +-6}
+ *      ([FP4-writeup], E2M1 paragraph), one fp32 scale per row of A
+ *      (token-wise) and per column of W (channel-wise) ([FP4-writeup],
+ *      granularity paragraph), ScaleShift calibration r = 6/amax, s = amax/6,
+ *      round to nearest, ties to the even code ([FP4-writeup], ScaleShift
+ *      paragraph)
+ *   A_clamped = clamp(A, -T, T), T = the alpha-quantile of |A| over the whole
+ *      tensor (order statistic of rank ceil(alpha * M * K) - 1), and the sparse
+ *      compensation dA = A - A_clamped ([FP4-writeup], outlier clamping and
+ *      compensation paragraph)
+ *
+ * Conventions shared by every call:
+ *   - All tensor pointers are DEVICE pointers, owned by the caller; the
+ *     library allocates no device memory.  Calls are asynchronous on the
+ *     given stream; argument checks happen on the host before anything is
+ *     enqueued, and a failed check enqueues nothing.
+ *   - Packed codes hold two 4-bit codes per byte, the even k in the low
+ *     nibble; code bit 3 is the sign, bits 2..0 index the magnitude grid.
+ *     Row codes of A are M x K/2 bytes; column codes of W are stored
+ *     transposed, N x K/2 bytes, so both GEMM operands have K contiguous.
+ *   - Shapes: K % 32 == 0 and 0 < K <= 16384 (else QG_ERR_UNSUPPORTED_SHAPE);
+ *     M, N >= 1 arbitrary.  Row strides (lda, ldw) are in elements, at least
+ *     the row length, and keep every row start 16-byte aligned.  Base
+ *     pointers are 16-byte aligned.
+ *   - Workspace: calls that take (ws, ws_bytes) use a caller-allocated device
+ *     buffer of at least qg_workspace_size(...) bytes, 256-byte aligned.  Its
+ *     first bytes hold a sticky device status word; initialise a new
+ *     workspace once with qg_workspace_init().  Calls on one workspace must
+ *     not overlap in time (use one stream, or one workspace per stream).
+ *   - Errors: nothing aborts, traps or throws.  Host-side argument errors are
+ *     returned immediately.  Device-side conditions (non-finite input, a
+ *     bounded wait that timed out, an internal capacity overflow) set bits in
+ *     the status word; qg_sync_status() synchronises the stream, returns the
+ *     condition and clears it.
+ *   - Inputs must be finite.  Calls that scan all of A for the threshold
+ *     (quantize_act, clamp_compensate, fp4_linear) report NaN/Inf as
+ *     QG_ERR_NONFINITE; the other calls give unspecified codes for them.
+ */
+#ifndef QGEMM_H
+#define QGEMM_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same definition as the CUDA runtime's; 0 / NULL is the legacy stream. */
+typedef struct CUstream_st* cudaStream_t;
+
+typedef enum { QG_F32 = 0, QG_BF16 = 1 } qg_dtype;
+
+typedef enum {
+    QG_OK = 0,
+    QG_ERR_INVALID_ARG = 1,       /* null pointer, bad stride, alpha out of (0, 1], ... */
+    QG_ERR_UNSUPPORTED_SHAPE = 2, /* K % 32 != 0, K > 16384, non-positive sizes */
+    QG_ERR_WORKSPACE = 3,         /* workspace missing, misaligned or too small */
+    QG_ERR_CUDA = 4,              /* a CUDA runtime call failed (launch, no device, ...) */
+    QG_ERR_NONFINITE = 5,         /* NaN or Inf found in A (device-side) */
+    QG_ERR_TIMEOUT = 6,           /* a bounded device wait gave up (device-side) */
+    QG_ERR_INTERNAL = 7           /* device-side capacity check failed */
+} qg_status;
+
+/* CSR form of dA (device arrays, caller-owned).  Rows ascending, columns
+ * ascending within a row; val holds a - sign(a) * T in double (exact for
+ * bf16 input).  nnz_capacity must be at least qg_nnz_capacity(M * K, alpha);
+ * *nnz_out (device int64) receives the count. */
+typedef struct {
+    int32_t* row_ptr;     /* M + 1 */
+    int32_t* col;         /* nnz_capacity */
+    double* val;          /* nnz_capacity */
+    int64_t nnz_capacity;
+    int64_t* nnz_out;     /* device, 1 element */
+} qg_csr;
+
+/* Which call a workspace is sized for. */
+typedef enum {
+    QG_OP_QUANTIZE_ROWS = 0,
+    QG_OP_QUANTIZE_COLS = 1,
+    QG_OP_CLAMP_COMPENSATE = 2,
+    QG_OP_QUANTIZE_ACT = 3,
+    QG_OP_SPMM = 4,
+    QG_OP_FP4_GEMM = 5,
+    QG_OP_FP4_LINEAR = 6
+} qg_op;
+
+const char* qg_status_string(qg_status s);
+const char* qg_version(void);
+
+/* Rank of the threshold in sorted |A|: ceil(alpha * n) - 1 evaluated in
+ * double, clamped to [0, n - 1].  ([FP4-writeup], outlier paragraph; the
+ * order-statistic reading of "quantile".) */
+int64_t qg_quantile_rank(double alpha, int64_t n);
+
+/* Upper bound on the clamped entries: n - (qg_quantile_rank(alpha, n) + 1). */
+int64_t qg_nnz_capacity(int64_t n, double alpha);
+
+/* Bytes of workspace that `op` needs for these sizes (N is ignored by the
+ * activation-only calls; alpha by the calls without a threshold).  Always a
+ * multiple of 256 and at least 256. */
+size_t qg_workspace_size(qg_op op, int64_t M, int64_t K, int64_t N, qg_dtype dtype,
+                         double alpha);
+
+/* Zero the workspace's status word and counters (enqueued on `stream`). */
+qg_status qg_workspace_init(void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Synchronise `stream`, then return and clear the workspace's device status
+ * (QG_OK when nothing was flagged; QG_ERR_CUDA when the stream had failed). */
+qg_status qg_sync_status(void* ws, cudaStream_t stream);
+
+/* Elementwise E2M1 encoding ([FP4-writeup], E2M1 + ScaleShift paragraphs,
+ * rounding only, no scaling): x (n fp32, n even) -> packed (n/2 bytes). */
+qg_status qg_e2m1_encode(const float* x, int64_t n, uint8_t* packed, void* ws,
+                         size_t ws_bytes, cudaStream_t stream);
+
+/* Token-wise (row) quantization of A without clamping ([FP4-writeup],
+ * granularity + ScaleShift paragraphs).  amax_i = max_k |A_ik|;
+ * r_i = fp32(6 / amax_i), s_i = fp32(amax_i / 6) (both 0 when amax_i is 0 or
+ * 6 / amax_i overflows); codes_ik = E2M1(fp32(A_ik * r_i)).
+ * A: M x K (stride lda elements) -> codes M x K/2, scales M (fp32). */
+qg_status qg_quantize_rows(const void* A, qg_dtype dtype, int64_t M, int64_t K, int64_t lda,
+                           uint8_t* codes, float* scales, void* ws, size_t ws_bytes,
+                           cudaStream_t stream);
+
+/* Channel-wise (column) quantization of W ([FP4-writeup], granularity
+ * paragraph), same arithmetic as qg_quantize_rows over the columns of W.
+ * W: K x N (stride ldw elements) -> codesT N x K/2 (transposed), scales N. */
+qg_status qg_quantize_cols(const void* W, qg_dtype dtype, int64_t K, int64_t N, int64_t ldw,
+                           uint8_t* codesT, float* scales, void* ws, size_t ws_bytes,
+                           cudaStream_t stream);
+
+/* Outlier clamping and compensation ([FP4-writeup], outlier paragraph):
+ * T = alpha-quantile of |A| (whole tensor), A_clamped = clamp(A, -T, T) in the
+ * input dtype (M x K, contiguous, may be NULL), dA in CSR, T_out (device fp32,
+ * 1 element).  0 < alpha <= 1. */
+qg_status qg_clamp_compensate(const void* A, qg_dtype dtype, int64_t M, int64_t K, int64_t lda,
+                              double alpha, void* A_clamped, const qg_csr* dA, float* T_out,
+                              void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Fused activation quantizer: threshold, clamp, dA (CSR) and token-wise
+ * quantization of A_clamped (amax_i = min(max_k |A_ik|, T)) in three passes
+ * over A ([FP4-writeup], outlier + granularity + ScaleShift paragraphs).
+ * Outputs as qg_quantize_rows plus dA and T_out. */
+qg_status qg_quantize_act(const void* A, qg_dtype dtype, int64_t M, int64_t K, int64_t lda,
+                          double alpha, uint8_t* codes, float* scales, const qg_csr* dA,
+                          float* T_out, void* ws, size_t ws_bytes, cudaStream_t stream);
+
+/* Compensation product C = dA . W (M x N, fp32, fully written), products and
+ * sums in fp32 with W in its stored dtype ([FP4-writeup], outlier paragraph:
+ * the compensation is kept in higher precision).  W: K x N, stride ldw. */
+qg_status qg_spmm_correction(const qg_csr* dA, int64_t M, const void* W, qg_dtype w_dtype,
+                             int64_t K, int64_t N, int64_t ldw, float* C, void* ws,
+                             size_t ws_bytes, cudaStream_t stream);
+
+/* FP4 GEMM on tcgen05 tensor cores: acc_ij = sum_k e2m1(codesA_ik) *
+ * e2m1(codesWT_jk) accumulated in fp32 (exact for K <= 16384), then
+ * Y_ij = acc_ij * sA_i * sW_j (+ C_ij when C != NULL), stored as fp32 or bf16
+ * (round to nearest even).  raw_acc (nullable, M x N fp32) receives acc itself.
+ * Y may be NULL when only raw_acc is wanted. */
+qg_status qg_fp4_gemm(const uint8_t* codesA, const float* sA, const uint8_t* codesWT,
+                      const float* sW, int64_t M, int64_t N, int64_t K, const float* C,
+                      void* Y, qg_dtype y_dtype, float* raw_acc, void* ws, size_t ws_bytes,
+                      cudaStream_t stream);
+
+/* The whole layer: qg_quantize_act(A) -> qg_spmm_correction(dA, W) ->
+ * qg_fp4_gemm(..., C) into Y (M x N, fp32 or bf16).  codesWT / sW come from
+ * qg_quantize_cols(W); W is the unquantized weight used by the correction.
+ * The activation codes, dA and C live in the workspace
+ * (qg_workspace_size(QG_OP_FP4_LINEAR, ...)). */
+qg_status qg_fp4_linear(const void* A, qg_dtype dtype, int64_t M, int64_t K,
+                        const uint8_t* codesWT, const float* sW, const void* W, int64_t N,
+                        double alpha, void* Y, qg_dtype y_dtype, void* ws, size_t ws_bytes,
+                        cudaStream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* QGEMM_H */

@@ -1,0 +1,325 @@
+"""Python binding of libqgemm.so, the B200 (sm_100a) FP4 quantized linear layer.
+
+Argument marshalling only: every step of the layer runs in the CUDA kernels
+behind the C ABI declared in ``include/qgemm.h``.  The functions named
+``qg_*`` mirror the C entry points one to one and take torch tensors (device
+memory and streams are torch's); the lower-case helpers below them allocate
+outputs with torch and raise :class:`QGError` on a non-OK status.
+
+There is no fallback: importing this package fails when ``lib/libqgemm.so``
+is missing (build it with ``python -m quantize_gemm_b200.build``).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from dataclasses import dataclass
+from typing import Optional
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "lib", "libqgemm.so")
+
+if not os.path.exists(LIB_PATH):
+    raise ImportError(
+        f"{LIB_PATH} is missing: build the CUDA library first "
+        "(python -m quantize_gemm_b200.build, or __graft_entry__.build())")
+
+_lib = ctypes.CDLL(LIB_PATH)
+
+QG_F32, QG_BF16 = 0, 1
+QG_OK, QG_ERR_INVALID_ARG, QG_ERR_UNSUPPORTED_SHAPE, QG_ERR_WORKSPACE, QG_ERR_CUDA, \
+    QG_ERR_NONFINITE, QG_ERR_TIMEOUT, QG_ERR_INTERNAL = range(8)
+(QG_OP_QUANTIZE_ROWS, QG_OP_QUANTIZE_COLS, QG_OP_CLAMP_COMPENSATE, QG_OP_QUANTIZE_ACT,
+ QG_OP_SPMM, QG_OP_FP4_GEMM, QG_OP_FP4_LINEAR) = range(7)
+
+# every symbol the header declares (checked by the CPU tests)
+EXPORTED = (
+    "qg_status_string", "qg_version", "qg_quantile_rank", "qg_nnz_capacity",
+    "qg_workspace_size", "qg_workspace_init", "qg_sync_status", "qg_e2m1_encode",
+    "qg_quantize_rows", "qg_quantize_cols", "qg_clamp_compensate", "qg_quantize_act",
+    "qg_spmm_correction", "qg_fp4_gemm", "qg_fp4_linear",
+)
+
+
+class _Csr(ctypes.Structure):
+    _fields_ = [("row_ptr", ctypes.c_void_p), ("col", ctypes.c_void_p),
+                ("val", ctypes.c_void_p), ("nnz_capacity", ctypes.c_int64),
+                ("nnz_out", ctypes.c_void_p)]
+
+
+_P = ctypes.c_void_p
+_I64 = ctypes.c_int64
+_INT = ctypes.c_int
+_SZ = ctypes.c_size_t
+_D = ctypes.c_double
+
+
+def _sig(name, res, args):
+    f = getattr(_lib, name)
+    f.restype = res
+    f.argtypes = args
+    return f
+
+
+_sig("qg_status_string", ctypes.c_char_p, [_INT])
+_sig("qg_version", ctypes.c_char_p, [])
+_sig("qg_quantile_rank", _I64, [_D, _I64])
+_sig("qg_nnz_capacity", _I64, [_I64, _D])
+_sig("qg_workspace_size", _SZ, [_INT, _I64, _I64, _I64, _INT, _D])
+_sig("qg_workspace_init", _INT, [_P, _SZ, _P])
+_sig("qg_sync_status", _INT, [_P, _P])
+_sig("qg_e2m1_encode", _INT, [_P, _I64, _P, _P, _SZ, _P])
+_sig("qg_quantize_rows", _INT, [_P, _INT, _I64, _I64, _I64, _P, _P, _P, _SZ, _P])
+_sig("qg_quantize_cols", _INT, [_P, _INT, _I64, _I64, _I64, _P, _P, _P, _SZ, _P])
+_sig("qg_clamp_compensate", _INT,
+     [_P, _INT, _I64, _I64, _I64, _D, _P, ctypes.POINTER(_Csr), _P, _P, _SZ, _P])
+_sig("qg_quantize_act", _INT,
+     [_P, _INT, _I64, _I64, _I64, _D, _P, _P, ctypes.POINTER(_Csr), _P, _P, _SZ, _P])
+_sig("qg_spmm_correction", _INT,
+     [ctypes.POINTER(_Csr), _I64, _P, _INT, _I64, _I64, _I64, _P, _P, _SZ, _P])
+_sig("qg_fp4_gemm", _INT,
+     [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _INT, _P, _P, _SZ, _P])
+_sig("qg_fp4_linear", _INT,
+     [_P, _INT, _I64, _I64, _P, _P, _P, _I64, _D, _P, _INT, _P, _SZ, _P])
+
+
+class QGError(RuntimeError):
+    def __init__(self, status: int, where: str = ""):
+        self.status = int(status)
+        super().__init__(f"{where}: {qg_status_string(status)} (status {status})")
+
+
+def qg_status_string(status: int) -> str:
+    return _lib.qg_status_string(int(status)).decode()
+
+
+def qg_version() -> str:
+    return _lib.qg_version().decode()
+
+
+def qg_quantile_rank(alpha: float, n: int) -> int:
+    return int(_lib.qg_quantile_rank(float(alpha), int(n)))
+
+
+def qg_nnz_capacity(n: int, alpha: float) -> int:
+    return int(_lib.qg_nnz_capacity(int(n), float(alpha)))
+
+
+def qg_workspace_size(op: int, M: int, K: int, N: int, dtype: int, alpha: float = 1.0) -> int:
+    return int(_lib.qg_workspace_size(int(op), int(M), int(K), int(N), int(dtype), float(alpha)))
+
+
+# ------------------------------------------------------------------ marshalling
+def _dt(t: torch.Tensor) -> int:
+    if t.dtype == torch.float32:
+        return QG_F32
+    if t.dtype == torch.bfloat16:
+        return QG_BF16
+    raise TypeError(f"unsupported dtype {t.dtype} (fp32 or bf16)")
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError("device tensor expected")
+    return ctypes.c_void_p(t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    if isinstance(stream, torch.cuda.Stream):
+        return ctypes.c_void_p(stream.cuda_stream)
+    return ctypes.c_void_p(int(stream))
+
+
+def _check(status: int, where: str):
+    if status != QG_OK:
+        raise QGError(status, where)
+
+
+@dataclass
+class CSR:
+    """dA in CSR form, device tensors (row_ptr int32 M+1, col int32, val f64)."""
+    row_ptr: torch.Tensor
+    col: torch.Tensor
+    val: torch.Tensor
+    nnz: torch.Tensor          # int64, 1 element (device)
+    capacity: int
+
+    @staticmethod
+    def empty(M: int, capacity: int, device="cuda") -> "CSR":
+        cap = max(int(capacity), 1)
+        return CSR(torch.empty(M + 1, dtype=torch.int32, device=device),
+                   torch.empty(cap, dtype=torch.int32, device=device),
+                   torch.empty(cap, dtype=torch.float64, device=device),
+                   torch.zeros(1, dtype=torch.int64, device=device), int(capacity))
+
+    def c(self) -> _Csr:
+        return _Csr(self.row_ptr.data_ptr(), self.col.data_ptr(), self.val.data_ptr(),
+                    max(self.capacity, 1), self.nnz.data_ptr())
+
+    def to_host(self):
+        n = int(self.nnz.item())
+        return (self.row_ptr.cpu().numpy(), self.col[:n].cpu().numpy(),
+                self.val[:n].cpu().numpy())
+
+
+class Workspace:
+    """Device workspace for one call type: status word, counters, scratch."""
+
+    def __init__(self, op: int, M: int, K: int, N: int = 1, dtype: int = QG_BF16,
+                 alpha: float = 1.0, device="cuda", stream=None):
+        self.nbytes = qg_workspace_size(op, M, K, N, dtype, alpha)
+        self.buf = torch.empty(self.nbytes, dtype=torch.uint8, device=device)
+        _check(_lib.qg_workspace_init(_ptr(self.buf), self.nbytes, _stream(stream)),
+               "qg_workspace_init")
+
+    @property
+    def ptr(self):
+        return _ptr(self.buf)
+
+    def sync_status(self, stream=None) -> int:
+        return qg_sync_status(self, stream)
+
+
+def qg_sync_status(ws: Workspace, stream=None) -> int:
+    return int(_lib.qg_sync_status(ws.ptr, _stream(stream)))
+
+
+# --------------------------------------------------------- the C entry points
+def qg_e2m1_encode(x: torch.Tensor, packed: torch.Tensor, ws: Workspace, stream=None) -> int:
+    return _lib.qg_e2m1_encode(_ptr(x), x.numel(), _ptr(packed), ws.ptr, ws.nbytes,
+                               _stream(stream))
+
+
+def qg_quantize_rows(A, codes, scales, ws: Workspace, lda=None, stream=None) -> int:
+    M, K = A.shape
+    return _lib.qg_quantize_rows(_ptr(A), _dt(A), M, K, A.stride(0) if lda is None else lda,
+                                 _ptr(codes), _ptr(scales), ws.ptr, ws.nbytes, _stream(stream))
+
+
+def qg_quantize_cols(W, codesT, scales, ws: Workspace, ldw=None, stream=None) -> int:
+    K, N = W.shape
+    return _lib.qg_quantize_cols(_ptr(W), _dt(W), K, N, W.stride(0) if ldw is None else ldw,
+                                 _ptr(codesT), _ptr(scales), ws.ptr, ws.nbytes, _stream(stream))
+
+
+def qg_clamp_compensate(A, alpha, A_clamped, csr: CSR, T_out, ws: Workspace, stream=None) -> int:
+    M, K = A.shape
+    c = csr.c()
+    return _lib.qg_clamp_compensate(_ptr(A), _dt(A), M, K, A.stride(0), float(alpha),
+                                    _ptr(A_clamped), ctypes.byref(c), _ptr(T_out), ws.ptr,
+                                    ws.nbytes, _stream(stream))
+
+
+def qg_quantize_act(A, alpha, codes, scales, csr: CSR, T_out, ws: Workspace, stream=None) -> int:
+    M, K = A.shape
+    c = csr.c()
+    return _lib.qg_quantize_act(_ptr(A), _dt(A), M, K, A.stride(0), float(alpha), _ptr(codes),
+                                _ptr(scales), ctypes.byref(c), _ptr(T_out), ws.ptr, ws.nbytes,
+                                _stream(stream))
+
+
+def qg_spmm_correction(csr: CSR, M, W, C, ws: Workspace, stream=None) -> int:
+    K, N = W.shape
+    c = csr.c()
+    return _lib.qg_spmm_correction(ctypes.byref(c), M, _ptr(W), _dt(W), K, N, W.stride(0),
+                                   _ptr(C), ws.ptr, ws.nbytes, _stream(stream))
+
+
+def qg_fp4_gemm(codesA, sA, codesWT, sW, M, N, K, C, Y, raw_acc, ws: Workspace,
+                stream=None) -> int:
+    y_dt = _dt(Y) if Y is not None else QG_F32
+    return _lib.qg_fp4_gemm(_ptr(codesA), _ptr(sA), _ptr(codesWT), _ptr(sW), M, N, K, _ptr(C),
+                            _ptr(Y), y_dt, _ptr(raw_acc), ws.ptr, ws.nbytes, _stream(stream))
+
+
+def qg_fp4_linear(A, codesWT, sW, W, alpha, Y, ws: Workspace, stream=None) -> int:
+    M, K = A.shape
+    N = W.shape[1]
+    return _lib.qg_fp4_linear(_ptr(A), _dt(A), M, K, _ptr(codesWT), _ptr(sW), _ptr(W), N,
+                              float(alpha), _ptr(Y), _dt(Y), ws.ptr, ws.nbytes, _stream(stream))
+
+
+# ----------------------------------------------------------- allocating helpers
+def e2m1_encode(x: torch.Tensor, ws: Optional[Workspace] = None) -> torch.Tensor:
+    ws = ws or Workspace(QG_OP_QUANTIZE_ROWS, 1, 32, device=x.device)
+    out = torch.empty(x.numel() // 2, dtype=torch.uint8, device=x.device)
+    _check(qg_e2m1_encode(x, out, ws), "qg_e2m1_encode")
+    return out
+
+
+def quantize_rows(A: torch.Tensor, ws: Optional[Workspace] = None):
+    M, K = A.shape
+    ws = ws or Workspace(QG_OP_QUANTIZE_ROWS, M, K, 1, _dt(A), device=A.device)
+    codes = torch.empty((M, K // 2), dtype=torch.uint8, device=A.device)
+    scales = torch.empty(M, dtype=torch.float32, device=A.device)
+    _check(qg_quantize_rows(A, codes, scales, ws), "qg_quantize_rows")
+    return codes, scales
+
+
+def quantize_cols(W: torch.Tensor, ws: Optional[Workspace] = None):
+    K, N = W.shape
+    ws = ws or Workspace(QG_OP_QUANTIZE_COLS, 1, K, N, _dt(W), device=W.device)
+    codesT = torch.empty((N, K // 2), dtype=torch.uint8, device=W.device)
+    scales = torch.empty(N, dtype=torch.float32, device=W.device)
+    _check(qg_quantize_cols(W, codesT, scales, ws), "qg_quantize_cols")
+    return codesT, scales
+
+
+def clamp_compensate(A: torch.Tensor, alpha: float, ws: Optional[Workspace] = None,
+                     want_clamped: bool = True):
+    M, K = A.shape
+    ws = ws or Workspace(QG_OP_CLAMP_COMPENSATE, M, K, 1, _dt(A), alpha, device=A.device)
+    csr = CSR.empty(M, qg_nnz_capacity(M * K, alpha), device=A.device)
+    A_c = torch.empty_like(A) if want_clamped else None
+    T = torch.empty(1, dtype=torch.float32, device=A.device)
+    _check(qg_clamp_compensate(A, alpha, A_c, csr, T, ws), "qg_clamp_compensate")
+    return A_c, csr, T
+
+
+def quantize_act(A: torch.Tensor, alpha: float, ws: Optional[Workspace] = None):
+    M, K = A.shape
+    ws = ws or Workspace(QG_OP_QUANTIZE_ACT, M, K, 1, _dt(A), alpha, device=A.device)
+    codes = torch.empty((M, K // 2), dtype=torch.uint8, device=A.device)
+    scales = torch.empty(M, dtype=torch.float32, device=A.device)
+    csr = CSR.empty(M, qg_nnz_capacity(M * K, alpha), device=A.device)
+    T = torch.empty(1, dtype=torch.float32, device=A.device)
+    _check(qg_quantize_act(A, alpha, codes, scales, csr, T, ws), "qg_quantize_act")
+    return codes, scales, csr, T
+
+
+def spmm_correction(csr: CSR, M: int, W: torch.Tensor, ws: Optional[Workspace] = None):
+    K, N = W.shape
+    ws = ws or Workspace(QG_OP_SPMM, M, K, N, _dt(W), device=W.device)
+    C = torch.empty((M, N), dtype=torch.float32, device=W.device)
+    _check(qg_spmm_correction(csr, M, W, C, ws), "qg_spmm_correction")
+    return C
+
+
+def fp4_gemm(codesA, sA, codesWT, sW, K: int, C=None, out_dtype=torch.float32,
+             raw: bool = False, ws: Optional[Workspace] = None):
+    M, N = codesA.shape[0], codesWT.shape[0]
+    ws = ws or Workspace(QG_OP_FP4_GEMM, M, K, N, QG_F32, device=codesA.device)
+    Y = torch.empty((M, N), dtype=out_dtype, device=codesA.device)
+    acc = torch.empty((M, N), dtype=torch.float32, device=codesA.device) if raw else None
+    _check(qg_fp4_gemm(codesA, sA, codesWT, sW, M, N, K, C, Y, acc, ws), "qg_fp4_gemm")
+    return (Y, acc) if raw else Y
+
+
+def fp4_linear(A, codesWT, sW, W, alpha: float, out_dtype=torch.float32,
+               ws: Optional[Workspace] = None):
+    M, K = A.shape
+    N = W.shape[1]
+    ws = ws or Workspace(QG_OP_FP4_LINEAR, M, K, N, _dt(A), alpha, device=A.device)
+    Y = torch.empty((M, N), dtype=out_dtype, device=A.device)
+    _check(qg_fp4_linear(A, codesWT, sW, W, alpha, Y, ws), "qg_fp4_linear")
+    return Y
+
+
+def check_status(ws: Workspace, where: str = "device status", stream=None):
+    _check(qg_sync_status(ws, stream), where)

@@ -1,0 +1,314 @@
+// api.cu -- the C ABI (include/qgemm.h): argument checks, workspace layout
+// and the launch sequences of each call.  No device memory is allocated here.
+#include <math.h>
+
+#include <mutex>
+
+#include "qg_internal.cuh"
+
+namespace qg {
+
+static const int kMaxDevices = 64;
+static int g_sms[kMaxDevices];
+static bool g_ready[kMaxDevices];
+static std::mutex g_mu;
+
+// One-time per-device setup (kernel attributes), with that device current.
+static cudaError_t ensure_device(int* dev_out) {
+    int dev = -1;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    if (dev < 0 || dev >= kMaxDevices) return cudaErrorInvalidDevice;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_ready[dev]) {
+        int sms = 0;
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e != cudaSuccess) return e;
+        e = act_setup();
+        if (e != cudaSuccess) return e;
+        e = gemm_setup();
+        if (e != cudaSuccess) return e;
+        g_sms[dev] = sms;
+        g_ready[dev] = true;
+    }
+    if (dev_out) *dev_out = dev;
+    return cudaSuccess;
+}
+
+int num_sms() {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices || g_sms[dev] <= 0)
+        return 148;
+    return g_sms[dev];
+}
+
+static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+static size_t elsize(qg_dtype d) { return d == QG_BF16 ? 2 : 4; }
+static bool dtype_ok(qg_dtype d) { return d == QG_F32 || d == QG_BF16; }
+
+static qg_status check_mk(int64_t M, int64_t K) {
+    if (M < 1 || K < 1) return QG_ERR_UNSUPPORTED_SHAPE;
+    if (K % 32 != 0 || K > 16384) return QG_ERR_UNSUPPORTED_SHAPE;
+    if (M > (int64_t)INT32_MAX - 1) return QG_ERR_UNSUPPORTED_SHAPE;
+    return QG_OK;
+}
+
+static qg_status check_ld(const void* A, qg_dtype dt, int64_t K, int64_t ld) {
+    if (A == nullptr || !aligned16(A)) return QG_ERR_INVALID_ARG;
+    if (ld < K || ((size_t)ld * elsize(dt)) % 16 != 0) return QG_ERR_INVALID_ARG;
+    return QG_OK;
+}
+
+static qg_status check_ws(void* ws, size_t ws_bytes, size_t need) {
+    if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0) return QG_ERR_WORKSPACE;
+    if (ws_bytes < need) return QG_ERR_WORKSPACE;
+    return QG_OK;
+}
+
+static bool alpha_ok(double a) { return a > 0.0 && a <= 1.0; }
+
+static qg_status cuda_status(cudaError_t e) { return e == cudaSuccess ? QG_OK : QG_ERR_CUDA; }
+
+template <class T>
+static T* at(void* ws, size_t off) {
+    return reinterpret_cast<T*>(static_cast<uint8_t*>(ws) + off);
+}
+
+static ActBuffers act_buffers(void* ws, const WsLayout& L) {
+    ActBuffers b;
+    b.status = at<uint32_t>(ws, L.status);
+    b.ctr = at<Counters>(ws, L.counters);
+    b.hist1 = at<uint32_t>(ws, L.hist1);
+    b.hist2 = L.hist2 ? at<uint32_t>(ws, L.hist2) : nullptr;
+    b.rowmax = at<uint32_t>(ws, L.rowmax);
+    b.rowcnt = at<uint32_t>(ws, L.rowcnt);
+    b.st_row = at<int32_t>(ws, L.st_row);
+    b.st_rank = at<int32_t>(ws, L.st_rank);
+    b.st_col = at<int32_t>(ws, L.st_col);
+    b.st_val = at<double>(ws, L.st_val);
+    b.cap = L.cap;
+    return b;
+}
+
+static qg_status check_csr(const qg_csr* dA, int64_t n, double alpha) {
+    if (dA == nullptr || dA->row_ptr == nullptr || dA->nnz_out == nullptr) return QG_ERR_INVALID_ARG;
+    int64_t k = (int64_t)ceil(alpha * (double)n) - 1;
+    if (k < 0) k = 0;
+    if (k > n - 1) k = n - 1;
+    const int64_t cap = n - (k + 1);
+    if (cap > 0 && (dA->col == nullptr || dA->val == nullptr)) return QG_ERR_INVALID_ARG;
+    if (dA->nnz_capacity < cap) return QG_ERR_INVALID_ARG;
+    if (cap > (int64_t)INT32_MAX) return QG_ERR_UNSUPPORTED_SHAPE;
+    return QG_OK;
+}
+
+}  // namespace qg
+
+using namespace qg;
+
+extern "C" {
+
+const char* qg_status_string(qg_status s) {
+    switch (s) {
+        case QG_OK: return "ok";
+        case QG_ERR_INVALID_ARG: return "invalid argument";
+        case QG_ERR_UNSUPPORTED_SHAPE: return "unsupported shape (need K % 32 == 0, 0 < K <= 16384, M, N >= 1)";
+        case QG_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+        case QG_ERR_CUDA: return "CUDA runtime error";
+        case QG_ERR_NONFINITE: return "non-finite value (NaN/Inf) in the input";
+        case QG_ERR_TIMEOUT: return "a bounded device wait timed out";
+        case QG_ERR_INTERNAL: return "internal capacity check failed";
+    }
+    return "unknown status";
+}
+
+const char* qg_version(void) { return "qgemm 0.1 sm_100a"; }
+
+int64_t qg_quantile_rank(double alpha, int64_t n) {
+    int64_t k = (int64_t)ceil(alpha * (double)n) - 1;
+    if (k < 0) k = 0;
+    if (k > n - 1) k = n - 1;
+    return k;
+}
+
+int64_t qg_nnz_capacity(int64_t n, double alpha) {
+    if (n <= 0) return 0;
+    return n - (qg_quantile_rank(alpha, n) + 1);
+}
+
+size_t qg_workspace_size(qg_op op, int64_t M, int64_t K, int64_t N, qg_dtype dtype, double alpha) {
+    if (M < 1) M = 1;
+    if (K < 2) K = 2;
+    if (N < 1) N = 1;
+    if (!(alpha > 0.0 && alpha <= 1.0)) alpha = 1.0;
+    return ws_layout(op, M, K, N, dtype, alpha).total;
+}
+
+qg_status qg_workspace_init(void* ws, size_t ws_bytes, cudaStream_t stream) {
+    if (ws == nullptr || (reinterpret_cast<uintptr_t>(ws) & (kAlign - 1)) != 0 || ws_bytes < 2 * kAlign)
+        return QG_ERR_WORKSPACE;
+    cudaError_t e = ensure_device(nullptr);
+    if (e != cudaSuccess) return QG_ERR_CUDA;
+    return cuda_status(cudaMemsetAsync(ws, 0, 2 * kAlign, stream));
+}
+
+qg_status qg_sync_status(void* ws, cudaStream_t stream) {
+    if (ws == nullptr) return QG_ERR_WORKSPACE;
+    if (cudaStreamSynchronize(stream) != cudaSuccess) return QG_ERR_CUDA;
+    uint32_t st = 0;
+    if (cudaMemcpy(&st, ws, sizeof(st), cudaMemcpyDeviceToHost) != cudaSuccess) return QG_ERR_CUDA;
+    if (st == 0) return QG_OK;
+    if (cudaMemset(ws, 0, sizeof(uint32_t)) != cudaSuccess) return QG_ERR_CUDA;
+    if (st & kStatusNonFinite) return QG_ERR_NONFINITE;
+    if (st & kStatusTimeout) return QG_ERR_TIMEOUT;
+    return QG_ERR_INTERNAL;
+}
+
+qg_status qg_e2m1_encode(const float* x, int64_t n, uint8_t* packed, void* ws, size_t ws_bytes,
+                         cudaStream_t stream) {
+    if (n < 0 || (n % 2) != 0) return QG_ERR_INVALID_ARG;
+    if (n == 0) return QG_OK;
+    if (!x || !packed || !aligned16(x) || !aligned16(packed)) return QG_ERR_INVALID_ARG;
+    qg_status st = check_ws(ws, ws_bytes, ws_layout(QG_OP_QUANTIZE_ROWS, 1, 32, 1, QG_F32, 1.0).total);
+    if (st != QG_OK) return st;
+    if (ensure_device(nullptr) != cudaSuccess) return QG_ERR_CUDA;
+    launch_e2m1_encode(x, n, packed, stream);
+    return cuda_status(cudaGetLastError());
+}
+
+qg_status qg_quantize_rows(const void* A, qg_dtype dtype, int64_t M, int64_t K, int64_t lda,
+                           uint8_t* codes, float* scales, void* ws, size_t ws_bytes,
+                           cudaStream_t stream) {
+    if (!dtype_ok(dtype)) return QG_ERR_INVALID_ARG;
+    qg_status st = check_mk(M, K);
+    if (st != QG_OK) return st;
+    if ((st = check_ld(A, dtype, K, lda)) != QG_OK) return st;
+    if (!codes || !scales || !aligned16(codes)) return QG_ERR_INVALID_ARG;
+    if ((st = check_ws(ws, ws_bytes, ws_layout(QG_OP_QUANTIZE_ROWS, M, K, 1, dtype, 1.0).total)) != QG_OK)
+        return st;
+    if (ensure_device(nullptr) != cudaSuccess) return QG_ERR_CUDA;
+    launch_quantize_rows(A, dtype, M, K, lda, codes, scales, stream);
+    return cuda_status(cudaGetLastError());
+}
+
+qg_status qg_quantize_cols(const void* W, qg_dtype dtype, int64_t K, int64_t N, int64_t ldw,
+                           uint8_t* codesT, float* scales, void* ws, size_t ws_bytes,
+                           cudaStream_t stream) {
+    if (!dtype_ok(dtype)) return QG_ERR_INVALID_ARG;
+    qg_status st = check_mk(N, K);
+    if (st != QG_OK) return st;
+    if (W == nullptr || !aligned16(W) || ldw < N) return QG_ERR_INVALID_ARG;
+    if (!codesT || !scales || !aligned16(codesT)) return QG_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(QG_OP_QUANTIZE_COLS, 1, K, N, dtype, 1.0);
+    if ((st = check_ws(ws, ws_bytes, L.total)) != QG_OK) return st;
+    if (ensure_device(nullptr) != cudaSuccess) return QG_ERR_CUDA;
+    launch_quantize_cols(W, dtype, K, N, ldw, codesT, scales, at<uint32_t>(ws, L.colmax), stream);
+    return cuda_status(cudaGetLastError());
+}
+
+qg_status qg_clamp_compensate(const void* A, qg_dtype dtype, int64_t M, int64_t K, int64_t lda,
+                              double alpha, void* A_clamped, const qg_csr* dA, float* T_out,
+                              void* ws, size_t ws_bytes, cudaStream_t stream) {
+    if (!dtype_ok(dtype) || !alpha_ok(alpha)) return QG_ERR_INVALID_ARG;
+    qg_status st = check_mk(M, K);
+    if (st != QG_OK) return st;
+    if ((st = check_ld(A, dtype, K, lda)) != QG_OK) return st;
+    if (A_clamped && !aligned16(A_clamped)) return QG_ERR_INVALID_ARG;
+    if (T_out == nullptr) return QG_ERR_INVALID_ARG;
+    if ((st = check_csr(dA, M * K, alpha)) != QG_OK) return st;
+    const WsLayout L = ws_layout(QG_OP_CLAMP_COMPENSATE, M, K, 1, dtype, alpha);
+    if ((st = check_ws(ws, ws_bytes, L.total)) != QG_OK) return st;
+    if (ensure_device(nullptr) != cudaSuccess) return QG_ERR_CUDA;
+    const int64_t rank = qg_quantile_rank(alpha, M * K);
+    return cuda_status(run_clamp_compensate(A, dtype, M, K, lda, rank, act_buffers(ws, L), A_clamped,
+                                            dA, T_out, stream));
+}
+
+qg_status qg_quantize_act(const void* A, qg_dtype dtype, int64_t M, int64_t K, int64_t lda,
+                          double alpha, uint8_t* codes, float* scales, const qg_csr* dA,
+                          float* T_out, void* ws, size_t ws_bytes, cudaStream_t stream) {
+    if (!dtype_ok(dtype) || !alpha_ok(alpha)) return QG_ERR_INVALID_ARG;
+    qg_status st = check_mk(M, K);
+    if (st != QG_OK) return st;
+    if ((st = check_ld(A, dtype, K, lda)) != QG_OK) return st;
+    if (!codes || !scales || !aligned16(codes) || T_out == nullptr) return QG_ERR_INVALID_ARG;
+    if ((st = check_csr(dA, M * K, alpha)) != QG_OK) return st;
+    const WsLayout L = ws_layout(QG_OP_QUANTIZE_ACT, M, K, 1, dtype, alpha);
+    if ((st = check_ws(ws, ws_bytes, L.total)) != QG_OK) return st;
+    if (ensure_device(nullptr) != cudaSuccess) return QG_ERR_CUDA;
+    const int64_t rank = qg_quantile_rank(alpha, M * K);
+    return cuda_status(run_quantize_act(A, dtype, M, K, lda, rank, act_buffers(ws, L), codes, scales,
+                                        dA, T_out, stream));
+}
+
+qg_status qg_spmm_correction(const qg_csr* dA, int64_t M, const void* W, qg_dtype w_dtype,
+                             int64_t K, int64_t N, int64_t ldw, float* C, void* ws,
+                             size_t ws_bytes, cudaStream_t stream) {
+    if (!dtype_ok(w_dtype)) return QG_ERR_INVALID_ARG;
+    if (M < 1 || N < 1 || K < 1) return QG_ERR_UNSUPPORTED_SHAPE;
+    if (dA == nullptr || dA->row_ptr == nullptr) return QG_ERR_INVALID_ARG;
+    if (W == nullptr || !aligned16(W) || ldw < N || C == nullptr || !aligned16(C)) return QG_ERR_INVALID_ARG;
+    qg_status st = check_ws(ws, ws_bytes, ws_layout(QG_OP_SPMM, M, K, N, w_dtype, 1.0).total);
+    if (st != QG_OK) return st;
+    if (ensure_device(nullptr) != cudaSuccess) return QG_ERR_CUDA;
+    launch_spmm(dA, M, W, w_dtype, N, ldw, C, stream);
+    return cuda_status(cudaGetLastError());
+}
+
+qg_status qg_fp4_gemm(const uint8_t* codesA, const float* sA, const uint8_t* codesWT,
+                      const float* sW, int64_t M, int64_t N, int64_t K, const float* C, void* Y,
+                      qg_dtype y_dtype, float* raw_acc, void* ws, size_t ws_bytes,
+                      cudaStream_t stream) {
+    if (!dtype_ok(y_dtype)) return QG_ERR_INVALID_ARG;
+    qg_status st = check_mk(M, K);
+    if (st != QG_OK) return st;
+    if ((st = check_mk(N, K)) != QG_OK) return st;
+    if (!codesA || !codesWT || !sA || !sW || !aligned16(codesA) || !aligned16(codesWT) ||
+        !aligned16(sW))
+        return QG_ERR_INVALID_ARG;
+    if (Y == nullptr && raw_acc == nullptr) return QG_ERR_INVALID_ARG;
+    if ((Y && !aligned16(Y)) || (C && !aligned16(C)) || (raw_acc && !aligned16(raw_acc)))
+        return QG_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(QG_OP_FP4_GEMM, M, K, N, y_dtype, 1.0);
+    if ((st = check_ws(ws, ws_bytes, L.total)) != QG_OK) return st;
+    if (ensure_device(nullptr) != cudaSuccess) return QG_ERR_CUDA;
+    return cuda_status(launch_fp4_gemm(codesA, sA, codesWT, sW, M, N, K, C, Y, y_dtype, raw_acc,
+                                       at<uint32_t>(ws, L.status), stream));
+}
+
+qg_status qg_fp4_linear(const void* A, qg_dtype dtype, int64_t M, int64_t K,
+                        const uint8_t* codesWT, const float* sW, const void* W, int64_t N,
+                        double alpha, void* Y, qg_dtype y_dtype, void* ws, size_t ws_bytes,
+                        cudaStream_t stream) {
+    if (!dtype_ok(dtype) || !dtype_ok(y_dtype) || !alpha_ok(alpha)) return QG_ERR_INVALID_ARG;
+    qg_status st = check_mk(M, K);
+    if (st != QG_OK) return st;
+    if ((st = check_mk(N, K)) != QG_OK) return st;
+    if ((st = check_ld(A, dtype, K, K)) != QG_OK) return st;
+    if (!codesWT || !sW || !W || !Y || !aligned16(codesWT) || !aligned16(sW) || !aligned16(W) ||
+        !aligned16(Y))
+        return QG_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(QG_OP_FP4_LINEAR, M, K, N, dtype, alpha);
+    if ((st = check_ws(ws, ws_bytes, L.total)) != QG_OK) return st;
+    if (L.cap > (int64_t)INT32_MAX) return QG_ERR_UNSUPPORTED_SHAPE;
+    if (ensure_device(nullptr) != cudaSuccess) return QG_ERR_CUDA;
+    qg_csr csr;
+    csr.row_ptr = at<int32_t>(ws, L.csr_row_ptr);
+    csr.col = at<int32_t>(ws, L.csr_col);
+    csr.val = at<double>(ws, L.csr_val);
+    csr.nnz_capacity = L.cap;
+    csr.nnz_out = at<int64_t>(ws, L.csr_nnz);
+    uint8_t* codes = at<uint8_t>(ws, L.act_codes);
+    float* scales = at<float>(ws, L.act_scales);
+    float* C = at<float>(ws, L.corr);
+    const int64_t rank = qg_quantile_rank(alpha, M * K);
+    cudaError_t e = run_quantize_act(A, dtype, M, K, K, rank, act_buffers(ws, L), codes, scales, &csr,
+                                     at<float>(ws, L.thr), stream);
+    if (e != cudaSuccess) return QG_ERR_CUDA;
+    launch_spmm(&csr, M, W, dtype, N, N, C, stream);
+    if ((e = cudaGetLastError()) != cudaSuccess) return QG_ERR_CUDA;
+    return cuda_status(launch_fp4_gemm(codes, scales, codesWT, sW, M, N, K, C, Y, y_dtype, nullptr,
+                                       at<uint32_t>(ws, L.status), stream));
+}
+
+}  // extern "C"

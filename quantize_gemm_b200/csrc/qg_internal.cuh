@@ -1,0 +1,241 @@
+// qg_internal.cuh -- device helpers and workspace layout shared by the
+// kernels of the FP4 linear-layer library (sm_100a only).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include <algorithm>
+
+#include "../../include/qgemm.h"
+
+#if defined(__CUDA_ARCH__) && (__CUDA_ARCH__ < 1000)
+#error "this library targets sm_100a (B200) only"
+#endif
+
+namespace qg {
+
+// ---------------------------------------------------------------- status word
+// Sticky device status bits, OR-ed into the first word of the workspace.
+enum : uint32_t {
+    kStatusNonFinite = 1u << 0,
+    kStatusTimeout = 1u << 1,
+    kStatusOverflow = 1u << 2,
+};
+
+// Counters that live right after the status word.
+struct Counters {
+    unsigned long long nnz;        // staging slots reserved so far
+    unsigned long long sel_below;  // entries strictly below the selected bin
+    uint32_t nonfinite;            // set when a NaN/Inf key was seen
+    uint32_t sel_bin;              // bin chosen by the last selection pass
+    uint32_t T_key;                // final threshold as |x| bit pattern
+    uint32_t pad;
+};
+
+// ---------------------------------------------------------------- workspace
+constexpr size_t kAlign = 256;
+constexpr int kHist1Bins = 1 << 15;   // 15-bit keys (bf16 |x|, fp32 |x| >> 16)
+constexpr int kHist2Bins = 1 << 16;   // fp32 refine: low 16 bits of |x|
+
+inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
+
+struct WsLayout {
+    size_t status = 0, counters = 0, hist1 = 0, hist2 = 0, rowmax = 0, rowcnt = 0;
+    size_t st_row = 0, st_rank = 0, st_col = 0, st_val = 0, colmax = 0;
+    size_t act_codes = 0, act_scales = 0, csr_row_ptr = 0, csr_col = 0, csr_val = 0,
+           csr_nnz = 0, thr = 0, corr = 0;
+    size_t total = 0;
+    int64_t cap = 0;
+};
+
+// Compute the layout for an op.  Offsets are relative to the workspace base.
+inline WsLayout ws_layout(qg_op op, int64_t M, int64_t K, int64_t N, qg_dtype dtype,
+                          double alpha) {
+    WsLayout L;
+    size_t off = 0;
+    auto take = [&](size_t bytes) {
+        size_t at = off;
+        off = align_up(off + (bytes ? bytes : 1));
+        return at;
+    };
+    L.status = take(16);
+    L.counters = take(sizeof(Counters));
+    bool act = (op == QG_OP_CLAMP_COMPENSATE || op == QG_OP_QUANTIZE_ACT ||
+                op == QG_OP_FP4_LINEAR);
+    if (act) {
+        int64_t n = M * K;
+        int64_t k = (int64_t)ceil(alpha * (double)n) - 1;
+        if (k < 0) k = 0;
+        if (k > n - 1) k = n - 1;
+        L.cap = n - (k + 1);
+        int64_t cap = L.cap > 0 ? L.cap : 1;
+        L.hist1 = take(sizeof(uint32_t) * kHist1Bins);
+        if (dtype == QG_F32) L.hist2 = take(sizeof(uint32_t) * kHist2Bins);
+        L.rowmax = take(sizeof(uint32_t) * (size_t)M);
+        L.rowcnt = take(sizeof(uint32_t) * (size_t)M);
+        L.st_row = take(sizeof(int32_t) * (size_t)cap);
+        L.st_rank = take(sizeof(int32_t) * (size_t)cap);
+        L.st_col = take(sizeof(int32_t) * (size_t)cap);
+        L.st_val = take(sizeof(double) * (size_t)cap);
+    }
+    if (op == QG_OP_QUANTIZE_COLS) L.colmax = take(sizeof(uint32_t) * (size_t)N);
+    if (op == QG_OP_FP4_LINEAR) {
+        int64_t cap = L.cap > 0 ? L.cap : 1;
+        L.act_codes = take((size_t)M * (size_t)(K / 2));
+        L.act_scales = take(sizeof(float) * (size_t)M);
+        L.csr_row_ptr = take(sizeof(int32_t) * (size_t)(M + 1));
+        L.csr_col = take(sizeof(int32_t) * (size_t)cap);
+        L.csr_val = take(sizeof(double) * (size_t)cap);
+        L.csr_nnz = take(sizeof(int64_t));
+        L.thr = take(sizeof(float));
+        L.corr = take(sizeof(float) * (size_t)M * (size_t)N);
+    }
+    L.total = off;
+    return L;
+}
+
+// ------------------------------------------------------------- device helpers
+#ifdef __CUDACC__
+
+__device__ __forceinline__ void flag_status(uint32_t* status, uint32_t bits) {
+    atomicOr(status, bits);
+}
+
+// E2M1 encoding of two fp32 values with the hardware converter
+// (cvt.rn.satfinite.e2m1x2.f32: round to nearest even, saturate at 6), then
+// the sign bit of each input is copied in so that a negative input that
+// rounds to zero keeps its sign (code 0x8).  lo lands in bits 3..0.
+__device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
+    uint16_t r;
+    asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u16.u8 %0, t;\n\t}"
+        : "=h"(r)
+        : "f"(hi), "f"(lo));
+    uint32_t sgn = ((__float_as_uint(lo) >> 31) << 3) | ((__float_as_uint(hi) >> 31) << 7);
+    return ((uint32_t)r & 0xFFu) | sgn;
+}
+
+// Eight values -> four packed bytes (element 0 in the low nibble of byte 0).
+__device__ __forceinline__ uint32_t e2m1x8(const float (&x)[8]) {
+    return e2m1x2(x[0], x[1]) | (e2m1x2(x[2], x[3]) << 8) | (e2m1x2(x[4], x[5]) << 16) |
+           (e2m1x2(x[6], x[7]) << 24);
+}
+
+// Scale factors of one row/column from its absolute maximum:
+// r = 6 / amax and s = amax / 6, IEEE correctly rounded; both 0 for a zero
+// (or so tiny that 6 / amax overflows) maximum.
+__device__ __forceinline__ void scale_factors(float amax, float& r, float& s) {
+    float rr = __fdiv_rn(6.0f, amax);
+    if (amax == 0.0f || isinf(rr)) {
+        r = 0.0f;
+        s = 0.0f;
+    } else {
+        r = rr;
+        s = __fdiv_rn(amax, 6.0f);
+    }
+}
+
+// Magnitude key of a value: the bit pattern without the sign.  For finite
+// values the keys order like |x|.
+__device__ __forceinline__ uint32_t key_of(float x) { return __float_as_uint(x) & 0x7FFFFFFFu; }
+__device__ __forceinline__ uint32_t key_of_bf16_bits(uint32_t b) { return b & 0x7FFFu; }
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t b) { return __uint_as_float(b << 16); }
+
+// Load 8 consecutive elements (16-byte aligned) as fp32.
+template <qg_dtype DT>
+__device__ __forceinline__ void load8(const void* base, int64_t idx, float (&x)[8]) {
+    if constexpr (DT == QG_BF16) {
+        uint4 v = __ldg(reinterpret_cast<const uint4*>(static_cast<const uint16_t*>(base) + idx));
+        uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            x[2 * i] = __uint_as_float(w[i] << 16);
+            x[2 * i + 1] = __uint_as_float(w[i] & 0xFFFF0000u);
+        }
+    } else {
+        const float4* p = reinterpret_cast<const float4*>(static_cast<const float*>(base) + idx);
+        float4 a = __ldg(p), b = __ldg(p + 1);
+        x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w;
+        x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+    }
+}
+
+// Magnitude key in the histogram's domain: bf16 -> 15-bit key, fp32 -> 31-bit.
+template <qg_dtype DT>
+__device__ __forceinline__ uint32_t mag_key(float x) {
+    if constexpr (DT == QG_BF16) return (__float_as_uint(x) >> 16) & 0x7FFFu;
+    else return __float_as_uint(x) & 0x7FFFFFFFu;
+}
+
+template <qg_dtype DT>
+__device__ __forceinline__ float key_to_float(uint32_t key) {
+    if constexpr (DT == QG_BF16) return __uint_as_float(key << 16);
+    else return __uint_as_float(key);
+}
+
+// Keys at or above this are Inf/NaN.
+template <qg_dtype DT>
+__device__ __forceinline__ uint32_t nonfinite_key() {
+    if constexpr (DT == QG_BF16) return 0x7F80u;
+    else return 0x7F800000u;
+}
+
+__device__ __forceinline__ int warp_inclusive_scan(int v) {
+    const int lane = threadIdx.x & 31;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        int t = __shfl_up_sync(0xFFFFFFFFu, v, d);
+        if (lane >= d) v += t;
+    }
+    return v;
+}
+
+__device__ __forceinline__ uint32_t warp_max_u32(uint32_t v) {
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) v = max(v, __shfl_xor_sync(0xFFFFFFFFu, v, d));
+    return v;
+}
+
+#endif  // __CUDACC__
+
+// Pointers into a workspace for the threshold / clamp passes.
+struct ActBuffers {
+    uint32_t* status;
+    Counters* ctr;
+    uint32_t* hist1;
+    uint32_t* hist2;
+    uint32_t* rowmax;
+    uint32_t* rowcnt;
+    int32_t *st_row, *st_rank, *st_col;
+    double* st_val;
+    int64_t cap;
+};
+
+// Launch sequences (kernel files) used by the C ABI layer.
+void launch_zero_u32(uint32_t* p, int64_t n, cudaStream_t s);
+void launch_e2m1_encode(const float* x, int64_t n, uint8_t* packed, cudaStream_t s);
+void launch_quantize_rows(const void* A, qg_dtype dt, int64_t M, int64_t K, int64_t lda,
+                          uint8_t* codes, float* scales, cudaStream_t s);
+void launch_quantize_cols(const void* W, qg_dtype dt, int64_t K, int64_t N, int64_t ldw,
+                          uint8_t* codesT, float* scales, uint32_t* colmax, cudaStream_t s);
+void launch_spmm(const qg_csr* dA, int64_t M, const void* W, qg_dtype dt, int64_t N, int64_t ldw,
+                 float* C, cudaStream_t s);
+cudaError_t launch_fp4_gemm(const uint8_t* codesA, const float* sA, const uint8_t* codesWT,
+                            const float* sW, int64_t M, int64_t N, int64_t K, const float* C,
+                            void* Y, qg_dtype y_dtype, float* raw_acc, uint32_t* status,
+                            cudaStream_t s);
+cudaError_t run_quantize_act(const void* A, qg_dtype dt, int64_t M, int64_t K, int64_t lda,
+                             int64_t rank, const ActBuffers& b, uint8_t* codes, float* scales,
+                             const qg_csr* dA, float* T_out, cudaStream_t s);
+cudaError_t run_clamp_compensate(const void* A, qg_dtype dt, int64_t M, int64_t K, int64_t lda,
+                                 int64_t rank, const ActBuffers& b, void* A_c, const qg_csr* dA,
+                                 float* T_out, cudaStream_t s);
+cudaError_t act_setup();
+cudaError_t gemm_setup();
+
+// Number of SMs of the current device (cached per device id).
+int num_sms();
+
+}  // namespace qg

@@ -1,0 +1,219 @@
+// quantize.cu -- token-wise (row) and channel-wise (column) E2M1 quantizers
+// and the elementwise encoder.
+//
+// Method: QbitAI write-up of "Optimizing LLM Training Using FP4 Quantization"
+// (news.movedaos.com/post/4103): granularity paragraph (rows of A,
+// columns of W) and ScaleShift paragraph (scale by 6 / amax, round to the
+// nearest E2M1 value; ties to the even code).
+//
+// All kernels are HBM-bound streaming passes with 16-byte loads.
+#include "qg_internal.cuh"
+
+namespace qg {
+
+// --------------------------------------------------------------------------
+// Elementwise encoder: packed[i] = e2m1(x[2i]) | e2m1(x[2i+1]) << 4.
+__global__ void e2m1_encode_kernel(const float* __restrict__ x, int64_t n,
+                                   uint8_t* __restrict__ packed) {
+    const int64_t nchunk = n / 8;
+    for (int64_t c = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; c < nchunk;
+         c += (int64_t)gridDim.x * blockDim.x) {
+        float v[8];
+        load8<QG_F32>(x, c * 8, v);
+        reinterpret_cast<uint32_t*>(packed)[c] = e2m1x8(v);
+    }
+    // tail (n even, n % 8 != 0)
+    if (blockIdx.x == 0) {
+        for (int64_t i = nchunk * 8 + 2 * threadIdx.x; i < n; i += 2 * blockDim.x)
+            packed[i / 2] = (uint8_t)e2m1x2(x[i], x[i + 1]);
+    }
+}
+
+void launch_e2m1_encode(const float* x, int64_t n, uint8_t* packed, cudaStream_t s) {
+    int64_t nchunk = n / 8;
+    int blocks = (int)std::min<int64_t>((nchunk + 255) / 256, (int64_t)num_sms() * 16);
+    if (blocks < 1) blocks = 1;
+    e2m1_encode_kernel<<<blocks, 256, 0, s>>>(x, n, packed);
+}
+
+// --------------------------------------------------------------------------
+// Token-wise quantization without clamp.  One CTA per row; the row stays in
+// registers between the max reduction and the encode, so A is read once.
+constexpr int kRowThreads = 256;
+
+template <qg_dtype DT, int CPT>
+__global__ void __launch_bounds__(kRowThreads)
+quantize_rows_kernel(const void* __restrict__ A, int64_t lda, int K,
+                     uint8_t* __restrict__ codes, float* __restrict__ scales) {
+    const int64_t row = blockIdx.x;
+    const int nchunks = K / 8;
+    float x[CPT][8];
+    uint32_t kmax = 0;
+#pragma unroll
+    for (int i = 0; i < CPT; ++i) {
+        const int c = threadIdx.x + kRowThreads * i;
+        if (c < nchunks) {
+            load8<DT>(A, row * lda + (int64_t)c * 8, x[i]);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) kmax = max(kmax, key_of(x[i][e]));
+        }
+    }
+    __shared__ uint32_t red[kRowThreads / 32];
+    kmax = warp_max_u32(kmax);
+    if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = kmax;
+    __syncthreads();
+    uint32_t m = 0;
+#pragma unroll
+    for (int w = 0; w < kRowThreads / 32; ++w) m = max(m, red[w]);
+    float r, s;
+    scale_factors(__uint_as_float(m), r, s);
+    if (threadIdx.x == 0) scales[row] = s;
+    uint32_t* out = reinterpret_cast<uint32_t*>(codes + row * (int64_t)(K / 2));
+#pragma unroll
+    for (int i = 0; i < CPT; ++i) {
+        const int c = threadIdx.x + kRowThreads * i;
+        if (c < nchunks) {
+            float y[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) y[e] = __fmul_rn(x[i][e], r);
+            out[c] = e2m1x8(y);
+        }
+    }
+}
+
+template <qg_dtype DT>
+static void launch_rows_dt(const void* A, int64_t M, int64_t K, int64_t lda, uint8_t* codes,
+                           float* scales, cudaStream_t s) {
+    const int64_t nchunks = K / 8;
+    const int cpt = (int)((nchunks + kRowThreads - 1) / kRowThreads);
+    dim3 grid((unsigned)M);
+    if (cpt <= 1) quantize_rows_kernel<DT, 1><<<grid, kRowThreads, 0, s>>>(A, lda, (int)K, codes, scales);
+    else if (cpt <= 2) quantize_rows_kernel<DT, 2><<<grid, kRowThreads, 0, s>>>(A, lda, (int)K, codes, scales);
+    else if (cpt <= 4) quantize_rows_kernel<DT, 4><<<grid, kRowThreads, 0, s>>>(A, lda, (int)K, codes, scales);
+    else quantize_rows_kernel<DT, 8><<<grid, kRowThreads, 0, s>>>(A, lda, (int)K, codes, scales);
+}
+
+void launch_quantize_rows(const void* A, qg_dtype dt, int64_t M, int64_t K, int64_t lda,
+                          uint8_t* codes, float* scales, cudaStream_t s) {
+    if (dt == QG_BF16) launch_rows_dt<QG_BF16>(A, M, K, lda, codes, scales, s);
+    else launch_rows_dt<QG_F32>(A, M, K, lda, codes, scales, s);
+}
+
+// --------------------------------------------------------------------------
+// Channel-wise quantization of W (K x N row-major) into codesT (N x K/2).
+// Pass 1: column maxima (split over K, combined with atomicMax on the keys).
+// Pass 2: a 32 (k) x 256 (n) tile goes through shared memory and each thread
+//         encodes one column's 32 values into 16 output bytes.
+template <qg_dtype DT>
+__device__ __forceinline__ float load1(const void* base, int64_t idx) {
+    if constexpr (DT == QG_BF16)
+        return __uint_as_float((uint32_t)static_cast<const uint16_t*>(base)[idx] << 16);
+    else
+        return static_cast<const float*>(base)[idx];
+}
+
+template <qg_dtype DT>
+__global__ void __launch_bounds__(256)
+colmax_kernel(const void* __restrict__ W, int64_t ldw, int K, int N, int rows_per_split,
+              uint32_t* __restrict__ colmax) {
+    const int c = blockIdx.x * 256 + threadIdx.x;  // chunk of 8 columns
+    const int n0 = c * 8;
+    if (n0 >= N) return;
+    const int k0 = blockIdx.y * rows_per_split;
+    const int k1 = min(K, k0 + rows_per_split);
+    uint32_t m[8] = {0, 0, 0, 0, 0, 0, 0, 0};
+    const bool vec = (n0 + 8 <= N) && ((ldw & 7) == 0 || DT == QG_F32) && ((ldw & 3) == 0);
+    for (int k = k0; k < k1; ++k) {
+        float x[8];
+        if (vec) {
+            load8<DT>(W, (int64_t)k * ldw + n0, x);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] = (n0 + e < N) ? load1<DT>(W, (int64_t)k * ldw + n0 + e) : 0.0f;
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) m[e] = max(m[e], key_of(x[e]));
+    }
+#pragma unroll
+    for (int e = 0; e < 8; ++e)
+        if (n0 + e < N && m[e] != 0) atomicMax(&colmax[n0 + e], m[e]);
+}
+
+constexpr int kColTileK = 32;
+constexpr int kColTileN = 256;
+
+template <qg_dtype DT>
+__global__ void __launch_bounds__(256)
+quantize_cols_kernel(const void* __restrict__ W, int64_t ldw, int K, int N,
+                     const uint32_t* __restrict__ colmax, uint8_t* __restrict__ codesT,
+                     float* __restrict__ scales) {
+    __shared__ float tile[kColTileK][kColTileN];
+    const int n_base = blockIdx.x * kColTileN;
+    const int k_base = blockIdx.y * kColTileK;
+    const int t = threadIdx.x;
+    // load: warp w covers rows w, w + 8, ...; lane covers 8 consecutive columns
+    const int lane = t & 31, warp = t >> 5;
+    const int nc = n_base + lane * 8;
+    const bool vec = (nc + 8 <= N) && ((ldw & 7) == 0 || DT == QG_F32) && ((ldw & 3) == 0);
+    for (int kr = warp; kr < kColTileK; kr += 8) {
+        const int k = k_base + kr;
+        float x[8];
+        if (vec) {
+            load8<DT>(W, (int64_t)k * ldw + nc, x);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) x[e] = (nc + e < N) ? load1<DT>(W, (int64_t)k * ldw + nc + e) : 0.0f;
+        }
+        float4* dst = reinterpret_cast<float4*>(&tile[kr][lane * 8]);
+        dst[0] = make_float4(x[0], x[1], x[2], x[3]);
+        dst[1] = make_float4(x[4], x[5], x[6], x[7]);
+    }
+    __syncthreads();
+    const int n = n_base + t;
+    if (n >= N) return;
+    float r, s;
+    scale_factors(__uint_as_float(colmax[n]), r, s);
+    if (blockIdx.y == 0) scales[n] = s;
+    uint32_t packed[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        float y[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) y[e] = __fmul_rn(tile[q * 8 + e][t], r);
+        packed[q] = e2m1x8(y);
+    }
+    uint4* dst = reinterpret_cast<uint4*>(codesT + (int64_t)n * (K / 2) + k_base / 2);
+    *dst = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+}
+
+__global__ void zero_u32_kernel(uint32_t* __restrict__ p, int64_t n) {
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x)
+        p[i] = 0u;
+}
+
+void launch_zero_u32(uint32_t* p, int64_t n, cudaStream_t s) {
+    int blocks = (int)std::min<int64_t>((n + 255) / 256, (int64_t)num_sms() * 4);
+    if (blocks < 1) blocks = 1;
+    zero_u32_kernel<<<blocks, 256, 0, s>>>(p, n);
+}
+
+void launch_quantize_cols(const void* W, qg_dtype dt, int64_t K, int64_t N, int64_t ldw,
+                          uint8_t* codesT, float* scales, uint32_t* colmax, cudaStream_t s) {
+    launch_zero_u32(colmax, N, s);
+    const int col_blocks = (int)((N + 2047) / 2048);
+    int splits = (int)std::max<int64_t>(1, std::min<int64_t>(K, (num_sms() * 8 + col_blocks - 1) / col_blocks));
+    const int rows_per = (int)((K + splits - 1) / splits);
+    splits = (int)((K + rows_per - 1) / rows_per);
+    dim3 g1(col_blocks, splits);
+    dim3 g2((unsigned)((N + kColTileN - 1) / kColTileN), (unsigned)(K / kColTileK));
+    if (dt == QG_BF16) {
+        colmax_kernel<QG_BF16><<<g1, 256, 0, s>>>(W, ldw, (int)K, (int)N, rows_per, colmax);
+        quantize_cols_kernel<QG_BF16><<<g2, 256, 0, s>>>(W, ldw, (int)K, (int)N, colmax, codesT, scales);
+    } else {
+        colmax_kernel<QG_F32><<<g1, 256, 0, s>>>(W, ldw, (int)K, (int)N, rows_per, colmax);
+        quantize_cols_kernel<QG_F32><<<g2, 256, 0, s>>>(W, ldw, (int)K, (int)N, colmax, codesT, scales);
+    }
+}
+
+}  // namespace qg

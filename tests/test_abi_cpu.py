@@ -1,0 +1,109 @@
+"""The C-ABI library without a GPU: it loads, exports every symbol that
+include/qgemm.h declares, and its host-only logic agrees with the oracle's
+rank convention and with the header's contracts."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import oracle
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "qgemm.h")
+
+
+def _header_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(qg_[a-z0-9_]+)\s*\(", text)))
+
+
+@pytest.fixture(scope="module")
+def qg():
+    import __graft_entry__
+    __graft_entry__.build()
+    import quantize_gemm_b200
+    return quantize_gemm_b200
+
+
+def test_header_declares_the_entry_points():
+    funcs = _header_functions()
+    for name in ("qg_quantize_rows", "qg_quantize_cols", "qg_clamp_compensate",
+                 "qg_quantize_act", "qg_spmm_correction", "qg_fp4_gemm", "qg_fp4_linear",
+                 "qg_sync_status", "qg_workspace_size"):
+        assert name in funcs
+
+
+def test_library_exports_every_declared_symbol(qg):
+    lib = ctypes.CDLL(qg.LIB_PATH)
+    for name in _header_functions():
+        assert hasattr(lib, name), f"{name} declared in qgemm.h but not exported"
+    assert set(_header_functions()) == set(qg.EXPORTED)
+
+
+def test_rank_convention_matches_oracle(qg):
+    for n in (1, 2, 10, 12, 131072, 4096 * 2048, 16384 * 11008):
+        for alpha in (1e-12, 0.1, 0.5, 0.9, 0.95, 0.99, 0.999, 0.9999, 1.0):
+            assert qg.qg_quantile_rank(alpha, n) == oracle.quantile_rank(alpha, n)
+            assert qg.qg_nnz_capacity(n, alpha) == oracle.nnz_capacity(n, alpha)
+
+
+def test_workspace_sizes(qg):
+    for op in range(7):
+        for (M, K, N, dt, a) in ((1, 32, 1, 0, 1.0), (256, 512, 512, 0, 0.99),
+                                 (4096, 2048, 5504, 1, 0.99), (16384, 11008, 4096, 1, 0.999)):
+            s = qg.qg_workspace_size(op, M, K, N, dt, a)
+            assert s >= 256 and s % 256 == 0
+    # the layer's workspace holds at least the fp32 correction and the CSR
+    M, K, N = 4096, 2048, 5504
+    s = qg.qg_workspace_size(qg.QG_OP_FP4_LINEAR, M, K, N, qg.QG_BF16, 0.99)
+    cap = qg.qg_nnz_capacity(M * K, 0.99)
+    assert s >= 4 * M * N + 12 * cap + M * K // 2
+    # staging grows as alpha falls
+    a = qg.qg_workspace_size(qg.QG_OP_QUANTIZE_ACT, M, K, 1, qg.QG_BF16, 0.999)
+    b = qg.qg_workspace_size(qg.QG_OP_QUANTIZE_ACT, M, K, 1, qg.QG_BF16, 0.99)
+    assert b > a
+
+
+def test_status_strings(qg):
+    for s in range(8):
+        assert qg.qg_status_string(s)
+    assert qg.qg_status_string(99) == "unknown status"
+
+
+def test_host_argument_checks_need_no_device(qg):
+    """Argument errors come back before any CUDA call is made."""
+    lib = qg._lib
+    P = ctypes.c_void_p
+    fake = P(1 << 20)   # never dereferenced: the checks reject the call first
+    # K not a multiple of 32
+    assert lib.qg_quantize_rows(fake, 1, 4, 48, 48, fake, fake, fake, 1 << 20, None) == \
+        qg.QG_ERR_UNSUPPORTED_SHAPE
+    # K too large
+    assert lib.qg_quantize_rows(fake, 1, 4, 16416, 16416, fake, fake, fake, 1 << 20, None) == \
+        qg.QG_ERR_UNSUPPORTED_SHAPE
+    # bad dtype
+    assert lib.qg_quantize_rows(fake, 7, 4, 64, 64, fake, fake, fake, 1 << 20, None) == \
+        qg.QG_ERR_INVALID_ARG
+    # misaligned A
+    assert lib.qg_quantize_rows(P((1 << 20) + 4), 1, 4, 64, 64, fake, fake, fake, 1 << 20,
+                                None) == qg.QG_ERR_INVALID_ARG
+    # lda smaller than K
+    assert lib.qg_quantize_rows(fake, 1, 4, 64, 32, fake, fake, fake, 1 << 20, None) == \
+        qg.QG_ERR_INVALID_ARG
+    # workspace too small
+    assert lib.qg_quantize_rows(fake, 1, 4, 64, 64, fake, fake, fake, 16, None) == \
+        qg.QG_ERR_WORKSPACE
+    # alpha out of range
+    csr = qg._Csr(1 << 20, 1 << 20, 1 << 20, 1000, 1 << 20)
+    for alpha in (0.0, -0.5, 1.5, float("nan")):
+        assert lib.qg_quantize_act(fake, 1, 4, 64, 64, alpha, fake, fake, ctypes.byref(csr),
+                                   fake, fake, 1 << 30, None) == qg.QG_ERR_INVALID_ARG
+    # CSR capacity below the bound n - ceil(alpha n)
+    small = qg._Csr(1 << 20, 1 << 20, 1 << 20, 1, 1 << 20)
+    assert lib.qg_quantize_act(fake, 1, 4, 64, 64, 0.5, fake, fake, ctypes.byref(small), fake,
+                               fake, 1 << 30, None) == qg.QG_ERR_INVALID_ARG
+    # GEMM with neither Y nor raw_acc
+    assert lib.qg_fp4_gemm(fake, fake, fake, fake, 128, 128, 256, None, None, 0, None, fake,
+                           1 << 20, None) == qg.QG_ERR_INVALID_ARG

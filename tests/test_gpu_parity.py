@@ -1,0 +1,369 @@
+"""CUDA path (through the C ABI) against the CPU oracle, element by element.
+
+Bars (from the layer's definition; see the header of include/qgemm.h):
+* codes, scales, threshold T, the CSR of dA and the raw FP4 accumulator are
+  bit-exact (integer / exactly representable results);
+* the correction C = dA . W (fp32 FMA chain) is within (n + 2) * 2^-24 of the
+  absolute sum |dA| . |W| per element, n = non-zeros in the row;
+* Y (fp32) satisfies max |Y - Yo| / max(|Yo|, 1e-3 * rms(Yo)) <= 1e-3 against
+  the oracle's fp64 evaluation of the same quantized operands;
+* Y (bf16) is within one bf16 ulp of Yo.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle_pins import unpack
+from workloads import WORKLOADS, make_layer_inputs, make_matrix
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def qg():
+    if not torch.cuda.is_available():
+        pytest.skip("needs a CUDA device")
+    import __graft_entry__
+    __graft_entry__.build()
+    import quantize_gemm_b200
+    torch.cuda.set_device(0)
+    return quantize_gemm_b200
+
+
+def _np(t):
+    return t.detach().cpu().numpy()
+
+
+def y_rel_err(Y, Yo):
+    Y = np.asarray(Y, dtype=np.float64)
+    floor = 1e-3 * np.sqrt(np.mean(Yo ** 2)) if Yo.size else 0.0
+    floor = max(floor, 1e-30)
+    return float(np.max(np.abs(Y - Yo) / np.maximum(np.abs(Yo), floor))) if Yo.size else 0.0
+
+
+def bf16_ulp(x):
+    x = np.abs(np.asarray(x, dtype=np.float64))
+    e = np.floor(np.log2(np.maximum(x, 2.0 ** -126)))
+    return 2.0 ** (e - 7)
+
+
+# ------------------------------------------------------------------ encoder
+def test_e2m1_exhaustive_all_fp32_patterns(qg):
+    """Every one of the 2^32 fp32 bit patterns (NaN patterns -> 0 on both
+    sides, since NaN is rejected before encoding)."""
+    ws = qg.Workspace(qg.QG_OP_QUANTIZE_ROWS, 1, 32, device="cuda")
+    CH = 1 << 28
+    for c in range(1 << 4):
+        start = c * CH
+        b = torch.arange(start, start + CH, dtype=torch.int64, device="cuda")
+        b = torch.where(b >= (1 << 31), b - (1 << 32), b).to(torch.int32)
+        x = b.view(torch.float32)
+        x = torch.where(torch.isnan(x), torch.zeros_like(x), x)
+        got = _np(qg.e2m1_encode(x, ws))
+        del b, x
+        want = oracle.e2m1_encode_bits_packed(start, CH)
+        bad = np.nonzero(got != want)[0]
+        assert bad.size == 0, (hex(start + 2 * int(bad[0])), got[bad[0]], want[bad[0]])
+    qg.check_status(ws)
+
+
+# ------------------------------------------------------------------ quantizers
+def _special_rows(K, dtype):
+    A = torch.zeros((6, K), dtype=torch.float32)
+    A[1] = -0.0
+    A[2, :] = 1e-45
+    A[2, 3] = -3e-45
+    A[3, :] = torch.linspace(-7, 7, K)
+    A[4, :] = 1e30
+    A[4, 1::2] = -2.5e30
+    # exact ties after scaling by r = 1 (amax = 6)
+    ties = torch.tensor([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0, 6.0])
+    A[5, :] = ties.repeat(K // 8) * torch.where(torch.arange(K) % 3 == 0, -1.0, 1.0)
+    return A.to(dtype)
+
+
+ROW_CASES = [
+    (1, 32, torch.float32), (3, 64, torch.bfloat16), (257, 512, torch.float32),
+    (100, 1056, torch.bfloat16), (64, 16384, torch.bfloat16), (32, 16384, torch.float32),
+    (129, 2048, torch.bfloat16), (7, 4128, torch.float32),
+]
+
+
+@pytest.mark.parametrize("M,K,dtype", ROW_CASES)
+def test_quantize_rows(qg, M, K, dtype):
+    A = make_matrix((M, K), ("student_t", 3), seed=M * 7 + K, device="cuda", dtype=dtype,
+                    scale=2.0)
+    codes, scales = qg.quantize_rows(A)
+    oc, os_ = oracle.quantize_rows(A.cpu())
+    assert np.array_equal(_np(scales), os_)
+    assert np.array_equal(_np(codes), oc)
+
+
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_quantize_rows_special_values(qg, dtype):
+    A = _special_rows(256, dtype).cuda()
+    codes, scales = qg.quantize_rows(A)
+    oc, os_ = oracle.quantize_rows(A.cpu())
+    assert np.array_equal(_np(scales), os_)
+    assert np.array_equal(_np(codes), oc)
+
+
+def test_quantize_rows_strided(qg):
+    base = make_matrix((40, 1024), seed=3, device="cuda", dtype=torch.bfloat16)
+    A = base[:, :512]            # lda = 1024 > K = 512
+    codes, scales = qg.quantize_rows(A)
+    oc, os_ = oracle.quantize_rows(A.contiguous().cpu())
+    assert np.array_equal(_np(codes), oc) and np.array_equal(_np(scales), os_)
+
+
+COL_CASES = [
+    (32, 1, torch.float32), (64, 7, torch.bfloat16), (512, 512, torch.float32),
+    (2048, 5504, torch.bfloat16), (5504, 2048, torch.bfloat16), (16384, 40, torch.bfloat16),
+    (96, 300, torch.float32),
+]
+
+
+@pytest.mark.parametrize("K,N,dtype", COL_CASES)
+def test_quantize_cols(qg, K, N, dtype):
+    W = make_matrix((K, N), seed=K + N, device="cuda", dtype=dtype, scale=0.02)
+    codesT, t = qg.quantize_cols(W)
+    oT, ot = oracle.quantize_cols(W.cpu())
+    assert np.array_equal(_np(t), ot)
+    assert np.array_equal(_np(codesT), oT)
+
+
+def test_quantize_cols_special_values(qg):
+    W = _special_rows(256, torch.float32).t().contiguous().cuda()   # columns = special rows
+    codesT, t = qg.quantize_cols(W)
+    oT, ot = oracle.quantize_cols(W.cpu())
+    assert np.array_equal(_np(t), ot) and np.array_equal(_np(codesT), oT)
+
+
+# ------------------------------------------------------------------ threshold + clamp
+def _act_inputs(name):
+    if name == "tiny":
+        return make_layer_inputs("tiny", 0, device="cuda")[0], 0.99
+    if name == "llama1.3b_attn_m512":
+        return make_layer_inputs("llama1.3b", 0, device="cuda", M=512)[0], 0.99
+    if name == "llama7b_down_m256":
+        return make_layer_inputs("llama7b", 4, device="cuda", M=256)[0], 0.99
+    if name == "llama13b_qkv_m128":
+        return make_layer_inputs("llama13b", 1, device="cuda", M=128)[0], 0.999
+    if name == "ragged_k1056_fp32":
+        return make_matrix((33, 1056), ("student_t", 3), seed=5, device="cuda"), 0.95
+    if name == "no_clamp":
+        return make_matrix((64, 512), seed=6, device="cuda", dtype=torch.bfloat16), 1.0
+    if name == "clamp_almost_all":
+        return make_matrix((16, 256), seed=7, device="cuda", dtype=torch.bfloat16), 1e-6
+    if name == "ties_at_T":
+        A = torch.ones((8, 64), device="cuda", dtype=torch.bfloat16)
+        A[::2, ::3] = -2.0
+        return A, 0.9
+    if name == "single_row":
+        return make_matrix((1, 8192), ("student_t", 4), seed=8, device="cuda",
+                           dtype=torch.bfloat16), 0.99
+    if name == "fp32_heavy_tail":
+        return make_matrix((200, 640), ("student_t", 3), seed=9, device="cuda",
+                           outliers=("random_entries", 0.002, 1e3)), 0.997
+    raise KeyError(name)
+
+
+ACT_CASES = ["tiny", "llama1.3b_attn_m512", "llama7b_down_m256", "llama13b_qkv_m128",
+             "ragged_k1056_fp32", "no_clamp", "clamp_almost_all", "ties_at_T", "single_row",
+             "fp32_heavy_tail"]
+
+
+def _check_act(qg, A, alpha, codes, scales, csr, T, exp):
+    assert float(_np(T)[0]) == exp["T"]
+    rp, col, val = csr.to_host()
+    assert np.array_equal(rp, exp["row_ptr"])
+    assert np.array_equal(col, exp["col"])
+    assert np.array_equal(val, exp["val"])
+    if codes is not None:
+        assert np.array_equal(_np(scales), exp["scales"])
+        assert np.array_equal(_np(codes), exp["codes"])
+
+
+@pytest.mark.parametrize("case", ACT_CASES)
+def test_quantize_act(qg, case):
+    A, alpha = _act_inputs(case)
+    M, K = A.shape
+    ws = qg.Workspace(qg.QG_OP_QUANTIZE_ACT, M, K, 1, qg._dt(A), alpha)
+    codes, scales, csr, T = qg.quantize_act(A, alpha, ws=ws)
+    qg.check_status(ws, case)
+    exp = oracle.quantize_act(A.cpu(), alpha)
+    _check_act(qg, A, alpha, codes, scales, csr, T, exp)
+    # same workspace again: identical bytes (canonical CSR, no stale state)
+    codes2, scales2, csr2, T2 = qg.quantize_act(A, alpha, ws=ws)
+    qg.check_status(ws, case)
+    _check_act(qg, A, alpha, codes2, scales2, csr2, T2, exp)
+
+
+@pytest.mark.parametrize("case", ["tiny", "llama7b_down_m256", "ragged_k1056_fp32", "ties_at_T"])
+def test_clamp_compensate(qg, case):
+    A, alpha = _act_inputs(case)
+    M, K = A.shape
+    ws = qg.Workspace(qg.QG_OP_CLAMP_COMPENSATE, M, K, 1, qg._dt(A), alpha)
+    A_c, csr, T = qg.clamp_compensate(A, alpha, ws=ws)
+    qg.check_status(ws, case)
+    Th = oracle.threshold(A.cpu(), alpha)
+    oa_c, orp, ocol, oval = oracle.clamp_compensate(A.cpu(), Th)
+    assert float(_np(T)[0]) == Th
+    assert np.array_equal(oracle.as_f32(A_c.cpu()), oa_c)
+    rp, col, val = csr.to_host()
+    assert np.array_equal(rp, orp) and np.array_equal(col, ocol) and np.array_equal(val, oval)
+    # the CSR without the clamped copy
+    _, csr2, _ = qg.clamp_compensate(A, alpha, ws=ws, want_clamped=False)
+    qg.check_status(ws, case)
+    rp2, col2, val2 = csr2.to_host()
+    assert np.array_equal(rp2, orp) and np.array_equal(col2, ocol) and np.array_equal(val2, oval)
+
+
+@pytest.mark.parametrize("bad", [float("nan"), float("inf"), float("-inf")])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_nonfinite_input_reported(qg, bad, dtype):
+    A = make_matrix((16, 256), seed=10, device="cuda", dtype=dtype)
+    A[5, 17] = bad
+    ws = qg.Workspace(qg.QG_OP_QUANTIZE_ACT, 16, 256, 1, qg._dt(A), 0.99)
+    qg.quantize_act(A, 0.99, ws=ws)
+    assert ws.sync_status() == qg.QG_ERR_NONFINITE
+    # the status is cleared by the read; a clean call on the same workspace is OK
+    A[5, 17] = 1.0
+    qg.quantize_act(A, 0.99, ws=ws)
+    assert ws.sync_status() == qg.QG_OK
+
+
+# ------------------------------------------------------------------ SpMM correction
+@pytest.mark.parametrize("case,N,wdtype", [("tiny", 512, torch.float32),
+                                            ("llama1.3b_attn_m512", 2048, torch.bfloat16),
+                                            ("ragged_k1056_fp32", 100, torch.float32),
+                                            ("clamp_almost_all", 264, torch.bfloat16)])
+def test_spmm_correction(qg, case, N, wdtype):
+    A, alpha = _act_inputs(case)
+    M, K = A.shape
+    W = make_matrix((K, N), seed=11, device="cuda", dtype=wdtype, scale=0.02)
+    _, csr, _ = qg.clamp_compensate(A, alpha, want_clamped=False)
+    C = _np(qg.spmm_correction(csr, M, W)).astype(np.float64)
+    rp, col, val = csr.to_host()
+    Co = oracle.spmm(rp, col, val, W.cpu())
+    S = oracle.spmm(rp, col, np.abs(val), W.cpu().abs())
+    n = np.diff(rp).astype(np.float64)[:, None]
+    bound = (n + 2) * 2.0 ** -24 * S
+    assert np.all(np.abs(C - Co) <= bound), float(np.max(np.abs(C - Co) - bound))
+
+
+# ------------------------------------------------------------------ FP4 GEMM
+GEMM_SHAPES = [(128, 256, 256), (1, 8, 32), (129, 257, 288), (300, 600, 1024),
+               (1024, 1024, 4096), (256, 512, 16384), (4096, 2048, 2048), (513, 5504, 2048)]
+
+
+def _rand_codes(rows, K, seed):
+    g = np.random.default_rng(seed)
+    return g.integers(0, 256, size=(rows, K // 2), dtype=np.uint8)
+
+
+@pytest.mark.parametrize("M,N,K", GEMM_SHAPES)
+def test_fp4_gemm_raw_accumulator_bit_exact(qg, M, N, K):
+    cA = _rand_codes(M, K, M + K)
+    cW = _rand_codes(N, K, N + 3 * K)
+    sA = np.ones(M, np.float32)
+    sW = np.ones(N, np.float32)
+    Y, acc = qg.fp4_gemm(torch.from_numpy(cA).cuda(), torch.from_numpy(sA).cuda(),
+                         torch.from_numpy(cW).cuda(), torch.from_numpy(sW).cuda(), K, raw=True)
+    acc = _np(acc)
+    rows = np.arange(M) if M * N * K <= (1 << 31) else \
+        np.unique(np.concatenate([np.random.default_rng(1).integers(0, M, 48), [0, M - 1]]))
+    want = oracle.gemm_acc(cA, cW, K, rows=rows)
+    assert np.array_equal(acc[rows], want.astype(np.float32))
+    assert np.array_equal(acc[rows].astype(np.float64), want)   # exact in fp32
+
+
+@pytest.mark.parametrize("M,N,K", [(128, 256, 256), (129, 257, 288), (300, 600, 1024),
+                                   (513, 5504, 2048)])
+@pytest.mark.parametrize("with_c", [False, True])
+def test_fp4_gemm_epilogue_fp32(qg, M, N, K, with_c):
+    g = np.random.default_rng(M + N)
+    cA, cW = _rand_codes(M, K, 5 + M), _rand_codes(N, K, 6 + N)
+    sA = (g.random(M) * 0.1 + 1e-3).astype(np.float32)
+    sW = (g.random(N) * 0.01 + 1e-4).astype(np.float32)
+    C = (g.standard_normal((M, N)) * 0.5).astype(np.float32) if with_c else None
+    Y = qg.fp4_gemm(torch.from_numpy(cA).cuda(), torch.from_numpy(sA).cuda(),
+                    torch.from_numpy(cW).cuda(), torch.from_numpy(sW).cuda(), K,
+                    C=torch.from_numpy(C).cuda() if with_c else None)
+    acc = oracle.gemm_acc(cA, cW, K)
+    Yo = acc * sA.astype(np.float64)[:, None] * sW.astype(np.float64)[None, :]
+    if with_c:
+        Yo = Yo + C.astype(np.float64)
+    assert y_rel_err(_np(Y), Yo) <= 1e-3
+
+
+def test_fp4_gemm_epilogue_bf16(qg):
+    M, N, K = 300, 600, 1024
+    g = np.random.default_rng(2)
+    cA, cW = _rand_codes(M, K, 21), _rand_codes(N, K, 22)
+    sA = (g.random(M) * 0.1 + 1e-3).astype(np.float32)
+    sW = (g.random(N) * 0.01 + 1e-4).astype(np.float32)
+    C = (g.standard_normal((M, N)) * 0.5).astype(np.float32)
+    Y = qg.fp4_gemm(torch.from_numpy(cA).cuda(), torch.from_numpy(sA).cuda(),
+                    torch.from_numpy(cW).cuda(), torch.from_numpy(sW).cuda(), K,
+                    C=torch.from_numpy(C).cuda(), out_dtype=torch.bfloat16)
+    acc = oracle.gemm_acc(cA, cW, K)
+    Yo = acc * sA.astype(np.float64)[:, None] * sW.astype(np.float64)[None, :] + C
+    err = np.abs(_np(Y.float()).astype(np.float64) - Yo)
+    assert np.all(err <= bf16_ulp(Yo))
+
+
+# ------------------------------------------------------------------ the layer
+def _linear_oracle(A, W, alpha, rows=None):
+    act = oracle.quantize_act(A.cpu(), alpha)
+    oT, ot = oracle.quantize_cols(W.cpu())
+    acc = oracle.gemm_acc(act["codes"], oT, A.shape[1], rows=rows)
+    return oracle.linear_y(acc, act["scales"], ot, act["row_ptr"], act["col"], act["val"],
+                           W.cpu(), rows=rows), act
+
+
+LAYER_CASES = [("tiny", 0, None), ("llama1.3b", 0, 256), ("llama1.3b", 1, 256),
+               ("llama1.3b", 2, 256), ("llama7b", 4, 128), ("llama13b", 1, 128)]
+
+
+@pytest.mark.parametrize("wl,layer,M", LAYER_CASES)
+def test_fp4_linear_small(qg, wl, layer, M):
+    A, W = make_layer_inputs(wl, layer, device="cuda", M=M)
+    alpha = WORKLOADS[wl].alphas[0]
+    codesT, t = qg.quantize_cols(W)
+    ws = qg.Workspace(qg.QG_OP_FP4_LINEAR, A.shape[0], A.shape[1], W.shape[1], qg._dt(A), alpha)
+    Y = qg.fp4_linear(A, codesT, t, W, alpha, ws=ws)
+    qg.check_status(ws)
+    Yo, _ = _linear_oracle(A, W, alpha)
+    assert y_rel_err(_np(Y), Yo) <= 1e-3
+    Yb = qg.fp4_linear(A, codesT, t, W, alpha, out_dtype=torch.bfloat16, ws=ws)
+    qg.check_status(ws)
+    rms = np.sqrt(np.mean(Yo ** 2))
+    assert np.all(np.abs(_np(Yb.float()).astype(np.float64) - Yo) <= bf16_ulp(Yo) + 1e-6 * rms)
+
+
+@pytest.mark.parametrize("wl,layer", [("llama1.3b", 1), ("llama7b", 1), ("llama13b", 4)])
+def test_fp4_linear_full_size_sampled(qg, wl, layer):
+    """Full BASELINE sizes, the launch configuration the benchmark times:
+    T, codes, scales and dA checked exactly over the whole tensor, Y on a
+    sample of rows computed by the oracle one by one."""
+    A, W = make_layer_inputs(wl, layer, device="cuda")
+    alpha = WORKLOADS[wl].alphas[0]
+    M, K = A.shape
+    N = W.shape[1]
+    codesT, t = qg.quantize_cols(W)
+    ws = qg.Workspace(qg.QG_OP_FP4_LINEAR, M, K, N, qg._dt(A), alpha)
+    Y = qg.fp4_linear(A, codesT, t, W, alpha, ws=ws)
+    qg.check_status(ws)
+    codes, scales, csr, T = qg.quantize_act(A, alpha)
+    rows = np.unique(np.concatenate([np.random.default_rng(M + N).integers(0, M, 24), [0, M - 1]]))
+    Yo, act = _linear_oracle(A, W, alpha, rows=rows)
+    assert float(_np(T)[0]) == act["T"]
+    assert np.array_equal(_np(codes), act["codes"]) and np.array_equal(_np(scales), act["scales"])
+    rp, col, val = csr.to_host()
+    assert np.array_equal(rp, act["row_ptr"]) and np.array_equal(col, act["col"])
+    assert np.array_equal(val, act["val"])
+    oT, ot = oracle.quantize_cols(W.cpu())
+    assert np.array_equal(_np(codesT), oT) and np.array_equal(_np(t), ot)
+    assert y_rel_err(_np(Y)[rows], Yo) <= 1e-3
