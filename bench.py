@@ -1,0 +1,473 @@
+"""Benchmark of the FP4 quantized linear layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference] [--no-e2e] [--no-cpu-baseline]
+
+A step is one forward pass of every linear layer of the workload (default:
+the LLaMA-1.3B-shaped linears, M = 4096 tokens, bf16): for each layer the
+weight is quantized column-wise (the method quantizes W and A at the start of
+every linear forward), then the activation goes through the fused threshold /
+clamp / quantize pass, the dA . W correction and the FP4 GEMM with its
+dequantization epilogue.  Inputs are synthetic (seeded, see workloads/) and
+resident in HBM before timing; L2 is flushed (256 MiB write) between timed
+steps.  One JSON line is printed by rank 0.
+
+Multi-GPU: one process per GPU (torchrun); every rank runs its own replica of
+the workload (weak scaling, no data-path collective); the timed region is
+bracketed by barrier + synchronize and the max over ranks is reported.
+
+--impl reference times the CPU oracle (the plain C restatement of the method)
+on the host cores, on a bounded sample of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+METRIC = "FP4 linear-layer TFLOPS & tokens/s (1 B200); quantizer GB/s; % roofline"
+L2_FLUSH_BYTES = 256 << 20
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return dict(hbm_gbs=float(p["hbm_gbs"]), bf16_tflops=float(p["bf16_tflops"]),
+                    bf16_tflops_sustained=float(p.get("bf16_tflops_sustained", p["bf16_tflops"])),
+                    sm_max_mhz=float(p.get("sm_max_mhz", 1965.0)), source="measured")
+    return dict(hbm_gbs=6650.0, bf16_tflops=1590.0, bf16_tflops_sustained=1400.0,
+                sm_max_mhz=1965.0, source="fallback")
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = os.path.join("/tmp", f"qg_clocks_{os.getpid()}.csv")
+
+    def start(self):
+        try:
+            self.f = open(self.path, "w")
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.f.close()
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        with open(self.path) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 9:
+                    continue
+                try:
+                    sm.append(float(parts[1]))
+                    smax.append(float(parts[2]))
+                except ValueError:
+                    continue
+                for name, v in zip(names, parts[5:9]):
+                    if v.lower() == "active":
+                        reasons.add(name)
+        os.remove(self.path)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": max(smax),
+                "samples": len(sm), "reasons": sorted(reasons)}
+
+
+# ------------------------------------------------------------------ our arm
+class Layer:
+    def __init__(self, qg, wl, li, device):
+        from workloads import make_layer_inputs
+        self.name = wl.layers[li].name
+        self.A, self.W = make_layer_inputs(wl, li, device=device)
+        self.alpha = wl.alphas[0]
+        M, K = self.A.shape
+        N = self.W.shape[1]
+        self.M, self.K, self.N = M, K, N
+        dt = qg._dt(self.A)
+        cap = qg.qg_nnz_capacity(M * K, self.alpha)
+        self.codesT = torch.empty((N, K // 2), dtype=torch.uint8, device=device)
+        self.t = torch.empty(N, dtype=torch.float32, device=device)
+        self.codes = torch.empty((M, K // 2), dtype=torch.uint8, device=device)
+        self.s = torch.empty(M, dtype=torch.float32, device=device)
+        self.csr = qg.CSR.empty(M, cap, device=device)
+        self.T = torch.empty(1, dtype=torch.float32, device=device)
+        self.C = torch.empty((M, N), dtype=torch.float32, device=device)
+        self.Y = torch.empty((M, N), dtype=torch.float32, device=device)
+        self.ws_cols = qg.Workspace(qg.QG_OP_QUANTIZE_COLS, 1, K, N, dt, device=device)
+        self.ws_act = qg.Workspace(qg.QG_OP_QUANTIZE_ACT, M, K, 1, dt, self.alpha, device=device)
+        self.ws_spmm = qg.Workspace(qg.QG_OP_SPMM, M, K, N, dt, device=device)
+        self.ws_gemm = qg.Workspace(qg.QG_OP_FP4_GEMM, M, K, N, qg.QG_F32, device=device)
+        self.ws_lin = qg.Workspace(qg.QG_OP_FP4_LINEAR, M, K, N, dt, self.alpha, device=device)
+        self.flops = 2 * M * N * K
+        self.a_bytes = M * K * self.A.element_size()
+        self.w_bytes = K * N * self.W.element_size()
+
+    def workspaces(self):
+        return (self.ws_cols, self.ws_act, self.ws_spmm, self.ws_gemm, self.ws_lin)
+
+
+KERNELS = ("quantize_cols", "quantize_act", "spmm", "fp4_gemm")
+
+
+def run_step(qg, layers, ev=None):
+    """One pass of the hot path over every layer.  With `ev`, record events
+    around each of the four calls of each layer (same stream)."""
+    def _chk(st, where):
+        if st != qg.QG_OK:
+            raise qg.QGError(st, where)
+    for i, L in enumerate(layers):
+        if ev is not None:
+            ev[i][0].record()
+        _chk(qg.qg_quantize_cols(L.W, L.codesT, L.t, L.ws_cols), "quantize_cols")
+        if ev is not None:
+            ev[i][1].record()
+        _chk(qg.qg_quantize_act(L.A, L.alpha, L.codes, L.s, L.csr, L.T, L.ws_act), "quantize_act")
+        if ev is not None:
+            ev[i][2].record()
+        _chk(qg.qg_spmm_correction(L.csr, L.M, L.W, L.C, L.ws_spmm), "spmm")
+        if ev is not None:
+            ev[i][3].record()
+        _chk(qg.qg_fp4_gemm(L.codes, L.s, L.codesT, L.t, L.M, L.N, L.K, L.C, L.Y, None,
+                            L.ws_gemm), "fp4_gemm")
+        if ev is not None:
+            ev[i][4].record()
+
+
+def our_arm(args, rank, world, device):
+    import quantize_gemm_b200 as qg
+    from workloads import WORKLOADS
+    wl = WORKLOADS[args.workload]
+    peaks = _peaks()
+    layers = [Layer(qg, wl, i, device) for i in range(len(wl.layers))]
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    stream = torch.cuda.current_stream()
+
+    for _ in range(args.warmup):
+        run_step(qg, layers)
+    torch.cuda.synchronize()
+    for L in layers:
+        for ws in L.workspaces():
+            qg.check_status(ws, f"warm-up {L.name}")
+
+    n_l = len(layers)
+    ev_steps = [[[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(n_l)]
+                for _ in range(args.steps)]
+    launches0 = qg.qg_launch_count()
+    sampler = ClockSampler(torch.cuda.current_device() if world == 1 else int(os.environ.get("LOCAL_RANK", 0)))
+    sampler.start()
+    time.sleep(0.3)
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    for k in range(args.steps):
+        flush.fill_(k & 0xFF)           # L2 flush outside the step's events
+        run_step(qg, layers, ev_steps[k])
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    wall = time.perf_counter() - wall0
+    clocks = sampler.stop()
+    launches = qg.qg_launch_count() - launches0
+    for L in layers:
+        for ws in L.workspaces():
+            qg.check_status(ws, f"timed {L.name}")
+
+    # per step and per kernel device times (ms)
+    step_ms = [sum(ev[i][0].elapsed_time(ev[i][4]) for i in range(n_l)) for ev in ev_steps]
+    per_kernel = {k: [] for k in KERNELS}
+    per_kernel_layer = {k: [[] for _ in range(n_l)] for k in KERNELS}
+    for ev in ev_steps:
+        for i in range(n_l):
+            for j, k in enumerate(KERNELS):
+                t = ev[i][j].elapsed_time(ev[i][j + 1])
+                per_kernel_layer[k][i].append(t)
+        for k in KERNELS:
+            per_kernel[k].append(sum(per_kernel_layer[k][i][-1] for i in range(n_l)))
+    total_ms = sum(step_ms)
+    if world > 1:
+        t = torch.tensor([total_ms], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    ms_per_step = total_ms / args.steps
+    flops_step = sum(L.flops for L in layers)
+    tokens_step = wl.M          # tokens through the whole layer stream
+    value = world * flops_step * args.steps / (total_ms * 1e-3) / 1e12
+
+    # roofline of each kernel, per launch
+    sm_mhz = clocks.get("sm_mhz") or peaks["sm_max_mhz"]
+    n_sm = torch.cuda.get_device_properties(device).multi_processor_count
+    fp4_peak = 4.0 * peaks["bf16_tflops_sustained"]
+    alu_peak = n_sm * 128 * 2 * sm_mhz * 1e6 / 1e12
+    rows = {}
+    for k in KERNELS:
+        kms = sum(per_kernel[k]) / args.steps
+        algo = 0.0
+        if k == "fp4_gemm":
+            algo = sum(L.flops for L in layers) / 1e12
+            bound, unit, peak = "tensor", "TFLOP/s", fp4_peak
+        elif k == "spmm":
+            algo = sum(2 * int(L.csr.nnz.item()) * L.N for L in layers) / 1e12
+            bound, unit, peak = "alu", "TFLOP/s", alu_peak
+        elif k == "quantize_act":
+            algo = sum(2 * L.a_bytes + L.M * L.K / 2 + 4 * L.M + 16 * int(L.csr.nnz.item())
+                       + 4 * (L.M + 1) + 8 * L.M for L in layers) / 1e9
+            bound, unit, peak = "hbm", "GB/s", peaks["hbm_gbs"]
+        else:
+            algo = sum(2 * L.w_bytes + L.K * L.N / 2 + 4 * L.N for L in layers) / 1e9
+            bound, unit, peak = "hbm", "GB/s", peaks["hbm_gbs"]
+        achieved = algo / (kms * 1e-3) if kms > 0 else 0.0
+        rows[k] = {"bound": bound, "achieved": round(achieved, 2), "peak": round(peak, 1),
+                   "unit": unit, "frac": round(achieved / peak, 4), "ms_per_step": round(kms, 4)}
+    dominant = max(KERNELS, key=lambda k: rows[k]["ms_per_step"])
+    traffic = _ncu_traffic(dominant, args.workload)
+    roofline = dict(rows[dominant])
+    roofline.pop("ms_per_step")
+    roofline["kernel"] = dominant
+    roofline["traffic"] = traffic
+    roofline["peak_source"] = (f"{peaks['source']}: 4 x bf16 sustained {peaks['bf16_tflops_sustained']}"
+                               if rows[dominant]["bound"] == "tensor" else
+                               f"{peaks['source']} HBM copy" if rows[dominant]["bound"] == "hbm" else
+                               f"SMs x 128 FMA x 2 x median SM clock {sm_mhz} MHz")
+    act_ms = sum(per_kernel["quantize_act"]) / args.steps
+    quant_gbs = rows["quantize_act"]["achieved"]
+
+    out = {
+        "metric": METRIC, "value": round(value, 3), "unit": "TFLOP/s", "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e2m1",
+        "data": "synthetic",
+        "config": {"workload": wl.name, "description": wl.description, "M": wl.M,
+                   "layers": [[L.name, L.K, L.N] for L in layers], "alpha": wl.alphas[0],
+                   "input_dtype": wl.dtype, "y_dtype": "f32",
+                   "l2": "flushed (256 MiB write between timed steps)",
+                   "parallelism": f"replicas x{world}"},
+        "tokens_per_s": round(world * tokens_step * args.steps / (total_ms * 1e-3), 1),
+        "quantizer_gbs": quant_gbs,
+        "kernels": rows,
+        "roofline": roofline,
+        "clocks": clocks,
+        "gpu_launches": int(launches),
+        "wall_s": round(wall, 3),
+    }
+    if not args.no_e2e:
+        out["e2e"] = e2e_arm(qg, args, layers, device, world)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(args, wl, layers)
+    return out
+
+
+def e2e_arm(qg, args, layers, device, world):
+    """Same metric through the public call qg_fp4_linear with host buffers:
+    pinned host A -> device, weight quantization, the layer, Y -> pinned host,
+    all inside the timed region."""
+    hostA = [L.A.cpu().pin_memory() for L in layers]
+    hostY = [torch.empty(L.Y.shape, dtype=L.Y.dtype).pin_memory() for L in layers]
+    devA = [torch.empty_like(L.A) for L in layers]
+
+    def step():
+        for L, hA, hY, dA in zip(layers, hostA, hostY, devA):
+            dA.copy_(hA, non_blocking=True)
+            st = qg.qg_quantize_cols(L.W, L.codesT, L.t, L.ws_cols)
+            if st != qg.QG_OK:
+                raise qg.QGError(st, "e2e quantize_cols")
+            st = qg.qg_fp4_linear(dA, L.codesT, L.t, L.W, L.alpha, L.Y, L.ws_lin)
+            if st != qg.QG_OK:
+                raise qg.QGError(st, "e2e fp4_linear")
+            hY.copy_(L.Y, non_blocking=True)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    total = 0.0
+    for k in range(args.steps):
+        flush.fill_(k & 0xFF)
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        step()
+        b.record()
+        torch.cuda.synchronize()
+        total += a.elapsed_time(b)
+    for L in layers:
+        qg.check_status(L.ws_lin, "e2e")
+    if world > 1:
+        t = torch.tensor([total], dtype=torch.float64, device=device)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total = float(t.item())
+    flops = sum(L.flops for L in layers)
+    return {"value": round(world * flops * args.steps / (total * 1e-3) / 1e12, 3),
+            "unit": "TFLOP/s",
+            "h2d_bytes_per_step": int(sum(L.a_bytes for L in layers)),
+            "d2h_bytes_per_step": int(sum(L.Y.numel() * L.Y.element_size() for L in layers)),
+            "ms_per_step": round(total / args.steps, 4)}
+
+
+def _ncu_traffic(kernel, workload):
+    """DRAM bytes per launch from a committed ncu summary, when it was taken
+    on the current source of that kernel (else None)."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(path):
+        return None
+    import hashlib
+    with open(path) as f:
+        data = json.load(f)
+    rec = data.get(f"{kernel}:{workload}")
+    if not rec:
+        return None
+    src = os.path.join(ROOT, rec["source"])
+    if not os.path.exists(src):
+        return None
+    with open(src, "rb") as f:
+        sha = hashlib.sha256(f.read()).hexdigest()[:16]
+    return rec["dram_bytes_per_launch"] if sha == rec["source_sha256_16"] else None
+
+
+# ------------------------------------------------------------------ CPU oracle
+def _oracle_sample(wl, A_list, W_list, rows_per_layer):
+    """Run the oracle on a bounded sample of one step: the full quantizers on
+    every layer, Y for `rows_per_layer` rows of each layer.  Returns (seconds,
+    flops the sample stands for after scaling the Y rows to M)."""
+    import oracle
+    t_total = 0.0
+    for A, W, alpha in zip(A_list, W_list, [wl.alphas[0]] * len(A_list)):
+        M, K = A.shape
+        N = W.shape[1]
+        t0 = time.perf_counter()
+        act = oracle.quantize_act(A, alpha)
+        oT, ot = oracle.quantize_cols(W)
+        t1 = time.perf_counter()
+        rows = np.linspace(0, M - 1, rows_per_layer).astype(np.int64)
+        acc = oracle.gemm_acc(act["codes"], oT, K, rows=rows)
+        oracle.linear_y(acc, act["scales"], ot, act["row_ptr"], act["col"], act["val"], W, rows=rows)
+        t2 = time.perf_counter()
+        t_total += (t1 - t0) + (t2 - t1) * (M / rows_per_layer)
+    return t_total
+
+
+def cpu_baseline(args, wl, layers):
+    import oracle
+    A_list = [oracle.as_f32(L.A.cpu()) for L in layers]
+    W_list = [oracle.as_f32(L.W.cpu()) for L in layers]
+    rows = 16
+    t_est = _oracle_sample(wl, A_list, W_list, rows)
+    flops = sum(L.flops for L in layers)
+    return {"value": round(flops / t_est / 1e12, 6), "unit": "TFLOP/s",
+            "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": (f"one step of {wl.name}: quantizers (threshold, clamp, dA, row and "
+                       f"column codes) on the full tensors; Y for {rows} evenly spaced rows per "
+                       f"layer, its time scaled by M/{rows}"),
+            "seconds_per_step_estimate": round(t_est, 3)}
+
+
+def reference_arm(args, rank, world):
+    """The CPU oracle as the reference arm (rank 0 only)."""
+    from workloads import WORKLOADS, make_layer_inputs
+    import oracle
+    wl = WORKLOADS[args.workload]
+    A_list, W_list = [], []
+    for i in range(len(wl.layers)):
+        A, W = make_layer_inputs(wl, i, device="cpu")
+        A_list.append(oracle.as_f32(A))
+        W_list.append(oracle.as_f32(W))
+    rows = 8
+    warm = min(args.warmup, 1)        # the oracle needs no warm-up beyond one pass
+    for _ in range(warm):
+        _oracle_sample(wl, A_list, W_list, rows)
+    total = 0.0
+    for _ in range(args.steps):
+        total += _oracle_sample(wl, A_list, W_list, rows)
+    flops = wl.flops()
+    value = flops * args.steps / total / 1e12
+    cores = oracle.num_threads()
+    sample = (f"each step: quantizers on the full tensors of every {wl.name} layer, Y for "
+              f"{rows} evenly spaced rows per layer with its time scaled by M/{rows}")
+    return {
+        "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
+        "n_gpus": world, "steps": args.steps, "warmup": warm,
+        "ms_per_step": round(1e3 * total / args.steps, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "M": wl.M,
+                   "layers": [[l.name, l.K, l.N] for l in wl.layers], "alpha": wl.alphas[0]},
+        "cpu_baseline": {"kind": "oracle", "cores": cores, "sample": sample,
+                         "value": round(value, 6), "unit": "TFLOP/s"},
+        "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="llama1.3b")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        print(json.dumps(reference_arm(args, rank, world)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=300),
+                                             device_id=torch.device("cuda", local))
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    import __graft_entry__
+    if rank == 0:
+        __graft_entry__.build()
+    if world > 1:
+        torch.distributed.barrier()
+    out = our_arm(args, rank, world, device)
+    if rank == 0:
+        print(json.dumps(out), flush=True)
+    if world > 1:
+        torch.distributed.barrier()
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

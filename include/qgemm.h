@@ -100,6 +100,10 @@ typedef enum {
 const char* qg_status_string(qg_status s);
 const char* qg_version(void);
 
+/* Number of kernel launches this library has enqueued in this process (all
+ * devices, all streams); graph replays of captured launches are not counted. */
+uint64_t qg_launch_count(void);
+
 /* Rank of the threshold in sorted |A|: ceil(alpha * n) - 1 evaluated in
  * double, clamped to [0, n - 1].  ([FP4-writeup], outlier paragraph; the
  * order-statistic reading of "quantile".) */

@@ -7,7 +7,7 @@ memory and streams are torch's); the lower-case helpers below them allocate
 outputs with torch and raise :class:`QGError` on a non-OK status.
 
 There is no fallback: importing this package fails when ``lib/libqgemm.so``
-is missing (build it with ``python -m quantize_gemm_b200.build``).
+is missing (build it with ``python quantize_gemm_b200/build.py``).
 """
 from __future__ import annotations
 
@@ -24,7 +24,7 @@ LIB_PATH = os.path.join(_HERE, "lib", "libqgemm.so")
 if not os.path.exists(LIB_PATH):
     raise ImportError(
         f"{LIB_PATH} is missing: build the CUDA library first "
-        "(python -m quantize_gemm_b200.build, or __graft_entry__.build())")
+        "(python quantize_gemm_b200/build.py, or __graft_entry__.build())")
 
 _lib = ctypes.CDLL(LIB_PATH)
 
@@ -39,7 +39,7 @@ EXPORTED = (
     "qg_status_string", "qg_version", "qg_quantile_rank", "qg_nnz_capacity",
     "qg_workspace_size", "qg_workspace_init", "qg_sync_status", "qg_e2m1_encode",
     "qg_quantize_rows", "qg_quantize_cols", "qg_clamp_compensate", "qg_quantize_act",
-    "qg_spmm_correction", "qg_fp4_gemm", "qg_fp4_linear",
+    "qg_spmm_correction", "qg_fp4_gemm", "qg_fp4_linear", "qg_launch_count",
 )
 
 
@@ -65,6 +65,7 @@ def _sig(name, res, args):
 
 _sig("qg_status_string", ctypes.c_char_p, [_INT])
 _sig("qg_version", ctypes.c_char_p, [])
+_sig("qg_launch_count", ctypes.c_uint64, [])
 _sig("qg_quantile_rank", _I64, [_D, _I64])
 _sig("qg_nnz_capacity", _I64, [_I64, _D])
 _sig("qg_workspace_size", _SZ, [_INT, _I64, _I64, _I64, _INT, _D])
@@ -97,6 +98,10 @@ def qg_status_string(status: int) -> str:
 
 def qg_version() -> str:
     return _lib.qg_version().decode()
+
+
+def qg_launch_count() -> int:
+    return int(_lib.qg_launch_count())
 
 
 def qg_quantile_rank(alpha: float, n: int) -> int:

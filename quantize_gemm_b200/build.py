@@ -1,6 +1,9 @@
 """Build libqgemm.so (the C-ABI library) in-tree with nvcc for sm_100a.
 
-    python -m quantize_gemm_b200.build [--force]
+    python quantize_gemm_b200/build.py [--force] [-v]
+
+(run it as a script, or through __graft_entry__.build(): importing the
+package loads the library, which must exist first)
 
 Each .cu file under csrc/ is compiled to an object under _build/ (in
 parallel), then linked into quantize_gemm_b200/lib/libqgemm.so with the static

@@ -361,6 +361,7 @@ static cudaError_t threshold_passes(const void* A, qg_dtype dt, int64_t M, int64
                                                                       b.hist1, b.rowmax, b.ctr);
         select_kernel<0><<<1, 1024, 0, s>>>(b.hist1, kHist1Bins, (unsigned long long)rank, b.ctr,
                                             b.status, T_out);
+        count_launch(2);
     } else {
         hist_rowmax_kernel<QG_F32><<<grid1, kHistThreads, shmem, s>>>(A, lda, (int)M, (int)K,
                                                                      b.hist1, b.rowmax, b.ctr);
@@ -372,6 +373,7 @@ static cudaError_t threshold_passes(const void* A, qg_dtype dt, int64_t M, int64
                                               b.ctr, b.hist2);
         select_kernel<2><<<1, 1024, 0, s>>>(b.hist2, kHist2Bins, (unsigned long long)rank, b.ctr,
                                             b.status, T_out);
+        count_launch(4);
     }
     return cudaGetLastError();
 }
@@ -382,6 +384,7 @@ static void finalize_csr(int64_t M, const ActBuffers& b, const qg_csr* dA, cudaS
     const int grid = std::max(1, num_sms() * 4);
     csr_scatter_kernel<<<grid, 256, 0, s>>>(b.ctr, b.cap, b.st_row, b.st_rank, b.st_col, b.st_val,
                                             dA->row_ptr, dA->col, dA->val);
+    count_launch(2);
 }
 
 template <qg_dtype DT, bool CODES>
@@ -392,6 +395,7 @@ static void launch_clamp(const void* A, int64_t M, int64_t K, int64_t lda, const
     clamp_quant_kernel<DT, CODES><<<grid, kQuantThreads, 0, s>>>(
         A, lda, (int)M, (int)K, b.rowmax, b.ctr, codes, scales, A_c, b.st_row, b.st_rank, b.st_col,
         b.st_val, b.cap, b.rowcnt, b.status);
+    count_launch(1);
 }
 
 cudaError_t act_setup() {

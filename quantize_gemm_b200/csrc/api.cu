@@ -2,6 +2,7 @@
 // and the launch sequences of each call.  No device memory is allocated here.
 #include <math.h>
 
+#include <atomic>
 #include <mutex>
 
 #include "qg_internal.cuh"
@@ -12,6 +13,9 @@ static const int kMaxDevices = 64;
 static int g_sms[kMaxDevices];
 static bool g_ready[kMaxDevices];
 static std::mutex g_mu;
+static std::atomic<unsigned long long> g_launches{0};
+
+void count_launch(int n) { g_launches.fetch_add((unsigned long long)n, std::memory_order_relaxed); }
 
 // One-time per-device setup (kernel attributes), with that device current.
 static cudaError_t ensure_device(int* dev_out) {
@@ -123,6 +127,8 @@ const char* qg_status_string(qg_status s) {
 }
 
 const char* qg_version(void) { return "qgemm 0.1 sm_100a"; }
+
+uint64_t qg_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
 
 int64_t qg_quantile_rank(double alpha, int64_t n) {
     int64_t k = (int64_t)ceil(alpha * (double)n) - 1;

@@ -484,6 +484,7 @@ cudaError_t launch_fp4_gemm(const uint8_t* codesA, const float* sA, const uint8_
     const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
     const int grid = (int)std::min<int64_t>(tiles, num_sms());
     fp4_gemm_kernel<<<grid, kThreads, kSmemBytes, s>>>(ta, tb, p);
+    count_launch(1);
     return cudaGetLastError();
 }
 

@@ -238,4 +238,7 @@ cudaError_t gemm_setup();
 // Number of SMs of the current device (cached per device id).
 int num_sms();
 
+// Count kernel launches enqueued by this library (reported by qg_launch_count).
+void count_launch(int n = 1);
+
 }  // namespace qg

@@ -34,6 +34,7 @@ void launch_e2m1_encode(const float* x, int64_t n, uint8_t* packed, cudaStream_t
     int blocks = (int)std::min<int64_t>((nchunk + 255) / 256, (int64_t)num_sms() * 16);
     if (blocks < 1) blocks = 1;
     e2m1_encode_kernel<<<blocks, 256, 0, s>>>(x, n, packed);
+    count_launch(1);
 }
 
 // --------------------------------------------------------------------------
@@ -91,6 +92,7 @@ static void launch_rows_dt(const void* A, int64_t M, int64_t K, int64_t lda, uin
     else if (cpt <= 2) quantize_rows_kernel<DT, 2><<<grid, kRowThreads, 0, s>>>(A, lda, (int)K, codes, scales);
     else if (cpt <= 4) quantize_rows_kernel<DT, 4><<<grid, kRowThreads, 0, s>>>(A, lda, (int)K, codes, scales);
     else quantize_rows_kernel<DT, 8><<<grid, kRowThreads, 0, s>>>(A, lda, (int)K, codes, scales);
+    count_launch(1);
 }
 
 void launch_quantize_rows(const void* A, qg_dtype dt, int64_t M, int64_t K, int64_t lda,
@@ -196,6 +198,7 @@ void launch_zero_u32(uint32_t* p, int64_t n, cudaStream_t s) {
     int blocks = (int)std::min<int64_t>((n + 255) / 256, (int64_t)num_sms() * 4);
     if (blocks < 1) blocks = 1;
     zero_u32_kernel<<<blocks, 256, 0, s>>>(p, n);
+    count_launch(1);
 }
 
 void launch_quantize_cols(const void* W, qg_dtype dt, int64_t K, int64_t N, int64_t ldw,
@@ -214,6 +217,7 @@ void launch_quantize_cols(const void* W, qg_dtype dt, int64_t K, int64_t N, int6
         colmax_kernel<QG_F32><<<g1, 256, 0, s>>>(W, ldw, (int)K, (int)N, rows_per, colmax);
         quantize_cols_kernel<QG_F32><<<g2, 256, 0, s>>>(W, ldw, (int)K, (int)N, colmax, codesT, scales);
     }
+    count_launch(2);
 }
 
 }  // namespace qg

@@ -85,6 +85,7 @@ void launch_spmm(const qg_csr* dA, int64_t M, const void* W, qg_dtype dt, int64_
     else
         spmm_rows_kernel<QG_F32><<<(unsigned)M, kSpmmThreads, 0, s>>>(dA->row_ptr, dA->col, dA->val,
                                                                        W, ldw, (int)N, C);
+    count_launch(1);
 }
 
 }  // namespace qg
