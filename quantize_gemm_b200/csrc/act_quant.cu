@@ -14,12 +14,15 @@
 //   fp32: a 2^15-bin pass on bits 30..16, then a 2^16-bin pass on bits 15..0
 //         restricted to the selected bucket.
 // The pass that builds the histogram also keeps each row's max |a|, so the
-// quantize pass knows amax_i = min(rowmax_i, T) without another reduction.
+// quantize pass knows amax_i = min(rowmax_i, T) without another reduction, and
+// its last CTA to finish selects the bin (no separate launch).
 //
-// dA is emitted in canonical CSR order without sorting: one warp owns a row
-// and walks it in column order, so each outlier knows its rank within the row;
-// entries go to a staging list through warp-aggregated slot reservation, and a
-// final scatter puts entry (row, rank) at row_ptr[row] + rank.
+// dA is emitted in canonical CSR order without sorting and without global
+// atomics in the common case: one warp owns a row and walks it in column
+// order, so each outlier knows its rank within the row; rank < row_slots goes
+// to the row's own staging region, later ones to an overflow list.  The last
+// CTA of the clamp pass scans the row counts into row_ptr; a scatter kernel
+// then moves entry (row, rank) to row_ptr[row] + rank.
 #include "qg_internal.cuh"
 
 namespace qg {
@@ -28,12 +31,113 @@ constexpr int kHistThreads = 1024;
 constexpr int kQuantThreads = 256;
 
 // --------------------------------------------------------------------------
-// Pass 1: shared-memory histogram of the 15-bit keys + per-row max key.
+// Selection of the bin that holds the entry of rank `rank` (0-based) in a
+// histogram of nbins = 1024 * per bins, by one CTA of 1024 threads.  Warp w
+// owns bins [w * 32 * per, (w + 1) * 32 * per); lanes read them coalesced.
+// Reads go around L1 (the bins were just written by atomics).
+struct SelectResult {
+    uint32_t bin;
+    unsigned long long below;   // entries in bins < bin
+    int found;
+};
+
+__device__ SelectResult block_select(const uint32_t* __restrict__ hist, int nbins,
+                                     unsigned long long rank) {
+    __shared__ unsigned long long s_warp[32];
+    __shared__ SelectResult s_res;
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int seg = nbins / 32;                 // bins per warp
+    const uint32_t* h = hist + (int64_t)warp * seg;
+    unsigned long long mine = 0;
+    for (int i = lane; i < seg; i += 32) mine += __ldcg(h + i);
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) mine += __shfl_xor_sync(0xFFFFFFFFu, mine, d);
+    if (lane == 0) s_warp[warp] = mine;
+    if (t == 0) s_res.found = 0;
+    __syncthreads();
+    if (warp == 0) {
+        // find the warp segment holding the rank
+        unsigned long long w = s_warp[lane], incl = w;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            unsigned long long u = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+            if (lane >= d) incl += u;
+        }
+        const unsigned long long excl = incl - w;
+        const unsigned hit = __ballot_sync(0xFFFFFFFFu, excl <= rank && rank < incl);
+        if (hit) {
+            const int ws = __ffs(hit) - 1;
+            unsigned long long cum = __shfl_sync(0xFFFFFFFFu, excl, ws);
+            const uint32_t* hs = hist + (int64_t)ws * seg;
+            // walk the segment 32 bins at a time
+            for (int base = 0; base < seg; base += 32) {
+                const unsigned long long c = __ldcg(hs + base + lane);
+                unsigned long long ci = c;
+#pragma unroll
+                for (int d = 1; d < 32; d <<= 1) {
+                    unsigned long long u = __shfl_up_sync(0xFFFFFFFFu, ci, d);
+                    if (lane >= d) ci += u;
+                }
+                const unsigned long long ce = cum + ci - c;
+                const unsigned h2 = __ballot_sync(0xFFFFFFFFu, ce <= rank && rank < cum + ci);
+                if (h2) {
+                    const int lb = __ffs(h2) - 1;
+                    if (lane == lb) {
+                        s_res.bin = (uint32_t)(ws * seg + base + lb);
+                        s_res.below = ce;
+                        s_res.found = 1;
+                    }
+                    break;
+                }
+                cum += __shfl_sync(0xFFFFFFFFu, ci, 31);
+            }
+        }
+    }
+    __syncthreads();
+    return s_res;
+}
+
+// Store the selection.  MODE 0: bf16 threshold; 1: fp32 bucket; 2: fp32 threshold.
+template <int MODE>
+__device__ void finish_select(const SelectResult& r, Counters* ctr, uint32_t* status,
+                              float* T_out) {
+    if (threadIdx.x != 0) return;
+    if (!r.found) {
+        // the histogram does not hold rank + 1 entries: inconsistent input
+        flag_status(status, kStatusOverflow);
+        ctr->T_key = 0x7FFFFFFFu;
+        if (MODE == 1) ctr->sel_bin = 0x7FFFu;
+    } else if (MODE == 1) {
+        ctr->sel_bin = r.bin;
+        ctr->sel_below = r.below;
+    } else {
+        const uint32_t key = (MODE == 0) ? r.bin : ((ctr->sel_bin << 16) | r.bin);
+        ctr->T_key = key;
+        *T_out = (MODE == 0) ? __uint_as_float(key << 16) : __uint_as_float(key);
+    }
+    if (MODE != 1 && ctr->nonfinite) flag_status(status, kStatusNonFinite);
+}
+
+// True in the CTA that finished last (after all CTAs' global writes).
+__device__ __forceinline__ bool last_block_done(uint32_t* counter) {
+    __shared__ int s_last;
+    __threadfence();
+    __syncthreads();
+    if (threadIdx.x == 0) s_last = (atomicAdd(counter, 1u) == gridDim.x - 1);
+    __syncthreads();
+    if (s_last) __threadfence();
+    return s_last != 0;
+}
+
+// --------------------------------------------------------------------------
+// Pass 1: shared-memory histogram of the 15-bit keys + per-row max key; the
+// last CTA selects the threshold bin (bf16) or the bucket (fp32).
 template <qg_dtype DT>
 __global__ void __launch_bounds__(kHistThreads, 1)
 hist_rowmax_kernel(const void* __restrict__ A, int64_t lda, int M, int K,
                    uint32_t* __restrict__ ghist, uint32_t* __restrict__ rowmax,
-                   Counters* __restrict__ ctr) {
+                   Counters* __restrict__ ctr, unsigned long long rank,
+                   uint32_t* __restrict__ status, float* __restrict__ T_out) {
     extern __shared__ uint32_t sh_hist[];
     for (int i = threadIdx.x; i < kHist1Bins; i += blockDim.x) sh_hist[i] = 0u;
     __syncthreads();
@@ -76,13 +180,20 @@ hist_rowmax_kernel(const void* __restrict__ A, int64_t lda, int M, int K,
         const uint32_t v = sh_hist[i];
         if (v) atomicAdd(&ghist[i], v);
     }
+    if (last_block_done(&ctr->done_hist)) {
+        const SelectResult r = block_select(ghist, kHist1Bins, rank);
+        if (DT == QG_BF16) finish_select<0>(r, ctr, status, T_out);
+        else finish_select<1>(r, ctr, status, T_out);
+    }
 }
 
 // fp32 only: histogram of the low 16 key bits of the entries whose high bits
-// equal the bucket chosen by the first selection.
-__global__ void __launch_bounds__(256)
+// equal the selected bucket; the last CTA selects the threshold.
+__global__ void __launch_bounds__(kHistThreads)
 refine_hist_kernel(const float* __restrict__ A, int64_t lda, int M, int K,
-                   const Counters* __restrict__ ctr, uint32_t* __restrict__ ghist2) {
+                   Counters* __restrict__ ctr, uint32_t* __restrict__ ghist2,
+                   unsigned long long rank, uint32_t* __restrict__ status,
+                   float* __restrict__ T_out) {
     const uint32_t hi = ctr->sel_bin;
     const int nchunks = K / 8;
     const int64_t total = (int64_t)M * nchunks;
@@ -98,75 +209,9 @@ refine_hist_kernel(const float* __restrict__ A, int64_t lda, int M, int K,
             if ((k >> 16) == hi) atomicAdd(&ghist2[k & 0xFFFFu], 1u);
         }
     }
-}
-
-// --------------------------------------------------------------------------
-// Selection: the bin holding the entry of rank `rank` (0-based) in a
-// histogram.  One CTA; each thread owns a run of consecutive bins.
-//   mode 0: bf16, bins are full keys           -> T
-//   mode 1: fp32 level 1 (bits 30..16)         -> sel_bin, sel_below
-//   mode 2: fp32 level 2 (bits 15..0) of rank - sel_below in bucket sel_bin -> T
-template <int MODE>
-__global__ void __launch_bounds__(1024)
-select_kernel(const uint32_t* __restrict__ hist, int nbins, unsigned long long rank,
-              Counters* __restrict__ ctr, uint32_t* __restrict__ status, float* __restrict__ T_out) {
-    __shared__ unsigned long long warp_tot[32];
-    __shared__ int found;
-    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    if (MODE == 2) rank -= ctr->sel_below;
-    if (t == 0) found = 0;
-    const int per = nbins / 1024;
-    const uint32_t* h = hist + (int64_t)t * per;
-    unsigned long long mine = 0;
-    for (int i = 0; i < per; ++i) mine += h[i];
-    // block-wide inclusive scan of `mine`
-    unsigned long long v = mine;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-        unsigned long long u = __shfl_up_sync(0xFFFFFFFFu, v, d);
-        if (lane >= d) v += u;
-    }
-    if (lane == 31) warp_tot[warp] = v;
-    __syncthreads();
-    if (warp == 0) {
-        unsigned long long w = warp_tot[lane];
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            unsigned long long u = __shfl_up_sync(0xFFFFFFFFu, w, d);
-            if (lane >= d) w += u;
-        }
-        warp_tot[lane] = w;
-    }
-    __syncthreads();
-    const unsigned long long incl = v + (warp > 0 ? warp_tot[warp - 1] : 0ull);
-    const unsigned long long excl = incl - mine;
-    if (excl <= rank && rank < incl) {
-        unsigned long long cum = excl;
-        int b = 0;
-        for (; b < per; ++b) {
-            if (rank < cum + h[b]) break;
-            cum += h[b];
-        }
-        const uint32_t bin = (uint32_t)(t * per + b);
-        found = 1;
-        if (MODE == 1) {
-            ctr->sel_bin = bin;
-            ctr->sel_below = cum;
-        } else {
-            const uint32_t key = (MODE == 0) ? bin : ((ctr->sel_bin << 16) | bin);
-            ctr->T_key = key;
-            *T_out = (MODE == 0) ? __uint_as_float(key << 16) : __uint_as_float(key);
-        }
-    }
-    __syncthreads();
-    if (t == 0) {
-        if (!found) {
-            // the histogram does not hold rank+1 entries: inconsistent input
-            flag_status(status, kStatusOverflow);
-            ctr->T_key = 0x7FFFFFFFu;
-            if (MODE == 1) ctr->sel_bin = 0x7FFFu;
-        }
-        if (MODE != 1 && ctr->nonfinite) flag_status(status, kStatusNonFinite);
+    if (last_block_done(&ctr->done_refine)) {
+        const SelectResult r = block_select(ghist2, kHist2Bins, rank - ctr->sel_below);
+        finish_select<2>(r, ctr, status, T_out);
     }
 }
 
@@ -176,81 +221,84 @@ select_kernel(const uint32_t* __restrict__ hist, int nbins, unsigned long long r
 // groups of the warp covering 1024 consecutive columns.
 //   WRITE_CODES = true : quantize_act (codes + scales)
 //   WRITE_CODES = false: clamp_compensate (A_clamped in the input dtype)
+// The last CTA to finish turns the row counts into row_ptr.
 template <qg_dtype DT, bool WRITE_CODES>
 __global__ void __launch_bounds__(kQuantThreads)
 clamp_quant_kernel(const void* __restrict__ A, int64_t lda, int M, int K,
                    const uint32_t* __restrict__ rowmax, Counters* __restrict__ ctr,
                    uint8_t* __restrict__ codes, float* __restrict__ scales,
-                   void* __restrict__ A_c,
-                   int32_t* __restrict__ st_row, int32_t* __restrict__ st_rank,
-                   int32_t* __restrict__ st_col, double* __restrict__ st_val, int64_t cap,
-                   uint32_t* __restrict__ rowcnt, uint32_t* __restrict__ status) {
+                   void* __restrict__ A_c, ActBuffers b, int32_t* __restrict__ row_ptr,
+                   int64_t* __restrict__ nnz_out) {
     const uint32_t Tk = ctr->T_key;
     const float T = key_to_float<DT>(Tk);
     const int lane = threadIdx.x & 31;
     const int wpc = blockDim.x >> 5;
     const int total_warps = gridDim.x * wpc;
     const int nchunks = K / 8;
+    const int row_slots = (int)b.row_slots;
     for (int row = blockIdx.x * wpc + (threadIdx.x >> 5); row < M; row += total_warps) {
         const int64_t base = (int64_t)row * lda;
-        const uint32_t akey = min(rowmax[row], Tk);
+        const uint32_t rmax = rowmax[row];
+        const uint32_t akey = min(rmax, Tk);
+        const bool any_out = rmax > Tk;
         float r = 0.0f, s = 0.0f;
         if (WRITE_CODES) {
             scale_factors(key_to_float<DT>(akey), r, s);
             if (lane == 0) scales[row] = s;
         }
+        int32_t* rcol = b.st_col + (int64_t)row * row_slots;
+        double* rval = b.st_val + (int64_t)row * row_slots;
         int row_rank = 0;
         for (int c0 = 0; c0 < nchunks; c0 += 128) {
             float x[4][8];
             uint32_t om[4];
-            int cnt[4], ex[4];
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
                 const int c = c0 + 32 * j + lane;
                 om[j] = 0;
                 if (c < nchunks) {
                     load8<DT>(A, base + (int64_t)c * 8, x[j]);
+                    if (any_out) {
 #pragma unroll
-                    for (int e = 0; e < 8; ++e)
-                        om[j] |= (mag_key<DT>(x[j][e]) > Tk ? 1u : 0u) << e;
+                        for (int e = 0; e < 8; ++e)
+                            om[j] |= (mag_key<DT>(x[j][e]) > Tk ? 1u : 0u) << e;
+                    }
                 }
             }
-            // ranks of this iteration's outliers in column order
-            int iter_total = 0;
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-                cnt[j] = __popc(om[j]);
-                const int incl = warp_inclusive_scan(cnt[j]);
-                ex[j] = iter_total + incl - cnt[j];
-                iter_total += __shfl_sync(0xFFFFFFFFu, incl, 31);
-            }
-            if (iter_total > 0) {
-                unsigned long long slot0 = 0;
-                if (lane == 0) slot0 = atomicAdd(&ctr->nnz, (unsigned long long)iter_total);
-                slot0 = __shfl_sync(0xFFFFFFFFu, slot0, 0);
+            if (any_out) {
+                // ranks of this iteration's outliers in column order
 #pragma unroll
                 for (int j = 0; j < 4; ++j) {
+                    const int cnt = __popc(om[j]);
+                    const int incl = warp_inclusive_scan(cnt);
+                    int idx = row_rank + incl - cnt;
+                    row_rank += __shfl_sync(0xFFFFFFFFu, incl, 31);
                     if (om[j] == 0) continue;
-                    int idx = ex[j];
                     const int c = c0 + 32 * j + lane;
 #pragma unroll
                     for (int e = 0; e < 8; ++e) {
                         if (!((om[j] >> e) & 1u)) continue;
-                        const unsigned long long slot = slot0 + (unsigned long long)idx;
-                        if (slot < (unsigned long long)cap) {
-                            const float a = x[j][e];
-                            st_row[slot] = row;
-                            st_rank[slot] = row_rank + idx;
-                            st_col[slot] = c * 8 + e;
-                            st_val[slot] = (double)a - (double)copysignf(T, a);
+                        const float a = x[j][e];
+                        const double d = (double)a - (double)copysignf(T, a);
+                        if (idx < row_slots) {
+                            rcol[idx] = c * 8 + e;
+                            rval[idx] = d;
                         } else {
-                            flag_status(status, kStatusOverflow);
+                            const unsigned long long o = atomicAdd(&ctr->nnz, 1ull);
+                            if (o < (unsigned long long)b.cap) {
+                                const int64_t slot = (int64_t)M * row_slots + (int64_t)o;
+                                b.st_row[o] = row;
+                                b.st_rank[o] = idx;
+                                b.st_col[slot] = c * 8 + e;
+                                b.st_val[slot] = d;
+                            } else {
+                                flag_status(b.status, kStatusOverflow);
+                            }
                         }
                         ++idx;
                     }
                 }
             }
-            row_rank += iter_total;
             // clamp, then encode (or store the clamped values)
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
@@ -281,66 +329,69 @@ clamp_quant_kernel(const void* __restrict__ A, int64_t lda, int M, int K,
                 }
             }
         }
-        if (lane == 0) rowcnt[row] = (uint32_t)row_rank;
+        if (lane == 0) b.rowcnt[row] = (uint32_t)row_rank;
     }
-}
 
-// --------------------------------------------------------------------------
-// CSR finalize: row_ptr = exclusive scan of the row counts (one CTA), then
-// scatter each staged entry to row_ptr[row] + rank.
-__global__ void __launch_bounds__(1024)
-csr_scan_kernel(const uint32_t* __restrict__ rowcnt, int M, int32_t* __restrict__ row_ptr,
-                int64_t* __restrict__ nnz_out, const Counters* __restrict__ ctr, int64_t cap,
-                uint32_t* __restrict__ status) {
-    __shared__ unsigned long long warp_tot[32];
-    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    const int per = (M + 1023) / 1024;
-    const int r0 = min(M, t * per), r1 = min(M, r0 + per);
-    unsigned long long mine = 0;
-    for (int i = r0; i < r1; ++i) mine += rowcnt[i];
-    unsigned long long v = mine;
-#pragma unroll
-    for (int d = 1; d < 32; d <<= 1) {
-        unsigned long long u = __shfl_up_sync(0xFFFFFFFFu, v, d);
-        if (lane >= d) v += u;
-    }
-    if (lane == 31) warp_tot[warp] = v;
-    __syncthreads();
-    if (warp == 0) {
-        unsigned long long w = warp_tot[lane];
+    // last CTA: row_ptr = exclusive scan of the row counts
+    if (last_block_done(&ctr->done_clamp)) {
+        __shared__ unsigned long long s_warp[kQuantThreads / 32];
+        const int t = threadIdx.x, w = t >> 5;
+        const int per = (M + kQuantThreads - 1) / kQuantThreads;
+        const int r0 = min(M, t * per), r1 = min(M, r0 + per);
+        unsigned long long mine = 0;
+        for (int i = r0; i < r1; ++i) mine += __ldcg(b.rowcnt + i);
+        unsigned long long v = mine;
 #pragma unroll
         for (int d = 1; d < 32; d <<= 1) {
-            unsigned long long u = __shfl_up_sync(0xFFFFFFFFu, w, d);
-            if (lane >= d) w += u;
+            unsigned long long u = __shfl_up_sync(0xFFFFFFFFu, v, d);
+            if (lane >= d) v += u;
         }
-        warp_tot[lane] = w;
-    }
-    __syncthreads();
-    unsigned long long run = v + (warp > 0 ? warp_tot[warp - 1] : 0ull) - mine;
-    for (int i = r0; i < r1; ++i) {
-        row_ptr[i] = (int32_t)run;
-        run += rowcnt[i];
-    }
-    if (t == 1023) {
-        const unsigned long long total = warp_tot[31];
-        row_ptr[M] = (int32_t)total;
-        *nnz_out = (int64_t)total;
-        if (total != ctr->nnz || total > (unsigned long long)cap) flag_status(status, kStatusOverflow);
+        if (lane == 31) s_warp[w] = v;
+        __syncthreads();
+        unsigned long long before = 0, total = 0;
+        for (int i = 0; i < kQuantThreads / 32; ++i) {
+            if (i < w) before += s_warp[i];
+            total += s_warp[i];
+        }
+        unsigned long long run = before + v - mine;
+        for (int i = r0; i < r1; ++i) {
+            row_ptr[i] = (int32_t)run;
+            run += __ldcg(b.rowcnt + i);
+        }
+        if (t == 0) {
+            row_ptr[M] = (int32_t)total;
+            *nnz_out = (int64_t)total;
+            if (total > (unsigned long long)b.cap) flag_status(b.status, kStatusOverflow);
+        }
     }
 }
 
+// Move staged entries to their CSR positions: a warp per row for the row
+// regions, then a thread per overflow entry.
 __global__ void __launch_bounds__(256)
-csr_scatter_kernel(const Counters* __restrict__ ctr, int64_t cap,
-                   const int32_t* __restrict__ st_row, const int32_t* __restrict__ st_rank,
-                   const int32_t* __restrict__ st_col, const double* __restrict__ st_val,
+csr_scatter_kernel(const Counters* __restrict__ ctr, ActBuffers b, int M,
                    const int32_t* __restrict__ row_ptr, int32_t* __restrict__ col,
                    double* __restrict__ val) {
-    const unsigned long long n = min(ctr->nnz, (unsigned long long)cap);
-    for (unsigned long long e = blockIdx.x * (unsigned long long)blockDim.x + threadIdx.x; e < n;
-         e += (unsigned long long)gridDim.x * blockDim.x) {
-        const int64_t dst = (int64_t)row_ptr[st_row[e]] + st_rank[e];
-        col[dst] = st_col[e];
-        val[dst] = st_val[e];
+    const int lane = threadIdx.x & 31;
+    const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+    const int nw = (gridDim.x * blockDim.x) >> 5;
+    const int row_slots = (int)b.row_slots;
+    for (int r = gw; r < M; r += nw) {
+        const int n = min((int)b.rowcnt[r], row_slots);
+        const int64_t dst = row_ptr[r];
+        const int64_t src = (int64_t)r * row_slots;
+        for (int j = lane; j < n; j += 32) {
+            col[dst + j] = b.st_col[src + j];
+            val[dst + j] = b.st_val[src + j];
+        }
+    }
+    const unsigned long long n_over = min(ctr->nnz, (unsigned long long)b.cap);
+    const int64_t base = (int64_t)M * row_slots;
+    for (unsigned long long e = blockIdx.x * (unsigned long long)blockDim.x + threadIdx.x;
+         e < n_over; e += (unsigned long long)gridDim.x * blockDim.x) {
+        const int64_t dst = (int64_t)row_ptr[b.st_row[e]] + b.st_rank[e];
+        col[dst] = b.st_col[base + e];
+        val[dst] = b.st_val[base + e];
     }
 }
 
@@ -357,45 +408,35 @@ static cudaError_t threshold_passes(const void* A, qg_dtype dt, int64_t M, int64
     const int grid1 = (int)std::min<int64_t>(nsm, (M + 31) / 32);
     const size_t shmem = sizeof(uint32_t) * kHist1Bins;
     if (dt == QG_BF16) {
-        hist_rowmax_kernel<QG_BF16><<<grid1, kHistThreads, shmem, s>>>(A, lda, (int)M, (int)K,
-                                                                      b.hist1, b.rowmax, b.ctr);
-        select_kernel<0><<<1, 1024, 0, s>>>(b.hist1, kHist1Bins, (unsigned long long)rank, b.ctr,
-                                            b.status, T_out);
-        count_launch(2);
+        hist_rowmax_kernel<QG_BF16><<<grid1, kHistThreads, shmem, s>>>(
+            A, lda, (int)M, (int)K, b.hist1, b.rowmax, b.ctr, (unsigned long long)rank, b.status,
+            T_out);
+        count_launch(1);
     } else {
-        hist_rowmax_kernel<QG_F32><<<grid1, kHistThreads, shmem, s>>>(A, lda, (int)M, (int)K,
-                                                                     b.hist1, b.rowmax, b.ctr);
-        select_kernel<1><<<1, 1024, 0, s>>>(b.hist1, kHist1Bins, (unsigned long long)rank, b.ctr,
-                                            b.status, T_out);
+        hist_rowmax_kernel<QG_F32><<<grid1, kHistThreads, shmem, s>>>(
+            A, lda, (int)M, (int)K, b.hist1, b.rowmax, b.ctr, (unsigned long long)rank, b.status,
+            T_out);
         const int64_t work = M * (K / 8);
-        const int g2 = (int)std::max<int64_t>(1, std::min<int64_t>((work + 255) / 256, nsm * 8));
-        refine_hist_kernel<<<g2, 256, 0, s>>>(static_cast<const float*>(A), lda, (int)M, (int)K,
-                                              b.ctr, b.hist2);
-        select_kernel<2><<<1, 1024, 0, s>>>(b.hist2, kHist2Bins, (unsigned long long)rank, b.ctr,
-                                            b.status, T_out);
-        count_launch(4);
+        const int g2 = (int)std::max<int64_t>(1, std::min<int64_t>((work + kHistThreads - 1) / kHistThreads, nsm * 2));
+        refine_hist_kernel<<<g2, kHistThreads, 0, s>>>(static_cast<const float*>(A), lda, (int)M,
+                                                       (int)K, b.ctr, b.hist2,
+                                                       (unsigned long long)rank, b.status, T_out);
+        count_launch(2);
     }
     return cudaGetLastError();
 }
 
-static void finalize_csr(int64_t M, const ActBuffers& b, const qg_csr* dA, cudaStream_t s) {
-    csr_scan_kernel<<<1, 1024, 0, s>>>(b.rowcnt, (int)M, dA->row_ptr, dA->nnz_out, b.ctr, b.cap,
-                                       b.status);
-    const int grid = std::max(1, num_sms() * 4);
-    csr_scatter_kernel<<<grid, 256, 0, s>>>(b.ctr, b.cap, b.st_row, b.st_rank, b.st_col, b.st_val,
-                                            dA->row_ptr, dA->col, dA->val);
-    count_launch(2);
-}
-
 template <qg_dtype DT, bool CODES>
 static void launch_clamp(const void* A, int64_t M, int64_t K, int64_t lda, const ActBuffers& b,
-                         uint8_t* codes, float* scales, void* A_c, cudaStream_t s) {
+                         uint8_t* codes, float* scales, void* A_c, const qg_csr* dA,
+                         cudaStream_t s) {
     const int wpc = kQuantThreads / 32;
     const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((M + wpc - 1) / wpc, (int64_t)num_sms() * 8));
     clamp_quant_kernel<DT, CODES><<<grid, kQuantThreads, 0, s>>>(
-        A, lda, (int)M, (int)K, b.rowmax, b.ctr, codes, scales, A_c, b.st_row, b.st_rank, b.st_col,
-        b.st_val, b.cap, b.rowcnt, b.status);
-    count_launch(1);
+        A, lda, (int)M, (int)K, b.rowmax, b.ctr, codes, scales, A_c, b, dA->row_ptr, dA->nnz_out);
+    const int g2 = (int)std::max<int64_t>(1, std::min<int64_t>((M * 32 + 255) / 256, (int64_t)num_sms() * 8));
+    csr_scatter_kernel<<<g2, 256, 0, s>>>(b.ctr, b, (int)M, dA->row_ptr, dA->col, dA->val);
+    count_launch(2);
 }
 
 cudaError_t act_setup() {
@@ -413,9 +454,8 @@ cudaError_t run_quantize_act(const void* A, qg_dtype dt, int64_t M, int64_t K, i
                              const qg_csr* dA, float* T_out, cudaStream_t s) {
     cudaError_t e = threshold_passes(A, dt, M, K, lda, rank, b, T_out, s);
     if (e != cudaSuccess) return e;
-    if (dt == QG_BF16) launch_clamp<QG_BF16, true>(A, M, K, lda, b, codes, scales, nullptr, s);
-    else launch_clamp<QG_F32, true>(A, M, K, lda, b, codes, scales, nullptr, s);
-    finalize_csr(M, b, dA, s);
+    if (dt == QG_BF16) launch_clamp<QG_BF16, true>(A, M, K, lda, b, codes, scales, nullptr, dA, s);
+    else launch_clamp<QG_F32, true>(A, M, K, lda, b, codes, scales, nullptr, dA, s);
     return cudaGetLastError();
 }
 
@@ -424,9 +464,8 @@ cudaError_t run_clamp_compensate(const void* A, qg_dtype dt, int64_t M, int64_t 
                                  float* T_out, cudaStream_t s) {
     cudaError_t e = threshold_passes(A, dt, M, K, lda, rank, b, T_out, s);
     if (e != cudaSuccess) return e;
-    if (dt == QG_BF16) launch_clamp<QG_BF16, false>(A, M, K, lda, b, nullptr, nullptr, A_c, s);
-    else launch_clamp<QG_F32, false>(A, M, K, lda, b, nullptr, nullptr, A_c, s);
-    finalize_csr(M, b, dA, s);
+    if (dt == QG_BF16) launch_clamp<QG_BF16, false>(A, M, K, lda, b, nullptr, nullptr, A_c, dA, s);
+    else launch_clamp<QG_F32, false>(A, M, K, lda, b, nullptr, nullptr, A_c, dA, s);
     return cudaGetLastError();
 }
 

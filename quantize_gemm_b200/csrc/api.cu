@@ -91,6 +91,7 @@ static ActBuffers act_buffers(void* ws, const WsLayout& L) {
     b.st_col = at<int32_t>(ws, L.st_col);
     b.st_val = at<double>(ws, L.st_val);
     b.cap = L.cap;
+    b.row_slots = L.row_slots;
     return b;
 }
 

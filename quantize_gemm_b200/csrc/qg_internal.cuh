@@ -27,13 +27,24 @@ enum : uint32_t {
 
 // Counters that live right after the status word.
 struct Counters {
-    unsigned long long nnz;        // staging slots reserved so far
+    unsigned long long nnz;        // dA entries that overflowed their row region
     unsigned long long sel_below;  // entries strictly below the selected bin
     uint32_t nonfinite;            // set when a NaN/Inf key was seen
     uint32_t sel_bin;              // bin chosen by the last selection pass
     uint32_t T_key;                // final threshold as |x| bit pattern
-    uint32_t pad;
+    uint32_t done_hist;            // CTAs finished with the histogram pass
+    uint32_t done_refine;          // CTAs finished with the fp32 refine pass
+    uint32_t done_clamp;           // CTAs finished with the clamp pass
 };
+
+// Staging of dA: every row owns `row_slots` entries (its first entries in
+// column order, stored at row * row_slots + rank); entries past that go to an
+// overflow list of (row, rank, col, val) with room for every clamped entry.
+inline int64_t staging_row_slots(int64_t M, int64_t K, int64_t cap) {
+    int64_t per = (cap + M - 1) / (M > 0 ? M : 1);
+    int64_t r = 2 * per + 16;
+    return r < K ? r : K;
+}
 
 // ---------------------------------------------------------------- workspace
 constexpr size_t kAlign = 256;
@@ -49,6 +60,7 @@ struct WsLayout {
            csr_nnz = 0, thr = 0, corr = 0;
     size_t total = 0;
     int64_t cap = 0;
+    int64_t row_slots = 0;
 };
 
 // Compute the layout for an op.  Offsets are relative to the workspace base.
@@ -76,10 +88,12 @@ inline WsLayout ws_layout(qg_op op, int64_t M, int64_t K, int64_t N, qg_dtype dt
         if (dtype == QG_F32) L.hist2 = take(sizeof(uint32_t) * kHist2Bins);
         L.rowmax = take(sizeof(uint32_t) * (size_t)M);
         L.rowcnt = take(sizeof(uint32_t) * (size_t)M);
-        L.st_row = take(sizeof(int32_t) * (size_t)cap);
-        L.st_rank = take(sizeof(int32_t) * (size_t)cap);
-        L.st_col = take(sizeof(int32_t) * (size_t)cap);
-        L.st_val = take(sizeof(double) * (size_t)cap);
+        L.row_slots = staging_row_slots(M, K, L.cap);
+        const size_t slots = (size_t)M * (size_t)L.row_slots + (size_t)cap;
+        L.st_row = take(sizeof(int32_t) * (size_t)cap);     // overflow list only
+        L.st_rank = take(sizeof(int32_t) * (size_t)cap);    // overflow list only
+        L.st_col = take(sizeof(int32_t) * slots);
+        L.st_val = take(sizeof(double) * slots);
     }
     if (op == QG_OP_QUANTIZE_COLS) L.colmax = take(sizeof(uint32_t) * (size_t)N);
     if (op == QG_OP_FP4_LINEAR) {
@@ -211,6 +225,7 @@ struct ActBuffers {
     int32_t *st_row, *st_rank, *st_col;
     double* st_val;
     int64_t cap;
+    int64_t row_slots;
 };
 
 // Launch sequences (kernel files) used by the C ABI layer.

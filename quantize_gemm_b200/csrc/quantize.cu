@@ -114,31 +114,49 @@ __device__ __forceinline__ float load1(const void* base, int64_t idx) {
         return static_cast<const float*>(base)[idx];
 }
 
+// Pass 1: a CTA owns 256 columns (8 per lane) and a range of rows; its 8 warps
+// split the rows, reduce in shared memory, and issue one atomicMax per column.
 template <qg_dtype DT>
 __global__ void __launch_bounds__(256)
 colmax_kernel(const void* __restrict__ W, int64_t ldw, int K, int N, int rows_per_split,
               uint32_t* __restrict__ colmax) {
-    const int c = blockIdx.x * 256 + threadIdx.x;  // chunk of 8 columns
-    const int n0 = c * 8;
-    if (n0 >= N) return;
+    __shared__ uint32_t red[8][256];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int n0 = blockIdx.x * 256 + lane * 8;
     const int k0 = blockIdx.y * rows_per_split;
     const int k1 = min(K, k0 + rows_per_split);
     uint32_t m[8] = {0, 0, 0, 0, 0, 0, 0, 0};
-    const bool vec = (n0 + 8 <= N) && ((ldw & 7) == 0 || DT == QG_F32) && ((ldw & 3) == 0);
-    for (int k = k0; k < k1; ++k) {
-        float x[8];
-        if (vec) {
+    if (n0 < N) {
+        const bool vec = (n0 + 8 <= N) && ((ldw & 7) == 0 || DT == QG_F32) && ((ldw & 3) == 0);
+        int k = k0 + warp;
+        for (; vec && k + 8 < k1; k += 16) {     // two rows in flight per lane
+            float x[8], y[8];
             load8<DT>(W, (int64_t)k * ldw + n0, x);
-        } else {
+            load8<DT>(W, (int64_t)(k + 8) * ldw + n0, y);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) x[e] = (n0 + e < N) ? load1<DT>(W, (int64_t)k * ldw + n0 + e) : 0.0f;
+            for (int e = 0; e < 8; ++e) m[e] = max(m[e], max(key_of(x[e]), key_of(y[e])));
         }
+        for (; k < k1; k += 8) {
+            float x[8];
+            if (vec) {
+                load8<DT>(W, (int64_t)k * ldw + n0, x);
+            } else {
 #pragma unroll
-        for (int e = 0; e < 8; ++e) m[e] = max(m[e], key_of(x[e]));
+                for (int e = 0; e < 8; ++e) x[e] = (n0 + e < N) ? load1<DT>(W, (int64_t)k * ldw + n0 + e) : 0.0f;
+            }
+#pragma unroll
+            for (int e = 0; e < 8; ++e) m[e] = max(m[e], key_of(x[e]));
+        }
     }
 #pragma unroll
-    for (int e = 0; e < 8; ++e)
-        if (n0 + e < N && m[e] != 0) atomicMax(&colmax[n0 + e], m[e]);
+    for (int e = 0; e < 8; ++e) red[warp][lane * 8 + e] = m[e];
+    __syncthreads();
+    const int c = threadIdx.x;          // one column per thread
+    uint32_t v = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) v = max(v, red[w][c]);
+    const int n = blockIdx.x * 256 + c;
+    if (n < N && v != 0) atomicMax(&colmax[n], v);
 }
 
 constexpr int kColTileK = 32;
@@ -204,8 +222,10 @@ void launch_zero_u32(uint32_t* p, int64_t n, cudaStream_t s) {
 void launch_quantize_cols(const void* W, qg_dtype dt, int64_t K, int64_t N, int64_t ldw,
                           uint8_t* codesT, float* scales, uint32_t* colmax, cudaStream_t s) {
     launch_zero_u32(colmax, N, s);
-    const int col_blocks = (int)((N + 2047) / 2048);
-    int splits = (int)std::max<int64_t>(1, std::min<int64_t>(K, (num_sms() * 8 + col_blocks - 1) / col_blocks));
+    // enough CTAs for two waves, but at least 64 rows per CTA
+    const int col_blocks = (int)((N + 255) / 256);
+    int splits = (int)std::max<int64_t>(1, (2 * num_sms() + col_blocks - 1) / col_blocks);
+    splits = (int)std::min<int64_t>(splits, std::max<int64_t>(1, K / 64));
     const int rows_per = (int)((K + splits - 1) / splits);
     splits = (int)((K + rows_per - 1) / rows_per);
     dim3 g1(col_blocks, splits);
