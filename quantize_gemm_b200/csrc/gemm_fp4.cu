@@ -17,9 +17,17 @@
 //   warp 0     TMA producer: 128-byte-swizzled 128 x 256 and BN x 256 FP4
 //              tiles of A and W^T into a kStages-deep shared-memory ring
 //   warp 1     TMEM allocator and MMA issuer (one thread): 4 MMAs of
-//              K = 64 per 256-wide k-block, accumulating in TMEM
-//   warps 2-5  epilogue: tcgen05.ld of the accumulator (one TMEM lane
-//              quarter each), scale, add C, store fp32 / bf16
+//              K = 64 per 256-wide k-block into one of two TMEM accumulators,
+//              so the next tile's MMAs run while the epilogue drains this one
+//   warps 2-5  epilogue, one TMEM lane quarter (32 rows) each, 32 columns at
+//              a time: tcgen05.ld of the accumulator, the C sub-tile arrives
+//              by TMA in swizzled shared memory, Y = acc * s_i * t_j + C is
+//              written back to the same buffer and leaves by a TMA store
+//              (double-buffered per warp).  A direct register-to-global path
+//              serves the raw-accumulator output and row pitches TMA cannot
+//              describe.
+// TMEM: accumulators at columns [0, BN) and [BN, 2 BN), constant block
+// scales (every byte 0x7F = 2^0) at [448, 512).
 // Every mbarrier wait is bounded; a wait that gives up sets the timeout bit in
 // the status word, raises a CTA-wide abort flag, waits (bounded) for copies
 // and MMAs in flight, frees TMEM and returns.
@@ -31,32 +39,43 @@ namespace qg {
 namespace gemm {
 
 constexpr int BM = 128;
-constexpr int BN = 256;
 constexpr int BK_BYTES = 128;       // 256 E2M1 values per row per k-block
 constexpr int UMMA_K_BYTES = 32;    // 64 E2M1 values per MMA
 constexpr int kStages = 4;
+constexpr int kAccStages = 2;
 constexpr int kEpiWarps = 4;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kTmemCols = 512;
-constexpr int kSfaCol = 448;        // constant block-scale region (0x7F = 2^0)
+constexpr int kSfaCol = 448;
 constexpr int kSfbCol = 480;
+constexpr int kEpiBuf = 32 * 32 * 4;   // one 32 x 32 fp32 sub-tile
 constexpr long long kWaitLimit = 2000000000LL;  // SM clocks (~1-2 s)
-
 constexpr int kStageABytes = BM * BK_BYTES;
-constexpr int kStageBBytes = BN * BK_BYTES;
+
+template <int BN>
+struct Cfg {
+    static_assert(BN % 32 == 0 && BN <= 224, "two accumulators + scales must fit in TMEM");
+    static constexpr int kStageBBytes = BN * BK_BYTES;
+    static constexpr size_t kOffB = (size_t)kStages * kStageABytes;
+    static constexpr size_t kOffEpi = kOffB + (size_t)kStages * kStageBBytes;
+    static constexpr size_t kOffBar = kOffEpi + (size_t)kEpiWarps * 2 * kEpiBuf;
+};
 
 struct alignas(8) Barriers {
     uint64_t full[kStages];
     uint64_t empty[kStages];
-    uint64_t acc_full;
-    uint64_t acc_empty;
+    uint64_t acc_full[kAccStages];
+    uint64_t acc_empty[kAccStages];
+    uint64_t cbar[kEpiWarps][2];
     uint64_t mma_done;
     uint32_t tmem_base;
     int abort;
 };
 
-constexpr size_t kSmemBytes =
-    1024 /*alignment slack*/ + (size_t)kStages * (kStageABytes + kStageBBytes) + sizeof(Barriers);
+template <int BN>
+constexpr size_t smem_bytes() {
+    return 1024 + Cfg<BN>::kOffBar + sizeof(Barriers);
+}
 
 // ------------------------------------------------------------------ PTX wraps
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -98,6 +117,12 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Barrie
         }
     }
 }
+// The same wait by a whole warp, with one verdict for all its lanes.
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, Barriers* B,
+                                               uint32_t* status) {
+    const bool ok = mbar_wait(bar, parity, B, status);
+    return __all_sync(0xFFFFFFFFu, ok);
+}
 // Bounded wait used during teardown (ignores the abort flag).
 __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
     const long long t0 = clock64();
@@ -112,6 +137,23 @@ __device__ __forceinline__ void tma_load_2d(const CUtensorMap* map, uint64_t* ba
         " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
         : "memory");
+}
+__device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int x, int y) {
+    asm volatile("cp.async.bulk.tensor.2d.global.shared::cta.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+                     reinterpret_cast<uint64_t>(map)),
+                 "r"(x), "r"(y), "r"(smem_u32(src))
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void bulk_wait_read() {
+    asm volatile("cp.async.bulk.wait_group.read %0;" ::"n"(N) : "memory");
+}
+__device__ __forceinline__ void bulk_wait_all() {
+    asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");
+}
+__device__ __forceinline__ void fence_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
 }
 
 __device__ __forceinline__ void tc_fence_before() {
@@ -140,6 +182,7 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr) {
 
 // Instruction descriptor of the block-scaled MMA: E2M1 x E2M1, UE8M0 scales,
 // both operands K-major, M = 128, N = BN, dense K = 64.
+template <int BN>
 __device__ __forceinline__ uint32_t mma_idesc() {
     return (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | (1u << 23) |
            ((uint32_t)(BM >> 4) << 24);
@@ -177,6 +220,11 @@ __device__ __forceinline__ void tmem_st32_const(uint32_t taddr, uint32_t c) {
         : "memory");
 }
 
+// Byte offset of 16-byte chunk `c` of row `r` in a 32-row TMA box with the
+// 128-byte (fp32 rows) or 64-byte (bf16 rows) swizzle.
+__device__ __forceinline__ uint32_t swz128(int r, int c) { return r * 128 + ((c ^ (r & 7)) << 4); }
+__device__ __forceinline__ uint32_t swz64(int r, int c) { return r * 64 + ((c ^ ((r >> 1) & 3)) << 4); }
+
 // ------------------------------------------------------------------ kernel
 struct Params {
     const float* sA;
@@ -187,6 +235,7 @@ struct Params {
     uint32_t* status;
     int M, N, K;
     int y_bf16;
+    int tma_epi;         // Y (and C) through TMA
 };
 
 __device__ __forceinline__ void tile_coords(int tile, int num_m, int& m_blk, int& n_blk) {
@@ -194,15 +243,49 @@ __device__ __forceinline__ void tile_coords(int tile, int num_m, int& m_blk, int
     n_blk = tile / num_m;
 }
 
+// Direct epilogue of one 32-column chunk: registers -> global (row per lane).
+__device__ __forceinline__ void epi_direct(const Params& p, const uint32_t (&v)[32], int row,
+                                           int col0, float s_row) {
+    const bool full = (p.N % 8) == 0 && (col0 + 32 <= p.N);
+    const int64_t off = (int64_t)row * p.N + col0;
+    if (p.raw_acc) {
+        if (full) {
+            float4* d = reinterpret_cast<float4*>(p.raw_acc + off);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                d[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                   __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+        } else {
+#pragma unroll
+            for (int j = 0; j < 32; ++j)
+                if (col0 + j < p.N) p.raw_acc[off + j] = __uint_as_float(v[j]);
+        }
+    }
+    if (p.Y == nullptr) return;
+#pragma unroll
+    for (int j = 0; j < 32; ++j) {
+        if (col0 + j >= p.N) continue;
+        float yy = __fmul_rn(__fmul_rn(__uint_as_float(v[j]), s_row), __ldg(p.sW + col0 + j));
+        if (p.C) yy = __fadd_rn(yy, __ldg(p.C + off + j));
+        if (p.y_bf16) static_cast<__nv_bfloat16*>(p.Y)[off + j] = __float2bfloat16_rn(yy);
+        else static_cast<float*>(p.Y)[off + j] = yy;
+    }
+}
+
+template <int BN>
 __global__ void __launch_bounds__(kThreads, 1)
 fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
-                const __grid_constant__ CUtensorMap tmap_b, const Params p) {
+                const __grid_constant__ CUtensorMap tmap_b,
+                const __grid_constant__ CUtensorMap tmap_y,
+                const __grid_constant__ CUtensorMap tmap_c, const Params p) {
+    using CF = Cfg<BN>;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     uint8_t* sa = smem;
-    uint8_t* sb = smem + (size_t)kStages * kStageABytes;
-    Barriers* B = reinterpret_cast<Barriers*>(sb + (size_t)kStages * kStageBBytes);
+    uint8_t* sb = smem + CF::kOffB;
+    uint8_t* sepi = smem + CF::kOffEpi;
+    Barriers* B = reinterpret_cast<Barriers*>(smem + CF::kOffBar);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -216,8 +299,14 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             mbar_init(&B->full[s], 1);
             mbar_init(&B->empty[s], 1);
         }
-        mbar_init(&B->acc_full, 1);
-        mbar_init(&B->acc_empty, kEpiWarps);
+        for (int s = 0; s < kAccStages; ++s) {
+            mbar_init(&B->acc_full[s], 1);
+            mbar_init(&B->acc_empty[s], kEpiWarps);
+        }
+        for (int w = 0; w < kEpiWarps; ++w) {
+            mbar_init(&B->cbar[w][0], 1);
+            mbar_init(&B->cbar[w][1], 1);
+        }
         mbar_init(&B->mma_done, 1);
         B->abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -252,9 +341,7 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     if (warp == 0) {
         // ---------------------------------------------------------- producer
         if (lane == 0) {
-            bool pend[kStages];
-            uint32_t pend_par[kStages];
-            for (int s = 0; s < kStages; ++s) pend[s] = false, pend_par[s] = 0;
+            uint32_t pend = 0, pend_par = 0;     // per-stage bit: load in flight / its parity
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
@@ -266,32 +353,34 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                         ok = false;
                         break;
                     }
-                    pend[stage] = false;
-                    mbar_expect_tx(&B->full[stage], (uint32_t)(kStageABytes + kStageBBytes));
+                    mbar_expect_tx(&B->full[stage], (uint32_t)(kStageABytes + CF::kStageBBytes));
                     tma_load_2d(&tmap_a, &B->full[stage], sa + (size_t)stage * kStageABytes,
                                 kb * BK_BYTES, m_blk * BM);
-                    tma_load_2d(&tmap_b, &B->full[stage], sb + (size_t)stage * kStageBBytes,
+                    tma_load_2d(&tmap_b, &B->full[stage], sb + (size_t)stage * CF::kStageBBytes,
                                 kb * BK_BYTES, n_blk * BN);
-                    pend[stage] = true;
-                    pend_par[stage] = phase;
+                    pend |= 1u << stage;
+                    pend_par = (pend_par & ~(1u << stage)) | (phase << stage);
                     if (++stage == kStages) stage = 0, phase ^= 1u;
                 }
             }
-            // copies still in flight complete before the CTA exits
-            for (int s = 0; s < kStages; ++s)
-                if (pend[s]) mbar_drain(&B->full[s], pend_par[s]);
+            // on abort, copies still in flight complete before the CTA exits
+            if (!ok) {
+                for (int s = 0; s < kStages; ++s)
+                    if ((pend >> s) & 1u) mbar_drain(&B->full[s], (pend_par >> s) & 1u);
+            }
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
         if (lane == 0) {
-            const uint32_t idesc = mma_idesc();
+            const uint32_t idesc = mma_idesc<BN>();
             const uint32_t sfa = tmem + kSfaCol, sfb = tmem + kSfbCol;
-            int stage = 0;
+            int stage = 0, as = 0;
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
             for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-                if (!mbar_wait(&B->acc_empty, acc_phase ^ 1u, B, p.status)) break;
+                if (!mbar_wait(&B->acc_empty[as], acc_phase ^ 1u, B, p.status)) break;
                 tc_fence_after();
+                const uint32_t d_tmem = tmem + (uint32_t)(as * BN);
                 for (int kb = 0; kb < num_kb; ++kb) {
                     if (!mbar_wait(&B->full[stage], phase, B, p.status)) {
                         ok = false;
@@ -299,10 +388,10 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     }
                     tc_fence_after();
                     const uint32_t a0 = smem_u32(sa + (size_t)stage * kStageABytes);
-                    const uint32_t b0 = smem_u32(sb + (size_t)stage * kStageBBytes);
+                    const uint32_t b0 = smem_u32(sb + (size_t)stage * CF::kStageBBytes);
 #pragma unroll
                     for (int ks = 0; ks < BK_BYTES / UMMA_K_BYTES; ++ks) {
-                        mma_mxf4(tmem, smem_desc(a0 + ks * UMMA_K_BYTES),
+                        mma_mxf4(d_tmem, smem_desc(a0 + ks * UMMA_K_BYTES),
                                  smem_desc(b0 + ks * UMMA_K_BYTES), idesc, sfa, sfb,
                                  (kb > 0 || ks > 0) ? 1u : 0u);
                     }
@@ -310,8 +399,8 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     if (++stage == kStages) stage = 0, phase ^= 1u;
                 }
                 if (!ok) break;
-                tc_commit(&B->acc_full);
-                acc_phase ^= 1u;
+                tc_commit(&B->acc_full[as]);
+                if (++as == kAccStages) as = 0, acc_phase ^= 1u;
             }
             // all issued MMAs complete before TMEM is released
             tc_commit(&B->mma_done);
@@ -319,98 +408,133 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         }
     } else {
         // ---------------------------------------------------------- epilogue
-        const int q = warp & 3;
+        const int ew = warp - 2;               // epilogue warp index (buffers)
+        const int q = warp & 3;                // TMEM lane quarter
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
+        uint8_t* buf0 = sepi + (size_t)ew * 2 * kEpiBuf;
+        const bool use_c = p.C != nullptr;
+        int as = 0;
         uint32_t acc_phase = 0;
-        const bool vec = (p.N % 8) == 0;
-        for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+        uint32_t cphase0 = 0, cphase1 = 0;
+        uint32_t cpend = 0;                    // C loads issued and not yet waited for
+        int nb = 0;                            // epilogue buffer of the next chunk
+        bool ok = true;
+        for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
             int m_blk, n_blk;
             tile_coords(tile, num_m, m_blk, n_blk);
-            if (!mbar_wait(&B->acc_full, acc_phase, B, p.status)) break;
-            acc_phase ^= 1u;
+            const int row0 = m_blk * BM + 32 * q;
+            const int row = row0 + lane;
+            const float s_row = row < p.M ? __ldg(p.sA + row) : 0.0f;
+            if (p.tma_epi && use_c && lane == 0) {
+                // first C sub-tile of this tile: its buffer's last store must be read out
+                bulk_wait_read<0>();
+                mbar_expect_tx(&B->cbar[ew][nb], kEpiBuf);
+                tma_load_2d(&tmap_c, &B->cbar[ew][nb], buf0 + nb * kEpiBuf, n_blk * BN, row0);
+            }
+            if (p.tma_epi && use_c) cpend |= 1u << nb;
+            if (!mbar_wait_warp(&B->acc_full[as], acc_phase, B, p.status)) {
+                ok = false;
+                break;
+            }
             tc_fence_after();
-            const int row = m_blk * BM + 32 * q + lane;
-            const bool row_ok = row < p.M;
-            const float s_row = row_ok ? p.sA[row] : 0.0f;
             for (int c = 0; c < BN / 32; ++c) {
+                const int col0 = n_blk * BN + c * 32;
                 uint32_t v[32];
-                tmem_ld32(tmem + lane_base + (uint32_t)(c * 32), v);
+                tmem_ld32(tmem + lane_base + (uint32_t)(as * BN + c * 32), v);
                 if (c == BN / 32 - 1) {
-                    // accumulator fully read: let the next tile's MMAs start
+                    // accumulator fully read: the next tile's MMAs may reuse it
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&B->acc_empty);
+                    if (lane == 0) mbar_arrive(&B->acc_empty[as]);
                 }
-                const int col0 = n_blk * BN + c * 32;
-                if (!row_ok || col0 >= p.N) continue;
-                const bool full = vec && (col0 + 32 <= p.N);
-                const int64_t off = (int64_t)row * p.N + col0;
-                if (p.raw_acc) {
-                    if (full) {
-                        float4* d = reinterpret_cast<float4*>(p.raw_acc + off);
-#pragma unroll
-                        for (int j = 0; j < 8; ++j)
-                            d[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
-                                               __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
-                    } else {
-#pragma unroll
-                        for (int j = 0; j < 32; ++j)
-                            if (col0 + j < p.N) p.raw_acc[off + j] = __uint_as_float(v[j]);
+                if (!p.tma_epi) {
+                    if (row < p.M && col0 < p.N) epi_direct(p, v, row, col0, s_row);
+                    continue;
+                }
+                const int cb = nb;
+                uint8_t* buf = buf0 + cb * kEpiBuf;
+                if (use_c && c + 1 < BN / 32) {
+                    // prefetch the next C sub-tile into the other buffer once the
+                    // store that last used it has finished reading it
+                    if (lane == 0) {
+                        bulk_wait_read<0>();
+                        mbar_expect_tx(&B->cbar[ew][cb ^ 1], kEpiBuf);
+                        tma_load_2d(&tmap_c, &B->cbar[ew][cb ^ 1], buf0 + (cb ^ 1) * kEpiBuf,
+                                    col0 + 32, row0);
                     }
+                    cpend |= 1u << (cb ^ 1);
                 }
-                if (p.Y == nullptr) continue;
-                float y[32];
-                if (full) {
-                    const float4* tw = reinterpret_cast<const float4*>(p.sW + col0);
+                float cv[32];
+                if (use_c) {
+                    const uint32_t par = cb ? cphase1 : cphase0;
+                    if (!mbar_wait_warp(&B->cbar[ew][cb], par, B, p.status)) {
+                        ok = false;
+                        break;
+                    }
+                    if (cb) cphase1 ^= 1u;
+                    else cphase0 ^= 1u;
+                    cpend &= ~(1u << cb);
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
-                        const float4 t = __ldg(tw + j);
-                        y[4 * j + 0] = __fmul_rn(__fmul_rn(__uint_as_float(v[4 * j + 0]), s_row), t.x);
-                        y[4 * j + 1] = __fmul_rn(__fmul_rn(__uint_as_float(v[4 * j + 1]), s_row), t.y);
-                        y[4 * j + 2] = __fmul_rn(__fmul_rn(__uint_as_float(v[4 * j + 2]), s_row), t.z);
-                        y[4 * j + 3] = __fmul_rn(__fmul_rn(__uint_as_float(v[4 * j + 3]), s_row), t.w);
+                        const float4 t = *reinterpret_cast<const float4*>(buf + swz128(lane, j));
+                        cv[4 * j] = t.x;
+                        cv[4 * j + 1] = t.y;
+                        cv[4 * j + 2] = t.z;
+                        cv[4 * j + 3] = t.w;
                     }
-                    if (p.C) {
-                        const float4* cc = reinterpret_cast<const float4*>(p.C + off);
+                } else {
+                    // this buffer's previous store must have finished reading it
+                    if (lane == 0) bulk_wait_read<1>();
+                    __syncwarp();
 #pragma unroll
-                        for (int j = 0; j < 8; ++j) {
-                            const float4 t = __ldg(cc + j);
-                            y[4 * j + 0] = __fadd_rn(y[4 * j + 0], t.x);
-                            y[4 * j + 1] = __fadd_rn(y[4 * j + 1], t.y);
-                            y[4 * j + 2] = __fadd_rn(y[4 * j + 2], t.z);
-                            y[4 * j + 3] = __fadd_rn(y[4 * j + 3], t.w);
+                    for (int j = 0; j < 32; ++j) cv[j] = 0.0f;
+                }
+                float y[32];
+                const float4* tw = reinterpret_cast<const float4*>(p.sW + col0);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
+                    if (col0 + 4 * j < p.N) t = __ldg(tw + j);
+                    y[4 * j + 0] = __fadd_rn(__fmul_rn(__fmul_rn(__uint_as_float(v[4 * j + 0]), s_row), t.x), cv[4 * j + 0]);
+                    y[4 * j + 1] = __fadd_rn(__fmul_rn(__fmul_rn(__uint_as_float(v[4 * j + 1]), s_row), t.y), cv[4 * j + 1]);
+                    y[4 * j + 2] = __fadd_rn(__fmul_rn(__fmul_rn(__uint_as_float(v[4 * j + 2]), s_row), t.z), cv[4 * j + 2]);
+                    y[4 * j + 3] = __fadd_rn(__fmul_rn(__fmul_rn(__uint_as_float(v[4 * j + 3]), s_row), t.w), cv[4 * j + 3]);
+                }
+                __syncwarp();   // every lane has read its C row before the buffer is overwritten
+                if (p.y_bf16) {
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        uint32_t w[4];
+#pragma unroll
+                        for (int i = 0; i < 4; ++i) {
+                            __nv_bfloat162 h = __floats2bfloat162_rn(y[8 * j + 2 * i], y[8 * j + 2 * i + 1]);
+                            w[i] = *reinterpret_cast<uint32_t*>(&h);
                         }
-                    }
-                    if (p.y_bf16) {
-                        uint4* d = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(p.Y) + off);
-#pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            uint32_t w[4];
-#pragma unroll
-                            for (int i = 0; i < 4; ++i) {
-                                __nv_bfloat162 h = __floats2bfloat162_rn(y[8 * j + 2 * i], y[8 * j + 2 * i + 1]);
-                                w[i] = *reinterpret_cast<uint32_t*>(&h);
-                            }
-                            d[j] = make_uint4(w[0], w[1], w[2], w[3]);
-                        }
-                    } else {
-                        float4* d = reinterpret_cast<float4*>(static_cast<float*>(p.Y) + off);
-#pragma unroll
-                        for (int j = 0; j < 8; ++j)
-                            d[j] = make_float4(y[4 * j], y[4 * j + 1], y[4 * j + 2], y[4 * j + 3]);
+                        *reinterpret_cast<uint4*>(buf + swz64(lane, j)) = make_uint4(w[0], w[1], w[2], w[3]);
                     }
                 } else {
 #pragma unroll
-                    for (int j = 0; j < 32; ++j) {
-                        if (col0 + j >= p.N) continue;
-                        float yy = __fmul_rn(__fmul_rn(__uint_as_float(v[j]), s_row), p.sW[col0 + j]);
-                        if (p.C) yy = __fadd_rn(yy, p.C[off + j]);
-                        if (p.y_bf16) static_cast<__nv_bfloat16*>(p.Y)[off + j] = __float2bfloat16_rn(yy);
-                        else static_cast<float*>(p.Y)[off + j] = yy;
-                    }
+                    for (int j = 0; j < 8; ++j)
+                        *reinterpret_cast<float4*>(buf + swz128(lane, j)) =
+                            make_float4(y[4 * j], y[4 * j + 1], y[4 * j + 2], y[4 * j + 3]);
                 }
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) {
+                    tma_store_2d(&tmap_y, buf, col0, row0);
+                    bulk_commit();
+                }
+                nb ^= 1;
             }
+            if (++as == kAccStages) as = 0, acc_phase ^= 1u;
         }
+        if (p.tma_epi && lane == 0) {
+            bulk_wait_all();
+            // on abort, C loads still in flight land before the CTA exits
+            if (cpend & 1u) mbar_drain(&B->cbar[ew][0], cphase0);
+            if (cpend & 2u) mbar_drain(&B->cbar[ew][1], cphase1);
+        }
+        __syncwarp();
     }
 
     tc_fence_before();
@@ -439,26 +563,52 @@ static EncodeTiledFn get_encode_fn() {
     return fn;
 }
 
-// 2-D map over packed codes: rows x (K/2) bytes, box (128 bytes) x box_rows.
-static bool make_code_map(CUtensorMap* map, const uint8_t* base, int64_t rows, int64_t kbytes,
-                          int box_rows) {
+static bool encode_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base, uint64_t inner,
+                      uint64_t rows, uint64_t row_bytes, uint32_t box_inner, uint32_t box_rows,
+                      CUtensorMapSwizzle swz) {
     EncodeTiledFn fn = get_encode_fn();
     if (!fn) return false;
-    cuuint64_t dims[2] = {(cuuint64_t)kbytes, (cuuint64_t)rows};
-    cuuint64_t strides[1] = {(cuuint64_t)kbytes};
-    cuuint32_t box[2] = {(cuuint32_t)BK_BYTES, (cuuint32_t)box_rows};
+    cuuint64_t dims[2] = {(cuuint64_t)inner, (cuuint64_t)rows};
+    cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+    cuuint32_t box[2] = {box_inner, box_rows};
     cuuint32_t estr[2] = {1, 1};
-    CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(base), dims,
-                    strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                    CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    return r == CUDA_SUCCESS;
+    return fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr,
+              CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Output tile width: the candidate with the least padding of the last tile.
+static int pick_bn(int64_t N) {
+    const int64_t w224 = ((N + 223) / 224) * 224 - N;
+    const int64_t w192 = ((N + 191) / 192) * 192 - N;
+    return (w192 < w224) ? 192 : 224;
+}
+
+template <int BN>
+static cudaError_t launch_bn(const CUtensorMap& ta, const uint8_t* codesWT, int64_t N, int64_t K,
+                             const CUtensorMap& ty, const CUtensorMap& tc, const Params& p,
+                             cudaStream_t s) {
+    CUtensorMap tb;
+    if (!encode_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, codesWT, K / 2, N, K / 2, BK_BYTES, BN,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    const int64_t tiles = ((p.M + BM - 1) / BM) * ((N + BN - 1) / BN);
+    const int grid = (int)std::min<int64_t>(tiles, num_sms());
+    fp4_gemm_kernel<BN><<<grid, kThreads, smem_bytes<BN>(), s>>>(ta, tb, ty, tc, p);
+    count_launch(1);
+    return cudaGetLastError();
 }
 
 }  // namespace gemm
 
 cudaError_t gemm_setup() {
-    return cudaFuncSetAttribute(gemm::fp4_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)gemm::kSmemBytes);
+    cudaError_t e = cudaFuncSetAttribute(gemm::fp4_gemm_kernel<224>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)gemm::smem_bytes<224>());
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(gemm::fp4_gemm_kernel<192>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)gemm::smem_bytes<192>());
 }
 
 // Returns cudaErrorInvalidValue when the tensor maps cannot be built.
@@ -467,9 +617,6 @@ cudaError_t launch_fp4_gemm(const uint8_t* codesA, const float* sA, const uint8_
                             void* Y, qg_dtype y_dtype, float* raw_acc, uint32_t* status,
                             cudaStream_t s) {
     using namespace gemm;
-    CUtensorMap ta, tb;
-    if (!make_code_map(&ta, codesA, M, K / 2, BM)) return cudaErrorInvalidValue;
-    if (!make_code_map(&tb, codesWT, N, K / 2, BN)) return cudaErrorInvalidValue;
     Params p;
     p.sA = sA;
     p.sW = sW;
@@ -481,11 +628,35 @@ cudaError_t launch_fp4_gemm(const uint8_t* codesA, const float* sA, const uint8_
     p.N = (int)N;
     p.K = (int)K;
     p.y_bf16 = (y_dtype == QG_BF16) ? 1 : 0;
-    const int64_t tiles = ((M + BM - 1) / BM) * ((N + BN - 1) / BN);
-    const int grid = (int)std::min<int64_t>(tiles, num_sms());
-    fp4_gemm_kernel<<<grid, kThreads, kSmemBytes, s>>>(ta, tb, p);
-    count_launch(1);
-    return cudaGetLastError();
+    // TMA epilogue: the row pitches of Y and C must be multiples of 16 bytes
+    const size_t ysz = (y_dtype == QG_BF16) ? 2 : 4;
+    p.tma_epi = (Y != nullptr && raw_acc == nullptr && ((size_t)N * ysz) % 16 == 0 &&
+                 ((size_t)N * 4) % 16 == 0)
+                    ? 1
+                    : 0;
+    CUtensorMap ta, ty, tc;
+    if (!encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, codesA, K / 2, M, K / 2, BK_BYTES, BM,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    ty = ta;
+    tc = ta;
+    if (p.tma_epi) {
+        if (y_dtype == QG_BF16) {
+            if (!encode_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, N, M, N * 2, 32, 32,
+                           CU_TENSOR_MAP_SWIZZLE_64B))
+                return cudaErrorInvalidValue;
+        } else {
+            if (!encode_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Y, N, M, N * 4, 32, 32,
+                           CU_TENSOR_MAP_SWIZZLE_128B))
+                return cudaErrorInvalidValue;
+        }
+        if (C != nullptr &&
+            !encode_2d(&tc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, C, N, M, N * 4, 32, 32,
+                       CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+    }
+    if (pick_bn(N) == 192) return launch_bn<192>(ta, codesWT, N, K, ty, tc, p, s);
+    return launch_bn<224>(ta, codesWT, N, K, ty, tc, p, s);
 }
 
 }  // namespace qg
