@@ -32,6 +32,8 @@ static cudaError_t ensure_device(int* dev_out) {
         if (e != cudaSuccess) return e;
         e = gemm_setup();
         if (e != cudaSuccess) return e;
+        e = spmm_setup();
+        if (e != cudaSuccess) return e;
         g_sms[dev] = sms;
         g_ready[dev] = true;
     }
@@ -255,10 +257,11 @@ qg_status qg_spmm_correction(const qg_csr* dA, int64_t M, const void* W, qg_dtyp
     if (M < 1 || N < 1 || K < 1) return QG_ERR_UNSUPPORTED_SHAPE;
     if (dA == nullptr || dA->row_ptr == nullptr) return QG_ERR_INVALID_ARG;
     if (W == nullptr || !aligned16(W) || ldw < N || C == nullptr || !aligned16(C)) return QG_ERR_INVALID_ARG;
-    qg_status st = check_ws(ws, ws_bytes, ws_layout(QG_OP_SPMM, M, K, N, w_dtype, 1.0).total);
+    const WsLayout L = ws_layout(QG_OP_SPMM, M, K, N, w_dtype, 1.0);
+    qg_status st = check_ws(ws, ws_bytes, L.total);
     if (st != QG_OK) return st;
     if (ensure_device(nullptr) != cudaSuccess) return QG_ERR_CUDA;
-    launch_spmm(dA, M, W, w_dtype, N, ldw, C, stream);
+    launch_spmm(dA, M, W, w_dtype, N, ldw, C, at<uint32_t>(ws, L.status), stream);
     return cuda_status(cudaGetLastError());
 }
 
@@ -312,7 +315,7 @@ qg_status qg_fp4_linear(const void* A, qg_dtype dtype, int64_t M, int64_t K,
     cudaError_t e = run_quantize_act(A, dtype, M, K, K, rank, act_buffers(ws, L), codes, scales, &csr,
                                      at<float>(ws, L.thr), stream);
     if (e != cudaSuccess) return QG_ERR_CUDA;
-    launch_spmm(&csr, M, W, dtype, N, N, C, stream);
+    launch_spmm(&csr, M, W, dtype, N, N, C, at<uint32_t>(ws, L.status), stream);
     if ((e = cudaGetLastError()) != cudaSuccess) return QG_ERR_CUDA;
     return cuda_status(launch_fp4_gemm(codes, scales, codesWT, sW, M, N, K, C, Y, y_dtype, nullptr,
                                        at<uint32_t>(ws, L.status), stream));

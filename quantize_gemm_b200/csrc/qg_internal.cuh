@@ -236,7 +236,7 @@ void launch_quantize_rows(const void* A, qg_dtype dt, int64_t M, int64_t K, int6
 void launch_quantize_cols(const void* W, qg_dtype dt, int64_t K, int64_t N, int64_t ldw,
                           uint8_t* codesT, float* scales, uint32_t* colmax, cudaStream_t s);
 void launch_spmm(const qg_csr* dA, int64_t M, const void* W, qg_dtype dt, int64_t N, int64_t ldw,
-                 float* C, cudaStream_t s);
+                 float* C, uint32_t* status, cudaStream_t s);
 cudaError_t launch_fp4_gemm(const uint8_t* codesA, const float* sA, const uint8_t* codesWT,
                             const float* sW, int64_t M, int64_t N, int64_t K, const float* C,
                             void* Y, qg_dtype y_dtype, float* raw_acc, uint32_t* status,
@@ -249,6 +249,7 @@ cudaError_t run_clamp_compensate(const void* A, qg_dtype dt, int64_t M, int64_t 
                                  float* T_out, cudaStream_t s);
 cudaError_t act_setup();
 cudaError_t gemm_setup();
+cudaError_t spmm_setup();
 
 // Number of SMs of the current device (cached per device id).
 int num_sms();
