@@ -115,98 +115,68 @@ spmm_slice_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restrict
 }
 
 // --------------------------------------------------------------------------
-// Fast path (bf16 W, N and ldw multiples of 8): the W row segments a warp needs
-// are fetched ahead with bulk async copies into a per-warp ring of 32 slots
-// (512 bytes each, one mbarrier per slot), so each warp keeps up to 16 KB of
-// W in flight without spending registers on it.  A warp owns 4 consecutive
-// rows: their CSR entries form one contiguous range, consumed in order; slot
-// j % 32 holds entry j and is refilled with entry j + 32 once every lane has
-// read it.  All waits are bounded; on a timeout the warp flags the status
-// word, waits (bounded) for its copies still in flight and stops.
-constexpr int kAsyncWarps = 4;
+// Fast path (bf16 W, N and ldw multiples of 8): W row segments are prefetched
+// with per-lane 16-byte cp.async copies into a per-lane ring of kDepth slots in
+// shared memory, so each warp keeps kDepth x 512 bytes of W in flight without
+// holding them in registers.  Every lane copies exactly the 16 bytes it will
+// read, so no synchronisation between lanes is needed: after committing the
+// copy of entry j + kDepth - 1, waiting until at most kDepth - 1 groups are
+// pending makes entry j's bytes visible to the lane that copied them.
+// A warp owns 4 consecutive rows, whose CSR entries form one contiguous
+// range consumed in order.
+constexpr int kAsyncWarps = 8;
 constexpr int kAsyncRowsPerWarp = 4;
-constexpr int kAsyncDepth = 32;
-constexpr int kAsyncSeg = kSpmmSlice * 2;   // bytes of one bf16 row segment
-constexpr long long kSpmmWaitLimit = 2000000000LL;
-constexpr size_t kAsyncSmem =
-    (size_t)kAsyncWarps * kAsyncDepth * kAsyncSeg + (size_t)kAsyncWarps * kAsyncDepth * 8;
+constexpr int kDepth = 16;
+constexpr size_t kAsyncSmem = (size_t)kAsyncWarps * kDepth * 32 * 16;
 
-__device__ __forceinline__ uint32_t smem_addr(const void* p) {
-    return (uint32_t)__cvta_generic_to_shared(p);
-}
-__device__ __forceinline__ bool slot_ready(uint64_t* bar, uint32_t parity) {
-    uint32_t ok;
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(smem_addr(bar)), "r"(parity)
-        : "memory");
-    return ok != 0;
-}
-__device__ __forceinline__ bool slot_wait(uint64_t* bar, uint32_t parity) {
-    if (slot_ready(bar, parity)) return true;
-    const long long t0 = clock64();
-    while (!slot_ready(bar, parity))
-        if (clock64() - t0 > kSpmmWaitLimit) return false;
-    return true;
-}
-__device__ __forceinline__ void slot_fetch(uint64_t* bar, void* dst, const void* src,
-                                           uint32_t bytes) {
-    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)),
-                 "r"(bytes)
+__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
+                     (uint32_t)__cvta_generic_to_shared(dst)),
+                 "l"(src)
                  : "memory");
-    asm volatile(
-        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
-            smem_addr(dst)),
-        "l"(src), "r"(bytes), "r"(smem_addr(bar))
-        : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() {
+    asm volatile("cp.async.commit_group;" ::: "memory");
+}
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 __global__ void __launch_bounds__(kAsyncWarps * 32)
 spmm_async_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col,
                   const double* __restrict__ val, const uint16_t* __restrict__ W, int64_t ldw,
-                  int M, int N, float* __restrict__ C, uint32_t* __restrict__ status) {
+                  int M, int N, float* __restrict__ C) {
     extern __shared__ __align__(128) uint8_t sm[];
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
-    uint8_t* ring = sm + (size_t)warp * kAsyncDepth * kAsyncSeg;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(sm + (size_t)kAsyncWarps * kAsyncDepth * kAsyncSeg) +
-                     warp * kAsyncDepth;
+    uint8_t* ring = sm + ((size_t)warp * kDepth * 32 + lane) * 16;   // slot s at ring + s * 512
     const int r_begin = (blockIdx.x * kAsyncWarps + warp) * kAsyncRowsPerWarp;
     if (r_begin >= M) return;
     const int r_end = min(M, r_begin + kAsyncRowsPerWarp);
-    if (lane == 0) {
-        for (int i = 0; i < kAsyncDepth; ++i)
-            asm volatile("mbarrier.init.shared::cta.b64 [%0], 1;" ::"r"(smem_addr(&bars[i])));
-        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    }
-    __syncwarp();
     const int n0 = blockIdx.y * kSpmmSlice;
-    const int ncols = min(kSpmmSlice, N - n0);
-    const uint32_t seg_bytes = (uint32_t)ncols * 2u;
-    const uint16_t* wslice = W + n0;
+    const bool lane_ok = n0 + lane * 8 < N;
+    const uint16_t* wlane = W + n0 + lane * 8;
     // row_ptr[r_begin .. r_end] held by lanes 0..4
     const int rp = (lane <= r_end - r_begin) ? row_ptr[r_begin + lane] : 0;
     const int P0 = __shfl_sync(0xFFFFFFFFu, rp, 0);
     const int P1 = __shfl_sync(0xFFFFFFFFu, rp, r_end - r_begin);
-    // prologue: entries P0 .. P0 + 31 into slots 0 .. 31
-    {
-        const int kn = (P0 + lane < P1) ? col[P0 + lane] : 0;
-        for (int t = 0; t < kAsyncDepth; ++t) {
-            const int k = __shfl_sync(0xFFFFFFFFu, kn, t);
-            if (lane == 0 && P0 + t < P1)
-                slot_fetch(&bars[t], ring + t * kAsyncSeg, wslice + (int64_t)k * ldw, seg_bytes);
-        }
+    // batches of 32 entries: current (kc, vc) and the next one's columns (kn)
+    int kc = (P0 + lane < P1) ? col[P0 + lane] : 0;
+    float vc = (P0 + lane < P1) ? (float)val[P0 + lane] : 0.0f;
+    int kn = (P0 + 32 + lane < P1) ? col[P0 + 32 + lane] : 0;
+    // prologue: entries P0 .. P0 + kDepth - 2
+#pragma unroll
+    for (int t = 0; t < kDepth - 1; ++t) {
+        const int k = __shfl_sync(0xFFFFFFFFu, kc, t);
+        if (lane_ok && P0 + t < P1) cp_async16(ring + t * 512, wlane + (int64_t)k * ldw);
+        cp_async_commit();
     }
-    const bool lane_ok = lane * 8 < ncols;
     float acc[8];
 #pragma unroll
     for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
     int row = r_begin;
     int rend = __shfl_sync(0xFFFFFFFFu, rp, 1);
-    int consumed = P0;            // entries consumed so far (absolute index)
-    bool ok = true;
     auto store_row = [&](int r) {
         if (lane_ok) {
             float4* d = reinterpret_cast<float4*>(C + (int64_t)r * N + n0 + lane * 8);
@@ -216,25 +186,25 @@ spmm_async_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restrict
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
     };
-    for (int B = P0; ok && B < P1; B += kAsyncDepth) {
-        const int cnt = min(kAsyncDepth, P1 - B);
-        const float vc = (B + lane < P1) ? (float)val[B + lane] : 0.0f;
-        const int kn = (B + kAsyncDepth + lane < P1) ? col[B + kAsyncDepth + lane] : 0;
-        const uint32_t par = (uint32_t)(((B - P0) / kAsyncDepth) & 1);
+    for (int B = P0; B < P1; B += 32) {
+        const int cnt = min(32, P1 - B);
         for (int t = 0; t < cnt; ++t) {
             const int j = B + t;
+            // look-ahead copy of entry j + kDepth - 1
+            const int li = t + kDepth - 1;
+            const int ka = __shfl_sync(0xFFFFFFFFu, kc, li & 31);
+            const int kb = __shfl_sync(0xFFFFFFFFu, kn, li & 31);
+            const int kl = li < 32 ? ka : kb;
+            if (lane_ok && j + kDepth - 1 < P1)
+                cp_async16(ring + ((j + kDepth - 1 - P0) % kDepth) * 512, wlane + (int64_t)kl * ldw);
+            cp_async_commit();
             while (j >= rend) {          // rows that end before entry j
                 store_row(row);
                 ++row;
                 rend = __shfl_sync(0xFFFFFFFFu, rp, row - r_begin + 1);
             }
-            const bool got = __all_sync(0xFFFFFFFFu, slot_wait(&bars[t], par));
-            if (!got) {
-                if (lane == 0) atomicOr(status, kStatusTimeout);
-                ok = false;
-                break;
-            }
-            const uint4 w = *reinterpret_cast<const uint4*>(ring + t * kAsyncSeg + lane * 16);
+            cp_async_wait<kDepth - 1>();
+            const uint4 w = *reinterpret_cast<const uint4*>(ring + ((j - P0) % kDepth) * 512);
             const float v = __shfl_sync(0xFFFFFFFFu, vc, t);
             const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
@@ -242,27 +212,13 @@ spmm_async_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restrict
                 acc[2 * i] = __fmaf_rn(v, __uint_as_float(ww[i] << 16), acc[2 * i]);
                 acc[2 * i + 1] = __fmaf_rn(v, __uint_as_float(ww[i] & 0xFFFF0000u), acc[2 * i + 1]);
             }
-            consumed = j + 1;
-            __syncwarp();                // every lane has read slot t
-            const int k = __shfl_sync(0xFFFFFFFFu, kn, t);
-            if (lane == 0 && j + kAsyncDepth < P1)
-                slot_fetch(&bars[t], ring + t * kAsyncSeg, wslice + (int64_t)k * ldw, seg_bytes);
         }
+        // advance the batches
+        kc = kn;
+        vc = (B + 32 + lane < P1) ? (float)val[B + 32 + lane] : 0.0f;
+        kn = (B + 64 + lane < P1) ? col[B + 64 + lane] : 0;
     }
-    if (!ok) {
-        // copies issued and not consumed: entries consumed .. min(P1, consumed + 31)
-        if (lane == 0) {
-            const int last = min(P1, consumed + kAsyncDepth);
-            for (int j = consumed; j < last; ++j) {
-                const int rel = j - P0;
-                const long long t0 = clock64();
-                while (!slot_ready(&bars[rel % kAsyncDepth], (uint32_t)((rel / kAsyncDepth) & 1)))
-                    if (clock64() - t0 > kSpmmWaitLimit) break;
-            }
-        }
-        __syncwarp();
-        return;
-    }
+    cp_async_wait<0>();
     while (row < r_end) {                // the last rows (and empty ones)
         store_row(row);
         ++row;
@@ -276,13 +232,13 @@ cudaError_t spmm_setup() {
 
 void launch_spmm(const qg_csr* dA, int64_t M, const void* W, qg_dtype dt, int64_t N, int64_t ldw,
                  float* C, uint32_t* status, cudaStream_t s) {
+    (void)status;   // no device-side waits that could time out
     if (dt == QG_BF16 && (N % 8) == 0 && (ldw % 8) == 0) {
         const int rows_per_cta = kAsyncWarps * kAsyncRowsPerWarp;
         dim3 grid((unsigned)((M + rows_per_cta - 1) / rows_per_cta),
                   (unsigned)((N + kSpmmSlice - 1) / kSpmmSlice));
         spmm_async_kernel<<<grid, kAsyncWarps * 32, kAsyncSmem, s>>>(
-            dA->row_ptr, dA->col, dA->val, static_cast<const uint16_t*>(W), ldw, (int)M, (int)N, C,
-            status);
+            dA->row_ptr, dA->col, dA->val, static_cast<const uint16_t*>(W), ldw, (int)M, (int)N, C);
         count_launch(1);
         return;
     }
