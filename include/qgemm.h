@@ -146,6 +146,27 @@ qg_status qg_quantize_cols(const void* W, qg_dtype dtype, int64_t K, int64_t N, 
                            uint8_t* codesT, float* scales, void* ws, size_t ws_bytes,
                            cudaStream_t stream);
 
+/* The same computation as qg_quantize_cols, for callers that cannot
+ * allocate device memory: code running under a fixed memory plan (an
+ * inference engine that has handed all device memory to its own pool and
+ * forbids further allocation while serving), or code that must not call
+ * cudaMalloc because it synchronises the device.  No workspace is taken and
+ * nothing is allocated: the column maxima live in a fixed array inside the
+ * library, sized for N <= 65536 columns (256 KB, held on every GPU that loads
+ * the library until the process exits).  The pages have no counterpart for
+ * this entry point; it is a deployment convenience.
+ *   - N > 65536 returns QG_ERR_UNSUPPORTED_SHAPE before anything is enqueued;
+ *     other argument checks are those of qg_quantize_cols.
+ *   - The first call on a device looks up the array's device address (a CUDA
+ *     runtime query); make that first call before any stream capture.
+ *   - Every call on a GPU uses that GPU's one array and zeroes what it needs
+ *     at the start; it keeps the last call's contents in between.  Calls
+ *     whose executions overlap on the same GPU (for example on two streams)
+ *     race on it: serialise them. */
+qg_status qg_quantize_cols_static(const void* W, qg_dtype dtype, int64_t K, int64_t N,
+                                  int64_t ldw, uint8_t* codesT, float* scales,
+                                  cudaStream_t stream);
+
 /* Outlier clamping and compensation ([FP4-writeup], outlier paragraph):
  * T = alpha-quantile of |A| (whole tensor), A_clamped = clamp(A, -T, T) in the
  * input dtype (M x K, contiguous, may be NULL), dA in CSR, T_out (device fp32,

@@ -40,6 +40,7 @@ EXPORTED = (
     "qg_workspace_size", "qg_workspace_init", "qg_sync_status", "qg_e2m1_encode",
     "qg_quantize_rows", "qg_quantize_cols", "qg_clamp_compensate", "qg_quantize_act",
     "qg_spmm_correction", "qg_fp4_gemm", "qg_fp4_linear", "qg_launch_count",
+    "qg_quantize_cols_static",
 )
 
 
@@ -74,6 +75,7 @@ _sig("qg_sync_status", _INT, [_P, _P])
 _sig("qg_e2m1_encode", _INT, [_P, _I64, _P, _P, _SZ, _P])
 _sig("qg_quantize_rows", _INT, [_P, _INT, _I64, _I64, _I64, _P, _P, _P, _SZ, _P])
 _sig("qg_quantize_cols", _INT, [_P, _INT, _I64, _I64, _I64, _P, _P, _P, _SZ, _P])
+_sig("qg_quantize_cols_static", _INT, [_P, _INT, _I64, _I64, _I64, _P, _P, _P])
 _sig("qg_clamp_compensate", _INT,
      [_P, _INT, _I64, _I64, _I64, _D, _P, ctypes.POINTER(_Csr), _P, _P, _SZ, _P])
 _sig("qg_quantize_act", _INT,
@@ -211,6 +213,14 @@ def qg_quantize_cols(W, codesT, scales, ws: Workspace, ldw=None, stream=None) ->
     K, N = W.shape
     return _lib.qg_quantize_cols(_ptr(W), _dt(W), K, N, W.stride(0) if ldw is None else ldw,
                                  _ptr(codesT), _ptr(scales), ws.ptr, ws.nbytes, _stream(stream))
+
+
+def qg_quantize_cols_static(W, codesT, scales, ldw=None, stream=None) -> int:
+    """qg_quantize_cols without a workspace (fixed in-library scratch, N <= 65536)."""
+    K, N = W.shape
+    return _lib.qg_quantize_cols_static(_ptr(W), _dt(W), K, N,
+                                        W.stride(0) if ldw is None else ldw, _ptr(codesT),
+                                        _ptr(scales), _stream(stream))
 
 
 def qg_clamp_compensate(A, alpha, A_clamped, csr: CSR, T_out, ws: Workspace, stream=None) -> int:

@@ -41,6 +41,8 @@ static cudaError_t ensure_device(int* dev_out) {
     return cudaSuccess;
 }
 
+cudaError_t device_setup() { return ensure_device(nullptr); }
+
 int num_sms() {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices || g_sms[dev] <= 0)

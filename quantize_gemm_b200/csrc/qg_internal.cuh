@@ -254,6 +254,10 @@ cudaError_t spmm_setup();
 // Number of SMs of the current device (cached per device id).
 int num_sms();
 
+// One-time per-device set-up of the library (kernel attributes, SM count),
+// for the current device.
+cudaError_t device_setup();
+
 // Count kernel launches enqueued by this library (reported by qg_launch_count).
 void count_launch(int n = 1);
 
