@@ -13,19 +13,27 @@
 // scaled FP4 MMA (tcgen05.mma kind::mxf4) with every block scale set to
 // UE8M0 1.0, which makes each MMA the plain E2M1 product.
 //
-// Structure (one CTA per SM, persistent over 128 x BN output tiles):
-//   warp 0     TMA producer: 128-byte-swizzled 128 x 256 and BN x 256 FP4
-//              tiles of A and W^T into a kStages-deep shared-memory ring
-//   warp 1     TMEM allocator and MMA issuer (one thread): 4 MMAs of
-//              K = 64 per 256-wide k-block into one of two TMEM accumulators,
-//              so the next tile's MMAs run while the epilogue drains this one
-//   warps 2-5  epilogue, one TMEM lane quarter (32 rows) each, 32 columns at
-//              a time: tcgen05.ld of the accumulator, the C sub-tile arrives
-//              by TMA in swizzled shared memory, Y = acc * s_i * t_j + C is
-//              written back to the same buffer and leaves by a TMA store
-//              (double-buffered per warp).  A direct register-to-global path
-//              serves the raw-accumulator output and row pitches TMA cannot
-//              describe.
+// Two variants of one kernel template, persistent over output tiles:
+//   PAIR = false  one CTA per SM computes 128 x BN tiles (tcgen05 cta_group::1)
+//   PAIR = true   a cluster of two CTAs (two SMs) computes 256 x BN tiles with
+//                 the 2-SM MMA (cta_group::2): each CTA loads its 128 rows of A
+//                 and half of the BN rows of W^T, so operand traffic from L2
+//                 per output element drops by about a third.  The leader CTA
+//                 (rank 0) issues the MMAs; the TMA loads of both CTAs signal
+//                 the leader's barriers; the leader's MMA commits signal both
+//                 CTAs' barriers.  Loads use no multicast.
+// Warp roles (192 threads per CTA):
+//   warp 0     TMA producer: 128-byte-swizzled FP4 tiles (256 values deep)
+//              into a kStages-deep shared-memory ring
+//   warp 1     TMEM allocator; in the (leader) CTA one thread issues the MMAs,
+//              K = 64 each, into one of two TMEM accumulators so the next
+//              tile's MMAs run while the epilogue drains this one
+//   warps 2-5  epilogue, one TMEM lane quarter (32 rows) each, 32 columns at a
+//              time: tcgen05.ld, the C sub-tile arrives by TMA in swizzled
+//              shared memory, Y = acc * s_i * t_j + C goes back into the same
+//              buffer and leaves by a TMA store (double-buffered per warp).  A
+//              direct register-to-global path serves the raw-accumulator
+//              output and row pitches that TMA cannot describe.
 // TMEM: accumulators at columns [0, BN) and [BN, 2 BN), constant block
 // scales (every byte 0x7F = 2^0) at [448, 512).
 // Every mbarrier wait is bounded; a wait that gives up sets the timeout bit in
@@ -38,10 +46,9 @@
 namespace qg {
 namespace gemm {
 
-constexpr int BM = 128;
+constexpr int BM = 128;             // rows of A per CTA
 constexpr int BK_BYTES = 128;       // 256 E2M1 values per row per k-block
 constexpr int UMMA_K_BYTES = 32;    // 64 E2M1 values per MMA
-constexpr int kStages = 4;
 constexpr int kAccStages = 2;
 constexpr int kEpiWarps = 4;
 constexpr int kThreads = 64 + 32 * kEpiWarps;
@@ -52,18 +59,23 @@ constexpr int kEpiBuf = 32 * 32 * 4;   // one 32 x 32 fp32 sub-tile
 constexpr long long kWaitLimit = 2000000000LL;  // SM clocks (~1-2 s)
 constexpr int kStageABytes = BM * BK_BYTES;
 
-template <int BN>
+template <int BN, bool PAIR>
 struct Cfg {
     static_assert(BN % 32 == 0 && BN <= 224, "two accumulators + scales must fit in TMEM");
-    static constexpr int kStageBBytes = BN * BK_BYTES;
+    static constexpr int kStages = PAIR ? 6 : 4;
+    static constexpr int kBRows = PAIR ? BN / 2 : BN;   // rows of W^T loaded by one CTA
+    static constexpr int kStageBBytes = kBRows * BK_BYTES;
+    static constexpr uint32_t kTxBytes = (PAIR ? 2u : 1u) * (kStageABytes + kStageBBytes);
+    static constexpr int kTileRows = PAIR ? 2 * BM : BM;
     static constexpr size_t kOffB = (size_t)kStages * kStageABytes;
     static constexpr size_t kOffEpi = kOffB + (size_t)kStages * kStageBBytes;
     static constexpr size_t kOffBar = kOffEpi + (size_t)kEpiWarps * 2 * kEpiBuf;
 };
 
+template <int S>
 struct alignas(8) Barriers {
-    uint64_t full[kStages];
-    uint64_t empty[kStages];
+    uint64_t full[S];
+    uint64_t empty[S];
     uint64_t acc_full[kAccStages];
     uint64_t acc_empty[kAccStages];
     uint64_t cbar[kEpiWarps][2];
@@ -72,9 +84,9 @@ struct alignas(8) Barriers {
     int abort;
 };
 
-template <int BN>
+template <int BN, bool PAIR>
 constexpr size_t smem_bytes() {
-    return 1024 + Cfg<BN>::kOffBar + sizeof(Barriers);
+    return 1024 + Cfg<BN, PAIR>::kOffBar + sizeof(Barriers<Cfg<BN, PAIR>::kStages>);
 }
 
 // ------------------------------------------------------------------ PTX wraps
@@ -92,6 +104,11 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
     asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
+// Arrive on a barrier given by its shared::cluster address (maybe the peer's).
+__device__ __forceinline__ void mbar_arrive_cluster(uint32_t cluster_addr) {
+    asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(cluster_addr)
+                 : "memory");
+}
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
@@ -103,24 +120,24 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
     return ok != 0;
 }
 // Bounded wait.  Returns false when the CTA is aborting or the limit passed.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, Barriers* B,
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, int* abort,
                                           uint32_t* status) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     while (true) {
         if (mbar_try_wait(bar, parity)) return true;
-        if (*reinterpret_cast<volatile int*>(&B->abort)) return false;
+        if (*reinterpret_cast<volatile int*>(abort)) return false;
         if (clock64() - t0 > kWaitLimit) {
-            *reinterpret_cast<volatile int*>(&B->abort) = 1;
+            *reinterpret_cast<volatile int*>(abort) = 1;
             flag_status(status, kStatusTimeout);
             return false;
         }
     }
 }
 // The same wait by a whole warp, with one verdict for all its lanes.
-__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, Barriers* B,
+__device__ __forceinline__ bool mbar_wait_warp(uint64_t* bar, uint32_t parity, int* abort,
                                                uint32_t* status) {
-    const bool ok = mbar_wait(bar, parity, B, status);
+    const bool ok = mbar_wait(bar, parity, abort, status);
     return __all_sync(0xFFFFFFFFu, ok);
 }
 // Bounded wait used during teardown (ignores the abort flag).
@@ -130,12 +147,37 @@ __device__ __forceinline__ void mbar_drain(uint64_t* bar, uint32_t parity) {
         if (clock64() - t0 > kWaitLimit) return;
 }
 
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                     : "memory");
+}
+// shared::cluster address of the same shared-memory object in CTA `rank`.
+__device__ __forceinline__ uint32_t map_to_rank(const void* p, uint32_t rank) {
+    uint32_t r;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+    return r;
+}
+
 __device__ __forceinline__ void tma_load_2d(const CUtensorMap* map, uint64_t* bar, void* dst,
                                             int x, int y) {
     asm volatile(
         "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
         " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
         "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+        : "memory");
+}
+// Load into this CTA's shared memory, completing on the leader CTA's barrier.
+__device__ __forceinline__ void tma_load_2d_pair(const CUtensorMap* map, uint32_t bar_cluster,
+                                                 void* dst, int x, int y) {
+    asm volatile(
+        "cp.async.bulk.tensor.2d.cta_group::2.shared::cluster.global.mbarrier::complete_tx::bytes"
+        " [%0], [%1, {%2, %3}], [%4];" ::"r"(smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(bar_cluster)
         : "memory");
 }
 __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void* src, int x, int y) {
@@ -162,10 +204,56 @@ __device__ __forceinline__ void tc_fence_before() {
 __device__ __forceinline__ void tc_fence_after() {
     asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
 }
-__device__ __forceinline__ void tc_commit(uint64_t* bar) {
-    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-                     smem_u32(bar))
-                 : "memory");
+// Commit this thread's outstanding MMAs to a barrier of this CTA (PAIR: the
+// barriers at the same offset in both CTAs of the pair).
+template <bool PAIR>
+__device__ __forceinline__ void tc_commit_all(uint64_t* bar) {
+    if constexpr (PAIR) {
+        asm volatile(
+            "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64"
+            " [%0], %1;" ::"r"(smem_u32(bar)),
+            "h"((uint16_t)0x3)
+            : "memory");
+    } else {
+        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                         smem_u32(bar))
+                     : "memory");
+    }
+}
+template <bool PAIR>
+__device__ __forceinline__ void tc_commit_local(uint64_t* bar) {
+    if constexpr (PAIR)
+        asm volatile("tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                         smem_u32(bar))
+                     : "memory");
+    else
+        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                         smem_u32(bar))
+                     : "memory");
+}
+
+template <bool PAIR>
+__device__ __forceinline__ void tmem_alloc(uint32_t* dst) {
+    if constexpr (PAIR) {
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(dst)),
+                     "r"(kTmemCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;");
+    } else {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_u32(dst)),
+                     "r"(kTmemCols));
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
+    }
+}
+template <bool PAIR>
+__device__ __forceinline__ void tmem_free(uint32_t taddr) {
+    if constexpr (PAIR)
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(taddr),
+                     "r"(kTmemCols));
+    else
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(taddr),
+                     "r"(kTmemCols));
 }
 
 // Shared-memory matrix descriptor: K-major, 128-byte swizzle, 8-row groups
@@ -181,21 +269,29 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr) {
 }
 
 // Instruction descriptor of the block-scaled MMA: E2M1 x E2M1, UE8M0 scales,
-// both operands K-major, M = 128, N = BN, dense K = 64.
-template <int BN>
+// both operands K-major, M = 128 (256 for the pair), N = BN, dense K = 64.
+template <int BN, bool PAIR>
 __device__ __forceinline__ uint32_t mma_idesc() {
-    return (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | (1u << 23) |
-           ((uint32_t)(BM >> 4) << 24);
+    constexpr uint32_t kM = PAIR ? 256u : 128u;
+    return (1u << 7) | (1u << 10) | ((uint32_t)(BN >> 3) << 17) | (1u << 23) | ((kM >> 4) << 24);
 }
 
+template <bool PAIR>
 __device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc,
                                          uint32_t idesc, uint32_t sfa, uint32_t sfb,
                                          uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;"
-        "\n\t}" ::"r"(d_tmem),
-        "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb));
+    if constexpr (PAIR)
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;"
+            "\n\t}" ::"r"(d_tmem),
+            "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb));
+    else
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::mxf4.block_scale.block32 [%0], %1, %2, %3, [%5], [%6], p;"
+            "\n\t}" ::"r"(d_tmem),
+            "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb));
 }
 
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
@@ -238,11 +334,6 @@ struct Params {
     int tma_epi;         // Y (and C) through TMA
 };
 
-__device__ __forceinline__ void tile_coords(int tile, int num_m, int& m_blk, int& n_blk) {
-    m_blk = tile % num_m;
-    n_blk = tile / num_m;
-}
-
 // Direct epilogue of one 32-column chunk: registers -> global (row per lane).
 __device__ __forceinline__ void epi_direct(const Params& p, const uint32_t (&v)[32], int row,
                                            int col0, float s_row) {
@@ -272,36 +363,41 @@ __device__ __forceinline__ void epi_direct(const Params& p, const uint32_t (&v)[
     }
 }
 
-template <int BN>
+template <int BN, bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
 fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 const __grid_constant__ CUtensorMap tmap_b,
                 const __grid_constant__ CUtensorMap tmap_y,
                 const __grid_constant__ CUtensorMap tmap_c, const Params p) {
-    using CF = Cfg<BN>;
+    using CF = Cfg<BN, PAIR>;
+    constexpr int S = CF::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     uint8_t* sa = smem;
     uint8_t* sb = smem + CF::kOffB;
     uint8_t* sepi = smem + CF::kOffEpi;
-    Barriers* B = reinterpret_cast<Barriers*>(smem + CF::kOffBar);
+    Barriers<S>* B = reinterpret_cast<Barriers<S>*>(smem + CF::kOffBar);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
-    const int num_m = (p.M + BM - 1) / BM;
+    const uint32_t rank = PAIR ? cluster_rank() : 0u;
+    const bool leader = rank == 0;
+    const int unit = PAIR ? (int)(blockIdx.x >> 1) : (int)blockIdx.x;    // CTA or CTA pair
+    const int n_units = PAIR ? (int)(gridDim.x >> 1) : (int)gridDim.x;
+    const int num_m = (p.M + CF::kTileRows - 1) / CF::kTileRows;
     const int num_n = (p.N + BN - 1) / BN;
     const int num_tiles = num_m * num_n;
     const int num_kb = (p.K / 2 + BK_BYTES - 1) / BK_BYTES;
 
     if (threadIdx.x == 0) {
-        for (int s = 0; s < kStages; ++s) {
+        for (int s = 0; s < S; ++s) {
             mbar_init(&B->full[s], 1);
             mbar_init(&B->empty[s], 1);
         }
         for (int s = 0; s < kAccStages; ++s) {
             mbar_init(&B->acc_full[s], 1);
-            mbar_init(&B->acc_empty[s], kEpiWarps);
+            mbar_init(&B->acc_empty[s], (PAIR ? 2 : 1) * kEpiWarps);
         }
         for (int w = 0; w < kEpiWarps; ++w) {
             mbar_init(&B->cbar[w][0], 1);
@@ -316,12 +412,7 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_a)) : "memory");
         asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(&tmap_b)) : "memory");
     }
-    if (warp == 1) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                         smem_u32(&B->tmem_base)),
-                     "r"(kTmemCols));
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;");
-    }
+    if (warp == 1) tmem_alloc<PAIR>(&B->tmem_base);
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
@@ -336,53 +427,70 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     }
     tc_fence_before();
     __syncthreads();
+    if constexpr (PAIR) cluster_sync();   // both CTAs' barriers and scales are ready
     tc_fence_after();
 
     if (warp == 0) {
         // ---------------------------------------------------------- producer
         if (lane == 0) {
-            uint32_t pend = 0, pend_par = 0;     // per-stage bit: load in flight / its parity
+            uint32_t pend = 0, pend_par = 0;     // per stage: load in flight / its parity
             int stage = 0;
             uint32_t phase = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-                int m_blk, n_blk;
-                tile_coords(tile, num_m, m_blk, n_blk);
+            for (int tile = unit; ok && tile < num_tiles; tile += n_units) {
+                const int m_blk = tile % num_m, n_blk = tile / num_m;
+                const int a_row = m_blk * CF::kTileRows + (int)rank * BM;
+                const int b_row = n_blk * BN + (int)rank * CF::kBRows;
                 for (int kb = 0; kb < num_kb; ++kb) {
-                    if (!mbar_wait(&B->empty[stage], phase ^ 1u, B, p.status)) {
+                    if (!mbar_wait(&B->empty[stage], phase ^ 1u, &B->abort, p.status)) {
                         ok = false;
                         break;
                     }
-                    mbar_expect_tx(&B->full[stage], (uint32_t)(kStageABytes + CF::kStageBBytes));
-                    tma_load_2d(&tmap_a, &B->full[stage], sa + (size_t)stage * kStageABytes,
-                                kb * BK_BYTES, m_blk * BM);
-                    tma_load_2d(&tmap_b, &B->full[stage], sb + (size_t)stage * CF::kStageBBytes,
-                                kb * BK_BYTES, n_blk * BN);
+                    uint8_t* da = sa + (size_t)stage * kStageABytes;
+                    uint8_t* db = sb + (size_t)stage * CF::kStageBBytes;
+                    if constexpr (PAIR) {
+                        if (leader) mbar_expect_tx(&B->full[stage], CF::kTxBytes);
+                        const uint32_t lb = map_to_rank(&B->full[stage], 0);
+                        tma_load_2d_pair(&tmap_a, lb, da, kb * BK_BYTES, a_row);
+                        tma_load_2d_pair(&tmap_b, lb, db, kb * BK_BYTES, b_row);
+                    } else {
+                        mbar_expect_tx(&B->full[stage], CF::kTxBytes);
+                        tma_load_2d(&tmap_a, &B->full[stage], da, kb * BK_BYTES, a_row);
+                        tma_load_2d(&tmap_b, &B->full[stage], db, kb * BK_BYTES, b_row);
+                    }
                     pend |= 1u << stage;
                     pend_par = (pend_par & ~(1u << stage)) | (phase << stage);
-                    if (++stage == kStages) stage = 0, phase ^= 1u;
+                    if (++stage == S) stage = 0, phase ^= 1u;
                 }
             }
-            // on abort, copies still in flight complete before the CTA exits
             if (!ok) {
-                for (int s = 0; s < kStages; ++s)
-                    if ((pend >> s) & 1u) mbar_drain(&B->full[s], (pend_par >> s) & 1u);
+                // on abort, copies still in flight land before the CTA exits
+                if (!PAIR || leader) {
+                    for (int s = 0; s < S; ++s)
+                        if ((pend >> s) & 1u) mbar_drain(&B->full[s], (pend_par >> s) & 1u);
+                } else {
+                    // the peer's loads complete on the leader's barriers: give
+                    // them a fixed grace period instead
+                    const long long t0 = clock64();
+                    while (clock64() - t0 < 2000000LL) {
+                    }
+                }
             }
         }
     } else if (warp == 1) {
         // ---------------------------------------------------------- MMA issuer
-        if (lane == 0) {
-            const uint32_t idesc = mma_idesc<BN>();
+        if (lane == 0 && leader) {
+            const uint32_t idesc = mma_idesc<BN, PAIR>();
             const uint32_t sfa = tmem + kSfaCol, sfb = tmem + kSfbCol;
             int stage = 0, as = 0;
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
-            for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-                if (!mbar_wait(&B->acc_empty[as], acc_phase ^ 1u, B, p.status)) break;
+            for (int tile = unit; ok && tile < num_tiles; tile += n_units) {
+                if (!mbar_wait(&B->acc_empty[as], acc_phase ^ 1u, &B->abort, p.status)) break;
                 tc_fence_after();
                 const uint32_t d_tmem = tmem + (uint32_t)(as * BN);
                 for (int kb = 0; kb < num_kb; ++kb) {
-                    if (!mbar_wait(&B->full[stage], phase, B, p.status)) {
+                    if (!mbar_wait(&B->full[stage], phase, &B->abort, p.status)) {
                         ok = false;
                         break;
                     }
@@ -391,19 +499,19 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     const uint32_t b0 = smem_u32(sb + (size_t)stage * CF::kStageBBytes);
 #pragma unroll
                     for (int ks = 0; ks < BK_BYTES / UMMA_K_BYTES; ++ks) {
-                        mma_mxf4(d_tmem, smem_desc(a0 + ks * UMMA_K_BYTES),
-                                 smem_desc(b0 + ks * UMMA_K_BYTES), idesc, sfa, sfb,
-                                 (kb > 0 || ks > 0) ? 1u : 0u);
+                        mma_mxf4<PAIR>(d_tmem, smem_desc(a0 + ks * UMMA_K_BYTES),
+                                       smem_desc(b0 + ks * UMMA_K_BYTES), idesc, sfa, sfb,
+                                       (kb > 0 || ks > 0) ? 1u : 0u);
                     }
-                    tc_commit(&B->empty[stage]);   // frees the stage when the MMAs finish
-                    if (++stage == kStages) stage = 0, phase ^= 1u;
+                    tc_commit_all<PAIR>(&B->empty[stage]);   // frees the stage (both CTAs)
+                    if (++stage == S) stage = 0, phase ^= 1u;
                 }
                 if (!ok) break;
-                tc_commit(&B->acc_full[as]);
+                tc_commit_all<PAIR>(&B->acc_full[as]);
                 if (++as == kAccStages) as = 0, acc_phase ^= 1u;
             }
             // all issued MMAs complete before TMEM is released
-            tc_commit(&B->mma_done);
+            tc_commit_local<PAIR>(&B->mma_done);
             mbar_drain(&B->mma_done, 0);
         }
     } else {
@@ -419,20 +527,21 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         uint32_t cpend = 0;                    // C loads issued and not yet waited for
         int nb = 0;                            // epilogue buffer of the next chunk
         bool ok = true;
-        for (int tile = blockIdx.x; ok && tile < num_tiles; tile += gridDim.x) {
-            int m_blk, n_blk;
-            tile_coords(tile, num_m, m_blk, n_blk);
-            const int row0 = m_blk * BM + 32 * q;
+        for (int tile = unit; ok && tile < num_tiles; tile += n_units) {
+            const int m_blk = tile % num_m, n_blk = tile / num_m;
+            const int row0 = m_blk * CF::kTileRows + (int)rank * BM + 32 * q;
             const int row = row0 + lane;
             const float s_row = row < p.M ? __ldg(p.sA + row) : 0.0f;
-            if (p.tma_epi && use_c && lane == 0) {
-                // first C sub-tile of this tile: its buffer's last store must be read out
-                bulk_wait_read<0>();
-                mbar_expect_tx(&B->cbar[ew][nb], kEpiBuf);
-                tma_load_2d(&tmap_c, &B->cbar[ew][nb], buf0 + nb * kEpiBuf, n_blk * BN, row0);
+            if (p.tma_epi && use_c) {
+                if (lane == 0) {
+                    // first C sub-tile of this tile; its buffer's last store must be read out
+                    bulk_wait_read<0>();
+                    mbar_expect_tx(&B->cbar[ew][nb], kEpiBuf);
+                    tma_load_2d(&tmap_c, &B->cbar[ew][nb], buf0 + nb * kEpiBuf, n_blk * BN, row0);
+                }
+                cpend |= 1u << nb;
             }
-            if (p.tma_epi && use_c) cpend |= 1u << nb;
-            if (!mbar_wait_warp(&B->acc_full[as], acc_phase, B, p.status)) {
+            if (!mbar_wait_warp(&B->acc_full[as], acc_phase, &B->abort, p.status)) {
                 ok = false;
                 break;
             }
@@ -445,7 +554,10 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     // accumulator fully read: the next tile's MMAs may reuse it
                     tc_fence_before();
                     __syncwarp();
-                    if (lane == 0) mbar_arrive(&B->acc_empty[as]);
+                    if (lane == 0) {
+                        if constexpr (PAIR) mbar_arrive_cluster(map_to_rank(&B->acc_empty[as], 0));
+                        else mbar_arrive(&B->acc_empty[as]);
+                    }
                 }
                 if (!p.tma_epi) {
                     if (row < p.M && col0 < p.N) epi_direct(p, v, row, col0, s_row);
@@ -467,7 +579,7 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 float cv[32];
                 if (use_c) {
                     const uint32_t par = cb ? cphase1 : cphase0;
-                    if (!mbar_wait_warp(&B->cbar[ew][cb], par, B, p.status)) {
+                    if (!mbar_wait_warp(&B->cbar[ew][cb], par, &B->abort, p.status)) {
                         ok = false;
                         break;
                     }
@@ -539,9 +651,9 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
 
     tc_fence_before();
     __syncthreads();
+    if constexpr (PAIR) cluster_sync();   // the peer no longer touches this CTA
     tc_fence_after();
-    if (warp == 1) asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
-                                "r"(kTmemCols));
+    if (warp == 1) tmem_free<PAIR>(tmem);
 }
 
 // ------------------------------------------------------------------ host side
@@ -584,31 +696,51 @@ static int pick_bn(int64_t N) {
     return (w192 < w224) ? 192 : 224;
 }
 
-template <int BN>
-static cudaError_t launch_bn(const CUtensorMap& ta, const uint8_t* codesWT, int64_t N, int64_t K,
-                             const CUtensorMap& ty, const CUtensorMap& tc, const Params& p,
-                             cudaStream_t s) {
+template <int BN, bool PAIR>
+static cudaError_t launch_variant(const CUtensorMap& ta, const uint8_t* codesWT, int64_t N,
+                                  int64_t K, const CUtensorMap& ty, const CUtensorMap& tc,
+                                  const Params& p, cudaStream_t s) {
+    using CF = Cfg<BN, PAIR>;
     CUtensorMap tb;
-    if (!encode_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, codesWT, K / 2, N, K / 2, BK_BYTES, BN,
-                   CU_TENSOR_MAP_SWIZZLE_128B))
+    if (!encode_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, codesWT, K / 2, N, K / 2, BK_BYTES,
+                   CF::kBRows, CU_TENSOR_MAP_SWIZZLE_128B))
         return cudaErrorInvalidValue;
-    const int64_t tiles = ((p.M + BM - 1) / BM) * ((N + BN - 1) / BN);
-    const int grid = (int)std::min<int64_t>(tiles, num_sms());
-    fp4_gemm_kernel<BN><<<grid, kThreads, smem_bytes<BN>(), s>>>(ta, tb, ty, tc, p);
+    const int64_t tiles = ((p.M + CF::kTileRows - 1) / CF::kTileRows) * ((N + BN - 1) / BN);
+    const int per_unit = PAIR ? 2 : 1;
+    const int units = (int)std::min<int64_t>(tiles, num_sms() / per_unit);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)(units * per_unit));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem_bytes<BN, PAIR>();
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = per_unit;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaError_t e = cudaLaunchKernelEx(&cfg, fp4_gemm_kernel<BN, PAIR>, ta, tb, ty, tc, p);
     count_launch(1);
-    return cudaGetLastError();
+    return e;
+}
+
+template <int BN, bool PAIR>
+static cudaError_t set_smem_attr() {
+    return cudaFuncSetAttribute(fp4_gemm_kernel<BN, PAIR>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                (int)smem_bytes<BN, PAIR>());
 }
 
 }  // namespace gemm
 
 cudaError_t gemm_setup() {
-    cudaError_t e = cudaFuncSetAttribute(gemm::fp4_gemm_kernel<224>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)gemm::smem_bytes<224>());
-    if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(gemm::fp4_gemm_kernel<192>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)gemm::smem_bytes<192>());
+    using namespace gemm;
+    cudaError_t e;
+    if ((e = set_smem_attr<224, false>()) != cudaSuccess) return e;
+    if ((e = set_smem_attr<192, false>()) != cudaSuccess) return e;
+    if ((e = set_smem_attr<224, true>()) != cudaSuccess) return e;
+    return set_smem_attr<192, true>();
 }
 
 // Returns cudaErrorInvalidValue when the tensor maps cannot be built.
@@ -655,8 +787,15 @@ cudaError_t launch_fp4_gemm(const uint8_t* codesA, const float* sA, const uint8_
                        CU_TENSOR_MAP_SWIZZLE_128B))
             return cudaErrorInvalidValue;
     }
-    if (pick_bn(N) == 192) return launch_bn<192>(ta, codesWT, N, K, ty, tc, p, s);
-    return launch_bn<224>(ta, codesWT, N, K, ty, tc, p, s);
+    // the CTA pair when there are enough 256-row tiles to fill the SMs in pairs
+    const bool pair = M > BM;
+    const int bn = pick_bn(N);
+    if (pair) {
+        if (bn == 192) return launch_variant<192, true>(ta, codesWT, N, K, ty, tc, p, s);
+        return launch_variant<224, true>(ta, codesWT, N, K, ty, tc, p, s);
+    }
+    if (bn == 192) return launch_variant<192, false>(ta, codesWT, N, K, ty, tc, p, s);
+    return launch_variant<224, false>(ta, codesWT, N, K, ty, tc, p, s);
 }
 
 }  // namespace qg
