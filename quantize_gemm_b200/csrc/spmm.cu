@@ -115,19 +115,24 @@ spmm_slice_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restrict
 }
 
 // --------------------------------------------------------------------------
-// Fast path (bf16 W, N and ldw multiples of 8): W row segments are prefetched
-// with per-lane 16-byte cp.async copies into a per-lane ring of kDepth slots in
-// shared memory, so each warp keeps kDepth x 512 bytes of W in flight without
-// holding them in registers.  Every lane copies exactly the 16 bytes it will
+// Fast path (bf16 W, N and ldw multiples of 8).  The kernel is bound by
+// instruction issue, so the work per non-zero is made as wide as possible:
+// a CTA owns a 512-column slice (each lane 16 columns, in two 256-column
+// halves so every load and store is coalesced), the bf16 pairs feed packed
+// fp32x2 FMAs (one rounding per product-sum, as fmaf), and W row segments are
+// prefetched with per-lane 16-byte cp.async copies into a per-lane ring of
+// kDepth slots in shared memory.  Every lane copies exactly the bytes it will
 // read, so no synchronisation between lanes is needed: after committing the
 // copy of entry j + kDepth - 1, waiting until at most kDepth - 1 groups are
 // pending makes entry j's bytes visible to the lane that copied them.
 // A warp owns 4 consecutive rows, whose CSR entries form one contiguous
 // range consumed in order.
-constexpr int kAsyncWarps = 8;
-constexpr int kAsyncRowsPerWarp = 4;
-constexpr int kDepth = 16;
-constexpr size_t kAsyncSmem = (size_t)kAsyncWarps * kDepth * 32 * 16;
+constexpr int kStreamWarps = 8;
+constexpr int kStreamRowsPerWarp = 4;
+constexpr int kStreamSlice = 512;
+constexpr int kDepth = 8;
+constexpr int kSlotBytes = 32 * 32;             // 32 lanes x 32 bytes
+constexpr size_t kAsyncSmem = (size_t)kStreamWarps * kDepth * kSlotBytes;
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
@@ -142,21 +147,33 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() {
     asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
+// acc0 += v * lo(w), acc1 += v * hi(w) for a bf16 pair w, as one packed FMA.
+__device__ __forceinline__ void fma_bf16x2(float& a0, float& a1, float v, uint32_t w) {
+    asm("{\n\t.reg .b32 lo, hi;\n\t.reg .b64 x, acc, vv;\n\t"
+        "shl.b32 lo, %3, 16;\n\tand.b32 hi, %3, 0xFFFF0000;\n\t"
+        "mov.b64 x, {lo, hi};\n\tmov.b64 acc, {%0, %1};\n\tmov.b64 vv, {%2, %2};\n\t"
+        "fma.rn.f32x2 acc, x, vv, acc;\n\tmov.b64 {%0, %1}, acc;\n\t}"
+        : "+f"(a0), "+f"(a1)
+        : "f"(v), "r"(w));
+}
 
-__global__ void __launch_bounds__(kAsyncWarps * 32)
-spmm_async_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col,
-                  const double* __restrict__ val, const uint16_t* __restrict__ W, int64_t ldw,
-                  int M, int N, float* __restrict__ C) {
+__global__ void __launch_bounds__(kStreamWarps * 32)
+spmm_stream_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col,
+                   const double* __restrict__ val, const uint16_t* __restrict__ W, int64_t ldw,
+                   int M, int N, float* __restrict__ C) {
     extern __shared__ __align__(128) uint8_t sm[];
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
-    uint8_t* ring = sm + ((size_t)warp * kDepth * 32 + lane) * 16;   // slot s at ring + s * 512
-    const int r_begin = (blockIdx.x * kAsyncWarps + warp) * kAsyncRowsPerWarp;
+    // slot s of this lane: half 0 at ring + s * 1024, half 1 at + 512 (16 bytes each)
+    uint8_t* ring = sm + (size_t)warp * kDepth * kSlotBytes + lane * 16;
+    const int r_begin = (blockIdx.x * kStreamWarps + warp) * kStreamRowsPerWarp;
     if (r_begin >= M) return;
-    const int r_end = min(M, r_begin + kAsyncRowsPerWarp);
-    const int n0 = blockIdx.y * kSpmmSlice;
-    const bool lane_ok = n0 + lane * 8 < N;
-    const uint16_t* wlane = W + n0 + lane * 8;
+    const int r_end = min(M, r_begin + kStreamRowsPerWarp);
+    const int n0 = blockIdx.y * kStreamSlice + lane * 8;     // half 0 columns n0 .. n0 + 7
+    const int n1 = n0 + 256;                                   // half 1 columns n1 .. n1 + 7
+    const bool ok0 = n0 < N, ok1 = n1 < N;
+    const uint16_t* w0 = W + n0;
+    const uint16_t* w1 = W + n1;
     // row_ptr[r_begin .. r_end] held by lanes 0..4
     const int rp = (lane <= r_end - r_begin) ? row_ptr[r_begin + lane] : 0;
     const int P0 = __shfl_sync(0xFFFFFFFFu, rp, 0);
@@ -165,26 +182,37 @@ spmm_async_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restrict
     int kc = (P0 + lane < P1) ? col[P0 + lane] : 0;
     float vc = (P0 + lane < P1) ? (float)val[P0 + lane] : 0.0f;
     int kn = (P0 + 32 + lane < P1) ? col[P0 + 32 + lane] : 0;
-    // prologue: entries P0 .. P0 + kDepth - 2
+    auto fetch = [&](int slot, int k) {
+        uint8_t* d = ring + slot * kSlotBytes;
+        const int64_t off = (int64_t)k * ldw;
+        if (ok0) cp_async16(d, w0 + off);
+        if (ok1) cp_async16(d + 512, w1 + off);
+    };
 #pragma unroll
     for (int t = 0; t < kDepth - 1; ++t) {
         const int k = __shfl_sync(0xFFFFFFFFu, kc, t);
-        if (lane_ok && P0 + t < P1) cp_async16(ring + t * 512, wlane + (int64_t)k * ldw);
+        if (P0 + t < P1) fetch(t, k);
         cp_async_commit();
     }
-    float acc[8];
+    float acc[16];
 #pragma unroll
-    for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+    for (int e = 0; e < 16; ++e) acc[e] = 0.0f;
     int row = r_begin;
     int rend = __shfl_sync(0xFFFFFFFFu, rp, 1);
     auto store_row = [&](int r) {
-        if (lane_ok) {
-            float4* d = reinterpret_cast<float4*>(C + (int64_t)r * N + n0 + lane * 8);
+        float* crow = C + (int64_t)r * N;
+        if (ok0) {
+            float4* d = reinterpret_cast<float4*>(crow + n0);
             d[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
             d[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
         }
+        if (ok1) {
+            float4* d = reinterpret_cast<float4*>(crow + n1);
+            d[0] = make_float4(acc[8], acc[9], acc[10], acc[11]);
+            d[1] = make_float4(acc[12], acc[13], acc[14], acc[15]);
+        }
 #pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = 0.0f;
+        for (int e = 0; e < 16; ++e) acc[e] = 0.0f;
     };
     for (int B = P0; B < P1; B += 32) {
         const int cnt = min(32, P1 - B);
@@ -194,9 +222,7 @@ spmm_async_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restrict
             const int li = t + kDepth - 1;
             const int ka = __shfl_sync(0xFFFFFFFFu, kc, li & 31);
             const int kb = __shfl_sync(0xFFFFFFFFu, kn, li & 31);
-            const int kl = li < 32 ? ka : kb;
-            if (lane_ok && j + kDepth - 1 < P1)
-                cp_async16(ring + ((j + kDepth - 1 - P0) % kDepth) * 512, wlane + (int64_t)kl * ldw);
+            if (j + kDepth - 1 < P1) fetch((j + kDepth - 1 - P0) % kDepth, li < 32 ? ka : kb);
             cp_async_commit();
             while (j >= rend) {          // rows that end before entry j
                 store_row(row);
@@ -204,14 +230,18 @@ spmm_async_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restrict
                 rend = __shfl_sync(0xFFFFFFFFu, rp, row - r_begin + 1);
             }
             cp_async_wait<kDepth - 1>();
-            const uint4 w = *reinterpret_cast<const uint4*>(ring + ((j - P0) % kDepth) * 512);
+            const uint8_t* src = ring + ((j - P0) % kDepth) * kSlotBytes;
+            const uint4 a = *reinterpret_cast<const uint4*>(src);
+            const uint4 b = *reinterpret_cast<const uint4*>(src + 512);
             const float v = __shfl_sync(0xFFFFFFFFu, vc, t);
-            const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-            for (int i = 0; i < 4; ++i) {
-                acc[2 * i] = __fmaf_rn(v, __uint_as_float(ww[i] << 16), acc[2 * i]);
-                acc[2 * i + 1] = __fmaf_rn(v, __uint_as_float(ww[i] & 0xFFFF0000u), acc[2 * i + 1]);
-            }
+            fma_bf16x2(acc[0], acc[1], v, a.x);
+            fma_bf16x2(acc[2], acc[3], v, a.y);
+            fma_bf16x2(acc[4], acc[5], v, a.z);
+            fma_bf16x2(acc[6], acc[7], v, a.w);
+            fma_bf16x2(acc[8], acc[9], v, b.x);
+            fma_bf16x2(acc[10], acc[11], v, b.y);
+            fma_bf16x2(acc[12], acc[13], v, b.z);
+            fma_bf16x2(acc[14], acc[15], v, b.w);
         }
         // advance the batches
         kc = kn;
@@ -226,7 +256,7 @@ spmm_async_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restrict
 }
 
 cudaError_t spmm_setup() {
-    return cudaFuncSetAttribute(spmm_async_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+    return cudaFuncSetAttribute(spmm_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)kAsyncSmem);
 }
 
@@ -234,10 +264,10 @@ void launch_spmm(const qg_csr* dA, int64_t M, const void* W, qg_dtype dt, int64_
                  float* C, uint32_t* status, cudaStream_t s) {
     (void)status;   // no device-side waits that could time out
     if (dt == QG_BF16 && (N % 8) == 0 && (ldw % 8) == 0) {
-        const int rows_per_cta = kAsyncWarps * kAsyncRowsPerWarp;
+        const int rows_per_cta = kStreamWarps * kStreamRowsPerWarp;
         dim3 grid((unsigned)((M + rows_per_cta - 1) / rows_per_cta),
-                  (unsigned)((N + kSpmmSlice - 1) / kSpmmSlice));
-        spmm_async_kernel<<<grid, kAsyncWarps * 32, kAsyncSmem, s>>>(
+                  (unsigned)((N + kStreamSlice - 1) / kStreamSlice));
+        spmm_stream_kernel<<<grid, kStreamWarps * 32, kAsyncSmem, s>>>(
             dA->row_ptr, dA->col, dA->val, static_cast<const uint16_t*>(W), ldw, (int)M, (int)N, C);
         count_launch(1);
         return;
