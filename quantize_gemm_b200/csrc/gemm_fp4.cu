@@ -31,7 +31,8 @@
 //   warps 2-5  epilogue, one TMEM lane quarter (32 rows) each, 32 columns at a
 //              time: tcgen05.ld, the C sub-tile arrives by TMA in swizzled
 //              shared memory, Y = acc * s_i * t_j + C goes back into the same
-//              buffer and leaves by a TMA store (double-buffered per warp).  A
+//              buffer and leaves by a TMA store (three buffers per warp, C
+//              requested two chunks ahead, TMEM loads one chunk ahead).  A
 //              direct register-to-global path serves the raw-accumulator
 //              output and row pitches that TMA cannot describe.
 // TMEM: accumulators at columns [0, BN) and [BN, 2 BN), constant block
@@ -56,20 +57,22 @@ constexpr int kTmemCols = 512;
 constexpr int kSfaCol = 448;
 constexpr int kSfbCol = 480;
 constexpr int kEpiBuf = 32 * 32 * 4;   // one 32 x 32 fp32 sub-tile
+constexpr int kEpiBufs = 3;            // sub-tile buffers per epilogue warp
 constexpr long long kWaitLimit = 2000000000LL;  // SM clocks (~1-2 s)
 constexpr int kStageABytes = BM * BK_BYTES;
 
 template <int BN, bool PAIR>
 struct Cfg {
     static_assert(BN % 32 == 0 && BN <= 224, "two accumulators + scales must fit in TMEM");
-    static constexpr int kStages = PAIR ? 6 : 4;
+    static constexpr int kStages = PAIR ? 5 : 3;
     static constexpr int kBRows = PAIR ? BN / 2 : BN;   // rows of W^T loaded by one CTA
     static constexpr int kStageBBytes = kBRows * BK_BYTES;
     static constexpr uint32_t kTxBytes = (PAIR ? 2u : 1u) * (kStageABytes + kStageBBytes);
     static constexpr int kTileRows = PAIR ? 2 * BM : BM;
     static constexpr size_t kOffB = (size_t)kStages * kStageABytes;
     static constexpr size_t kOffEpi = kOffB + (size_t)kStages * kStageBBytes;
-    static constexpr size_t kOffBar = kOffEpi + (size_t)kEpiWarps * 2 * kEpiBuf;
+    static constexpr size_t kOffSw = kOffEpi + (size_t)kEpiWarps * kEpiBufs * kEpiBuf;
+    static constexpr size_t kOffBar = kOffSw + (size_t)kEpiWarps * BN * 4;
 };
 
 template <int S>
@@ -78,7 +81,7 @@ struct alignas(8) Barriers {
     uint64_t empty[S];
     uint64_t acc_full[kAccStages];
     uint64_t acc_empty[kAccStages];
-    uint64_t cbar[kEpiWarps][2];
+    uint64_t cbar[kEpiWarps][kEpiBufs];
     uint64_t mma_done;
     uint32_t tmem_base;
     int abort;
@@ -294,6 +297,37 @@ __device__ __forceinline__ void mma_mxf4(uint32_t d_tmem, uint64_t adesc, uint64
             "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate), "r"(sfa), "r"(sfb));
 }
 
+// Start a load of 32 accumulator columns (this warp's 32 lanes) into v; the
+// registers are valid only after tmem_ld_wait(v).
+__device__ __forceinline__ void tmem_ld32_issue(uint32_t taddr, uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+        "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]),
+          "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]),
+          "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]),
+          "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]),
+          "=r"(v[31])
+        : "r"(taddr));
+}
+// Wait for the loads issued so far; v is named so that no use of it can be
+// scheduled before the wait.
+__device__ __forceinline__ void tmem_ld_wait(uint32_t (&v)[32]) {
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(v[0]), "+r"(v[1]), "+r"(v[2]), "+r"(v[3]), "+r"(v[4]), "+r"(v[5]),
+                   "+r"(v[6]), "+r"(v[7]), "+r"(v[8]), "+r"(v[9]), "+r"(v[10]), "+r"(v[11]),
+                   "+r"(v[12]), "+r"(v[13]), "+r"(v[14]), "+r"(v[15]), "+r"(v[16]), "+r"(v[17]),
+                   "+r"(v[18]), "+r"(v[19]), "+r"(v[20]), "+r"(v[21]), "+r"(v[22]), "+r"(v[23]),
+                   "+r"(v[24]), "+r"(v[25]), "+r"(v[26]), "+r"(v[27]), "+r"(v[28]), "+r"(v[29]),
+                   "+r"(v[30]), "+r"(v[31])
+                 :
+                 : "memory");
+}
+__device__ __forceinline__ void tmem_ld_wait_all() {
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
     asm volatile(
         "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
@@ -399,10 +433,8 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             mbar_init(&B->acc_full[s], 1);
             mbar_init(&B->acc_empty[s], (PAIR ? 2 : 1) * kEpiWarps);
         }
-        for (int w = 0; w < kEpiWarps; ++w) {
-            mbar_init(&B->cbar[w][0], 1);
-            mbar_init(&B->cbar[w][1], 1);
-        }
+        for (int w = 0; w < kEpiWarps; ++w)
+            for (int b = 0; b < kEpiBufs; ++b) mbar_init(&B->cbar[w][b], 1);
         mbar_init(&B->mma_done, 1);
         B->abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -516,76 +548,84 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         }
     } else {
         // ---------------------------------------------------------- epilogue
+        // This warp walks its 32-column chunks of all its tiles as one stream:
+        // chunk g uses sub-tile buffer g % 3; with a correction C, the C
+        // sub-tile of chunk g + 2 is requested once chunk g is stored.
+        constexpr int NC = BN / 32;
         const int ew = warp - 2;               // epilogue warp index (buffers)
         const int q = warp & 3;                // TMEM lane quarter
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-        uint8_t* buf0 = sepi + (size_t)ew * 2 * kEpiBuf;
-        const bool use_c = p.C != nullptr;
+        uint8_t* bufs = sepi + (size_t)ew * kEpiBufs * kEpiBuf;
+        float* sw = reinterpret_cast<float*>(smem + CF::kOffSw) + ew * BN;
+        const bool use_c = p.tma_epi && p.C != nullptr;
+        const int my_tiles = unit < num_tiles ? (num_tiles - unit + n_units - 1) / n_units : 0;
+        const int total = my_tiles * NC;
+        uint32_t cphase = 0;                   // bit b: parity of the next wait on cbar[ew][b]
+        uint32_t cpend = 0;                    // bit b: a C load into buffer b not yet waited for
+        auto c_load = [&](int g) {
+            const int ti = g / NC, c = g - ti * NC;
+            const int tile = unit + ti * n_units;
+            const int mb = tile % num_m, nbk = tile / num_m;
+            const int b = g % kEpiBufs;
+            if (lane == 0) {
+                mbar_expect_tx(&B->cbar[ew][b], kEpiBuf);
+                tma_load_2d(&tmap_c, &B->cbar[ew][b], bufs + b * kEpiBuf, nbk * BN + c * 32,
+                            mb * CF::kTileRows + (int)rank * BM + 32 * q);
+            }
+            cpend |= 1u << b;
+        };
+        if (use_c) {
+            if (total > 0) c_load(0);
+            if (total > 1) c_load(1);
+        }
         int as = 0;
         uint32_t acc_phase = 0;
-        uint32_t cphase0 = 0, cphase1 = 0;
-        uint32_t cpend = 0;                    // C loads issued and not yet waited for
-        int nb = 0;                            // epilogue buffer of the next chunk
         bool ok = true;
-        for (int tile = unit; ok && tile < num_tiles; tile += n_units) {
+        uint32_t va[32], vb[32];
+        for (int ti = 0; ok && ti < my_tiles; ++ti) {
+            const int tile = unit + ti * n_units;
             const int m_blk = tile % num_m, n_blk = tile / num_m;
             const int row0 = m_blk * CF::kTileRows + (int)rank * BM + 32 * q;
             const int row = row0 + lane;
             const float s_row = row < p.M ? __ldg(p.sA + row) : 0.0f;
-            if (p.tma_epi && use_c) {
-                if (lane == 0) {
-                    // first C sub-tile of this tile; its buffer's last store must be read out
-                    bulk_wait_read<0>();
-                    mbar_expect_tx(&B->cbar[ew][nb], kEpiBuf);
-                    tma_load_2d(&tmap_c, &B->cbar[ew][nb], buf0 + nb * kEpiBuf, n_blk * BN, row0);
-                }
-                cpend |= 1u << nb;
+            // this tile's column scales into the warp's shared-memory copy
+            __syncwarp();
+            for (int i = lane; i < BN; i += 32) {
+                const int n = n_blk * BN + i;
+                sw[i] = n < p.N ? __ldg(p.sW + n) : 0.0f;
             }
+            __syncwarp();
             if (!mbar_wait_warp(&B->acc_full[as], acc_phase, &B->abort, p.status)) {
                 ok = false;
                 break;
             }
             tc_fence_after();
-            for (int c = 0; c < BN / 32; ++c) {
-                const int col0 = n_blk * BN + c * 32;
-                uint32_t v[32];
-                tmem_ld32(tmem + lane_base + (uint32_t)(as * BN + c * 32), v);
-                if (c == BN / 32 - 1) {
-                    // accumulator fully read: the next tile's MMAs may reuse it
-                    tc_fence_before();
-                    __syncwarp();
-                    if (lane == 0) {
-                        if constexpr (PAIR) mbar_arrive_cluster(map_to_rank(&B->acc_empty[as], 0));
-                        else mbar_arrive(&B->acc_empty[as]);
-                    }
+            const uint32_t tbase = tmem + lane_base + (uint32_t)(as * BN);
+            auto release_acc = [&]() {
+                // accumulator fully read: the next tile's MMAs may reuse it
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    if constexpr (PAIR) mbar_arrive_cluster(map_to_rank(&B->acc_empty[as], 0));
+                    else mbar_arrive(&B->acc_empty[as]);
                 }
+            };
+            // one 32-column chunk: Y = acc * s_i * t_j + C, staged and stored by TMA
+            auto chunk = [&](const uint32_t (&v)[32], int c) -> bool {
+                const int col0 = n_blk * BN + c * 32;
                 if (!p.tma_epi) {
                     if (row < p.M && col0 < p.N) epi_direct(p, v, row, col0, s_row);
-                    continue;
+                    return true;
                 }
-                const int cb = nb;
-                uint8_t* buf = buf0 + cb * kEpiBuf;
-                if (use_c && c + 1 < BN / 32) {
-                    // prefetch the next C sub-tile into the other buffer once the
-                    // store that last used it has finished reading it
-                    if (lane == 0) {
-                        bulk_wait_read<0>();
-                        mbar_expect_tx(&B->cbar[ew][cb ^ 1], kEpiBuf);
-                        tma_load_2d(&tmap_c, &B->cbar[ew][cb ^ 1], buf0 + (cb ^ 1) * kEpiBuf,
-                                    col0 + 32, row0);
-                    }
-                    cpend |= 1u << (cb ^ 1);
-                }
+                const int g = ti * NC + c;
+                const int b = g % kEpiBufs;
+                uint8_t* buf = bufs + b * kEpiBuf;
                 float cv[32];
                 if (use_c) {
-                    const uint32_t par = cb ? cphase1 : cphase0;
-                    if (!mbar_wait_warp(&B->cbar[ew][cb], par, &B->abort, p.status)) {
-                        ok = false;
-                        break;
-                    }
-                    if (cb) cphase1 ^= 1u;
-                    else cphase0 ^= 1u;
-                    cpend &= ~(1u << cb);
+                    if (!mbar_wait_warp(&B->cbar[ew][b], (cphase >> b) & 1u, &B->abort, p.status))
+                        return false;
+                    cphase ^= 1u << b;
+                    cpend &= ~(1u << b);
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         const float4 t = *reinterpret_cast<const float4*>(buf + swz128(lane, j));
@@ -595,18 +635,17 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                         cv[4 * j + 3] = t.w;
                     }
                 } else {
-                    // this buffer's previous store must have finished reading it
-                    if (lane == 0) bulk_wait_read<1>();
+                    // buffer b was last read by the store of chunk g - 3
+                    if (lane == 0) bulk_wait_read<2>();
                     __syncwarp();
 #pragma unroll
                     for (int j = 0; j < 32; ++j) cv[j] = 0.0f;
                 }
                 float y[32];
-                const float4* tw = reinterpret_cast<const float4*>(p.sW + col0);
+                const float4* tw = reinterpret_cast<const float4*>(sw + c * 32);
 #pragma unroll
                 for (int j = 0; j < 8; ++j) {
-                    float4 t = make_float4(0.f, 0.f, 0.f, 0.f);
-                    if (col0 + 4 * j < p.N) t = __ldg(tw + j);
+                    const float4 t = tw[j];
                     y[4 * j + 0] = __fadd_rn(__fmul_rn(__fmul_rn(__uint_as_float(v[4 * j + 0]), s_row), t.x), cv[4 * j + 0]);
                     y[4 * j + 1] = __fadd_rn(__fmul_rn(__fmul_rn(__uint_as_float(v[4 * j + 1]), s_row), t.y), cv[4 * j + 1]);
                     y[4 * j + 2] = __fadd_rn(__fmul_rn(__fmul_rn(__uint_as_float(v[4 * j + 2]), s_row), t.z), cv[4 * j + 2]);
@@ -636,15 +675,40 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     tma_store_2d(&tmap_y, buf, col0, row0);
                     bulk_commit();
                 }
-                nb ^= 1;
+                if (use_c && g + 2 < total) {
+                    // buffer (g + 2) % 3 was last read by the store of chunk g - 1
+                    if (lane == 0) bulk_wait_read<1>();
+                    c_load(g + 2);
+                }
+                return true;
+            };
+            tmem_ld32_issue(tbase, va);
+            for (int c = 0; c < NC; c += 2) {
+                tmem_ld_wait(va);
+                if (c + 1 < NC) tmem_ld32_issue(tbase + (uint32_t)((c + 1) * 32), vb);
+                else release_acc();
+                if (!chunk(va, c)) {
+                    ok = false;
+                    break;
+                }
+                if (c + 1 < NC) {
+                    tmem_ld_wait(vb);
+                    if (c + 2 < NC) tmem_ld32_issue(tbase + (uint32_t)((c + 2) * 32), va);
+                    else release_acc();
+                    if (!chunk(vb, c + 1)) {
+                        ok = false;
+                        break;
+                    }
+                }
             }
             if (++as == kAccStages) as = 0, acc_phase ^= 1u;
         }
+        tmem_ld_wait_all();
         if (p.tma_epi && lane == 0) {
             bulk_wait_all();
             // on abort, C loads still in flight land before the CTA exits
-            if (cpend & 1u) mbar_drain(&B->cbar[ew][0], cphase0);
-            if (cpend & 2u) mbar_drain(&B->cbar[ew][1], cphase1);
+            for (int b = 0; b < kEpiBufs; ++b)
+                if ((cpend >> b) & 1u) mbar_drain(&B->cbar[ew][b], (cphase >> b) & 1u);
         }
         __syncwarp();
     }

@@ -117,8 +117,8 @@ spmm_slice_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restrict
 // --------------------------------------------------------------------------
 // Fast path (bf16 W, N and ldw multiples of 8).  The kernel is bound by
 // instruction issue, so the work per non-zero is made as wide as possible:
-// a CTA owns a 512-column slice (each lane 16 columns, in two 256-column
-// halves so every load and store is coalesced), the bf16 pairs feed packed
+// a CTA owns a 1024-column slice (each lane 32 columns, in four 256-column
+// quarters so every load and store is coalesced), the bf16 pairs feed packed
 // fp32x2 FMAs (one rounding per product-sum, as fmaf), and W row segments are
 // prefetched with per-lane 16-byte cp.async copies into a per-lane ring of
 // kDepth slots in shared memory.  Every lane copies exactly the bytes it will
@@ -129,9 +129,10 @@ spmm_slice_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restrict
 // range consumed in order.
 constexpr int kStreamWarps = 8;
 constexpr int kStreamRowsPerWarp = 4;
-constexpr int kStreamSlice = 512;
-constexpr int kDepth = 8;
-constexpr int kSlotBytes = 32 * 32;             // 32 lanes x 32 bytes
+constexpr int kStreamParts = 4;                   // 256-column quarters per slice
+constexpr int kStreamSlice = 256 * kStreamParts;
+constexpr int kDepth = 4;
+constexpr int kSlotBytes = kStreamParts * 512;    // 32 lanes x 16 bytes per quarter
 constexpr size_t kAsyncSmem = (size_t)kStreamWarps * kDepth * kSlotBytes;
 
 __device__ __forceinline__ void cp_async16(void* dst, const void* src) {
@@ -164,16 +165,16 @@ spmm_stream_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restric
     extern __shared__ __align__(128) uint8_t sm[];
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
-    // slot s of this lane: half 0 at ring + s * 1024, half 1 at + 512 (16 bytes each)
+    // slot s of this lane: quarter h at ring + s * kSlotBytes + h * 512 (16 bytes)
     uint8_t* ring = sm + (size_t)warp * kDepth * kSlotBytes + lane * 16;
     const int r_begin = (blockIdx.x * kStreamWarps + warp) * kStreamRowsPerWarp;
     if (r_begin >= M) return;
     const int r_end = min(M, r_begin + kStreamRowsPerWarp);
-    const int n0 = blockIdx.y * kStreamSlice + lane * 8;     // half 0 columns n0 .. n0 + 7
-    const int n1 = n0 + 256;                                   // half 1 columns n1 .. n1 + 7
-    const bool ok0 = n0 < N, ok1 = n1 < N;
-    const uint16_t* w0 = W + n0;
-    const uint16_t* w1 = W + n1;
+    const int nbase = blockIdx.y * kStreamSlice + lane * 8;   // quarter h: nbase + 256 h
+    bool okh[kStreamParts];
+#pragma unroll
+    for (int h = 0; h < kStreamParts; ++h) okh[h] = nbase + 256 * h < N;
+    const uint16_t* wl = W + nbase;
     // row_ptr[r_begin .. r_end] held by lanes 0..4
     const int rp = (lane <= r_end - r_begin) ? row_ptr[r_begin + lane] : 0;
     const int P0 = __shfl_sync(0xFFFFFFFFu, rp, 0);
@@ -184,9 +185,10 @@ spmm_stream_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restric
     int kn = (P0 + 32 + lane < P1) ? col[P0 + 32 + lane] : 0;
     auto fetch = [&](int slot, int k) {
         uint8_t* d = ring + slot * kSlotBytes;
-        const int64_t off = (int64_t)k * ldw;
-        if (ok0) cp_async16(d, w0 + off);
-        if (ok1) cp_async16(d + 512, w1 + off);
+        const uint16_t* src = wl + (int64_t)k * ldw;
+#pragma unroll
+        for (int h = 0; h < kStreamParts; ++h)
+            if (okh[h]) cp_async16(d + h * 512, src + 256 * h);
     };
 #pragma unroll
     for (int t = 0; t < kDepth - 1; ++t) {
@@ -194,25 +196,23 @@ spmm_stream_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restric
         if (P0 + t < P1) fetch(t, k);
         cp_async_commit();
     }
-    float acc[16];
+    float acc[8 * kStreamParts];
 #pragma unroll
-    for (int e = 0; e < 16; ++e) acc[e] = 0.0f;
+    for (int e = 0; e < 8 * kStreamParts; ++e) acc[e] = 0.0f;
     int row = r_begin;
     int rend = __shfl_sync(0xFFFFFFFFu, rp, 1);
     auto store_row = [&](int r) {
-        float* crow = C + (int64_t)r * N;
-        if (ok0) {
-            float4* d = reinterpret_cast<float4*>(crow + n0);
-            d[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
-            d[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
-        }
-        if (ok1) {
-            float4* d = reinterpret_cast<float4*>(crow + n1);
-            d[0] = make_float4(acc[8], acc[9], acc[10], acc[11]);
-            d[1] = make_float4(acc[12], acc[13], acc[14], acc[15]);
+        float* crow = C + (int64_t)r * N + nbase;
+#pragma unroll
+        for (int h = 0; h < kStreamParts; ++h) {
+            if (okh[h]) {
+                float4* d = reinterpret_cast<float4*>(crow + 256 * h);
+                d[0] = make_float4(acc[8 * h + 0], acc[8 * h + 1], acc[8 * h + 2], acc[8 * h + 3]);
+                d[1] = make_float4(acc[8 * h + 4], acc[8 * h + 5], acc[8 * h + 6], acc[8 * h + 7]);
+            }
         }
 #pragma unroll
-        for (int e = 0; e < 16; ++e) acc[e] = 0.0f;
+        for (int e = 0; e < 8 * kStreamParts; ++e) acc[e] = 0.0f;
     };
     for (int B = P0; B < P1; B += 32) {
         const int cnt = min(32, P1 - B);
@@ -231,17 +231,15 @@ spmm_stream_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restric
             }
             cp_async_wait<kDepth - 1>();
             const uint8_t* src = ring + ((j - P0) % kDepth) * kSlotBytes;
-            const uint4 a = *reinterpret_cast<const uint4*>(src);
-            const uint4 b = *reinterpret_cast<const uint4*>(src + 512);
             const float v = __shfl_sync(0xFFFFFFFFu, vc, t);
-            fma_bf16x2(acc[0], acc[1], v, a.x);
-            fma_bf16x2(acc[2], acc[3], v, a.y);
-            fma_bf16x2(acc[4], acc[5], v, a.z);
-            fma_bf16x2(acc[6], acc[7], v, a.w);
-            fma_bf16x2(acc[8], acc[9], v, b.x);
-            fma_bf16x2(acc[10], acc[11], v, b.y);
-            fma_bf16x2(acc[12], acc[13], v, b.z);
-            fma_bf16x2(acc[14], acc[15], v, b.w);
+#pragma unroll
+            for (int h = 0; h < kStreamParts; ++h) {
+                const uint4 a = *reinterpret_cast<const uint4*>(src + h * 512);
+                fma_bf16x2(acc[8 * h + 0], acc[8 * h + 1], v, a.x);
+                fma_bf16x2(acc[8 * h + 2], acc[8 * h + 3], v, a.y);
+                fma_bf16x2(acc[8 * h + 4], acc[8 * h + 5], v, a.z);
+                fma_bf16x2(acc[8 * h + 6], acc[8 * h + 7], v, a.w);
+            }
         }
         // advance the batches
         kc = kn;
