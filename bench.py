@@ -1,7 +1,7 @@
 """Benchmark of the FP4 quantized linear layer on B200.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
-                    [--impl ours|reference] [--no-e2e] [--no-cpu-baseline]
+                    [--layer I] [--impl ours|reference] [--no-e2e] [--no-cpu-baseline]
 
 A step is one forward pass of every linear layer of the workload (default:
 the LLaMA-1.3B-shaped linears, M = 4096 tokens, bf16): for each layer the
@@ -127,13 +127,15 @@ class Layer:
         self.ws_act = qg.Workspace(qg.QG_OP_QUANTIZE_ACT, M, K, 1, dt, self.alpha, device=device)
         self.ws_spmm = qg.Workspace(qg.QG_OP_SPMM, M, K, N, dt, device=device)
         self.ws_gemm = qg.Workspace(qg.QG_OP_FP4_GEMM, M, K, N, qg.QG_F32, device=device)
-        self.ws_lin = qg.Workspace(qg.QG_OP_FP4_LINEAR, M, K, N, dt, self.alpha, device=device)
+        self.ws_lin = None          # allocated by the e2e arm (it holds its own M x N correction)
+        self.dt = dt
         self.flops = 2 * M * N * K
         self.a_bytes = M * K * self.A.element_size()
         self.w_bytes = K * N * self.W.element_size()
 
     def workspaces(self):
-        return (self.ws_cols, self.ws_act, self.ws_spmm, self.ws_gemm, self.ws_lin)
+        return tuple(w for w in (self.ws_cols, self.ws_act, self.ws_spmm, self.ws_gemm, self.ws_lin)
+                     if w is not None)
 
 
 KERNELS = ("quantize_cols", "quantize_act", "spmm", "fp4_gemm")
@@ -168,7 +170,8 @@ def our_arm(args, rank, world, device):
     from workloads import WORKLOADS
     wl = WORKLOADS[args.workload]
     peaks = _peaks()
-    layers = [Layer(qg, wl, i, device) for i in range(len(wl.layers))]
+    idx = range(len(wl.layers)) if args.layer is None else [args.layer]
+    layers = [Layer(qg, wl, i, device) for i in idx]
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream()
 
@@ -221,7 +224,7 @@ def our_arm(args, rank, world, device):
         total_ms = float(t.item())
     ms_per_step = total_ms / args.steps
     flops_step = sum(L.flops for L in layers)
-    tokens_step = wl.M          # tokens through the whole layer stream
+    tokens_step = wl.M          # tokens through the layers of the step
     value = world * flops_step * args.steps / (total_ms * 1e-3) / 1e12
 
     # roofline of each kernel, per launch
@@ -267,7 +270,8 @@ def our_arm(args, rank, world, device):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e2m1",
         "data": "synthetic",
-        "config": {"workload": wl.name, "description": wl.description, "M": wl.M,
+        "config": {"workload": wl.name if args.layer is None else f"{wl.name}:{layers[0].name}",
+                   "description": wl.description, "M": wl.M,
                    "layers": [[L.name, L.K, L.N] for L in layers], "alpha": wl.alphas[0],
                    "input_dtype": wl.dtype, "y_dtype": "f32",
                    "l2": "flushed (256 MiB write between timed steps)",
@@ -291,6 +295,9 @@ def e2e_arm(qg, args, layers, device, world):
     """Same metric through the public call qg_fp4_linear with host buffers:
     pinned host A -> device, weight quantization, the layer, Y -> pinned host,
     all inside the timed region."""
+    for L in layers:
+        if L.ws_lin is None:
+            L.ws_lin = qg.Workspace(qg.QG_OP_FP4_LINEAR, L.M, L.K, L.N, L.dt, L.alpha, device=device)
     hostA = [L.A.cpu().pin_memory() for L in layers]
     hostY = [torch.empty(L.Y.shape, dtype=L.Y.dtype).pin_memory() for L in layers]
     devA = [torch.empty_like(L.A) for L in layers]
@@ -396,8 +403,9 @@ def reference_arm(args, rank, world):
     from workloads import WORKLOADS, make_layer_inputs
     import oracle
     wl = WORKLOADS[args.workload]
+    idx = list(range(len(wl.layers))) if args.layer is None else [args.layer]
     A_list, W_list = [], []
-    for i in range(len(wl.layers)):
+    for i in idx:
         A, W = make_layer_inputs(wl, i, device="cpu")
         A_list.append(oracle.as_f32(A))
         W_list.append(oracle.as_f32(W))
@@ -408,7 +416,7 @@ def reference_arm(args, rank, world):
     total = 0.0
     for _ in range(args.steps):
         total += _oracle_sample(wl, A_list, W_list, rows)
-    flops = wl.flops()
+    flops = sum(2 * wl.M * wl.layers[i].K * wl.layers[i].N for i in idx)
     value = flops * args.steps / total / 1e12
     cores = oracle.num_threads()
     sample = (f"each step: quantizers on the full tensors of every {wl.name} layer, Y for "
@@ -418,8 +426,9 @@ def reference_arm(args, rank, world):
         "n_gpus": world, "steps": args.steps, "warmup": warm,
         "ms_per_step": round(1e3 * total / args.steps, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name, "M": wl.M,
-                   "layers": [[l.name, l.K, l.N] for l in wl.layers], "alpha": wl.alphas[0]},
+        "config": {"workload": wl.name if args.layer is None else f"{wl.name}:{wl.layers[idx[0]].name}",
+                   "M": wl.M, "layers": [[wl.layers[i].name, wl.layers[i].K, wl.layers[i].N] for i in idx],
+                   "alpha": wl.alphas[0]},
         "cpu_baseline": {"kind": "oracle", "cores": cores, "sample": sample,
                          "value": round(value, 6), "unit": "TFLOP/s"},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
@@ -433,6 +442,8 @@ def main():
     ap.add_argument("--steps", type=int, default=1000)
     ap.add_argument("--warmup", type=int, default=10)
     ap.add_argument("--workload", default="llama1.3b")
+    ap.add_argument("--layer", type=int, default=None,
+                    help="run one linear of the workload (index), e.g. for profiling")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
