@@ -32,65 +32,65 @@ constexpr int kQuantThreads = 256;
 
 // --------------------------------------------------------------------------
 // Selection of the bin that holds the entry of rank `rank` (0-based) in a
-// histogram of nbins = 1024 * per bins, by one CTA of 1024 threads.  Warp w
-// owns bins [w * 32 * per, (w + 1) * 32 * per); lanes read them coalesced.
-// Reads go around L1 (the bins were just written by atomics).
+// histogram of 1024 * PER bins, by one CTA of 1024 threads.  Reads go around
+// L1 (the bins were just written by atomics).
 struct SelectResult {
     uint32_t bin;
     unsigned long long below;   // entries in bins < bin
     int found;
 };
 
-__device__ SelectResult block_select(const uint32_t* __restrict__ hist, int nbins,
-                                     unsigned long long rank) {
+template <int PER>
+__device__ SelectResult block_select(const uint32_t* __restrict__ hist, unsigned long long rank) {
+    // 1024 threads; warp w owns bins [w * 32 * PER, (w + 1) * 32 * PER); lane l
+    // holds bins w * 32 * PER + 32 i + l, i < PER, in registers (one round of
+    // coalesced loads), so the walk inside the chosen segment reloads nothing.
     __shared__ unsigned long long s_warp[32];
     __shared__ SelectResult s_res;
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
-    const int seg = nbins / 32;                 // bins per warp
+    const int seg = 32 * PER;
     const uint32_t* h = hist + (int64_t)warp * seg;
+    uint32_t v[PER];
+#pragma unroll
+    for (int i = 0; i < PER; ++i) v[i] = __ldcg(h + 32 * i + lane);
     unsigned long long mine = 0;
-    for (int i = lane; i < seg; i += 32) mine += __ldcg(h + i);
+#pragma unroll
+    for (int i = 0; i < PER; ++i) mine += v[i];
 #pragma unroll
     for (int d = 16; d > 0; d >>= 1) mine += __shfl_xor_sync(0xFFFFFFFFu, mine, d);
     if (lane == 0) s_warp[warp] = mine;
     if (t == 0) s_res.found = 0;
     __syncthreads();
-    if (warp == 0) {
-        // find the warp segment holding the rank
-        unsigned long long w = s_warp[lane], incl = w;
+    unsigned long long before = 0, incl = 0;
+    for (int w = 0; w < 32; ++w) {
+        const unsigned long long c = s_warp[w];
+        if (w < warp) before += c;
+        if (w <= warp) incl += c;
+    }
+    if (before <= rank && rank < incl) {
+        // this warp's segment holds the rank: walk it 32 bins at a time
+        unsigned long long cum = before;
 #pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            unsigned long long u = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-            if (lane >= d) incl += u;
-        }
-        const unsigned long long excl = incl - w;
-        const unsigned hit = __ballot_sync(0xFFFFFFFFu, excl <= rank && rank < incl);
-        if (hit) {
-            const int ws = __ffs(hit) - 1;
-            unsigned long long cum = __shfl_sync(0xFFFFFFFFu, excl, ws);
-            const uint32_t* hs = hist + (int64_t)ws * seg;
-            // walk the segment 32 bins at a time
-            for (int base = 0; base < seg; base += 32) {
-                const unsigned long long c = __ldcg(hs + base + lane);
-                unsigned long long ci = c;
+        for (int i = 0; i < PER; ++i) {
+            const unsigned long long c = v[i];
+            unsigned long long ci = c;
 #pragma unroll
-                for (int d = 1; d < 32; d <<= 1) {
-                    unsigned long long u = __shfl_up_sync(0xFFFFFFFFu, ci, d);
-                    if (lane >= d) ci += u;
-                }
-                const unsigned long long ce = cum + ci - c;
-                const unsigned h2 = __ballot_sync(0xFFFFFFFFu, ce <= rank && rank < cum + ci);
-                if (h2) {
-                    const int lb = __ffs(h2) - 1;
-                    if (lane == lb) {
-                        s_res.bin = (uint32_t)(ws * seg + base + lb);
-                        s_res.below = ce;
-                        s_res.found = 1;
-                    }
-                    break;
-                }
-                cum += __shfl_sync(0xFFFFFFFFu, ci, 31);
+            for (int d = 1; d < 32; d <<= 1) {
+                unsigned long long u = __shfl_up_sync(0xFFFFFFFFu, ci, d);
+                if (lane >= d) ci += u;
             }
+            const unsigned long long ce = cum + ci - c;
+            const unsigned hit = __ballot_sync(0xFFFFFFFFu, ce <= rank && rank < cum + ci);
+            if (hit) {
+                const int lb = __ffs(hit) - 1;
+                if (lane == lb) {
+                    s_res.bin = (uint32_t)(warp * seg + 32 * i + lb);
+                    s_res.below = ce;
+                    s_res.found = 1;
+                }
+                break;
+            }
+            cum += __shfl_sync(0xFFFFFFFFu, ci, 31);
         }
     }
     __syncthreads();
@@ -181,7 +181,7 @@ hist_rowmax_kernel(const void* __restrict__ A, int64_t lda, int M, int K,
         if (v) atomicAdd(&ghist[i], v);
     }
     if (last_block_done(&ctr->done_hist)) {
-        const SelectResult r = block_select(ghist, kHist1Bins, rank);
+        const SelectResult r = block_select<kHist1Bins / 1024>(ghist, rank);
         if (DT == QG_BF16) finish_select<0>(r, ctr, status, T_out);
         else finish_select<1>(r, ctr, status, T_out);
     }
@@ -210,7 +210,7 @@ refine_hist_kernel(const float* __restrict__ A, int64_t lda, int M, int K,
         }
     }
     if (last_block_done(&ctr->done_refine)) {
-        const SelectResult r = block_select(ghist2, kHist2Bins, rank - ctr->sel_below);
+        const SelectResult r = block_select<kHist2Bins / 1024>(ghist2, rank - ctr->sel_below);
         finish_select<2>(r, ctr, status, T_out);
     }
 }
@@ -332,13 +332,16 @@ clamp_quant_kernel(const void* __restrict__ A, int64_t lda, int M, int K,
         if (lane == 0) b.rowcnt[row] = (uint32_t)row_rank;
     }
 
-    // last CTA: row_ptr = exclusive scan of the row counts
+    // last CTA: row_ptr = exclusive scan of the row counts.  Thread t owns a
+    // contiguous run of rows; its counts are read with independent loads (no
+    // load waits on another), then written back as running sums.
     if (last_block_done(&ctr->done_clamp)) {
         __shared__ unsigned long long s_warp[kQuantThreads / 32];
         const int t = threadIdx.x, w = t >> 5;
         const int per = (M + kQuantThreads - 1) / kQuantThreads;
         const int r0 = min(M, t * per), r1 = min(M, r0 + per);
         unsigned long long mine = 0;
+#pragma unroll 8
         for (int i = r0; i < r1; ++i) mine += __ldcg(b.rowcnt + i);
         unsigned long long v = mine;
 #pragma unroll
@@ -354,9 +357,11 @@ clamp_quant_kernel(const void* __restrict__ A, int64_t lda, int M, int K,
             total += s_warp[i];
         }
         unsigned long long run = before + v - mine;
+#pragma unroll 8
         for (int i = r0; i < r1; ++i) {
+            const uint32_t c = __ldcg(b.rowcnt + i);
             row_ptr[i] = (int32_t)run;
-            run += __ldcg(b.rowcnt + i);
+            run += c;
         }
         if (t == 0) {
             row_ptr[M] = (int32_t)total;

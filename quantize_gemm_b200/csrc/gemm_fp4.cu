@@ -31,8 +31,9 @@
 //   warps 2-5  epilogue, one TMEM lane quarter (32 rows) each, 32 columns at a
 //              time: tcgen05.ld, the C sub-tile arrives by TMA in swizzled
 //              shared memory, Y = acc * s_i * t_j + C goes back into the same
-//              buffer and leaves by a TMA store (three buffers per warp, C
-//              requested two chunks ahead, TMEM loads one chunk ahead).  A
+//              buffer and leaves by a TMA store (kEpiBufs buffers per warp, C
+//              requested kEpiBufs - 1 chunks ahead, TMEM loads one chunk
+//              ahead).  A
 //              direct register-to-global path serves the raw-accumulator
 //              output and row pitches that TMA cannot describe.
 // TMEM: accumulators at columns [0, BN) and [BN, 2 BN), constant block
@@ -56,15 +57,28 @@ constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kTmemCols = 512;
 constexpr int kSfaCol = 448;
 constexpr int kSfbCol = 480;
+// Pipeline depths (overridable at build time for tuning sweeps).
+#ifndef QG_GEMM_PAIR_STAGES
+#define QG_GEMM_PAIR_STAGES 5
+#endif
+#ifndef QG_GEMM_SOLO_STAGES
+#define QG_GEMM_SOLO_STAGES 3
+#endif
+#ifndef QG_GEMM_EPI_BUFS
+#define QG_GEMM_EPI_BUFS 3
+#endif
+#ifndef QG_GEMM_FORCE_BN
+#define QG_GEMM_FORCE_BN 0
+#endif
 constexpr int kEpiBuf = 32 * 32 * 4;   // one 32 x 32 fp32 sub-tile
-constexpr int kEpiBufs = 3;            // sub-tile buffers per epilogue warp
+constexpr int kEpiBufs = QG_GEMM_EPI_BUFS;   // sub-tile buffers per epilogue warp (>= 2)
 constexpr long long kWaitLimit = 2000000000LL;  // SM clocks (~1-2 s)
 constexpr int kStageABytes = BM * BK_BYTES;
 
 template <int BN, bool PAIR>
 struct Cfg {
     static_assert(BN % 32 == 0 && BN <= 224, "two accumulators + scales must fit in TMEM");
-    static constexpr int kStages = PAIR ? 5 : 3;
+    static constexpr int kStages = PAIR ? QG_GEMM_PAIR_STAGES : QG_GEMM_SOLO_STAGES;
     static constexpr int kBRows = PAIR ? BN / 2 : BN;   // rows of W^T loaded by one CTA
     static constexpr int kStageBBytes = kBRows * BK_BYTES;
     static constexpr uint32_t kTxBytes = (PAIR ? 2u : 1u) * (kStageABytes + kStageBBytes);
@@ -549,8 +563,8 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     } else {
         // ---------------------------------------------------------- epilogue
         // This warp walks its 32-column chunks of all its tiles as one stream:
-        // chunk g uses sub-tile buffer g % 3; with a correction C, the C
-        // sub-tile of chunk g + 2 is requested once chunk g is stored.
+        // chunk g uses sub-tile buffer g % kEpiBufs; with a correction C, the C
+        // sub-tile of chunk g + kEpiBufs - 1 is requested once chunk g is stored.
         constexpr int NC = BN / 32;
         const int ew = warp - 2;               // epilogue warp index (buffers)
         const int q = warp & 3;                // TMEM lane quarter
@@ -574,10 +588,8 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             }
             cpend |= 1u << b;
         };
-        if (use_c) {
-            if (total > 0) c_load(0);
-            if (total > 1) c_load(1);
-        }
+        if (use_c)
+            for (int g = 0; g < kEpiBufs - 1 && g < total; ++g) c_load(g);
         int as = 0;
         uint32_t acc_phase = 0;
         bool ok = true;
@@ -635,8 +647,8 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                         cv[4 * j + 3] = t.w;
                     }
                 } else {
-                    // buffer b was last read by the store of chunk g - 3
-                    if (lane == 0) bulk_wait_read<2>();
+                    // buffer b was last read by the store of chunk g - kEpiBufs
+                    if (lane == 0) bulk_wait_read<kEpiBufs - 1>();
                     __syncwarp();
 #pragma unroll
                     for (int j = 0; j < 32; ++j) cv[j] = 0.0f;
@@ -675,10 +687,10 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     tma_store_2d(&tmap_y, buf, col0, row0);
                     bulk_commit();
                 }
-                if (use_c && g + 2 < total) {
-                    // buffer (g + 2) % 3 was last read by the store of chunk g - 1
+                if (use_c && g + kEpiBufs - 1 < total) {
+                    // that buffer was last read by the store of chunk g - 1
                     if (lane == 0) bulk_wait_read<1>();
-                    c_load(g + 2);
+                    c_load(g + kEpiBufs - 1);
                 }
                 return true;
             };
@@ -853,7 +865,7 @@ cudaError_t launch_fp4_gemm(const uint8_t* codesA, const float* sA, const uint8_
     }
     // the CTA pair when there are enough 256-row tiles to fill the SMs in pairs
     const bool pair = M > BM;
-    const int bn = pick_bn(N);
+    const int bn = QG_GEMM_FORCE_BN ? QG_GEMM_FORCE_BN : pick_bn(N);
     if (pair) {
         if (bn == 192) return launch_variant<192, true>(ta, codesWT, N, K, ty, tc, p, s);
         return launch_variant<224, true>(ta, codesWT, N, K, ty, tc, p, s);
