@@ -51,6 +51,26 @@ def _peaks():
                 sm_max_mhz=1965.0, source="fallback")
 
 
+# ------------------------------------------------------------------ ranks
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """The largest value of x over all ranks (x itself on one rank).  Uses a
+    device tensor under NCCL and a host tensor under gloo."""
+    if world <= 1:
+        return float(x)
+    import torch.distributed as dist
+    dev = device if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([float(x)], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(work_per_rank_per_step: float, steps: int, max_ms: float,
+                       world: int) -> float:
+    """Whole-job throughput: the work all ranks did over the slowest rank's
+    time (units of work per second)."""
+    return world * work_per_rank_per_step * steps / (max_ms * 1e-3)
+
+
 # ------------------------------------------------------------------ clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -217,15 +237,11 @@ def our_arm(args, rank, world, device):
                 per_kernel_layer[k][i].append(t)
         for k in KERNELS:
             per_kernel[k].append(sum(per_kernel_layer[k][i][-1] for i in range(n_l)))
-    total_ms = sum(step_ms)
-    if world > 1:
-        t = torch.tensor([total_ms], dtype=torch.float64, device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(step_ms), world, device)
     ms_per_step = total_ms / args.steps
     flops_step = sum(L.flops for L in layers)
     tokens_step = wl.M          # tokens through the layers of the step
-    value = world * flops_step * args.steps / (total_ms * 1e-3) / 1e12
+    value = weak_scaling_value(flops_step, args.steps, total_ms, world) / 1e12
 
     # roofline of each kernel, per launch
     sm_mhz = clocks.get("sm_mhz") or peaks["sm_max_mhz"]
@@ -276,7 +292,7 @@ def our_arm(args, rank, world, device):
                    "input_dtype": wl.dtype, "y_dtype": "f32",
                    "l2": "flushed (256 MiB write between timed steps)",
                    "parallelism": f"replicas x{world}"},
-        "tokens_per_s": round(world * tokens_step * args.steps / (total_ms * 1e-3), 1),
+        "tokens_per_s": round(weak_scaling_value(tokens_step, args.steps, total_ms, world), 1),
         "quantizer_gbs": quant_gbs,
         "kernels": rows,
         "roofline": roofline,
@@ -294,51 +310,79 @@ def our_arm(args, rank, world, device):
 def e2e_arm(qg, args, layers, device, world):
     """Same metric through the public call qg_fp4_linear with host buffers:
     pinned host A -> device, weight quantization, the layer, Y -> pinned host,
-    all inside the timed region."""
+    all inside the timed region.  Uploads run on one copy stream, downloads on
+    another, the layers on the compute stream, ordered by events, so the PCIe
+    transfers of one layer overlap the computation of its neighbours."""
     for L in layers:
         if L.ws_lin is None:
             L.ws_lin = qg.Workspace(qg.QG_OP_FP4_LINEAR, L.M, L.K, L.N, L.dt, L.alpha, device=device)
     hostA = [L.A.cpu().pin_memory() for L in layers]
     hostY = [torch.empty(L.Y.shape, dtype=L.Y.dtype).pin_memory() for L in layers]
     devA = [torch.empty_like(L.A) for L in layers]
+    cs = torch.cuda.current_stream()
+    hs = torch.cuda.Stream(device=device)
+    ds = torch.cuda.Stream(device=device)
+    n = len(layers)
+    ev_up = [torch.cuda.Event() for _ in range(n)]
+    ev_done = [torch.cuda.Event() for _ in range(n)]
+    ev_down = [torch.cuda.Event() for _ in range(n)]
+    started = [False]
 
-    def step():
-        for L, hA, hY, dA in zip(layers, hostA, hostY, devA):
-            dA.copy_(hA, non_blocking=True)
+    def step(t0=None, t1=None):
+        if t0 is not None:
+            t0.record(cs)
+        start = torch.cuda.Event()
+        start.record(cs)
+        hs.wait_event(start)
+        for i in range(n):
+            if started[0]:
+                hs.wait_event(ev_done[i])       # the last step has finished reading devA[i]
+            with torch.cuda.stream(hs):
+                devA[i].copy_(hostA[i], non_blocking=True)
+            ev_up[i].record(hs)
+        for i, L in enumerate(layers):
+            cs.wait_event(ev_up[i])
+            if started[0]:
+                cs.wait_event(ev_down[i])       # the last step's Y[i] has left the device
             st = qg.qg_quantize_cols(L.W, L.codesT, L.t, L.ws_cols)
             if st != qg.QG_OK:
                 raise qg.QGError(st, "e2e quantize_cols")
-            st = qg.qg_fp4_linear(dA, L.codesT, L.t, L.W, L.alpha, L.Y, L.ws_lin)
+            st = qg.qg_fp4_linear(devA[i], L.codesT, L.t, L.W, L.alpha, L.Y, L.ws_lin)
             if st != qg.QG_OK:
                 raise qg.QGError(st, "e2e fp4_linear")
-            hY.copy_(L.Y, non_blocking=True)
+            ev_done[i].record(cs)
+            ds.wait_event(ev_done[i])
+            with torch.cuda.stream(ds):
+                hostY[i].copy_(L.Y, non_blocking=True)
+            ev_down[i].record(ds)
+        for i in range(n):
+            cs.wait_event(ev_down[i])
+        started[0] = True
+        if t1 is not None:
+            t1.record(cs)
 
     for _ in range(args.warmup):
         step()
     torch.cuda.synchronize()
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     total = 0.0
-    for k in range(max(1, args.steps // 10)):
+    e2e_steps = max(1, args.steps // 10)
+    for k in range(e2e_steps):
         flush.fill_(k & 0xFF)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        a.record()
-        step()
-        b.record()
+        step(a, b)
         torch.cuda.synchronize()
         total += a.elapsed_time(b)
     for L in layers:
         qg.check_status(L.ws_lin, "e2e")
-    if world > 1:
-        t = torch.tensor([total], dtype=torch.float64, device=device)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total = float(t.item())
+    total = max_over_ranks(total, world, device)
     flops = sum(L.flops for L in layers)
-    e2e_steps = max(1, args.steps // 10)
-    return {"value": round(world * flops * e2e_steps / (total * 1e-3) / 1e12, 3),
+    return {"value": round(weak_scaling_value(flops, e2e_steps, total, world) / 1e12, 3),
             "unit": "TFLOP/s", "steps": e2e_steps,
             "h2d_bytes_per_step": int(sum(L.a_bytes for L in layers)),
             "d2h_bytes_per_step": int(sum(L.Y.numel() * L.Y.element_size() for L in layers)),
-            "ms_per_step": round(total / e2e_steps, 4)}
+            "ms_per_step": round(total / e2e_steps, 4),
+            "overlap": "uploads, layers and downloads on three streams ordered by events"}
 
 
 def _ncu_traffic(kernel, workload):

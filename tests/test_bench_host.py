@@ -1,0 +1,71 @@
+"""Host-side logic of bench.py that the multi-GPU runs rely on, on CPU:
+max-over-ranks timing with a world_size-2 gloo group, the weak-scaling
+aggregate, and the seeded workload generator."""
+import os
+import socket
+
+import pytest
+import torch
+import torch.multiprocessing as mp
+
+import bench
+from workloads import WORKLOADS, make_layer_inputs, seed_for
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    import torch.distributed as dist
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        ms = 10.0 + 5.0 * rank                       # rank 1 is the slow one
+        m = bench.max_over_ranks(ms, world)
+        v = bench.weak_scaling_value(100.0, 4, m, world)
+        out[rank] = (m, v)
+    finally:
+        dist.destroy_process_group()
+
+
+def test_max_over_ranks_and_weak_scaling_with_gloo():
+    world = 2
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    manager = ctx.Manager()
+    out = manager.dict()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, out)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    for r in range(world):
+        m, v = out[r]
+        assert m == 15.0                              # the slowest rank's time
+        assert v == pytest.approx(2 * 100.0 * 4 / 15e-3)
+
+
+def test_single_rank_needs_no_process_group():
+    assert bench.max_over_ranks(3.5, 1) == 3.5
+    assert bench.weak_scaling_value(10.0, 2, 4.0, 1) == pytest.approx(5000.0)
+
+
+def test_workload_generator_is_seeded_and_shaped():
+    A1, W1 = make_layer_inputs("tiny", 0, device="cpu")
+    A2, W2 = make_layer_inputs("tiny", 0, device="cpu")
+    assert torch.equal(A1, A2) and torch.equal(W1, W2)
+    wl = WORKLOADS["tiny"]
+    assert A1.shape == (wl.M, wl.layers[0].K) and W1.shape == (wl.layers[0].K, wl.layers[0].N)
+    assert A1.dtype == torch.float32
+    # the 8-channel outliers: 0.5% of entries scaled by 50 lie in 8 columns
+    big = (A1.abs() > 10).nonzero()
+    assert 0 < big.shape[0] <= round(0.005 * A1.numel())
+    assert len(set(big[:, 1].tolist())) <= 8
+    A3, _ = make_layer_inputs("llama1.3b", 0, device="cpu", M=64)
+    assert A3.dtype == torch.bfloat16 and A3.shape == (64, 2048)
+    assert seed_for(WORKLOADS["llama7b"], 3) == 2003
