@@ -40,7 +40,7 @@ struct SelectResult {
     int found;
 };
 
-template <int PER>
+template <int PER, bool SMEM = false>
 __device__ SelectResult block_select(const uint32_t* __restrict__ hist, unsigned long long rank) {
     // 1024 threads; warp w owns bins [w * 32 * PER, (w + 1) * 32 * PER); lane l
     // holds bins w * 32 * PER + 32 i + l, i < PER, in registers (one round of
@@ -52,7 +52,7 @@ __device__ SelectResult block_select(const uint32_t* __restrict__ hist, unsigned
     const uint32_t* h = hist + (int64_t)warp * seg;
     uint32_t v[PER];
 #pragma unroll
-    for (int i = 0; i < PER; ++i) v[i] = __ldcg(h + 32 * i + lane);
+    for (int i = 0; i < PER; ++i) v[i] = SMEM ? h[32 * i + lane] : __ldcg(h + 32 * i + lane);
     unsigned long long mine = 0;
 #pragma unroll
     for (int i = 0; i < PER; ++i) mine += v[i];
@@ -184,6 +184,285 @@ hist_rowmax_kernel(const void* __restrict__ A, int64_t lda, int M, int K,
         const SelectResult r = block_select<kHist1Bins / 1024>(ghist, rank);
         if (DT == QG_BF16) finish_select<0>(r, ctr, status, T_out);
         else finish_select<1>(r, ctr, status, T_out);
+    }
+}
+
+// --------------------------------------------------------------------------
+// bf16 threshold by a band histogram.  A full 2^15-bin histogram costs one
+// shared-memory atomic per element; here only the elements whose key falls in
+// a narrow band around the order statistic take one, the rest are counted
+// with SWAR arithmetic on the packed bf16 pairs.  The band comes from a
+// sample of A; the result does not depend on it: when the order
+// statistic is not inside the band, an exact two-level count over all of A
+// takes its place (slow, but exact).
+//
+// SWAR compare of the two 15-bit keys of m = w & 0x7FFF7FFF with a constant
+// c in [0, 0x7FFF]: key + (0x8000 - c) sets bit 15 of its half iff key >= c,
+// and key + (0x7FFF - c) iff key > c; no sum leaves its 16-bit half.
+constexpr int kBandBins = 4096;            // band width in keys
+constexpr int kBandThreads = 1024;
+constexpr int kSampleBins = 4096;          // sample histogram of key >> 3
+constexpr int64_t kSampleTarget = 16384;   // sampled elements
+constexpr int kSampleRows = 64;            // from this many rows
+
+__device__ __forceinline__ uint32_t swar_ge(uint32_t m, uint32_t c) {
+    return (m + (0x8000u - c) * 0x10001u) & 0x80008000u;
+}
+__device__ __forceinline__ uint32_t swar_gt(uint32_t m, uint32_t c) {
+    return (m + (0x7FFFu - c) * 0x10001u) & 0x80008000u;
+}
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
+// Bins of a 4096-bin shared histogram holding the entries of ranks r[0..2]
+// (each r < total): thread t owns bins 4t..4t+3; one block scan.
+__device__ void block_select3(const uint32_t* sh, const unsigned long long (&r)[3],
+                              uint32_t* s_out /* 3 entries, shared */) {
+    __shared__ uint32_t s_w[32];
+    const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+    const uint4 v = reinterpret_cast<const uint4*>(sh)[t];
+    const uint32_t mine = v.x + v.y + v.z + v.w;
+    uint32_t incl = (uint32_t)warp_inclusive_scan((int)mine);
+    if (lane == 31) s_w[w] = incl;
+    __syncthreads();
+    uint32_t before = 0;
+    for (int i = 0; i < w; ++i) before += s_w[i];
+    uint32_t c = before + incl - mine;   // entries in bins < 4t
+    const uint32_t b[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+#pragma unroll
+        for (int k = 0; k < 3; ++k)
+            if (c <= r[k] && r[k] < (unsigned long long)c + b[q]) s_out[k] = 4 * t + q;
+        c += b[q];
+    }
+    __syncthreads();
+}
+
+// One CTA: zero the counters and band bins, histogram the keys >> 3 of a
+// sample (windows of 64 rows spread evenly over A), and put the band around
+// the sample quantile with a margin of six standard deviations of a sample
+// quantile's rank plus 32.
+__global__ void __launch_bounds__(kBandThreads, 1)
+band_prep_kernel(const uint16_t* __restrict__ A, int64_t lda, int M, int K,
+                 Counters* __restrict__ ctr, uint32_t* __restrict__ band_bins,
+                 unsigned long long rank) {
+    __shared__ __align__(16) uint32_t sh[kSampleBins];
+    __shared__ uint32_t s_sel[3];
+    const int t = threadIdx.x;
+    uint32_t* cz = reinterpret_cast<uint32_t*>(ctr);
+    for (int i = t; i < (int)(sizeof(Counters) / 4); i += blockDim.x) cz[i] = 0u;
+    for (int i = t; i < kBandBins; i += blockDim.x) band_bins[i] = 0u;
+    for (int i = t; i < kSampleBins; i += blockDim.x) sh[i] = 0u;
+    __syncthreads();
+    // R rows evenly spaced over M; from each a window of cpr 16-byte chunks
+    // whose start moves from row to row
+    const int nch = K / 8;
+    const int R = M < kSampleRows ? M : kSampleRows;
+    const int per_row = (int)((kSampleTarget / 8 + R - 1) / R);
+    const int cpr = nch < per_row ? nch : per_row;
+    const int64_t total = (int64_t)R * cpr;
+    for (int64_t q0 = t; q0 < total; q0 += 2 * (int64_t)blockDim.x) {
+        uint4 v[2];
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            const int64_t q = q0 + (int64_t)u * blockDim.x;
+            v[u] = make_uint4(0u, 0u, 0u, 0u);
+            if (q < total) {
+                const int64_t ri = q / cpr;
+                const int64_t off = (ri * 977) % (int64_t)(nch - cpr + 1);
+                const int c = (int)(off + (q - ri * cpr));
+                const int64_t row = ri * M / R;
+                v[u] = __ldg(reinterpret_cast<const uint4*>(A + row * lda) + c);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < 2; ++u) {
+            if (q0 + (int64_t)u * blockDim.x >= total) continue;
+            const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                atomicAdd(&sh[(w[i] & 0x7FFFu) >> 3], 1u);
+                atomicAdd(&sh[(w[i] >> 19) & 0xFFFu], 1u);
+            }
+        }
+    }
+    __syncthreads();
+    const double n = (double)M * (double)K;
+    const double ns = (double)total * 8.0;
+    const double p = ((double)rank + 0.5) / n;
+    const double center = p * ns;
+    const double margin = 6.0 * sqrt(ns * p * (1.0 - p)) + 32.0;
+    const double top = ns - 1.0;
+    const unsigned long long r[3] = {
+        (unsigned long long)fmin(fmax(floor(center - margin), 0.0), top),
+        (unsigned long long)fmin(fmax(ceil(center + margin), 0.0), top),
+        (unsigned long long)fmin(fmax(center, 0.0), top)};
+    if (t < 3) s_sel[t] = 0u;
+    __syncthreads();
+    block_select3(sh, r, s_sel);
+    if (t == 0) {
+        uint32_t lo = s_sel[0] << 3, hi = (s_sel[1] << 3) + 7u;
+        const uint32_t mid = s_sel[2] << 3;
+        if (hi - lo + 1 > (uint32_t)kBandBins) {
+            lo = max(lo, mid > (uint32_t)(kBandBins / 2) ? mid - kBandBins / 2 : 0u);
+            hi = min(hi, lo + kBandBins - 1);
+        }
+        ctr->band_lo = lo;
+        ctr->band_hi = hi;
+    }
+}
+
+// Exact selection of the key of rank `rank` over all of A by one CTA (the
+// band missed): a count of the 4096 buckets key >> 3, then of the 8 keys of
+// the chosen bucket.  sh holds kBandBins counters.
+__device__ SelectResult cta_exact_select(const uint16_t* __restrict__ A, int64_t lda, int M, int K,
+                                         uint32_t* sh, unsigned long long rank) {
+    const int nch = K / 8;
+    const int64_t total = (int64_t)M * nch;
+    SelectResult r1;
+    uint32_t bucket = 0;
+    for (int level = 0; level < 2; ++level) {
+        for (int i = threadIdx.x; i < kBandBins; i += blockDim.x) sh[i] = 0u;
+        __syncthreads();
+        for (int64_t q = threadIdx.x; q < total; q += blockDim.x) {
+            const int64_t row = q / nch;
+            const int c = (int)(q - row * nch);
+            const uint4 v = __ldcg(reinterpret_cast<const uint4*>(A + row * lda) + c);
+            const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const uint32_t key = (i & 1) ? ((w[i >> 1] >> 16) & 0x7FFFu) : (w[i >> 1] & 0x7FFFu);
+                if (level == 0) atomicAdd(&sh[key >> 3], 1u);
+                else if ((key >> 3) == bucket) atomicAdd(&sh[key & 7u], 1u);
+            }
+        }
+        __syncthreads();
+        if (level == 0) {
+            r1 = block_select<kBandBins / 1024, true>(sh, rank);
+            __syncthreads();
+            if (!r1.found) return r1;
+            bucket = r1.bin;
+        } else {
+            SelectResult r2 = block_select<kBandBins / 1024, true>(sh, rank - r1.below);
+            r2.bin = bucket * 8 + r2.bin;
+            r2.below += r1.below;
+            return r2;
+        }
+    }
+    return r1;
+}
+
+// Full pass over A: per-row max key, count of keys at or above the band's
+// low end, shared histogram of the keys inside the band.  The last CTA
+// selects the threshold from the band, or runs the exact fallback when the
+// band does not hold it.
+__global__ void __launch_bounds__(kBandThreads, 1)
+band_hist_rowmax_kernel(const uint16_t* __restrict__ A, int64_t lda, int M, int K,
+                        uint32_t* __restrict__ band_bins, uint32_t* __restrict__ rowmax,
+                        Counters* __restrict__ ctr, unsigned long long rank,
+                        uint32_t* __restrict__ status, float* __restrict__ T_out) {
+    __shared__ uint32_t sh[kBandBins];
+    __shared__ unsigned long long s_ge[kBandThreads / 32];
+    for (int i = threadIdx.x; i < kBandBins; i += blockDim.x) sh[i] = 0u;
+    __syncthreads();
+    const uint32_t lo = ctr->band_lo, hi = ctr->band_hi;
+    const int lane = threadIdx.x & 31;
+    const int wpc = blockDim.x >> 5;
+    const int total_warps = gridDim.x * wpc;
+    const int nchunks = K / 8;
+    const int steps_per_row = (nchunks + 127) / 128;
+    unsigned long long n_ge = 0;
+    uint32_t bad = 0;
+
+    int row = blockIdx.x * wpc + (threadIdx.x >> 5), step = 0;
+    uint4 nxt[4];
+    auto load_step = [&](int r, int st, uint4 (&dst)[4]) {
+        const uint16_t* base = A + (int64_t)r * lda;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int c = st * 128 + 32 * j + lane;
+            dst[j] = (c < nchunks) ? __ldg(reinterpret_cast<const uint4*>(base) + c)
+                                   : make_uint4(0u, 0u, 0u, 0u);
+        }
+    };
+    if (row < M) load_step(row, 0, nxt);
+    uint32_t mx = 0, cnt = 0, mx1 = 0, cnt1 = 0;
+    while (row < M) {
+        uint4 cur[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) cur[j] = nxt[j];
+        int nrow = row, nstep = step + 1;
+        if (nstep == steps_per_row) nrow = row + total_warps, nstep = 0;
+        if (nrow < M) load_step(nrow, nstep, nxt);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            if (step * 128 + 32 * j + lane >= nchunks) continue;   // past K
+            const uint32_t w[4] = {cur[j].x, cur[j].y, cur[j].z, cur[j].w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint32_t m = w[i] & 0x7FFF7FFFu;
+                // two accumulator chains each (shorter dependency chains)
+                if (i & 1) mx1 = max_u16x2(mx1, m);
+                else mx = max_u16x2(mx, m);
+                const uint32_t ge = swar_ge(m, lo);
+                if (i & 1) cnt1 += ge >> 15;
+                else cnt += ge >> 15;
+                const uint32_t in = ge & ~swar_gt(m, hi);
+                if (in) {
+                    if (in & 0x8000u) atomicAdd(&sh[(m & 0xFFFFu) - lo], 1u);
+                    if (in >> 16) atomicAdd(&sh[(m >> 16) - lo], 1u);
+                }
+            }
+        }
+        if (nstep == 0) {
+            // row done: its max key and its count of keys >= lo
+            mx = max_u16x2(mx, mx1);
+            cnt += cnt1;
+            const uint32_t km = warp_max_u32(max(mx & 0xFFFFu, mx >> 16));
+            if (lane == 0) rowmax[row] = km;
+            bad |= (km >= nonfinite_key<QG_BF16>()) ? 1u : 0u;
+            n_ge += (cnt & 0xFFFFu) + (cnt >> 16);
+            mx = mx1 = 0;
+            cnt = cnt1 = 0;
+        }
+        row = nrow;
+        step = nstep;
+    }
+#pragma unroll
+    for (int d = 16; d > 0; d >>= 1) n_ge += __shfl_xor_sync(0xFFFFFFFFu, n_ge, d);
+    if (lane == 0) s_ge[threadIdx.x >> 5] = n_ge;
+    if (bad && lane == 0) atomicOr(&ctr->nonfinite, 1u);
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        unsigned long long tot = 0;
+        for (int i = 0; i < wpc; ++i) tot += s_ge[i];
+        if (tot) atomicAdd(&ctr->band_below, tot);
+    }
+    for (int i = threadIdx.x; i < kBandBins; i += blockDim.x) {
+        const uint32_t v = sh[i];
+        if (v) atomicAdd(&band_bins[i], v);
+    }
+    if (last_block_done(&ctr->done_band)) {
+        // band_below holds the count of keys >= lo
+        const unsigned long long n = (unsigned long long)M * (unsigned long long)K;
+        const unsigned long long nbelow = n - __ldcg(&ctr->band_below);
+        SelectResult r;
+        r.found = 0;
+        if (rank >= nbelow) {
+            r = block_select<kBandBins / 1024>(band_bins, rank - nbelow);
+            r.bin += lo;
+            r.below += nbelow;
+        }
+        __syncthreads();
+        if (!r.found) {
+            if (threadIdx.x == 0) ctr->band_missed = 1u;
+            r = cta_exact_select(A, lda, M, K, sh, rank);
+        }
+        finish_select<0>(r, ctr, status, T_out);
     }
 }
 
@@ -371,6 +650,209 @@ clamp_quant_kernel(const void* __restrict__ A, int64_t lda, int M, int K,
     }
 }
 
+// --------------------------------------------------------------------------
+// The same pass for bf16 A with codes out, written for instruction count: the
+// bf16 pairs stay packed until they are scaled.  Per 32-bit word (two bf16):
+// the outlier test is a SWAR compare of the two magnitudes with T (one add,
+// one and), the clamp is a bit select (only in warps that hold an outlier),
+// the scale one packed fp32x2 multiply (IEEE round to nearest, as
+// __fmul_rn), the encode one cvt.  The next step's loads are issued before
+// this step's work.  Warps walk rows grid-stride; a step covers 1024 columns
+// of one row.
+constexpr int kQ3Threads = 256;
+#ifndef QG_CLAMP_MIN_BLOCKS
+#define QG_CLAMP_MIN_BLOCKS 3
+#endif
+constexpr int kQ3MinBlocks = QG_CLAMP_MIN_BLOCKS;   // resident CTAs per SM (register cap)
+
+// Scale a bf16 pair by r and encode it: one byte, element 0 in the low nibble.
+__device__ __forceinline__ uint32_t bf16x2_encode(uint32_t w, float r) {
+    const float lo = __uint_as_float(w << 16), hi = __uint_as_float(w & 0xFFFF0000u);
+    float a, b;
+    asm("{\n\t.reg .b64 p, q, t;\n\tmov.b64 p, {%2, %3};\n\tmov.b64 q, {%4, %4};\n\t"
+        "mul.rn.f32x2 t, p, q;\n\tmov.b64 {%0, %1}, t;\n\t}"
+        : "=f"(a), "=f"(b)
+        : "f"(lo), "f"(hi), "f"(r));
+    return e2m1x2(a, b);
+}
+
+__global__ void __launch_bounds__(kQ3Threads, kQ3MinBlocks)
+clamp_quant_bf16_kernel(const uint16_t* __restrict__ A, int64_t lda, int M, int K,
+                        const uint32_t* __restrict__ rowmax, Counters* __restrict__ ctr,
+                        uint8_t* __restrict__ codes, float* __restrict__ scales, ActBuffers b,
+                        int32_t* __restrict__ row_ptr, int64_t* __restrict__ nnz_out) {
+    // (an unselected threshold reads as the largest finite-or-not key)
+    const uint32_t Tk = min(ctr->T_key, 0x7FFFu);
+    const uint32_t tk2 = Tk | (Tk << 16);
+    const uint32_t cT = (0x7FFFu - Tk) * 0x10001u;   // SWAR: key > T sets bit 15
+    const float T = __uint_as_float(Tk << 16);
+    const int lane = threadIdx.x & 31;
+    const int wpc = blockDim.x >> 5;
+    const int total_warps = gridDim.x * wpc;
+    const int nchunks = K / 8;                       // 16-byte chunks per row
+    const int steps_per_row = (nchunks + 127) / 128;
+    const int row_slots = (int)b.row_slots;
+
+    int row = blockIdx.x * wpc + (threadIdx.x >> 5), step = 0;
+    uint4 nxt[4];
+    auto load_step = [&](int r, int st, uint4 (&dst)[4]) {
+        const uint16_t* base = A + (int64_t)r * lda;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int c = st * 128 + 32 * j + lane;
+            dst[j] = (c < nchunks) ? __ldg(reinterpret_cast<const uint4*>(base) + c)
+                                   : make_uint4(0u, 0u, 0u, 0u);
+        }
+    };
+    if (row < M) load_step(row, 0, nxt);
+
+    float r = 0.0f;
+    int row_rank = 0;
+    while (row < M) {
+        if (step == 0) {
+            const uint32_t rmax = rowmax[row];
+            float s;
+            scale_factors(__uint_as_float(min(rmax, Tk) << 16), r, s);
+            if (lane == 0) scales[row] = s;
+            row_rank = 0;
+        }
+        uint32_t w[4][4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            w[j][0] = nxt[j].x;
+            w[j][1] = nxt[j].y;
+            w[j][2] = nxt[j].z;
+            w[j][3] = nxt[j].w;
+        }
+        int nrow = row, nstep = step + 1;
+        if (nstep == steps_per_row) nrow = row + total_warps, nstep = 0;
+        if (nrow < M) load_step(nrow, nstep, nxt);
+
+        // outlier test: bit 15 / 31 of (|w| + cT) per word, OR-ed over the
+        // step; zero-filled columns past K never exceed T
+        uint32_t any = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+#pragma unroll
+            for (int i = 0; i < 4; ++i) any |= (w[j][i] & 0x7FFF7FFFu) + cT;
+        }
+        any &= 0x80008000u;
+        if (__any_sync(0xFFFFFFFFu, any != 0)) {
+            // this lane's outliers: element e of chunk j at bit 8 j + e
+            uint32_t ob = 0;
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint32_t gt = ((w[j][i] & 0x7FFF7FFFu) + cT) & 0x80008000u;
+                    ob |= (((gt >> 15) & 1u) | ((gt >> 30) & 2u)) << (8 * j + 2 * i);
+                }
+            }
+            // ranks in column order: chunks j-major, then lanes, then
+            // elements; the four per-lane counts are scanned as two pairs of
+            // 16-bit fields
+            const uint32_t c01 = __popc(ob & 0xFFu) | (__popc(ob & 0xFF00u) << 16);
+            const uint32_t c23 = __popc(ob & 0xFF0000u) | (__popc(ob & 0xFF000000u) << 16);
+            const uint32_t i01 = (uint32_t)warp_inclusive_scan((int)c01);
+            const uint32_t i23 = (uint32_t)warp_inclusive_scan((int)c23);
+            const uint32_t t01 = __shfl_sync(0xFFFFFFFFu, i01, 31);
+            const uint32_t t23 = __shfl_sync(0xFFFFFFFFu, i23, 31);
+            const uint32_t e01 = i01 - c01, e23 = i23 - c23;
+            // first rank of this lane's outliers in chunk j
+            const int b0 = row_rank + (int)(e01 & 0xFFFF);
+            const int b1 = row_rank + (int)(t01 & 0xFFFF) + (int)(e01 >> 16);
+            const int b2 = row_rank + (int)(t01 & 0xFFFF) + (int)(t01 >> 16) + (int)(e23 & 0xFFFF);
+            const int b3 = row_rank + (int)(t01 & 0xFFFF) + (int)(t01 >> 16) + (int)(t23 & 0xFFFF) +
+                           (int)(e23 >> 16);
+            const uint16_t* arow = A + (int64_t)row * lda;
+            for (uint32_t mm = ob; mm != 0; mm &= mm - 1) {
+                const int bit = __ffs(mm) - 1;
+                const int j = bit >> 3;
+                const int col = (step * 128 + 32 * j + lane) * 8 + (bit & 7);
+                const int idx = (j == 0 ? b0 : j == 1 ? b1 : j == 2 ? b2 : b3) +
+                                __popc(ob & ((1u << bit) - 1u) & (0xFFu << (8 * j)));
+                const float a = __uint_as_float((uint32_t)__ldg(arow + col) << 16);
+                const double d = (double)a - (double)copysignf(T, a);
+                if (idx < row_slots) {
+                    b.st_col[(int64_t)row * row_slots + idx] = col;
+                    b.st_val[(int64_t)row * row_slots + idx] = d;
+                } else {
+                    const unsigned long long o = atomicAdd(&ctr->nnz, 1ull);
+                    if (o < (unsigned long long)b.cap) {
+                        const int64_t slot = (int64_t)M * row_slots + (int64_t)o;
+                        b.st_row[o] = row;
+                        b.st_rank[o] = idx;
+                        b.st_col[slot] = col;
+                        b.st_val[slot] = d;
+                    } else {
+                        flag_status(b.status, kStatusOverflow);
+                    }
+                }
+            }
+            // flagged halves -> sign(x) * T
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+#pragma unroll
+                for (int i = 0; i < 4; ++i) {
+                    const uint32_t gt = ((w[j][i] & 0x7FFF7FFFu) + cT) & 0x80008000u;
+                    const uint32_t g = (gt >> 15) * 0xFFFFu;
+                    w[j][i] = (w[j][i] & ~g) | (g & ((w[j][i] & 0x80008000u) | tk2));
+                }
+            }
+            row_rank += (int)(t01 & 0xFFFF) + (int)(t01 >> 16) + (int)(t23 & 0xFFFF) + (int)(t23 >> 16);
+        }
+        uint32_t* out = reinterpret_cast<uint32_t*>(codes + (int64_t)row * (K / 2));
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int c = step * 128 + 32 * j + lane;
+            if (c < nchunks) {
+                const uint32_t q01 = __byte_perm(bf16x2_encode(w[j][0], r), bf16x2_encode(w[j][1], r), 0x0040);
+                const uint32_t q23 = __byte_perm(bf16x2_encode(w[j][2], r), bf16x2_encode(w[j][3], r), 0x0040);
+                out[c] = __byte_perm(q01, q23, 0x5410);
+            }
+        }
+        if (nstep == 0 && lane == 0) b.rowcnt[row] = (uint32_t)row_rank;
+        row = nrow;
+        step = nstep;
+    }
+
+    // last CTA: row_ptr = exclusive scan of the row counts
+    if (last_block_done(&ctr->done_clamp)) {
+        __shared__ unsigned long long s_warp[kQ3Threads / 32];
+        const int t = threadIdx.x, wi = t >> 5;
+        const int per = (M + kQ3Threads - 1) / kQ3Threads;
+        const int r0 = min(M, t * per), r1 = min(M, r0 + per);
+        unsigned long long mine = 0;
+#pragma unroll 8
+        for (int i = r0; i < r1; ++i) mine += __ldcg(b.rowcnt + i);
+        unsigned long long v = mine;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            unsigned long long u = __shfl_up_sync(0xFFFFFFFFu, v, d);
+            if (lane >= d) v += u;
+        }
+        if (lane == 31) s_warp[wi] = v;
+        __syncthreads();
+        unsigned long long before = 0, total = 0;
+        for (int i = 0; i < kQ3Threads / 32; ++i) {
+            if (i < wi) before += s_warp[i];
+            total += s_warp[i];
+        }
+        unsigned long long run = before + v - mine;
+#pragma unroll 8
+        for (int i = r0; i < r1; ++i) {
+            const uint32_t c = __ldcg(b.rowcnt + i);
+            row_ptr[i] = (int32_t)run;
+            run += c;
+        }
+        if (t == 0) {
+            row_ptr[M] = (int32_t)total;
+            *nnz_out = (int64_t)total;
+            if (total > (unsigned long long)b.cap) flag_status(b.status, kStatusOverflow);
+        }
+    }
+}
+
 // Move staged entries to their CSR positions: a warp per row for the row
 // regions, then a thread per overflow entry.
 __global__ void __launch_bounds__(256)
@@ -405,19 +887,24 @@ csr_scatter_kernel(const Counters* __restrict__ ctr, ActBuffers b, int M,
 static cudaError_t threshold_passes(const void* A, qg_dtype dt, int64_t M, int64_t K,
                                     int64_t lda, int64_t rank, const ActBuffers& b, float* T_out,
                                     cudaStream_t s) {
-    // counters and histograms are contiguous in the workspace
-    uint32_t* zbeg = reinterpret_cast<uint32_t*>(b.ctr);
-    uint32_t* zend = (dt == QG_F32 ? b.hist2 + kHist2Bins : b.hist1 + kHist1Bins);
-    launch_zero_u32(zbeg, zend - zbeg, s);
     const int nsm = num_sms();
     const int grid1 = (int)std::min<int64_t>(nsm, (M + 31) / 32);
     const size_t shmem = sizeof(uint32_t) * kHist1Bins;
     if (dt == QG_BF16) {
-        hist_rowmax_kernel<QG_BF16><<<grid1, kHistThreads, shmem, s>>>(
-            A, lda, (int)M, (int)K, b.hist1, b.rowmax, b.ctr, (unsigned long long)rank, b.status,
-            T_out);
-        count_launch(1);
+        // the band bins live at the start of hist1; the prep kernel zeroes
+        // them and the counters
+        const uint16_t* Ab = static_cast<const uint16_t*>(A);
+        band_prep_kernel<<<1, kBandThreads, shmem, s>>>(Ab, lda, (int)M, (int)K, b.ctr, b.hist1,
+                                                        (unsigned long long)rank);
+        band_hist_rowmax_kernel<<<grid1, kBandThreads, 0, s>>>(Ab, lda, (int)M, (int)K, b.hist1,
+                                                               b.rowmax, b.ctr,
+                                                               (unsigned long long)rank, b.status,
+                                                               T_out);
+        count_launch(2);
     } else {
+        // counters and histograms are contiguous in the workspace
+        uint32_t* zbeg = reinterpret_cast<uint32_t*>(b.ctr);
+        launch_zero_u32(zbeg, (b.hist2 + kHist2Bins) - zbeg, s);
         hist_rowmax_kernel<QG_F32><<<grid1, kHistThreads, shmem, s>>>(
             A, lda, (int)M, (int)K, b.hist1, b.rowmax, b.ctr, (unsigned long long)rank, b.status,
             T_out);
@@ -436,16 +923,26 @@ static void launch_clamp(const void* A, int64_t M, int64_t K, int64_t lda, const
                          uint8_t* codes, float* scales, void* A_c, const qg_csr* dA,
                          cudaStream_t s) {
     const int wpc = kQuantThreads / 32;
-    const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((M + wpc - 1) / wpc, (int64_t)num_sms() * 8));
-    clamp_quant_kernel<DT, CODES><<<grid, kQuantThreads, 0, s>>>(
-        A, lda, (int)M, (int)K, b.rowmax, b.ctr, codes, scales, A_c, b, dA->row_ptr, dA->nnz_out);
+    if (DT == QG_BF16 && CODES) {
+        const int g = (int)std::max<int64_t>(1, std::min<int64_t>((M + wpc - 1) / wpc, (int64_t)num_sms() * kQ3MinBlocks));
+        clamp_quant_bf16_kernel<<<g, kQ3Threads, 0, s>>>(static_cast<const uint16_t*>(A), lda, (int)M,
+                                                         (int)K, b.rowmax, b.ctr, codes, scales, b,
+                                                         dA->row_ptr, dA->nnz_out);
+    } else {
+        const int grid = (int)std::max<int64_t>(1, std::min<int64_t>((M + wpc - 1) / wpc, (int64_t)num_sms() * 8));
+        clamp_quant_kernel<DT, CODES><<<grid, kQuantThreads, 0, s>>>(
+            A, lda, (int)M, (int)K, b.rowmax, b.ctr, codes, scales, A_c, b, dA->row_ptr, dA->nnz_out);
+    }
     const int g2 = (int)std::max<int64_t>(1, std::min<int64_t>((M * 32 + 255) / 256, (int64_t)num_sms() * 8));
     csr_scatter_kernel<<<g2, 256, 0, s>>>(b.ctr, b, (int)M, dA->row_ptr, dA->col, dA->val);
     count_launch(2);
 }
 
 cudaError_t act_setup() {
-    cudaError_t e = cudaFuncSetAttribute(hist_rowmax_kernel<QG_BF16>,
+    cudaError_t e = cudaFuncSetAttribute(band_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)(sizeof(uint32_t) * kHist1Bins));
+    if (e != cudaSuccess) return e;
+    e = cudaFuncSetAttribute(hist_rowmax_kernel<QG_BF16>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)(sizeof(uint32_t) * kHist1Bins));
     if (e != cudaSuccess) return e;

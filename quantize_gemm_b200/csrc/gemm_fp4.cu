@@ -766,7 +766,18 @@ static bool encode_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base
 }
 
 // Output tile width: the candidate with the least padding of the last tile.
-static int pick_bn(int64_t N) {
+// Tile width: the persistent grid runs ceil(tiles / units) rounds of tiles
+// whose time grows with BN, so pick the width with the smaller rounds x BN;
+// on a tie, the one that pads N less.
+static int pick_bn(int64_t M, int64_t N, bool pair) {
+    const int64_t row_tiles = (M + (pair ? 255 : 127)) / (pair ? 256 : 128);
+    const int64_t units = std::max<int64_t>(1, num_sms() / (pair ? 2 : 1));
+    auto cost = [&](int64_t bn) {
+        const int64_t tiles = row_tiles * ((N + bn - 1) / bn);
+        return ((tiles + units - 1) / units) * bn;
+    };
+    const int64_t c224 = cost(224), c192 = cost(192);
+    if (c224 != c192) return c224 < c192 ? 224 : 192;
     const int64_t w224 = ((N + 223) / 224) * 224 - N;
     const int64_t w192 = ((N + 191) / 192) * 192 - N;
     return (w192 < w224) ? 192 : 224;
@@ -865,7 +876,7 @@ cudaError_t launch_fp4_gemm(const uint8_t* codesA, const float* sA, const uint8_
     }
     // the CTA pair when there are enough 256-row tiles to fill the SMs in pairs
     const bool pair = M > BM;
-    const int bn = QG_GEMM_FORCE_BN ? QG_GEMM_FORCE_BN : pick_bn(N);
+    const int bn = QG_GEMM_FORCE_BN ? QG_GEMM_FORCE_BN : pick_bn(p.M, N, pair);
     if (pair) {
         if (bn == 192) return launch_variant<192, true>(ta, codesWT, N, K, ty, tc, p, s);
         return launch_variant<224, true>(ta, codesWT, N, K, ty, tc, p, s);

@@ -35,6 +35,15 @@ struct Counters {
     uint32_t done_hist;            // CTAs finished with the histogram pass
     uint32_t done_refine;          // CTAs finished with the fp32 refine pass
     uint32_t done_clamp;           // CTAs finished with the clamp pass
+    // bf16 band pass: keys in [band_lo, band_hi] are histogrammed, the ones
+    // at or above band_lo counted (band_below holds that count, from which
+    // the number below the band follows); band_missed is set when the order
+    // statistic fell outside the band and an exact fallback ran
+    unsigned long long band_below;
+    uint32_t band_lo;
+    uint32_t band_hi;
+    uint32_t done_band;
+    uint32_t band_missed;
 };
 
 // Staging of dA: every row owns `row_slots` entries (its first entries in
@@ -118,17 +127,16 @@ __device__ __forceinline__ void flag_status(uint32_t* status, uint32_t bits) {
     atomicOr(status, bits);
 }
 
-// E2M1 encoding of two fp32 values with the hardware converter
-// (cvt.rn.satfinite.e2m1x2.f32: round to nearest even, saturate at 6), then
-// the sign bit of each input is copied in so that a negative input that
-// rounds to zero keeps its sign (code 0x8).  lo lands in bits 3..0.
+// Two fp32 values -> one byte of E2M1 codes by the hardware conversion
+// (cvt.rn.satfinite.e2m1x2.f32: round to nearest even, saturate at 6; a
+// negative input that rounds to zero keeps its sign, code 0x8, which a check
+// over every non-NaN fp32 pattern confirmed).  lo lands in bits 3..0.
 __device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
     uint16_t r;
     asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u16.u8 %0, t;\n\t}"
         : "=h"(r)
         : "f"(hi), "f"(lo));
-    uint32_t sgn = ((__float_as_uint(lo) >> 31) << 3) | ((__float_as_uint(hi) >> 31) << 7);
-    return ((uint32_t)r & 0xFFu) | sgn;
+    return (uint32_t)r & 0xFFu;
 }
 
 // Eight values -> four packed bytes (element 0 in the low nibble of byte 0).

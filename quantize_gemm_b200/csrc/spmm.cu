@@ -116,57 +116,42 @@ spmm_slice_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restrict
 
 // --------------------------------------------------------------------------
 // Fast path (bf16 W, N and ldw multiples of 8).  The kernel is bound by
-// instruction issue, so the work per non-zero is made as wide as possible:
-// a CTA owns a 1024-column slice (each lane 32 columns, in four 256-column
-// quarters so every load and store is coalesced), the bf16 pairs feed packed
-// fp32x2 FMAs (one rounding per product-sum, as fmaf), and W row segments are
-// prefetched with per-lane 16-byte cp.async copies into a per-lane ring of
-// kDepth slots in shared memory.  Every lane copies exactly the bytes it will
-// read, so no synchronisation between lanes is needed: after committing the
-// copy of entry j + kDepth - 1, waiting until at most kDepth - 1 groups are
-// pending makes entry j's bytes visible to the lane that copied them.
+// instruction issue, so the work per non-zero is made as wide and as lean as
+// possible: a CTA owns a 1024-column slice (each lane 32 columns, in four
+// 256-column quarters so every load and store is coalesced), W row segments
+// go straight from L2 into a register ring kDepth entries deep (the ring
+// position is a compile-time index: the entry loop is unrolled by kDepth),
+// and each bf16 pair feeds one packed fp32x2 FMA (one rounding per
+// product-sum, as fmaf) on accumulators kept as 64-bit register pairs.
 // A warp owns 4 consecutive rows, whose CSR entries form one contiguous
 // range consumed in order.
 constexpr int kStreamWarps = 8;
 constexpr int kStreamRowsPerWarp = 4;
-constexpr int kStreamParts = 4;                   // 256-column quarters per slice
+#ifndef QG_SPMM_PARTS
+#define QG_SPMM_PARTS 4
+#endif
+#ifndef QG_SPMM_DEPTH
+#define QG_SPMM_DEPTH 4
+#endif
+constexpr int kStreamParts = QG_SPMM_PARTS;       // 256-column quarters per slice
 constexpr int kStreamSlice = 256 * kStreamParts;
-constexpr int kDepth = 4;
-constexpr int kSlotBytes = kStreamParts * 512;    // 32 lanes x 16 bytes per quarter
-constexpr size_t kAsyncSmem = (size_t)kStreamWarps * kDepth * kSlotBytes;
+constexpr int kDepth = QG_SPMM_DEPTH;             // entries in flight per warp
 
-__device__ __forceinline__ void cp_async16(void* dst, const void* src) {
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(
-                     (uint32_t)__cvta_generic_to_shared(dst)),
-                 "l"(src)
-                 : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() {
-    asm volatile("cp.async.commit_group;" ::: "memory");
-}
-template <int N>
-__device__ __forceinline__ void cp_async_wait() {
-    asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
-}
-// acc0 += v * lo(w), acc1 += v * hi(w) for a bf16 pair w, as one packed FMA.
-__device__ __forceinline__ void fma_bf16x2(float& a0, float& a1, float v, uint32_t w) {
-    asm("{\n\t.reg .b32 lo, hi;\n\t.reg .b64 x, acc, vv;\n\t"
-        "shl.b32 lo, %3, 16;\n\tand.b32 hi, %3, 0xFFFF0000;\n\t"
-        "mov.b64 x, {lo, hi};\n\tmov.b64 acc, {%0, %1};\n\tmov.b64 vv, {%2, %2};\n\t"
-        "fma.rn.f32x2 acc, x, vv, acc;\n\tmov.b64 {%0, %1}, acc;\n\t}"
-        : "+f"(a0), "+f"(a1)
-        : "f"(v), "r"(w));
+// acc += vv * (lo(w), hi(w)) for a bf16 pair w; acc and vv hold fp32 pairs.
+__device__ __forceinline__ void fma_bf16x2(uint64_t& acc, uint64_t vv, uint32_t w) {
+    asm("{\n\t.reg .b32 lo, hi;\n\t.reg .b64 x;\n\t"
+        "shl.b32 lo, %2, 16;\n\tand.b32 hi, %2, 0xFFFF0000;\n\t"
+        "mov.b64 x, {lo, hi};\n\tfma.rn.f32x2 %0, x, %1, %0;\n\t}"
+        : "+l"(acc)
+        : "l"(vv), "r"(w));
 }
 
-__global__ void __launch_bounds__(kStreamWarps * 32)
+__global__ void __launch_bounds__(kStreamWarps * 32, 2)
 spmm_stream_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col,
                    const double* __restrict__ val, const uint16_t* __restrict__ W, int64_t ldw,
                    int M, int N, float* __restrict__ C) {
-    extern __shared__ __align__(128) uint8_t sm[];
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
-    // slot s of this lane: quarter h at ring + s * kSlotBytes + h * 512 (16 bytes)
-    uint8_t* ring = sm + (size_t)warp * kDepth * kSlotBytes + lane * 16;
     const int r_begin = (blockIdx.x * kStreamWarps + warp) * kStreamRowsPerWarp;
     if (r_begin >= M) return;
     const int r_end = min(M, r_begin + kStreamRowsPerWarp);
@@ -178,85 +163,80 @@ spmm_stream_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restric
     // row_ptr[r_begin .. r_end] held by lanes 0..4
     const int rp = (lane <= r_end - r_begin) ? row_ptr[r_begin + lane] : 0;
     const int P0 = __shfl_sync(0xFFFFFFFFu, rp, 0);
-    const int P1 = __shfl_sync(0xFFFFFFFFu, rp, r_end - r_begin);
+    const int n = __shfl_sync(0xFFFFFFFFu, rp, r_end - r_begin) - P0;
     // batches of 32 entries: current (kc, vc) and the next one's columns (kn)
-    int kc = (P0 + lane < P1) ? col[P0 + lane] : 0;
-    float vc = (P0 + lane < P1) ? (float)val[P0 + lane] : 0.0f;
-    int kn = (P0 + 32 + lane < P1) ? col[P0 + 32 + lane] : 0;
-    auto fetch = [&](int slot, int k) {
-        uint8_t* d = ring + slot * kSlotBytes;
-        const uint16_t* src = wl + (int64_t)k * ldw;
+    int kc = (lane < n) ? col[P0 + lane] : 0;
+    float vc = (lane < n) ? (float)val[P0 + lane] : 0.0f;
+    int kn = (32 + lane < n) ? col[P0 + 32 + lane] : 0;
+
+    uint4 buf[kDepth][kStreamParts];
+    auto fetch = [&](uint4 (&d)[kStreamParts], int k) {
+        const uint4* src = reinterpret_cast<const uint4*>(wl + (int64_t)k * ldw);
 #pragma unroll
         for (int h = 0; h < kStreamParts; ++h)
-            if (okh[h]) cp_async16(d + h * 512, src + 256 * h);
+            d[h] = okh[h] ? __ldg(src + 32 * h) : make_uint4(0u, 0u, 0u, 0u);
     };
 #pragma unroll
-    for (int t = 0; t < kDepth - 1; ++t) {
-        const int k = __shfl_sync(0xFFFFFFFFu, kc, t);
-        if (P0 + t < P1) fetch(t, k);
-        cp_async_commit();
-    }
-    float acc[8 * kStreamParts];
+    for (int u = 0; u < kDepth; ++u)
+        if (u < n) fetch(buf[u], __shfl_sync(0xFFFFFFFFu, kc, u));
+
+    uint64_t acc[4 * kStreamParts];
 #pragma unroll
-    for (int e = 0; e < 8 * kStreamParts; ++e) acc[e] = 0.0f;
+    for (int e = 0; e < 4 * kStreamParts; ++e) acc[e] = 0ull;
     int row = r_begin;
-    int rend = __shfl_sync(0xFFFFFFFFu, rp, 1);
+    int rend = __shfl_sync(0xFFFFFFFFu, rp, 1) - P0;   // entries of rows <= row end here
     auto store_row = [&](int r) {
         float* crow = C + (int64_t)r * N + nbase;
 #pragma unroll
         for (int h = 0; h < kStreamParts; ++h) {
             if (okh[h]) {
-                float4* d = reinterpret_cast<float4*>(crow + 256 * h);
-                d[0] = make_float4(acc[8 * h + 0], acc[8 * h + 1], acc[8 * h + 2], acc[8 * h + 3]);
-                d[1] = make_float4(acc[8 * h + 4], acc[8 * h + 5], acc[8 * h + 6], acc[8 * h + 7]);
+                ulonglong2* d = reinterpret_cast<ulonglong2*>(crow + 256 * h);
+                d[0] = make_ulonglong2(acc[4 * h + 0], acc[4 * h + 1]);
+                d[1] = make_ulonglong2(acc[4 * h + 2], acc[4 * h + 3]);
             }
         }
 #pragma unroll
-        for (int e = 0; e < 8 * kStreamParts; ++e) acc[e] = 0.0f;
+        for (int e = 0; e < 4 * kStreamParts; ++e) acc[e] = 0ull;
     };
-    for (int B = P0; B < P1; B += 32) {
-        const int cnt = min(32, P1 - B);
-        for (int t = 0; t < cnt; ++t) {
-            const int j = B + t;
-            // look-ahead copy of entry j + kDepth - 1
-            const int li = t + kDepth - 1;
-            const int ka = __shfl_sync(0xFFFFFFFFu, kc, li & 31);
-            const int kb = __shfl_sync(0xFFFFFFFFu, kn, li & 31);
-            if (j + kDepth - 1 < P1) fetch((j + kDepth - 1 - P0) % kDepth, li < 32 ? ka : kb);
-            cp_async_commit();
-            while (j >= rend) {          // rows that end before entry j
+    for (int q = 0; q < n; q += kDepth) {
+#pragma unroll
+        for (int u = 0; u < kDepth; ++u) {
+            const int j = q + u;                 // entry index within the warp's range
+            if (j >= n) break;
+            while (j >= rend) {                  // rows that end before entry j
                 store_row(row);
                 ++row;
-                rend = __shfl_sync(0xFFFFFFFFu, rp, row - r_begin + 1);
+                rend = __shfl_sync(0xFFFFFFFFu, rp, row - r_begin + 1) - P0;
             }
-            cp_async_wait<kDepth - 1>();
-            const uint8_t* src = ring + ((j - P0) % kDepth) * kSlotBytes;
-            const float v = __shfl_sync(0xFFFFFFFFu, vc, t);
+            const float v = __shfl_sync(0xFFFFFFFFu, vc, j & 31);
+            uint64_t vv;
+            asm("mov.b64 %0, {%1, %1};" : "=l"(vv) : "f"(v));
 #pragma unroll
             for (int h = 0; h < kStreamParts; ++h) {
-                const uint4 a = *reinterpret_cast<const uint4*>(src + h * 512);
-                fma_bf16x2(acc[8 * h + 0], acc[8 * h + 1], v, a.x);
-                fma_bf16x2(acc[8 * h + 2], acc[8 * h + 3], v, a.y);
-                fma_bf16x2(acc[8 * h + 4], acc[8 * h + 5], v, a.z);
-                fma_bf16x2(acc[8 * h + 6], acc[8 * h + 7], v, a.w);
+                fma_bf16x2(acc[4 * h + 0], vv, buf[u][h].x);
+                fma_bf16x2(acc[4 * h + 1], vv, buf[u][h].y);
+                fma_bf16x2(acc[4 * h + 2], vv, buf[u][h].z);
+                fma_bf16x2(acc[4 * h + 3], vv, buf[u][h].w);
+            }
+            // refill this ring position with entry j + kDepth
+            const int la = (j + kDepth) & 31;
+            const int ka = __shfl_sync(0xFFFFFFFFu, kc, la);
+            const int kb = __shfl_sync(0xFFFFFFFFu, kn, la);
+            if (j + kDepth < n) fetch(buf[u], ((j & 31) + kDepth < 32) ? ka : kb);
+            if ((j & 31) == 31) {                // advance the batches
+                kc = kn;
+                vc = (j + 1 + lane < n) ? (float)val[P0 + j + 1 + lane] : 0.0f;
+                kn = (j + 33 + lane < n) ? col[P0 + j + 33 + lane] : 0;
             }
         }
-        // advance the batches
-        kc = kn;
-        vc = (B + 32 + lane < P1) ? (float)val[B + 32 + lane] : 0.0f;
-        kn = (B + 64 + lane < P1) ? col[B + 64 + lane] : 0;
     }
-    cp_async_wait<0>();
     while (row < r_end) {                // the last rows (and empty ones)
         store_row(row);
         ++row;
     }
 }
 
-cudaError_t spmm_setup() {
-    return cudaFuncSetAttribute(spmm_stream_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)kAsyncSmem);
-}
+cudaError_t spmm_setup() { return cudaSuccess; }
 
 void launch_spmm(const qg_csr* dA, int64_t M, const void* W, qg_dtype dt, int64_t N, int64_t ldw,
                  float* C, uint32_t* status, cudaStream_t s) {
@@ -265,7 +245,7 @@ void launch_spmm(const qg_csr* dA, int64_t M, const void* W, qg_dtype dt, int64_
         const int rows_per_cta = kStreamWarps * kStreamRowsPerWarp;
         dim3 grid((unsigned)((M + rows_per_cta - 1) / rows_per_cta),
                   (unsigned)((N + kStreamSlice - 1) / kStreamSlice));
-        spmm_stream_kernel<<<grid, kStreamWarps * 32, kAsyncSmem, s>>>(
+        spmm_stream_kernel<<<grid, kStreamWarps * 32, 0, s>>>(
             dA->row_ptr, dA->col, dA->val, static_cast<const uint16_t*>(W), ldw, (int)M, (int)N, C);
         count_launch(1);
         return;

@@ -166,12 +166,26 @@ def _act_inputs(name):
     if name == "fp32_heavy_tail":
         return make_matrix((200, 640), ("student_t", 3), seed=9, device="cuda",
                            outliers=("random_entries", 0.002, 1e3)), 0.997
+    if name == "bf16_ragged_k1056":
+        return make_matrix((300, 1056), ("student_t", 4), seed=11, device="cuda",
+                           dtype=torch.bfloat16), 0.99
+    if name in ("band_miss_low", "band_miss_high"):
+        # M=512, K=256: the bf16 threshold pass samples whole rows 0, 8, 16, ...
+        # (all even).  Here the even rows are all zeros (or 1000x larger than
+        # the rest), so the sampled quantile is far from the true one and the
+        # exact fallback has to produce the threshold.
+        A = make_matrix((512, 256), ("student_t", 4), seed=12, device="cuda")
+        if name == "band_miss_low":
+            A[0::2] = 0.0
+        else:
+            A[0::2] *= 1000.0
+        return A.to(torch.bfloat16), 0.99
     raise KeyError(name)
 
 
 ACT_CASES = ["tiny", "llama1.3b_attn_m512", "llama7b_down_m256", "llama13b_qkv_m128",
              "ragged_k1056_fp32", "no_clamp", "clamp_almost_all", "ties_at_T", "single_row",
-             "fp32_heavy_tail"]
+             "fp32_heavy_tail", "bf16_ragged_k1056", "band_miss_low", "band_miss_high"]
 
 
 def _check_act(qg, A, alpha, codes, scales, csr, T, exp):
