@@ -136,20 +136,40 @@ constexpr int kStreamRowsPerWarp = 4;
 constexpr int kStreamParts = QG_SPMM_PARTS;       // 256-column quarters per slice
 constexpr int kStreamSlice = 256 * kStreamParts;
 constexpr int kDepth = QG_SPMM_DEPTH;             // entries in flight per warp
+static_assert(32 % kDepth == 0, "entry batches of 32 hold whole ring turns");
 
 // acc += vv * (lo(w), hi(w)) for a bf16 pair w; acc and vv hold fp32 pairs.
+// The low half can be moved up by a shift (which the compiler may place on
+// the FMA pipe) or by a byte permute (ALU pipe); ALU_LO picks the second, so
+// a caller can spread the unpacking over both pipes.
+template <bool ALU_LO>
 __device__ __forceinline__ void fma_bf16x2(uint64_t& acc, uint64_t vv, uint32_t w) {
-    asm("{\n\t.reg .b32 lo, hi;\n\t.reg .b64 x;\n\t"
-        "shl.b32 lo, %2, 16;\n\tand.b32 hi, %2, 0xFFFF0000;\n\t"
-        "mov.b64 x, {lo, hi};\n\tfma.rn.f32x2 %0, x, %1, %0;\n\t}"
-        : "+l"(acc)
-        : "l"(vv), "r"(w));
+    if (ALU_LO) {
+        asm("{\n\t.reg .b32 lo, hi;\n\t.reg .b64 x;\n\t"
+            "prmt.b32 lo, %2, 0, 0x1044;\n\tand.b32 hi, %2, 0xFFFF0000;\n\t"
+            "mov.b64 x, {lo, hi};\n\tfma.rn.f32x2 %0, x, %1, %0;\n\t}"
+            : "+l"(acc)
+            : "l"(vv), "r"(w));
+    } else {
+        asm("{\n\t.reg .b32 lo, hi;\n\t.reg .b64 x;\n\t"
+            "shl.b32 lo, %2, 16;\n\tand.b32 hi, %2, 0xFFFF0000;\n\t"
+            "mov.b64 x, {lo, hi};\n\tfma.rn.f32x2 %0, x, %1, %0;\n\t}"
+            : "+l"(acc)
+            : "l"(vv), "r"(w));
+    }
 }
+#ifndef QG_SPMM_ALU_WORDS
+#define QG_SPMM_ALU_WORDS 1     // words per 16-byte segment unpacked on the ALU (0..4)
+#endif
 
-__global__ void __launch_bounds__(kStreamWarps * 32, 2)
-spmm_stream_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col,
-                   const double* __restrict__ val, const uint16_t* __restrict__ W, int64_t ldw,
-                   int M, int N, float* __restrict__ C) {
+// FULL: every quarter of the slice is inside N (all slices but the last when
+// N is not a multiple of the slice width), so loads and stores need no checks.
+template <bool FULL>
+__device__ __forceinline__ void spmm_stream_body(const int32_t* __restrict__ row_ptr,
+                                                 const int32_t* __restrict__ col,
+                                                 const double* __restrict__ val,
+                                                 const uint16_t* __restrict__ W, int64_t ldw,
+                                                 int M, int N, float* __restrict__ C) {
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const int r_begin = (blockIdx.x * kStreamWarps + warp) * kStreamRowsPerWarp;
@@ -158,23 +178,33 @@ spmm_stream_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restric
     const int nbase = blockIdx.y * kStreamSlice + lane * 8;   // quarter h: nbase + 256 h
     bool okh[kStreamParts];
 #pragma unroll
-    for (int h = 0; h < kStreamParts; ++h) okh[h] = nbase + 256 * h < N;
+    for (int h = 0; h < kStreamParts; ++h) okh[h] = FULL || nbase + 256 * h < N;
     const uint16_t* wl = W + nbase;
     // row_ptr[r_begin .. r_end] held by lanes 0..4
     const int rp = (lane <= r_end - r_begin) ? row_ptr[r_begin + lane] : 0;
     const int P0 = __shfl_sync(0xFFFFFFFFu, rp, 0);
     const int n = __shfl_sync(0xFFFFFFFFu, rp, r_end - r_begin) - P0;
-    // batches of 32 entries: current (kc, vc) and the next one's columns (kn)
+    // per batch of 32 entries B .. B + 31: lane l holds the value of entry
+    // B + l (vc) and the column of entry B + kDepth + l (ks), the one whose
+    // W segment is fetched while entry B + l is consumed
     int kc = (lane < n) ? col[P0 + lane] : 0;
     float vc = (lane < n) ? (float)val[P0 + lane] : 0.0f;
-    int kn = (32 + lane < n) ? col[P0 + 32 + lane] : 0;
+    int ks;
+    {
+        const int kn = (32 + lane < n) ? col[P0 + 32 + lane] : 0;
+        const int a = __shfl_sync(0xFFFFFFFFu, kc, (lane + kDepth) & 31);
+        const int b = __shfl_sync(0xFFFFFFFFu, kn, (lane + kDepth) & 31);
+        ks = (lane + kDepth < 32) ? a : b;
+    }
 
     uint4 buf[kDepth][kStreamParts];
     auto fetch = [&](uint4 (&d)[kStreamParts], int k) {
         const uint4* src = reinterpret_cast<const uint4*>(wl + (int64_t)k * ldw);
 #pragma unroll
-        for (int h = 0; h < kStreamParts; ++h)
-            d[h] = okh[h] ? __ldg(src + 32 * h) : make_uint4(0u, 0u, 0u, 0u);
+        for (int h = 0; h < kStreamParts; ++h) {
+            if (FULL) d[h] = __ldg(src + 32 * h);
+            else d[h] = okh[h] ? __ldg(src + 32 * h) : make_uint4(0u, 0u, 0u, 0u);
+        }
     };
 #pragma unroll
     for (int u = 0; u < kDepth; ++u)
@@ -208,32 +238,45 @@ spmm_stream_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restric
                 ++row;
                 rend = __shfl_sync(0xFFFFFFFFu, rp, row - r_begin + 1) - P0;
             }
-            const float v = __shfl_sync(0xFFFFFFFFu, vc, j & 31);
+            const int t = (q & 31) + u;          // position in the batch
+            const float v = __shfl_sync(0xFFFFFFFFu, vc, t);
+            const int kf = __shfl_sync(0xFFFFFFFFu, ks, t);
             uint64_t vv;
             asm("mov.b64 %0, {%1, %1};" : "=l"(vv) : "f"(v));
 #pragma unroll
             for (int h = 0; h < kStreamParts; ++h) {
-                fma_bf16x2(acc[4 * h + 0], vv, buf[u][h].x);
-                fma_bf16x2(acc[4 * h + 1], vv, buf[u][h].y);
-                fma_bf16x2(acc[4 * h + 2], vv, buf[u][h].z);
-                fma_bf16x2(acc[4 * h + 3], vv, buf[u][h].w);
+                fma_bf16x2<(0 < QG_SPMM_ALU_WORDS)>(acc[4 * h + 0], vv, buf[u][h].x);
+                fma_bf16x2<(1 < QG_SPMM_ALU_WORDS)>(acc[4 * h + 1], vv, buf[u][h].y);
+                fma_bf16x2<(2 < QG_SPMM_ALU_WORDS)>(acc[4 * h + 2], vv, buf[u][h].z);
+                fma_bf16x2<(3 < QG_SPMM_ALU_WORDS)>(acc[4 * h + 3], vv, buf[u][h].w);
             }
             // refill this ring position with entry j + kDepth
-            const int la = (j + kDepth) & 31;
-            const int ka = __shfl_sync(0xFFFFFFFFu, kc, la);
-            const int kb = __shfl_sync(0xFFFFFFFFu, kn, la);
-            if (j + kDepth < n) fetch(buf[u], ((j & 31) + kDepth < 32) ? ka : kb);
-            if ((j & 31) == 31) {                // advance the batches
-                kc = kn;
-                vc = (j + 1 + lane < n) ? (float)val[P0 + j + 1 + lane] : 0.0f;
-                kn = (j + 33 + lane < n) ? col[P0 + j + 33 + lane] : 0;
-            }
+            if (j + kDepth < n) fetch(buf[u], kf);
+        }
+        if ((q & 31) == 32 - kDepth) {           // batch done: load the next one
+            const int B = q + kDepth;
+            kc = (B + lane < n) ? col[P0 + B + lane] : 0;
+            vc = (B + lane < n) ? (float)val[P0 + B + lane] : 0.0f;
+            const int kn = (B + 32 + lane < n) ? col[P0 + B + 32 + lane] : 0;
+            const int a = __shfl_sync(0xFFFFFFFFu, kc, (lane + kDepth) & 31);
+            const int b = __shfl_sync(0xFFFFFFFFu, kn, (lane + kDepth) & 31);
+            ks = (lane + kDepth < 32) ? a : b;
         }
     }
     while (row < r_end) {                // the last rows (and empty ones)
         store_row(row);
         ++row;
     }
+}
+
+__global__ void __launch_bounds__(kStreamWarps * 32, 2)
+spmm_stream_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col,
+                   const double* __restrict__ val, const uint16_t* __restrict__ W, int64_t ldw,
+                   int M, int N, float* __restrict__ C) {
+    if ((int)(blockIdx.y + 1) * kStreamSlice <= N)
+        spmm_stream_body<true>(row_ptr, col, val, W, ldw, M, N, C);
+    else
+        spmm_stream_body<false>(row_ptr, col, val, W, ldw, M, N, C);
 }
 
 cudaError_t spmm_setup() { return cudaSuccess; }
