@@ -683,7 +683,6 @@ clamp_quant_bf16_kernel(const uint16_t* __restrict__ A, int64_t lda, int M, int 
                         int32_t* __restrict__ row_ptr, int64_t* __restrict__ nnz_out) {
     // (an unselected threshold reads as the largest finite-or-not key)
     const uint32_t Tk = min(ctr->T_key, 0x7FFFu);
-    const uint32_t tk2 = Tk | (Tk << 16);
     const uint32_t cT = (0x7FFFu - Tk) * 0x10001u;   // SWAR: key > T sets bit 15
     const float T = __uint_as_float(Tk << 16);
     const int lane = threadIdx.x & 31;
@@ -728,25 +727,34 @@ clamp_quant_bf16_kernel(const uint16_t* __restrict__ A, int64_t lda, int M, int 
         if (nstep == steps_per_row) nrow = row + total_warps, nstep = 0;
         if (nrow < M) load_step(nrow, nstep, nxt);
 
-        // outlier test: bit 15 / 31 of (|w| + cT) per word, OR-ed over the
-        // step; zero-filled columns past K never exceed T
-        uint32_t any = 0;
+        // outlier test: the 16x2 max of |w| over the step, then bit 15 / 31
+        // of (max + cT); zero-filled columns past K never exceed T
+        uint32_t mx0 = 0, mx1 = 0;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) any |= (w[j][i] & 0x7FFF7FFFu) + cT;
+            for (int i = 0; i < 4; ++i) {
+                if (i & 1) mx1 = max_u16x2(mx1, w[j][i] & 0x7FFF7FFFu);
+                else mx0 = max_u16x2(mx0, w[j][i] & 0x7FFF7FFFu);
+            }
         }
-        any &= 0x80008000u;
+        const uint32_t any = (max_u16x2(mx0, mx1) + cT) & 0x80008000u;
         if (__any_sync(0xFFFFFFFFu, any != 0)) {
-            // this lane's outliers: element e of chunk j at bit 8 j + e
+            // this lane's outliers: element e of chunk j at bit 8 j + e.  The
+            // flags sit in bit 7 of bytes 1 and 3 of (|w| + cT); a byte
+            // permute gathers four of them into one word, and a multiply
+            // packs the four bit-7s into a nibble
             uint32_t ob = 0;
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
+                uint32_t g[4];
 #pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint32_t gt = ((w[j][i] & 0x7FFF7FFFu) + cT) & 0x80008000u;
-                    ob |= (((gt >> 15) & 1u) | ((gt >> 30) & 2u)) << (8 * j + 2 * i);
-                }
+                for (int i = 0; i < 4; ++i) g[i] = (w[j][i] & 0x7FFF7FFFu) + cT;
+                const uint32_t p01 = (__byte_perm(g[0], g[1], 0x7531) >> 7) & 0x01010101u;
+                const uint32_t p23 = (__byte_perm(g[2], g[3], 0x7531) >> 7) & 0x01010101u;
+                const uint32_t nib01 = (p01 * 0x01020408u) >> 24;
+                const uint32_t nib23 = (p23 * 0x01020408u) >> 24;
+                ob |= (nib01 | (nib23 << 4)) << (8 * j);
             }
             // ranks in column order: chunks j-major, then lanes, then
             // elements; the four per-lane counts are scanned as two pairs of
@@ -789,18 +797,12 @@ clamp_quant_bf16_kernel(const uint16_t* __restrict__ A, int64_t lda, int M, int 
                     }
                 }
             }
-            // flagged halves -> sign(x) * T
-#pragma unroll
-            for (int j = 0; j < 4; ++j) {
-#pragma unroll
-                for (int i = 0; i < 4; ++i) {
-                    const uint32_t gt = ((w[j][i] & 0x7FFF7FFFu) + cT) & 0x80008000u;
-                    const uint32_t g = (gt >> 15) * 0xFFFFu;
-                    w[j][i] = (w[j][i] & ~g) | (g & ((w[j][i] & 0x80008000u) | tk2));
-                }
-            }
             row_rank += (int)(t01 & 0xFFFF) + (int)(t01 >> 16) + (int)(t23 & 0xFFFF) + (int)(t23 >> 16);
         }
+        // codes of the clamped row: an outlier x (|x| > T, so amax = T) has
+        // |x r| >= |T r|, and T r is 6 within an ulp, so the saturating
+        // conversion of x r gives +-6 -- the code of sign(x) T r; hence the
+        // row is encoded without writing the clamp back into registers
         uint32_t* out = reinterpret_cast<uint32_t*>(codes + (int64_t)row * (K / 2));
 #pragma unroll
         for (int j = 0; j < 4; ++j) {

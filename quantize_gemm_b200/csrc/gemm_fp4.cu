@@ -765,7 +765,6 @@ static bool encode_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
-// Output tile width: the candidate with the least padding of the last tile.
 // Tile width: the persistent grid runs ceil(tiles / units) rounds of tiles
 // whose time grows with BN, so pick the width with the smaller rounds x BN;
 // on a tie, the one that pads N less.
