@@ -22,20 +22,21 @@
 //                 (rank 0) issues the MMAs; the TMA loads of both CTAs signal
 //                 the leader's barriers; the leader's MMA commits signal both
 //                 CTAs' barriers.  Loads use no multicast.
-// Warp roles (192 threads per CTA):
+// Warp roles (64 + 32 * kEpiWarps threads per CTA, kEpiWarps = 4 by default):
 //   warp 0     TMA producer: 128-byte-swizzled FP4 tiles (256 values deep)
 //              into a kStages-deep shared-memory ring
 //   warp 1     TMEM allocator; in the (leader) CTA one thread issues the MMAs,
 //              K = 64 each, into one of two TMEM accumulators so the next
 //              tile's MMAs run while the epilogue drains this one
-//   warps 2-5  epilogue, one TMEM lane quarter (32 rows) each, 32 columns at a
-//              time: tcgen05.ld, the C sub-tile arrives by TMA in swizzled
-//              shared memory, Y = acc * s_i * t_j + C goes back into the same
-//              buffer and leaves by a TMA store (kEpiBufs buffers per warp, C
-//              requested kEpiBufs - 1 chunks ahead, TMEM loads one chunk
-//              ahead).  A
-//              direct register-to-global path serves the raw-accumulator
-//              output and row pitches that TMA cannot describe.
+//   warps 2..  epilogue, one (or, with 8 warps, two) per TMEM lane quarter of
+//              32 rows, 32 columns at a time: tcgen05.ld, the C sub-tile
+//              arrives by TMA in swizzled shared memory, Y = acc * s_i * t_j
+//              + C goes back into the same buffer and leaves by a TMA store
+//              (kEpiBufs buffers per warp, C requested kEpiBufs - 1 chunks
+//              ahead, TMEM loads one chunk ahead, the next tile's scales
+//              loaded while this tile drains).  A separate instantiation
+//              (TMA_EPI = false) stores registers directly, for the raw-
+//              accumulator output and row pitches that TMA cannot describe.
 // TMEM: accumulators at columns [0, BN) and [BN, 2 BN), constant block
 // scales (every byte 0x7F = 2^0) at [448, 512).
 // Every mbarrier wait is bounded; a wait that gives up sets the timeout bit in
@@ -52,7 +53,12 @@ constexpr int BM = 128;             // rows of A per CTA
 constexpr int BK_BYTES = 128;       // 256 E2M1 values per row per k-block
 constexpr int UMMA_K_BYTES = 32;    // 64 E2M1 values per MMA
 constexpr int kAccStages = 2;
-constexpr int kEpiWarps = 4;
+#ifndef QG_GEMM_EPI_WARPS
+#define QG_GEMM_EPI_WARPS 4
+#endif
+constexpr int kEpiWarps = QG_GEMM_EPI_WARPS;     // 4 or 8 (one or two per TMEM lane quarter)
+constexpr int kEpiSplit = kEpiWarps / 4;         // chunk stride of one epilogue warp
+static_assert(kEpiWarps == 4 || kEpiWarps == 8, "one or two epilogue warps per lane quarter");
 constexpr int kThreads = 64 + 32 * kEpiWarps;
 constexpr int kTmemCols = 512;
 constexpr int kSfaCol = 448;
@@ -65,7 +71,7 @@ constexpr int kSfbCol = 480;
 #define QG_GEMM_SOLO_STAGES 3
 #endif
 #ifndef QG_GEMM_EPI_BUFS
-#define QG_GEMM_EPI_BUFS 3
+#define QG_GEMM_EPI_BUFS 4
 #endif
 #ifndef QG_GEMM_FORCE_BN
 #define QG_GEMM_FORCE_BN 0
@@ -86,7 +92,7 @@ struct Cfg {
     static constexpr size_t kOffB = (size_t)kStages * kStageABytes;
     static constexpr size_t kOffEpi = kOffB + (size_t)kStages * kStageBBytes;
     static constexpr size_t kOffSw = kOffEpi + (size_t)kEpiWarps * kEpiBufs * kEpiBuf;
-    static constexpr size_t kOffBar = kOffSw + (size_t)kEpiWarps * BN * 4;
+    static constexpr size_t kOffBar = kOffSw + (size_t)kEpiWarps * ((BN / 32 + kEpiSplit - 1) / kEpiSplit) * 32 * 4;
 };
 
 template <int S>
@@ -105,6 +111,8 @@ template <int BN, bool PAIR>
 constexpr size_t smem_bytes() {
     return 1024 + Cfg<BN, PAIR>::kOffBar + sizeof(Barriers<Cfg<BN, PAIR>::kStages>);
 }
+static_assert(smem_bytes<224, true>() <= 232448 && smem_bytes<224, false>() <= 232448,
+              "pipeline stages and epilogue buffers must fit in 227 KB of shared memory");
 
 // ------------------------------------------------------------------ PTX wraps
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
@@ -411,7 +419,10 @@ __device__ __forceinline__ void epi_direct(const Params& p, const uint32_t (&v)[
     }
 }
 
-template <int BN, bool PAIR>
+// TMA_EPI: Y (and C) go through the swizzled sub-tile buffers and TMA; the
+// other instantiation stores registers directly (raw accumulator output, or
+// row pitches TMA cannot describe), so neither path's registers burden the other.
+template <int BN, bool PAIR, bool TMA_EPI>
 __global__ void __launch_bounds__(kThreads, 1)
 fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 const __grid_constant__ CUtensorMap tmap_b,
@@ -562,22 +573,28 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         }
     } else {
         // ---------------------------------------------------------- epilogue
-        // This warp walks its 32-column chunks of all its tiles as one stream:
-        // chunk g uses sub-tile buffer g % kEpiBufs; with a correction C, the C
-        // sub-tile of chunk g + kEpiBufs - 1 is requested once chunk g is stored.
+        // Two warps per TMEM lane quarter when kEpiSplit == 2: warp ew takes
+        // the chunks c with c % kEpiSplit == ew / 4.  Each warp walks its
+        // chunks of all its tiles as one stream: chunk g uses sub-tile buffer
+        // g % kEpiBufs; with a correction C, the C sub-tile of chunk
+        // g + kEpiBufs - 1 is requested once chunk g is stored.  The next
+        // tile's row and column scales are loaded while this tile is drained.
         constexpr int NC = BN / 32;
+        constexpr int SWR = (NC + kEpiSplit - 1) / kEpiSplit;   // this warp's chunks per tile, at most
         const int ew = warp - 2;               // epilogue warp index (buffers)
         const int q = warp & 3;                // TMEM lane quarter
+        const int par = ew / 4;                // chunk residue class of this warp
+        const int my_nc = (NC - par + kEpiSplit - 1) / kEpiSplit;   // its chunks per tile
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
         uint8_t* bufs = sepi + (size_t)ew * kEpiBufs * kEpiBuf;
-        float* sw = reinterpret_cast<float*>(smem + CF::kOffSw) + ew * BN;
-        const bool use_c = p.tma_epi && p.C != nullptr;
+        float* sw = reinterpret_cast<float*>(smem + CF::kOffSw) + ew * SWR * 32;
+        const bool use_c = TMA_EPI && p.C != nullptr;
         const int my_tiles = unit < num_tiles ? (num_tiles - unit + n_units - 1) / n_units : 0;
-        const int total = my_tiles * NC;
+        const int total = my_tiles * my_nc;
         uint32_t cphase = 0;                   // bit b: parity of the next wait on cbar[ew][b]
         uint32_t cpend = 0;                    // bit b: a C load into buffer b not yet waited for
         auto c_load = [&](int g) {
-            const int ti = g / NC, c = g - ti * NC;
+            const int ti = g / my_nc, c = par + kEpiSplit * (g - ti * my_nc);
             const int tile = unit + ti * n_units;
             const int mb = tile % num_m, nbk = tile / num_m;
             const int b = g % kEpiBufs;
@@ -590,6 +607,22 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         };
         if (use_c)
             for (int g = 0; g < kEpiBufs - 1 && g < total; ++g) c_load(g);
+        // scales of tile ti into registers (consumed one tile later)
+        float swr[SWR];
+        float srow_next = 0.0f;
+        auto fetch_scales = [&](int ti) {
+            const int tile = unit + ti * n_units;
+            const int m_blk = tile % num_m, n_blk = tile / num_m;
+#pragma unroll
+            for (int k = 0; k < SWR; ++k) {
+                const int c = par + kEpiSplit * k;           // k-th chunk of this warp
+                const int n = n_blk * BN + c * 32 + lane;
+                swr[k] = (k < my_nc && n < p.N) ? __ldg(p.sW + n) : 0.0f;
+            }
+            const int r = m_blk * CF::kTileRows + (int)rank * BM + 32 * q + lane;
+            srow_next = r < p.M ? __ldg(p.sA + r) : 0.0f;
+        };
+        if (my_tiles > 0) fetch_scales(0);
         int as = 0;
         uint32_t acc_phase = 0;
         bool ok = true;
@@ -599,14 +632,13 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             const int m_blk = tile % num_m, n_blk = tile / num_m;
             const int row0 = m_blk * CF::kTileRows + (int)rank * BM + 32 * q;
             const int row = row0 + lane;
-            const float s_row = row < p.M ? __ldg(p.sA + row) : 0.0f;
             // this tile's column scales into the warp's shared-memory copy
+            __syncwarp();   // the previous tile's chunks have read sw
+#pragma unroll
+            for (int k = 0; k < SWR; ++k) sw[32 * k + lane] = swr[k];   // chunk h's scales at sw[32 h]
+            const float s_row = srow_next;
             __syncwarp();
-            for (int i = lane; i < BN; i += 32) {
-                const int n = n_blk * BN + i;
-                sw[i] = n < p.N ? __ldg(p.sW + n) : 0.0f;
-            }
-            __syncwarp();
+            if (ti + 1 < my_tiles) fetch_scales(ti + 1);
             if (!mbar_wait_warp(&B->acc_full[as], acc_phase, &B->abort, p.status)) {
                 ok = false;
                 break;
@@ -614,7 +646,8 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             tc_fence_after();
             const uint32_t tbase = tmem + lane_base + (uint32_t)(as * BN);
             auto release_acc = [&]() {
-                // accumulator fully read: the next tile's MMAs may reuse it
+                // this warp's chunks fully read: the next tile's MMAs may reuse
+                // the accumulator once every epilogue warp has arrived
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) {
@@ -622,17 +655,28 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     else mbar_arrive(&B->acc_empty[as]);
                 }
             };
-            // one 32-column chunk: Y = acc * s_i * t_j + C, staged and stored by TMA
-            auto chunk = [&](const uint32_t (&v)[32], int c) -> bool {
+            // one 32-column chunk: Y = acc * s_i * t_j (+ C), staged and stored by TMA
+            auto chunk = [&](uint32_t (&v)[32], int h) -> bool {
+                const int c = par + kEpiSplit * h;
                 const int col0 = n_blk * BN + c * 32;
-                if (!p.tma_epi) {
+                if constexpr (!TMA_EPI) {
                     if (row < p.M && col0 < p.N) epi_direct(p, v, row, col0, s_row);
                     return true;
                 }
-                const int g = ti * NC + c;
+                const int g = ti * my_nc + h;
                 const int b = g % kEpiBufs;
                 uint8_t* buf = bufs + b * kEpiBuf;
-                float cv[32];
+                // y overwrites the accumulator registers (as fp32 bit patterns)
+                const float4* tw = reinterpret_cast<const float4*>(sw + h * 32);
+#pragma unroll
+                for (int j = 0; j < 8; ++j) {
+                    const float4 t = tw[j];
+                    const float tt[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+                    for (int e = 0; e < 4; ++e)
+                        v[4 * j + e] = __float_as_uint(
+                            __fmul_rn(__fmul_rn(__uint_as_float(v[4 * j + e]), s_row), tt[e]));
+                }
                 if (use_c) {
                     if (!mbar_wait_warp(&B->cbar[ew][b], (cphase >> b) & 1u, &B->abort, p.status))
                         return false;
@@ -641,27 +685,14 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
 #pragma unroll
                     for (int j = 0; j < 8; ++j) {
                         const float4 t = *reinterpret_cast<const float4*>(buf + swz128(lane, j));
-                        cv[4 * j] = t.x;
-                        cv[4 * j + 1] = t.y;
-                        cv[4 * j + 2] = t.z;
-                        cv[4 * j + 3] = t.w;
+                        const float tt[4] = {t.x, t.y, t.z, t.w};
+#pragma unroll
+                        for (int e = 0; e < 4; ++e)
+                            v[4 * j + e] = __float_as_uint(__fadd_rn(__uint_as_float(v[4 * j + e]), tt[e]));
                     }
                 } else {
                     // buffer b was last read by the store of chunk g - kEpiBufs
                     if (lane == 0) bulk_wait_read<kEpiBufs - 1>();
-                    __syncwarp();
-#pragma unroll
-                    for (int j = 0; j < 32; ++j) cv[j] = 0.0f;
-                }
-                float y[32];
-                const float4* tw = reinterpret_cast<const float4*>(sw + c * 32);
-#pragma unroll
-                for (int j = 0; j < 8; ++j) {
-                    const float4 t = tw[j];
-                    y[4 * j + 0] = __fadd_rn(__fmul_rn(__fmul_rn(__uint_as_float(v[4 * j + 0]), s_row), t.x), cv[4 * j + 0]);
-                    y[4 * j + 1] = __fadd_rn(__fmul_rn(__fmul_rn(__uint_as_float(v[4 * j + 1]), s_row), t.y), cv[4 * j + 1]);
-                    y[4 * j + 2] = __fadd_rn(__fmul_rn(__fmul_rn(__uint_as_float(v[4 * j + 2]), s_row), t.z), cv[4 * j + 2]);
-                    y[4 * j + 3] = __fadd_rn(__fmul_rn(__fmul_rn(__uint_as_float(v[4 * j + 3]), s_row), t.w), cv[4 * j + 3]);
                 }
                 __syncwarp();   // every lane has read its C row before the buffer is overwritten
                 if (p.y_bf16) {
@@ -670,16 +701,17 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                         uint32_t w[4];
 #pragma unroll
                         for (int i = 0; i < 4; ++i) {
-                            __nv_bfloat162 h = __floats2bfloat162_rn(y[8 * j + 2 * i], y[8 * j + 2 * i + 1]);
-                            w[i] = *reinterpret_cast<uint32_t*>(&h);
+                            __nv_bfloat162 hh = __floats2bfloat162_rn(__uint_as_float(v[8 * j + 2 * i]),
+                                                                      __uint_as_float(v[8 * j + 2 * i + 1]));
+                            w[i] = *reinterpret_cast<uint32_t*>(&hh);
                         }
                         *reinterpret_cast<uint4*>(buf + swz64(lane, j)) = make_uint4(w[0], w[1], w[2], w[3]);
                     }
                 } else {
 #pragma unroll
                     for (int j = 0; j < 8; ++j)
-                        *reinterpret_cast<float4*>(buf + swz128(lane, j)) =
-                            make_float4(y[4 * j], y[4 * j + 1], y[4 * j + 2], y[4 * j + 3]);
+                        *reinterpret_cast<uint4*>(buf + swz128(lane, j)) =
+                            make_uint4(v[4 * j], v[4 * j + 1], v[4 * j + 2], v[4 * j + 3]);
                 }
                 fence_async_smem();
                 __syncwarp();
@@ -694,20 +726,21 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 }
                 return true;
             };
-            tmem_ld32_issue(tbase, va);
-            for (int c = 0; c < NC; c += 2) {
+            const uint32_t coff = (uint32_t)(par * 32), cstep = (uint32_t)(kEpiSplit * 32);
+            tmem_ld32_issue(tbase + coff, va);
+            for (int h = 0; h < my_nc; h += 2) {
                 tmem_ld_wait(va);
-                if (c + 1 < NC) tmem_ld32_issue(tbase + (uint32_t)((c + 1) * 32), vb);
+                if (h + 1 < my_nc) tmem_ld32_issue(tbase + coff + (uint32_t)(h + 1) * cstep, vb);
                 else release_acc();
-                if (!chunk(va, c)) {
+                if (!chunk(va, h)) {
                     ok = false;
                     break;
                 }
-                if (c + 1 < NC) {
+                if (h + 1 < my_nc) {
                     tmem_ld_wait(vb);
-                    if (c + 2 < NC) tmem_ld32_issue(tbase + (uint32_t)((c + 2) * 32), va);
+                    if (h + 2 < my_nc) tmem_ld32_issue(tbase + coff + (uint32_t)(h + 2) * cstep, va);
                     else release_acc();
-                    if (!chunk(vb, c + 1)) {
+                    if (!chunk(vb, h + 1)) {
                         ok = false;
                         break;
                     }
@@ -716,7 +749,7 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             if (++as == kAccStages) as = 0, acc_phase ^= 1u;
         }
         tmem_ld_wait_all();
-        if (p.tma_epi && lane == 0) {
+        if (TMA_EPI && lane == 0) {
             bulk_wait_all();
             // on abort, C loads still in flight land before the CTA exits
             for (int b = 0; b < kEpiBufs; ++b)
@@ -782,7 +815,7 @@ static int pick_bn(int64_t M, int64_t N, bool pair) {
     return (w192 < w224) ? 192 : 224;
 }
 
-template <int BN, bool PAIR>
+template <int BN, bool PAIR, bool TMA_EPI>
 static cudaError_t launch_variant(const CUtensorMap& ta, const uint8_t* codesWT, int64_t N,
                                   int64_t K, const CUtensorMap& ty, const CUtensorMap& tc,
                                   const Params& p, cudaStream_t s) {
@@ -806,14 +839,18 @@ static cudaError_t launch_variant(const CUtensorMap& ta, const uint8_t* codesWT,
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, fp4_gemm_kernel<BN, PAIR>, ta, tb, ty, tc, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, fp4_gemm_kernel<BN, PAIR, TMA_EPI>, ta, tb, ty, tc, p);
     count_launch(1);
     return e;
 }
 
 template <int BN, bool PAIR>
 static cudaError_t set_smem_attr() {
-    return cudaFuncSetAttribute(fp4_gemm_kernel<BN, PAIR>,
+    cudaError_t e = cudaFuncSetAttribute(fp4_gemm_kernel<BN, PAIR, true>,
+                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem_bytes<BN, PAIR>());
+    if (e != cudaSuccess) return e;
+    return cudaFuncSetAttribute(fp4_gemm_kernel<BN, PAIR, false>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)smem_bytes<BN, PAIR>());
 }
@@ -877,11 +914,19 @@ cudaError_t launch_fp4_gemm(const uint8_t* codesA, const float* sA, const uint8_
     const bool pair = M > BM;
     const int bn = QG_GEMM_FORCE_BN ? QG_GEMM_FORCE_BN : pick_bn(p.M, N, pair);
     if (pair) {
-        if (bn == 192) return launch_variant<192, true>(ta, codesWT, N, K, ty, tc, p, s);
-        return launch_variant<224, true>(ta, codesWT, N, K, ty, tc, p, s);
+        if (p.tma_epi) {
+            if (bn == 192) return launch_variant<192, true, true>(ta, codesWT, N, K, ty, tc, p, s);
+            return launch_variant<224, true, true>(ta, codesWT, N, K, ty, tc, p, s);
+        }
+        if (bn == 192) return launch_variant<192, true, false>(ta, codesWT, N, K, ty, tc, p, s);
+        return launch_variant<224, true, false>(ta, codesWT, N, K, ty, tc, p, s);
     }
-    if (bn == 192) return launch_variant<192, false>(ta, codesWT, N, K, ty, tc, p, s);
-    return launch_variant<224, false>(ta, codesWT, N, K, ty, tc, p, s);
+    if (p.tma_epi) {
+        if (bn == 192) return launch_variant<192, false, true>(ta, codesWT, N, K, ty, tc, p, s);
+        return launch_variant<224, false, true>(ta, codesWT, N, K, ty, tc, p, s);
+    }
+    if (bn == 192) return launch_variant<192, false, false>(ta, codesWT, N, K, ty, tc, p, s);
+    return launch_variant<224, false, false>(ta, codesWT, N, K, ty, tc, p, s);
 }
 
 }  // namespace qg
