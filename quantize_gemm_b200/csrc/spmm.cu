@@ -126,7 +126,10 @@ spmm_slice_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restrict
 // A warp owns 4 consecutive rows, whose CSR entries form one contiguous
 // range consumed in order.
 constexpr int kStreamWarps = 8;
-constexpr int kStreamRowsPerWarp = 4;
+#ifndef QG_SPMM_RPW
+#define QG_SPMM_RPW 4
+#endif
+constexpr int kStreamRowsPerWarp = QG_SPMM_RPW;   // consecutive rows owned by one warp
 #ifndef QG_SPMM_PARTS
 #define QG_SPMM_PARTS 4
 #endif
