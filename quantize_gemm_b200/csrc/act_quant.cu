@@ -32,20 +32,21 @@ constexpr int kQuantThreads = 256;
 
 // --------------------------------------------------------------------------
 // Selection of the bin that holds the entry of rank `rank` (0-based) in a
-// histogram of 1024 * PER bins, by one CTA of 1024 threads.  Reads go around
-// L1 (the bins were just written by atomics).
+// histogram of NT * PER bins, by one CTA of NT threads.  Reads go around L1
+// (the bins were just written by atomics, maybe by other SMs).
 struct SelectResult {
     uint32_t bin;
     unsigned long long below;   // entries in bins < bin
     int found;
 };
 
-template <int PER, bool SMEM = false>
+template <int PER, bool SMEM = false, int NT = 1024>
 __device__ SelectResult block_select(const uint32_t* __restrict__ hist, unsigned long long rank) {
-    // 1024 threads; warp w owns bins [w * 32 * PER, (w + 1) * 32 * PER); lane l
+    // NT threads; warp w owns bins [w * 32 * PER, (w + 1) * 32 * PER); lane l
     // holds bins w * 32 * PER + 32 i + l, i < PER, in registers (one round of
     // coalesced loads), so the walk inside the chosen segment reloads nothing.
-    __shared__ unsigned long long s_warp[32];
+    constexpr int NW = NT / 32;
+    __shared__ unsigned long long s_warp[NW];
     __shared__ SelectResult s_res;
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const int seg = 32 * PER;
@@ -62,7 +63,7 @@ __device__ SelectResult block_select(const uint32_t* __restrict__ hist, unsigned
     if (t == 0) s_res.found = 0;
     __syncthreads();
     unsigned long long before = 0, incl = 0;
-    for (int w = 0; w < 32; ++w) {
+    for (int w = 0; w < NW; ++w) {
         const unsigned long long c = s_warp[w];
         if (w < warp) before += c;
         if (w <= warp) incl += c;
@@ -111,11 +112,11 @@ __device__ void finish_select(const SelectResult& r, Counters* ctr, uint32_t* st
         ctr->sel_bin = r.bin;
         ctr->sel_below = r.below;
     } else {
-        const uint32_t key = (MODE == 0) ? r.bin : ((ctr->sel_bin << 16) | r.bin);
+        const uint32_t key = (MODE == 0) ? r.bin : ((__ldcg(&ctr->sel_bin) << 16) | r.bin);
         ctr->T_key = key;
         *T_out = (MODE == 0) ? __uint_as_float(key << 16) : __uint_as_float(key);
     }
-    if (MODE != 1 && ctr->nonfinite) flag_status(status, kStatusNonFinite);
+    if (MODE != 1 && __ldcg(&ctr->nonfinite)) flag_status(status, kStatusNonFinite);
 }
 
 // True in the CTA that finished last (after all CTAs' global writes).
@@ -218,70 +219,83 @@ __device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
 }
 
 // Bins of a 4096-bin shared histogram holding the entries of ranks r[0..2]
-// (each r < total): thread t owns bins 4t..4t+3; one block scan.
+// (each r < total), by NT threads: thread t owns 4096 / NT consecutive bins;
+// one block scan.
+template <int NT>
 __device__ void block_select3(const uint32_t* sh, const unsigned long long (&r)[3],
                               uint32_t* s_out /* 3 entries, shared */) {
-    __shared__ uint32_t s_w[32];
+    constexpr int B = kSampleBins / NT;
+    __shared__ uint32_t s_w[NT / 32];
     const int t = threadIdx.x, lane = t & 31, w = t >> 5;
-    const uint4 v = reinterpret_cast<const uint4*>(sh)[t];
-    const uint32_t mine = v.x + v.y + v.z + v.w;
-    uint32_t incl = (uint32_t)warp_inclusive_scan((int)mine);
+    uint32_t b[B];
+#pragma unroll
+    for (int i = 0; i < B / 4; ++i) {
+        const uint4 v = reinterpret_cast<const uint4*>(sh)[t * (B / 4) + i];
+        b[4 * i] = v.x;
+        b[4 * i + 1] = v.y;
+        b[4 * i + 2] = v.z;
+        b[4 * i + 3] = v.w;
+    }
+    uint32_t mine = 0;
+#pragma unroll
+    for (int i = 0; i < B; ++i) mine += b[i];
+    const uint32_t incl = (uint32_t)warp_inclusive_scan((int)mine);
     if (lane == 31) s_w[w] = incl;
     __syncthreads();
     uint32_t before = 0;
     for (int i = 0; i < w; ++i) before += s_w[i];
-    uint32_t c = before + incl - mine;   // entries in bins < 4t
-    const uint32_t b[4] = {v.x, v.y, v.z, v.w};
+    uint32_t c = before + incl - mine;   // entries in bins < B t
 #pragma unroll
-    for (int q = 0; q < 4; ++q) {
+    for (int q = 0; q < B; ++q) {
 #pragma unroll
         for (int k = 0; k < 3; ++k)
-            if (c <= r[k] && r[k] < (unsigned long long)c + b[q]) s_out[k] = 4 * t + q;
+            if (c <= r[k] && r[k] < (unsigned long long)c + b[q]) s_out[k] = B * t + q;
         c += b[q];
     }
     __syncthreads();
 }
 
-// One CTA: zero the counters and band bins, histogram the keys >> 3 of a
-// sample (windows of 64 rows spread evenly over A), and put the band around
-// the sample quantile with a margin of six standard deviations of a sample
-// quantile's rank plus 32.
-__global__ void __launch_bounds__(kBandThreads, 1)
-band_prep_kernel(const uint16_t* __restrict__ A, int64_t lda, int M, int K,
-                 Counters* __restrict__ ctr, uint32_t* __restrict__ band_bins,
-                 unsigned long long rank) {
-    __shared__ __align__(16) uint32_t sh[kSampleBins];
+// One CTA of NT threads: zero the counters and band bins, histogram the keys
+// >> 3 of a sample (windows of 64 rows spread evenly over A) in sh, and put
+// the band around the sample quantile with a margin of six standard
+// deviations of a sample quantile's rank plus 32.
+template <int NT>
+__device__ void cta_sample_band(const uint16_t* __restrict__ A, int64_t lda, int M, int K,
+                                Counters* __restrict__ ctr, uint32_t* __restrict__ band_bins,
+                                unsigned long long rank, uint32_t* sh) {
     __shared__ uint32_t s_sel[3];
     const int t = threadIdx.x;
     uint32_t* cz = reinterpret_cast<uint32_t*>(ctr);
-    for (int i = t; i < (int)(sizeof(Counters) / 4); i += blockDim.x) cz[i] = 0u;
-    for (int i = t; i < kBandBins; i += blockDim.x) band_bins[i] = 0u;
-    for (int i = t; i < kSampleBins; i += blockDim.x) sh[i] = 0u;
+    for (int i = t; i < (int)(sizeof(Counters) / 4); i += NT) cz[i] = 0u;
+    for (int i = t; i < kBandBins; i += NT) band_bins[i] = 0u;
+    for (int i = t; i < kSampleBins; i += NT) sh[i] = 0u;
     __syncthreads();
-    // R rows evenly spaced over M; from each a window of cpr 16-byte chunks
-    // whose start moves from row to row
+    // R rows evenly spaced over M (row ri * M / R); from each a window of cpr
+    // 16-byte chunks whose start moves from row to row
     const int nch = K / 8;
     const int R = M < kSampleRows ? M : kSampleRows;
     const int per_row = (int)((kSampleTarget / 8 + R - 1) / R);
     const int cpr = nch < per_row ? nch : per_row;
-    const int64_t total = (int64_t)R * cpr;
-    for (int64_t q0 = t; q0 < total; q0 += 2 * (int64_t)blockDim.x) {
-        uint4 v[2];
+    const int total = R * cpr;
+    const int mq = M / R, mr = M % R;
+    constexpr int U = (int)((kSampleTarget / 8 + NT - 1) / NT);   // loads per thread per round
+    for (int q0 = t; q0 < total; q0 += U * NT) {
+        uint4 v[U];
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            const int64_t q = q0 + (int64_t)u * blockDim.x;
+        for (int u = 0; u < U; ++u) {
+            const int q = q0 + u * NT;
             v[u] = make_uint4(0u, 0u, 0u, 0u);
             if (q < total) {
-                const int64_t ri = q / cpr;
-                const int64_t off = (ri * 977) % (int64_t)(nch - cpr + 1);
-                const int c = (int)(off + (q - ri * cpr));
-                const int64_t row = ri * M / R;
+                const int ri = q / cpr;
+                const int off = (ri * 977) % (nch - cpr + 1);
+                const int c = off + (q - ri * cpr);
+                const int64_t row = (int64_t)ri * mq + (ri * mr) / R;
                 v[u] = __ldg(reinterpret_cast<const uint4*>(A + row * lda) + c);
             }
         }
 #pragma unroll
-        for (int u = 0; u < 2; ++u) {
-            if (q0 + (int64_t)u * blockDim.x >= total) continue;
+        for (int u = 0; u < U; ++u) {
+            if (q0 + u * NT >= total) continue;
             const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
@@ -303,7 +317,7 @@ band_prep_kernel(const uint16_t* __restrict__ A, int64_t lda, int M, int K,
         (unsigned long long)fmin(fmax(center, 0.0), top)};
     if (t < 3) s_sel[t] = 0u;
     __syncthreads();
-    block_select3(sh, r, s_sel);
+    block_select3<NT>(sh, r, s_sel);
     if (t == 0) {
         uint32_t lo = s_sel[0] << 3, hi = (s_sel[1] << 3) + 7u;
         const uint32_t mid = s_sel[2] << 3;
@@ -316,9 +330,18 @@ band_prep_kernel(const uint16_t* __restrict__ A, int64_t lda, int M, int K,
     }
 }
 
-// Exact selection of the key of rank `rank` over all of A by one CTA (the
-// band missed): a count of the 4096 buckets key >> 3, then of the 8 keys of
-// the chosen bucket.  sh holds kBandBins counters.
+__global__ void __launch_bounds__(kBandThreads, 1)
+band_prep_kernel(const uint16_t* __restrict__ A, int64_t lda, int M, int K,
+                 Counters* __restrict__ ctr, uint32_t* __restrict__ band_bins,
+                 unsigned long long rank) {
+    __shared__ __align__(16) uint32_t sh[kSampleBins];
+    cta_sample_band<kBandThreads>(A, lda, M, K, ctr, band_bins, rank, sh);
+}
+
+// Exact selection of the key of rank `rank` over all of A by one CTA of NT
+// threads (the band missed): a count of the 4096 buckets key >> 3, then of
+// the 8 keys of the chosen bucket.  sh holds kBandBins counters.
+template <int NT>
 __device__ SelectResult cta_exact_select(const uint16_t* __restrict__ A, int64_t lda, int M, int K,
                                          uint32_t* sh, unsigned long long rank) {
     const int nch = K / 8;
@@ -326,9 +349,9 @@ __device__ SelectResult cta_exact_select(const uint16_t* __restrict__ A, int64_t
     SelectResult r1;
     uint32_t bucket = 0;
     for (int level = 0; level < 2; ++level) {
-        for (int i = threadIdx.x; i < kBandBins; i += blockDim.x) sh[i] = 0u;
+        for (int i = threadIdx.x; i < kBandBins; i += NT) sh[i] = 0u;
         __syncthreads();
-        for (int64_t q = threadIdx.x; q < total; q += blockDim.x) {
+        for (int64_t q = threadIdx.x; q < total; q += NT) {
             const int64_t row = q / nch;
             const int c = (int)(q - row * nch);
             const uint4 v = __ldcg(reinterpret_cast<const uint4*>(A + row * lda) + c);
@@ -342,12 +365,12 @@ __device__ SelectResult cta_exact_select(const uint16_t* __restrict__ A, int64_t
         }
         __syncthreads();
         if (level == 0) {
-            r1 = block_select<kBandBins / 1024, true>(sh, rank);
+            r1 = block_select<kBandBins / NT, true, NT>(sh, rank);
             __syncthreads();
             if (!r1.found) return r1;
             bucket = r1.bin;
         } else {
-            SelectResult r2 = block_select<kBandBins / 1024, true>(sh, rank - r1.below);
+            SelectResult r2 = block_select<kBandBins / NT, true, NT>(sh, rank - r1.below);
             r2.bin = bucket * 8 + r2.bin;
             r2.below += r1.below;
             return r2;
@@ -356,29 +379,17 @@ __device__ SelectResult cta_exact_select(const uint16_t* __restrict__ A, int64_t
     return r1;
 }
 
-// Full pass over A: per-row max key, count of keys at or above the band's
-// low end, shared histogram of the keys inside the band.  The last CTA
-// selects the threshold from the band, or runs the exact fallback when the
-// band does not hold it.
-__global__ void __launch_bounds__(kBandThreads, 1)
-band_hist_rowmax_kernel(const uint16_t* __restrict__ A, int64_t lda, int M, int K,
-                        uint32_t* __restrict__ band_bins, uint32_t* __restrict__ rowmax,
-                        Counters* __restrict__ ctr, unsigned long long rank,
-                        uint32_t* __restrict__ status, float* __restrict__ T_out) {
-    __shared__ uint32_t sh[kBandBins];
-    __shared__ unsigned long long s_ge[kBandThreads / 32];
-    for (int i = threadIdx.x; i < kBandBins; i += blockDim.x) sh[i] = 0u;
-    __syncthreads();
-    const uint32_t lo = ctr->band_lo, hi = ctr->band_hi;
+// The band pass over the rows of warp gwarp, gwarp + nwarps, ...: per-row max
+// key into rowmax, count of keys >= lo into n_ge, keys in [lo, hi] into the
+// shared histogram sh (at key - lo), non-finite keys into bad.
+__device__ __forceinline__ void band_rows(const uint16_t* __restrict__ A, int64_t lda, int M, int K,
+                                          uint32_t lo, uint32_t hi, uint32_t* sh,
+                                          uint32_t* __restrict__ rowmax, int gwarp, int nwarps,
+                                          unsigned long long& n_ge, uint32_t& bad) {
     const int lane = threadIdx.x & 31;
-    const int wpc = blockDim.x >> 5;
-    const int total_warps = gridDim.x * wpc;
     const int nchunks = K / 8;
     const int steps_per_row = (nchunks + 127) / 128;
-    unsigned long long n_ge = 0;
-    uint32_t bad = 0;
-
-    int row = blockIdx.x * wpc + (threadIdx.x >> 5), step = 0;
+    int row = gwarp, step = 0;
     uint4 nxt[4];
     auto load_step = [&](int r, int st, uint4 (&dst)[4]) {
         const uint16_t* base = A + (int64_t)r * lda;
@@ -396,7 +407,7 @@ band_hist_rowmax_kernel(const uint16_t* __restrict__ A, int64_t lda, int M, int 
 #pragma unroll
         for (int j = 0; j < 4; ++j) cur[j] = nxt[j];
         int nrow = row, nstep = step + 1;
-        if (nstep == steps_per_row) nrow = row + total_warps, nstep = 0;
+        if (nstep == steps_per_row) nrow = row + nwarps, nstep = 0;
         if (nrow < M) load_step(nrow, nstep, nxt);
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -432,6 +443,14 @@ band_hist_rowmax_kernel(const uint16_t* __restrict__ A, int64_t lda, int M, int 
         row = nrow;
         step = nstep;
     }
+}
+
+// A CTA's share of the band pass into the global counters and bins.
+template <int NT>
+__device__ void band_flush(const uint32_t* sh, uint32_t* __restrict__ band_bins,
+                           unsigned long long n_ge, uint32_t bad, Counters* __restrict__ ctr) {
+    __shared__ unsigned long long s_ge[NT / 32];
+    const int lane = threadIdx.x & 31;
 #pragma unroll
     for (int d = 16; d > 0; d >>= 1) n_ge += __shfl_xor_sync(0xFFFFFFFFu, n_ge, d);
     if (lane == 0) s_ge[threadIdx.x >> 5] = n_ge;
@@ -439,31 +458,107 @@ band_hist_rowmax_kernel(const uint16_t* __restrict__ A, int64_t lda, int M, int 
     __syncthreads();
     if (threadIdx.x == 0) {
         unsigned long long tot = 0;
-        for (int i = 0; i < wpc; ++i) tot += s_ge[i];
+        for (int i = 0; i < NT / 32; ++i) tot += s_ge[i];
         if (tot) atomicAdd(&ctr->band_below, tot);
     }
-    for (int i = threadIdx.x; i < kBandBins; i += blockDim.x) {
+    for (int i = threadIdx.x; i < kBandBins; i += NT) {
         const uint32_t v = sh[i];
         if (v) atomicAdd(&band_bins[i], v);
     }
-    if (last_block_done(&ctr->done_band)) {
-        // band_below holds the count of keys >= lo
-        const unsigned long long n = (unsigned long long)M * (unsigned long long)K;
-        const unsigned long long nbelow = n - __ldcg(&ctr->band_below);
-        SelectResult r;
-        r.found = 0;
-        if (rank >= nbelow) {
-            r = block_select<kBandBins / 1024>(band_bins, rank - nbelow);
-            r.bin += lo;
-            r.below += nbelow;
-        }
-        __syncthreads();
-        if (!r.found) {
-            if (threadIdx.x == 0) ctr->band_missed = 1u;
-            r = cta_exact_select(A, lda, M, K, sh, rank);
-        }
-        finish_select<0>(r, ctr, status, T_out);
+}
+
+// Selection over NB global bins (written by other SMs: read around L1) by NT
+// threads in one pass: thread t sums its NB / NT consecutive bins, one block
+// scan locates the thread that holds the rank, which walks its own bins.
+template <int NT, int NB>
+__device__ SelectResult block_select_seq(const uint32_t* __restrict__ hist, unsigned long long rank) {
+    constexpr int B = NB / NT;
+    static_assert(B % 4 == 0, "whole 16-byte groups per thread");
+    __shared__ unsigned long long s_w[NT / 32];
+    __shared__ SelectResult s_res;
+    const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+    uint32_t v[B];
+#pragma unroll
+    for (int i = 0; i < B / 4; ++i) {
+        const uint4 q = __ldcg(reinterpret_cast<const uint4*>(hist) + t * (B / 4) + i);
+        v[4 * i] = q.x;
+        v[4 * i + 1] = q.y;
+        v[4 * i + 2] = q.z;
+        v[4 * i + 3] = q.w;
     }
+    unsigned long long mine = 0;
+#pragma unroll
+    for (int i = 0; i < B; ++i) mine += v[i];
+    unsigned long long incl = mine;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const unsigned long long u = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+        if (lane >= d) incl += u;
+    }
+    if (lane == 31) s_w[w] = incl;
+    if (t == 0) s_res.found = 0;
+    __syncthreads();
+    unsigned long long c = incl - mine;
+    for (int i = 0; i < w; ++i) c += s_w[i];
+    if (c <= rank && rank < c + mine) {
+#pragma unroll
+        for (int i = 0; i < B; ++i) {
+            if (c <= rank && rank < c + v[i]) {
+                s_res.bin = (uint32_t)(B * t + i);
+                s_res.below = c;
+                s_res.found = 1;
+            }
+            c += v[i];
+        }
+    }
+    __syncthreads();
+    return s_res;
+}
+
+// After every CTA's flush: the threshold from the band, or from the exact
+// fallback when the band does not hold the order statistic (one CTA).
+template <int NT>
+__device__ void band_select(const uint16_t* __restrict__ A, int64_t lda, int M, int K,
+                            const uint32_t* band_bins, Counters* __restrict__ ctr,
+                            unsigned long long rank, uint32_t* __restrict__ status,
+                            float* __restrict__ T_out, uint32_t* sh) {
+    const uint32_t lo = __ldcg(&ctr->band_lo);
+    // band_below holds the count of keys >= lo
+    const unsigned long long n = (unsigned long long)M * (unsigned long long)K;
+    const unsigned long long nbelow = n - __ldcg(&ctr->band_below);
+    SelectResult r;
+    r.found = 0;
+    if (rank >= nbelow) {
+        r = block_select_seq<NT, kBandBins>(band_bins, rank - nbelow);
+        r.bin += lo;
+        r.below += nbelow;
+    }
+    __syncthreads();
+    if (!r.found) {
+        if (threadIdx.x == 0) ctr->band_missed = 1u;
+        r = cta_exact_select<NT>(A, lda, M, K, sh, rank);
+    }
+    finish_select<0>(r, ctr, status, T_out);
+}
+
+// Full pass over A (grid-stride rows); the last CTA selects the threshold.
+__global__ void __launch_bounds__(kBandThreads, 1)
+band_hist_rowmax_kernel(const uint16_t* __restrict__ A, int64_t lda, int M, int K,
+                        uint32_t* __restrict__ band_bins, uint32_t* __restrict__ rowmax,
+                        Counters* __restrict__ ctr, unsigned long long rank,
+                        uint32_t* __restrict__ status, float* __restrict__ T_out) {
+    __shared__ uint32_t sh[kBandBins];
+    for (int i = threadIdx.x; i < kBandBins; i += blockDim.x) sh[i] = 0u;
+    __syncthreads();
+    const uint32_t lo = __ldcg(&ctr->band_lo), hi = __ldcg(&ctr->band_hi);
+    const int wpc = kBandThreads / 32;
+    unsigned long long n_ge = 0;
+    uint32_t bad = 0;
+    band_rows(A, lda, M, K, lo, hi, sh, rowmax, blockIdx.x * wpc + (threadIdx.x >> 5),
+              gridDim.x * wpc, n_ge, bad);
+    band_flush<kBandThreads>(sh, band_bins, n_ge, bad, ctr);
+    if (last_block_done(&ctr->done_band))
+        band_select<kBandThreads>(A, lda, M, K, band_bins, ctr, rank, status, T_out, sh);
 }
 
 // fp32 only: histogram of the low 16 key bits of the entries whose high bits
@@ -676,23 +771,26 @@ __device__ __forceinline__ uint32_t bf16x2_encode(uint32_t w, float r) {
     return e2m1x2(a, b);
 }
 
-__global__ void __launch_bounds__(kQ3Threads, kQ3MinBlocks)
-clamp_quant_bf16_kernel(const uint16_t* __restrict__ A, int64_t lda, int M, int K,
-                        const uint32_t* __restrict__ rowmax, Counters* __restrict__ ctr,
-                        uint8_t* __restrict__ codes, float* __restrict__ scales, ActBuffers b,
-                        int32_t* __restrict__ row_ptr, int64_t* __restrict__ nnz_out) {
+// The clamp / quantize pass over rows first, first + stride, ... (< row_end)
+// of this warp; M is the matrix height (the overflow slots follow M row
+// regions).
+__device__ __forceinline__ void clamp_rows_bf16(const uint16_t* __restrict__ A, int64_t lda, int M,
+                                                int K, uint32_t T_key,
+                                                const uint32_t* __restrict__ rowmax,
+                                                Counters* __restrict__ ctr,
+                                                uint8_t* __restrict__ codes,
+                                                float* __restrict__ scales, const ActBuffers& b,
+                                                int first, int stride, int row_end) {
     // (an unselected threshold reads as the largest finite-or-not key)
-    const uint32_t Tk = min(ctr->T_key, 0x7FFFu);
+    const uint32_t Tk = min(T_key, 0x7FFFu);
     const uint32_t cT = (0x7FFFu - Tk) * 0x10001u;   // SWAR: key > T sets bit 15
     const float T = __uint_as_float(Tk << 16);
     const int lane = threadIdx.x & 31;
-    const int wpc = blockDim.x >> 5;
-    const int total_warps = gridDim.x * wpc;
     const int nchunks = K / 8;                       // 16-byte chunks per row
     const int steps_per_row = (nchunks + 127) / 128;
     const int row_slots = (int)b.row_slots;
 
-    int row = blockIdx.x * wpc + (threadIdx.x >> 5), step = 0;
+    int row = first, step = 0;
     uint4 nxt[4];
     auto load_step = [&](int r, int st, uint4 (&dst)[4]) {
         const uint16_t* base = A + (int64_t)r * lda;
@@ -703,13 +801,13 @@ clamp_quant_bf16_kernel(const uint16_t* __restrict__ A, int64_t lda, int M, int 
                                    : make_uint4(0u, 0u, 0u, 0u);
         }
     };
-    if (row < M) load_step(row, 0, nxt);
+    if (row < row_end) load_step(row, 0, nxt);
 
     float r = 0.0f;
     int row_rank = 0;
-    while (row < M) {
+    while (row < row_end) {
         if (step == 0) {
-            const uint32_t rmax = rowmax[row];
+            const uint32_t rmax = __ldcg(rowmax + row);
             float s;
             scale_factors(__uint_as_float(min(rmax, Tk) << 16), r, s);
             if (lane == 0) scales[row] = s;
@@ -724,8 +822,8 @@ clamp_quant_bf16_kernel(const uint16_t* __restrict__ A, int64_t lda, int M, int 
             w[j][3] = nxt[j].w;
         }
         int nrow = row, nstep = step + 1;
-        if (nstep == steps_per_row) nrow = row + total_warps, nstep = 0;
-        if (nrow < M) load_step(nrow, nstep, nxt);
+        if (nstep == steps_per_row) nrow = row + stride, nstep = 0;
+        if (nrow < row_end) load_step(nrow, nstep, nxt);
 
         // outlier test: the 16x2 max of |w| over the step, then bit 15 / 31
         // of (max + cT); zero-filled columns past K never exceed T
@@ -817,70 +915,311 @@ clamp_quant_bf16_kernel(const uint16_t* __restrict__ A, int64_t lda, int M, int 
         row = nrow;
         step = nstep;
     }
+}
 
-    // last CTA: row_ptr = exclusive scan of the row counts
-    if (last_block_done(&ctr->done_clamp)) {
-        __shared__ unsigned long long s_warp[kQ3Threads / 32];
-        const int t = threadIdx.x, wi = t >> 5;
-        const int per = (M + kQ3Threads - 1) / kQ3Threads;
-        const int r0 = min(M, t * per), r1 = min(M, r0 + per);
-        unsigned long long mine = 0;
+// row_ptr = exclusive scan of the row counts, by one CTA of NT threads.
+template <int NT>
+__device__ void cta_scan_rowcnt(const ActBuffers& b, int M, int32_t* __restrict__ row_ptr,
+                                int64_t* __restrict__ nnz_out) {
+    __shared__ unsigned long long s_warp[NT / 32];
+    const int t = threadIdx.x, wi = t >> 5, lane = t & 31;
+    const int per = (M + NT - 1) / NT;
+    const int r0 = min(M, t * per), r1 = min(M, r0 + per);
+    unsigned long long mine = 0;
 #pragma unroll 8
-        for (int i = r0; i < r1; ++i) mine += __ldcg(b.rowcnt + i);
-        unsigned long long v = mine;
+    for (int i = r0; i < r1; ++i) mine += __ldcg(b.rowcnt + i);
+    unsigned long long v = mine;
 #pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            unsigned long long u = __shfl_up_sync(0xFFFFFFFFu, v, d);
-            if (lane >= d) v += u;
-        }
-        if (lane == 31) s_warp[wi] = v;
-        __syncthreads();
-        unsigned long long before = 0, total = 0;
-        for (int i = 0; i < kQ3Threads / 32; ++i) {
-            if (i < wi) before += s_warp[i];
-            total += s_warp[i];
-        }
-        unsigned long long run = before + v - mine;
+    for (int d = 1; d < 32; d <<= 1) {
+        unsigned long long u = __shfl_up_sync(0xFFFFFFFFu, v, d);
+        if (lane >= d) v += u;
+    }
+    if (lane == 31) s_warp[wi] = v;
+    __syncthreads();
+    unsigned long long before = 0, total = 0;
+    for (int i = 0; i < NT / 32; ++i) {
+        if (i < wi) before += s_warp[i];
+        total += s_warp[i];
+    }
+    unsigned long long run = before + v - mine;
 #pragma unroll 8
-        for (int i = r0; i < r1; ++i) {
-            const uint32_t c = __ldcg(b.rowcnt + i);
-            row_ptr[i] = (int32_t)run;
-            run += c;
-        }
-        if (t == 0) {
-            row_ptr[M] = (int32_t)total;
-            *nnz_out = (int64_t)total;
-            if (total > (unsigned long long)b.cap) flag_status(b.status, kStatusOverflow);
-        }
+    for (int i = r0; i < r1; ++i) {
+        const uint32_t c = __ldcg(b.rowcnt + i);
+        row_ptr[i] = (int32_t)run;
+        run += c;
+    }
+    if (t == 0) {
+        row_ptr[M] = (int32_t)total;
+        *nnz_out = (int64_t)total;
+        if (total > (unsigned long long)b.cap) flag_status(b.status, kStatusOverflow);
     }
 }
 
-// Move staged entries to their CSR positions: a warp per row for the row
-// regions, then a thread per overflow entry.
+__global__ void __launch_bounds__(kQ3Threads, kQ3MinBlocks)
+clamp_quant_bf16_kernel(const uint16_t* __restrict__ A, int64_t lda, int M, int K,
+                        const uint32_t* __restrict__ rowmax, Counters* __restrict__ ctr,
+                        uint8_t* __restrict__ codes, float* __restrict__ scales, ActBuffers b,
+                        int32_t* __restrict__ row_ptr, int64_t* __restrict__ nnz_out) {
+    const int wpc = kQ3Threads / 32;
+    clamp_rows_bf16(A, lda, M, K, __ldcg(&ctr->T_key), rowmax, ctr, codes, scales, b,
+                    blockIdx.x * wpc + (threadIdx.x >> 5), gridDim.x * wpc, M);
+    if (last_block_done(&ctr->done_clamp)) cta_scan_rowcnt<kQ3Threads>(b, M, row_ptr, nnz_out);
+}
+
+// Move staged entries to their CSR positions: warp gwarp, gwarp + nwarps, ...
+// per row for the row regions, then thread gtid, gtid + nthreads, ... per
+// overflow entry.  Staged data is read around L1 (other SMs wrote it).
+__device__ __forceinline__ void scatter_entries(const Counters* __restrict__ ctr,
+                                                const ActBuffers& b, int M,
+                                                const int32_t* __restrict__ row_ptr,
+                                                int32_t* __restrict__ col,
+                                                double* __restrict__ val, int gwarp, int nwarps,
+                                                int64_t gtid, int64_t nthreads) {
+    const int lane = threadIdx.x & 31;
+    const int row_slots = (int)b.row_slots;
+    for (int r = gwarp; r < M; r += nwarps) {
+        const int n = min((int)__ldcg(b.rowcnt + r), row_slots);
+        const int64_t dst = __ldcg(row_ptr + r);
+        const int64_t src = (int64_t)r * row_slots;
+        for (int j = lane; j < n; j += 32) {
+            col[dst + j] = __ldcg(b.st_col + src + j);
+            val[dst + j] = __ldcg(b.st_val + src + j);
+        }
+    }
+    const unsigned long long n_over = min(__ldcg(&ctr->nnz), (unsigned long long)b.cap);
+    const int64_t base = (int64_t)M * row_slots;
+    for (unsigned long long e = (unsigned long long)gtid; e < n_over; e += (unsigned long long)nthreads) {
+        const int64_t dst = (int64_t)__ldcg(row_ptr + __ldcg(b.st_row + e)) + __ldcg(b.st_rank + e);
+        col[dst] = __ldcg(b.st_col + base + e);
+        val[dst] = __ldcg(b.st_val + base + e);
+    }
+}
+
 __global__ void __launch_bounds__(256)
 csr_scatter_kernel(const Counters* __restrict__ ctr, ActBuffers b, int M,
                    const int32_t* __restrict__ row_ptr, int32_t* __restrict__ col,
                    double* __restrict__ val) {
-    const int lane = threadIdx.x & 31;
-    const int gw = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-    const int nw = (gridDim.x * blockDim.x) >> 5;
-    const int row_slots = (int)b.row_slots;
-    for (int r = gw; r < M; r += nw) {
-        const int n = min((int)b.rowcnt[r], row_slots);
-        const int64_t dst = row_ptr[r];
-        const int64_t src = (int64_t)r * row_slots;
-        for (int j = lane; j < n; j += 32) {
-            col[dst + j] = b.st_col[src + j];
-            val[dst + j] = b.st_val[src + j];
-        }
+    scatter_entries(ctr, b, M, row_ptr, col, val, (blockIdx.x * blockDim.x + threadIdx.x) >> 5,
+                    (gridDim.x * blockDim.x) >> 5, blockIdx.x * (int64_t)blockDim.x + threadIdx.x,
+                    (int64_t)gridDim.x * blockDim.x);
+}
+
+// Exclusive scan of n counts (in[0..n)) into out[0..n) by one CTA of NT
+// threads; the total goes to *total.  Reads and writes this CTA's own data.
+template <int NT>
+__device__ void cta_local_scan(const uint32_t* in, int n, uint32_t* out, uint32_t* total) {
+    __shared__ uint32_t s_w[NT / 32];
+    const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+    const int per = (n + NT - 1) / NT;
+    const int a = min(n, t * per), e = min(n, a + per);
+    uint32_t mine = 0;
+    for (int i = a; i < e; ++i) mine += in[i];
+    const uint32_t incl = (uint32_t)warp_inclusive_scan((int)mine);
+    if (lane == 31) s_w[w] = incl;
+    __syncthreads();
+    uint32_t run = incl - mine, all = 0;
+    for (int i = 0; i < NT / 32; ++i) {
+        if (i < w) run += s_w[i];
+        all += s_w[i];
     }
-    const unsigned long long n_over = min(ctr->nnz, (unsigned long long)b.cap);
-    const int64_t base = (int64_t)M * row_slots;
-    for (unsigned long long e = blockIdx.x * (unsigned long long)blockDim.x + threadIdx.x;
-         e < n_over; e += (unsigned long long)gridDim.x * blockDim.x) {
-        const int64_t dst = (int64_t)row_ptr[b.st_row[e]] + b.st_rank[e];
-        col[dst] = b.st_col[base + e];
-        val[dst] = b.st_val[base + e];
+    for (int i = a; i < e; ++i) {
+        const uint32_t c = in[i];
+        out[i] = run;
+        run += c;
+    }
+    if (t == 0) *total = all;
+}
+
+// The last CTA: exclusive scan of the per-CTA totals in place (offsets), the
+// grand total into row_ptr[M] and nnz_out, and the capacity check.
+template <int NT>
+__device__ void cta_scan_offsets(uint32_t* cta_tot, int ncta, const ActBuffers& b, int M,
+                                 int32_t* __restrict__ row_ptr, int64_t* __restrict__ nnz_out) {
+    __shared__ unsigned long long s_w[NT / 32];
+    const int t = threadIdx.x, lane = t & 31, w = t >> 5;
+    const int per = (ncta + NT - 1) / NT;
+    const int a = min(ncta, t * per), e = min(ncta, a + per);
+    unsigned long long mine = 0;
+    for (int i = a; i < e; ++i) mine += __ldcg(cta_tot + i);
+    unsigned long long incl = mine;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const unsigned long long u = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+        if (lane >= d) incl += u;
+    }
+    if (lane == 31) s_w[w] = incl;
+    __syncthreads();
+    unsigned long long run = incl - mine, all = 0;
+    for (int i = 0; i < NT / 32; ++i) {
+        if (i < w) run += s_w[i];
+        all += s_w[i];
+    }
+    for (int i = a; i < e; ++i) {
+        const uint32_t c = __ldcg(cta_tot + i);
+        cta_tot[i] = (uint32_t)run;
+        run += c;
+    }
+    if (t == 0) {
+        row_ptr[M] = (int32_t)all;
+        *nnz_out = (int64_t)all;
+        if (all > (unsigned long long)b.cap) flag_status(b.status, kStatusOverflow);
+    }
+}
+
+// --------------------------------------------------------------------------
+// The whole bf16 quantize_act in one cooperative launch (all CTAs resident):
+//   phase 0  CTA 0 samples A and sets the band (the others wait)
+//   phase 1  band pass: row maxima, band histogram, count below the band
+//   phase 2  the last CTA to finish phase 1 selects T, then releases the rest
+//   phase 3  clamp / quantize / dA staging
+//   phase 4  the last CTA to finish phase 3 scans the row counts into row_ptr
+//   phase 5  CSR scatter
+// The grid barriers are a count and a generation word in the workspace
+// (count returns to 0 after every barrier).  Every wait is bounded: a CTA
+// that gives up sets the timeout bit and returns (the workspace barrier words
+// are then reset by qg_sync_status / qg_workspace_init).
+constexpr int kFusedThreads = 256;
+constexpr int kFusedMinBlocks = 3;
+constexpr int kCtaTotOffset = 8192;   // per-CTA totals in hist1 (after the band bins)
+constexpr int kFusedMaxGrid = 8192;
+constexpr long long kGridWaitLimit = 2000000000LL;   // SM clocks (~1-2 s)
+
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Arrive at a grid barrier.  Returns (in every thread) true in the CTA that
+// arrived last, which then runs its serial work and calls grid_release; the
+// others call grid_wait with gen0.
+__device__ __forceinline__ bool grid_arrive(GridSync* g, uint32_t& gen0) {
+    __shared__ int s_last;
+    __shared__ uint32_t s_gen;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        s_gen = ld_acquire_u32(&g->gen);
+        __threadfence();
+        const uint32_t old = atomicAdd(&g->count, 1u);
+        s_last = (old == gridDim.x - 1) ? 1 : 0;
+        if (s_last) __threadfence();
+    }
+    __syncthreads();
+    gen0 = s_gen;
+    return s_last != 0;
+}
+__device__ __forceinline__ void grid_release(GridSync* g) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        g->count = 0u;
+        __threadfence();
+        atomicAdd(&g->gen, 1u);
+    }
+}
+__device__ __forceinline__ bool grid_wait(GridSync* g, uint32_t gen0, uint32_t* status) {
+    __shared__ int s_ok;
+    if (threadIdx.x == 0) {
+        int ok = 1;
+        const long long t0 = clock64();
+        while (ld_acquire_u32(&g->gen) == gen0) {
+            if (clock64() - t0 > kGridWaitLimit) {
+                ok = 0;
+                flag_status(status, kStatusTimeout);
+                break;
+            }
+        }
+        __threadfence();
+        s_ok = ok;
+    }
+    __syncthreads();
+    return s_ok != 0;
+}
+
+__global__ void __launch_bounds__(kFusedThreads, kFusedMinBlocks)
+act_fused_bf16_kernel(const uint16_t* __restrict__ A, int64_t lda, int M, int K,
+                      unsigned long long rank, ActBuffers b, uint8_t* __restrict__ codes,
+                      float* __restrict__ scales, int32_t* __restrict__ row_ptr,
+                      int32_t* __restrict__ col, double* __restrict__ val,
+                      int64_t* __restrict__ nnz_out, float* __restrict__ T_out) {
+    __shared__ __align__(16) uint32_t sh[kBandBins];   // sample bins, band bins, fallback counts
+    constexpr int wpc = kFusedThreads / 32;
+    const int gwarp = blockIdx.x * wpc + (threadIdx.x >> 5), nwarps = gridDim.x * wpc;
+    GridSync* g = b.gsync;
+    uint32_t gen0;
+
+    // phase 0 (the other CTAs pull their first band row into L2 meanwhile)
+    if (blockIdx.x == 0) {
+        cta_sample_band<kFusedThreads>(A, lda, M, K, b.ctr, b.hist1, rank, sh);
+    } else if (gwarp < M) {
+        const char* rowp = reinterpret_cast<const char*>(A + (int64_t)gwarp * lda);
+        for (int c = threadIdx.x & 31; c < K * 2 / 128; c += 32)
+            asm volatile("prefetch.global.L2 [%0];" ::"l"(rowp + (int64_t)c * 128));
+    }
+    if (grid_arrive(g, gen0)) grid_release(g);
+    else if (!grid_wait(g, gen0, b.status)) return;
+
+    // phase 1
+    for (int i = threadIdx.x; i < kBandBins; i += kFusedThreads) sh[i] = 0u;
+    __syncthreads();
+    {
+        const uint32_t lo = __ldcg(&b.ctr->band_lo), hi = __ldcg(&b.ctr->band_hi);
+        unsigned long long n_ge = 0;
+        uint32_t bad = 0;
+        band_rows(A, lda, M, K, lo, hi, sh, b.rowmax, gwarp, nwarps, n_ge, bad);
+        band_flush<kFusedThreads>(sh, b.hist1, n_ge, bad, b.ctr);
+    }
+    // phase 2
+    if (grid_arrive(g, gen0)) {
+        band_select<kFusedThreads>(A, lda, M, K, b.hist1, b.ctr, rank, b.status, T_out, sh);
+        grid_release(g);
+    } else if (!grid_wait(g, gen0, b.status)) {
+        return;
+    }
+
+    // phase 3: CTA c clamps rows [r0, r1), a warp per row, then scans its
+    // rows' counts locally (the prefix overwrites rowmax, no longer needed)
+    const int rpc = (M + (int)gridDim.x - 1) / (int)gridDim.x;
+    const int r0 = min(M, (int)blockIdx.x * rpc), r1 = min(M, r0 + rpc);
+    clamp_rows_bf16(A, lda, M, K, __ldcg(&b.ctr->T_key), b.rowmax, b.ctr, codes, scales, b,
+                    r0 + (int)(threadIdx.x >> 5), wpc, r1);
+    uint32_t* cta_off = b.hist1 + kCtaTotOffset;   // per-CTA totals, then offsets
+    __syncthreads();
+    cta_local_scan<kFusedThreads>(b.rowcnt + r0, r1 - r0, b.rowmax + r0, cta_off + blockIdx.x);
+    // phase 4: the last CTA turns the CTA totals into offsets
+    if (grid_arrive(g, gen0)) {
+        cta_scan_offsets<kFusedThreads>(cta_off, (int)gridDim.x, b, M, row_ptr, nnz_out);
+        grid_release(g);
+    } else if (!grid_wait(g, gen0, b.status)) {
+        return;
+    }
+
+    // phase 5: row_ptr and the row regions of this CTA's rows, then a slice of
+    // the overflow list
+    const uint32_t off = __ldcg(cta_off + blockIdx.x);
+    for (int r = r0 + (int)threadIdx.x; r < r1; r += kFusedThreads)
+        row_ptr[r] = (int32_t)(b.rowmax[r] + off);
+    {
+        const int lane = threadIdx.x & 31;
+        const int row_slots = (int)b.row_slots;
+        for (int r = r0 + (int)(threadIdx.x >> 5); r < r1; r += wpc) {
+            const int n = min((int)b.rowcnt[r], row_slots);
+            const int64_t dst = (int64_t)b.rowmax[r] + off;
+            const int64_t src = (int64_t)r * row_slots;
+            for (int jj = lane; jj < n; jj += 32) {
+                col[dst + jj] = __ldcg(b.st_col + src + jj);
+                val[dst + jj] = __ldcg(b.st_val + src + jj);
+            }
+        }
+        const unsigned long long n_over = min(__ldcg(&b.ctr->nnz), (unsigned long long)b.cap);
+        const int64_t base = (int64_t)M * row_slots;
+        for (unsigned long long e = blockIdx.x * (unsigned long long)kFusedThreads + threadIdx.x;
+             e < n_over; e += (unsigned long long)gridDim.x * kFusedThreads) {
+            const int rr = __ldcg(b.st_row + e);
+            const int64_t dst = (int64_t)__ldcg(b.rowmax + rr) + __ldcg(cta_off + rr / rpc) +
+                                __ldcg(b.st_rank + e);
+            col[dst] = __ldcg(b.st_col + base + e);
+            val[dst] = __ldcg(b.st_val + base + e);
+        }
     }
 }
 
@@ -896,7 +1235,7 @@ static cudaError_t threshold_passes(const void* A, qg_dtype dt, int64_t M, int64
         // the band bins live at the start of hist1; the prep kernel zeroes
         // them and the counters
         const uint16_t* Ab = static_cast<const uint16_t*>(A);
-        band_prep_kernel<<<1, kBandThreads, shmem, s>>>(Ab, lda, (int)M, (int)K, b.ctr, b.hist1,
+        band_prep_kernel<<<1, kBandThreads, 0, s>>>(Ab, lda, (int)M, (int)K, b.ctr, b.hist1,
                                                         (unsigned long long)rank);
         band_hist_rowmax_kernel<<<grid1, kBandThreads, 0, s>>>(Ab, lda, (int)M, (int)K, b.hist1,
                                                                b.rowmax, b.ctr,
@@ -940,10 +1279,20 @@ static void launch_clamp(const void* A, int64_t M, int64_t K, int64_t lda, const
     count_launch(2);
 }
 
+// Resident CTAs per SM of the cooperative kernel, per device (0: not usable).
+static int g_fused_blocks[64];
+
 cudaError_t act_setup() {
-    cudaError_t e = cudaFuncSetAttribute(band_prep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)(sizeof(uint32_t) * kHist1Bins));
+    int dev = 0, coop = 0, nb = 0;
+    cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev);
+    if (e != cudaSuccess) return e;
+    if (coop) {
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, act_fused_bf16_kernel, kFusedThreads, 0);
+        if (e != cudaSuccess) return e;
+    }
+    if (dev >= 0 && dev < 64) g_fused_blocks[dev] = coop ? nb : 0;
     e = cudaFuncSetAttribute(hist_rowmax_kernel<QG_BF16>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)(sizeof(uint32_t) * kHist1Bins));
@@ -953,9 +1302,44 @@ cudaError_t act_setup() {
                                 (int)(sizeof(uint32_t) * kHist1Bins));
 }
 
+// The bf16 path as one cooperative launch; false when it cannot be used here.
+static bool launch_act_fused(const void* A, int64_t M, int64_t K, int64_t lda, int64_t rank,
+                             const ActBuffers& b, uint8_t* codes, float* scales, const qg_csr* dA,
+                             float* T_out, cudaStream_t s) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    const int nb = g_fused_blocks[dev];
+    if (nb < 1) return false;
+    const int64_t want = (M + kFusedThreads / 32 - 1) / (kFusedThreads / 32);   // a warp per row
+    const int grid = (int)std::max<int64_t>(
+        1, std::min<int64_t>({want, (int64_t)nb * num_sms(), (int64_t)kFusedMaxGrid}));
+    const uint16_t* Ab = static_cast<const uint16_t*>(A);
+    int Mi = (int)M, Ki = (int)K;
+    unsigned long long rk = (unsigned long long)rank;
+    ActBuffers bb = b;
+    int32_t* row_ptr = dA->row_ptr;
+    int32_t* col = dA->col;
+    double* val = dA->val;
+    int64_t* nnz_out = dA->nnz_out;
+    void* args[] = {(void*)&Ab, (void*)&lda, (void*)&Mi, (void*)&Ki, (void*)&rk, (void*)&bb,
+                    (void*)&codes, (void*)&scales, (void*)&row_ptr, (void*)&col, (void*)&val,
+                    (void*)&nnz_out, (void*)&T_out};
+    const cudaError_t e = cudaLaunchCooperativeKernel((const void*)act_fused_bf16_kernel,
+                                                      dim3((unsigned)grid), dim3(kFusedThreads),
+                                                      args, 0, s);
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();   // not sticky: fall back to the multi-kernel sequence
+        return false;
+    }
+    count_launch(1);
+    return true;
+}
+
 cudaError_t run_quantize_act(const void* A, qg_dtype dt, int64_t M, int64_t K, int64_t lda,
                              int64_t rank, const ActBuffers& b, uint8_t* codes, float* scales,
                              const qg_csr* dA, float* T_out, cudaStream_t s) {
+    if (dt == QG_BF16 && launch_act_fused(A, M, K, lda, rank, b, codes, scales, dA, T_out, s))
+        return cudaSuccess;
     cudaError_t e = threshold_passes(A, dt, M, K, lda, rank, b, T_out, s);
     if (e != cudaSuccess) return e;
     if (dt == QG_BF16) launch_clamp<QG_BF16, true>(A, M, K, lda, b, codes, scales, nullptr, dA, s);

@@ -85,6 +85,7 @@ static T* at(void* ws, size_t off) {
 static ActBuffers act_buffers(void* ws, const WsLayout& L) {
     ActBuffers b;
     b.status = at<uint32_t>(ws, L.status);
+    b.gsync = at<GridSync>(ws, L.gsync);
     b.ctr = at<Counters>(ws, L.counters);
     b.hist1 = at<uint32_t>(ws, L.hist1);
     b.hist2 = L.hist2 ? at<uint32_t>(ws, L.hist2) : nullptr;
@@ -170,6 +171,11 @@ qg_status qg_sync_status(void* ws, cudaStream_t stream) {
     if (cudaMemcpy(&st, ws, sizeof(st), cudaMemcpyDeviceToHost) != cudaSuccess) return QG_ERR_CUDA;
     if (st == 0) return QG_OK;
     if (cudaMemset(ws, 0, sizeof(uint32_t)) != cudaSuccess) return QG_ERR_CUDA;
+    if (st & kStatusTimeout) {
+        // a wait that gave up may have left a grid barrier half-counted
+        if (cudaMemset(static_cast<uint8_t*>(ws) + kGridSyncOffset, 0, sizeof(GridSync)) != cudaSuccess)
+            return QG_ERR_CUDA;
+    }
     if (st & kStatusNonFinite) return QG_ERR_NONFINITE;
     if (st & kStatusTimeout) return QG_ERR_TIMEOUT;
     return QG_ERR_INTERNAL;

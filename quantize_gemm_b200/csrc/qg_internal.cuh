@@ -62,7 +62,16 @@ constexpr int kHist2Bins = 1 << 16;   // fp32 refine: low 16 bits of |x|
 
 inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
+// Grid barrier of the cooperative activation kernel (inside the status block,
+// so qg_workspace_init zeroes it; the count is back to 0 after every barrier).
+struct GridSync {
+    uint32_t count;
+    uint32_t gen;
+};
+constexpr size_t kGridSyncOffset = 16;   // bytes from the workspace base
+
 struct WsLayout {
+    size_t gsync = 0;
     size_t status = 0, counters = 0, hist1 = 0, hist2 = 0, rowmax = 0, rowcnt = 0;
     size_t st_row = 0, st_rank = 0, st_col = 0, st_val = 0, colmax = 0;
     size_t act_codes = 0, act_scales = 0, csr_row_ptr = 0, csr_col = 0, csr_val = 0,
@@ -82,7 +91,8 @@ inline WsLayout ws_layout(qg_op op, int64_t M, int64_t K, int64_t N, qg_dtype dt
         off = align_up(off + (bytes ? bytes : 1));
         return at;
     };
-    L.status = take(16);
+    L.status = take(32);   // status word at +0, GridSync at +16
+    L.gsync = L.status + kGridSyncOffset;
     L.counters = take(sizeof(Counters));
     bool act = (op == QG_OP_CLAMP_COMPENSATE || op == QG_OP_QUANTIZE_ACT ||
                 op == QG_OP_FP4_LINEAR);
@@ -225,6 +235,7 @@ __device__ __forceinline__ uint32_t warp_max_u32(uint32_t v) {
 // Pointers into a workspace for the threshold / clamp passes.
 struct ActBuffers {
     uint32_t* status;
+    GridSync* gsync;
     Counters* ctr;
     uint32_t* hist1;
     uint32_t* hist2;
