@@ -1089,20 +1089,26 @@ __device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
     asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
     return v;
 }
+__device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
 
 // Arrive at a grid barrier.  Returns (in every thread) true in the CTA that
 // arrived last, which then runs its serial work and calls grid_release; the
-// others call grid_wait with gen0.
+// others call grid_wait with gen0.  The arrival is an acq_rel atomic (this
+// CTA's writes, ordered by bar.sync, are released; the last CTA acquires
+// everyone's).
 __device__ __forceinline__ bool grid_arrive(GridSync* g, uint32_t& gen0) {
     __shared__ int s_last;
     __shared__ uint32_t s_gen;
     __syncthreads();
     if (threadIdx.x == 0) {
-        s_gen = ld_acquire_u32(&g->gen);
-        __threadfence();
-        const uint32_t old = atomicAdd(&g->count, 1u);
+        s_gen = ld_relaxed_u32(&g->gen);
+        uint32_t old;
+        asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(&g->count) : "memory");
         s_last = (old == gridDim.x - 1) ? 1 : 0;
-        if (s_last) __threadfence();
     }
     __syncthreads();
     gen0 = s_gen;
@@ -1111,9 +1117,8 @@ __device__ __forceinline__ bool grid_arrive(GridSync* g, uint32_t& gen0) {
 __device__ __forceinline__ void grid_release(GridSync* g) {
     __syncthreads();
     if (threadIdx.x == 0) {
-        g->count = 0u;
-        __threadfence();
-        atomicAdd(&g->gen, 1u);
+        asm volatile("st.relaxed.gpu.global.u32 [%0], 0;" ::"l"(&g->count) : "memory");
+        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&g->gen) : "memory");
     }
 }
 __device__ __forceinline__ bool grid_wait(GridSync* g, uint32_t gen0, uint32_t* status) {
@@ -1128,7 +1133,6 @@ __device__ __forceinline__ bool grid_wait(GridSync* g, uint32_t gen0, uint32_t* 
                 break;
             }
         }
-        __threadfence();
         s_ok = ok;
     }
     __syncthreads();
