@@ -212,11 +212,6 @@ __device__ __forceinline__ uint32_t swar_ge(uint32_t m, uint32_t c) {
 __device__ __forceinline__ uint32_t swar_gt(uint32_t m, uint32_t c) {
     return (m + (0x7FFFu - c) * 0x10001u) & 0x80008000u;
 }
-__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
-    uint32_t d;
-    asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
-    return d;
-}
 
 // Bins of a 4096-bin shared histogram holding the entries of ranks r[0..2]
 // (each r < total), by NT threads: thread t owns 4096 / NT consecutive bins;
@@ -1082,62 +1077,6 @@ constexpr int kFusedThreads = 256;
 constexpr int kFusedMinBlocks = 3;
 constexpr int kCtaTotOffset = 8192;   // per-CTA totals in hist1 (after the band bins)
 constexpr int kFusedMaxGrid = 8192;
-constexpr long long kGridWaitLimit = 2000000000LL;   // SM clocks (~1-2 s)
-
-__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-__device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t* p) {
-    uint32_t v;
-    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-    return v;
-}
-
-// Arrive at a grid barrier.  Returns (in every thread) true in the CTA that
-// arrived last, which then runs its serial work and calls grid_release; the
-// others call grid_wait with gen0.  The arrival is an acq_rel atomic (this
-// CTA's writes, ordered by bar.sync, are released; the last CTA acquires
-// everyone's).
-__device__ __forceinline__ bool grid_arrive(GridSync* g, uint32_t& gen0) {
-    __shared__ int s_last;
-    __shared__ uint32_t s_gen;
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        s_gen = ld_relaxed_u32(&g->gen);
-        uint32_t old;
-        asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(&g->count) : "memory");
-        s_last = (old == gridDim.x - 1) ? 1 : 0;
-    }
-    __syncthreads();
-    gen0 = s_gen;
-    return s_last != 0;
-}
-__device__ __forceinline__ void grid_release(GridSync* g) {
-    __syncthreads();
-    if (threadIdx.x == 0) {
-        asm volatile("st.relaxed.gpu.global.u32 [%0], 0;" ::"l"(&g->count) : "memory");
-        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&g->gen) : "memory");
-    }
-}
-__device__ __forceinline__ bool grid_wait(GridSync* g, uint32_t gen0, uint32_t* status) {
-    __shared__ int s_ok;
-    if (threadIdx.x == 0) {
-        int ok = 1;
-        const long long t0 = clock64();
-        while (ld_acquire_u32(&g->gen) == gen0) {
-            if (clock64() - t0 > kGridWaitLimit) {
-                ok = 0;
-                flag_status(status, kStatusTimeout);
-                break;
-            }
-        }
-        s_ok = ok;
-    }
-    __syncthreads();
-    return s_ok != 0;
-}
 
 __global__ void __launch_bounds__(kFusedThreads, kFusedMinBlocks)
 act_fused_bf16_kernel(const uint16_t* __restrict__ A, int64_t lda, int M, int K,

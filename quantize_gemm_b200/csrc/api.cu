@@ -30,6 +30,8 @@ static cudaError_t ensure_device(int* dev_out) {
         if (e != cudaSuccess) return e;
         e = act_setup();
         if (e != cudaSuccess) return e;
+        e = cols_setup();
+        if (e != cudaSuccess) return e;
         e = gemm_setup();
         if (e != cudaSuccess) return e;
         e = spmm_setup();
@@ -219,6 +221,10 @@ qg_status qg_quantize_cols(const void* W, qg_dtype dtype, int64_t K, int64_t N, 
     const WsLayout L = ws_layout(QG_OP_QUANTIZE_COLS, 1, K, N, dtype, 1.0);
     if ((st = check_ws(ws, ws_bytes, L.total)) != QG_OK) return st;
     if (ensure_device(nullptr) != cudaSuccess) return QG_ERR_CUDA;
+    if (dtype == QG_BF16 &&
+        launch_quantize_cols_fused(W, K, N, ldw, codesT, scales, at<uint32_t>(ws, L.colmax),
+                                   at<GridSync>(ws, L.gsync), at<uint32_t>(ws, L.status), stream))
+        return cuda_status(cudaGetLastError());
     launch_quantize_cols(W, dtype, K, N, ldw, codesT, scales, at<uint32_t>(ws, L.colmax), stream);
     return cuda_status(cudaGetLastError());
 }

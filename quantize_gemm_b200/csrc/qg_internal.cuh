@@ -114,7 +114,9 @@ inline WsLayout ws_layout(qg_op op, int64_t M, int64_t K, int64_t N, qg_dtype dt
         L.st_col = take(sizeof(int32_t) * slots);
         L.st_val = take(sizeof(double) * slots);
     }
-    if (op == QG_OP_QUANTIZE_COLS) L.colmax = take(sizeof(uint32_t) * (size_t)N);
+    // column maxima: N words (fp32 path); the cooperative bf16 kernel keeps
+    // per-split partial maxima, up to 32 splits
+    if (op == QG_OP_QUANTIZE_COLS) L.colmax = take(sizeof(uint32_t) * 32 * (size_t)N);
     if (op == QG_OP_FP4_LINEAR) {
         int64_t cap = L.cap > 0 ? L.cap : 1;
         L.act_codes = take((size_t)M * (size_t)(K / 2));
@@ -214,6 +216,13 @@ __device__ __forceinline__ uint32_t nonfinite_key() {
     else return 0x7F800000u;
 }
 
+// Per-16-bit-half unsigned maximum.
+__device__ __forceinline__ uint32_t max_u16x2(uint32_t a, uint32_t b) {
+    uint32_t d;
+    asm("max.u16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+    return d;
+}
+
 __device__ __forceinline__ int warp_inclusive_scan(int v) {
     const int lane = threadIdx.x & 31;
 #pragma unroll
@@ -228,6 +237,69 @@ __device__ __forceinline__ uint32_t warp_max_u32(uint32_t v) {
 #pragma unroll
     for (int d = 16; d > 0; d >>= 1) v = max(v, __shfl_xor_sync(0xFFFFFFFFu, v, d));
     return v;
+}
+
+// ------------------------------------------------------- grid barrier
+// For cooperative launches (every CTA resident).  A count and a generation
+// word (GridSync, in the workspace status block, zero between barriers):
+// grid_arrive returns true in the CTA that arrived last, which runs its
+// serial work and calls grid_release; the other CTAs call grid_wait.  Waits
+// are bounded: a CTA that gives up sets the timeout bit and must return.
+constexpr long long kGridWaitLimit = 2000000000LL;   // SM clocks (~1-2 s)
+
+__device__ __forceinline__ uint32_t ld_acquire_u32(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+__device__ __forceinline__ uint32_t ld_relaxed_u32(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+// Arrive at a grid barrier.  Returns (in every thread) true in the CTA that
+// arrived last, which then runs its serial work and calls grid_release; the
+// others call grid_wait with gen0.  The arrival is an acq_rel atomic (this
+// CTA's writes, ordered by bar.sync, are released; the last CTA acquires
+// everyone's).
+__device__ __forceinline__ bool grid_arrive(GridSync* g, uint32_t& gen0) {
+    __shared__ int s_last;
+    __shared__ uint32_t s_gen;
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        s_gen = ld_relaxed_u32(&g->gen);
+        uint32_t old;
+        asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(old) : "l"(&g->count) : "memory");
+        s_last = (old == gridDim.x - 1) ? 1 : 0;
+    }
+    __syncthreads();
+    gen0 = s_gen;
+    return s_last != 0;
+}
+__device__ __forceinline__ void grid_release(GridSync* g) {
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        asm volatile("st.relaxed.gpu.global.u32 [%0], 0;" ::"l"(&g->count) : "memory");
+        asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(&g->gen) : "memory");
+    }
+}
+__device__ __forceinline__ bool grid_wait(GridSync* g, uint32_t gen0, uint32_t* status) {
+    __shared__ int s_ok;
+    if (threadIdx.x == 0) {
+        int ok = 1;
+        const long long t0 = clock64();
+        while (ld_acquire_u32(&g->gen) == gen0) {
+            if (clock64() - t0 > kGridWaitLimit) {
+                ok = 0;
+                flag_status(status, kStatusTimeout);
+                break;
+            }
+        }
+        s_ok = ok;
+    }
+    __syncthreads();
+    return s_ok != 0;
 }
 
 #endif  // __CUDACC__
@@ -267,6 +339,10 @@ cudaError_t run_clamp_compensate(const void* A, qg_dtype dt, int64_t M, int64_t 
                                  int64_t rank, const ActBuffers& b, void* A_c, const qg_csr* dA,
                                  float* T_out, cudaStream_t s);
 cudaError_t act_setup();
+cudaError_t cols_setup();
+bool launch_quantize_cols_fused(const void* W, int64_t K, int64_t N, int64_t ldw, uint8_t* codesT,
+                                float* scales, uint32_t* colpart, GridSync* gsync,
+                                uint32_t* status, cudaStream_t s);
 cudaError_t gemm_setup();
 cudaError_t spmm_setup();
 

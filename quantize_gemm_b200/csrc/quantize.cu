@@ -206,6 +206,203 @@ quantize_cols_kernel(const void* __restrict__ W, int64_t ldw, int K, int N,
     *dst = make_uint4(packed[0], packed[1], packed[2], packed[3]);
 }
 
+// --------------------------------------------------------------------------
+// bf16 W in one cooperative launch (all CTAs resident):
+//   phase 1  unit (split s, 256-column block): the max key of each column over
+//            the split's rows -> colpart[s][n] (no atomics, nothing to zero)
+//   barrier
+//   phase 2  tiles of 32 rows x 256 columns, a CTA's tiles consecutive in
+//            (column block, row tile) order: the column scales from the
+//            partial maxima (once per column block), the tile through shared
+//            memory (W is read a second time, mostly from L2), one thread
+//            per column encodes 32 values into 16 output bytes.
+constexpr int kColsFusedThreads = 256;
+constexpr int kColsMaxSplits = 32;
+
+__global__ void __launch_bounds__(kColsFusedThreads)
+quantize_cols_fused_bf16_kernel(const uint16_t* __restrict__ W, int64_t ldw, int K, int N,
+                                int splits, int rows_per_split, uint32_t* __restrict__ colpart,
+                                uint8_t* __restrict__ codesT, float* __restrict__ scales,
+                                GridSync* __restrict__ gsync, uint32_t* __restrict__ status) {
+    __shared__ uint32_t red[8][256];
+    __shared__ __align__(16) uint16_t tile[kColTileK][kColTileN];
+    __shared__ float s_r[kColTileN];
+    const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
+    const int cblocks = (N + 255) / 256;
+    const bool ld_vec = (ldw & 7) == 0;
+
+    // phase 1
+    for (int u = blockIdx.x; u < cblocks * splits; u += gridDim.x) {
+        const int cb = u % cblocks, sp = u / cblocks;
+        const int n0 = cb * 256 + lane * 8;
+        const int k0 = sp * rows_per_split, k1 = min(K, k0 + rows_per_split);
+        uint32_t m[4] = {0u, 0u, 0u, 0u};   // 16x2 maxima of the lane's 8 columns
+        if (n0 < N) {
+            if (ld_vec && n0 + 8 <= N) {
+                int k = k0 + warp;
+                for (; k + 24 < k1; k += 32) {      // four rows in flight per lane
+                    uint4 a[4];
+#pragma unroll
+                    for (int u = 0; u < 4; ++u)
+                        a[u] = __ldg(reinterpret_cast<const uint4*>(W + (int64_t)(k + 8 * u) * ldw + n0));
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        m[0] = max_u16x2(m[0], a[u].x & 0x7FFF7FFFu);
+                        m[1] = max_u16x2(m[1], a[u].y & 0x7FFF7FFFu);
+                        m[2] = max_u16x2(m[2], a[u].z & 0x7FFF7FFFu);
+                        m[3] = max_u16x2(m[3], a[u].w & 0x7FFF7FFFu);
+                    }
+                }
+                for (; k < k1; k += 8) {
+                    const uint4 a = __ldg(reinterpret_cast<const uint4*>(W + (int64_t)k * ldw + n0));
+                    m[0] = max_u16x2(m[0], a.x & 0x7FFF7FFFu);
+                    m[1] = max_u16x2(m[1], a.y & 0x7FFF7FFFu);
+                    m[2] = max_u16x2(m[2], a.z & 0x7FFF7FFFu);
+                    m[3] = max_u16x2(m[3], a.w & 0x7FFF7FFFu);
+                }
+            } else {
+                for (int k = k0 + warp; k < k1; k += 8) {
+#pragma unroll
+                    for (int e = 0; e < 8; ++e) {
+                        if (n0 + e >= N) continue;
+                        const uint32_t key = W[(int64_t)k * ldw + n0 + e] & 0x7FFFu;
+                        const uint32_t sh = (e & 1) ? 16 : 0;
+                        m[e >> 1] = max_u16x2(m[e >> 1], key << sh);
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) red[warp][lane * 8 + e] = (e & 1) ? (m[e >> 1] >> 16) : (m[e >> 1] & 0xFFFFu);
+        __syncthreads();
+        uint32_t v = 0;
+#pragma unroll
+        for (int w = 0; w < 8; ++w) v = max(v, red[w][t]);
+        const int n = cb * 256 + t;
+        if (n < N) colpart[(int64_t)sp * N + n] = v;
+        __syncthreads();   // red is reused by the next unit
+    }
+
+    uint32_t gen0;
+    if (grid_arrive(gsync, gen0)) grid_release(gsync);
+    else if (!grid_wait(gsync, gen0, status)) return;
+
+    // phase 2
+    const int ktiles = K / kColTileK;
+    const int total = cblocks * ktiles;
+    const int per = (total + gridDim.x - 1) / gridDim.x;
+    const int t0 = blockIdx.x * per, t1 = min(total, t0 + per);
+    int cur_cb = -1;
+    // this thread's part of a tile: rows warp + 8 u (u < 4), columns lane * 8 .. + 7
+    auto load_tile = [&](int ti, uint4 (&v)[4]) {
+        const int cb = ti / ktiles, kt = ti - cb * ktiles;
+        const int nc = cb * kColTileN + lane * 8;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) {
+            const int k = kt * kColTileK + warp + 8 * u;
+            v[u] = make_uint4(0u, 0u, 0u, 0u);
+            if (ld_vec && nc + 8 <= N) {
+                v[u] = __ldg(reinterpret_cast<const uint4*>(W + (int64_t)k * ldw + nc));
+            } else if (nc < N) {
+                uint16_t h[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) h[e] = (nc + e < N) ? W[(int64_t)k * ldw + nc + e] : (uint16_t)0;
+                v[u] = make_uint4(h[0] | ((uint32_t)h[1] << 16), h[2] | ((uint32_t)h[3] << 16),
+                                  h[4] | ((uint32_t)h[5] << 16), h[6] | ((uint32_t)h[7] << 16));
+            }
+        }
+    };
+    uint4 nxt[4];
+    if (t0 < t1) load_tile(t0, nxt);
+    for (int ti = t0; ti < t1; ++ti) {
+        const int cb = ti / ktiles, kt = ti - cb * ktiles;
+        const int n_base = cb * kColTileN, k_base = kt * kColTileK;
+        __syncthreads();   // the previous tile's reads of tile / s_r are done
+        if (cb != cur_cb) {
+            const int n = n_base + t;
+            float r = 0.0f, sc = 0.0f;
+            if (n < N) {
+                uint32_t key = 0;
+                for (int sp = 0; sp < splits; ++sp) key = max(key, __ldcg(colpart + (int64_t)sp * N + n));
+                scale_factors(__uint_as_float(key << 16), r, sc);
+                if (kt == 0) scales[n] = sc;
+            }
+            s_r[t] = r;
+            cur_cb = cb;
+        }
+#pragma unroll
+        for (int u = 0; u < 4; ++u) *reinterpret_cast<uint4*>(&tile[warp + 8 * u][lane * 8]) = nxt[u];
+        __syncthreads();
+        if (ti + 1 < t1) load_tile(ti + 1, nxt);   // in flight while this tile is encoded
+        const int n = n_base + t;
+        if (n < N) {
+            const float r = s_r[t];
+            uint32_t packed[4];
+#pragma unroll
+            for (int q = 0; q < 4; ++q) {
+                float y[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    y[e] = __fmul_rn(__uint_as_float((uint32_t)tile[q * 8 + e][t] << 16), r);
+                packed[q] = e2m1x8(y);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(codesT + (int64_t)n * (K / 2) + k_base / 2);
+            *dst = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        }
+    }
+}
+
+// Resident CTAs per SM of the cooperative column kernel, per device.
+static int g_cols_blocks[64];
+
+cudaError_t cols_setup() {
+    int dev = 0, coop = 0, nb = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    e = cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev);
+    if (e != cudaSuccess) return e;
+    if (coop) {
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, quantize_cols_fused_bf16_kernel,
+                                                          kColsFusedThreads, 0);
+        if (e != cudaSuccess) return e;
+    }
+    if (dev >= 0 && dev < 64) g_cols_blocks[dev] = coop ? nb : 0;
+    return cudaSuccess;
+}
+
+size_t cols_fused_scratch_words(int64_t N) { return (size_t)kColsMaxSplits * (size_t)N; }
+
+bool launch_quantize_cols_fused(const void* W, int64_t K, int64_t N, int64_t ldw, uint8_t* codesT,
+                                float* scales, uint32_t* colpart, GridSync* gsync,
+                                uint32_t* status, cudaStream_t s) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+    const int nb = g_cols_blocks[dev];
+    if (nb < 1) return false;
+    const int cblocks = (int)((N + 255) / 256);
+    const int ktiles = (int)(K / kColTileK);
+    const int grid = (int)std::max<int64_t>(
+        1, std::min<int64_t>((int64_t)nb * num_sms(), (int64_t)cblocks * ktiles));
+    // splits: at most one unit per CTA, at least 32 rows per split
+    int splits = (int)std::max<int64_t>(1, grid / cblocks);
+    splits = (int)std::min<int64_t>({(int64_t)splits, (int64_t)kColsMaxSplits, std::max<int64_t>(1, K / 32)});
+    const int rows_per = (int)((K + splits - 1) / splits);
+    splits = (int)((K + rows_per - 1) / rows_per);
+    const uint16_t* Wb = static_cast<const uint16_t*>(W);
+    int Ki = (int)K, Ni = (int)N;
+    void* args[] = {(void*)&Wb, (void*)&ldw, (void*)&Ki, (void*)&Ni, (void*)&splits, (void*)&rows_per,
+                    (void*)&colpart, (void*)&codesT, (void*)&scales, (void*)&gsync, (void*)&status};
+    const cudaError_t e = cudaLaunchCooperativeKernel((const void*)quantize_cols_fused_bf16_kernel,
+                                                      dim3((unsigned)grid), dim3(kColsFusedThreads),
+                                                      args, 0, s);
+    if (e != cudaSuccess) {
+        (void)cudaGetLastError();
+        return false;
+    }
+    count_launch(1);
+    return true;
+}
+
 __global__ void zero_u32_kernel(uint32_t* __restrict__ p, int64_t n) {
     for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
          i += (int64_t)gridDim.x * blockDim.x)
