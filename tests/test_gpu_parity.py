@@ -133,10 +133,22 @@ def test_quantize_cols(qg, K, N, dtype):
     assert np.array_equal(_np(codesT), oT)
 
 
-def test_quantize_cols_special_values(qg):
-    W = _special_rows(256, torch.float32).t().contiguous().cuda()   # columns = special rows
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16])
+def test_quantize_cols_special_values(qg, dtype):
+    W = _special_rows(256, dtype).t().contiguous().cuda()   # columns = special rows
     codesT, t = qg.quantize_cols(W)
     oT, ot = oracle.quantize_cols(W.cpu())
+    assert np.array_equal(_np(t), ot) and np.array_equal(_np(codesT), oT)
+
+
+@pytest.mark.parametrize("width", [600, 604])
+def test_quantize_cols_strided_bf16(qg, width):
+    """A column block of a wider bf16 matrix: row pitch 600 (16-byte rows) and
+    604 (rows not 16-byte multiples, element loads)."""
+    Wide = make_matrix((288, width), seed=width, device="cuda", dtype=torch.bfloat16, scale=0.02)
+    W = Wide[:, :300]
+    codesT, t = qg.quantize_cols(W)
+    oT, ot = oracle.quantize_cols(W.cpu().contiguous())
     assert np.array_equal(_np(t), ot) and np.array_equal(_np(codesT), oT)
 
 
