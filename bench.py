@@ -125,11 +125,11 @@ class ClockSampler:
 
 # ------------------------------------------------------------------ our arm
 class Layer:
-    def __init__(self, qg, wl, li, device):
+    def __init__(self, qg, wl, li, device, alpha=None):
         from workloads import make_layer_inputs
         self.name = wl.layers[li].name
         self.A, self.W = make_layer_inputs(wl, li, device=device)
-        self.alpha = wl.alphas[0]
+        self.alpha = wl.alphas[0] if alpha is None else alpha
         M, K = self.A.shape
         N = self.W.shape[1]
         self.M, self.K, self.N = M, K, N
@@ -191,7 +191,7 @@ def our_arm(args, rank, world, device):
     wl = WORKLOADS[args.workload]
     peaks = _peaks()
     idx = range(len(wl.layers)) if args.layer is None else [args.layer]
-    layers = [Layer(qg, wl, i, device) for i in idx]
+    layers = [Layer(qg, wl, i, device, args.alpha) for i in idx]
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
     stream = torch.cuda.current_stream()
 
@@ -288,7 +288,7 @@ def our_arm(args, rank, world, device):
         "data": "synthetic",
         "config": {"workload": wl.name if args.layer is None else f"{wl.name}:{layers[0].name}",
                    "description": wl.description, "M": wl.M,
-                   "layers": [[L.name, L.K, L.N] for L in layers], "alpha": wl.alphas[0],
+                   "layers": [[L.name, L.K, L.N] for L in layers], "alpha": layers[0].alpha,
                    "input_dtype": wl.dtype, "y_dtype": "f32",
                    "l2": "flushed (256 MiB write between timed steps)",
                    "parallelism": f"replicas x{world}"},
@@ -406,13 +406,14 @@ def _ncu_traffic(kernel, workload):
 
 
 # ------------------------------------------------------------------ CPU oracle
-def _oracle_sample(wl, A_list, W_list, rows_per_layer):
+def _oracle_sample(wl, A_list, W_list, rows_per_layer, alpha=None):
     """Run the oracle on a bounded sample of one step: the full quantizers on
     every layer, Y for `rows_per_layer` rows of each layer.  Returns (seconds,
     flops the sample stands for after scaling the Y rows to M)."""
     import oracle
     t_total = 0.0
-    for A, W, alpha in zip(A_list, W_list, [wl.alphas[0]] * len(A_list)):
+    alpha = wl.alphas[0] if alpha is None else alpha
+    for A, W in zip(A_list, W_list):
         M, K = A.shape
         N = W.shape[1]
         t0 = time.perf_counter()
@@ -432,7 +433,7 @@ def cpu_baseline(args, wl, layers):
     A_list = [oracle.as_f32(L.A.cpu()) for L in layers]
     W_list = [oracle.as_f32(L.W.cpu()) for L in layers]
     rows = 16
-    t_est = _oracle_sample(wl, A_list, W_list, rows)
+    t_est = _oracle_sample(wl, A_list, W_list, rows, layers[0].alpha)
     flops = sum(L.flops for L in layers)
     return {"value": round(flops / t_est / 1e12, 6), "unit": "TFLOP/s",
             "cores": oracle.num_threads(), "kind": "oracle",
@@ -456,10 +457,10 @@ def reference_arm(args, rank, world):
     rows = 8
     warm = min(args.warmup, 1)        # the oracle needs no warm-up beyond one pass
     for _ in range(warm):
-        _oracle_sample(wl, A_list, W_list, rows)
+        _oracle_sample(wl, A_list, W_list, rows, args.alpha)
     total = 0.0
     for _ in range(args.steps):
-        total += _oracle_sample(wl, A_list, W_list, rows)
+        total += _oracle_sample(wl, A_list, W_list, rows, args.alpha)
     flops = sum(2 * wl.M * wl.layers[i].K * wl.layers[i].N for i in idx)
     value = flops * args.steps / total / 1e12
     cores = oracle.num_threads()
@@ -472,12 +473,75 @@ def reference_arm(args, rank, world):
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": wl.name if args.layer is None else f"{wl.name}:{wl.layers[idx[0]].name}",
                    "M": wl.M, "layers": [[wl.layers[i].name, wl.layers[i].K, wl.layers[i].N] for i in idx],
-                   "alpha": wl.alphas[0]},
+                   "alpha": wl.alphas[0] if args.alpha is None else args.alpha},
         "cpu_baseline": {"kind": "oracle", "cores": cores, "sample": sample,
                          "value": round(value, 6), "unit": "TFLOP/s"},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,
                 "d2h_bytes_per_step": 0},
     }
+
+
+def quantizer_sweep(device, reps=20, warm=5):
+    """The quantizers alone over A = M x 4096 bf16, Student-t(3), M = 256 * 2^j
+    (1M .. 256M elements), alpha = 0.99; quantize_cols on a 4096 x M weight of
+    the same element count.  Median of `reps` CUDA-event timings, L2 flushed
+    (256 MiB write) before each; GB/s from algorithmic bytes."""
+    import quantize_gemm_b200 as qg
+    from workloads import make_matrix
+    peaks = _peaks()
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    def timed(fn):
+        for _ in range(warm):
+            fn()
+        ts = []
+        for _ in range(reps):
+            flush.fill_(1)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        ts.sort()
+        return ts[len(ts) // 2]
+
+    K, alpha = 4096, 0.99
+    for j in range(9):
+        M = 256 * 2 ** j
+        n = M * K
+        A = make_matrix((M, K), ("student_t", 3), seed=5000 + j, device=device, dtype=torch.bfloat16)
+        codes = torch.empty((M, K // 2), dtype=torch.uint8, device=device)
+        s = torch.empty(M, dtype=torch.float32, device=device)
+        ws_r = qg.Workspace(qg.QG_OP_QUANTIZE_ROWS, M, K, 1, qg.QG_BF16, device=device)
+        t_rows = timed(lambda: qg.qg_quantize_rows(A, codes, s, ws_r))
+        ws_a = qg.Workspace(qg.QG_OP_QUANTIZE_ACT, M, K, 1, qg.QG_BF16, alpha, device=device)
+        csr = qg.CSR.empty(M, qg.qg_nnz_capacity(n, alpha), device=device)
+        T = torch.empty(1, dtype=torch.float32, device=device)
+        t_act = timed(lambda: qg.qg_quantize_act(A, alpha, codes, s, csr, T, ws_a))
+        qg.check_status(ws_a, "sweep quantize_act")
+        nnz = int(csr.nnz.item())
+        del A, csr, ws_a, ws_r
+        W = make_matrix((K, M), ("normal",), seed=6000 + j, device=device, dtype=torch.bfloat16,
+                        scale=0.02)
+        codesT = torch.empty((M, K // 2), dtype=torch.uint8, device=device)
+        tw = torch.empty(M, dtype=torch.float32, device=device)
+        ws_c = qg.Workspace(qg.QG_OP_QUANTIZE_COLS, 1, K, M, qg.QG_BF16, device=device)
+        t_cols = timed(lambda: qg.qg_quantize_cols(W, codesT, tw, ws_c))
+        qg.check_status(ws_c, "sweep quantize_cols")
+        del W, ws_c, codesT, codes
+        torch.cuda.empty_cache()
+        by = {"quantize_rows": 2 * n + n / 2 + 4 * M,
+              "quantize_act": 2 * 2 * n + n / 2 + 4 * M + 16 * nnz + 4 * (M + 1) + 8 * M,
+              "quantize_cols": 2 * 2 * n + n / 2 + 4 * M}
+        line = {"sweep": "quantizers", "elements": n, "M": M, "K": K, "alpha": alpha, "nnz": nnz,
+                "dtype": "bf16", "l2": "flushed before each rep", "reps": reps}
+        for k, t in (("quantize_rows", t_rows), ("quantize_act", t_act), ("quantize_cols", t_cols)):
+            gbs = by[k] / (t * 1e-3) / 1e9
+            line[k] = {"ms": round(t, 4), "GB/s": round(gbs, 1),
+                       "frac_measured": round(gbs / peaks["hbm_gbs"], 4),
+                       "frac_8TBs": round(gbs / 8000.0, 4)}
+        print(json.dumps(line), flush=True)
 
 
 def main():
@@ -491,6 +555,11 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--alpha", type=float, default=None,
+                    help="quantile of the clamp (default: the workload's first)")
+    ap.add_argument("--quantizer-sweep", action="store_true",
+                    help="time the three quantizers over 1M..256M bf16 elements (one JSON line "
+                         "per size) instead of the layer stream")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -515,6 +584,10 @@ def main():
     import __graft_entry__
     if rank == 0:
         __graft_entry__.build()
+    if args.quantizer_sweep:
+        if rank == 0:
+            quantizer_sweep(device)
+        return
     if world > 1:
         torch.distributed.barrier()
     out = our_arm(args, rank, world, device)

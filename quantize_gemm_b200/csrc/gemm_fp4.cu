@@ -409,6 +409,29 @@ __device__ __forceinline__ void epi_direct(const Params& p, const uint32_t (&v)[
         }
     }
     if (p.Y == nullptr) return;
+    if (full && !p.y_bf16) {
+        // 16-byte loads of C and the column scales, 16-byte stores of Y
+        float* yrow = static_cast<float*>(p.Y) + off;
+        const float4* tw = reinterpret_cast<const float4*>(p.sW + col0);
+        const float4* crow = p.C ? reinterpret_cast<const float4*>(p.C + off) : nullptr;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) {
+            const float4 t = __ldg(tw + j);
+            float4 y = make_float4(__fmul_rn(__fmul_rn(__uint_as_float(v[4 * j]), s_row), t.x),
+                                   __fmul_rn(__fmul_rn(__uint_as_float(v[4 * j + 1]), s_row), t.y),
+                                   __fmul_rn(__fmul_rn(__uint_as_float(v[4 * j + 2]), s_row), t.z),
+                                   __fmul_rn(__fmul_rn(__uint_as_float(v[4 * j + 3]), s_row), t.w));
+            if (crow) {
+                const float4 c = __ldg(crow + j);
+                y.x = __fadd_rn(y.x, c.x);
+                y.y = __fadd_rn(y.y, c.y);
+                y.z = __fadd_rn(y.z, c.z);
+                y.w = __fadd_rn(y.w, c.w);
+            }
+            reinterpret_cast<float4*>(yrow)[j] = y;
+        }
+        return;
+    }
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
         if (col0 + j >= p.N) continue;
@@ -885,8 +908,11 @@ cudaError_t launch_fp4_gemm(const uint8_t* codesA, const float* sA, const uint8_
     p.y_bf16 = (y_dtype == QG_BF16) ? 1 : 0;
     // TMA epilogue: the row pitches of Y and C must be multiples of 16 bytes
     const size_t ysz = (y_dtype == QG_BF16) ? 2 : 4;
-    p.tma_epi = (Y != nullptr && raw_acc == nullptr && ((size_t)N * ysz) % 16 == 0 &&
-                 ((size_t)N * 4) % 16 == 0)
+#ifndef QG_GEMM_DIRECT_EPI
+#define QG_GEMM_DIRECT_EPI 0
+#endif
+    p.tma_epi = (!QG_GEMM_DIRECT_EPI && Y != nullptr && raw_acc == nullptr &&
+                 ((size_t)N * ysz) % 16 == 0 && ((size_t)N * 4) % 16 == 0)
                     ? 1
                     : 0;
     CUtensorMap ta, ty, tc;

@@ -324,6 +324,25 @@ def test_fp4_gemm_epilogue_fp32(qg, M, N, K, with_c):
     assert y_rel_err(_np(Y), Yo) <= 1e-3
 
 
+@pytest.mark.parametrize("M,N,K", [(300, 600, 1024), (129, 257, 288), (256, 5504, 512)])
+def test_fp4_gemm_direct_epilogue(qg, M, N, K):
+    """Raw accumulator requested: the register-to-global epilogue writes Y too
+    (16-byte stores for whole 32-column chunks when N % 8 == 0, scalar stores
+    otherwise); Y with C must match like the TMA epilogue's."""
+    g = np.random.default_rng(M + 7 * N)
+    cA, cW = _rand_codes(M, K, 31 + M), _rand_codes(N, K, 32 + N)
+    sA = (g.random(M) * 0.1 + 1e-3).astype(np.float32)
+    sW = (g.random(N) * 0.01 + 1e-4).astype(np.float32)
+    C = (g.standard_normal((M, N)) * 0.5).astype(np.float32)
+    Y, acc = qg.fp4_gemm(torch.from_numpy(cA).cuda(), torch.from_numpy(sA).cuda(),
+                         torch.from_numpy(cW).cuda(), torch.from_numpy(sW).cuda(), K,
+                         C=torch.from_numpy(C).cuda(), raw=True)
+    want = oracle.gemm_acc(cA, cW, K)
+    assert np.array_equal(_np(acc).astype(np.float64), want)
+    Yo = want * sA.astype(np.float64)[:, None] * sW.astype(np.float64)[None, :] + C.astype(np.float64)
+    assert y_rel_err(_np(Y), Yo) <= 1e-3
+
+
 def test_fp4_gemm_epilogue_bf16(qg):
     M, N, K = 300, 600, 1024
     g = np.random.default_rng(2)
