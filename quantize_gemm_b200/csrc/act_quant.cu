@@ -440,6 +440,69 @@ __device__ __forceinline__ void band_rows(const uint16_t* __restrict__ A, int64_
     }
 }
 
+// The band pass over (row, 1024-column step) units u = gwarp, gwarp + nwarps,
+// ... (u = row * steps + step): the unit's max key into rowmax[u], count of
+// keys >= lo into n_ge, keys in [lo, hi] into sh (at key - lo), non-finite
+// keys into bad.  Finer than whole rows, so the warps finish together.
+__device__ __forceinline__ void band_units(const uint16_t* __restrict__ A, int64_t lda, int M, int K,
+                                           uint32_t lo, uint32_t hi, uint32_t* sh,
+                                           uint32_t* __restrict__ rowmax, int gwarp, int nwarps,
+                                           unsigned long long& n_ge, uint32_t& bad) {
+    const int lane = threadIdx.x & 31;
+    const int nchunks = K / 8;
+    const int steps = (nchunks + 127) / 128;
+    const int64_t units = (int64_t)M * steps;
+    auto load_unit = [&](int64_t u, uint4 (&dst)[4]) {
+        const int64_t r = u / steps;
+        const int st = (int)(u - r * steps);
+        const uint16_t* base = A + r * lda;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const int c = st * 128 + 32 * j + lane;
+            dst[j] = (c < nchunks) ? __ldg(reinterpret_cast<const uint4*>(base) + c)
+                                   : make_uint4(0u, 0u, 0u, 0u);
+        }
+    };
+    int64_t u = gwarp;
+    uint4 nxt[4];
+    if (u < units) load_unit(u, nxt);
+    while (u < units) {
+        uint4 cur[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) cur[j] = nxt[j];
+        const int64_t nu = u + nwarps;
+        if (nu < units) load_unit(nu, nxt);
+        const int st = (int)(u % steps);
+        uint32_t mx = 0, mx1 = 0, cnt = 0, cnt1 = 0;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            if (st * 128 + 32 * j + lane >= nchunks) continue;   // past K
+            const uint32_t w[4] = {cur[j].x, cur[j].y, cur[j].z, cur[j].w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const uint32_t m = w[i] & 0x7FFF7FFFu;
+                if (i & 1) mx1 = max_u16x2(mx1, m);
+                else mx = max_u16x2(mx, m);
+                const uint32_t ge = swar_ge(m, lo);
+                if (i & 1) cnt1 += ge >> 15;
+                else cnt += ge >> 15;
+                const uint32_t in = ge & ~swar_gt(m, hi);
+                if (in) {
+                    if (in & 0x8000u) atomicAdd(&sh[(m & 0xFFFFu) - lo], 1u);
+                    if (in >> 16) atomicAdd(&sh[(m >> 16) - lo], 1u);
+                }
+            }
+        }
+        mx = max_u16x2(mx, mx1);
+        cnt += cnt1;
+        const uint32_t km = warp_max_u32(max(mx & 0xFFFFu, mx >> 16));
+        if (lane == 0) rowmax[u] = km;
+        bad |= (km >= nonfinite_key<QG_BF16>()) ? 1u : 0u;
+        n_ge += (cnt & 0xFFFFu) + (cnt >> 16);
+        u = nu;
+    }
+}
+
 // A CTA's share of the band pass into the global counters and bins.
 template <int NT>
 __device__ void band_flush(const uint32_t* sh, uint32_t* __restrict__ band_bins,
@@ -775,7 +838,8 @@ __device__ __forceinline__ void clamp_rows_bf16(const uint16_t* __restrict__ A, 
                                                 Counters* __restrict__ ctr,
                                                 uint8_t* __restrict__ codes,
                                                 float* __restrict__ scales, const ActBuffers& b,
-                                                int first, int stride, int row_end) {
+                                                int first, int stride, int row_end,
+                                                int nparts = 1) {
     // (an unselected threshold reads as the largest finite-or-not key)
     const uint32_t Tk = min(T_key, 0x7FFFu);
     const uint32_t cT = (0x7FFFu - Tk) * 0x10001u;   // SWAR: key > T sets bit 15
@@ -802,7 +866,8 @@ __device__ __forceinline__ void clamp_rows_bf16(const uint16_t* __restrict__ A, 
     int row_rank = 0;
     while (row < row_end) {
         if (step == 0) {
-            const uint32_t rmax = __ldcg(rowmax + row);
+            uint32_t rmax = 0;   // the row's max key: over its nparts partial maxima
+            for (int q = 0; q < nparts; ++q) rmax = max(rmax, __ldcg(rowmax + (int64_t)row * nparts + q));
             float s;
             scale_factors(__uint_as_float(min(rmax, Tk) << 16), r, s);
             if (lane == 0) scales[row] = s;
@@ -1108,7 +1173,7 @@ act_fused_bf16_kernel(const uint16_t* __restrict__ A, int64_t lda, int M, int K,
         const uint32_t lo = __ldcg(&b.ctr->band_lo), hi = __ldcg(&b.ctr->band_hi);
         unsigned long long n_ge = 0;
         uint32_t bad = 0;
-        band_rows(A, lda, M, K, lo, hi, sh, b.rowmax, gwarp, nwarps, n_ge, bad);
+        band_units(A, lda, M, K, lo, hi, sh, b.rowmax, gwarp, nwarps, n_ge, bad);
         band_flush<kFusedThreads>(sh, b.hist1, n_ge, bad, b.ctr);
     }
     // phase 2
@@ -1120,14 +1185,14 @@ act_fused_bf16_kernel(const uint16_t* __restrict__ A, int64_t lda, int M, int K,
     }
 
     // phase 3: CTA c clamps rows [r0, r1), a warp per row, then scans its
-    // rows' counts locally (the prefix overwrites rowmax, no longer needed)
+    // rows' counts locally into rowpre
     const int rpc = (M + (int)gridDim.x - 1) / (int)gridDim.x;
     const int r0 = min(M, (int)blockIdx.x * rpc), r1 = min(M, r0 + rpc);
     clamp_rows_bf16(A, lda, M, K, __ldcg(&b.ctr->T_key), b.rowmax, b.ctr, codes, scales, b,
-                    r0 + (int)(threadIdx.x >> 5), wpc, r1);
+                    r0 + (int)(threadIdx.x >> 5), wpc, r1, (K / 8 + 127) / 128);
     uint32_t* cta_off = b.hist1 + kCtaTotOffset;   // per-CTA totals, then offsets
     __syncthreads();
-    cta_local_scan<kFusedThreads>(b.rowcnt + r0, r1 - r0, b.rowmax + r0, cta_off + blockIdx.x);
+    cta_local_scan<kFusedThreads>(b.rowcnt + r0, r1 - r0, b.rowpre + r0, cta_off + blockIdx.x);
     // phase 4: the last CTA turns the CTA totals into offsets
     if (grid_arrive(g, gen0)) {
         cta_scan_offsets<kFusedThreads>(cta_off, (int)gridDim.x, b, M, row_ptr, nnz_out);
@@ -1140,13 +1205,13 @@ act_fused_bf16_kernel(const uint16_t* __restrict__ A, int64_t lda, int M, int K,
     // the overflow list
     const uint32_t off = __ldcg(cta_off + blockIdx.x);
     for (int r = r0 + (int)threadIdx.x; r < r1; r += kFusedThreads)
-        row_ptr[r] = (int32_t)(b.rowmax[r] + off);
+        row_ptr[r] = (int32_t)(b.rowpre[r] + off);
     {
         const int lane = threadIdx.x & 31;
         const int row_slots = (int)b.row_slots;
         for (int r = r0 + (int)(threadIdx.x >> 5); r < r1; r += wpc) {
             const int n = min((int)b.rowcnt[r], row_slots);
-            const int64_t dst = (int64_t)b.rowmax[r] + off;
+            const int64_t dst = (int64_t)b.rowpre[r] + off;
             const int64_t src = (int64_t)r * row_slots;
             for (int jj = lane; jj < n; jj += 32) {
                 col[dst + jj] = __ldcg(b.st_col + src + jj);
@@ -1158,7 +1223,7 @@ act_fused_bf16_kernel(const uint16_t* __restrict__ A, int64_t lda, int M, int K,
         for (unsigned long long e = blockIdx.x * (unsigned long long)kFusedThreads + threadIdx.x;
              e < n_over; e += (unsigned long long)gridDim.x * kFusedThreads) {
             const int rr = __ldcg(b.st_row + e);
-            const int64_t dst = (int64_t)__ldcg(b.rowmax + rr) + __ldcg(cta_off + rr / rpc) +
+            const int64_t dst = (int64_t)__ldcg(b.rowpre + rr) + __ldcg(cta_off + rr / rpc) +
                                 __ldcg(b.st_rank + e);
             col[dst] = __ldcg(b.st_col + base + e);
             val[dst] = __ldcg(b.st_val + base + e);

@@ -93,6 +93,7 @@ static ActBuffers act_buffers(void* ws, const WsLayout& L) {
     b.hist2 = L.hist2 ? at<uint32_t>(ws, L.hist2) : nullptr;
     b.rowmax = at<uint32_t>(ws, L.rowmax);
     b.rowcnt = at<uint32_t>(ws, L.rowcnt);
+    b.rowpre = at<uint32_t>(ws, L.rowpre);
     b.st_row = at<int32_t>(ws, L.st_row);
     b.st_rank = at<int32_t>(ws, L.st_rank);
     b.st_col = at<int32_t>(ws, L.st_col);

@@ -72,6 +72,7 @@ constexpr size_t kGridSyncOffset = 16;   // bytes from the workspace base
 
 struct WsLayout {
     size_t gsync = 0;
+    size_t rowpre = 0;
     size_t status = 0, counters = 0, hist1 = 0, hist2 = 0, rowmax = 0, rowcnt = 0;
     size_t st_row = 0, st_rank = 0, st_col = 0, st_val = 0, colmax = 0;
     size_t act_codes = 0, act_scales = 0, csr_row_ptr = 0, csr_col = 0, csr_val = 0,
@@ -105,8 +106,12 @@ inline WsLayout ws_layout(qg_op op, int64_t M, int64_t K, int64_t N, qg_dtype dt
         int64_t cap = L.cap > 0 ? L.cap : 1;
         L.hist1 = take(sizeof(uint32_t) * kHist1Bins);
         if (dtype == QG_F32) L.hist2 = take(sizeof(uint32_t) * kHist2Bins);
-        L.rowmax = take(sizeof(uint32_t) * (size_t)M);
+        // row maxima: one per (row, 1024-column step) for the cooperative
+        // bf16 kernel (the other kernels use the first M words, one per row)
+        const int64_t steps = (K / 8 + 127) / 128;
+        L.rowmax = take(sizeof(uint32_t) * (size_t)M * (size_t)steps);
         L.rowcnt = take(sizeof(uint32_t) * (size_t)M);
+        L.rowpre = take(sizeof(uint32_t) * (size_t)M);
         L.row_slots = staging_row_slots(M, K, L.cap);
         const size_t slots = (size_t)M * (size_t)L.row_slots + (size_t)cap;
         L.st_row = take(sizeof(int32_t) * (size_t)cap);     // overflow list only
@@ -313,6 +318,7 @@ struct ActBuffers {
     uint32_t* hist2;
     uint32_t* rowmax;
     uint32_t* rowcnt;
+    uint32_t* rowpre;    // CTA-local prefix of the row counts (cooperative kernel)
     int32_t *st_row, *st_rank, *st_col;
     double* st_val;
     int64_t cap;
