@@ -818,16 +818,6 @@ constexpr int kQ3Threads = 256;
 #endif
 constexpr int kQ3MinBlocks = QG_CLAMP_MIN_BLOCKS;   // resident CTAs per SM (register cap)
 
-// Scale a bf16 pair by r and encode it: one byte, element 0 in the low nibble.
-__device__ __forceinline__ uint32_t bf16x2_encode(uint32_t w, float r) {
-    const float lo = __uint_as_float(w << 16), hi = __uint_as_float(w & 0xFFFF0000u);
-    float a, b;
-    asm("{\n\t.reg .b64 p, q, t;\n\tmov.b64 p, {%2, %3};\n\tmov.b64 q, {%4, %4};\n\t"
-        "mul.rn.f32x2 t, p, q;\n\tmov.b64 {%0, %1}, t;\n\t}"
-        : "=f"(a), "=f"(b)
-        : "f"(lo), "f"(hi), "f"(r));
-    return e2m1x2(a, b);
-}
 
 // The clamp / quantize pass over rows first, first + stride, ... (< row_end)
 // of this warp; M is the matrix height (the overflow slots follow M row

@@ -156,6 +156,17 @@ __device__ __forceinline__ uint32_t e2m1x2(float lo, float hi) {
     return (uint32_t)r & 0xFFu;
 }
 
+// Scale a bf16 pair by r and encode it: one byte, element 0 in the low nibble.
+__device__ __forceinline__ uint32_t bf16x2_encode(uint32_t w, float r) {
+    const float lo = __uint_as_float(w << 16), hi = __uint_as_float(w & 0xFFFF0000u);
+    float a, b;
+    asm("{\n\t.reg .b64 p, q, t;\n\tmov.b64 p, {%2, %3};\n\tmov.b64 q, {%4, %4};\n\t"
+        "mul.rn.f32x2 t, p, q;\n\tmov.b64 {%0, %1}, t;\n\t}"
+        : "=f"(a), "=f"(b)
+        : "f"(lo), "f"(hi), "f"(r));
+    return e2m1x2(a, b);
+}
+
 // Eight values -> four packed bytes (element 0 in the low nibble of byte 0).
 __device__ __forceinline__ uint32_t e2m1x8(const float (&x)[8]) {
     return e2m1x2(x[0], x[1]) | (e2m1x2(x[2], x[3]) << 8) | (e2m1x2(x[4], x[5]) << 16) |

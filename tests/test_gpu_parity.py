@@ -87,6 +87,7 @@ ROW_CASES = [
     (1, 32, torch.float32), (3, 64, torch.bfloat16), (257, 512, torch.float32),
     (100, 1056, torch.bfloat16), (64, 16384, torch.bfloat16), (32, 16384, torch.float32),
     (129, 2048, torch.bfloat16), (7, 4128, torch.float32),
+    (50, 3072, torch.bfloat16), (77, 4096, torch.bfloat16), (5, 4064, torch.bfloat16),
 ]
 
 
