@@ -32,8 +32,10 @@
  *     transposed, N x K/2 bytes, so both GEMM operands have K contiguous.
  *   - Shapes: K % 32 == 0 and 0 < K <= 16384 (else QG_ERR_UNSUPPORTED_SHAPE);
  *     M, N >= 1 arbitrary.  Row strides (lda, ldw) are in elements, at least
- *     the row length, and keep every row start 16-byte aligned.  Base
- *     pointers are 16-byte aligned.
+ *     the row length; lda keeps every row start of A 16-byte aligned (checked).
+ *     ldw may be any value >= N: rows of W that are not 16-byte multiples
+ *     are read element by element (slower).  Base pointers are 16-byte
+ *     aligned.
  *   - Workspace: calls that take (ws, ws_bytes) use a caller-allocated device
  *     buffer of at least qg_workspace_size(...) bytes, 256-byte aligned.  Its
  *     first bytes hold a sticky device status word; initialise a new

@@ -8,21 +8,27 @@
 // granularity + ScaleShift paragraphs for the row quantization of A_clamped.
 //
 // The threshold is the exact order statistic T = sorted(|A|)[k] over the whole
-// tensor, found by a radix histogram of the magnitude bit patterns (integer
-// keys order like |x| for finite values):
-//   bf16: one pass, 2^15 bins = every possible magnitude;
+// tensor; integer keys (the magnitude bit patterns) order like |x| for finite
+// values.
+//   bf16: a sample of A puts a band of at most 4096 keys around the sample
+//         quantile; one pass counts the keys below the band and histograms
+//         the keys inside it (SWAR on packed bf16 pairs), and the order
+//         statistic is selected from the band -- or, when it is not inside
+//         it, by an exact two-level count over all of A (same result).
 //   fp32: a 2^15-bin pass on bits 30..16, then a 2^16-bin pass on bits 15..0
 //         restricted to the selected bucket.
-// The pass that builds the histogram also keeps each row's max |a|, so the
-// quantize pass knows amax_i = min(rowmax_i, T) without another reduction, and
-// its last CTA to finish selects the bin (no separate launch).
+// The pass that finds T also keeps each row's max |a|, so the quantize pass
+// knows amax_i = min(rowmax_i, T) without another reduction.
 //
-// dA is emitted in canonical CSR order without sorting and without global
-// atomics in the common case: one warp owns a row and walks it in column
-// order, so each outlier knows its rank within the row; rank < row_slots goes
-// to the row's own staging region, later ones to an overflow list.  The last
-// CTA of the clamp pass scans the row counts into row_ptr; a scatter kernel
-// then moves entry (row, rank) to row_ptr[row] + rank.
+// dA is emitted in canonical CSR order without sorting: one warp owns a row
+// and walks it in column order, so each outlier knows its rank within the
+// row; rank < row_slots goes to the row's own staging region, later ones to
+// an overflow list.  The row counts are scanned into row_ptr and a scatter
+// moves entry (row, rank) to row_ptr[row] + rank.
+//
+// bf16 quantize_act runs as one cooperative kernel (act_fused_bf16_kernel,
+// phases separated by bounded grid barriers); fp32 input, clamp_compensate
+// and devices without cooperative launch use the multi-kernel sequence.
 #include "qg_internal.cuh"
 
 namespace qg {

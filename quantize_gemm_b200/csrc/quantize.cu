@@ -6,7 +6,9 @@
 // columns of W) and ScaleShift paragraph (scale by 6 / amax, round to the
 // nearest E2M1 value; ties to the even code).
 //
-// All kernels are HBM-bound streaming passes with 16-byte loads.
+// Streaming passes with 16-byte loads: the bf16 row quantizer holds a row in
+// registers (a warp per row); the bf16 column quantizer is one cooperative
+// kernel (partial column maxima, a grid barrier, then 32 x 256 tiles).
 #include "qg_internal.cuh"
 
 namespace qg {

@@ -116,8 +116,9 @@ spmm_slice_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restrict
 
 // --------------------------------------------------------------------------
 // Fast path (bf16 W, N and ldw multiples of 8).  The kernel is bound by
-// instruction issue, so the work per non-zero is made as wide and as lean as
-// possible: a CTA owns a 1024-column slice (each lane 32 columns, in four
+// instruction issue and L2 bandwidth at large shapes and by the latency of the
+// W-row reads at small ones, so the work per non-zero is made as wide and as
+// lean as possible and each warp keeps several rows' segments in flight: a CTA owns a 1024-column slice (each lane 32 columns, in four
 // 256-column quarters so every load and store is coalesced), W row segments
 // go straight from L2 into a register ring kDepth entries deep (the ring
 // position is a compile-time index: the entry loop is unrolled by kDepth),
