@@ -19,6 +19,11 @@ write-up of "Optimizing Large Language Model Training Using FP4 Quantization"
   for A, channel-wise for W) with the ScaleShift calibration.
 * ``gemm_acc`` / ``linear_y`` / ``spmm``: Y = acc * s_i * t_j + dA * W, the
   layer output in double.
+* ``dgrad`` / ``wgrad``: the gradient GEMMs with FP4 operands (the write-up's
+  paragraphs on the FP4 GEMM and on the differentiable gradient estimator say
+  the training runs its matrix products in FP4; how gradients are quantized
+  is not stated).  Reading: each operand is quantized with the forward's
+  rule along the contraction dimension, one scale per outer index, no clamp.
 
 Pins: every function here is checked in ``tests/test_oracle_pins.py``
 against values fixed by the pages or the mathematics (worked examples,
@@ -287,3 +292,37 @@ def dequant_rows(codes, scales) -> np.ndarray:
     q[:, 0::2] = lo
     q[:, 1::2] = hi
     return q * np.asarray(scales, dtype=np.float64)[:, None]
+
+
+# -- gradient GEMMs -------------------------------------------------------------------
+def scaled_product(acc, s_rows, s_cols) -> np.ndarray:
+    """acc[i, j] * s_rows[i] * s_cols[j] in double."""
+    return (np.asarray(acc, dtype=np.float64)
+            * np.asarray(s_rows, dtype=np.float32).astype(np.float64)[:, None]
+            * np.asarray(s_cols, dtype=np.float32).astype(np.float64)[None, :])
+
+
+def dgrad(dY, W, rows=None) -> np.ndarray:
+    """dA = Q(dY) Q(W)^T (double) for the listed rows of dA (None: all).
+
+    dY is M x N and W the forward weight, K x N; both are quantized per row,
+    i.e. along N, the contraction dimension; dA is M x K.
+    """
+    cd, sd = quantize_rows(dY)
+    cw, sw = quantize_rows(W)
+    N = 2 * cd.shape[1]
+    acc = gemm_acc(cd, cw, N, rows)
+    return scaled_product(acc, sd if rows is None else sd[np.asarray(rows)], sw)
+
+
+def wgrad(A, dY, rows=None) -> np.ndarray:
+    """dW = Q(A)^T Q(dY) (double) for the listed rows of dW (None: all).
+
+    A is M x K and dY is M x N; both are quantized per column, i.e. along the
+    M tokens, the contraction dimension; dW is K x N.
+    """
+    ca, sa = quantize_cols(A)
+    cd, sd = quantize_cols(dY)
+    M = 2 * ca.shape[1]
+    acc = gemm_acc(ca, cd, M, rows)
+    return scaled_product(acc, sa if rows is None else sa[np.asarray(rows)], sd)

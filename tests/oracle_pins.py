@@ -390,6 +390,67 @@ def pin_quantize_act_composition(orc, seed=11):
     assert np.array_equal(out["scales"], (amax / np.float32(6)).astype(np.float32))
 
 
+def pin_dgrad_exact_on_grid(orc, seed=12):
+    """dY rows and W rows on their own scaled grids (spread exponents): the
+    quantization along N is exact, so dA == dY @ W^T exactly.  Quantizing
+    along the wrong dimension, a transposed operand or a lost scale breaks it
+    (M, N, K all differ)."""
+    rng = np.random.default_rng(seed)
+    M, N, K = 12, 64, 20
+    dY, *_ = _on_grid_matrix(rng, M, N, rng.integers(-4, 5, size=M).astype(np.float64))
+    W, *_ = _on_grid_matrix(rng, K, N, rng.integers(-9, -1, size=K).astype(np.float64))
+    exact = dY.astype(np.float64) @ W.astype(np.float64).T
+    got = orc.dgrad(dY, W)
+    assert got.shape == (M, K) and np.array_equal(got, exact)
+    rows = [11, 0, 5]
+    assert np.array_equal(orc.dgrad(dY, W, rows=rows), exact[rows])
+
+
+def pin_wgrad_exact_on_grid(orc, seed=13):
+    """A columns and dY columns on their own scaled grids: the quantization
+    along the M tokens is exact, so dW == A^T @ dY exactly."""
+    rng = np.random.default_rng(seed)
+    M, K, N = 64, 18, 26
+    AT, *_ = _on_grid_matrix(rng, K, M, rng.integers(-5, 4, size=K).astype(np.float64))
+    dYT, *_ = _on_grid_matrix(rng, N, M, rng.integers(-12, -3, size=N).astype(np.float64))
+    A, dY = np.ascontiguousarray(AT.T), np.ascontiguousarray(dYT.T)
+    exact = A.astype(np.float64).T @ dY.astype(np.float64)
+    got = orc.wgrad(A, dY)
+    assert got.shape == (K, N) and np.array_equal(got, exact)
+    rows = [17, 3]
+    assert np.array_equal(orc.wgrad(A, dY, rows=rows), exact[rows])
+
+
+def pin_grads_within_rounding_bound(orc, seed=14):
+    """Off-grid inputs: |Q(x) - x| <= s for every element (the widest grid
+    gap, 4 to 6, is 2 in units of s), so each gradient lies within
+    sum(s_x |y| + |x| s_y + s_x s_y) of the exact product."""
+    rng = np.random.default_rng(seed)
+    M, K, N = 96, 40, 32
+    A = rng.standard_t(4, size=(M, K)).astype(np.float32)
+    W = (rng.standard_normal((K, N)) * 0.05).astype(np.float32)
+    dY = (rng.standard_normal((M, N)) * 1e-3).astype(np.float32)
+    a64, w64, d64 = (x.astype(np.float64) for x in (A, W, dY))
+    # dgrad: scales per row of dY and per row of W (along N)
+    sd = np.abs(d64).max(axis=1) / 6
+    sw = np.abs(w64).max(axis=1) / 6
+    bound = (sd[:, None] * (np.abs(w64).sum(axis=1))[None, :]
+             + (np.abs(d64).sum(axis=1))[:, None] * sw[None, :]
+             + N * sd[:, None] * sw[None, :])
+    got = orc.dgrad(dY, W)
+    err = np.abs(got - d64 @ w64.T)
+    assert np.all(err <= bound * (1 + 1e-6)) and err.max() > 0
+    # wgrad: scales per column of A and per column of dY (along M)
+    sa = np.abs(a64).max(axis=0) / 6
+    sy = np.abs(d64).max(axis=0) / 6
+    bound = (sa[:, None] * (np.abs(d64).sum(axis=0))[None, :]
+             + (np.abs(a64).sum(axis=0))[:, None] * sy[None, :]
+             + M * sa[:, None] * sy[None, :])
+    got = orc.wgrad(A, dY)
+    err = np.abs(got - a64.T @ d64)
+    assert np.all(err <= bound * (1 + 1e-6)) and err.max() > 0
+
+
 ALL_PINS = [
     pin_grid, pin_encoder_ties, pin_encoder_nearest_search, pin_row_worked_example,
     pin_col_worked_example, pin_threshold_worked_example, pin_act_worked_example,
@@ -397,5 +458,6 @@ ALL_PINS = [
     pin_quantize_rows_identity, pin_quantize_rows_properties, pin_quantize_degenerate_rows,
     pin_quantize_cols_transpose, pin_gemm_vs_integer_matmul, pin_spmm_vs_scipy,
     pin_linear_no_clamp_is_dequant_matmul, pin_linear_exact_on_grid,
-    pin_quantize_act_composition,
+    pin_quantize_act_composition, pin_dgrad_exact_on_grid, pin_wgrad_exact_on_grid,
+    pin_grads_within_rounding_bound,
 ]

@@ -3,7 +3,6 @@ catch every one of them.  The copies are built in a temporary directory on the
 CPU; the oracle in the repository is never modified."""
 import importlib.util
 import os
-import shutil
 import sys
 
 import pytest
@@ -45,13 +44,15 @@ MUTANTS = [
 ]
 
 
-def _build_variant(tmp_path, name, find, repl):
-    src = open(os.path.join(ORACLE_DIR, "qg_oracle.c")).read()
-    assert src.count(find) >= 1, f"mutation anchor not found: {name}"
+def _build_variant(tmp_path, name, find, repl, target="qg_oracle.c"):
     pkg = tmp_path / f"orc_{name}"
     pkg.mkdir()
-    (pkg / "qg_oracle.c").write_text(src.replace(find, repl, 1))
-    shutil.copy(os.path.join(ORACLE_DIR, "__init__.py"), pkg / "__init__.py")
+    for fname in ("qg_oracle.c", "__init__.py"):
+        src = open(os.path.join(ORACLE_DIR, fname)).read()
+        if fname == target:
+            assert src.count(find) >= 1, f"mutation anchor not found: {name}"
+            src = src.replace(find, repl, 1)
+        (pkg / fname).write_text(src)
     modname = f"orc_mutant_{name}"
     spec = importlib.util.spec_from_file_location(modname, pkg / "__init__.py",
                                                   submodule_search_locations=[str(pkg)])
@@ -61,9 +62,24 @@ def _build_variant(tmp_path, name, find, repl):
     return mod
 
 
-@pytest.mark.parametrize("name,find,repl", MUTANTS, ids=[m[0] for m in MUTANTS])
-def test_planted_mistake_is_caught(tmp_path, name, find, repl):
-    mod = _build_variant(tmp_path, name, find, repl)
+# the same, planted in the Python compositions of the gradient GEMMs
+PY_MUTANTS = [
+    ("dgrad_row_scale_dropped", "return scaled_product(acc, sd if rows is None",
+     "return scaled_product(acc, 1.0 + 0 * sd if rows is None"),
+    ("dgrad_weight_scale_of_dy", "cw, sw = quantize_rows(W)",
+     "cw, sw = quantize_rows(W)\n    sw = sw * 0 + sd.max()"),
+    ("wgrad_contraction_halved", "M = 2 * ca.shape[1]", "M = ca.shape[1]"),
+    ("wgrad_dy_per_row", "cd, sd = quantize_cols(dY)",
+     "cd, sd = quantize_cols(dY)\n    sd = sd * 0 + quantize_rows(dY)[1].max()"),
+]
+
+
+@pytest.mark.parametrize("name,find,repl,target",
+                         [m + ("qg_oracle.c",) for m in MUTANTS]
+                         + [m + ("__init__.py",) for m in PY_MUTANTS],
+                         ids=[m[0] for m in MUTANTS + PY_MUTANTS])
+def test_planted_mistake_is_caught(tmp_path, name, find, repl, target):
+    mod = _build_variant(tmp_path, name, find, repl, target)
     caught = []
     for pin in oracle_pins.ALL_PINS:
         try:
