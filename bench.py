@@ -544,6 +544,82 @@ def quantizer_sweep(device, reps=20, warm=5):
         print(json.dumps(line), flush=True)
 
 
+def grads_sweep(device, workload, reps=20, warm=5):
+    """Forward layer, dgrad and wgrad of every linear of a workload, each
+    timed alone (median of `reps` CUDA-event timings, L2 flushed before each),
+    with the FP4 GEMM of the same shape timed on its own beside it.  One JSON
+    line per linear; TFLOP/s counts 2*M*K*N per product."""
+    import quantize_gemm_b200 as qg
+    from workloads import WORKLOADS, make_layer_inputs, make_matrix
+    peaks = _peaks()
+    fp4_peak = 4.0 * peaks["bf16_tflops_sustained"]
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    wl = WORKLOADS[workload]
+
+    def timed(fn):
+        for _ in range(warm):
+            fn()
+        ts = []
+        for _ in range(reps):
+            flush.fill_(1)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        ts.sort()
+        return ts[len(ts) // 2]
+
+    for li, layer in enumerate(wl.layers):
+        A, W = make_layer_inputs(wl, li, device=device)
+        M, K = A.shape
+        N = W.shape[1]
+        dY = make_matrix((M, N), seed=9000 + li, device=device, dtype=A.dtype, scale=1e-3)
+        alpha = wl.alphas[0]
+        codesT, t = qg.quantize_cols(W)
+        ws_f = qg.Workspace(qg.QG_OP_FP4_LINEAR, M, K, N, qg._dt(A), alpha, device=device)
+        Y = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+        t_fwd = timed(lambda: qg.qg_fp4_linear(A, codesT, t, W, alpha, Y, ws_f))
+        qg.check_status(ws_f, "grads forward")
+        del ws_f, Y
+        ws_d = qg.Workspace(qg.QG_OP_FP4_DGRAD, M, K, N, qg.QG_F32, device=device)
+        dA = torch.empty((M, K), dtype=torch.bfloat16, device=device)
+        t_dgrad = timed(lambda: qg.qg_fp4_dgrad(dY, W, dA, ws_d))
+        qg.check_status(ws_d, "grads dgrad")
+        del ws_d, dA
+        ws_w = qg.Workspace(qg.QG_OP_FP4_WGRAD, M, K, N, qg.QG_F32, device=device)
+        dW = torch.empty((K, N), dtype=torch.bfloat16, device=device)
+        t_wgrad = timed(lambda: qg.qg_fp4_wgrad(A, dY, dW, ws_w))
+        qg.check_status(ws_w, "grads wgrad")
+        del ws_w, dW
+        # the GEMMs alone on codes of the same shapes
+        gemm_ms = {}
+        for name, (m, n, k) in (("dgrad", (M, K, N)), ("wgrad", (K, N, M))):
+            cA = torch.randint(0, 256, (m, k // 2), dtype=torch.uint8, device=device)
+            cB = torch.randint(0, 256, (n, k // 2), dtype=torch.uint8, device=device)
+            sa = torch.full((m,), 1e-3, device=device)
+            sb = torch.full((n,), 1e-3, device=device)
+            out = torch.empty((m, n), dtype=torch.bfloat16, device=device)
+            ws_g = qg.Workspace(qg.QG_OP_FP4_GEMM, m, k, n, qg.QG_F32, device=device)
+            gemm_ms[name] = timed(lambda: qg.qg_fp4_gemm(cA, sa, cB, sb, m, n, k, None, out, None,
+                                                         ws_g))
+            qg.check_status(ws_g, "grads gemm")
+            del cA, cB, out, ws_g
+        torch.cuda.empty_cache()
+        fl = 2.0 * M * K * N
+        line = {"sweep": "grads", "workload": wl.name, "layer": layer.name, "M": M, "K": K,
+                "N": N, "dtype": wl.dtype, "out": "bf16", "l2": "flushed before each rep",
+                "reps": reps, "fp4_peak_tflops": fp4_peak}
+        for k, tm in (("forward", t_fwd), ("dgrad", t_dgrad), ("wgrad", t_wgrad),
+                      ("dgrad_gemm_only", gemm_ms["dgrad"]), ("wgrad_gemm_only", gemm_ms["wgrad"])):
+            tf = fl / (tm * 1e-3) / 1e12
+            line[k] = {"ms": round(tm, 4), "TFLOP/s": round(tf, 1),
+                       "frac_measured": round(tf / fp4_peak, 4)}
+        print(json.dumps(line), flush=True)
+        del A, W, dY, codesT, t
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -560,6 +636,9 @@ def main():
     ap.add_argument("--quantizer-sweep", action="store_true",
                     help="time the three quantizers over 1M..256M bf16 elements (one JSON line "
                          "per size) instead of the layer stream")
+    ap.add_argument("--grads", action="store_true",
+                    help="time forward, dgrad and wgrad of each linear of --workload (one JSON "
+                         "line per linear) instead of the layer stream")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3
@@ -584,9 +663,12 @@ def main():
     import __graft_entry__
     if rank == 0:
         __graft_entry__.build()
-    if args.quantizer_sweep:
+    if args.quantizer_sweep or args.grads:
         if rank == 0:
-            quantizer_sweep(device)
+            if args.quantizer_sweep:
+                quantizer_sweep(device)
+            else:
+                grads_sweep(device, args.workload)
         return
     if world > 1:
         torch.distributed.barrier()

@@ -96,7 +96,9 @@ typedef enum {
     QG_OP_QUANTIZE_ACT = 3,
     QG_OP_SPMM = 4,
     QG_OP_FP4_GEMM = 5,
-    QG_OP_FP4_LINEAR = 6
+    QG_OP_FP4_LINEAR = 6,
+    QG_OP_FP4_DGRAD = 7,    /* sized with (M, K, N) of the forward layer */
+    QG_OP_FP4_WGRAD = 8     /* sized with (M, K, N) of the forward layer */
 } qg_op;
 
 const char* qg_status_string(qg_status s);
@@ -211,6 +213,32 @@ qg_status qg_fp4_linear(const void* A, qg_dtype dtype, int64_t M, int64_t K,
                         const uint8_t* codesWT, const float* sW, const void* W, int64_t N,
                         double alpha, void* Y, qg_dtype y_dtype, void* ws, size_t ws_bytes,
                         cudaStream_t stream);
+
+/* Backward GEMMs of the layer with FP4 operands (the training method also
+ * runs the gradient GEMMs in FP4: [FP4-writeup], the paragraphs on the FP4
+ * GEMM and on the differentiable gradient estimator).  The pages do not state
+ * how gradients are quantized; the reading used here is the forward's rule:
+ * each operand is quantized along the contraction dimension with one fp32
+ * scale per outer index (ScaleShift, E2M1, ties to the even code), no clamp.
+ *
+ * dgrad: dA (M x K) = sum over n of Q(dY)[m, n] * Q(W)[k, n], with dY (M x N)
+ *   quantized per row m and W (K x N, the forward weight) per row k; the
+ *   contraction is over N, so N % 32 == 0 and N <= 16384.
+ * wgrad: dW (K x N) = sum over m of Q(A)[m, k] * Q(dY)[m, n], with A (M x K)
+ *   quantized per column k and dY per column n; the contraction is over the
+ *   M tokens, so M % 32 == 0 and M <= 16384.
+ * All matrices row-major and contiguous (16-byte aligned); output fp32 or
+ * bf16 (out_dtype).  The codes and scales of both operands live in the
+ * workspace (qg_workspace_size(QG_OP_FP4_DGRAD / QG_OP_FP4_WGRAD, M, K, N,
+ * any dtype, 1.0); the size does not depend on the dtype).  Errors: as
+ * qg_fp4_gemm, plus QG_ERR_UNSUPPORTED_SHAPE when the contraction dimension
+ * breaks the rule above. */
+qg_status qg_fp4_dgrad(const void* dY, qg_dtype dy_dtype, int64_t M, int64_t N, const void* W,
+                       qg_dtype w_dtype, int64_t K, void* dA, qg_dtype out_dtype, void* ws,
+                       size_t ws_bytes, cudaStream_t stream);
+qg_status qg_fp4_wgrad(const void* A, qg_dtype a_dtype, int64_t M, int64_t K, const void* dY,
+                       qg_dtype dy_dtype, int64_t N, void* dW, qg_dtype out_dtype, void* ws,
+                       size_t ws_bytes, cudaStream_t stream);
 
 #ifdef __cplusplus
 }

@@ -32,7 +32,7 @@ QG_F32, QG_BF16 = 0, 1
 QG_OK, QG_ERR_INVALID_ARG, QG_ERR_UNSUPPORTED_SHAPE, QG_ERR_WORKSPACE, QG_ERR_CUDA, \
     QG_ERR_NONFINITE, QG_ERR_TIMEOUT, QG_ERR_INTERNAL = range(8)
 (QG_OP_QUANTIZE_ROWS, QG_OP_QUANTIZE_COLS, QG_OP_CLAMP_COMPENSATE, QG_OP_QUANTIZE_ACT,
- QG_OP_SPMM, QG_OP_FP4_GEMM, QG_OP_FP4_LINEAR) = range(7)
+ QG_OP_SPMM, QG_OP_FP4_GEMM, QG_OP_FP4_LINEAR, QG_OP_FP4_DGRAD, QG_OP_FP4_WGRAD) = range(9)
 
 # every symbol the header declares (checked by the CPU tests)
 EXPORTED = (
@@ -40,7 +40,7 @@ EXPORTED = (
     "qg_workspace_size", "qg_workspace_init", "qg_sync_status", "qg_e2m1_encode",
     "qg_quantize_rows", "qg_quantize_cols", "qg_clamp_compensate", "qg_quantize_act",
     "qg_spmm_correction", "qg_fp4_gemm", "qg_fp4_linear", "qg_launch_count",
-    "qg_quantize_cols_static",
+    "qg_quantize_cols_static", "qg_fp4_dgrad", "qg_fp4_wgrad",
 )
 
 
@@ -86,6 +86,8 @@ _sig("qg_fp4_gemm", _INT,
      [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _INT, _P, _P, _SZ, _P])
 _sig("qg_fp4_linear", _INT,
      [_P, _INT, _I64, _I64, _P, _P, _P, _I64, _D, _P, _INT, _P, _SZ, _P])
+_sig("qg_fp4_dgrad", _INT, [_P, _INT, _I64, _I64, _P, _INT, _I64, _P, _INT, _P, _SZ, _P])
+_sig("qg_fp4_wgrad", _INT, [_P, _INT, _I64, _I64, _P, _INT, _I64, _P, _INT, _P, _SZ, _P])
 
 
 class QGError(RuntimeError):
@@ -260,6 +262,28 @@ def qg_fp4_linear(A, codesWT, sW, W, alpha, Y, ws: Workspace, stream=None) -> in
                               float(alpha), _ptr(Y), _dt(Y), ws.ptr, ws.nbytes, _stream(stream))
 
 
+def _contig(*ts):
+    for t in ts:
+        if not t.is_contiguous():
+            raise ValueError("the backward entry points take row-major contiguous matrices")
+
+
+def qg_fp4_dgrad(dY, W, dA, ws: Workspace, stream=None) -> int:
+    _contig(dY, W, dA)
+    M, N = dY.shape
+    K = W.shape[0]
+    return _lib.qg_fp4_dgrad(_ptr(dY), _dt(dY), M, N, _ptr(W), _dt(W), K, _ptr(dA), _dt(dA),
+                             ws.ptr, ws.nbytes, _stream(stream))
+
+
+def qg_fp4_wgrad(A, dY, dW, ws: Workspace, stream=None) -> int:
+    _contig(A, dY, dW)
+    M, K = A.shape
+    N = dY.shape[1]
+    return _lib.qg_fp4_wgrad(_ptr(A), _dt(A), M, K, _ptr(dY), _dt(dY), N, _ptr(dW), _dt(dW),
+                             ws.ptr, ws.nbytes, _stream(stream))
+
+
 # ----------------------------------------------------------- allocating helpers
 def e2m1_encode(x: torch.Tensor, ws: Optional[Workspace] = None) -> torch.Tensor:
     ws = ws or Workspace(QG_OP_QUANTIZE_ROWS, 1, 32, device=x.device)
@@ -334,6 +358,26 @@ def fp4_linear(A, codesWT, sW, W, alpha: float, out_dtype=torch.float32,
     Y = torch.empty((M, N), dtype=out_dtype, device=A.device)
     _check(qg_fp4_linear(A, codesWT, sW, W, alpha, Y, ws), "qg_fp4_linear")
     return Y
+
+
+def fp4_dgrad(dY, W, out_dtype=torch.float32, ws: Optional[Workspace] = None):
+    """dA = Q(dY) Q(W)^T with dY (M x N) and W (K x N) quantized along N."""
+    M, N = dY.shape
+    K = W.shape[0]
+    ws = ws or Workspace(QG_OP_FP4_DGRAD, M, K, N, QG_F32, device=dY.device)
+    dA = torch.empty((M, K), dtype=out_dtype, device=dY.device)
+    _check(qg_fp4_dgrad(dY, W, dA, ws), "qg_fp4_dgrad")
+    return dA
+
+
+def fp4_wgrad(A, dY, out_dtype=torch.float32, ws: Optional[Workspace] = None):
+    """dW = Q(A)^T Q(dY) with A (M x K) and dY (M x N) quantized along the M tokens."""
+    M, K = A.shape
+    N = dY.shape[1]
+    ws = ws or Workspace(QG_OP_FP4_WGRAD, M, K, N, QG_F32, device=A.device)
+    dW = torch.empty((K, N), dtype=out_dtype, device=A.device)
+    _check(qg_fp4_wgrad(A, dY, dW, ws), "qg_fp4_wgrad")
+    return dW
 
 
 def check_status(ws: Workspace, where: str = "device status", stream=None):

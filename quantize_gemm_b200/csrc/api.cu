@@ -336,4 +336,68 @@ qg_status qg_fp4_linear(const void* A, qg_dtype dtype, int64_t M, int64_t K,
                                        at<uint32_t>(ws, L.status), stream));
 }
 
+// Column quantization of a whole row-major matrix X (rows x cols) into
+// codesT (cols x rows/2) + scales (cols): the cooperative bf16 kernel or the
+// multi-kernel sequence (colmax: 32 * cols words of scratch).
+static cudaError_t quantize_cols_any(const void* X, qg_dtype dt, int64_t rows, int64_t cols,
+                                     uint8_t* codesT, float* scales, uint32_t* colmax, void* ws,
+                                     const WsLayout& L, cudaStream_t stream) {
+    if (dt == QG_BF16 &&
+        launch_quantize_cols_fused(X, rows, cols, cols, codesT, scales, colmax,
+                                   at<GridSync>(ws, L.gsync), at<uint32_t>(ws, L.status), stream))
+        return cudaGetLastError();
+    launch_quantize_cols(X, dt, rows, cols, cols, codesT, scales, colmax, stream);
+    return cudaGetLastError();
+}
+
+qg_status qg_fp4_dgrad(const void* dY, qg_dtype dy_dtype, int64_t M, int64_t N, const void* W,
+                       qg_dtype w_dtype, int64_t K, void* dA, qg_dtype out_dtype, void* ws,
+                       size_t ws_bytes, cudaStream_t stream) {
+    if (!dtype_ok(dy_dtype) || !dtype_ok(w_dtype) || !dtype_ok(out_dtype)) return QG_ERR_INVALID_ARG;
+    qg_status st = check_mk(M, N);              // contraction over N
+    if (st != QG_OK) return st;
+    if ((st = check_mk(K, N)) != QG_OK) return st;
+    if ((st = check_ld(dY, dy_dtype, N, N)) != QG_OK) return st;
+    if ((st = check_ld(W, w_dtype, N, N)) != QG_OK) return st;
+    if (dA == nullptr || !aligned16(dA)) return QG_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(QG_OP_FP4_DGRAD, M, K, N, QG_F32, 1.0);
+    if ((st = check_ws(ws, ws_bytes, L.total)) != QG_OK) return st;
+    if (ensure_device(nullptr) != cudaSuccess) return QG_ERR_CUDA;
+    uint8_t* ca = at<uint8_t>(ws, L.g_codes_a);
+    float* sa = at<float>(ws, L.g_scales_a);
+    uint8_t* cb = at<uint8_t>(ws, L.g_codes_b);
+    float* sb = at<float>(ws, L.g_scales_b);
+    launch_quantize_rows(dY, dy_dtype, M, N, N, ca, sa, stream);
+    launch_quantize_rows(W, w_dtype, K, N, N, cb, sb, stream);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return QG_ERR_CUDA;
+    return cuda_status(launch_fp4_gemm(ca, sa, cb, sb, M, K, N, nullptr, dA, out_dtype, nullptr,
+                                       at<uint32_t>(ws, L.status), stream));
+}
+
+qg_status qg_fp4_wgrad(const void* A, qg_dtype a_dtype, int64_t M, int64_t K, const void* dY,
+                       qg_dtype dy_dtype, int64_t N, void* dW, qg_dtype out_dtype, void* ws,
+                       size_t ws_bytes, cudaStream_t stream) {
+    if (!dtype_ok(a_dtype) || !dtype_ok(dy_dtype) || !dtype_ok(out_dtype)) return QG_ERR_INVALID_ARG;
+    qg_status st = check_mk(K, M);              // contraction over the M tokens
+    if (st != QG_OK) return st;
+    if ((st = check_mk(N, M)) != QG_OK) return st;
+    if (A == nullptr || dY == nullptr || !aligned16(A) || !aligned16(dY)) return QG_ERR_INVALID_ARG;
+    if (dW == nullptr || !aligned16(dW)) return QG_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(QG_OP_FP4_WGRAD, M, K, N, QG_F32, 1.0);
+    if ((st = check_ws(ws, ws_bytes, L.total)) != QG_OK) return st;
+    if (ensure_device(nullptr) != cudaSuccess) return QG_ERR_CUDA;
+    uint8_t* ca = at<uint8_t>(ws, L.g_codes_a);
+    float* sa = at<float>(ws, L.g_scales_a);
+    uint8_t* cb = at<uint8_t>(ws, L.g_codes_b);
+    float* sb = at<float>(ws, L.g_scales_b);
+    uint32_t* colmax = at<uint32_t>(ws, L.colmax);
+    cudaError_t e = quantize_cols_any(A, a_dtype, M, K, ca, sa, colmax, ws, L, stream);
+    if (e != cudaSuccess) return QG_ERR_CUDA;
+    e = quantize_cols_any(dY, dy_dtype, M, N, cb, sb, colmax, ws, L, stream);
+    if (e != cudaSuccess) return QG_ERR_CUDA;
+    return cuda_status(launch_fp4_gemm(ca, sa, cb, sb, K, N, M, nullptr, dW, out_dtype, nullptr,
+                                       at<uint32_t>(ws, L.status), stream));
+}
+
 }  // extern "C"

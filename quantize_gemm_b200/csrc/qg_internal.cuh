@@ -73,6 +73,7 @@ constexpr size_t kGridSyncOffset = 16;   // bytes from the workspace base
 struct WsLayout {
     size_t gsync = 0;
     size_t rowpre = 0;
+    size_t g_codes_a = 0, g_scales_a = 0, g_codes_b = 0, g_scales_b = 0;
     size_t status = 0, counters = 0, hist1 = 0, hist2 = 0, rowmax = 0, rowcnt = 0;
     size_t st_row = 0, st_rank = 0, st_col = 0, st_val = 0, colmax = 0;
     size_t act_codes = 0, act_scales = 0, csr_row_ptr = 0, csr_col = 0, csr_val = 0,
@@ -122,6 +123,23 @@ inline WsLayout ws_layout(qg_op op, int64_t M, int64_t K, int64_t N, qg_dtype dt
     // column maxima: N words (fp32 path); the cooperative bf16 kernel keeps
     // per-split partial maxima, up to 32 splits
     if (op == QG_OP_QUANTIZE_COLS) L.colmax = take(sizeof(uint32_t) * 32 * (size_t)N);
+    // backward GEMMs (forward dims M, K, N): the two operands' codes + scales
+    //   dgrad: a = dY rows (M x N/2, M), b = W rows (K x N/2, K)
+    //   wgrad: a = A columns (K x M/2, K), b = dY columns (N x M/2, N), plus
+    //          the column quantizer's partial maxima
+    if (op == QG_OP_FP4_DGRAD) {
+        L.g_codes_a = take((size_t)M * (size_t)(N / 2));
+        L.g_scales_a = take(sizeof(float) * (size_t)M);
+        L.g_codes_b = take((size_t)K * (size_t)(N / 2));
+        L.g_scales_b = take(sizeof(float) * (size_t)K);
+    }
+    if (op == QG_OP_FP4_WGRAD) {
+        L.g_codes_a = take((size_t)K * (size_t)(M / 2));
+        L.g_scales_a = take(sizeof(float) * (size_t)K);
+        L.g_codes_b = take((size_t)N * (size_t)(M / 2));
+        L.g_scales_b = take(sizeof(float) * (size_t)N);
+        L.colmax = take(sizeof(uint32_t) * 32 * (size_t)(K > N ? K : N));
+    }
     if (op == QG_OP_FP4_LINEAR) {
         int64_t cap = L.cap > 0 ? L.cap : 1;
         L.act_codes = take((size_t)M * (size_t)(K / 2));

@@ -31,7 +31,7 @@ def test_header_declares_the_entry_points():
     funcs = _header_functions()
     for name in ("qg_quantize_rows", "qg_quantize_cols", "qg_clamp_compensate",
                  "qg_quantize_act", "qg_spmm_correction", "qg_fp4_gemm", "qg_fp4_linear",
-                 "qg_sync_status", "qg_workspace_size"):
+                 "qg_sync_status", "qg_workspace_size", "qg_fp4_dgrad", "qg_fp4_wgrad"):
         assert name in funcs
 
 
@@ -50,7 +50,7 @@ def test_rank_convention_matches_oracle(qg):
 
 
 def test_workspace_sizes(qg):
-    for op in range(7):
+    for op in range(9):
         for (M, K, N, dt, a) in ((1, 32, 1, 0, 1.0), (256, 512, 512, 0, 0.99),
                                  (4096, 2048, 5504, 1, 0.99), (16384, 11008, 4096, 1, 0.999)):
             s = qg.qg_workspace_size(op, M, K, N, dt, a)
@@ -107,3 +107,19 @@ def test_host_argument_checks_need_no_device(qg):
     # GEMM with neither Y nor raw_acc
     assert lib.qg_fp4_gemm(fake, fake, fake, fake, 128, 128, 256, None, None, 0, None, fake,
                            1 << 20, None) == qg.QG_ERR_INVALID_ARG
+    # gradient GEMMs: the contraction dimension (N for dgrad, M for wgrad)
+    # must be a multiple of 32 and at most 16384; the outer ones are free
+    big = 1 << 30
+    assert lib.qg_fp4_dgrad(fake, 1, 64, 48, fake, 1, 64, fake, 0, fake, big, None) == \
+        qg.QG_ERR_UNSUPPORTED_SHAPE
+    assert lib.qg_fp4_dgrad(fake, 1, 64, 16416, fake, 1, 64, fake, 0, fake, big, None) == \
+        qg.QG_ERR_UNSUPPORTED_SHAPE
+    assert lib.qg_fp4_wgrad(fake, 1, 48, 64, fake, 1, 64, fake, 0, fake, big, None) == \
+        qg.QG_ERR_UNSUPPORTED_SHAPE
+    assert lib.qg_fp4_wgrad(fake, 5, 64, 64, fake, 1, 64, fake, 0, fake, big, None) == \
+        qg.QG_ERR_INVALID_ARG
+    assert lib.qg_fp4_dgrad(fake, 1, 64, 64, fake, 1, 64, P((1 << 20) + 8), 0, fake, big,
+                            None) == qg.QG_ERR_INVALID_ARG
+    need = qg.qg_workspace_size(qg.QG_OP_FP4_WGRAD, 64, 64, 64, 1, 1.0)
+    assert lib.qg_fp4_wgrad(fake, 1, 64, 64, fake, 1, 64, fake, 0, fake, need - 256, None) == \
+        qg.QG_ERR_WORKSPACE

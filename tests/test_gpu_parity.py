@@ -413,3 +413,82 @@ def test_fp4_linear_full_size_sampled(qg, wl, layer):
     oT, ot = oracle.quantize_cols(W.cpu())
     assert np.array_equal(_np(codesT), oT) and np.array_equal(_np(t), ot)
     assert y_rel_err(_np(Y)[rows], Yo) <= 1e-3
+
+
+# ------------------------------------------------------------ gradient GEMMs
+GRAD_CASES = [  # (M, K, N, dtype): ragged outer sizes, warp-row and CTA-row quantizers
+    (256, 512, 512, torch.float32), (300, 600, 1056, torch.bfloat16),
+    (77, 1000, 4096, torch.bfloat16), (64, 200, 5504, torch.bfloat16),
+    (1024, 96, 160, torch.bfloat16), (32, 33, 32, torch.float32),
+]
+
+
+def _grad_inputs(M, K, N, dtype, seed):
+    A = make_matrix((M, K), ("student_t", 4), seed=seed, dtype=dtype)
+    W = make_matrix((K, N), seed=seed + 1, dtype=dtype, scale=0.02)
+    dY = make_matrix((M, N), seed=seed + 2, dtype=dtype, scale=1e-3)
+    return A, W, dY
+
+
+@pytest.mark.parametrize("M,K,N,dtype", GRAD_CASES)
+def test_fp4_dgrad(qg, M, K, N, dtype):
+    A, W, dY = _grad_inputs(M, K, N, dtype, seed=M + K)
+    # forward Y = A W (M x N); backward dA = dY W^T with W (K x N): contraction over N
+    ws = qg.Workspace(qg.QG_OP_FP4_DGRAD, M, K, N, qg.QG_F32)
+    dA = qg.fp4_dgrad(dY.cuda(), W.cuda(), ws=ws)
+    qg.check_status(ws)
+    assert dA.shape == (M, K)
+    Do = oracle.dgrad(dY, W)
+    assert y_rel_err(_np(dA), Do) <= 1e-3
+    dAb = qg.fp4_dgrad(dY.cuda(), W.cuda(), out_dtype=torch.bfloat16)
+    rms = np.sqrt(np.mean(Do ** 2))
+    assert np.all(np.abs(_np(dAb.float()).astype(np.float64) - Do) <= bf16_ulp(Do) + 1e-6 * rms)
+
+
+@pytest.mark.parametrize("M,K,N,dtype", GRAD_CASES)
+def test_fp4_wgrad(qg, M, K, N, dtype):
+    if M % 32:
+        pytest.skip("wgrad contracts over M")
+    A, W, dY = _grad_inputs(M, K, N, dtype, seed=M + N)
+    dW = qg.fp4_wgrad(A.cuda(), dY.cuda())
+    assert dW.shape == (K, N)
+    Wo = oracle.wgrad(A, dY)
+    assert y_rel_err(_np(dW), Wo) <= 1e-3
+    dWb = qg.fp4_wgrad(A.cuda(), dY.cuda(), out_dtype=torch.bfloat16)
+    rms = np.sqrt(np.mean(Wo ** 2))
+    assert np.all(np.abs(_np(dWb.float()).astype(np.float64) - Wo) <= bf16_ulp(Wo) + 1e-6 * rms)
+
+
+def test_fp4_grads_exact_on_grid(qg):
+    """Operands already on their scaled grids along the contraction dimension:
+    both gradients equal the exact products (fp32 output, power-of-two
+    scales, integer-valued accumulators)."""
+    from oracle_pins import _on_grid_matrix
+    g = np.random.default_rng(31)
+    M, K, N = 96, 72, 160
+    dY, *_ = _on_grid_matrix(g, M, N, g.integers(-4, 4, size=M).astype(np.float64))
+    W, *_ = _on_grid_matrix(g, K, N, g.integers(-8, -2, size=K).astype(np.float64))
+    dA = qg.fp4_dgrad(torch.from_numpy(dY).cuda(), torch.from_numpy(W).cuda())
+    assert np.array_equal(_np(dA).astype(np.float64), dY.astype(np.float64) @ W.astype(np.float64).T)
+    AT, *_ = _on_grid_matrix(g, K, M, g.integers(-3, 3, size=K).astype(np.float64))
+    dYT, *_ = _on_grid_matrix(g, N, M, g.integers(-9, -5, size=N).astype(np.float64))
+    A, dY2 = np.ascontiguousarray(AT.T), np.ascontiguousarray(dYT.T)
+    dW = qg.fp4_wgrad(torch.from_numpy(A).cuda(), torch.from_numpy(dY2).cuda())
+    assert np.array_equal(_np(dW).astype(np.float64), A.astype(np.float64).T @ dY2.astype(np.float64))
+
+
+@pytest.mark.parametrize("wl,layer", [("llama1.3b", 1), ("llama7b", 4)])
+def test_fp4_grads_full_size_sampled(qg, wl, layer):
+    """A layer of the benchmark workloads at full size: dgrad and wgrad on a
+    sample of output rows computed by the oracle one by one."""
+    A, W = make_layer_inputs(wl, layer, device="cuda")
+    M, K = A.shape
+    N = W.shape[1]
+    dY = make_matrix((M, N), seed=77, device="cuda", dtype=A.dtype, scale=1e-3)
+    dA = qg.fp4_dgrad(dY, W)
+    dW = qg.fp4_wgrad(A, dY)
+    g = np.random.default_rng(M + K + N)
+    rows = np.unique(np.concatenate([g.integers(0, M, 12), [0, M - 1]]))
+    assert y_rel_err(_np(dA)[rows], oracle.dgrad(dY.cpu(), W.cpu(), rows=rows)) <= 1e-3
+    rows = np.unique(np.concatenate([g.integers(0, K, 12), [0, K - 1]]))
+    assert y_rel_err(_np(dW)[rows], oracle.wgrad(A.cpu(), dY.cpu(), rows=rows)) <= 1e-3
