@@ -84,28 +84,38 @@ quantize_rows_kernel(const void* __restrict__ A, int64_t lda, int K,
     }
 }
 
-// bf16, K <= 4096: a warp per row, the whole row in registers (SPR steps of
-// 1024 columns, each lane four 16-byte chunks per step); the row's max by a
-// 16x2 max and a warp reduction, then one packed fp32x2 multiply and one
-// conversion per bf16 pair.  Warps walk rows grid-stride.
+// bf16, K <= 16384: G warps per row (G = 1, 2, 4), each holding its segment
+// of SPR steps of 1024 columns in registers (each lane four 16-byte chunks per
+// step); the row's max by a 16x2 max, a warp reduction and, for G > 1, a
+// shared-memory exchange between the row's warps; then one packed fp32x2
+// multiply and one conversion per bf16 pair.  Row groups walk the rows
+// grid-stride; the loop bound is uniform over the CTA, so every thread
+// reaches each barrier.
 constexpr int kRowWarpThreads = 256;
 
-template <int SPR>
+template <int SPR, int G>
 __global__ void __launch_bounds__(kRowWarpThreads, SPR >= 4 ? 2 : 3)
 quantize_rows_bf16_kernel(const uint16_t* __restrict__ A, int64_t lda, int M, int K,
                           uint8_t* __restrict__ codes, float* __restrict__ scales) {
-    const int lane = threadIdx.x & 31;
-    const int wpc = kRowWarpThreads / 32;
+    constexpr int wpc = kRowWarpThreads / 32;
+    constexpr int rpc = wpc / G;                 // rows per CTA per turn
+    __shared__ uint32_t part[2][wpc];
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int sub = warp % G, slot = warp / G;
     const int nchunks = K / 8;
-    for (int row = blockIdx.x * wpc + (threadIdx.x >> 5); row < M; row += gridDim.x * wpc) {
-        const uint4* src = reinterpret_cast<const uint4*>(A + (int64_t)row * lda);
+    const int c0 = sub * SPR * 128 + lane;       // this lane's first chunk
+    int turn = 0;
+    for (int row0 = blockIdx.x * rpc; row0 < M; row0 += gridDim.x * rpc, turn ^= 1) {
+        const int row = row0 + slot;
+        const bool active = row < M;
+        const uint4* src = reinterpret_cast<const uint4*>(A + (int64_t)(active ? row : 0) * lda);
         uint4 v[SPR][4];
 #pragma unroll
         for (int st = 0; st < SPR; ++st)
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                const int c = st * 128 + 32 * j + lane;
-                v[st][j] = (c < nchunks) ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
+                const int c = c0 + st * 128 + 32 * j;
+                v[st][j] = (active && c < nchunks) ? __ldg(src + c) : make_uint4(0u, 0u, 0u, 0u);
             }
         uint32_t m0 = 0, m1 = 0;
 #pragma unroll
@@ -116,16 +126,23 @@ quantize_rows_bf16_kernel(const uint16_t* __restrict__ A, int64_t lda, int M, in
                 m1 = max_u16x2(m1, max_u16x2(v[st][j].z & 0x7FFF7FFFu, v[st][j].w & 0x7FFF7FFFu));
             }
         const uint32_t mm = max_u16x2(m0, m1);
-        const uint32_t key = warp_max_u32(max(mm & 0xFFFFu, mm >> 16));
+        uint32_t key = warp_max_u32(max(mm & 0xFFFFu, mm >> 16));
+        if constexpr (G > 1) {
+            if (lane == 0) part[turn][warp] = key;
+            __syncthreads();
+#pragma unroll
+            for (int g = 0; g < G; ++g) key = max(key, part[turn][slot * G + g]);
+        }
+        if (!active) continue;
         float r, sc;
         scale_factors(__uint_as_float(key << 16), r, sc);
-        if (lane == 0) scales[row] = sc;
+        if (sub == 0 && lane == 0) scales[row] = sc;
         uint32_t* out = reinterpret_cast<uint32_t*>(codes + (int64_t)row * (K / 2));
 #pragma unroll
         for (int st = 0; st < SPR; ++st)
 #pragma unroll
             for (int j = 0; j < 4; ++j) {
-                const int c = st * 128 + 32 * j + lane;
+                const int c = c0 + st * 128 + 32 * j;
                 if (c < nchunks) {
                     const uint32_t q01 = __byte_perm(bf16x2_encode(v[st][j].x, r), bf16x2_encode(v[st][j].y, r), 0x0040);
                     const uint32_t q23 = __byte_perm(bf16x2_encode(v[st][j].z, r), bf16x2_encode(v[st][j].w, r), 0x0040);
@@ -133,6 +150,16 @@ quantize_rows_bf16_kernel(const uint16_t* __restrict__ A, int64_t lda, int M, in
                 }
             }
     }
+}
+
+template <int SPR, int G>
+static void launch_rows_bf16(const uint16_t* A, int64_t M, int64_t K, int64_t lda, uint8_t* codes,
+                             float* scales, cudaStream_t s) {
+    constexpr int rpc = kRowWarpThreads / 32 / G;
+    const int grid = (int)std::max<int64_t>(
+        1, std::min<int64_t>((M + rpc - 1) / rpc, (int64_t)num_sms() * (SPR >= 4 ? 2 : 3)));
+    quantize_rows_bf16_kernel<SPR, G><<<grid, kRowWarpThreads, 0, s>>>(A, lda, (int)M, (int)K, codes,
+                                                                      scales);
 }
 
 template <qg_dtype DT>
@@ -150,16 +177,18 @@ static void launch_rows_dt(const void* A, int64_t M, int64_t K, int64_t lda, uin
 
 void launch_quantize_rows(const void* A, qg_dtype dt, int64_t M, int64_t K, int64_t lda,
                           uint8_t* codes, float* scales, cudaStream_t s) {
-    if (dt == QG_BF16 && K <= 4096) {
-        const int wpc = kRowWarpThreads / 32;
-        const int spr = (int)((K / 8 + 127) / 128);
-        const int grid = (int)std::max<int64_t>(
-            1, std::min<int64_t>((M + wpc - 1) / wpc, (int64_t)num_sms() * (spr >= 4 ? 2 : 3)));
+    if (dt == QG_BF16 && K <= 16384) {
+        // steps of 1024 columns; G warps per row, SPR steps per warp
+        const int steps = (int)((K / 8 + 127) / 128);
         const uint16_t* Ab = static_cast<const uint16_t*>(A);
-        if (spr <= 1) quantize_rows_bf16_kernel<1><<<grid, kRowWarpThreads, 0, s>>>(Ab, lda, (int)M, (int)K, codes, scales);
-        else if (spr == 2) quantize_rows_bf16_kernel<2><<<grid, kRowWarpThreads, 0, s>>>(Ab, lda, (int)M, (int)K, codes, scales);
-        else if (spr == 3) quantize_rows_bf16_kernel<3><<<grid, kRowWarpThreads, 0, s>>>(Ab, lda, (int)M, (int)K, codes, scales);
-        else quantize_rows_bf16_kernel<4><<<grid, kRowWarpThreads, 0, s>>>(Ab, lda, (int)M, (int)K, codes, scales);
+        if (steps <= 1) launch_rows_bf16<1, 1>(Ab, M, K, lda, codes, scales, s);
+        else if (steps == 2) launch_rows_bf16<2, 1>(Ab, M, K, lda, codes, scales, s);
+        else if (steps == 3) launch_rows_bf16<3, 1>(Ab, M, K, lda, codes, scales, s);
+        else if (steps == 4) launch_rows_bf16<4, 1>(Ab, M, K, lda, codes, scales, s);
+        else if (steps <= 6) launch_rows_bf16<3, 2>(Ab, M, K, lda, codes, scales, s);
+        else if (steps <= 8) launch_rows_bf16<4, 2>(Ab, M, K, lda, codes, scales, s);
+        else if (steps <= 12) launch_rows_bf16<3, 4>(Ab, M, K, lda, codes, scales, s);
+        else launch_rows_bf16<4, 4>(Ab, M, K, lda, codes, scales, s);
         count_launch(1);
         return;
     }

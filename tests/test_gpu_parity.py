@@ -88,6 +88,10 @@ ROW_CASES = [
     (100, 1056, torch.bfloat16), (64, 16384, torch.bfloat16), (32, 16384, torch.float32),
     (129, 2048, torch.bfloat16), (7, 4128, torch.float32),
     (50, 3072, torch.bfloat16), (77, 4096, torch.bfloat16), (5, 4064, torch.bfloat16),
+    # bf16 rows split over 2 or 4 warps (4096 < K <= 16384), ragged last segments
+    (33, 4128, torch.bfloat16), (19, 5504, torch.bfloat16), (70, 8192, torch.bfloat16),
+    (17, 11008, torch.bfloat16), (9, 16384, torch.bfloat16), (1, 15360, torch.bfloat16),
+    (300, 12320, torch.bfloat16),
 ]
 
 
@@ -110,9 +114,10 @@ def test_quantize_rows_special_values(qg, dtype):
     assert np.array_equal(_np(codes), oc)
 
 
-def test_quantize_rows_strided(qg):
-    base = make_matrix((40, 1024), seed=3, device="cuda", dtype=torch.bfloat16)
-    A = base[:, :512]            # lda = 1024 > K = 512
+@pytest.mark.parametrize("K,ld", [(512, 1024), (6144, 6152)])
+def test_quantize_rows_strided(qg, K, ld):
+    base = make_matrix((40, ld), seed=3, device="cuda", dtype=torch.bfloat16)
+    A = base[:, :K]              # lda > K
     codes, scales = qg.quantize_rows(A)
     oc, os_ = oracle.quantize_rows(A.contiguous().cpu())
     assert np.array_equal(_np(codes), oc) and np.array_equal(_np(scales), os_)
@@ -183,15 +188,16 @@ def _act_inputs(name):
         return make_matrix((300, 1056), ("student_t", 4), seed=11, device="cuda",
                            dtype=torch.bfloat16), 0.99
     if name in ("band_miss_low", "band_miss_high"):
-        # M=512, K=256: the bf16 threshold pass samples whole rows 0, 8, 16, ...
-        # (all even).  Here the even rows are all zeros (or 1000x larger than
-        # the rest), so the sampled quantile is far from the true one and the
-        # exact fallback has to produce the threshold.
+        # M=512, K=256: the bf16 threshold pass samples rows 0, 8, 16, ...
+        # only.  Here those rows are all zeros (every other row zero), or
+        # 1000x larger than the rest (1/8 of the rows: the true quantile lies
+        # well below the sampled one), so the band misses the order statistic
+        # and the exact fallback has to produce the threshold.
         A = make_matrix((512, 256), ("student_t", 4), seed=12, device="cuda")
         if name == "band_miss_low":
             A[0::2] = 0.0
         else:
-            A[0::2] *= 1000.0
+            A[0::8] *= 1000.0
         return A.to(torch.bfloat16), 0.99
     raise KeyError(name)
 
@@ -210,6 +216,32 @@ def _check_act(qg, A, alpha, codes, scales, csr, T, exp):
     if codes is not None:
         assert np.array_equal(_np(scales), exp["scales"])
         assert np.array_equal(_np(codes), exp["codes"])
+
+
+def test_quantize_act_workspace_shared_with_other_paths(qg):
+    """One workspace used in turn by the cooperative bf16 kernel, the
+    multi-kernel clamp_compensate sequence and the fp32 path: each call must
+    start from its own state (the cooperative kernel's clean-counter
+    shortcut must not trust counters another path left behind)."""
+    A, alpha = _act_inputs("llama1.3b_attn_m512")
+    Af = make_matrix(tuple(A.shape), ("student_t", 4), seed=99, device="cuda")
+    M, K = A.shape
+    ws = qg.Workspace(qg.QG_OP_QUANTIZE_ACT, M, K, 1, qg.QG_F32, alpha)
+    exp = oracle.quantize_act(A.cpu(), alpha)
+    exp_f = oracle.quantize_act(Af.cpu(), alpha)
+    for step in range(3):
+        out = qg.quantize_act(A, alpha, ws=ws)
+        qg.check_status(ws, "fused")
+        _check_act(qg, A, alpha, *out, exp)
+        _, csr, T = qg.clamp_compensate(A, alpha, ws=ws, want_clamped=False)
+        qg.check_status(ws, "clamp_compensate")
+        _check_act(qg, A, alpha, None, None, csr, T, exp)
+        out = qg.quantize_act(A, alpha, ws=ws)
+        qg.check_status(ws, "fused after multi-kernel")
+        _check_act(qg, A, alpha, *out, exp)
+        out = qg.quantize_act(Af, alpha, ws=ws)
+        qg.check_status(ws, "fp32")
+        _check_act(qg, Af, alpha, *out, exp_f)
 
 
 @pytest.mark.parametrize("case", ACT_CASES)
