@@ -19,6 +19,12 @@ write-up of "Optimizing Large Language Model Training Using FP4 Quantization"
   for A, channel-wise for W) with the ScaleShift calibration.
 * ``gemm_acc`` / ``linear_y`` / ``spmm``: Y = acc * s_i * t_j + dA * W, the
   layer output in double.
+* ``mx_exponent`` / ``mx_quantize_rows`` / ``mx_quantize_cols`` / ``mx_gemm``:
+  the MXFP4 block-scaled variant (the micro-scaling section of the lecture
+  page "FP4量化训练的硬件挑战：NVIDIA Blackwell架构上的微缩放格式（Micro-scaling）实现",
+  zyxy.net/?p=24232, and the micro-scaling paragraph of the low-precision
+  training survey at 10100.com/article/123065115): blocks of 32 along K, each
+  with the E8M0 scale 2^e, e the smallest exponent with 6 * 2^e >= block max.
 * ``dgrad`` / ``wgrad``: the gradient GEMMs with FP4 operands (the write-up's
   paragraphs on the FP4 GEMM and on the differentiable gradient estimator say
   the training runs its matrix products in FP4; how gradients are quantized
@@ -85,6 +91,11 @@ def _load():
     lib.orc_gemm_acc_rows.argtypes = [P, P, I64, I64, I64, P, I64, P]
     lib.orc_linear_y_rows.argtypes = [P, P, P, P, P, P, P, I64, I64, I64, P, I64, P]
     lib.orc_spmm.argtypes = [P, P, P, P, I64, I64, P]
+    lib.orc_mx_exponent.restype = ctypes.c_int
+    lib.orc_mx_exponent.argtypes = [ctypes.c_float]
+    lib.orc_mx_quantize_rows.argtypes = [P, I64, I64, P, P]
+    lib.orc_mx_quantize_cols.argtypes = [P, I64, I64, P, P]
+    lib.orc_mx_gemm_rows.argtypes = [P, P, P, P, I64, I64, I64, P, I64, P]
     lib.orc_num_threads.restype = ctypes.c_int
     _lib = lib
     return lib
@@ -326,3 +337,56 @@ def wgrad(A, dY, rows=None) -> np.ndarray:
     M = 2 * ca.shape[1]
     acc = gemm_acc(ca, cd, M, rows)
     return scaled_product(acc, sa if rows is None else sa[np.asarray(rows)], sd)
+
+
+# -- MXFP4 block-scaled variant -------------------------------------------------------
+def mx_exponent(amax: float) -> int:
+    """Smallest e in [-127, 127] with 6 * 2^e >= amax (-127 for amax == 0)."""
+    return int(_load().orc_mx_exponent(ctypes.c_float(amax)))
+
+
+def mx_quantize_rows(A):
+    """Rows of A (M x K) in blocks of 32: (codes uint8 M x K/2, E8M0 uint8 M x K/32)."""
+    a = as_f32(A)
+    M, K = a.shape
+    assert K % 32 == 0
+    codes = np.empty((M, K // 2), dtype=np.uint8)
+    scales = np.empty((M, K // 32), dtype=np.uint8)
+    _load().orc_mx_quantize_rows(_ptr(a), M, K, _ptr(codes), _ptr(scales))
+    return codes, scales
+
+
+def mx_quantize_cols(W):
+    """Columns of W (K x N) in blocks of 32 along K, transposed:
+    (codesT uint8 N x K/2, E8M0 uint8 N x K/32)."""
+    w = as_f32(W)
+    K, N = w.shape
+    assert K % 32 == 0
+    codesT = np.empty((N, K // 2), dtype=np.uint8)
+    scalesT = np.empty((N, K // 32), dtype=np.uint8)
+    _load().orc_mx_quantize_cols(_ptr(w), K, N, _ptr(codesT), _ptr(scalesT))
+    return codesT, scalesT
+
+
+def mx_gemm(codesA, sA, codesWT, sW, K: int, rows=None) -> np.ndarray:
+    """Y = sum over blocks of 2^(eA + eW) * (block dot product of the codes),
+    in double, for the listed rows (None: all)."""
+    cA = np.ascontiguousarray(codesA, dtype=np.uint8)
+    cW = np.ascontiguousarray(codesWT, dtype=np.uint8)
+    sa = np.ascontiguousarray(sA, dtype=np.uint8)
+    sw = np.ascontiguousarray(sW, dtype=np.uint8)
+    M, N = cA.shape[0], cW.shape[0]
+    r, nr = _rows_arg(rows)
+    R = nr if r is not None else M
+    Y = np.empty((R, N), dtype=np.float64)
+    _load().orc_mx_gemm_rows(_ptr(cA), _ptr(sa), _ptr(cW), _ptr(sw), M, N, K,
+                             _ptr(r) if r is not None else None, nr, _ptr(Y))
+    return Y
+
+
+def mx_dequant_rows(codes, scales) -> np.ndarray:
+    """Dequantized M x K matrix (double): grid value of each code times its
+    block's 2^e."""
+    q = dequant_rows(codes, np.ones(np.asarray(codes).shape[0], dtype=np.float32))
+    e = np.asarray(scales, dtype=np.int64) - 127
+    return q * np.ldexp(1.0, np.repeat(e, 32, axis=1))

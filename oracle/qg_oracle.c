@@ -286,6 +286,100 @@ void orc_spmm(const int32_t* row_ptr, const int32_t* col, const double* val, con
     }
 }
 
+/* ------------------------------------------------------------------------ */
+/* MXFP4 block-scaled variant.
+ *
+ * [MX-lecture] "FP4量化训练的硬件挑战：NVIDIA Blackwell架构上的微缩放格式（Micro-
+ * scaling）实现" (zyxy.net/?p=24232), section 3 on micro-scaling: split the
+ * tensor into small groups, give each group its own scale (max scaling: from
+ * the group's largest magnitude), divide the group by its scale and round to
+ * FP4, multiply back to dequantize.
+ * [LP-survey] (10100.com/article/123065115), custom number formats: micro-
+ * scaling pairs a per-block scale, usually E8M0 (a bare power of two), with
+ * low-precision elements.
+ *
+ * Readings: groups are 32 consecutive elements along the contraction
+ * dimension (K); the block scale is the smallest power of two X = 2^e with
+ * 6 * X >= amax (the block's largest magnitude lands inside the E2M1 range
+ * without clipping), e limited to [-127, 127] and stored as the E8M0 byte
+ * e + 127; a block whose amax is 0 gets e = -127.  Codes are
+ * E2M1(fp32(x * 2^-e)) with the encoder above; the dequantized value of a
+ * code is grid(code) * 2^e.                                                 */
+int orc_mx_exponent(float amax) {
+    int e = -127;
+    while (e < 127 && ldexp(6.0, e) < (double)amax) ++e;
+    return e;
+}
+
+/* One block of n (<= 32) values with stride `stride`: codes into out_codes
+ * (unpacked, one per value), the E8M0 byte returned.                        */
+static uint8_t mx_block(const float* x, int64_t stride, int n, uint8_t* out_codes) {
+    float amax = 0.0f;
+    for (int t = 0; t < n; ++t)
+        if (fabsf(x[t * stride]) > amax) amax = fabsf(x[t * stride]);
+    const int e = orc_mx_exponent(amax);
+    const float inv = ldexpf(1.0f, -e);
+    for (int t = 0; t < n; ++t) out_codes[t] = orc_e2m1_encode(x[t * stride] * inv);
+    return (uint8_t)(e + 127);
+}
+
+/* Rows of A (M x K, K % 32 == 0): codes M x K/2, E8M0 scales M x K/32.      */
+void orc_mx_quantize_rows(const float* A, int64_t M, int64_t K, uint8_t* codes,
+                          uint8_t* scales) {
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < M; ++i) {
+        uint8_t q[32];
+        for (int64_t b = 0; b < K / 32; ++b) {
+            scales[i * (K / 32) + b] = mx_block(A + i * K + 32 * b, 1, 32, q);
+            for (int t = 0; t < 32; t += 2)
+                codes[i * (K / 2) + 16 * b + t / 2] = (uint8_t)(q[t] | (q[t + 1] << 4));
+        }
+    }
+}
+
+/* Columns of W (K x N, K % 32 == 0), blocks along K: codes written transposed
+ * N x K/2, scales N x K/32.                                                 */
+void orc_mx_quantize_cols(const float* W, int64_t K, int64_t N, uint8_t* codesT,
+                          uint8_t* scalesT) {
+#pragma omp parallel for schedule(static)
+    for (int64_t j = 0; j < N; ++j) {
+        uint8_t q[32];
+        for (int64_t b = 0; b < K / 32; ++b) {
+            scalesT[j * (K / 32) + b] = mx_block(W + 32 * b * N + j, N, 32, q);
+            for (int t = 0; t < 32; t += 2)
+                codesT[j * (K / 2) + 16 * b + t / 2] = (uint8_t)(q[t] | (q[t + 1] << 4));
+        }
+    }
+}
+
+/* Y_ij = sum over blocks b of 2^(eA_ib + eW_jb) * sum_{k in b} e2m1(qA_ik) e2m1(qW_jk),
+ * in double, for the listed rows (rows == NULL: all M).                     */
+void orc_mx_gemm_rows(const uint8_t* codesA, const uint8_t* sA, const uint8_t* codesWT,
+                      const uint8_t* sW, int64_t M, int64_t N, int64_t K, const int64_t* rows,
+                      int64_t nrows, double* Y) {
+    const int64_t R = rows ? nrows : M;
+    const int64_t nb = K / 32;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t r = 0; r < R; ++r) {
+        const int64_t i = rows ? rows[r] : r;
+        for (int64_t j = 0; j < N; ++j) {
+            double y = 0.0;
+            for (int64_t b = 0; b < nb; ++b) {
+                double part = 0.0;
+                for (int64_t k = 32 * b; k < 32 * b + 32; ++k) {
+                    const uint8_t ba = codesA[i * (K / 2) + k / 2];
+                    const uint8_t bw = codesWT[j * (K / 2) + k / 2];
+                    const uint8_t ca = (k & 1) ? (uint8_t)(ba >> 4) : (uint8_t)(ba & 15u);
+                    const uint8_t cw = (k & 1) ? (uint8_t)(bw >> 4) : (uint8_t)(bw & 15u);
+                    part += orc_e2m1_value(ca) * orc_e2m1_value(cw);
+                }
+                y += ldexp(part, ((int)sA[i * nb + b] - 127) + ((int)sW[j * nb + b] - 127));
+            }
+            Y[r * N + j] = y;
+        }
+    }
+}
+
 int orc_num_threads(void) {
 #ifdef _OPENMP
     return omp_get_max_threads();

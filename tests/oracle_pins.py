@@ -451,6 +451,127 @@ def pin_grads_within_rounding_bound(orc, seed=14):
     assert np.all(err <= bound * (1 + 1e-6)) and err.max() > 0
 
 
+# ------------------------------------------------------------ MXFP4 variant
+def _mx_exponent_by_bits(amax: float) -> int:
+    """The block exponent from the fp32 fields alone: with amax = m * 2^E,
+    m in [1, 2), 6 * 2^e >= amax holds first at e = E - 2 when m <= 1.5 and
+    at e = E - 1 when m > 1.5; clamped to [-127, 127]; -127 for zero."""
+    a = np.float32(amax)
+    if a == 0:
+        return -127
+    bits = int(np.array([a], dtype=np.float32).view(np.uint32)[0])
+    ex, man = (bits >> 23) & 0xFF, bits & 0x7FFFFF
+    if ex == 0:                       # subnormal: far below 6 * 2^-127
+        return -127
+    E = ex - 127
+    e = E - 2 if man <= 0x400000 else E - 1
+    return max(-127, min(127, e))
+
+
+def pin_mx_worked_example(orc):
+    g = golden()["mx_block_quantization"]
+    codes, scales = orc.mx_quantize_rows(np.array(g["rows"], dtype=np.float32))
+    assert np.array_equal(unpack(codes), np.array(g["codes_unpacked"], dtype=np.uint8))
+    assert np.array_equal(scales, np.array(g["scales_e8m0"], dtype=np.uint8))
+    dq = orc.mx_dequant_rows(codes, scales)
+    for r, want in enumerate(g["dequant_first"]):
+        assert np.array_equal(dq[r, :len(want)], np.array(want))
+    for k, e in g["exponents"].items():
+        assert orc.mx_exponent(float(k)) == e
+
+
+def pin_mx_exponent_vs_bit_fields(orc, seed=20):
+    rng = np.random.default_rng(seed)
+    vals = [0.0, 1e-45, 1e-40, 2.0 ** -126, 3.4e38, 6.0, 3.0, 1.5, 0.75]
+    for e in range(-125, 126, 7):
+        for m in (1.0, 1.25, 1.5, 1.75, 1.9999999):
+            vals.append(m * 2.0 ** e)
+            vals.append(np.nextafter(np.float32(m * 2.0 ** e), np.float32(np.inf)))
+            vals.append(np.nextafter(np.float32(m * 2.0 ** e), np.float32(0)))
+    vals += list((rng.standard_normal(2000) * 10.0 ** rng.integers(-30, 30, 2000)).astype(np.float32))
+    for v in vals:
+        v = abs(float(np.float32(v)))
+        assert orc.mx_exponent(v) == _mx_exponent_by_bits(v), v
+
+
+def _mx_on_grid_rows(rng, M, K, espan=30):
+    """Rows of 32-blocks, each block on grid * 2^e_b with its max 4 or 6 * 2^e_b,
+    e_b in [-espan, espan)."""
+    grid = format_grid()[:8]
+    nb = K // 32
+    codes = rng.integers(0, 8, size=(M, K))
+    top = np.where(rng.random((M, nb)) < 0.5, 6, 7)            # grid 4 or 6
+    codes = np.minimum(codes, np.repeat(top, 32, axis=1))
+    pos = rng.integers(0, 32, size=(M, nb)) + 32 * np.arange(nb)
+    codes[np.arange(M)[:, None], pos] = top
+    sign = np.where(rng.random((M, K)) < 0.5, -1.0, 1.0)
+    eb = rng.integers(-espan, espan, size=(M, nb))
+    A = sign * grid[codes] * np.ldexp(1.0, np.repeat(eb, 32, axis=1))
+    return A.astype(np.float32), codes, sign, eb
+
+
+def pin_mx_rows_on_grid_identity(orc, seed=21):
+    rng = np.random.default_rng(seed)
+    A, codes, sign, eb = _mx_on_grid_rows(rng, 9, 128)
+    q, s = orc.mx_quantize_rows(A)
+    assert np.array_equal(s.astype(np.int64) - 127, eb)
+    want = (codes | np.where(sign < 0, 8, 0)).astype(np.uint8)
+    assert np.array_equal(unpack(q), want)
+    assert np.array_equal(orc.mx_dequant_rows(q, s), A.astype(np.float64))
+
+
+def pin_mx_rows_properties(orc, seed=22):
+    """Off-grid rows: the exponent is minimal, nothing clips, and every value
+    is within one block unit 2^e of its dequantized value (the widest grid
+    gap, 4 to 6, is 2 units); a block of zeros keeps only sign bits."""
+    rng = np.random.default_rng(seed)
+    A = (rng.standard_t(3, size=(17, 256)) * 10.0 ** rng.integers(-5, 5, size=(17, 1))).astype(np.float32)
+    A[3, 32:64] = 0.0
+    A[4, 64:96] = -0.0
+    q, s = orc.mx_quantize_rows(A)
+    e = s.astype(np.int64) - 127
+    amax = np.abs(A.astype(np.float64)).reshape(17, 8, 32).max(axis=2)
+    nz = amax > 0
+    assert np.all(np.ldexp(6.0, e)[nz] >= amax[nz])
+    assert np.all((np.ldexp(6.0, e - 1) < amax)[nz & (e > -127)])
+    assert np.all(e[~nz] == -127)
+    dq = orc.mx_dequant_rows(q, s)
+    unit = np.ldexp(1.0, np.repeat(e, 32, axis=1))
+    assert np.all(np.abs(dq - A) <= unit)
+    u = unpack(q)
+    assert np.all(u[3, 32:64] == 0) and np.all(u[4, 64:96] == 8)
+
+
+def pin_mx_cols_are_rows_of_transpose(orc, seed=23):
+    rng = np.random.default_rng(seed)
+    W = (rng.standard_normal((96, 40)) * 0.02).astype(np.float32)
+    qT, sT = orc.mx_quantize_cols(W)
+    qr, sr = orc.mx_quantize_rows(np.ascontiguousarray(W.T))
+    assert np.array_equal(qT, qr) and np.array_equal(sT, sr)
+
+
+def pin_mx_gemm(orc, seed=24):
+    """On-grid operands (block exponents within +-4, so every sum is exact in
+    double): the block-scaled product is A @ W exactly; off-grid: it equals
+    the product of the dequantized operands (numpy matmul)."""
+    rng = np.random.default_rng(seed)
+    M, N, K = 7, 11, 96
+    A, *_ = _mx_on_grid_rows(rng, M, K, espan=4)
+    WT, *_ = _mx_on_grid_rows(rng, N, K, espan=4)
+    qa, sa = orc.mx_quantize_rows(A)
+    qw, sw = orc.mx_quantize_rows(WT)
+    Y = orc.mx_gemm(qa, sa, qw, sw, K)
+    assert np.array_equal(Y, A.astype(np.float64) @ WT.astype(np.float64).T)
+    B = rng.standard_t(4, size=(M, K)).astype(np.float32)
+    W = rng.standard_normal((K, N)).astype(np.float32)
+    qb, sb = orc.mx_quantize_rows(B)
+    qwt, swt = orc.mx_quantize_cols(W)
+    Y = orc.mx_gemm(qb, sb, qwt, swt, K)
+    ref = orc.mx_dequant_rows(qb, sb) @ orc.mx_dequant_rows(qwt, swt).T
+    assert np.allclose(Y, ref, rtol=1e-12, atol=1e-300)
+    assert np.array_equal(orc.mx_gemm(qb, sb, qwt, swt, K, rows=[6, 2]), Y[[6, 2]])
+
+
 ALL_PINS = [
     pin_grid, pin_encoder_ties, pin_encoder_nearest_search, pin_row_worked_example,
     pin_col_worked_example, pin_threshold_worked_example, pin_act_worked_example,
@@ -459,5 +580,7 @@ ALL_PINS = [
     pin_quantize_cols_transpose, pin_gemm_vs_integer_matmul, pin_spmm_vs_scipy,
     pin_linear_no_clamp_is_dequant_matmul, pin_linear_exact_on_grid,
     pin_quantize_act_composition, pin_dgrad_exact_on_grid, pin_wgrad_exact_on_grid,
-    pin_grads_within_rounding_bound,
+    pin_grads_within_rounding_bound, pin_mx_worked_example, pin_mx_exponent_vs_bit_fields,
+    pin_mx_rows_on_grid_identity, pin_mx_rows_properties, pin_mx_cols_are_rows_of_transpose,
+    pin_mx_gemm,
 ]

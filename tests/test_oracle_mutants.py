@@ -41,6 +41,15 @@ MUTANTS = [
     ("spmm_wrong_row_of_w", "const float* w = W + (int64_t)col[p] * N;\n            for (int64_t j = 0; j < N; ++j) c[j]",
      "const float* w = W + (int64_t)(col[p] > 0 ? col[p] - 1 : 0) * N;\n            for (int64_t j = 0; j < N; ++j) c[j]"),
     ("delta_in_single", "val[nnz] = (double)a - (double)ac;", "val[nnz] = (double)(float)(a * 1.0000001f - ac);"),
+    ("mx_exponent_floor_rule", "ldexp(6.0, e) < (double)amax", "ldexp(8.0, e) <= (double)amax"),
+    ("mx_exponent_not_minimal", "while (e < 127 && ldexp(6.0, e) < (double)amax) ++e;",
+     "while (e < 127 && ldexp(6.0, e) < (double)amax) ++e;\n    if (amax > 0.0f && e < 127) ++e;"),
+    ("mx_block_of_16", "mx_block(A + i * K + 32 * b, 1, 32, q)",
+     "mx_block(A + i * K + 32 * b, 1, 16, q); mx_block(A + i * K + 32 * b + 16, 1, 16, q + 16)"),
+    ("mx_gemm_scale_difference", "((int)sA[i * nb + b] - 127) + ((int)sW[j * nb + b] - 127)",
+     "((int)sA[i * nb + b] - 127) - ((int)sW[j * nb + b] - 127)"),
+    ("mx_cols_reads_transposed", "mx_block(W + 32 * b * N + j, N, 32, q)",
+     "mx_block(W + 32 * b + j * K, 1, 32, q)"),
 ]
 
 
