@@ -620,6 +620,72 @@ def grads_sweep(device, workload, reps=20, warm=5):
         del A, W, dY, codesT, t
 
 
+def mx_sweep(device, workload, reps=20, warm=5):
+    """MXFP4 variant on every linear of a workload: the block row quantizer
+    on A, the block column quantizer on W and the block-scaled GEMM (fp32 Y),
+    each timed alone (median of `reps`, L2 flushed before each), beside the
+    per-row/per-column FP4 GEMM of the same shape.  One JSON line per linear."""
+    import quantize_gemm_b200 as qg
+    from workloads import WORKLOADS, make_layer_inputs
+    peaks = _peaks()
+    fp4_peak = 4.0 * peaks["bf16_tflops_sustained"]
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+    wl = WORKLOADS[workload]
+
+    def timed(fn):
+        for _ in range(warm):
+            fn()
+        ts = []
+        for _ in range(reps):
+            flush.fill_(1)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        ts.sort()
+        return ts[len(ts) // 2]
+
+    for li, layer in enumerate(wl.layers):
+        A, W = make_layer_inputs(wl, li, device=device)
+        M, K = A.shape
+        N = W.shape[1]
+        ws_q = qg.Workspace(qg.QG_OP_QUANTIZE_ROWS, M, K, 1, qg._dt(A), device=device)
+        codes = torch.empty((M, K // 2), dtype=torch.uint8, device=device)
+        sa = torch.empty(qg.qg_mx_scale_bytes(M, K), dtype=torch.uint8, device=device)
+        codesT = torch.empty((N, K // 2), dtype=torch.uint8, device=device)
+        sw = torch.empty(qg.qg_mx_scale_bytes(N, K), dtype=torch.uint8, device=device)
+        t_rows = timed(lambda: qg.qg_mx_quantize_rows(A, codes, sa, ws_q))
+        t_cols = timed(lambda: qg.qg_mx_quantize_cols(W, codesT, sw, ws_q))
+        qg.check_status(ws_q, "mx quantizers")
+        Y = torch.empty((M, N), dtype=torch.float32, device=device)
+        ws_g = qg.Workspace(qg.QG_OP_FP4_GEMM, M, K, N, qg.QG_F32, device=device)
+        t_mx = timed(lambda: qg.qg_mx_gemm(codes, sa, codesT, sw, M, N, K, None, Y, None, ws_g))
+        s_row = torch.full((M,), 1e-3, device=device)
+        s_col = torch.full((N,), 1e-3, device=device)
+        t_fp4 = timed(lambda: qg.qg_fp4_gemm(codes, s_row, codesT, s_col, M, N, K, None, Y, None,
+                                             ws_g))
+        qg.check_status(ws_g, "mx gemm")
+        fl = 2.0 * M * K * N
+        b = qg._dt(A) == qg.QG_BF16 and 2 or 4
+        line = {"sweep": "mx", "workload": wl.name, "layer": layer.name, "M": M, "K": K, "N": N,
+                "dtype": wl.dtype, "y": "f32", "l2": "flushed before each rep", "reps": reps,
+                "fp4_peak_tflops": fp4_peak, "hbm_gbs": peaks["hbm_gbs"]}
+        for k, tm, by in (("mx_quantize_rows", t_rows, b * M * K + M * K / 2 + M * K / 32),
+                          ("mx_quantize_cols", t_cols, b * K * N + K * N / 2 + K * N / 32)):
+            gbs = by / (tm * 1e-3) / 1e9
+            line[k] = {"ms": round(tm, 4), "GB/s": round(gbs, 1),
+                       "frac_measured": round(gbs / peaks["hbm_gbs"], 4)}
+        for k, tm in (("mx_gemm", t_mx), ("fp4_gemm_row_col_scales", t_fp4)):
+            tf = fl / (tm * 1e-3) / 1e12
+            line[k] = {"ms": round(tm, 4), "TFLOP/s": round(tf, 1),
+                       "frac_measured": round(tf / fp4_peak, 4)}
+        print(json.dumps(line), flush=True)
+        del A, W, codes, codesT, sa, sw, Y, ws_q, ws_g
+        torch.cuda.empty_cache()
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -636,6 +702,9 @@ def main():
     ap.add_argument("--quantizer-sweep", action="store_true",
                     help="time the three quantizers over 1M..256M bf16 elements (one JSON line "
                          "per size) instead of the layer stream")
+    ap.add_argument("--mx", action="store_true",
+                    help="time the MXFP4 block-scaled quantizers and GEMM on each linear of "
+                         "--workload (one JSON line per linear) instead of the layer stream")
     ap.add_argument("--grads", action="store_true",
                     help="time forward, dgrad and wgrad of each linear of --workload (one JSON "
                          "line per linear) instead of the layer stream")
@@ -663,10 +732,12 @@ def main():
     import __graft_entry__
     if rank == 0:
         __graft_entry__.build()
-    if args.quantizer_sweep or args.grads:
+    if args.quantizer_sweep or args.grads or args.mx:
         if rank == 0:
             if args.quantizer_sweep:
                 quantizer_sweep(device)
+            elif args.mx:
+                mx_sweep(device, args.workload)
             else:
                 grads_sweep(device, args.workload)
         return

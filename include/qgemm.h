@@ -240,6 +240,47 @@ qg_status qg_fp4_wgrad(const void* A, qg_dtype a_dtype, int64_t M, int64_t K, co
                        qg_dtype dy_dtype, int64_t N, void* dW, qg_dtype out_dtype, void* ws,
                        size_t ws_bytes, cudaStream_t stream);
 
+/* MXFP4 block-scaled variant: E2M1 codes with one E8M0 scale per 32
+ * consecutive elements along K (the micro-scaling section of the lecture page
+ * "FP4量化训练的硬件挑战：NVIDIA Blackwell架构上的微缩放格式（Micro-scaling）实现",
+ * zyxy.net/?p=24232: group, scale by the group's max, divide, round to FP4;
+ * the E8M0 block scale from the micro-scaling paragraph of the low-precision
+ * training survey at 10100.com/article/123065115).  Reading: the block scale
+ * is 2^e with e the smallest exponent such that 6 * 2^e >= the block's largest
+ * magnitude (no clipping), e in [-127, 126] stored as the byte e + 127 (a zero
+ * block gets e = -127); codes E2M1(fp32(x * 2^-e)), ties to the even code.
+ *
+ * Codes: row-major, two codes per byte (even k in the low nibble): rows of A
+ * as M x K/2, columns of W transposed as N x K/2.  Scales: the layout the GEMM
+ * reads, in 512-byte atoms: rows in blocks of 128, K in groups of 128 (four
+ * 32-blocks); one atom per (row block, k group), k group fastest, with
+ * 2 * ceil(K / 256) groups per row block; in an atom, row r (0..127 inside its
+ * block) and 32-block j (0..3 inside the group) sit at byte
+ * (r % 32) * 16 + (r / 32) * 4 + j.  Padding rows and blocks hold 127 (2^0).
+ * qg_mx_scale_bytes(rows, K) = ceil(rows / 128) * ceil(K / 256) * 1024 is the
+ * buffer size (0 for an invalid K).  K % 32 == 0 and K <= 16384; all pointers
+ * 16-byte aligned; A row pitch lda (elements) with lda * element size a
+ * multiple of 16; W row pitch ldw >= N.  Non-finite inputs set the workspace
+ * status (QG_ERR_NONFINITE from qg_sync_status) and give unspecified codes.
+ * Workspace: qg_workspace_size(QG_OP_QUANTIZE_ROWS, ...) for the quantizers,
+ * qg_workspace_size(QG_OP_FP4_GEMM, M, K, N, ...) for the GEMM.
+ *
+ * qg_mx_gemm: Y = sum over 32-blocks b of 2^(eA_ib + eW_jb) * sum_{k in b}
+ * e2m1(qA_ik) * e2m1(qW_jk) (+ C), on the block-scaled FP4 tensor-core MMA
+ * with the scales applied by the hardware; fp32 accumulation; Y fp32 or bf16,
+ * raw_acc (nullable) receives the fp32 accumulator instead of / besides Y. */
+size_t qg_mx_scale_bytes(int64_t rows, int64_t K);
+qg_status qg_mx_quantize_rows(const void* A, qg_dtype dtype, int64_t M, int64_t K, int64_t lda,
+                              uint8_t* codes, uint8_t* scales, void* ws, size_t ws_bytes,
+                              cudaStream_t stream);
+qg_status qg_mx_quantize_cols(const void* W, qg_dtype dtype, int64_t K, int64_t N, int64_t ldw,
+                              uint8_t* codesT, uint8_t* scalesT, void* ws, size_t ws_bytes,
+                              cudaStream_t stream);
+qg_status qg_mx_gemm(const uint8_t* codesA, const uint8_t* sA, const uint8_t* codesWT,
+                     const uint8_t* sW, int64_t M, int64_t N, int64_t K, const float* C, void* Y,
+                     qg_dtype y_dtype, float* raw_acc, void* ws, size_t ws_bytes,
+                     cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

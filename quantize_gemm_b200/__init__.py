@@ -40,7 +40,8 @@ EXPORTED = (
     "qg_workspace_size", "qg_workspace_init", "qg_sync_status", "qg_e2m1_encode",
     "qg_quantize_rows", "qg_quantize_cols", "qg_clamp_compensate", "qg_quantize_act",
     "qg_spmm_correction", "qg_fp4_gemm", "qg_fp4_linear", "qg_launch_count",
-    "qg_quantize_cols_static", "qg_fp4_dgrad", "qg_fp4_wgrad",
+    "qg_quantize_cols_static", "qg_fp4_dgrad", "qg_fp4_wgrad", "qg_mx_scale_bytes",
+    "qg_mx_quantize_rows", "qg_mx_quantize_cols", "qg_mx_gemm",
 )
 
 
@@ -86,6 +87,10 @@ _sig("qg_fp4_gemm", _INT,
      [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _INT, _P, _P, _SZ, _P])
 _sig("qg_fp4_linear", _INT,
      [_P, _INT, _I64, _I64, _P, _P, _P, _I64, _D, _P, _INT, _P, _SZ, _P])
+_sig("qg_mx_scale_bytes", _SZ, [_I64, _I64])
+_sig("qg_mx_quantize_rows", _INT, [_P, _INT, _I64, _I64, _I64, _P, _P, _P, _SZ, _P])
+_sig("qg_mx_quantize_cols", _INT, [_P, _INT, _I64, _I64, _I64, _P, _P, _P, _SZ, _P])
+_sig("qg_mx_gemm", _INT, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _INT, _P, _P, _SZ, _P])
 _sig("qg_fp4_dgrad", _INT, [_P, _INT, _I64, _I64, _P, _INT, _I64, _P, _INT, _P, _SZ, _P])
 _sig("qg_fp4_wgrad", _INT, [_P, _INT, _I64, _I64, _P, _INT, _I64, _P, _INT, _P, _SZ, _P])
 
@@ -284,6 +289,50 @@ def qg_fp4_wgrad(A, dY, dW, ws: Workspace, stream=None) -> int:
                              ws.ptr, ws.nbytes, _stream(stream))
 
 
+def qg_mx_scale_bytes(rows: int, K: int) -> int:
+    return int(_lib.qg_mx_scale_bytes(rows, K))
+
+
+def qg_mx_quantize_rows(A, codes, scales, ws: Workspace, lda=None, stream=None) -> int:
+    M, K = A.shape
+    return _lib.qg_mx_quantize_rows(_ptr(A), _dt(A), M, K, A.stride(0) if lda is None else lda,
+                                    _ptr(codes), _ptr(scales), ws.ptr, ws.nbytes, _stream(stream))
+
+
+def qg_mx_quantize_cols(W, codesT, scalesT, ws: Workspace, ldw=None, stream=None) -> int:
+    K, N = W.shape
+    return _lib.qg_mx_quantize_cols(_ptr(W), _dt(W), K, N, W.stride(0) if ldw is None else ldw,
+                                    _ptr(codesT), _ptr(scalesT), ws.ptr, ws.nbytes, _stream(stream))
+
+
+def qg_mx_gemm(codesA, sA, codesWT, sW, M, N, K, C, Y, raw_acc, ws: Workspace, stream=None) -> int:
+    y_dt = _dt(Y) if Y is not None else QG_F32
+    return _lib.qg_mx_gemm(_ptr(codesA), _ptr(sA), _ptr(codesWT), _ptr(sW), M, N, K, _ptr(C),
+                           _ptr(Y), y_dt, _ptr(raw_acc), ws.ptr, ws.nbytes, _stream(stream))
+
+
+def mx_scale_index(rows: int, K: int, device="cpu") -> torch.Tensor:
+    """Byte offset, in the GEMM's scale-atom layout, of the scale of row r and
+    32-block j, as a rows x K/32 int64 tensor (layout bookkeeping only)."""
+    groups = 2 * ((K + 255) // 256)
+    r = torch.arange(rows, device=device, dtype=torch.int64)[:, None]
+    j = torch.arange(K // 32, device=device, dtype=torch.int64)[None, :]
+    return (((r // 128) * groups + j // 4) * 512 + (r % 32) * 16 + ((r % 128) // 32) * 4 + j % 4)
+
+
+def mx_scales_to_rows(tiled: torch.Tensor, rows: int, K: int) -> torch.Tensor:
+    """Atom layout -> plain rows x K/32 bytes."""
+    return tiled.reshape(-1)[mx_scale_index(rows, K, tiled.device)]
+
+
+def mx_scales_from_rows(plain: torch.Tensor, K: int) -> torch.Tensor:
+    """Plain rows x K/32 bytes -> atom layout (padding bytes 127)."""
+    rows = plain.shape[0]
+    out = torch.full((qg_mx_scale_bytes(rows, K),), 127, dtype=torch.uint8, device=plain.device)
+    out[mx_scale_index(rows, K, plain.device).reshape(-1)] = plain.reshape(-1).to(torch.uint8)
+    return out
+
+
 # ----------------------------------------------------------- allocating helpers
 def e2m1_encode(x: torch.Tensor, ws: Optional[Workspace] = None) -> torch.Tensor:
     ws = ws or Workspace(QG_OP_QUANTIZE_ROWS, 1, 32, device=x.device)
@@ -378,6 +427,36 @@ def fp4_wgrad(A, dY, out_dtype=torch.float32, ws: Optional[Workspace] = None):
     dW = torch.empty((K, N), dtype=out_dtype, device=A.device)
     _check(qg_fp4_wgrad(A, dY, dW, ws), "qg_fp4_wgrad")
     return dW
+
+
+def mx_quantize_rows(A: torch.Tensor, ws: Optional[Workspace] = None):
+    """(codes M x K/2, scales in the atom layout) of the rows of A."""
+    M, K = A.shape
+    ws = ws or Workspace(QG_OP_QUANTIZE_ROWS, M, K, 1, _dt(A), device=A.device)
+    codes = torch.empty((M, K // 2), dtype=torch.uint8, device=A.device)
+    scales = torch.empty(qg_mx_scale_bytes(M, K), dtype=torch.uint8, device=A.device)
+    _check(qg_mx_quantize_rows(A, codes, scales, ws), "qg_mx_quantize_rows")
+    return codes, scales
+
+
+def mx_quantize_cols(W: torch.Tensor, ws: Optional[Workspace] = None):
+    """(codesT N x K/2, scales in the atom layout) of the columns of W (K x N)."""
+    K, N = W.shape
+    ws = ws or Workspace(QG_OP_QUANTIZE_ROWS, 1, K, 1, _dt(W), device=W.device)
+    codesT = torch.empty((N, K // 2), dtype=torch.uint8, device=W.device)
+    scalesT = torch.empty(qg_mx_scale_bytes(N, K), dtype=torch.uint8, device=W.device)
+    _check(qg_mx_quantize_cols(W, codesT, scalesT, ws), "qg_mx_quantize_cols")
+    return codesT, scalesT
+
+
+def mx_gemm(codesA, sA, codesWT, sW, K: int, C=None, out_dtype=torch.float32, raw: bool = False,
+            ws: Optional[Workspace] = None):
+    M, N = codesA.shape[0], codesWT.shape[0]
+    ws = ws or Workspace(QG_OP_FP4_GEMM, M, K, N, QG_F32, device=codesA.device)
+    Y = torch.empty((M, N), dtype=out_dtype, device=codesA.device)
+    acc = torch.empty((M, N), dtype=torch.float32, device=codesA.device) if raw else None
+    _check(qg_mx_gemm(codesA, sA, codesWT, sW, M, N, K, C, Y, acc, ws), "qg_mx_gemm")
+    return (Y, acc) if raw else Y
 
 
 def check_status(ws: Workspace, where: str = "device status", stream=None):

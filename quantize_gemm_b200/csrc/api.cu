@@ -400,4 +400,60 @@ qg_status qg_fp4_wgrad(const void* A, qg_dtype a_dtype, int64_t M, int64_t K, co
                                        at<uint32_t>(ws, L.status), stream));
 }
 
+size_t qg_mx_scale_bytes(int64_t rows, int64_t K) {
+    if (rows < 1 || K < 32 || K % 32 != 0) return 0;
+    return (size_t)((rows + 127) / 128) * (size_t)((K + 255) / 256) * 1024u;
+}
+
+qg_status qg_mx_quantize_rows(const void* A, qg_dtype dtype, int64_t M, int64_t K, int64_t lda,
+                              uint8_t* codes, uint8_t* scales, void* ws, size_t ws_bytes,
+                              cudaStream_t stream) {
+    if (!dtype_ok(dtype)) return QG_ERR_INVALID_ARG;
+    qg_status st = check_mk(M, K);
+    if (st != QG_OK) return st;
+    if ((st = check_ld(A, dtype, K, lda)) != QG_OK) return st;
+    if (!codes || !scales || !aligned16(codes) || !aligned16(scales)) return QG_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(QG_OP_QUANTIZE_ROWS, M, K, 1, dtype, 1.0);
+    if ((st = check_ws(ws, ws_bytes, L.total)) != QG_OK) return st;
+    if (ensure_device(nullptr) != cudaSuccess) return QG_ERR_CUDA;
+    launch_mx_quantize_rows(A, dtype, M, K, lda, codes, scales, at<uint32_t>(ws, L.status), stream);
+    return cuda_status(cudaGetLastError());
+}
+
+qg_status qg_mx_quantize_cols(const void* W, qg_dtype dtype, int64_t K, int64_t N, int64_t ldw,
+                              uint8_t* codesT, uint8_t* scalesT, void* ws, size_t ws_bytes,
+                              cudaStream_t stream) {
+    if (!dtype_ok(dtype)) return QG_ERR_INVALID_ARG;
+    qg_status st = check_mk(N, K);
+    if (st != QG_OK) return st;
+    if (W == nullptr || ldw < N) return QG_ERR_INVALID_ARG;
+    if (!codesT || !scalesT || !aligned16(codesT) || !aligned16(scalesT)) return QG_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(QG_OP_QUANTIZE_ROWS, 1, K, 1, dtype, 1.0);
+    if ((st = check_ws(ws, ws_bytes, L.total)) != QG_OK) return st;
+    if (ensure_device(nullptr) != cudaSuccess) return QG_ERR_CUDA;
+    launch_mx_quantize_cols(W, dtype, K, N, ldw, codesT, scalesT, at<uint32_t>(ws, L.status), stream);
+    return cuda_status(cudaGetLastError());
+}
+
+qg_status qg_mx_gemm(const uint8_t* codesA, const uint8_t* sA, const uint8_t* codesWT,
+                     const uint8_t* sW, int64_t M, int64_t N, int64_t K, const float* C, void* Y,
+                     qg_dtype y_dtype, float* raw_acc, void* ws, size_t ws_bytes,
+                     cudaStream_t stream) {
+    if (!dtype_ok(y_dtype)) return QG_ERR_INVALID_ARG;
+    qg_status st = check_mk(M, K);
+    if (st != QG_OK) return st;
+    if ((st = check_mk(N, K)) != QG_OK) return st;
+    if (!codesA || !codesWT || !sA || !sW || !aligned16(codesA) || !aligned16(codesWT) ||
+        !aligned16(sA) || !aligned16(sW))
+        return QG_ERR_INVALID_ARG;
+    if (Y == nullptr && raw_acc == nullptr) return QG_ERR_INVALID_ARG;
+    if ((Y && !aligned16(Y)) || (C && !aligned16(C)) || (raw_acc && !aligned16(raw_acc)))
+        return QG_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(QG_OP_FP4_GEMM, M, K, N, y_dtype, 1.0);
+    if ((st = check_ws(ws, ws_bytes, L.total)) != QG_OK) return st;
+    if (ensure_device(nullptr) != cudaSuccess) return QG_ERR_CUDA;
+    return cuda_status(launch_fp4_gemm_mx(codesA, sA, codesWT, sW, M, N, K, C, Y, y_dtype, raw_acc,
+                                          at<uint32_t>(ws, L.status), stream));
+}
+
 }  // extern "C"

@@ -39,6 +39,14 @@
 //              accumulator output and row pitches that TMA cannot describe.
 // TMEM: accumulators at columns [0, BN) and [BN, 2 BN), constant block
 // scales (every byte 0x7F = 2^0) at [448, 512).
+// MX = true (MXFP4 operands, solo CTAs, BN = 128): every stage also brings the
+// stage's E8M0 block scales of both operands (two 512-byte atoms each, see
+// qg_mx_quantize_rows) by a bulk copy; the MMA thread moves them into a TMEM
+// slot of the stage with tcgen05.cp (32 rows x 16 bytes, repeated into the four
+// lane quarters) and points each MMA at them.  The block-scaled MMA reads the
+// scales of row r from lane r, column slot + r / 32, and the scale-factor id
+// of the instruction descriptor picks the byte pair of its two 32-blocks.
+// The epilogue then writes the accumulator as is (+ C).
 // Every mbarrier wait is bounded; a wait that gives up sets the timeout bit in
 // the status word, raises a CTA-wide abort flag, waits (bounded) for copies
 // and MMAs in flight, frees TMEM and returns.
@@ -76,21 +84,31 @@ constexpr int kSfbCol = 480;
 #ifndef QG_GEMM_FORCE_BN
 #define QG_GEMM_FORCE_BN 0
 #endif
+#ifndef QG_GEMM_MX_STAGES
+#define QG_GEMM_MX_STAGES 4
+#endif
+constexpr int kMxSfCol = 256;        // MX: per-stage scale slots, 16 columns each
+constexpr int kMxAtom = 512;         // 32 rows x 16 bytes of E8M0 scales (128 rows x 4 blocks)
+constexpr int kMxStageSf = 4 * kMxAtom;   // two atoms of A, two of W^T per 256-deep stage
 constexpr int kEpiBuf = 32 * 32 * 4;   // one 32 x 32 fp32 sub-tile
 constexpr int kEpiBufs = QG_GEMM_EPI_BUFS;   // sub-tile buffers per epilogue warp (>= 2)
 constexpr long long kWaitLimit = 2000000000LL;  // SM clocks (~1-2 s)
 constexpr int kStageABytes = BM * BK_BYTES;
 
-template <int BN, bool PAIR>
+template <int BN, bool PAIR, bool MX = false>
 struct Cfg {
     static_assert(BN % 32 == 0 && BN <= 224, "two accumulators + scales must fit in TMEM");
-    static constexpr int kStages = PAIR ? QG_GEMM_PAIR_STAGES : QG_GEMM_SOLO_STAGES;
+    static_assert(!MX || (!PAIR && BN == 128), "MX tiles: one CTA, 128 x 128");
+    static constexpr int kStages = MX ? QG_GEMM_MX_STAGES : PAIR ? QG_GEMM_PAIR_STAGES : QG_GEMM_SOLO_STAGES;
+    static_assert(!MX || kMxSfCol + 16 * kStages <= kSfaCol, "MX scale slots below the constant scales");
     static constexpr int kBRows = PAIR ? BN / 2 : BN;   // rows of W^T loaded by one CTA
     static constexpr int kStageBBytes = kBRows * BK_BYTES;
-    static constexpr uint32_t kTxBytes = (PAIR ? 2u : 1u) * (kStageABytes + kStageBBytes);
+    static constexpr int kStageSfBytes = MX ? kMxStageSf : 0;
+    static constexpr uint32_t kTxBytes = (PAIR ? 2u : 1u) * (kStageABytes + kStageBBytes) + kStageSfBytes;
     static constexpr int kTileRows = PAIR ? 2 * BM : BM;
     static constexpr size_t kOffB = (size_t)kStages * kStageABytes;
-    static constexpr size_t kOffEpi = kOffB + (size_t)kStages * kStageBBytes;
+    static constexpr size_t kOffSf = kOffB + (size_t)kStages * kStageBBytes;
+    static constexpr size_t kOffEpi = kOffSf + (size_t)kStages * kStageSfBytes;
     static constexpr size_t kOffSw = kOffEpi + (size_t)kEpiWarps * kEpiBufs * kEpiBuf;
     static constexpr size_t kOffBar = kOffSw + (size_t)kEpiWarps * ((BN / 32 + kEpiSplit - 1) / kEpiSplit) * 32 * 4;
 };
@@ -107,11 +125,12 @@ struct alignas(8) Barriers {
     int abort;
 };
 
-template <int BN, bool PAIR>
+template <int BN, bool PAIR, bool MX = false>
 constexpr size_t smem_bytes() {
-    return 1024 + Cfg<BN, PAIR>::kOffBar + sizeof(Barriers<Cfg<BN, PAIR>::kStages>);
+    return 1024 + Cfg<BN, PAIR, MX>::kOffBar + sizeof(Barriers<Cfg<BN, PAIR, MX>::kStages>);
 }
-static_assert(smem_bytes<224, true>() <= 232448 && smem_bytes<224, false>() <= 232448,
+static_assert(smem_bytes<224, true>() <= 232448 && smem_bytes<224, false>() <= 232448 &&
+                  smem_bytes<128, false, true>() <= 232448,
               "pipeline stages and epilogue buffers must fit in 227 KB of shared memory");
 
 // ------------------------------------------------------------------ PTX wraps
@@ -210,6 +229,26 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void*
                      reinterpret_cast<uint64_t>(map)),
                  "r"(x), "r"(y), "r"(smem_u32(src))
                  : "memory");
+}
+// Plain bulk copy global -> this CTA's shared memory (16-byte aligned, size a
+// multiple of 16), completing on a barrier of this CTA.
+__device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_u32(dst)),
+        "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+        : "memory");
+}
+// One scale atom (32 rows x 16 bytes, no swizzle, 8-row groups 128 bytes
+// apart) from shared memory into TMEM columns [taddr, taddr + 4) of all four
+// lane quarters.
+__device__ __forceinline__ void tc_cp_scales(uint32_t taddr, uint32_t saddr) {
+    uint64_t d = 0;
+    d |= (uint64_t)((saddr >> 4) & 0x3FFFu);
+    d |= (uint64_t)(2048 >> 4) << 16;   // leading byte offset (one 16-byte column: unused)
+    d |= (uint64_t)(128 >> 4) << 32;    // stride byte offset: next 8-row group
+    d |= (uint64_t)1 << 46;             // descriptor version, no swizzle
+    asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(d) : "memory");
 }
 __device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
 template <int N>
@@ -388,6 +427,10 @@ struct Params {
     int M, N, K;
     int y_bf16;
     int tma_epi;         // Y (and C) through TMA
+    int unit_scales;     // MX: no row / column scales in the epilogue
+    const uint8_t* sfA;  // MX: E8M0 scale atoms of A, [row block][k group]
+    const uint8_t* sfB;  // MX: the same for W^T
+    int sf_groups;       // MX: 128-deep k groups per row block (even)
 };
 
 // Direct epilogue of one 32-column chunk: registers -> global (row per lane).
@@ -416,7 +459,7 @@ __device__ __forceinline__ void epi_direct(const Params& p, const uint32_t (&v)[
         const float4* crow = p.C ? reinterpret_cast<const float4*>(p.C + off) : nullptr;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
-            const float4 t = __ldg(tw + j);
+            const float4 t = p.unit_scales ? make_float4(1.0f, 1.0f, 1.0f, 1.0f) : __ldg(tw + j);
             float4 y = make_float4(__fmul_rn(__fmul_rn(__uint_as_float(v[4 * j]), s_row), t.x),
                                    __fmul_rn(__fmul_rn(__uint_as_float(v[4 * j + 1]), s_row), t.y),
                                    __fmul_rn(__fmul_rn(__uint_as_float(v[4 * j + 2]), s_row), t.z),
@@ -435,7 +478,8 @@ __device__ __forceinline__ void epi_direct(const Params& p, const uint32_t (&v)[
 #pragma unroll
     for (int j = 0; j < 32; ++j) {
         if (col0 + j >= p.N) continue;
-        float yy = __fmul_rn(__fmul_rn(__uint_as_float(v[j]), s_row), __ldg(p.sW + col0 + j));
+        const float tj = p.unit_scales ? 1.0f : __ldg(p.sW + col0 + j);
+        float yy = __fmul_rn(__fmul_rn(__uint_as_float(v[j]), s_row), tj);
         if (p.C) yy = __fadd_rn(yy, __ldg(p.C + off + j));
         if (p.y_bf16) static_cast<__nv_bfloat16*>(p.Y)[off + j] = __float2bfloat16_rn(yy);
         else static_cast<float*>(p.Y)[off + j] = yy;
@@ -445,19 +489,20 @@ __device__ __forceinline__ void epi_direct(const Params& p, const uint32_t (&v)[
 // TMA_EPI: Y (and C) go through the swizzled sub-tile buffers and TMA; the
 // other instantiation stores registers directly (raw accumulator output, or
 // row pitches TMA cannot describe), so neither path's registers burden the other.
-template <int BN, bool PAIR, bool TMA_EPI>
+template <int BN, bool PAIR, bool TMA_EPI, bool MX = false>
 __global__ void __launch_bounds__(kThreads, 1)
 fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 const __grid_constant__ CUtensorMap tmap_b,
                 const __grid_constant__ CUtensorMap tmap_y,
                 const __grid_constant__ CUtensorMap tmap_c, const Params p) {
-    using CF = Cfg<BN, PAIR>;
+    using CF = Cfg<BN, PAIR, MX>;
     constexpr int S = CF::kStages;
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
     uint8_t* sa = smem;
     uint8_t* sb = smem + CF::kOffB;
+    uint8_t* ssf = smem + CF::kOffSf;
     uint8_t* sepi = smem + CF::kOffEpi;
     Barriers<S>* B = reinterpret_cast<Barriers<S>*>(smem + CF::kOffBar);
 
@@ -537,6 +582,15 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                         mbar_expect_tx(&B->full[stage], CF::kTxBytes);
                         tma_load_2d(&tmap_a, &B->full[stage], da, kb * BK_BYTES, a_row);
                         tma_load_2d(&tmap_b, &B->full[stage], db, kb * BK_BYTES, b_row);
+                        if constexpr (MX) {
+                            // the stage's two k groups are adjacent atoms
+                            uint8_t* ds = ssf + (size_t)stage * kMxStageSf;
+                            const size_t ka = (size_t)2 * kb * kMxAtom;
+                            bulk_load(ds, p.sfA + (size_t)m_blk * p.sf_groups * kMxAtom + ka,
+                                      2 * kMxAtom, &B->full[stage]);
+                            bulk_load(ds + 2 * kMxAtom, p.sfB + (size_t)n_blk * p.sf_groups * kMxAtom + ka,
+                                      2 * kMxAtom, &B->full[stage]);
+                        }
                     }
                     pend |= 1u << stage;
                     pend_par = (pend_par & ~(1u << stage)) | (phase << stage);
@@ -577,11 +631,32 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     tc_fence_after();
                     const uint32_t a0 = smem_u32(sa + (size_t)stage * kStageABytes);
                     const uint32_t b0 = smem_u32(sb + (size_t)stage * CF::kStageBBytes);
+                    if constexpr (MX) {
+                        // this stage's scales into its TMEM slot: A atoms at +0, +4,
+                        // W^T atoms at +8, +12; the copies run before the MMAs
+                        const uint32_t slot = tmem + (uint32_t)(kMxSfCol + 16 * stage);
+                        const uint32_t s0 = smem_u32(ssf + (size_t)stage * kMxStageSf);
 #pragma unroll
-                    for (int ks = 0; ks < BK_BYTES / UMMA_K_BYTES; ++ks) {
-                        mma_mxf4<PAIR>(d_tmem, smem_desc(a0 + ks * UMMA_K_BYTES),
-                                       smem_desc(b0 + ks * UMMA_K_BYTES), idesc, sfa, sfb,
-                                       (kb > 0 || ks > 0) ? 1u : 0u);
+                        for (int g = 0; g < 4; ++g) tc_cp_scales(slot + 4u * g, s0 + kMxAtom * g);
+#pragma unroll
+                        for (int ks = 0; ks < BK_BYTES / UMMA_K_BYTES; ++ks) {
+                            // MMA ks covers 32-blocks 2 ks, 2 ks + 1: atom ks / 2, bytes
+                            // 2 (ks % 2) and up (scale-factor ids, bits 29-30 and 4-5)
+                            const uint32_t id = 2u * (uint32_t)(ks & 1);
+                            mma_mxf4<PAIR>(d_tmem, smem_desc(a0 + ks * UMMA_K_BYTES),
+                                           smem_desc(b0 + ks * UMMA_K_BYTES),
+                                           idesc | (id << 29) | (id << 4),
+                                           slot + 4u * (uint32_t)(ks >> 1),
+                                           slot + 8u + 4u * (uint32_t)(ks >> 1),
+                                           (kb > 0 || ks > 0) ? 1u : 0u);
+                        }
+                    } else {
+#pragma unroll
+                        for (int ks = 0; ks < BK_BYTES / UMMA_K_BYTES; ++ks) {
+                            mma_mxf4<PAIR>(d_tmem, smem_desc(a0 + ks * UMMA_K_BYTES),
+                                           smem_desc(b0 + ks * UMMA_K_BYTES), idesc, sfa, sfb,
+                                           (kb > 0 || ks > 0) ? 1u : 0u);
+                        }
                     }
                     tc_commit_all<PAIR>(&B->empty[stage]);   // frees the stage (both CTAs)
                     if (++stage == S) stage = 0, phase ^= 1u;
@@ -640,10 +715,12 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             for (int k = 0; k < SWR; ++k) {
                 const int c = par + kEpiSplit * k;           // k-th chunk of this warp
                 const int n = n_blk * BN + c * 32 + lane;
-                swr[k] = (k < my_nc && n < p.N) ? __ldg(p.sW + n) : 0.0f;
+                if constexpr (MX) swr[k] = 1.0f;
+                else swr[k] = (k < my_nc && n < p.N) ? __ldg(p.sW + n) : 0.0f;
             }
             const int r = m_blk * CF::kTileRows + (int)rank * BM + 32 * q + lane;
-            srow_next = r < p.M ? __ldg(p.sA + r) : 0.0f;
+            if constexpr (MX) srow_next = 1.0f;
+            else srow_next = r < p.M ? __ldg(p.sA + r) : 0.0f;
         };
         if (my_tiles > 0) fetch_scales(0);
         int as = 0;
@@ -838,11 +915,11 @@ static int pick_bn(int64_t M, int64_t N, bool pair) {
     return (w192 < w224) ? 192 : 224;
 }
 
-template <int BN, bool PAIR, bool TMA_EPI>
+template <int BN, bool PAIR, bool TMA_EPI, bool MX = false>
 static cudaError_t launch_variant(const CUtensorMap& ta, const uint8_t* codesWT, int64_t N,
                                   int64_t K, const CUtensorMap& ty, const CUtensorMap& tc,
                                   const Params& p, cudaStream_t s) {
-    using CF = Cfg<BN, PAIR>;
+    using CF = Cfg<BN, PAIR, MX>;
     CUtensorMap tb;
     if (!encode_2d(&tb, CU_TENSOR_MAP_DATA_TYPE_UINT8, codesWT, K / 2, N, K / 2, BK_BYTES,
                    CF::kBRows, CU_TENSOR_MAP_SWIZZLE_128B))
@@ -853,7 +930,7 @@ static cudaError_t launch_variant(const CUtensorMap& ta, const uint8_t* codesWT,
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(units * per_unit));
     cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = smem_bytes<BN, PAIR>();
+    cfg.dynamicSmemBytes = smem_bytes<BN, PAIR, MX>();
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -862,20 +939,20 @@ static cudaError_t launch_variant(const CUtensorMap& ta, const uint8_t* codesWT,
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, fp4_gemm_kernel<BN, PAIR, TMA_EPI>, ta, tb, ty, tc, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, fp4_gemm_kernel<BN, PAIR, TMA_EPI, MX>, ta, tb, ty, tc, p);
     count_launch(1);
     return e;
 }
 
-template <int BN, bool PAIR>
+template <int BN, bool PAIR, bool MX = false>
 static cudaError_t set_smem_attr() {
-    cudaError_t e = cudaFuncSetAttribute(fp4_gemm_kernel<BN, PAIR, true>,
+    cudaError_t e = cudaFuncSetAttribute(fp4_gemm_kernel<BN, PAIR, true, MX>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem_bytes<BN, PAIR>());
+                                         (int)smem_bytes<BN, PAIR, MX>());
     if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(fp4_gemm_kernel<BN, PAIR, false>,
+    return cudaFuncSetAttribute(fp4_gemm_kernel<BN, PAIR, false, MX>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)smem_bytes<BN, PAIR>());
+                                (int)smem_bytes<BN, PAIR, MX>());
 }
 
 }  // namespace gemm
@@ -886,6 +963,7 @@ cudaError_t gemm_setup() {
     if ((e = set_smem_attr<224, false>()) != cudaSuccess) return e;
     if ((e = set_smem_attr<192, false>()) != cudaSuccess) return e;
     if ((e = set_smem_attr<224, true>()) != cudaSuccess) return e;
+    if ((e = set_smem_attr<128, false, true>()) != cudaSuccess) return e;
     return set_smem_attr<192, true>();
 }
 
@@ -906,6 +984,10 @@ cudaError_t launch_fp4_gemm(const uint8_t* codesA, const float* sA, const uint8_
     p.N = (int)N;
     p.K = (int)K;
     p.y_bf16 = (y_dtype == QG_BF16) ? 1 : 0;
+    p.unit_scales = 0;
+    p.sfA = nullptr;
+    p.sfB = nullptr;
+    p.sf_groups = 0;
     // TMA epilogue: the row pitches of Y and C must be multiples of 16 bytes
     const size_t ysz = (y_dtype == QG_BF16) ? 2 : 4;
 #ifndef QG_GEMM_DIRECT_EPI
@@ -953,6 +1035,57 @@ cudaError_t launch_fp4_gemm(const uint8_t* codesA, const float* sA, const uint8_
     }
     if (bn == 192) return launch_variant<192, false, false>(ta, codesWT, N, K, ty, tc, p, s);
     return launch_variant<224, false, false>(ta, codesWT, N, K, ty, tc, p, s);
+}
+
+// MXFP4 GEMM: Y = sum over 32-blocks of 2^(eA + eW) * (block product) (+ C).
+cudaError_t launch_fp4_gemm_mx(const uint8_t* codesA, const uint8_t* sfA, const uint8_t* codesWT,
+                               const uint8_t* sfW, int64_t M, int64_t N, int64_t K, const float* C,
+                               void* Y, qg_dtype y_dtype, float* raw_acc, uint32_t* status,
+                               cudaStream_t s) {
+    using namespace gemm;
+    Params p;
+    p.sA = nullptr;
+    p.sW = nullptr;
+    p.C = C;
+    p.Y = Y;
+    p.raw_acc = raw_acc;
+    p.status = status;
+    p.M = (int)M;
+    p.N = (int)N;
+    p.K = (int)K;
+    p.y_bf16 = (y_dtype == QG_BF16) ? 1 : 0;
+    p.unit_scales = 1;
+    p.sfA = sfA;
+    p.sfB = sfW;
+    p.sf_groups = (int)(2 * ((K + 255) / 256));
+    const size_t ysz = (y_dtype == QG_BF16) ? 2 : 4;
+    p.tma_epi = (!QG_GEMM_DIRECT_EPI && Y != nullptr && raw_acc == nullptr &&
+                 ((size_t)N * ysz) % 16 == 0 && ((size_t)N * 4) % 16 == 0)
+                    ? 1
+                    : 0;
+    CUtensorMap ta, ty, tc;
+    if (!encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, codesA, K / 2, M, K / 2, BK_BYTES, BM,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    ty = ta;
+    tc = ta;
+    if (p.tma_epi) {
+        if (y_dtype == QG_BF16) {
+            if (!encode_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, N, M, N * 2, 32, 32,
+                           CU_TENSOR_MAP_SWIZZLE_64B))
+                return cudaErrorInvalidValue;
+        } else {
+            if (!encode_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Y, N, M, N * 4, 32, 32,
+                           CU_TENSOR_MAP_SWIZZLE_128B))
+                return cudaErrorInvalidValue;
+        }
+        if (C != nullptr &&
+            !encode_2d(&tc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, C, N, M, N * 4, 32, 32,
+                       CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+        return launch_variant<128, false, true, true>(ta, codesWT, N, K, ty, tc, p, s);
+    }
+    return launch_variant<128, false, false, true>(ta, codesWT, N, K, ty, tc, p, s);
 }
 
 }  // namespace qg

@@ -363,6 +363,14 @@ void launch_quantize_cols(const void* W, qg_dtype dt, int64_t K, int64_t N, int6
                           uint8_t* codesT, float* scales, uint32_t* colmax, cudaStream_t s);
 void launch_spmm(const qg_csr* dA, int64_t M, const void* W, qg_dtype dt, int64_t N, int64_t ldw,
                  float* C, uint32_t* status, cudaStream_t s);
+void launch_mx_quantize_rows(const void* A, qg_dtype dt, int64_t M, int64_t K, int64_t lda,
+                             uint8_t* codes, uint8_t* sf, uint32_t* status, cudaStream_t s);
+void launch_mx_quantize_cols(const void* W, qg_dtype dt, int64_t K, int64_t N, int64_t ldw,
+                             uint8_t* codesT, uint8_t* sf, uint32_t* status, cudaStream_t s);
+cudaError_t launch_fp4_gemm_mx(const uint8_t* codesA, const uint8_t* sfA, const uint8_t* codesWT,
+                               const uint8_t* sfW, int64_t M, int64_t N, int64_t K, const float* C,
+                               void* Y, qg_dtype y_dtype, float* raw_acc, uint32_t* status,
+                               cudaStream_t s);
 cudaError_t launch_fp4_gemm(const uint8_t* codesA, const float* sA, const uint8_t* codesWT,
                             const float* sW, int64_t M, int64_t N, int64_t K, const float* C,
                             void* Y, qg_dtype y_dtype, float* raw_acc, uint32_t* status,

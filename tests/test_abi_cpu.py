@@ -6,6 +6,7 @@ import os
 import re
 
 import pytest
+import torch
 
 import oracle
 
@@ -31,7 +32,8 @@ def test_header_declares_the_entry_points():
     funcs = _header_functions()
     for name in ("qg_quantize_rows", "qg_quantize_cols", "qg_clamp_compensate",
                  "qg_quantize_act", "qg_spmm_correction", "qg_fp4_gemm", "qg_fp4_linear",
-                 "qg_sync_status", "qg_workspace_size", "qg_fp4_dgrad", "qg_fp4_wgrad"):
+                 "qg_sync_status", "qg_workspace_size", "qg_fp4_dgrad", "qg_fp4_wgrad",
+                 "qg_mx_quantize_rows", "qg_mx_quantize_cols", "qg_mx_gemm", "qg_mx_scale_bytes"):
         assert name in funcs
 
 
@@ -123,3 +125,31 @@ def test_host_argument_checks_need_no_device(qg):
     need = qg.qg_workspace_size(qg.QG_OP_FP4_WGRAD, 64, 64, 64, 1, 1.0)
     assert lib.qg_fp4_wgrad(fake, 1, 64, 64, fake, 1, 64, fake, 0, fake, need - 256, None) == \
         qg.QG_ERR_WORKSPACE
+
+
+def test_mx_scale_layout_host(qg):
+    """The atom layout is a bijection between (row, 32-block) pairs of the
+    padded matrix and the buffer's bytes; padding rows/blocks hold 127."""
+    for rows, K in ((1, 32), (128, 256), (129, 288), (300, 5504), (40, 13824)):
+        nbytes = qg.qg_mx_scale_bytes(rows, K)
+        assert nbytes == -(-rows // 128) * -(-K // 256) * 1024
+        rp = -(-rows // 128) * 128
+        kp = 8 * -(-K // 256) * 32
+        idx = qg.mx_scale_index(rp, kp)
+        assert idx.numel() == nbytes and torch.unique(idx).numel() == nbytes
+        plain = torch.randint(0, 255, (rows, K // 32), dtype=torch.uint8)
+        tiled = qg.mx_scales_from_rows(plain, K)
+        assert tiled.numel() == nbytes
+        assert torch.equal(qg.mx_scales_to_rows(tiled, rows, K), plain)
+        assert int((tiled == 127).sum()) >= nbytes - plain.numel()
+    assert qg.qg_mx_scale_bytes(4, 48) == 0 and qg.qg_mx_scale_bytes(0, 64) == 0
+    # host argument checks of the MX calls
+    lib = qg._lib
+    P = ctypes.c_void_p
+    fake = P(1 << 20)
+    assert lib.qg_mx_quantize_rows(fake, 1, 4, 48, 48, fake, fake, fake, 1 << 20, None) == \
+        qg.QG_ERR_UNSUPPORTED_SHAPE
+    assert lib.qg_mx_quantize_rows(fake, 1, 4, 64, 64, fake, P((1 << 20) + 4), fake, 1 << 20,
+                                   None) == qg.QG_ERR_INVALID_ARG
+    assert lib.qg_mx_gemm(fake, fake, fake, fake, 128, 128, 256, None, None, 0, None, fake,
+                          1 << 20, None) == qg.QG_ERR_INVALID_ARG

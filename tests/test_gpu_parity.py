@@ -524,3 +524,119 @@ def test_fp4_grads_full_size_sampled(qg, wl, layer):
     assert y_rel_err(_np(dA)[rows], oracle.dgrad(dY.cpu(), W.cpu(), rows=rows)) <= 1e-3
     rows = np.unique(np.concatenate([g.integers(0, K, 12), [0, K - 1]]))
     assert y_rel_err(_np(dW)[rows], oracle.wgrad(A.cpu(), dY.cpu(), rows=rows)) <= 1e-3
+
+
+# ------------------------------------------------------------ MXFP4 variant
+def _mx_plain(qg, tiled, rows, K):
+    return _np(qg.mx_scales_to_rows(tiled, rows, K))
+
+
+MX_ROW_CASES = [(1, 32, torch.float32), (5, 64, torch.bfloat16), (128, 256, torch.bfloat16),
+                (129, 288, torch.float32), (300, 5504, torch.bfloat16), (77, 16384, torch.bfloat16),
+                (256, 4096, torch.float32)]
+
+
+@pytest.mark.parametrize("M,K,dtype", MX_ROW_CASES)
+def test_mx_quantize_rows(qg, M, K, dtype):
+    A = make_matrix((M, K), ("student_t", 3), seed=M + 3 * K, device="cuda", dtype=dtype,
+                    scale=float(10.0 ** ((M % 7) - 3)))
+    codes, tiled = qg.mx_quantize_rows(A)
+    oc, os_ = oracle.mx_quantize_rows(A.cpu())
+    assert np.array_equal(_np(codes), oc)
+    assert np.array_equal(_mx_plain(qg, tiled, M, K), os_)
+    # padding rows / blocks of the atoms hold 2^0
+    idx = qg.mx_scale_index(M, K).reshape(-1).numpy()
+    pad = np.ones(tiled.numel(), dtype=bool)
+    pad[idx] = False
+    assert np.all(_np(tiled)[pad] == 127)
+
+
+def test_mx_quantize_rows_special_values(qg):
+    K = 256
+    A = np.zeros((6, K), dtype=np.float32)
+    A[1, :] = -0.0
+    A[2, :32] = 1e-42                       # subnormal block
+    A[3, :] = np.float32(3.0e38) * np.sign(np.random.default_rng(1).standard_normal(K))
+    A[4, ::3] = 6.0 * 2.0 ** -20            # block max exactly on 6 * 2^e
+    A[5, :] = np.linspace(-7.0, 7.0, K, dtype=np.float32)
+    for dt in (torch.float32, torch.bfloat16):
+        At = torch.from_numpy(A).to(dt)
+        codes, tiled = qg.mx_quantize_rows(At.cuda())
+        oc, os_ = oracle.mx_quantize_rows(At)
+        assert np.array_equal(_np(codes), oc)
+        assert np.array_equal(_mx_plain(qg, tiled, 6, K), os_)
+
+
+MX_COL_CASES = [(32, 1, torch.float32), (64, 200, torch.bfloat16), (288, 130, torch.bfloat16),
+                (2048, 5504, torch.bfloat16), (512, 512, torch.float32)]
+
+
+@pytest.mark.parametrize("K,N,dtype", MX_COL_CASES)
+def test_mx_quantize_cols(qg, K, N, dtype):
+    W = make_matrix((K, N), seed=K + N, device="cuda", dtype=dtype, scale=0.02)
+    codesT, tiled = qg.mx_quantize_cols(W)
+    oT, osT = oracle.mx_quantize_cols(W.cpu())
+    assert np.array_equal(_np(codesT), oT)
+    assert np.array_equal(_mx_plain(qg, tiled, N, K), osT)
+
+
+MX_GEMM_CASES = [(128, 128, 256), (1, 8, 32), (300, 200, 288), (129, 640, 1024), (512, 384, 5504),
+                 (256, 1000, 4096)]
+
+
+@pytest.mark.parametrize("M,N,K", MX_GEMM_CASES)
+def test_mx_gemm(qg, M, N, K):
+    """Oracle codes and scales through the block-scaled MMA: fp32 Y within the
+    layer tolerance of the oracle's double evaluation, bf16 within one ulp."""
+    A = make_matrix((M, K), ("student_t", 4), seed=M + K, dtype=torch.float32)
+    W = make_matrix((K, N), seed=N + K + 1, dtype=torch.float32, scale=0.02)
+    qa, sa = oracle.mx_quantize_rows(A)
+    qw, sw = oracle.mx_quantize_cols(W)
+    Yo = oracle.mx_gemm(qa, sa, qw, sw, K)
+    ta = qg.mx_scales_from_rows(torch.from_numpy(sa), K).cuda()
+    tw = qg.mx_scales_from_rows(torch.from_numpy(sw), K).cuda()
+    ca, cw = torch.from_numpy(qa).cuda(), torch.from_numpy(qw).cuda()
+    Y = qg.mx_gemm(ca, ta, cw, tw, K)
+    assert y_rel_err(_np(Y), Yo) <= 1e-3
+    Yb = qg.mx_gemm(ca, ta, cw, tw, K, out_dtype=torch.bfloat16)
+    rms = np.sqrt(np.mean(Yo ** 2))
+    assert np.all(np.abs(_np(Yb.float()).astype(np.float64) - Yo) <= bf16_ulp(Yo) + 1e-6 * rms)
+    C = torch.randn((M, N), device="cuda") * float(rms)
+    Yc = qg.mx_gemm(ca, ta, cw, tw, K, C=C)
+    assert y_rel_err(_np(Yc), Yo + _np(C).astype(np.float64)) <= 1e-3
+
+
+def test_mx_gemm_exact_on_grid(qg):
+    """Blocks on their scaled grids with exponents within +-2: every partial
+    sum is exact in fp32, so the raw accumulator equals A @ W exactly."""
+    from oracle_pins import _mx_on_grid_rows
+    g = np.random.default_rng(41)
+    M, N, K = 200, 136, 768
+    A, *_ = _mx_on_grid_rows(g, M, K, espan=2)
+    WT, *_ = _mx_on_grid_rows(g, N, K, espan=2)
+    codes, ta = qg.mx_quantize_rows(torch.from_numpy(A).cuda())
+    codesW, tw = qg.mx_quantize_rows(torch.from_numpy(WT).cuda())
+    Y, acc = qg.mx_gemm(codes, ta, codesW, tw, K, raw=True)
+    exact = A.astype(np.float64) @ WT.astype(np.float64).T
+    assert np.array_equal(_np(acc).astype(np.float64), exact)
+    assert np.array_equal(_np(Y).astype(np.float64), exact)
+
+
+@pytest.mark.parametrize("wl,layer", [("llama1.3b", 1), ("llama7b", 1)])
+def test_mx_pipeline_full_size_sampled(qg, wl, layer):
+    """A layer of the benchmark workloads at full size through the MX path
+    (GPU quantizers, GPU GEMM): codes and scales exact over the whole
+    tensors, Y on sampled rows against the oracle."""
+    A, W = make_layer_inputs(wl, layer, device="cuda")
+    M, K = A.shape
+    N = W.shape[1]
+    codes, ta = qg.mx_quantize_rows(A)
+    codesT, tw = qg.mx_quantize_cols(W)
+    Y = qg.mx_gemm(codes, ta, codesT, tw, K)
+    oc, os_ = oracle.mx_quantize_rows(A.cpu())
+    oT, osT = oracle.mx_quantize_cols(W.cpu())
+    assert np.array_equal(_np(codes), oc) and np.array_equal(_mx_plain(qg, ta, M, K), os_)
+    assert np.array_equal(_np(codesT), oT) and np.array_equal(_mx_plain(qg, tw, N, K), osT)
+    rows = np.unique(np.concatenate([np.random.default_rng(M + N).integers(0, M, 16), [0, M - 1]]))
+    Yo = oracle.mx_gemm(oc, os_, oT, osT, K, rows=rows)
+    assert y_rel_err(_np(Y)[rows], Yo) <= 1e-3
