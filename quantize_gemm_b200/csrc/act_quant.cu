@@ -1134,8 +1134,11 @@ __device__ void cta_scan_offsets(uint32_t* cta_tot, int ncta, const ActBuffers& 
 // (count returns to 0 after every barrier).  Every wait is bounded: a CTA
 // that gives up sets the timeout bit and returns (the workspace barrier words
 // are then reset by qg_sync_status / qg_workspace_init).
-constexpr int kFusedThreads = 256;
-constexpr int kFusedMinBlocks = 3;
+// 16 warps per CTA, two CTAs per SM (64 registers): fewer, larger CTAs make
+// the grid barriers, the band flush and the CTA-offset scan cheaper than
+// 256-thread CTAs at the same warp count per SM.
+constexpr int kFusedThreads = 512;
+constexpr int kFusedMinBlocks = 2;
 constexpr int kCtaTotOffset = 8192;   // per-CTA totals in hist1 (after the band bins)
 constexpr int kFusedMaxGrid = 8192;
 
