@@ -209,7 +209,7 @@ hist_rowmax_kernel(const void* __restrict__ A, int64_t lda, int M, int K,
 constexpr int kBandBins = 4096;            // band width in keys
 constexpr int kBandThreads = 1024;
 constexpr int kSampleBins = 4096;          // sample histogram of key >> 3
-constexpr int64_t kSampleTarget = 16384;   // sampled elements
+constexpr int64_t kSampleTarget = 8192;    // sampled elements
 constexpr int kSampleRows = 64;            // from this many rows
 
 __device__ __forceinline__ uint32_t swar_ge(uint32_t m, uint32_t c) {
@@ -259,7 +259,10 @@ __device__ void block_select3(const uint32_t* sh, const unsigned long long (&r)[
 // One CTA of NT threads: zero the counters and band bins, histogram the keys
 // >> 3 of a sample (windows of 64 rows spread evenly over A) in sh, and put
 // the band around the sample quantile with a margin of six standard
-// deviations of a sample quantile's rank plus 32.
+// deviations of a sample quantile's rank plus 32.  A margin that runs past
+// the sample's largest (smallest) key opens the band upwards (downwards), up
+// to its 4096-key width, so an extreme quantile is not missed for want of
+// sampled keys above it.
 template <int NT>
 __device__ void cta_sample_band(const uint16_t* __restrict__ A, int64_t lda, int M, int K,
                                 Counters* __restrict__ ctr, uint32_t* __restrict__ band_bins,
@@ -322,6 +325,8 @@ __device__ void cta_sample_band(const uint16_t* __restrict__ A, int64_t lda, int
     if (t == 0) {
         uint32_t lo = s_sel[0] << 3, hi = (s_sel[1] << 3) + 7u;
         const uint32_t mid = s_sel[2] << 3;
+        if (center + margin >= top) hi = 0x7FFFu;
+        if (center - margin <= 0.0) lo = 0u;
         if (hi - lo + 1 > (uint32_t)kBandBins) {
             lo = max(lo, mid > (uint32_t)(kBandBins / 2) ? mid - kBandBins / 2 : 0u);
             hi = min(hi, lo + kBandBins - 1);
