@@ -2,6 +2,7 @@
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
                     [--layer I] [--impl ours|reference] [--no-e2e] [--no-cpu-baseline]
+                    [--no-graph]
 
 A step is one forward pass of every linear layer of the workload (default:
 the LLaMA-1.3B-shaped linears, M = 4096 tokens, bf16): for each layer the
@@ -10,7 +11,14 @@ every linear forward), then the activation goes through the fused threshold /
 clamp / quantize pass, the dA . W correction and the FP4 GEMM with its
 dequantization epilogue.  Inputs are synthetic (seeded, see workloads/) and
 resident in HBM before timing; L2 is flushed (256 MiB write) between timed
-steps.  One JSON line is printed by rank 0.
+steps.  The step's library calls are captured once into a CUDA graph and the
+graph is replayed once per timed step (the cooperative and cluster launches
+capture like any other); the step time is the device time between two events
+around each replay.  Per-kernel times come from a second pass over the same
+steps, launched eagerly with events between the calls (`kernels`,
+`roofline`; those intervals also carry the launch gaps the events add, so
+they sum to `breakdown_ms_per_step`, a little above `ms_per_step`).  One JSON
+line is printed by rank 0.
 
 Multi-GPU: one process per GPU (torchrun); every rank runs its own replica of
 the workload (weak scaling, no data-path collective); the timed region is
@@ -185,6 +193,36 @@ def run_step(qg, layers, ev=None):
             ev[i][4].record()
 
 
+def capture_step(qg, layers):
+    """Capture one step (run_step) into a CUDA graph.  Returns (graph, library
+    launches in the step), or (None, None) when capture is not available;
+    the captured step is replayed once and must leave the workspaces' status
+    clean."""
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    graph = torch.cuda.CUDAGraph()
+    try:
+        with torch.cuda.stream(side):
+            run_step(qg, layers)         # on the capture stream once before capturing
+        torch.cuda.current_stream().wait_stream(side)
+        torch.cuda.synchronize()
+        n1 = qg.qg_launch_count()
+        with torch.cuda.graph(graph):
+            run_step(qg, layers)
+        per_step = qg.qg_launch_count() - n1
+        graph.replay()
+        torch.cuda.synchronize()
+        for L in layers:
+            for ws in L.workspaces():
+                qg.check_status(ws, f"graph {L.name}")
+    except Exception as ex:   # capture unsupported here: run eagerly
+        print(f"bench: CUDA graph capture unavailable ({type(ex).__name__}); eager launches",
+              file=sys.stderr)
+        torch.cuda.synchronize()
+        return None, None
+    return graph, per_step
+
+
 def our_arm(args, rank, world, device):
     import quantize_gemm_b200 as qg
     from workloads import WORKLOADS
@@ -203,9 +241,17 @@ def our_arm(args, rank, world, device):
             qg.check_status(ws, f"warm-up {L.name}")
 
     n_l = len(layers)
+    # Timed region 1 (the headline): the step's library calls captured once
+    # into a CUDA graph and replayed once per step, each replay between two
+    # events on the stream (none inside the graph); eager launches without
+    # graph support.  Timed region 2 (the breakdown): the same steps launched
+    # eagerly with events between the calls, for per-kernel times (those
+    # intervals also hold the launch gaps the events add).
+    graph, launches_per_step = (None, None) if args.no_graph else capture_step(qg, layers)
+    ev_step = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+               for _ in range(args.steps)]
     ev_steps = [[[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(n_l)]
                 for _ in range(args.steps)]
-    launches0 = qg.qg_launch_count()
     sampler = ClockSampler(torch.cuda.current_device() if world == 1 else int(os.environ.get("LOCAL_RANK", 0)))
     sampler.start()
     time.sleep(0.3)
@@ -213,30 +259,39 @@ def our_arm(args, rank, world, device):
         torch.distributed.barrier()
     torch.cuda.synchronize()
     wall0 = time.perf_counter()
+    launches0 = qg.qg_launch_count()
     for k in range(args.steps):
         flush.fill_(k & 0xFF)           # L2 flush outside the step's events
-        run_step(qg, layers, ev_steps[k])
+        ev_step[k][0].record()
+        if graph is not None:
+            graph.replay()
+        else:
+            run_step(qg, layers)
+        ev_step[k][1].record()
     torch.cuda.synchronize()
     if world > 1:
         torch.distributed.barrier()
     wall = time.perf_counter() - wall0
+    launches = (launches_per_step * args.steps if graph is not None
+                else qg.qg_launch_count() - launches0)
+    for k in range(args.steps):         # region 2
+        flush.fill_(k & 0xFF)
+        run_step(qg, layers, ev_steps[k])
+    torch.cuda.synchronize()
     clocks = sampler.stop()
-    launches = qg.qg_launch_count() - launches0
     for L in layers:
         for ws in L.workspaces():
             qg.check_status(ws, f"timed {L.name}")
 
-    # per step and per kernel device times (ms)
-    step_ms = [sum(ev[i][0].elapsed_time(ev[i][4]) for i in range(n_l)) for ev in ev_steps]
+    step_ms = [a.elapsed_time(b) for a, b in ev_step]
     per_kernel = {k: [] for k in KERNELS}
     per_kernel_layer = {k: [[] for _ in range(n_l)] for k in KERNELS}
     for ev in ev_steps:
         for i in range(n_l):
-            for j, k in enumerate(KERNELS):
-                t = ev[i][j].elapsed_time(ev[i][j + 1])
-                per_kernel_layer[k][i].append(t)
-        for k in KERNELS:
-            per_kernel[k].append(sum(per_kernel_layer[k][i][-1] for i in range(n_l)))
+            for j, kn in enumerate(KERNELS):
+                per_kernel_layer[kn][i].append(ev[i][j].elapsed_time(ev[i][j + 1]))
+        for kn in KERNELS:
+            per_kernel[kn].append(sum(per_kernel_layer[kn][i][-1] for i in range(n_l)))
     total_ms = max_over_ranks(sum(step_ms), world, device)
     ms_per_step = total_ms / args.steps
     flops_step = sum(L.flops for L in layers)
@@ -298,6 +353,8 @@ def our_arm(args, rank, world, device):
         "roofline": roofline,
         "clocks": clocks,
         "gpu_launches": int(launches),
+        "cuda_graph": graph is not None,
+        "breakdown_ms_per_step": round(sum(sum(v) for v in per_kernel.values()) / args.steps, 4),
         "wall_s": round(wall, 3),
     }
     if not args.no_e2e:
@@ -697,6 +754,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="launch the timed steps eagerly instead of replaying a captured CUDA graph")
     ap.add_argument("--alpha", type=float, default=None,
                     help="quantile of the clamp (default: the workload's first)")
     ap.add_argument("--quantizer-sweep", action="store_true",
