@@ -124,13 +124,13 @@ spmm_slice_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restrict
 // position is a compile-time index: the entry loop is unrolled by kDepth),
 // and each bf16 pair feeds one packed fp32x2 FMA (one rounding per
 // product-sum, as fmaf) on accumulators kept as 64-bit register pairs.
-// A warp owns 4 consecutive rows, whose CSR entries form one contiguous
+// A warp owns RPW consecutive rows, whose CSR entries form one contiguous
 // range consumed in order.
 constexpr int kStreamWarps = 8;
-#ifndef QG_SPMM_RPW
-#define QG_SPMM_RPW 4
-#endif
-constexpr int kStreamRowsPerWarp = QG_SPMM_RPW;   // consecutive rows owned by one warp
+// A warp owns RPW consecutive rows (4, 2 or 1): the launcher takes the
+// largest RPW that still gives every SM eight CTAs' worth of work, so narrow
+// or short problems get more, smaller CTAs.
+constexpr int kStreamMaxRowsPerWarp = 4;
 #ifndef QG_SPMM_PARTS
 #define QG_SPMM_PARTS 4
 #endif
@@ -168,7 +168,7 @@ __device__ __forceinline__ void fma_bf16x2(uint64_t& acc, uint64_t vv, uint32_t 
 
 // FULL: every quarter of the slice is inside N (all slices but the last when
 // N is not a multiple of the slice width), so loads and stores need no checks.
-template <bool FULL>
+template <int RPW, bool FULL>
 __device__ __forceinline__ void spmm_stream_body(const int32_t* __restrict__ row_ptr,
                                                  const int32_t* __restrict__ col,
                                                  const double* __restrict__ val,
@@ -176,15 +176,15 @@ __device__ __forceinline__ void spmm_stream_body(const int32_t* __restrict__ row
                                                  int M, int N, float* __restrict__ C) {
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
-    const int r_begin = (blockIdx.x * kStreamWarps + warp) * kStreamRowsPerWarp;
+    const int r_begin = (blockIdx.x * kStreamWarps + warp) * RPW;
     if (r_begin >= M) return;
-    const int r_end = min(M, r_begin + kStreamRowsPerWarp);
+    const int r_end = min(M, r_begin + RPW);
     const int nbase = blockIdx.y * kStreamSlice + lane * 8;   // quarter h: nbase + 256 h
     bool okh[kStreamParts];
 #pragma unroll
     for (int h = 0; h < kStreamParts; ++h) okh[h] = FULL || nbase + 256 * h < N;
     const uint16_t* wl = W + nbase;
-    // row_ptr[r_begin .. r_end] held by lanes 0..4
+    // row_ptr[r_begin .. r_end] held by lanes 0 .. RPW
     const int rp = (lane <= r_end - r_begin) ? row_ptr[r_begin + lane] : 0;
     const int P0 = __shfl_sync(0xFFFFFFFFu, rp, 0);
     const int n = __shfl_sync(0xFFFFFFFFu, rp, r_end - r_begin) - P0;
@@ -273,14 +273,15 @@ __device__ __forceinline__ void spmm_stream_body(const int32_t* __restrict__ row
     }
 }
 
+template <int RPW>
 __global__ void __launch_bounds__(kStreamWarps * 32, 2)
 spmm_stream_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col,
                    const double* __restrict__ val, const uint16_t* __restrict__ W, int64_t ldw,
                    int M, int N, float* __restrict__ C) {
     if ((int)(blockIdx.y + 1) * kStreamSlice <= N)
-        spmm_stream_body<true>(row_ptr, col, val, W, ldw, M, N, C);
+        spmm_stream_body<RPW, true>(row_ptr, col, val, W, ldw, M, N, C);
     else
-        spmm_stream_body<false>(row_ptr, col, val, W, ldw, M, N, C);
+        spmm_stream_body<RPW, false>(row_ptr, col, val, W, ldw, M, N, C);
 }
 
 cudaError_t spmm_setup() { return cudaSuccess; }
@@ -289,11 +290,18 @@ void launch_spmm(const qg_csr* dA, int64_t M, const void* W, qg_dtype dt, int64_
                  float* C, uint32_t* status, cudaStream_t s) {
     (void)status;   // no device-side waits that could time out
     if (dt == QG_BF16 && (N % 8) == 0 && (ldw % 8) == 0) {
-        const int rows_per_cta = kStreamWarps * kStreamRowsPerWarp;
-        dim3 grid((unsigned)((M + rows_per_cta - 1) / rows_per_cta),
-                  (unsigned)((N + kStreamSlice - 1) / kStreamSlice));
-        spmm_stream_kernel<<<grid, kStreamWarps * 32, 0, s>>>(
-            dA->row_ptr, dA->col, dA->val, static_cast<const uint16_t*>(W), ldw, (int)M, (int)N, C);
+        const int64_t slices = (N + kStreamSlice - 1) / kStreamSlice;
+        const int64_t want = 8 * (int64_t)num_sms();
+        int rpw = kStreamMaxRowsPerWarp;
+        while (rpw > 1 && ((M + kStreamWarps * rpw - 1) / (kStreamWarps * rpw)) * slices < want) rpw /= 2;
+        dim3 grid((unsigned)((M + kStreamWarps * rpw - 1) / (kStreamWarps * rpw)), (unsigned)slices);
+        const uint16_t* Wb = static_cast<const uint16_t*>(W);
+        if (rpw == 4)
+            spmm_stream_kernel<4><<<grid, kStreamWarps * 32, 0, s>>>(dA->row_ptr, dA->col, dA->val, Wb, ldw, (int)M, (int)N, C);
+        else if (rpw == 2)
+            spmm_stream_kernel<2><<<grid, kStreamWarps * 32, 0, s>>>(dA->row_ptr, dA->col, dA->val, Wb, ldw, (int)M, (int)N, C);
+        else
+            spmm_stream_kernel<1><<<grid, kStreamWarps * 32, 0, s>>>(dA->row_ptr, dA->col, dA->val, Wb, ldw, (int)M, (int)N, C);
         count_launch(1);
         return;
     }
