@@ -231,7 +231,6 @@ def our_arm(args, rank, world, device):
     idx = range(len(wl.layers)) if args.layer is None else [args.layer]
     layers = [Layer(qg, wl, i, device, args.alpha) for i in idx]
     flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
-    stream = torch.cuda.current_stream()
 
     for _ in range(args.warmup):
         run_step(qg, layers)
