@@ -640,3 +640,21 @@ def test_mx_pipeline_full_size_sampled(qg, wl, layer):
     rows = np.unique(np.concatenate([np.random.default_rng(M + N).integers(0, M, 16), [0, M - 1]]))
     Yo = oracle.mx_gemm(oc, os_, oT, osT, K, rows=rows)
     assert y_rel_err(_np(Y)[rows], Yo) <= 1e-3
+
+
+def test_mx_quantizers_flag_nonfinite(qg):
+    """A NaN or Inf in a block sets the workspace status (reported as
+    QG_ERR_NONFINITE) in both MX quantizers; finite inputs leave it clean."""
+    A = make_matrix((64, 256), seed=5, device="cuda", dtype=torch.bfloat16)
+    ws = qg.Workspace(qg.QG_OP_QUANTIZE_ROWS, 64, 256, 1, qg.QG_BF16)
+    qg.mx_quantize_rows(A, ws=ws)
+    assert qg.qg_sync_status(ws) == qg.QG_OK
+    for bad in (float("nan"), float("inf")):
+        B = A.clone()
+        B[7, 100] = bad
+        qg.mx_quantize_rows(B, ws=ws)
+        assert qg.qg_sync_status(ws) == qg.QG_ERR_NONFINITE
+        qg.mx_quantize_cols(B, ws=ws)
+        assert qg.qg_sync_status(ws) == qg.QG_ERR_NONFINITE
+    qg.mx_quantize_cols(A, ws=ws)
+    assert qg.qg_sync_status(ws) == qg.QG_OK
