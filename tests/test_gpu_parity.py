@@ -423,7 +423,7 @@ def test_fp4_linear_small(qg, wl, layer, M):
 
 @pytest.mark.parametrize("wl,layer", [("llama1.3b", 1), ("llama7b", 1), ("llama13b", 4)])
 def test_fp4_linear_full_size_sampled(qg, wl, layer):
-    """Full BASELINE sizes, the launch configuration the benchmark times:
+    """Full workload sizes, the launch configuration the benchmark times:
     T, codes, scales and dA checked exactly over the whole tensor, Y on a
     sample of rows computed by the oracle one by one."""
     A, W = make_layer_inputs(wl, layer, device="cuda")
