@@ -153,3 +153,44 @@ def test_mx_scale_layout_host(qg):
                                    None) == qg.QG_ERR_INVALID_ARG
     assert lib.qg_mx_gemm(fake, fake, fake, fake, 128, 128, 256, None, None, 0, None, fake,
                           1 << 20, None) == qg.QG_ERR_INVALID_ARG
+
+
+C_CLIENT = r"""
+#include <stdio.h>
+#include "qgemm.h"
+int main(void) {
+    printf("%s\n", qg_status_string(QG_ERR_TIMEOUT));
+    printf("%lld\n", (long long)qg_quantile_rank(0.99, 1000));
+    printf("%zu\n", qg_workspace_size(QG_OP_FP4_LINEAR, 4096, 2048, 5504, QG_BF16, 0.99));
+    printf("%zu\n", qg_mx_scale_bytes(300, 5504));
+    /* rejected on the host before any CUDA call: K not a multiple of 32 */
+    printf("%d\n", (int)qg_quantize_rows((const void*)0x100000, QG_BF16, 4, 48, 48,
+                                         (uint8_t*)0x100000, (float*)0x100000,
+                                         (void*)0x100000, 1 << 20, (cudaStream_t)0));
+    return 0;
+}
+"""
+
+
+def test_header_is_plain_c_and_links(qg, tmp_path):
+    """include/qgemm.h compiles as C99 with warnings as errors, and a C
+    program linked against libqgemm.so gets the same host-side answers as the
+    Python binding (no device needed)."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    src = tmp_path / "client.c"
+    src.write_text(C_CLIENT)
+    exe = tmp_path / "client"
+    inc = os.path.join(ROOT, "include")
+    libdir = os.path.dirname(qg.LIB_PATH)
+    subprocess.check_call([cc, "-std=c99", "-Wall", "-Wextra", "-Werror", "-I", inc, str(src),
+                           "-o", str(exe), "-L", libdir, "-lqgemm", f"-Wl,-rpath,{libdir}"])
+    out = subprocess.check_output([str(exe)], text=True).splitlines()
+    assert out[0] == qg.qg_status_string(qg.QG_ERR_TIMEOUT)
+    assert int(out[1]) == qg.qg_quantile_rank(0.99, 1000)
+    assert int(out[2]) == qg.qg_workspace_size(qg.QG_OP_FP4_LINEAR, 4096, 2048, 5504, qg.QG_BF16, 0.99)
+    assert int(out[3]) == qg.qg_mx_scale_bytes(300, 5504)
+    assert int(out[4]) == qg.QG_ERR_UNSUPPORTED_SHAPE
