@@ -462,45 +462,79 @@ def _ncu_traffic(kernel, workload):
 
 
 # ------------------------------------------------------------------ CPU oracle
-def _oracle_sample(wl, A_list, W_list, rows_per_layer, alpha=None):
-    """Run the oracle on a bounded sample of one step: the full quantizers on
-    every layer, Y for `rows_per_layer` rows of each layer.  Returns (seconds,
-    flops the sample stands for after scaling the Y rows to M)."""
+def _oracle_sample(wl, A_list, W_list, frac, alpha=None, step=0):
+    """Time the oracle on a bounded sample of one step and return the seconds
+    the whole step would take.  For each layer a fraction `frac` of the work:
+    the activation quantizer (threshold, clamp, dA, row codes) on a slice of
+    about frac * M rows, the W quantizer on about frac * N columns, Y for about
+    frac * M evenly spaced rows; each part's time is scaled by its inverse
+    fraction.  `step` rotates the slices through the tensors.  frac = 1 runs
+    the quantizers on the full tensors (Y is then sampled by `_Y_ROWS_FULL`)."""
     import oracle
     t_total = 0.0
     alpha = wl.alphas[0] if alpha is None else alpha
     for A, W in zip(A_list, W_list):
         M, K = A.shape
         N = W.shape[1]
+        ra = M if frac >= 1 else max(32, min(M, int(round(frac * M))))
+        cs = N if frac >= 1 else max(32, min(N, int(round(frac * N))))
+        ry = _Y_ROWS_FULL if frac >= 1 else max(1, min(M, int(round(frac * M))))
+        r0 = (step * ra) % (M - ra + 1)
+        c0 = (step * cs) % (N - cs + 1)
+        A_s = A[r0:r0 + ra]
+        W_s = W if cs == N else np.ascontiguousarray(W[:, c0:c0 + cs])
         t0 = time.perf_counter()
-        act = oracle.quantize_act(A, alpha)
-        oT, ot = oracle.quantize_cols(W)
+        act = oracle.quantize_act(A_s, alpha)
         t1 = time.perf_counter()
-        rows = np.linspace(0, M - 1, rows_per_layer).astype(np.int64)
+        oracle.quantize_cols(W_s)
+        t2 = time.perf_counter()
+        # Y needs the codes of all N columns; their time is the W quantizer's,
+        # already sampled above, so the full-column codes are made untimed.
+        oT, ot = _codes_cache(W)
+        rows = (np.linspace(0, ra - 1, ry).astype(np.int64) + step) % ra
+        t3 = time.perf_counter()
         acc = oracle.gemm_acc(act["codes"], oT, K, rows=rows)
         oracle.linear_y(acc, act["scales"], ot, act["row_ptr"], act["col"], act["val"], W, rows=rows)
-        t2 = time.perf_counter()
-        t_total += (t1 - t0) + (t2 - t1) * (M / rows_per_layer)
+        t4 = time.perf_counter()
+        t_total += (t1 - t0) * (M / ra) + (t2 - t1) * (N / cs) + (t4 - t3) * (M / ry)
     return t_total
+
+
+_Y_ROWS_FULL = 16
+_CODES = {}
+
+
+def _codes_cache(W):
+    """The oracle's column codes of W, computed once per weight."""
+    import oracle
+    key = id(W)
+    if key not in _CODES:
+        _CODES[key] = oracle.quantize_cols(W)
+    return _CODES[key]
 
 
 def cpu_baseline(args, wl, layers):
     import oracle
     A_list = [oracle.as_f32(L.A.cpu()) for L in layers]
     W_list = [oracle.as_f32(L.W.cpu()) for L in layers]
-    rows = 16
-    t_est = _oracle_sample(wl, A_list, W_list, rows, layers[0].alpha)
+    t_est = _oracle_sample(wl, A_list, W_list, 1.0, layers[0].alpha)
     flops = sum(L.flops for L in layers)
     return {"value": round(flops / t_est / 1e12, 6), "unit": "TFLOP/s",
             "cores": oracle.num_threads(), "kind": "oracle",
             "sample": (f"one step of {wl.name}: quantizers (threshold, clamp, dA, row and "
-                       f"column codes) on the full tensors; Y for {rows} evenly spaced rows per "
-                       f"layer, its time scaled by M/{rows}"),
+                       f"column codes) on the full tensors; Y for {_Y_ROWS_FULL} evenly spaced "
+                       f"rows per layer, its time scaled by M/{_Y_ROWS_FULL}"),
             "seconds_per_step_estimate": round(t_est, 3)}
 
 
+REFERENCE_BUDGET_S = 150.0   # wall time the reference arm's warm-up + timed steps aim for
+
+
 def reference_arm(args, rank, world):
-    """The CPU oracle as the reference arm (rank 0 only)."""
+    """The CPU oracle as the reference arm (rank 0 only).  Every step times the
+    oracle on a sample of the step whose size is set so that the W warm-up and
+    K timed steps together take about REFERENCE_BUDGET_S seconds; the value is
+    the step's FLOPs over the step time the samples stand for."""
     from workloads import WORKLOADS, make_layer_inputs
     import oracle
     wl = WORKLOADS[args.workload]
@@ -510,21 +544,34 @@ def reference_arm(args, rank, world):
         A, W = make_layer_inputs(wl, i, device="cpu")
         A_list.append(oracle.as_f32(A))
         W_list.append(oracle.as_f32(W))
-    rows = 8
-    warm = min(args.warmup, 1)        # the oracle needs no warm-up beyond one pass
-    for _ in range(warm):
-        _oracle_sample(wl, A_list, W_list, rows, args.alpha)
+    for W in W_list:
+        _codes_cache(W)
+    # calibrate: one small sample gives the full step's estimated time
+    probe = 1.0 / 256
+    t_step = _oracle_sample(wl, A_list, W_list, probe, args.alpha)
+    n_runs = max(1, args.steps + args.warmup)
+    frac = min(1.0, REFERENCE_BUDGET_S / n_runs / max(t_step, 1e-9))
+    for s in range(args.warmup):
+        _oracle_sample(wl, A_list, W_list, frac, args.alpha, step=s)
     total = 0.0
-    for _ in range(args.steps):
-        total += _oracle_sample(wl, A_list, W_list, rows, args.alpha)
+    for s in range(args.steps):
+        total += _oracle_sample(wl, A_list, W_list, frac, args.alpha, step=args.warmup + s)
     flops = sum(2 * wl.M * wl.layers[i].K * wl.layers[i].N for i in idx)
     value = flops * args.steps / total / 1e12
     cores = oracle.num_threads()
-    sample = (f"each step: quantizers on the full tensors of every {wl.name} layer, Y for "
-              f"{rows} evenly spaced rows per layer with its time scaled by M/{rows}")
+    if frac >= 1:
+        sample = (f"each step: quantizers on the full tensors of every {wl.name} layer, Y for "
+                  f"{_Y_ROWS_FULL} evenly spaced rows per layer with its time scaled by "
+                  f"M/{_Y_ROWS_FULL}")
+    else:
+        sample = (f"each step: on every {wl.name} layer, a fraction {frac:.3g} of the work "
+                  f"(activation quantizer on a slice of >= 32 rows, W quantizer on >= 32 "
+                  f"columns, Y for >= 1 row; slices rotate across steps), each part's time "
+                  f"scaled by its inverse fraction; sized so the {args.warmup} + {args.steps} "
+                  f"steps take about {REFERENCE_BUDGET_S:.0f} s")
     return {
         "impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s",
-        "n_gpus": world, "steps": args.steps, "warmup": warm,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
         "ms_per_step": round(1e3 * total / args.steps, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": wl.name if args.layer is None else f"{wl.name}:{wl.layers[idx[0]].name}",
