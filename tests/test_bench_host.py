@@ -69,3 +69,29 @@ def test_workload_generator_is_seeded_and_shaped():
     A3, _ = make_layer_inputs("llama1.3b", 0, device="cpu", M=64)
     assert A3.dtype == torch.bfloat16 and A3.shape == (64, 2048)
     assert seed_for(WORKLOADS["llama7b"], 3) == 2003
+
+
+def _ref_args(steps, warmup):
+    import argparse
+    return argparse.Namespace(workload="tiny", layer=None, steps=steps, warmup=warmup, alpha=None)
+
+
+@pytest.mark.parametrize("budget", [bench.REFERENCE_BUDGET_S, 1e-3])
+def test_reference_arm_line_and_bounded_sample(monkeypatch, budget):
+    """The reference arm (the oracle on the host) prints the contract's fields;
+    with a tiny time budget every step falls back to the smallest sample (32-row
+    and 32-column slices, one Y row per layer) and still reports the metric."""
+    monkeypatch.setattr(bench, "REFERENCE_BUDGET_S", budget)
+    line = bench.reference_arm(_ref_args(steps=4, warmup=3), 0, 1)
+    for key in ("impl", "metric", "value", "unit", "n_gpus", "steps", "warmup", "ms_per_step",
+                "higher_is_better", "config", "cpu_baseline", "e2e"):
+        assert key in line
+    assert line["impl"] == "reference" and line["steps"] == 4 and line["warmup"] == 3
+    assert line["value"] > 0 and line["e2e"]["value"] == line["value"]
+    assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
+    assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    sample = line["cpu_baseline"]["sample"]
+    if budget < 1:
+        assert "fraction" in sample
+    else:
+        assert "full tensors" in sample
