@@ -789,6 +789,44 @@ def mx_sweep(device, workload, reps=20, warm=5):
         torch.cuda.empty_cache()
 
 
+def fp4_peak_sweep(device, reps=10, warm=3, iters=1 << 16):
+    """The tensor pipe's E2M1 rate from the library's MMA-only loop
+    (qg_fp4_mma_loop: operands in shared memory, the GEMM's MMA shape, no
+    global traffic), one CTA per SM and 2-SM pairs; median of `reps` CUDA-event
+    timings on the launching stream, clocks sampled meanwhile.  One JSON line
+    per form, with the ratio to the FP4 denominator the other lines use
+    (4 x the measured sustained bf16 rate)."""
+    import quantize_gemm_b200 as qg
+    peaks = _peaks()
+    fp4_denominator = 4.0 * peaks["bf16_tflops_sustained"]
+    ws = qg.Workspace(qg.QG_OP_FP4_GEMM, 1, 32, 1, qg.QG_F32, device=device)
+    stream = torch.cuda.current_stream(device)
+    for pair in (False, True):
+        for _ in range(warm):
+            qg.fp4_mma_loop(iters, pair, ws, stream=stream)
+        clocks = ClockSampler(device.index or 0)
+        clocks.start()
+        ts, flops = [], 0.0
+        for _ in range(reps):
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            flops = qg.fp4_mma_loop(iters, pair, ws, stream=stream)
+            b.record(stream)
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        clk = clocks.stop()
+        qg.check_status(ws, "fp4 mma loop")
+        ts.sort()
+        ms = ts[len(ts) // 2]
+        tf = flops / (ms * 1e-3) / 1e12
+        line = {"sweep": "fp4_peak", "form": "2-SM pairs (cta_group::2)" if pair else "one CTA per SM",
+                "mma": "256 x 224 x 64" if pair else "128 x 224 x 64", "iters": iters,
+                "reps": reps, "ms": round(ms, 4), "TFLOP/s": round(tf, 1),
+                "ratio_to_4x_bf16_sustained": round(tf / fp4_denominator, 4),
+                "fp4_denominator_tflops": fp4_denominator, "clocks": clk}
+        print(json.dumps(line), flush=True)
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -810,6 +848,9 @@ def main():
     ap.add_argument("--mx", action="store_true",
                     help="time the MXFP4 block-scaled quantizers and GEMM on each linear of "
                          "--workload (one JSON line per linear) instead of the layer stream")
+    ap.add_argument("--fp4-peak", action="store_true",
+                    help="time the library's MMA-only tensor-pipe loop (E2M1 rate of the tensor "
+                         "cores, solo and 2-SM pairs) instead of the layer stream")
     ap.add_argument("--grads", action="store_true",
                     help="time forward, dgrad and wgrad of each linear of --workload (one JSON "
                          "line per linear) instead of the layer stream")
@@ -837,10 +878,12 @@ def main():
     import __graft_entry__
     if rank == 0:
         __graft_entry__.build()
-    if args.quantizer_sweep or args.grads or args.mx:
+    if args.quantizer_sweep or args.grads or args.mx or args.fp4_peak:
         if rank == 0:
             if args.quantizer_sweep:
                 quantizer_sweep(device)
+            elif args.fp4_peak:
+                fp4_peak_sweep(device)
             elif args.mx:
                 mx_sweep(device, args.workload)
             else:

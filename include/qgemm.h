@@ -281,6 +281,22 @@ qg_status qg_mx_gemm(const uint8_t* codesA, const uint8_t* sA, const uint8_t* co
                      qg_dtype y_dtype, float* raw_acc, void* ws, size_t ws_bytes,
                      cudaStream_t stream);
 
+/* ---- tensor-pipe E2M1 rate (measurement) -----------------------------------
+ * The ceiling of qg_fp4_gemm's mainloop ([FP4-writeup], FP4 GEMM paragraph:
+ * the matrix product is the part FP4 accelerates).  One launch over the whole
+ * GPU: every SM (pair != 0: every 2-SM cluster that can be resident, 2-SM MMA)
+ * issues iters x 4 block-scaled E2M1 MMAs of the GEMM's shape, 128 x 224 x 64
+ * per SM (256 x 224 x 64 per pair), on operands that stay in shared memory,
+ * accumulating in TMEM; no global memory is read or written besides the
+ * status word.  Time the launch with CUDA events on `stream`; *flops_out
+ * (host pointer) receives the MMA flops of the launch, 2 x 128 x 224 x 64 x 4
+ * x iters per CTA.  1 <= iters <= 2^20 (else QG_ERR_INVALID_ARG; 2^20 takes
+ * about a quarter of a second).  ws: qg_workspace_size(QG_OP_FP4_GEMM, 1, 32,
+ * 1, QG_F32, 1.0) bytes at least; a completion wait that runs out (~2 s of SM
+ * clocks) sets the timeout bit (QG_ERR_TIMEOUT from qg_sync_status). */
+qg_status qg_fp4_mma_loop(int64_t iters, int pair, double* flops_out, void* ws, size_t ws_bytes,
+                          cudaStream_t stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -41,7 +41,7 @@ EXPORTED = (
     "qg_quantize_rows", "qg_quantize_cols", "qg_clamp_compensate", "qg_quantize_act",
     "qg_spmm_correction", "qg_fp4_gemm", "qg_fp4_linear", "qg_launch_count",
     "qg_quantize_cols_static", "qg_fp4_dgrad", "qg_fp4_wgrad", "qg_mx_scale_bytes",
-    "qg_mx_quantize_rows", "qg_mx_quantize_cols", "qg_mx_gemm",
+    "qg_mx_quantize_rows", "qg_mx_quantize_cols", "qg_mx_gemm", "qg_fp4_mma_loop",
 )
 
 
@@ -91,6 +91,7 @@ _sig("qg_mx_scale_bytes", _SZ, [_I64, _I64])
 _sig("qg_mx_quantize_rows", _INT, [_P, _INT, _I64, _I64, _I64, _P, _P, _P, _SZ, _P])
 _sig("qg_mx_quantize_cols", _INT, [_P, _INT, _I64, _I64, _I64, _P, _P, _P, _SZ, _P])
 _sig("qg_mx_gemm", _INT, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _INT, _P, _P, _SZ, _P])
+_sig("qg_fp4_mma_loop", _INT, [_I64, _INT, ctypes.POINTER(_D), _P, _SZ, _P])
 _sig("qg_fp4_dgrad", _INT, [_P, _INT, _I64, _I64, _P, _INT, _I64, _P, _INT, _P, _SZ, _P])
 _sig("qg_fp4_wgrad", _INT, [_P, _INT, _I64, _I64, _P, _INT, _I64, _P, _INT, _P, _SZ, _P])
 
@@ -311,6 +312,14 @@ def qg_mx_gemm(codesA, sA, codesWT, sW, M, N, K, C, Y, raw_acc, ws: Workspace, s
                            _ptr(Y), y_dt, _ptr(raw_acc), ws.ptr, ws.nbytes, _stream(stream))
 
 
+def qg_fp4_mma_loop(iters: int, pair: bool, ws: Workspace, stream=None):
+    """(status, MMA flops of the launch)."""
+    flops = _D(0.0)
+    st = _lib.qg_fp4_mma_loop(int(iters), 1 if pair else 0, ctypes.byref(flops), ws.ptr, ws.nbytes,
+                              _stream(stream))
+    return st, flops.value
+
+
 def mx_scale_index(rows: int, K: int, device="cpu") -> torch.Tensor:
     """Byte offset, in the GEMM's scale-atom layout, of the scale of row r and
     32-block j, as a rows x K/32 int64 tensor (layout bookkeeping only)."""
@@ -457,6 +466,15 @@ def mx_gemm(codesA, sA, codesWT, sW, K: int, C=None, out_dtype=torch.float32, ra
     acc = torch.empty((M, N), dtype=torch.float32, device=codesA.device) if raw else None
     _check(qg_mx_gemm(codesA, sA, codesWT, sW, M, N, K, C, Y, acc, ws), "qg_mx_gemm")
     return (Y, acc) if raw else Y
+
+
+def fp4_mma_loop(iters: int, pair: bool = True, ws: Optional[Workspace] = None, stream=None) -> float:
+    """Enqueue the tensor-pipe E2M1 MMA loop; returns its flops (time it with
+    CUDA events on `stream`)."""
+    ws = ws or Workspace(QG_OP_FP4_GEMM, 1, 32, 1, QG_F32)
+    st, flops = qg_fp4_mma_loop(iters, pair, ws, stream)
+    _check(st, "qg_fp4_mma_loop")
+    return flops
 
 
 def check_status(ws: Workspace, where: str = "device status", stream=None):

@@ -36,6 +36,8 @@ static cudaError_t ensure_device(int* dev_out) {
         if (e != cudaSuccess) return e;
         e = spmm_setup();
         if (e != cudaSuccess) return e;
+        e = mma_peak_setup();
+        if (e != cudaSuccess) return e;
         g_sms[dev] = sms;
         g_ready[dev] = true;
     }
@@ -454,6 +456,17 @@ qg_status qg_mx_gemm(const uint8_t* codesA, const uint8_t* sA, const uint8_t* co
     if (ensure_device(nullptr) != cudaSuccess) return QG_ERR_CUDA;
     return cuda_status(launch_fp4_gemm_mx(codesA, sA, codesWT, sW, M, N, K, C, Y, y_dtype, raw_acc,
                                           at<uint32_t>(ws, L.status), stream));
+}
+
+qg_status qg_fp4_mma_loop(int64_t iters, int pair, double* flops_out, void* ws, size_t ws_bytes,
+                          cudaStream_t stream) {
+    if (iters < 1 || iters > ((int64_t)1 << 20) || flops_out == nullptr) return QG_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(QG_OP_FP4_GEMM, 1, 32, 1, QG_F32, 1.0);
+    qg_status st = check_ws(ws, ws_bytes, L.total);
+    if (st != QG_OK) return st;
+    if (ensure_device(nullptr) != cudaSuccess) return QG_ERR_CUDA;
+    return cuda_status(launch_fp4_mma_loop(iters, pair != 0, flops_out, at<uint32_t>(ws, L.status),
+                                           stream));
 }
 
 }  // extern "C"

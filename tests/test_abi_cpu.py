@@ -155,6 +155,24 @@ def test_mx_scale_layout_host(qg):
                           1 << 20, None) == qg.QG_ERR_INVALID_ARG
 
 
+
+def test_mma_loop_host_checks(qg):
+    """The tensor-pipe loop rejects out-of-range iteration counts, a missing
+    flops pointer and a short workspace before anything is enqueued."""
+    lib = qg._lib
+    P = ctypes.c_void_p
+    fake = P(1 << 20)
+    flops = ctypes.c_double(-1.0)
+    ws_need = qg.qg_workspace_size(qg.QG_OP_FP4_GEMM, 1, 32, 1, qg.QG_F32, 1.0)
+    for iters in (0, -1, (1 << 20) + 1):
+        assert lib.qg_fp4_mma_loop(iters, 1, ctypes.byref(flops), fake, ws_need, None) == \
+            qg.QG_ERR_INVALID_ARG
+    assert lib.qg_fp4_mma_loop(16, 0, None, fake, ws_need, None) == qg.QG_ERR_INVALID_ARG
+    assert lib.qg_fp4_mma_loop(16, 0, ctypes.byref(flops), fake, ws_need - 256, None) == \
+        qg.QG_ERR_WORKSPACE
+    assert flops.value == -1.0   # nothing written on a rejected call
+
+
 C_CLIENT = r"""
 #include <stdio.h>
 #include "qgemm.h"
