@@ -36,8 +36,6 @@ static cudaError_t ensure_device(int* dev_out) {
         if (e != cudaSuccess) return e;
         e = spmm_setup();
         if (e != cudaSuccess) return e;
-        e = mma_peak_setup();
-        if (e != cudaSuccess) return e;
         g_sms[dev] = sms;
         g_ready[dev] = true;
     }

@@ -194,22 +194,23 @@ fp4_mma_loop_kernel(long long iters, uint32_t* status) {
     }
 }
 
-}  // namespace peak
-
-cudaError_t mma_peak_setup() {
-    cudaError_t e = cudaFuncSetAttribute(peak::fp4_mma_loop_kernel<false>,
-                                         cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)peak::kSmemBytes);
-    if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(peak::fp4_mma_loop_kernel<true>,
-                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)peak::kSmemBytes);
+// The shared-memory size is set here, on use, rather than in the library's
+// device setup, which the layer's calls share.
+static cudaError_t set_smem_attr(bool pair) {
+    return cudaFuncSetAttribute(pair ? (const void*)fp4_mma_loop_kernel<true>
+                                     : (const void*)fp4_mma_loop_kernel<false>,
+                                cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
 }
+
+}  // namespace peak
 
 // One launch over the whole GPU: a CTA per SM (pair: as many 2-CTA clusters as
 // can be resident at once).  *flops = 2 x 128 x 224 x 64 x 4 x iters per CTA.
 cudaError_t launch_fp4_mma_loop(int64_t iters, bool pair, double* flops, uint32_t* status,
                                 cudaStream_t s) {
     using namespace peak;
+    cudaError_t e = set_smem_attr(pair);
+    if (e != cudaSuccess) return e;
     cudaLaunchConfig_t cfg = {};
     cfg.blockDim = dim3(kThreads);
     cfg.dynamicSmemBytes = kSmemBytes;
@@ -225,13 +226,13 @@ cudaError_t launch_fp4_mma_loop(int64_t iters, bool pair, double* flops, uint32_
     if (pair) {
         cfg.gridDim = dim3(2);
         int clusters = 0;
-        cudaError_t e = cudaOccupancyMaxActiveClusters(&clusters, fp4_mma_loop_kernel<true>, &cfg);
+        e = cudaOccupancyMaxActiveClusters(&clusters, fp4_mma_loop_kernel<true>, &cfg);
         if (e != cudaSuccess) return e;
         if (clusters < 1) return cudaErrorInvalidConfiguration;
         ctas = std::min(2 * clusters, ctas / 2 * 2);
     }
     cfg.gridDim = dim3((unsigned)ctas);
-    cudaError_t e = pair ? cudaLaunchKernelEx(&cfg, fp4_mma_loop_kernel<true>, (long long)iters, status)
+    e = pair ? cudaLaunchKernelEx(&cfg, fp4_mma_loop_kernel<true>, (long long)iters, status)
                          : cudaLaunchKernelEx(&cfg, fp4_mma_loop_kernel<false>, (long long)iters, status);
     count_launch(1);
     if (flops) *flops = 2.0 * 128.0 * kBN * 64.0 * 4.0 * (double)iters * (double)ctas;

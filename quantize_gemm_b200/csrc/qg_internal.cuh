@@ -388,7 +388,6 @@ bool launch_quantize_cols_fused(const void* W, int64_t K, int64_t N, int64_t ldw
                                 uint32_t* status, cudaStream_t s);
 cudaError_t gemm_setup();
 cudaError_t spmm_setup();
-cudaError_t mma_peak_setup();
 // MMA-only loop on the tensor pipe (a CTA per SM, or 2-SM pairs); *flops gets
 // the MMA flops of the launch.
 cudaError_t launch_fp4_mma_loop(int64_t iters, bool pair, double* flops, uint32_t* status,
