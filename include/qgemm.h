@@ -180,8 +180,9 @@ qg_status qg_clamp_compensate(const void* A, qg_dtype dtype, int64_t M, int64_t 
                               void* ws, size_t ws_bytes, cudaStream_t stream);
 
 /* Fused activation quantizer: threshold, clamp, dA (CSR) and token-wise
- * quantization of A_clamped (amax_i = min(max_k |A_ik|, T)) in three passes
- * over A ([FP4-writeup], outlier + granularity + ScaleShift paragraphs).
+ * quantization of A_clamped (amax_i = min(max_k |A_ik|, T)), in two passes
+ * over A for bf16 input (one cooperative launch) and three for fp32
+ * ([FP4-writeup], outlier + granularity + ScaleShift paragraphs).
  * Outputs as qg_quantize_rows plus dA and T_out. */
 qg_status qg_quantize_act(const void* A, qg_dtype dtype, int64_t M, int64_t K, int64_t lda,
                           double alpha, uint8_t* codes, float* scales, const qg_csr* dA,
