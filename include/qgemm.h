@@ -162,7 +162,12 @@ qg_status qg_quantize_cols(const void* W, qg_dtype dtype, int64_t K, int64_t N, 
  *   - N > 65536 returns QG_ERR_UNSUPPORTED_SHAPE before anything is enqueued;
  *     other argument checks are those of qg_quantize_cols.
  *   - The first call on a device looks up the array's device address (a CUDA
- *     runtime query); make that first call before any stream capture.
+ *     runtime query); make that first call before any stream capture.  The
+ *     address is kept for the life of the process: after a cudaDeviceReset
+ *     it is stale, so do not call this entry point again after a reset.
+ *   - For either dtype it runs the two-pass kernels (column maxima, then the
+ *     codes) rather than the single cooperative bf16 kernel of
+ *     qg_quantize_cols: same results, somewhat slower on bf16 weights.
  *   - Every call on a GPU uses that GPU's one array and zeroes what it needs
  *     at the start; it keeps the last call's contents in between.  Calls
  *     whose executions overlap on the same GPU (for example on two streams)
@@ -207,13 +212,27 @@ qg_status qg_fp4_gemm(const uint8_t* codesA, const float* sA, const uint8_t* cod
 
 /* The whole layer: qg_quantize_act(A) -> qg_spmm_correction(dA, W) ->
  * qg_fp4_gemm(..., C) into Y (M x N, fp32 or bf16).  codesWT / sW come from
- * qg_quantize_cols(W); W is the unquantized weight used by the correction.
- * The activation codes, dA and C live in the workspace
- * (qg_workspace_size(QG_OP_FP4_LINEAR, ...)). */
+ * qg_quantize_cols(W); W is the unquantized weight used by the correction,
+ * K x N row-major and contiguous, stored in the SAME dtype as A (`dtype`
+ * describes both; the call has no separate weight dtype, so a weight in the
+ * other dtype is read wrongly without an error).  The activation codes, dA
+ * and C live in the workspace (qg_workspace_size(QG_OP_FP4_LINEAR, ...)). */
 qg_status qg_fp4_linear(const void* A, qg_dtype dtype, int64_t M, int64_t K,
                         const uint8_t* codesWT, const float* sW, const void* W, int64_t N,
                         double alpha, void* Y, qg_dtype y_dtype, void* ws, size_t ws_bytes,
                         cudaStream_t stream);
+
+/* Where qg_fp4_linear leaves its intermediate results inside a workspace
+ * sized for (M, K, N, dtype, alpha), as byte offsets from the workspace base
+ * (each a multiple of 256), for a caller that wants to inspect them after the
+ * call: parts[0] activation codes (M x K/2 bytes), parts[1] activation scales
+ * (M fp32), parts[2] dA row_ptr (M + 1 int32), parts[3] dA col (int32),
+ * parts[4] dA val (double), parts[5] the dA entry count (int64), parts[6] the
+ * threshold T (fp32).  `parts` is a host array of 7 elements.  Nothing is
+ * enqueued.  Errors: QG_ERR_INVALID_ARG (null parts, bad dtype or alpha),
+ * QG_ERR_UNSUPPORTED_SHAPE (as qg_fp4_linear). */
+qg_status qg_fp4_linear_parts(int64_t M, int64_t K, int64_t N, qg_dtype dtype, double alpha,
+                              size_t* parts);
 
 /* Backward GEMMs of the layer with FP4 operands (the training method also
  * runs the gradient GEMMs in FP4: [FP4-writeup], the paragraphs on the FP4
@@ -294,9 +313,17 @@ qg_status qg_mx_gemm(const uint8_t* codesA, const uint8_t* sA, const uint8_t* co
  * x iters per CTA.  1 <= iters <= 2^20 (else QG_ERR_INVALID_ARG; 2^20 takes
  * about a quarter of a second).  ws: qg_workspace_size(QG_OP_FP4_GEMM, 1, 32,
  * 1, QG_F32, 1.0) bytes at least; a completion wait that runs out (~2 s of SM
- * clocks) sets the timeout bit (QG_ERR_TIMEOUT from qg_sync_status). */
-qg_status qg_fp4_mma_loop(int64_t iters, int pair, double* flops_out, void* ws, size_t ws_bytes,
-                          cudaStream_t stream);
+ * clocks) sets the timeout bit (QG_ERR_TIMEOUT from qg_sync_status), and the
+ * kernel then waits once more (bounded) before it releases its TMEM.
+ * acc_out (nullable device pointer, 16-byte aligned, 128 x 224 fp32,
+ * row-major) receives CTA 0's accumulator after the last MMA, for checking the
+ * loop's products: the operand tiles are fixed functions of the CTA index
+ * (32-bit words h(i) = ((i * 2654435761 + cta) ^ (. >> 15)) * 2246822519 over
+ * the A tile, 128 rows of 128 bytes, then the W^T tile, 224 rows; 128-byte
+ * swizzle; a pair takes W^T rows 0..111 of CTA 0 and 0..111 of CTA 1), so
+ * acc = iters x (A tile . W^T tile^T) over their 256 E2M1 values per row. */
+qg_status qg_fp4_mma_loop(int64_t iters, int pair, double* flops_out, float* acc_out, void* ws,
+                          size_t ws_bytes, cudaStream_t stream);
 
 #ifdef __cplusplus
 }

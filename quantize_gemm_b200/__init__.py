@@ -42,6 +42,7 @@ EXPORTED = (
     "qg_spmm_correction", "qg_fp4_gemm", "qg_fp4_linear", "qg_launch_count",
     "qg_quantize_cols_static", "qg_fp4_dgrad", "qg_fp4_wgrad", "qg_mx_scale_bytes",
     "qg_mx_quantize_rows", "qg_mx_quantize_cols", "qg_mx_gemm", "qg_fp4_mma_loop",
+    "qg_fp4_linear_parts",
 )
 
 
@@ -87,11 +88,12 @@ _sig("qg_fp4_gemm", _INT,
      [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _INT, _P, _P, _SZ, _P])
 _sig("qg_fp4_linear", _INT,
      [_P, _INT, _I64, _I64, _P, _P, _P, _I64, _D, _P, _INT, _P, _SZ, _P])
+_sig("qg_fp4_linear_parts", _INT, [_I64, _I64, _I64, _INT, _D, ctypes.POINTER(_SZ)])
 _sig("qg_mx_scale_bytes", _SZ, [_I64, _I64])
 _sig("qg_mx_quantize_rows", _INT, [_P, _INT, _I64, _I64, _I64, _P, _P, _P, _SZ, _P])
 _sig("qg_mx_quantize_cols", _INT, [_P, _INT, _I64, _I64, _I64, _P, _P, _P, _SZ, _P])
 _sig("qg_mx_gemm", _INT, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _INT, _P, _P, _SZ, _P])
-_sig("qg_fp4_mma_loop", _INT, [_I64, _INT, ctypes.POINTER(_D), _P, _SZ, _P])
+_sig("qg_fp4_mma_loop", _INT, [_I64, _INT, ctypes.POINTER(_D), _P, _P, _SZ, _P])
 _sig("qg_fp4_dgrad", _INT, [_P, _INT, _I64, _I64, _P, _INT, _I64, _P, _INT, _P, _SZ, _P])
 _sig("qg_fp4_wgrad", _INT, [_P, _INT, _I64, _I64, _P, _INT, _I64, _P, _INT, _P, _SZ, _P])
 
@@ -268,6 +270,33 @@ def qg_fp4_linear(A, codesWT, sW, W, alpha, Y, ws: Workspace, stream=None) -> in
                               float(alpha), _ptr(Y), _dt(Y), ws.ptr, ws.nbytes, _stream(stream))
 
 
+def qg_fp4_linear_parts(M: int, K: int, N: int, dtype: int, alpha: float):
+    """(status, the 7 byte offsets of qg_fp4_linear's intermediates in its workspace)."""
+    arr = (_SZ * 7)()
+    st = _lib.qg_fp4_linear_parts(int(M), int(K), int(N), int(dtype), float(alpha), arr)
+    return st, [int(x) for x in arr]
+
+
+def linear_parts(ws: Workspace, M: int, K: int, N: int, dtype: int, alpha: float) -> dict:
+    """Views into `ws` of what qg_fp4_linear left there: activation codes and
+    scales, dA (as a CSR) and T."""
+    st, off = qg_fp4_linear_parts(M, K, N, dtype, alpha)
+    _check(st, "qg_fp4_linear_parts")
+    b = ws.buf
+
+    def view(i, n, dt):
+        item = torch.empty((), dtype=dt).element_size()
+        return b[off[i]:off[i] + n * item].view(dt)
+
+    nnz = view(5, 1, torch.int64)
+    cap = max(qg_nnz_capacity(M * K, alpha), 1)
+    return {"codes": view(0, M * (K // 2), torch.uint8).view(M, K // 2),
+            "scales": view(1, M, torch.float32),
+            "csr": CSR(view(2, M + 1, torch.int32), view(3, cap, torch.int32),
+                       view(4, cap, torch.float64), nnz, cap),
+            "T": view(6, 1, torch.float32)}
+
+
 def _contig(*ts):
     for t in ts:
         if not t.is_contiguous():
@@ -312,11 +341,12 @@ def qg_mx_gemm(codesA, sA, codesWT, sW, M, N, K, C, Y, raw_acc, ws: Workspace, s
                            _ptr(Y), y_dt, _ptr(raw_acc), ws.ptr, ws.nbytes, _stream(stream))
 
 
-def qg_fp4_mma_loop(iters: int, pair: bool, ws: Workspace, stream=None):
-    """(status, MMA flops of the launch)."""
+def qg_fp4_mma_loop(iters: int, pair: bool, ws: Workspace, stream=None, acc_out=None):
+    """(status, MMA flops of the launch); acc_out (128 x 224 fp32, optional)
+    receives CTA 0's accumulator."""
     flops = _D(0.0)
-    st = _lib.qg_fp4_mma_loop(int(iters), 1 if pair else 0, ctypes.byref(flops), ws.ptr, ws.nbytes,
-                              _stream(stream))
+    st = _lib.qg_fp4_mma_loop(int(iters), 1 if pair else 0, ctypes.byref(flops), _ptr(acc_out),
+                              ws.ptr, ws.nbytes, _stream(stream))
     return st, flops.value
 
 
@@ -468,11 +498,13 @@ def mx_gemm(codesA, sA, codesWT, sW, K: int, C=None, out_dtype=torch.float32, ra
     return (Y, acc) if raw else Y
 
 
-def fp4_mma_loop(iters: int, pair: bool = True, ws: Optional[Workspace] = None, stream=None) -> float:
+def fp4_mma_loop(iters: int, pair: bool = True, ws: Optional[Workspace] = None, stream=None,
+                 acc_out: Optional[torch.Tensor] = None) -> float:
     """Enqueue the tensor-pipe E2M1 MMA loop; returns its flops (time it with
-    CUDA events on `stream`)."""
+    CUDA events on `stream`).  acc_out (128 x 224 fp32) receives CTA 0's
+    accumulator."""
     ws = ws or Workspace(QG_OP_FP4_GEMM, 1, 32, 1, QG_F32)
-    st, flops = qg_fp4_mma_loop(iters, pair, ws, stream)
+    st, flops = qg_fp4_mma_loop(iters, pair, ws, stream, acc_out)
     _check(st, "qg_fp4_mma_loop")
     return flops
 

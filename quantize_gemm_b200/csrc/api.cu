@@ -52,16 +52,7 @@ int num_sms() {
     return g_sms[dev];
 }
 
-static bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 static size_t elsize(qg_dtype d) { return d == QG_BF16 ? 2 : 4; }
-static bool dtype_ok(qg_dtype d) { return d == QG_F32 || d == QG_BF16; }
-
-static qg_status check_mk(int64_t M, int64_t K) {
-    if (M < 1 || K < 1) return QG_ERR_UNSUPPORTED_SHAPE;
-    if (K % 32 != 0 || K > 16384) return QG_ERR_UNSUPPORTED_SHAPE;
-    if (M > (int64_t)INT32_MAX - 1) return QG_ERR_UNSUPPORTED_SHAPE;
-    return QG_OK;
-}
 
 static qg_status check_ld(const void* A, qg_dtype dt, int64_t K, int64_t ld) {
     if (A == nullptr || !aligned16(A)) return QG_ERR_INVALID_ARG;
@@ -77,7 +68,6 @@ static qg_status check_ws(void* ws, size_t ws_bytes, size_t need) {
 
 static bool alpha_ok(double a) { return a > 0.0 && a <= 1.0; }
 
-static qg_status cuda_status(cudaError_t e) { return e == cudaSuccess ? QG_OK : QG_ERR_CUDA; }
 
 template <class T>
 static T* at(void* ws, size_t off) {
@@ -336,6 +326,23 @@ qg_status qg_fp4_linear(const void* A, qg_dtype dtype, int64_t M, int64_t K,
                                        at<uint32_t>(ws, L.status), stream));
 }
 
+qg_status qg_fp4_linear_parts(int64_t M, int64_t K, int64_t N, qg_dtype dtype, double alpha,
+                              size_t* parts) {
+    if (parts == nullptr || !dtype_ok(dtype) || !alpha_ok(alpha)) return QG_ERR_INVALID_ARG;
+    qg_status st = check_mk(M, K);
+    if (st != QG_OK) return st;
+    if ((st = check_mk(N, K)) != QG_OK) return st;
+    const WsLayout L = ws_layout(QG_OP_FP4_LINEAR, M, K, N, dtype, alpha);
+    parts[0] = L.act_codes;
+    parts[1] = L.act_scales;
+    parts[2] = L.csr_row_ptr;
+    parts[3] = L.csr_col;
+    parts[4] = L.csr_val;
+    parts[5] = L.csr_nnz;
+    parts[6] = L.thr;
+    return QG_OK;
+}
+
 // Column quantization of a whole row-major matrix X (rows x cols) into
 // codesT (cols x rows/2) + scales (cols): the cooperative bf16 kernel or the
 // multi-kernel sequence (colmax: 32 * cols words of scratch).
@@ -456,15 +463,16 @@ qg_status qg_mx_gemm(const uint8_t* codesA, const uint8_t* sA, const uint8_t* co
                                           at<uint32_t>(ws, L.status), stream));
 }
 
-qg_status qg_fp4_mma_loop(int64_t iters, int pair, double* flops_out, void* ws, size_t ws_bytes,
-                          cudaStream_t stream) {
+qg_status qg_fp4_mma_loop(int64_t iters, int pair, double* flops_out, float* acc_out, void* ws,
+                          size_t ws_bytes, cudaStream_t stream) {
     if (iters < 1 || iters > ((int64_t)1 << 20) || flops_out == nullptr) return QG_ERR_INVALID_ARG;
+    if (acc_out != nullptr && !aligned16(acc_out)) return QG_ERR_INVALID_ARG;
     const WsLayout L = ws_layout(QG_OP_FP4_GEMM, 1, 32, 1, QG_F32, 1.0);
     qg_status st = check_ws(ws, ws_bytes, L.total);
     if (st != QG_OK) return st;
     if (ensure_device(nullptr) != cudaSuccess) return QG_ERR_CUDA;
-    return cuda_status(launch_fp4_mma_loop(iters, pair != 0, flops_out, at<uint32_t>(ws, L.status),
-                                           stream));
+    return cuda_status(launch_fp4_mma_loop(iters, pair != 0, flops_out, acc_out,
+                                           at<uint32_t>(ws, L.status), stream));
 }
 
 }  // extern "C"

@@ -14,7 +14,11 @@
 // 256 x 224 x 64 per 2-SM pair (cta_group::2).  Nothing is read from or
 // written to global memory except the status word, so the launch time is the
 // tensor pipe's time for the MMAs.  The wait for the last MMA is bounded; a
-// wait that runs out sets the timeout bit of the status word.
+// wait that runs out sets the timeout bit of the status word, and a second
+// bounded wait lets MMAs still in flight finish before TMEM is released.
+// Optionally (acc_out != NULL) CTA 0 copies its accumulator, 128 rows x 224
+// columns, to global memory afterwards, so a test can check the MMAs against
+// a CPU product of the same operand tiles.
 #include "qg_internal.cuh"
 
 namespace qg {
@@ -66,7 +70,7 @@ __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr) {
 
 template <bool PAIR>
 __global__ void __launch_bounds__(kThreads, 1)
-fp4_mma_loop_kernel(long long iters, uint32_t* status) {
+fp4_mma_loop_kernel(long long iters, uint32_t* status, float* acc_out) {
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -169,17 +173,51 @@ fp4_mma_loop_kernel(long long iters, uint32_t* status) {
                              smem_u32(bar))
                          : "memory");
     }
-    // every thread waits (bounded) for the MMAs to complete
-    if (!mbar_try_wait(bar, 0)) {
+    // every thread waits (bounded) for the MMAs to complete; after a timeout a
+    // second bounded wait gives MMAs still in flight time to finish before
+    // the accumulator is read or TMEM is released
+    bool done = mbar_try_wait(bar, 0);
+    if (!done) {
         const long long t0 = clock64();
-        while (!mbar_try_wait(bar, 0)) {
+        while (!(done = mbar_try_wait(bar, 0))) {
             if (clock64() - t0 > kWaitLimit) {
                 if ((threadIdx.x & 31) == 0) flag_status(status, kStatusTimeout);
                 break;
             }
         }
+        if (!done) {
+            const long long t1 = clock64();
+            while (!(done = mbar_try_wait(bar, 0)) && clock64() - t1 < kWaitLimit) {
+            }
+        }
     }
     __syncwarp();
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+    if (acc_out != nullptr && blockIdx.x == 0 && __all_sync(0xFFFFFFFFu, done)) {
+        // warp w holds accumulator rows 32 w .. 32 w + 31 (one per lane)
+        const int row = 32 * warp + (threadIdx.x & 31);
+        const uint32_t lanes = (uint32_t)(32 * warp) << 16;
+        for (int c0 = 0; c0 < kBN; c0 += 32) {
+            uint32_t v[32];
+            asm volatile(
+                "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,"
+                "%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,"
+                "%31}, [%32];"
+                : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]),
+                  "=r"(v[6]), "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]),
+                  "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]),
+                  "=r"(v[18]), "=r"(v[19]), "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]),
+                  "=r"(v[24]), "=r"(v[25]), "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]),
+                  "=r"(v[30]), "=r"(v[31])
+                : "r"(tmem + lanes + (uint32_t)c0));
+            asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+            float4* d = reinterpret_cast<float4*>(acc_out + (size_t)row * kBN + c0);
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                d[j] = make_float4(__uint_as_float(v[4 * j]), __uint_as_float(v[4 * j + 1]),
+                                   __uint_as_float(v[4 * j + 2]), __uint_as_float(v[4 * j + 3]));
+        }
+    }
     asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
     __syncthreads();
     if constexpr (PAIR) cluster_sync();   // the peer's MMAs no longer use this CTA
@@ -206,8 +244,9 @@ static cudaError_t set_smem_attr(bool pair) {
 
 // One launch over the whole GPU: a CTA per SM (pair: as many 2-CTA clusters as
 // can be resident at once).  *flops = 2 x 128 x 224 x 64 x 4 x iters per CTA.
-cudaError_t launch_fp4_mma_loop(int64_t iters, bool pair, double* flops, uint32_t* status,
-                                cudaStream_t s) {
+// acc_out (nullable): CTA 0's accumulator, 128 x 224 fp32, row-major.
+cudaError_t launch_fp4_mma_loop(int64_t iters, bool pair, double* flops, float* acc_out,
+                                uint32_t* status, cudaStream_t s) {
     using namespace peak;
     cudaError_t e = set_smem_attr(pair);
     if (e != cudaSuccess) return e;
@@ -232,8 +271,8 @@ cudaError_t launch_fp4_mma_loop(int64_t iters, bool pair, double* flops, uint32_
         ctas = std::min(2 * clusters, ctas / 2 * 2);
     }
     cfg.gridDim = dim3((unsigned)ctas);
-    e = pair ? cudaLaunchKernelEx(&cfg, fp4_mma_loop_kernel<true>, (long long)iters, status)
-                         : cudaLaunchKernelEx(&cfg, fp4_mma_loop_kernel<false>, (long long)iters, status);
+    e = pair ? cudaLaunchKernelEx(&cfg, fp4_mma_loop_kernel<true>, (long long)iters, status, acc_out)
+             : cudaLaunchKernelEx(&cfg, fp4_mma_loop_kernel<false>, (long long)iters, status, acc_out);
     count_launch(1);
     if (flops) *flops = 2.0 * 128.0 * kBN * 64.0 * 4.0 * (double)iters * (double)ctas;
     return e;

@@ -354,6 +354,18 @@ struct ActBuffers {
     int64_t row_slots;
 };
 
+// Host-side argument checks shared by the C entry points.
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+inline bool dtype_ok(qg_dtype d) { return d == QG_F32 || d == QG_BF16; }
+// Rows x K operand: K a multiple of 32 and at most 16384, both sizes positive.
+inline qg_status check_mk(int64_t M, int64_t K) {
+    if (M < 1 || K < 1) return QG_ERR_UNSUPPORTED_SHAPE;
+    if (K % 32 != 0 || K > 16384) return QG_ERR_UNSUPPORTED_SHAPE;
+    if (M > (int64_t)INT32_MAX - 1) return QG_ERR_UNSUPPORTED_SHAPE;
+    return QG_OK;
+}
+inline qg_status cuda_status(cudaError_t e) { return e == cudaSuccess ? QG_OK : QG_ERR_CUDA; }
+
 // Launch sequences (kernel files) used by the C ABI layer.
 void launch_zero_u32(uint32_t* p, int64_t n, cudaStream_t s);
 void launch_e2m1_encode(const float* x, int64_t n, uint8_t* packed, cudaStream_t s);
@@ -390,8 +402,8 @@ cudaError_t gemm_setup();
 cudaError_t spmm_setup();
 // MMA-only loop on the tensor pipe (a CTA per SM, or 2-SM pairs); *flops gets
 // the MMA flops of the launch.
-cudaError_t launch_fp4_mma_loop(int64_t iters, bool pair, double* flops, uint32_t* status,
-                                cudaStream_t s);
+cudaError_t launch_fp4_mma_loop(int64_t iters, bool pair, double* flops, float* acc_out,
+                                uint32_t* status, cudaStream_t s);
 
 // Number of SMs of the current device (cached per device id).
 int num_sms();

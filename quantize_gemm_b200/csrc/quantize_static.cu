@@ -7,7 +7,12 @@
 // 256 KB), which every GPU that loads this library holds until the process
 // exits.  Host code cannot use the array's name as a device address, so the
 // address is looked up once per device (cudaGetSymbolAddress, with that device
-// current) on the first call made on that device, and cached.
+// current) on the first call made on that device, and cached; a
+// cudaDeviceReset ends the context that address belongs to, so the cache is
+// only valid until then.  Both dtypes run the two-pass kernels of
+// qg_quantize_cols's fp32 path (column maxima, then codes): the cooperative
+// bf16 kernel of qg_quantize_cols keeps per-split maxima and a grid barrier in
+// its workspace, which would need a larger fixed array.
 #include <mutex>
 
 #include "qg_internal.cuh"
@@ -42,17 +47,18 @@ using namespace qg;
 extern "C" qg_status qg_quantize_cols_static(const void* W, qg_dtype dtype, int64_t K, int64_t N,
                                              int64_t ldw, uint8_t* codesT, float* scales,
                                              cudaStream_t stream) {
-    if (dtype != QG_F32 && dtype != QG_BF16) return QG_ERR_INVALID_ARG;
-    if (N < 1 || K < 1 || K % 32 != 0 || K > 16384) return QG_ERR_UNSUPPORTED_SHAPE;
+    // the checks of qg_quantize_cols (same helpers), then the array's capacity
+    if (!dtype_ok(dtype)) return QG_ERR_INVALID_ARG;
+    qg_status st = check_mk(N, K);
+    if (st != QG_OK) return st;
     if (N > kStaticColsMax) return QG_ERR_UNSUPPORTED_SHAPE;
-    if (W == nullptr || (reinterpret_cast<uintptr_t>(W) & 15u) != 0 || ldw < N) return QG_ERR_INVALID_ARG;
-    if (codesT == nullptr || scales == nullptr || (reinterpret_cast<uintptr_t>(codesT) & 15u) != 0)
-        return QG_ERR_INVALID_ARG;
+    if (W == nullptr || !aligned16(W) || ldw < N) return QG_ERR_INVALID_ARG;
+    if (!codesT || !scales || !aligned16(codesT)) return QG_ERR_INVALID_ARG;
     if (device_setup() != cudaSuccess) return QG_ERR_CUDA;
     uint32_t* colmax = static_scratch();
     if (colmax == nullptr) return QG_ERR_CUDA;
     // the same two kernels as qg_quantize_cols; the column maxima are zeroed
     // first, since the array keeps whatever the previous call left in it
     launch_quantize_cols(W, dtype, K, N, ldw, codesT, scales, colmax, stream);
-    return cudaGetLastError() == cudaSuccess ? QG_OK : QG_ERR_CUDA;
+    return cuda_status(cudaGetLastError());
 }

@@ -124,6 +124,28 @@ def pin_encoder_nearest_search(orc, seed=1):
     assert bad.size == 0, (xs[bad[:8]], got[bad[:8]], want[bad[:8]])
 
 
+def pin_encode_bits_packed(orc, seed=15):
+    """The packed sweep over consecutive fp32 bit patterns (the exhaustive GPU
+    encoder test's reference) equals the independent nearest-value search on
+    the same patterns, packed two per byte with the even pattern in the low
+    nibble, NaN patterns mapped to code 0: ranges around zero, 1, the top grid
+    value, the largest finite values into Inf and NaN (both signs), and random
+    starts (odd ones included)."""
+    rng = np.random.default_rng(seed)
+    starts = [0x00000000, 0x3F7FFF00, 0x40BFFF01, 0x7F7FFF80, 0x7FBFFFF0, 0x807FFF00,
+              0xBF7FFFF1, 0xFF7FFF80, 0xFFFFFE00]
+    starts += [int(s) for s in rng.integers(0, (1 << 32) - 4096, size=6)]
+    for start in starts:
+        n = 2048
+        bits = (np.arange(n, dtype=np.uint64) + np.uint64(start)).astype(np.uint32)
+        x = bits.view(np.float32)
+        want_codes = ref_encode(np.where(np.isnan(x), np.float32(0.0), x))
+        want = pack(want_codes)
+        got = orc.e2m1_encode_bits_packed(start, n)
+        bad = np.nonzero(got != want)[0]
+        assert bad.size == 0, (hex(start), int(bad[0]), got[bad[0]], want[bad[0]])
+
+
 def pin_row_worked_example(orc):
     g = golden()["row_quantization"]
     codes, s = orc.quantize_rows(np.array([g["row"]], dtype=np.float32))
@@ -573,7 +595,8 @@ def pin_mx_gemm(orc, seed=24):
 
 
 ALL_PINS = [
-    pin_grid, pin_encoder_ties, pin_encoder_nearest_search, pin_row_worked_example,
+    pin_grid, pin_encoder_ties, pin_encoder_nearest_search, pin_encode_bits_packed,
+    pin_row_worked_example,
     pin_col_worked_example, pin_threshold_worked_example, pin_act_worked_example,
     pin_gemm_worked_example, pin_threshold_vs_sort_and_quantile, pin_clamp_invariants,
     pin_quantize_rows_identity, pin_quantize_rows_properties, pin_quantize_degenerate_rows,

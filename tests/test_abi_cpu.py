@@ -165,10 +165,12 @@ def test_mma_loop_host_checks(qg):
     flops = ctypes.c_double(-1.0)
     ws_need = qg.qg_workspace_size(qg.QG_OP_FP4_GEMM, 1, 32, 1, qg.QG_F32, 1.0)
     for iters in (0, -1, (1 << 20) + 1):
-        assert lib.qg_fp4_mma_loop(iters, 1, ctypes.byref(flops), fake, ws_need, None) == \
+        assert lib.qg_fp4_mma_loop(iters, 1, ctypes.byref(flops), None, fake, ws_need, None) == \
             qg.QG_ERR_INVALID_ARG
-    assert lib.qg_fp4_mma_loop(16, 0, None, fake, ws_need, None) == qg.QG_ERR_INVALID_ARG
-    assert lib.qg_fp4_mma_loop(16, 0, ctypes.byref(flops), fake, ws_need - 256, None) == \
+    assert lib.qg_fp4_mma_loop(16, 0, None, None, fake, ws_need, None) == qg.QG_ERR_INVALID_ARG
+    assert lib.qg_fp4_mma_loop(16, 0, ctypes.byref(flops), P((1 << 20) + 4), fake, ws_need,
+                               None) == qg.QG_ERR_INVALID_ARG   # misaligned accumulator output
+    assert lib.qg_fp4_mma_loop(16, 0, ctypes.byref(flops), None, fake, ws_need - 256, None) == \
         qg.QG_ERR_WORKSPACE
     assert flops.value == -1.0   # nothing written on a rejected call
 
@@ -212,3 +214,23 @@ def test_header_is_plain_c_and_links(qg, tmp_path):
     assert int(out[2]) == qg.qg_workspace_size(qg.QG_OP_FP4_LINEAR, 4096, 2048, 5504, qg.QG_BF16, 0.99)
     assert int(out[3]) == qg.qg_mx_scale_bytes(300, 5504)
     assert int(out[4]) == qg.QG_ERR_UNSUPPORTED_SHAPE
+
+
+def test_linear_parts_offsets(qg):
+    """The intermediates of qg_fp4_linear sit at distinct 256-byte-aligned
+    offsets inside the workspace, far enough apart for their sizes."""
+    for (M, K, N, dt, alpha) in ((16384, 11008, 4096, qg.QG_BF16, 0.99),
+                                 (256, 512, 512, qg.QG_F32, 0.99), (1, 32, 1, qg.QG_BF16, 1.0)):
+        st, off = qg.qg_fp4_linear_parts(M, K, N, dt, alpha)
+        assert st == qg.QG_OK
+        total = qg.qg_workspace_size(qg.QG_OP_FP4_LINEAR, M, K, N, dt, alpha)
+        cap = max(qg.qg_nnz_capacity(M * K, alpha), 1)
+        sizes = [M * (K // 2), 4 * M, 4 * (M + 1), 4 * cap, 8 * cap, 8, 4]
+        assert all(o % 256 == 0 for o in off)
+        spans = sorted(zip(off, sizes))
+        for (o1, s1), (o2, _) in zip(spans, spans[1:]):
+            assert o1 + s1 <= o2
+        assert spans[-1][0] + spans[-1][1] <= total
+    assert qg.qg_fp4_linear_parts(64, 48, 64, qg.QG_BF16, 0.99)[0] == qg.QG_ERR_UNSUPPORTED_SHAPE
+    assert qg.qg_fp4_linear_parts(64, 64, 64, qg.QG_BF16, 0.0)[0] == qg.QG_ERR_INVALID_ARG
+    assert qg._lib.qg_fp4_linear_parts(64, 64, 64, qg.QG_BF16, 0.99, None) == qg.QG_ERR_INVALID_ARG

@@ -424,8 +424,9 @@ def test_fp4_linear_small(qg, wl, layer, M):
 @pytest.mark.parametrize("wl,layer", [("llama1.3b", 1), ("llama7b", 1), ("llama13b", 4)])
 def test_fp4_linear_full_size_sampled(qg, wl, layer):
     """Full workload sizes, the launch configuration the benchmark times:
-    T, codes, scales and dA checked exactly over the whole tensor, Y on a
-    sample of rows computed by the oracle one by one."""
+    T, codes, scales and dA, as the layer call left them in its workspace,
+    checked exactly over the whole tensor, Y on a sample of rows computed by
+    the oracle one by one."""
     A, W = make_layer_inputs(wl, layer, device="cuda")
     alpha = WORKLOADS[wl].alphas[0]
     M, K = A.shape
@@ -434,7 +435,8 @@ def test_fp4_linear_full_size_sampled(qg, wl, layer):
     ws = qg.Workspace(qg.QG_OP_FP4_LINEAR, M, K, N, qg._dt(A), alpha)
     Y = qg.fp4_linear(A, codesT, t, W, alpha, ws=ws)
     qg.check_status(ws)
-    codes, scales, csr, T = qg.quantize_act(A, alpha)
+    parts = qg.linear_parts(ws, M, K, N, qg._dt(A), alpha)   # what the layer call used
+    codes, scales, csr, T = parts["codes"], parts["scales"], parts["csr"], parts["T"]
     rows = np.unique(np.concatenate([np.random.default_rng(M + N).integers(0, M, 24), [0, M - 1]]))
     Yo, act = _linear_oracle(A, W, alpha, rows=rows)
     assert float(_np(T)[0]) == act["T"]

@@ -41,6 +41,12 @@ MUTANTS = [
     ("spmm_wrong_row_of_w", "const float* w = W + (int64_t)col[p] * N;\n            for (int64_t j = 0; j < N; ++j) c[j]",
      "const float* w = W + (int64_t)(col[p] > 0 ? col[p] - 1 : 0) * N;\n            for (int64_t j = 0; j < N; ++j) c[j]"),
     ("delta_in_single", "val[nnz] = (double)a - (double)ac;", "val[nnz] = (double)(float)(a * 1.0000001f - ac);"),
+    ("bits_packed_nibbles_swapped", "packed[j] = (uint8_t)(c0 | (c1 << 4));",
+     "packed[j] = (uint8_t)(c1 | (c0 << 4));"),
+    ("bits_packed_start_off_by_one", "uint32_t b0 = start + (uint32_t)(2 * j), b1 = b0 + 1u;",
+     "uint32_t b0 = start + (uint32_t)(2 * j) + 1u, b1 = b0 + 1u;"),
+    ("bits_packed_nan_keeps_sign", "uint8_t c0 = isnan(x0) ? 0u : orc_e2m1_encode(x0);",
+     "uint8_t c0 = isnan(x0) ? (uint8_t)(signbit(x0) ? 8u : 0u) : orc_e2m1_encode(x0);"),
     ("mx_exponent_floor_rule", "ldexp(6.0, e) < (double)amax", "ldexp(8.0, e) <= (double)amax"),
     ("mx_exponent_not_minimal", "while (e < 127 && ldexp(6.0, e) < (double)amax) ++e;",
      "while (e < 127 && ldexp(6.0, e) < (double)amax) ++e;\n    if (amax > 0.0f && e < 127) ++e;"),
