@@ -158,29 +158,30 @@ class Layer:
         self.s = torch.empty(M, dtype=torch.float32, device=device)
         self.csr = qg.CSR.empty(M, cap, device=device)
         self.T = torch.empty(1, dtype=torch.float32, device=device)
-        self.C = torch.empty((M, N), dtype=torch.float32, device=device)
         self.Y = torch.empty((M, N), dtype=torch.float32, device=device)
         self.ws_cols = qg.Workspace(qg.QG_OP_QUANTIZE_COLS, 1, K, N, dt, device=device)
         self.ws_act = qg.Workspace(qg.QG_OP_QUANTIZE_ACT, M, K, 1, dt, a_size, device=device)
-        self.ws_spmm = qg.Workspace(qg.QG_OP_SPMM, M, K, N, dt, device=device)
-        self.ws_gemm = qg.Workspace(qg.QG_OP_FP4_GEMM, M, K, N, qg.QG_F32, device=device)
-        self.ws_lin = None          # allocated by the e2e arm (it holds its own M x N correction)
+        self.ws_gemm = qg.Workspace(qg.QG_OP_FP4_GEMM_COMPENSATED, M, K, N, qg.QG_F32,
+                                    device=device)
+        self.ws_lin = None          # allocated by the e2e arm
         self.dt = dt
         self.flops = 2 * M * N * K
         self.a_bytes = M * K * self.A.element_size()
         self.w_bytes = K * N * self.W.element_size()
 
     def workspaces(self):
-        return tuple(w for w in (self.ws_cols, self.ws_act, self.ws_spmm, self.ws_gemm, self.ws_lin)
+        return tuple(w for w in (self.ws_cols, self.ws_act, self.ws_gemm, self.ws_lin)
                      if w is not None)
 
 
-KERNELS = ("quantize_cols", "quantize_act", "spmm", "fp4_gemm")
+KERNELS = ("quantize_cols", "quantize_act", "fp4_gemm_compensated")
 
 
 def run_step(qg, layers, ev=None):
-    """One pass of the hot path over every layer.  With `ev`, record events
-    around each of the four calls of each layer (same stream)."""
+    """One pass of the hot path over every layer: the weight quantizer, the
+    fused activation quantizer (threshold, clamp, dA, codes) and the FP4 GEMM
+    whose kernel also computes dA . W.  With `ev`, record events around each
+    of the three calls of each layer (same stream)."""
     def _chk(st, where):
         if st != qg.QG_OK:
             raise qg.QGError(st, where)
@@ -193,13 +194,10 @@ def run_step(qg, layers, ev=None):
         _chk(qg.qg_quantize_act(L.A, L.alpha, L.codes, L.s, L.csr, L.T, L.ws_act), "quantize_act")
         if ev is not None:
             ev[i][2].record()
-        _chk(qg.qg_spmm_correction(L.csr, L.M, L.W, L.C, L.ws_spmm), "spmm")
+        _chk(qg.qg_fp4_gemm_compensated(L.codes, L.s, L.codesT, L.t, L.M, L.N, L.K, L.csr, L.W,
+                                        L.Y, L.ws_gemm), "fp4_gemm_compensated")
         if ev is not None:
             ev[i][3].record()
-        _chk(qg.qg_fp4_gemm(L.codes, L.s, L.codesT, L.t, L.M, L.N, L.K, L.C, L.Y, None,
-                            L.ws_gemm), "fp4_gemm")
-        if ev is not None:
-            ev[i][4].record()
 
 
 def capture_step(qg, layers):
@@ -245,8 +243,8 @@ def _measure(qg, layers, steps, flush, world, device, no_graph):
     graph, launches_per_step = (None, None) if no_graph else capture_step(qg, layers)
     ev_step = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
                for _ in range(steps)]
-    ev_steps = [[[torch.cuda.Event(enable_timing=True) for _ in range(5)] for _ in range(n_l)]
-                for _ in range(steps)]
+    ev_steps = [[[torch.cuda.Event(enable_timing=True) for _ in range(len(KERNELS) + 1)]
+                 for _ in range(n_l)] for _ in range(steps)]
     sampler = ClockSampler(torch.cuda.current_device() if world == 1 else int(os.environ.get("LOCAL_RANK", 0)))
     sampler.start()
     time.sleep(0.3)
@@ -299,26 +297,33 @@ def _kernel_rows(layers, per_kernel, steps, peaks, sm_mhz, n_sm):
     for k in KERNELS:
         kms = sum(per_kernel[k]) / steps
         t = kms * 1e-3
-        if k == "fp4_gemm":
-            # the GEMM moves the FP4 codes, the scales, the fp32 correction C
-            # (read) and Y (fp32, written); its bound is whichever of the
-            # tensor-core time and the HBM time of those bytes is longer
+        if k == "fp4_gemm_compensated":
+            # three ceilings: the FP4 MMAs on the tensor cores (2 M N K), the
+            # compensation's fp32 FMAs on the CUDA cores (2 nnz N), and the
+            # HBM bytes (codes, scales, the CSR, W read once, Y written); the
+            # kernel's roofline time is the largest of the three
             flops = sum(L.flops for L in layers)
-            byts = sum(L.M * L.K / 2 + L.N * L.K / 2 + 4 * (L.M + L.N) + 4 * L.M * L.N
+            alu_flops = sum(2 * int(L.csr.nnz.item()) * L.N for L in layers)
+            byts = sum(L.M * L.K / 2 + L.N * L.K / 2 + 4 * (L.M + L.N) + 4 * (L.M + 1)
+                       + 12 * int(L.csr.nnz.item()) + L.w_bytes
                        + L.Y.element_size() * L.M * L.N for L in layers)
             t_tensor = flops / (fp4_peak * 1e12)
+            t_alu = alu_flops / (alu_peak * 1e12)
             t_hbm = byts / (peaks["hbm_gbs"] * 1e9)
-            if t_tensor >= t_hbm:
+            worst = max(t_tensor, t_alu, t_hbm)
+            if worst == t_tensor:
                 bound, unit, peak, algo = "tensor", "TFLOP/s", fp4_peak, flops / 1e12
+            elif worst == t_alu:
+                bound, unit, peak, algo = "alu", "TFLOP/s", alu_peak, alu_flops / 1e12
             else:
                 bound, unit, peak, algo = "hbm", "GB/s", peaks["hbm_gbs"], byts / 1e9
-            extra = {"tflops": round(flops / t / 1e12, 1) if t > 0 else 0.0,
+            extra = {"fp4_tflops": round(flops / t / 1e12, 1) if t > 0 else 0.0,
                      "frac_of_9pf_datasheet": round(flops / t / 9e15, 4) if t > 0 else 0.0,
-                     "roofline_ms": round(1e3 * max(t_tensor, t_hbm), 4)}
-        elif k == "spmm":
-            algo = sum(2 * int(L.csr.nnz.item()) * L.N for L in layers) / 1e12
-            bound, unit, peak = "alu", "TFLOP/s", alu_peak
-            extra = {}
+                     "compensation_tflops": round(alu_flops / t / 1e12, 2) if t > 0 else 0.0,
+                     "ceilings_ms": {"tensor": round(1e3 * t_tensor, 4),
+                                     "alu": round(1e3 * t_alu, 4), "hbm": round(1e3 * t_hbm, 4)},
+                     "w_row_gather_bytes": sum(int(L.csr.nnz.item()) * L.N * L.W.element_size()
+                                               for L in layers)}
         elif k == "quantize_act":
             algo = sum(2 * L.a_bytes + L.M * L.K / 2 + 4 * L.M + 16 * int(L.csr.nnz.item())
                        + 4 * (L.M + 1) + 8 * L.M for L in layers) / 1e9

@@ -98,7 +98,8 @@ typedef enum {
     QG_OP_FP4_GEMM = 5,
     QG_OP_FP4_LINEAR = 6,
     QG_OP_FP4_DGRAD = 7,    /* sized with (M, K, N) of the forward layer */
-    QG_OP_FP4_WGRAD = 8     /* sized with (M, K, N) of the forward layer */
+    QG_OP_FP4_WGRAD = 8,    /* sized with (M, K, N) of the forward layer */
+    QG_OP_FP4_GEMM_COMPENSATED = 9
 } qg_op;
 
 const char* qg_status_string(qg_status s);
@@ -210,13 +211,36 @@ qg_status qg_fp4_gemm(const uint8_t* codesA, const float* sA, const uint8_t* cod
                       void* Y, qg_dtype y_dtype, float* raw_acc, void* ws, size_t ws_bytes,
                       cudaStream_t stream);
 
-/* The whole layer: qg_quantize_act(A) -> qg_spmm_correction(dA, W) ->
- * qg_fp4_gemm(..., C) into Y (M x N, fp32 or bf16).  codesWT / sW come from
- * qg_quantize_cols(W); W is the unquantized weight used by the correction,
+/* The compensated FP4 GEMM, the layer's product in one kernel:
+ *   Y_ij = acc_ij * sA_i * sW_j + sum over the entries (i, k) of dA of
+ *          dA_ik * W_kj
+ * ([FP4-writeup], FP4 GEMM + outlier clamping and compensation paragraphs),
+ * with acc the FP4 product as in qg_fp4_gemm and the compensation summed in
+ * fp32 (one fused multiply-add per entry, in the row's CSR order, W read in
+ * its stored dtype): the same arithmetic as qg_spmm_correction followed by
+ * qg_fp4_gemm with that C, bit for bit, but the compensation is computed by
+ * extra warps of the GEMM kernel while the tensor cores run, tile by tile, and
+ * no M x N correction matrix is written to or read from memory.
+ *   dA: CSR over M rows with column indices < K (as qg_quantize_act leaves it);
+ *   W: K x N, row pitch ldw >= N elements, 16-byte aligned, dtype w_dtype;
+ *   Y: M x N, fp32 or bf16 (y_dtype), contiguous.
+ * Workspace: qg_workspace_size(QG_OP_FP4_GEMM_COMPENSATED, M, K, N, any, 1.0)
+ * (a fixed ~37 MB of scratch slots: two 128 x 224 fp32 tiles per CTA).
+ * Errors as qg_fp4_gemm. */
+qg_status qg_fp4_gemm_compensated(const uint8_t* codesA, const float* sA, const uint8_t* codesWT,
+                                  const float* sW, int64_t M, int64_t N, int64_t K,
+                                  const qg_csr* dA, const void* W, qg_dtype w_dtype, int64_t ldw,
+                                  void* Y, qg_dtype y_dtype, void* ws, size_t ws_bytes,
+                                  cudaStream_t stream);
+
+/* The whole layer: qg_quantize_act(A) -> qg_fp4_gemm_compensated(codes, dA,
+ * W) into Y (M x N, fp32 or bf16).  codesWT / sW come from
+ * qg_quantize_cols(W); W is the unquantized weight used by the compensation,
  * K x N row-major and contiguous, stored in the SAME dtype as A (`dtype`
  * describes both; the call has no separate weight dtype, so a weight in the
  * other dtype is read wrongly without an error).  The activation codes, dA
- * and C live in the workspace (qg_workspace_size(QG_OP_FP4_LINEAR, ...)). */
+ * and the GEMM's scratch slots live in the workspace
+ * (qg_workspace_size(QG_OP_FP4_LINEAR, ...)); no M x N intermediate exists. */
 qg_status qg_fp4_linear(const void* A, qg_dtype dtype, int64_t M, int64_t K,
                         const uint8_t* codesWT, const float* sW, const void* W, int64_t N,
                         double alpha, void* Y, qg_dtype y_dtype, void* ws, size_t ws_bytes,

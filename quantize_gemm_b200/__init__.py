@@ -32,7 +32,8 @@ QG_F32, QG_BF16 = 0, 1
 QG_OK, QG_ERR_INVALID_ARG, QG_ERR_UNSUPPORTED_SHAPE, QG_ERR_WORKSPACE, QG_ERR_CUDA, \
     QG_ERR_NONFINITE, QG_ERR_TIMEOUT, QG_ERR_INTERNAL = range(8)
 (QG_OP_QUANTIZE_ROWS, QG_OP_QUANTIZE_COLS, QG_OP_CLAMP_COMPENSATE, QG_OP_QUANTIZE_ACT,
- QG_OP_SPMM, QG_OP_FP4_GEMM, QG_OP_FP4_LINEAR, QG_OP_FP4_DGRAD, QG_OP_FP4_WGRAD) = range(9)
+ QG_OP_SPMM, QG_OP_FP4_GEMM, QG_OP_FP4_LINEAR, QG_OP_FP4_DGRAD, QG_OP_FP4_WGRAD,
+ QG_OP_FP4_GEMM_COMPENSATED) = range(10)
 
 # every symbol the header declares (checked by the CPU tests)
 EXPORTED = (
@@ -42,7 +43,7 @@ EXPORTED = (
     "qg_spmm_correction", "qg_fp4_gemm", "qg_fp4_linear", "qg_launch_count",
     "qg_quantize_cols_static", "qg_fp4_dgrad", "qg_fp4_wgrad", "qg_mx_scale_bytes",
     "qg_mx_quantize_rows", "qg_mx_quantize_cols", "qg_mx_gemm", "qg_fp4_mma_loop",
-    "qg_fp4_linear_parts",
+    "qg_fp4_linear_parts", "qg_fp4_gemm_compensated",
 )
 
 
@@ -86,6 +87,9 @@ _sig("qg_spmm_correction", _INT,
      [ctypes.POINTER(_Csr), _I64, _P, _INT, _I64, _I64, _I64, _P, _P, _SZ, _P])
 _sig("qg_fp4_gemm", _INT,
      [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _INT, _P, _P, _SZ, _P])
+_sig("qg_fp4_gemm_compensated", _INT,
+     [_P, _P, _P, _P, _I64, _I64, _I64, ctypes.POINTER(_Csr), _P, _INT, _I64, _P, _INT, _P, _SZ,
+      _P])
 _sig("qg_fp4_linear", _INT,
      [_P, _INT, _I64, _I64, _P, _P, _P, _I64, _D, _P, _INT, _P, _SZ, _P])
 _sig("qg_fp4_linear_parts", _INT, [_I64, _I64, _I64, _INT, _D, ctypes.POINTER(_SZ)])
@@ -263,6 +267,15 @@ def qg_fp4_gemm(codesA, sA, codesWT, sW, M, N, K, C, Y, raw_acc, ws: Workspace,
                             _ptr(Y), y_dt, _ptr(raw_acc), ws.ptr, ws.nbytes, _stream(stream))
 
 
+def qg_fp4_gemm_compensated(codesA, sA, codesWT, sW, M, N, K, csr: CSR, W, Y, ws: Workspace,
+                            ldw=None, stream=None) -> int:
+    c = csr.c()
+    return _lib.qg_fp4_gemm_compensated(_ptr(codesA), _ptr(sA), _ptr(codesWT), _ptr(sW), M, N, K,
+                                        ctypes.byref(c), _ptr(W), _dt(W),
+                                        W.stride(0) if ldw is None else ldw, _ptr(Y), _dt(Y),
+                                        ws.ptr, ws.nbytes, _stream(stream))
+
+
 def qg_fp4_linear(A, codesWT, sW, W, alpha, Y, ws: Workspace, stream=None) -> int:
     M, K = A.shape
     N = W.shape[1]
@@ -436,6 +449,17 @@ def fp4_gemm(codesA, sA, codesWT, sW, K: int, C=None, out_dtype=torch.float32,
     acc = torch.empty((M, N), dtype=torch.float32, device=codesA.device) if raw else None
     _check(qg_fp4_gemm(codesA, sA, codesWT, sW, M, N, K, C, Y, acc, ws), "qg_fp4_gemm")
     return (Y, acc) if raw else Y
+
+
+def fp4_gemm_compensated(codesA, sA, codesWT, sW, K: int, csr: CSR, W, out_dtype=torch.float32,
+                         ws: Optional[Workspace] = None):
+    """Y = acc * sA_i * sW_j + dA . W in one kernel (dA as a CSR over the rows)."""
+    M, N = codesA.shape[0], codesWT.shape[0]
+    ws = ws or Workspace(QG_OP_FP4_GEMM_COMPENSATED, M, K, N, QG_F32, device=codesA.device)
+    Y = torch.empty((M, N), dtype=out_dtype, device=codesA.device)
+    _check(qg_fp4_gemm_compensated(codesA, sA, codesWT, sW, M, N, K, csr, W, Y, ws),
+           "qg_fp4_gemm_compensated")
+    return Y
 
 
 def fp4_linear(A, codesWT, sW, W, alpha: float, out_dtype=torch.float32,

@@ -315,15 +315,37 @@ qg_status qg_fp4_linear(const void* A, qg_dtype dtype, int64_t M, int64_t K,
     csr.nnz_out = at<int64_t>(ws, L.csr_nnz);
     uint8_t* codes = at<uint8_t>(ws, L.act_codes);
     float* scales = at<float>(ws, L.act_scales);
-    float* C = at<float>(ws, L.corr);
     const int64_t rank = qg_quantile_rank(alpha, M * K);
     cudaError_t e = run_quantize_act(A, dtype, M, K, K, rank, act_buffers(ws, L), codes, scales, &csr,
                                      at<float>(ws, L.thr), stream);
     if (e != cudaSuccess) return QG_ERR_CUDA;
-    launch_spmm(&csr, M, W, dtype, N, N, C, at<uint32_t>(ws, L.status), stream);
-    if ((e = cudaGetLastError()) != cudaSuccess) return QG_ERR_CUDA;
-    return cuda_status(launch_fp4_gemm(codes, scales, codesWT, sW, M, N, K, C, Y, y_dtype, nullptr,
-                                       at<uint32_t>(ws, L.status), stream));
+    return cuda_status(launch_fp4_gemm_corr(codes, scales, codesWT, sW, M, N, K, &csr, W, dtype, N,
+                                            at<float>(ws, L.corr_scratch), Y, y_dtype,
+                                            at<uint32_t>(ws, L.status), stream));
+}
+
+qg_status qg_fp4_gemm_compensated(const uint8_t* codesA, const float* sA, const uint8_t* codesWT,
+                                  const float* sW, int64_t M, int64_t N, int64_t K,
+                                  const qg_csr* dA, const void* W, qg_dtype w_dtype, int64_t ldw,
+                                  void* Y, qg_dtype y_dtype, void* ws, size_t ws_bytes,
+                                  cudaStream_t stream) {
+    if (!dtype_ok(y_dtype) || !dtype_ok(w_dtype)) return QG_ERR_INVALID_ARG;
+    qg_status st = check_mk(M, K);
+    if (st != QG_OK) return st;
+    if ((st = check_mk(N, K)) != QG_OK) return st;
+    if (!codesA || !codesWT || !sA || !sW || !aligned16(codesA) || !aligned16(codesWT) ||
+        !aligned16(sW))
+        return QG_ERR_INVALID_ARG;
+    if (Y == nullptr || !aligned16(Y)) return QG_ERR_INVALID_ARG;
+    if (dA == nullptr || dA->row_ptr == nullptr || dA->col == nullptr || dA->val == nullptr)
+        return QG_ERR_INVALID_ARG;
+    if (W == nullptr || !aligned16(W) || ldw < N) return QG_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(QG_OP_FP4_GEMM_COMPENSATED, M, K, N, y_dtype, 1.0);
+    if ((st = check_ws(ws, ws_bytes, L.total)) != QG_OK) return st;
+    if (ensure_device(nullptr) != cudaSuccess) return QG_ERR_CUDA;
+    return cuda_status(launch_fp4_gemm_corr(codesA, sA, codesWT, sW, M, N, K, dA, W, w_dtype, ldw,
+                                            at<float>(ws, L.corr_scratch), Y, y_dtype,
+                                            at<uint32_t>(ws, L.status), stream));
 }
 
 qg_status qg_fp4_linear_parts(int64_t M, int64_t K, int64_t N, qg_dtype dtype, double alpha,

@@ -47,6 +47,18 @@
 // scales of row r from lane r, column slot + r / 32, and the scale-factor id
 // of the instruction descriptor picks the byte pair of its two 32-blocks.
 // The epilogue then writes the accumulator as is (+ C).
+// CORR = true (the layer's compensated GEMM): kCorrWarps more warps compute
+// the compensation dA . W of each output tile on the CUDA cores while the
+// tensor pipe runs the tile's MMAs.  A correction warp owns a contiguous block
+// of the CTA's 128 rows; lane l owns the 8 columns [8 l, 8 l + 8) of the
+// tile; the warp walks its rows' CSR entries as one stream, keeping a ring of
+// W-row segments (16 bytes per lane per entry) in flight, and accumulates
+// each row with fp32 FMAs in the row's CSR order.  Finished rows go to this
+// CTA's slot of a small scratch ring in global memory (2 slots of 128 x BN
+// fp32 per CTA, rewritten every other tile, so it stays in L2), and the
+// epilogue TMA-loads them exactly as it loads a caller's C.  Two barrier
+// pairs (corr_full / corr_empty) hand the slots between the two roles.  The
+// dense M x N fp32 correction never exists.
 // Every mbarrier wait is bounded; a wait that gives up sets the timeout bit in
 // the status word, raises a CTA-wide abort flag, waits (bounded) for copies
 // and MMAs in flight, frees TMEM and returns.
@@ -67,7 +79,15 @@ constexpr int kAccStages = 2;
 constexpr int kEpiWarps = QG_GEMM_EPI_WARPS;     // 4 or 8 (one or two per TMEM lane quarter)
 constexpr int kEpiSplit = kEpiWarps / 4;         // chunk stride of one epilogue warp
 static_assert(kEpiWarps == 4 || kEpiWarps == 8, "one or two epilogue warps per lane quarter");
-constexpr int kThreads = 64 + 32 * kEpiWarps;
+constexpr int kCorrWarps = 6;                    // correction warps (CORR)
+// Threads of a CTA: producer, MMA, epilogue warps (+ correction warps).  With
+// the correction warps a CTA has 384 threads, which leaves 168 registers per
+// thread: what the TMA epilogue needs.
+template <bool CORR>
+constexpr int threads_of() { return 64 + 32 * kEpiWarps + (CORR ? 32 * kCorrWarps : 0); }
+constexpr int kThreads = threads_of<false>();
+constexpr int kCorrMaxCtas = 160;                // scratch slots are sized for this many CTAs
+constexpr int kCorrSlots = 2;
 constexpr int kTmemCols = 512;
 constexpr int kSfaCol = 448;
 constexpr int kSfbCol = 480;
@@ -120,6 +140,8 @@ struct alignas(8) Barriers {
     uint64_t acc_full[kAccStages];
     uint64_t acc_empty[kAccStages];
     uint64_t cbar[kEpiWarps][kEpiBufs];
+    uint64_t corr_full[kCorrSlots];    // a tile's correction rows are in its scratch slot
+    uint64_t corr_empty[kCorrSlots];   // the epilogue has loaded them: the slot is free
     uint64_t mma_done;
     uint32_t tmem_base;
     int abort;
@@ -416,6 +438,145 @@ __device__ __forceinline__ void tmem_st32_const(uint32_t taddr, uint32_t c) {
 __device__ __forceinline__ uint32_t swz128(int r, int c) { return r * 128 + ((c ^ (r & 7)) << 4); }
 __device__ __forceinline__ uint32_t swz64(int r, int c) { return r * 64 + ((c ^ ((r >> 1) & 3)) << 4); }
 
+// ------------------------------------------------------------------ correction
+// acc (an fp32 pair) += v * (lo(w), hi(w)) for a bf16 pair w: one rounding per
+// product-sum, as fmaf.
+__device__ __forceinline__ void fma2_bf16(uint64_t& acc, uint64_t vv, uint32_t w) {
+    asm("{\n\t.reg .b32 lo, hi;\n\t.reg .b64 x;\n\t"
+        "shl.b32 lo, %2, 16;\n\tand.b32 hi, %2, 0xFFFF0000;\n\t"
+        "mov.b64 x, {lo, hi};\n\tfma.rn.f32x2 %0, x, %1, %0;\n\t}"
+        : "+l"(acc)
+        : "l"(vv), "r"(w));
+}
+// acc += v * (a, b) for an fp32 pair (a in the low word).
+__device__ __forceinline__ void fma2_f32(uint64_t& acc, uint64_t vv, uint32_t a, uint32_t b) {
+    asm("{\n\t.reg .b64 x;\n\tmov.b64 x, {%2, %3};\n\tfma.rn.f32x2 %0, x, %1, %0;\n\t}"
+        : "+l"(acc)
+        : "l"(vv), "r"(a), "r"(b));
+}
+
+// The compensation rows r_begin .. r_end - 1 (at most 31 rows) of dA . W,
+// 8 columns per lane starting at c0: for each row, the fp32 FMA chain over the
+// row's CSR entries in order, value (fp32 of the stored double) times the W
+// row segment.  The warp's entries form one contiguous CSR range, consumed as
+// a stream with D W-row segments in flight (the ring position is a
+// compile-time index: the loop over entries is unrolled by D); lane l holds
+// entry values and the columns of the entries D ahead, batch by batch of 32.
+// Row r's 8 sums go to dst + (r - r_begin) * dst_ld (lanes with lane_on).
+// vec: the 8 columns are inside W and 16-byte aligned (else element loads,
+// zero past N).
+template <bool WBF16, int D>
+__device__ __forceinline__ void corr_rows(const int32_t* __restrict__ row_ptr,
+                                          const int32_t* __restrict__ col,
+                                          const double* __restrict__ val,
+                                          const void* __restrict__ W, int64_t ldw, int r_begin,
+                                          int r_end, int N, int c0, bool lane_on, bool vec,
+                                          float* __restrict__ dst, int dst_ld) {
+    static_assert(32 % D == 0, "entry batches of 32 hold whole ring turns");
+    constexpr int SEG = WBF16 ? 1 : 2;          // 16-byte words per lane per W row segment
+    const int lane = threadIdx.x & 31;
+    const int nrows = r_end - r_begin;
+    const int rp = (lane <= nrows) ? __ldg(row_ptr + r_begin + lane) : 0;
+    const int P0 = __shfl_sync(0xFFFFFFFFu, rp, 0);
+    const int n = __shfl_sync(0xFFFFFFFFu, rp, nrows) - P0;
+    int kc = (lane < n) ? __ldg(col + P0 + lane) : 0;
+    float vc = (lane < n) ? (float)__ldg(val + P0 + lane) : 0.0f;
+    int ks;
+    {
+        const int kn = (32 + lane < n) ? __ldg(col + P0 + 32 + lane) : 0;
+        const int a = __shfl_sync(0xFFFFFFFFu, kc, (lane + D) & 31);
+        const int b = __shfl_sync(0xFFFFFFFFu, kn, (lane + D) & 31);
+        ks = (lane + D < 32) ? a : b;
+    }
+    auto fetch = [&](uint4 (&d)[SEG], int k) {
+#pragma unroll
+        for (int s = 0; s < SEG; ++s) d[s] = make_uint4(0u, 0u, 0u, 0u);
+        if (!lane_on) return;
+        if constexpr (WBF16) {
+            const uint16_t* src = static_cast<const uint16_t*>(W) + (int64_t)k * ldw + c0;
+            if (vec) {
+                d[0] = __ldg(reinterpret_cast<const uint4*>(src));
+            } else {
+                uint32_t w[4] = {0u, 0u, 0u, 0u};
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    if (c0 + e < N) w[e >> 1] |= (uint32_t)__ldg(src + e) << (16 * (e & 1));
+                d[0] = make_uint4(w[0], w[1], w[2], w[3]);
+            }
+        } else {
+            const float* src = static_cast<const float*>(W) + (int64_t)k * ldw + c0;
+            if (vec) {
+                d[0] = __ldg(reinterpret_cast<const uint4*>(src));
+                d[1] = __ldg(reinterpret_cast<const uint4*>(src) + 1);
+            } else {
+                uint32_t w[8];
+#pragma unroll
+                for (int e = 0; e < 8; ++e) w[e] = (c0 + e < N) ? __float_as_uint(__ldg(src + e)) : 0u;
+                d[0] = make_uint4(w[0], w[1], w[2], w[3]);
+                d[1] = make_uint4(w[4], w[5], w[6], w[7]);
+            }
+        }
+    };
+    uint4 buf[D][SEG];
+#pragma unroll
+    for (int u = 0; u < D; ++u)
+        if (u < n) fetch(buf[u], __shfl_sync(0xFFFFFFFFu, kc, u));
+    uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+    int row = r_begin;
+    int rend = __shfl_sync(0xFFFFFFFFu, rp, 1) - P0;   // entries of rows <= row end here
+    auto store_row = [&](int r) {
+        if (lane_on) {
+            ulonglong2* d = reinterpret_cast<ulonglong2*>(dst + (int64_t)(r - r_begin) * dst_ld);
+            d[0] = make_ulonglong2(acc[0], acc[1]);
+            d[1] = make_ulonglong2(acc[2], acc[3]);
+        }
+#pragma unroll
+        for (int e = 0; e < 4; ++e) acc[e] = 0ull;
+    };
+    for (int q = 0; q < n; q += D) {
+#pragma unroll
+        for (int u = 0; u < D; ++u) {
+            const int j = q + u;                 // entry index within the warp's range
+            if (j >= n) break;
+            while (j >= rend) {                  // rows that end before entry j
+                store_row(row);
+                ++row;
+                rend = __shfl_sync(0xFFFFFFFFu, rp, row - r_begin + 1) - P0;
+            }
+            const int t = (q & 31) + u;          // position in the batch
+            const float v = __shfl_sync(0xFFFFFFFFu, vc, t);
+            const int kf = __shfl_sync(0xFFFFFFFFu, ks, t);
+            uint64_t vv;
+            asm("mov.b64 %0, {%1, %1};" : "=l"(vv) : "f"(v));
+            if constexpr (WBF16) {
+                fma2_bf16(acc[0], vv, buf[u][0].x);
+                fma2_bf16(acc[1], vv, buf[u][0].y);
+                fma2_bf16(acc[2], vv, buf[u][0].z);
+                fma2_bf16(acc[3], vv, buf[u][0].w);
+            } else {
+                fma2_f32(acc[0], vv, buf[u][0].x, buf[u][0].y);
+                fma2_f32(acc[1], vv, buf[u][0].z, buf[u][0].w);
+                fma2_f32(acc[2], vv, buf[u][SEG - 1].x, buf[u][SEG - 1].y);
+                fma2_f32(acc[3], vv, buf[u][SEG - 1].z, buf[u][SEG - 1].w);
+            }
+            if (j + D < n) fetch(buf[u], kf);    // refill this ring position
+        }
+        if ((q & 31) == 32 - D) {                // batch done: load the next one
+            const int Bn = q + D;
+            kc = (Bn + lane < n) ? __ldg(col + P0 + Bn + lane) : 0;
+            vc = (Bn + lane < n) ? (float)__ldg(val + P0 + Bn + lane) : 0.0f;
+            const int kn = (Bn + 32 + lane < n) ? __ldg(col + P0 + Bn + 32 + lane) : 0;
+            const int a = __shfl_sync(0xFFFFFFFFu, kc, (lane + D) & 31);
+            const int b = __shfl_sync(0xFFFFFFFFu, kn, (lane + D) & 31);
+            ks = (lane + D < 32) ? a : b;
+        }
+    }
+    while (row < r_end) {                        // the last rows (and empty ones)
+        store_row(row);
+        ++row;
+    }
+}
+
 // ------------------------------------------------------------------ kernel
 struct Params {
     const float* sA;
@@ -431,11 +592,22 @@ struct Params {
     const uint8_t* sfA;  // MX: E8M0 scale atoms of A, [row block][k group]
     const uint8_t* sfB;  // MX: the same for W^T
     int sf_groups;       // MX: 128-deep k groups per row block (even)
+    // CORR: dA in CSR, the unquantized W (K x N, row pitch ldw elements, bf16
+    // or fp32) and the scratch slots (kCorrSlots x 128 x BN fp32 per CTA)
+    const int32_t* row_ptr;
+    const int32_t* col;
+    const double* val;
+    const void* Wc;
+    int64_t ldw;
+    int w_bf16;
+    float* corr;
 };
 
 // Direct epilogue of one 32-column chunk: registers -> global (row per lane).
+// crow: this row's correction at column col0 (a caller's C or a scratch slot),
+// or null; read with coherent loads, since a slot is rewritten in the kernel.
 __device__ __forceinline__ void epi_direct(const Params& p, const uint32_t (&v)[32], int row,
-                                           int col0, float s_row) {
+                                           int col0, float s_row, const float* crow) {
     const bool full = (p.N % 8) == 0 && (col0 + 32 <= p.N);
     const int64_t off = (int64_t)row * p.N + col0;
     if (p.raw_acc) {
@@ -456,7 +628,7 @@ __device__ __forceinline__ void epi_direct(const Params& p, const uint32_t (&v)[
         // 16-byte loads of C and the column scales, 16-byte stores of Y
         float* yrow = static_cast<float*>(p.Y) + off;
         const float4* tw = reinterpret_cast<const float4*>(p.sW + col0);
-        const float4* crow = p.C ? reinterpret_cast<const float4*>(p.C + off) : nullptr;
+        const float4* c4 = reinterpret_cast<const float4*>(crow);
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
             const float4 t = p.unit_scales ? make_float4(1.0f, 1.0f, 1.0f, 1.0f) : __ldg(tw + j);
@@ -464,8 +636,8 @@ __device__ __forceinline__ void epi_direct(const Params& p, const uint32_t (&v)[
                                    __fmul_rn(__fmul_rn(__uint_as_float(v[4 * j + 1]), s_row), t.y),
                                    __fmul_rn(__fmul_rn(__uint_as_float(v[4 * j + 2]), s_row), t.z),
                                    __fmul_rn(__fmul_rn(__uint_as_float(v[4 * j + 3]), s_row), t.w));
-            if (crow) {
-                const float4 c = __ldg(crow + j);
+            if (c4) {
+                const float4 c = __ldcg(c4 + j);
                 y.x = __fadd_rn(y.x, c.x);
                 y.y = __fadd_rn(y.y, c.y);
                 y.z = __fadd_rn(y.z, c.z);
@@ -480,7 +652,7 @@ __device__ __forceinline__ void epi_direct(const Params& p, const uint32_t (&v)[
         if (col0 + j >= p.N) continue;
         const float tj = p.unit_scales ? 1.0f : __ldg(p.sW + col0 + j);
         float yy = __fmul_rn(__fmul_rn(__uint_as_float(v[j]), s_row), tj);
-        if (p.C) yy = __fadd_rn(yy, __ldg(p.C + off + j));
+        if (crow) yy = __fadd_rn(yy, __ldcg(crow + j));
         if (p.y_bf16) static_cast<__nv_bfloat16*>(p.Y)[off + j] = __float2bfloat16_rn(yy);
         else static_cast<float*>(p.Y)[off + j] = yy;
     }
@@ -489,14 +661,15 @@ __device__ __forceinline__ void epi_direct(const Params& p, const uint32_t (&v)[
 // TMA_EPI: Y (and C) go through the swizzled sub-tile buffers and TMA; the
 // other instantiation stores registers directly (raw accumulator output, or
 // row pitches TMA cannot describe), so neither path's registers burden the other.
-template <int BN, bool PAIR, bool TMA_EPI, bool MX = false>
-__global__ void __launch_bounds__(kThreads, 1)
+template <int BN, bool PAIR, bool TMA_EPI, bool MX = false, bool CORR = false>
+__global__ void __launch_bounds__(threads_of<CORR>(), 1)
 fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 const __grid_constant__ CUtensorMap tmap_b,
                 const __grid_constant__ CUtensorMap tmap_y,
                 const __grid_constant__ CUtensorMap tmap_c, const Params p) {
     using CF = Cfg<BN, PAIR, MX>;
     constexpr int S = CF::kStages;
+    static_assert(!(CORR && MX), "the compensated GEMM uses per-row / per-column scales");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
         (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~(uintptr_t)1023);
@@ -528,6 +701,10 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         }
         for (int w = 0; w < kEpiWarps; ++w)
             for (int b = 0; b < kEpiBufs; ++b) mbar_init(&B->cbar[w][b], 1);
+        for (int s = 0; s < kCorrSlots; ++s) {
+            mbar_init(&B->corr_full[s], kCorrWarps);
+            mbar_init(&B->corr_empty[s], kEpiWarps);
+        }
         mbar_init(&B->mma_done, 1);
         B->abort = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -543,7 +720,7 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     tc_fence_after();
     const uint32_t tmem = B->tmem_base;
 
-    if (warp >= 2) {
+    if (warp >= 2 && warp < 2 + kEpiWarps) {
         // constant block scales: every byte 0x7F (UE8M0 2^0) in the scale region
         const uint32_t q = (uint32_t)(warp & 3);
         tmem_st32_const(tmem + ((32u * q) << 16) + kSfaCol, 0x7F7F7F7Fu);
@@ -669,7 +846,7 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             tc_commit_local<PAIR>(&B->mma_done);
             mbar_drain(&B->mma_done, 0);
         }
-    } else {
+    } else if (warp < 2 + kEpiWarps) {
         // ---------------------------------------------------------- epilogue
         // Two warps per TMEM lane quarter when kEpiSplit == 2: warp ew takes
         // the chunks c with c % kEpiSplit == ew / 4.  Each warp walks its
@@ -686,25 +863,38 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
         uint8_t* bufs = sepi + (size_t)ew * kEpiBufs * kEpiBuf;
         float* sw = reinterpret_cast<float*>(smem + CF::kOffSw) + ew * SWR * 32;
-        const bool use_c = TMA_EPI && p.C != nullptr;
+        const bool use_c = TMA_EPI && (CORR || p.C != nullptr);
         const int my_tiles = unit < num_tiles ? (num_tiles - unit + n_units - 1) / n_units : 0;
         const int total = my_tiles * my_nc;
         uint32_t cphase = 0;                   // bit b: parity of the next wait on cbar[ew][b]
         uint32_t cpend = 0;                    // bit b: a C load into buffer b not yet waited for
-        auto c_load = [&](int g) {
+        // C sub-tile of chunk g: from the caller's C, or (CORR) from this CTA's
+        // scratch slot of the chunk's tile, once the correction warps have
+        // filled it.  False when a wait gave up.
+        auto c_load = [&](int g) -> bool {
             const int ti = g / my_nc, c = par + kEpiSplit * (g - ti * my_nc);
             const int tile = unit + ti * n_units;
             const int mb = tile % num_m, nbk = tile / num_m;
             const int b = g % kEpiBufs;
+            int x = nbk * BN + c * 32, y = mb * CF::kTileRows + (int)rank * BM + 32 * q;
+            if constexpr (CORR) {
+                if (g == ti * my_nc &&
+                    !mbar_wait_warp(&B->corr_full[ti & 1], (uint32_t)(ti >> 1) & 1u, &B->abort,
+                                    p.status))
+                    return false;
+                x = c * 32;
+                y = ((int)blockIdx.x * kCorrSlots + (ti & 1)) * BM + 32 * q;
+            }
             if (lane == 0) {
                 mbar_expect_tx(&B->cbar[ew][b], kEpiBuf);
-                tma_load_2d(&tmap_c, &B->cbar[ew][b], bufs + b * kEpiBuf, nbk * BN + c * 32,
-                            mb * CF::kTileRows + (int)rank * BM + 32 * q);
+                tma_load_2d(&tmap_c, &B->cbar[ew][b], bufs + b * kEpiBuf, x, y);
             }
             cpend |= 1u << b;
+            return true;
         };
+        bool ok = true;
         if (use_c)
-            for (int g = 0; g < kEpiBufs - 1 && g < total; ++g) c_load(g);
+            for (int g = 0; ok && g < kEpiBufs - 1 && g < total; ++g) ok = c_load(g);
         // scales of tile ti into registers (consumed one tile later)
         float swr[SWR];
         float srow_next = 0.0f;
@@ -725,7 +915,6 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         if (my_tiles > 0) fetch_scales(0);
         int as = 0;
         uint32_t acc_phase = 0;
-        bool ok = true;
         uint32_t va[32], vb[32];
         for (int ti = 0; ok && ti < my_tiles; ++ti) {
             const int tile = unit + ti * n_units;
@@ -744,6 +933,17 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 break;
             }
             tc_fence_after();
+            // direct epilogue with the fused correction: this tile's slot rows
+            const float* cslot = nullptr;
+            if constexpr (CORR && !TMA_EPI) {
+                if (!mbar_wait_warp(&B->corr_full[ti & 1], (uint32_t)(ti >> 1) & 1u, &B->abort,
+                                    p.status)) {
+                    ok = false;
+                    break;
+                }
+                cslot = p.corr + ((size_t)((int)blockIdx.x * kCorrSlots + (ti & 1)) * BM +
+                                  32 * q + lane) * BN;
+            }
             const uint32_t tbase = tmem + lane_base + (uint32_t)(as * BN);
             auto release_acc = [&]() {
                 // this warp's chunks fully read: the next tile's MMAs may reuse
@@ -760,7 +960,14 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 const int c = par + kEpiSplit * h;
                 const int col0 = n_blk * BN + c * 32;
                 if constexpr (!TMA_EPI) {
-                    if (row < p.M && col0 < p.N) epi_direct(p, v, row, col0, s_row);
+                    const float* crow = CORR ? cslot + c * 32
+                                             : (p.C ? p.C + (int64_t)row * p.N + col0 : nullptr);
+                    if (row < p.M && col0 < p.N) epi_direct(p, v, row, col0, s_row, crow);
+                    if (CORR && h == my_nc - 1) {
+                        // every chunk of the tile is read: the slot may be refilled
+                        __syncwarp();
+                        if (lane == 0) mbar_arrive(&B->corr_empty[ti & 1]);
+                    }
                     return true;
                 }
                 const int g = ti * my_nc + h;
@@ -789,6 +996,11 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
 #pragma unroll
                         for (int e = 0; e < 4; ++e)
                             v[4 * j + e] = __float_as_uint(__fadd_rn(__uint_as_float(v[4 * j + e]), tt[e]));
+                    }
+                    if (CORR && h == my_nc - 1 && lane == 0) {
+                        // the tile's last C sub-tile has landed: every TMA read of
+                        // its scratch slot is done, the slot may be refilled
+                        mbar_arrive(&B->corr_empty[ti & 1]);
                     }
                 } else {
                     // buffer b was last read by the store of chunk g - kEpiBufs
@@ -822,7 +1034,7 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 if (use_c && g + kEpiBufs - 1 < total) {
                     // that buffer was last read by the store of chunk g - 1
                     if (lane == 0) bulk_wait_read<1>();
-                    c_load(g + kEpiBufs - 1);
+                    if (!c_load(g + kEpiBufs - 1)) return false;
                 }
                 return true;
             };
@@ -856,6 +1068,44 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 if ((cpend >> b) & 1u) mbar_drain(&B->cbar[ew][b], (cphase >> b) & 1u);
         }
         __syncwarp();
+    } else if constexpr (CORR) {
+        // ---------------------------------------------------------- correction
+        // Warp cw owns rows [r_lo, r_hi) of the CTA's 128 (one contiguous CSR
+        // range per tile); tiles in the CTA's order, slot ti % 2.
+        const int cw = warp - 2 - kEpiWarps;
+        const int r_lo = (cw * BM) / kCorrWarps, r_hi = ((cw + 1) * BM) / kCorrWarps;
+        const int my_tiles = unit < num_tiles ? (num_tiles - unit + n_units - 1) / n_units : 0;
+        const bool lane_on = lane * 8 < BN;
+        for (int ti = 0; ti < my_tiles; ++ti) {
+            const int tile = unit + ti * n_units;
+            const int m_blk = tile % num_m, n_blk = tile / num_m;
+            const int slot = ti & 1;
+            if (!mbar_wait_warp(&B->corr_empty[slot], ((uint32_t)(ti >> 1) & 1u) ^ 1u, &B->abort,
+                                p.status))
+                break;
+            const int row0 = m_blk * CF::kTileRows + (int)rank * BM;
+            const int rb = min(p.M, row0 + r_lo), re = min(p.M, row0 + r_hi);
+            const int c0 = n_blk * BN + lane * 8;
+            float* dst = p.corr + ((size_t)((int)blockIdx.x * kCorrSlots + slot) * BM + r_lo) * BN +
+                         lane * 8;
+            const bool on = lane_on && c0 < p.N;
+            if (rb < re) {
+                if (p.w_bf16) {
+                    const bool vec = c0 + 8 <= p.N && (p.ldw % 8) == 0;
+                    corr_rows<true, 16>(p.row_ptr, p.col, p.val, p.Wc, p.ldw, rb, re, p.N, c0, on,
+                                        vec, dst, BN);
+                } else {
+                    const bool vec = c0 + 8 <= p.N && (p.ldw % 4) == 0;
+                    corr_rows<false, 8>(p.row_ptr, p.col, p.val, p.Wc, p.ldw, rb, re, p.N, c0, on,
+                                        vec, dst, BN);
+                }
+            }
+            // the rows are written (generic proxy); the epilogue reads them by
+            // TMA (async proxy) once every correction warp has arrived
+            asm volatile("fence.proxy.async.global;" ::: "memory");
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&B->corr_full[slot]);
+        }
     }
 
     tc_fence_before();
@@ -915,7 +1165,19 @@ static int pick_bn(int64_t M, int64_t N, bool pair) {
     return (w192 < w224) ? 192 : 224;
 }
 
-template <int BN, bool PAIR, bool TMA_EPI, bool MX = false>
+// CTAs of the persistent grid (units of one CTA or one pair, at most one per
+// SM, and at most kCorrMaxCtas with the fused correction).
+template <int BN, bool PAIR, bool CORR = false>
+static int grid_ctas(int64_t M, int64_t N) {
+    using CF = Cfg<BN, PAIR, false>;
+    const int64_t tiles = ((M + CF::kTileRows - 1) / CF::kTileRows) * ((N + BN - 1) / BN);
+    const int per_unit = PAIR ? 2 : 1;
+    int64_t units = std::min<int64_t>(tiles, num_sms() / per_unit);
+    if (CORR) units = std::min<int64_t>(units, kCorrMaxCtas / per_unit);
+    return (int)std::max<int64_t>(units, 1) * per_unit;
+}
+
+template <int BN, bool PAIR, bool TMA_EPI, bool MX = false, bool CORR = false>
 static cudaError_t launch_variant(const CUtensorMap& ta, const uint8_t* codesWT, int64_t N,
                                   int64_t K, const CUtensorMap& ty, const CUtensorMap& tc,
                                   const Params& p, cudaStream_t s) {
@@ -926,10 +1188,12 @@ static cudaError_t launch_variant(const CUtensorMap& ta, const uint8_t* codesWT,
         return cudaErrorInvalidValue;
     const int64_t tiles = ((p.M + CF::kTileRows - 1) / CF::kTileRows) * ((N + BN - 1) / BN);
     const int per_unit = PAIR ? 2 : 1;
-    const int units = (int)std::min<int64_t>(tiles, num_sms() / per_unit);
+    int64_t max_units = num_sms() / per_unit;
+    if (CORR) max_units = std::min<int64_t>(max_units, kCorrMaxCtas / per_unit);
+    const int units = (int)std::min<int64_t>(tiles, max_units);
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(units * per_unit));
-    cfg.blockDim = dim3(kThreads);
+    cfg.blockDim = dim3(threads_of<CORR>());
     cfg.dynamicSmemBytes = smem_bytes<BN, PAIR, MX>();
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
@@ -939,18 +1203,19 @@ static cudaError_t launch_variant(const CUtensorMap& ta, const uint8_t* codesWT,
     attr[0].val.clusterDim.z = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaError_t e = cudaLaunchKernelEx(&cfg, fp4_gemm_kernel<BN, PAIR, TMA_EPI, MX>, ta, tb, ty, tc, p);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, fp4_gemm_kernel<BN, PAIR, TMA_EPI, MX, CORR>, ta, tb,
+                                       ty, tc, p);
     count_launch(1);
     return e;
 }
 
-template <int BN, bool PAIR, bool MX = false>
+template <int BN, bool PAIR, bool MX = false, bool CORR = false>
 static cudaError_t set_smem_attr() {
-    cudaError_t e = cudaFuncSetAttribute(fp4_gemm_kernel<BN, PAIR, true, MX>,
+    cudaError_t e = cudaFuncSetAttribute(fp4_gemm_kernel<BN, PAIR, true, MX, CORR>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem_bytes<BN, PAIR, MX>());
     if (e != cudaSuccess) return e;
-    return cudaFuncSetAttribute(fp4_gemm_kernel<BN, PAIR, false, MX>,
+    return cudaFuncSetAttribute(fp4_gemm_kernel<BN, PAIR, false, MX, CORR>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
                                 (int)smem_bytes<BN, PAIR, MX>());
 }
@@ -964,8 +1229,16 @@ cudaError_t gemm_setup() {
     if ((e = set_smem_attr<192, false>()) != cudaSuccess) return e;
     if ((e = set_smem_attr<224, true>()) != cudaSuccess) return e;
     if ((e = set_smem_attr<128, false, true>()) != cudaSuccess) return e;
-    return set_smem_attr<192, true>();
+    if ((e = set_smem_attr<192, true>()) != cudaSuccess) return e;
+    if ((e = set_smem_attr<224, false, false, true>()) != cudaSuccess) return e;
+    if ((e = set_smem_attr<192, false, false, true>()) != cudaSuccess) return e;
+    if ((e = set_smem_attr<224, true, false, true>()) != cudaSuccess) return e;
+    return set_smem_attr<192, true, false, true>();
 }
+
+static_assert(kCorrScratchBytes ==
+                  (size_t)gemm::kCorrMaxCtas * gemm::kCorrSlots * gemm::BM * 224 * sizeof(float),
+              "scratch of the fused correction: two 128 x 224 fp32 slots per CTA");
 
 // Returns cudaErrorInvalidValue when the tensor maps cannot be built.
 cudaError_t launch_fp4_gemm(const uint8_t* codesA, const float* sA, const uint8_t* codesWT,
@@ -973,7 +1246,7 @@ cudaError_t launch_fp4_gemm(const uint8_t* codesA, const float* sA, const uint8_
                             void* Y, qg_dtype y_dtype, float* raw_acc, uint32_t* status,
                             cudaStream_t s) {
     using namespace gemm;
-    Params p;
+    Params p{};
     p.sA = sA;
     p.sW = sW;
     p.C = C;
@@ -1037,13 +1310,89 @@ cudaError_t launch_fp4_gemm(const uint8_t* codesA, const float* sA, const uint8_
     return launch_variant<224, false, false>(ta, codesWT, N, K, ty, tc, p, s);
 }
 
+// The compensated GEMM: Y = acc * sA_i * sW_j + (dA . W)_ij, the correction
+// computed inside the GEMM kernel (CORR) into scratch slots of `scratch`
+// (corr_scratch_bytes()).  Returns cudaErrorInvalidValue when the tensor maps
+// cannot be built.
+cudaError_t launch_fp4_gemm_corr(const uint8_t* codesA, const float* sA, const uint8_t* codesWT,
+                                 const float* sW, int64_t M, int64_t N, int64_t K,
+                                 const qg_csr* dA, const void* W, qg_dtype w_dtype, int64_t ldw,
+                                 float* scratch, void* Y, qg_dtype y_dtype, uint32_t* status,
+                                 cudaStream_t s) {
+    using namespace gemm;
+    Params p{};
+    p.sA = sA;
+    p.sW = sW;
+    p.C = nullptr;
+    p.Y = Y;
+    p.raw_acc = nullptr;
+    p.status = status;
+    p.M = (int)M;
+    p.N = (int)N;
+    p.K = (int)K;
+    p.y_bf16 = (y_dtype == QG_BF16) ? 1 : 0;
+    p.unit_scales = 0;
+    p.sfA = nullptr;
+    p.sfB = nullptr;
+    p.sf_groups = 0;
+    p.row_ptr = dA->row_ptr;
+    p.col = dA->col;
+    p.val = dA->val;
+    p.Wc = W;
+    p.ldw = ldw;
+    p.w_bf16 = (w_dtype == QG_BF16) ? 1 : 0;
+    p.corr = scratch;
+    const size_t ysz = (y_dtype == QG_BF16) ? 2 : 4;
+    p.tma_epi = (!QG_GEMM_DIRECT_EPI && ((size_t)N * ysz) % 16 == 0) ? 1 : 0;
+    const bool pair = M > BM;
+    const int bn = QG_GEMM_FORCE_BN ? QG_GEMM_FORCE_BN : pick_bn(p.M, N, pair);
+    const int ctas = pair ? (bn == 192 ? grid_ctas<192, true, true>(M, N) : grid_ctas<224, true, true>(M, N))
+                          : (bn == 192 ? grid_ctas<192, false, true>(M, N) : grid_ctas<224, false, true>(M, N));
+    CUtensorMap ta, ty, tc;
+    if (!encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, codesA, K / 2, M, K / 2, BK_BYTES, BM,
+                   CU_TENSOR_MAP_SWIZZLE_128B))
+        return cudaErrorInvalidValue;
+    ty = ta;
+    tc = ta;
+    if (p.tma_epi) {
+        if (y_dtype == QG_BF16) {
+            if (!encode_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, Y, N, M, N * 2, 32, 32,
+                           CU_TENSOR_MAP_SWIZZLE_64B))
+                return cudaErrorInvalidValue;
+        } else {
+            if (!encode_2d(&ty, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, Y, N, M, N * 4, 32, 32,
+                           CU_TENSOR_MAP_SWIZZLE_128B))
+                return cudaErrorInvalidValue;
+        }
+        // the scratch as a (ctas x slots x 128) x bn fp32 matrix
+        if (!encode_2d(&tc, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, scratch, bn,
+                       (uint64_t)ctas * kCorrSlots * BM, (uint64_t)bn * 4, 32, 32,
+                       CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+    }
+    if (pair) {
+        if (p.tma_epi) {
+            if (bn == 192) return launch_variant<192, true, true, false, true>(ta, codesWT, N, K, ty, tc, p, s);
+            return launch_variant<224, true, true, false, true>(ta, codesWT, N, K, ty, tc, p, s);
+        }
+        if (bn == 192) return launch_variant<192, true, false, false, true>(ta, codesWT, N, K, ty, tc, p, s);
+        return launch_variant<224, true, false, false, true>(ta, codesWT, N, K, ty, tc, p, s);
+    }
+    if (p.tma_epi) {
+        if (bn == 192) return launch_variant<192, false, true, false, true>(ta, codesWT, N, K, ty, tc, p, s);
+        return launch_variant<224, false, true, false, true>(ta, codesWT, N, K, ty, tc, p, s);
+    }
+    if (bn == 192) return launch_variant<192, false, false, false, true>(ta, codesWT, N, K, ty, tc, p, s);
+    return launch_variant<224, false, false, false, true>(ta, codesWT, N, K, ty, tc, p, s);
+}
+
 // MXFP4 GEMM: Y = sum over 32-blocks of 2^(eA + eW) * (block product) (+ C).
 cudaError_t launch_fp4_gemm_mx(const uint8_t* codesA, const uint8_t* sfA, const uint8_t* codesWT,
                                const uint8_t* sfW, int64_t M, int64_t N, int64_t K, const float* C,
                                void* Y, qg_dtype y_dtype, float* raw_acc, uint32_t* status,
                                cudaStream_t s) {
     using namespace gemm;
-    Params p;
+    Params p{};
     p.sA = nullptr;
     p.sW = nullptr;
     p.C = C;

@@ -70,6 +70,10 @@ struct GridSync {
 };
 constexpr size_t kGridSyncOffset = 16;   // bytes from the workspace base
 
+// Scratch of the compensated GEMM: two slots of 128 rows x 224 fp32 columns
+// per CTA, for up to 160 CTAs (36.7 MB; it stays in L2).
+constexpr size_t kCorrScratchBytes = (size_t)160 * 2 * 128 * 224 * 4;
+
 struct WsLayout {
     size_t gsync = 0;
     size_t rowpre = 0;
@@ -77,7 +81,7 @@ struct WsLayout {
     size_t status = 0, counters = 0, hist1 = 0, hist2 = 0, rowmax = 0, rowcnt = 0;
     size_t st_row = 0, st_rank = 0, st_col = 0, st_val = 0, colmax = 0;
     size_t act_codes = 0, act_scales = 0, csr_row_ptr = 0, csr_col = 0, csr_val = 0,
-           csr_nnz = 0, thr = 0, corr = 0;
+           csr_nnz = 0, thr = 0, corr_scratch = 0;
     size_t total = 0;
     int64_t cap = 0;
     int64_t row_slots = 0;
@@ -149,8 +153,10 @@ inline WsLayout ws_layout(qg_op op, int64_t M, int64_t K, int64_t N, qg_dtype dt
         L.csr_val = take(sizeof(double) * (size_t)cap);
         L.csr_nnz = take(sizeof(int64_t));
         L.thr = take(sizeof(float));
-        L.corr = take(sizeof(float) * (size_t)M * (size_t)N);
     }
+    // the compensated GEMM's scratch slots (the layer call and the GEMM alone)
+    if (op == QG_OP_FP4_LINEAR || op == QG_OP_FP4_GEMM_COMPENSATED)
+        L.corr_scratch = take(kCorrScratchBytes);
     L.total = off;
     return L;
 }
@@ -387,6 +393,11 @@ cudaError_t launch_fp4_gemm(const uint8_t* codesA, const float* sA, const uint8_
                             const float* sW, int64_t M, int64_t N, int64_t K, const float* C,
                             void* Y, qg_dtype y_dtype, float* raw_acc, uint32_t* status,
                             cudaStream_t s);
+cudaError_t launch_fp4_gemm_corr(const uint8_t* codesA, const float* sA, const uint8_t* codesWT,
+                                 const float* sW, int64_t M, int64_t N, int64_t K,
+                                 const qg_csr* dA, const void* W, qg_dtype w_dtype, int64_t ldw,
+                                 float* scratch, void* Y, qg_dtype y_dtype, uint32_t* status,
+                                 cudaStream_t s);
 cudaError_t run_quantize_act(const void* A, qg_dtype dt, int64_t M, int64_t K, int64_t lda,
                              int64_t rank, const ActBuffers& b, uint8_t* codes, float* scales,
                              const qg_csr* dA, float* T_out, cudaStream_t s);

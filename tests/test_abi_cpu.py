@@ -52,16 +52,23 @@ def test_rank_convention_matches_oracle(qg):
 
 
 def test_workspace_sizes(qg):
-    for op in range(9):
+    for op in range(10):
         for (M, K, N, dt, a) in ((1, 32, 1, 0, 1.0), (256, 512, 512, 0, 0.99),
                                  (4096, 2048, 5504, 1, 0.99), (16384, 11008, 4096, 1, 0.999)):
             s = qg.qg_workspace_size(op, M, K, N, dt, a)
             assert s >= 256 and s % 256 == 0
-    # the layer's workspace holds at least the fp32 correction and the CSR
+    # the layer's workspace holds the activation codes, the CSR and the fixed
+    # scratch slots of the compensated GEMM, but no M x N correction: it does
+    # not grow with N
     M, K, N = 4096, 2048, 5504
     s = qg.qg_workspace_size(qg.QG_OP_FP4_LINEAR, M, K, N, qg.QG_BF16, 0.99)
     cap = qg.qg_nnz_capacity(M * K, 0.99)
-    assert s >= 4 * M * N + 12 * cap + M * K // 2
+    scratch = 160 * 2 * 128 * 224 * 4
+    assert s >= scratch + 12 * cap + M * K // 2
+    assert s == qg.qg_workspace_size(qg.QG_OP_FP4_LINEAR, M, K, 4 * N, qg.QG_BF16, 0.99)
+    assert s < 4 * M * N
+    g = qg.qg_workspace_size(qg.QG_OP_FP4_GEMM_COMPENSATED, M, K, N, qg.QG_F32, 1.0)
+    assert scratch <= g < scratch + 4096
     # staging grows as alpha falls
     a = qg.qg_workspace_size(qg.QG_OP_QUANTIZE_ACT, M, K, 1, qg.QG_BF16, 0.999)
     b = qg.qg_workspace_size(qg.QG_OP_QUANTIZE_ACT, M, K, 1, qg.QG_BF16, 0.99)
@@ -234,3 +241,32 @@ def test_linear_parts_offsets(qg):
     assert qg.qg_fp4_linear_parts(64, 48, 64, qg.QG_BF16, 0.99)[0] == qg.QG_ERR_UNSUPPORTED_SHAPE
     assert qg.qg_fp4_linear_parts(64, 64, 64, qg.QG_BF16, 0.0)[0] == qg.QG_ERR_INVALID_ARG
     assert qg._lib.qg_fp4_linear_parts(64, 64, 64, qg.QG_BF16, 0.99, None) == qg.QG_ERR_INVALID_ARG
+
+
+def test_compensated_gemm_host_checks(qg):
+    """The compensated GEMM rejects a missing CSR, a short weight pitch, a
+    misaligned W and a short workspace before anything is enqueued."""
+    lib = qg._lib
+    P = ctypes.c_void_p
+    fake = P(1 << 20)
+    big = 1 << 30
+    csr = qg._Csr(1 << 20, 1 << 20, 1 << 20, 1000, 1 << 20)
+    nocol = qg._Csr(1 << 20, 0, 1 << 20, 1000, 1 << 20)
+    M, N, K = 256, 512, 512
+    args = lambda c, W, ldw, ws_bytes: (fake, fake, fake, fake, M, N, K, c, W, 1, ldw, fake, 0,
+                                        fake, ws_bytes, None)
+    need = qg.qg_workspace_size(qg.QG_OP_FP4_GEMM_COMPENSATED, M, K, N, qg.QG_F32, 1.0)
+    before = qg.qg_launch_count()
+    assert lib.qg_fp4_gemm_compensated(*args(None, fake, N, big)) == qg.QG_ERR_INVALID_ARG
+    assert lib.qg_fp4_gemm_compensated(*args(ctypes.byref(nocol), fake, N, big)) == \
+        qg.QG_ERR_INVALID_ARG
+    assert lib.qg_fp4_gemm_compensated(*args(ctypes.byref(csr), fake, N - 1, big)) == \
+        qg.QG_ERR_INVALID_ARG
+    assert lib.qg_fp4_gemm_compensated(*args(ctypes.byref(csr), P((1 << 20) + 2), N, big)) == \
+        qg.QG_ERR_INVALID_ARG
+    assert lib.qg_fp4_gemm_compensated(*args(ctypes.byref(csr), fake, N, need - 256)) == \
+        qg.QG_ERR_WORKSPACE
+    bad_k = (fake, fake, fake, fake, M, N, 48, ctypes.byref(csr), fake, 1, N, fake, 0, fake, big,
+             None)
+    assert lib.qg_fp4_gemm_compensated(*bad_k) == qg.QG_ERR_UNSUPPORTED_SHAPE
+    assert qg.qg_launch_count() == before

@@ -392,6 +392,54 @@ def test_fp4_gemm_epilogue_bf16(qg):
     assert np.all(err <= bf16_ulp(Yo))
 
 
+# ------------------------------------------------------------ compensated GEMM
+COMP_CASES = [  # (activation case, N, W dtype, Y dtype)
+    ("tiny", 512, torch.float32, torch.float32),
+    ("llama1.3b_attn_m512", 2048, torch.bfloat16, torch.float32),
+    ("llama1.3b_attn_m512", 2048, torch.bfloat16, torch.bfloat16),
+    ("llama7b_down_m256", 4096, torch.bfloat16, torch.float32),
+    ("ragged_k1056_fp32", 100, torch.float32, torch.float32),     # ragged last column group
+    ("bf16_ragged_k1056", 257, torch.bfloat16, torch.float32),    # Y pitch not 16 B: direct stores
+    ("bf16_ragged_k1056", 264, torch.bfloat16, torch.bfloat16),
+    ("clamp_almost_all", 264, torch.bfloat16, torch.float32),     # every row full of entries
+    ("no_clamp", 600, torch.bfloat16, torch.float32),             # no entries at all
+    ("ties_at_T", 64, torch.bfloat16, torch.float32),             # 8 rows: one CTA, not a pair
+    ("single_row", 1056, torch.bfloat16, torch.bfloat16),
+]
+
+
+@pytest.mark.parametrize("case,N,wdtype,ydtype", COMP_CASES)
+def test_fp4_gemm_compensated(qg, case, N, wdtype, ydtype):
+    """The GEMM with the compensation computed inside it equals, bit for bit,
+    the two-kernel path (SpMM into C, then the GEMM adding C), and Y is within
+    the layer's tolerance of the oracle."""
+    A, alpha = _act_inputs(case)
+    M, K = A.shape
+    W = make_matrix((K, N), seed=K + 3 * N, device="cuda", dtype=wdtype, scale=0.02)
+    codes, scales, csr, T = qg.quantize_act(A, alpha)
+    codesT, t = qg.quantize_cols(W)
+    ws = qg.Workspace(qg.QG_OP_FP4_GEMM_COMPENSATED, M, K, N, qg.QG_F32)
+    Y = qg.fp4_gemm_compensated(codes, scales, codesT, t, K, csr, W, out_dtype=ydtype, ws=ws)
+    qg.check_status(ws, case)
+    C = qg.spmm_correction(csr, M, W)
+    Y2 = qg.fp4_gemm(codes, scales, codesT, t, K, C=C, out_dtype=ydtype)
+    torch.cuda.synchronize()
+    assert torch.equal(Y, Y2)
+    # the same workspace again: the scratch slots keep the last call's rows
+    Y3 = qg.fp4_gemm_compensated(codes, scales, codesT, t, K, csr, W, out_dtype=ydtype, ws=ws)
+    qg.check_status(ws, case)
+    assert torch.equal(Y3, Y)
+    rp, col, val = csr.to_host()
+    oT, ot = oracle.quantize_cols(W.cpu())
+    acc = oracle.gemm_acc(_np(codes), oT, K)
+    Yo = oracle.linear_y(acc, _np(scales), ot, rp, col, val, W.cpu())
+    if ydtype == torch.float32:
+        assert y_rel_err(_np(Y), Yo) <= 1e-3
+    else:
+        rms = np.sqrt(np.mean(Yo ** 2))
+        assert np.all(np.abs(_np(Y.float()).astype(np.float64) - Yo) <= bf16_ulp(Yo) + 1e-6 * rms)
+
+
 # ------------------------------------------------------------------ the layer
 def _linear_oracle(A, W, alpha, rows=None):
     act = oracle.quantize_act(A.cpu(), alpha)
