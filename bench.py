@@ -287,6 +287,16 @@ def _measure(qg, layers, steps, flush, world, device, no_graph):
                 graph=used_graph, wall=wall)
 
 
+def _mma_loop_peak():
+    """The E2M1 rate measured by the library's MMA-only loop (2-SM pairs, the
+    GEMM's form for M > 128), from the committed summary, or None."""
+    path = os.path.join(ROOT, "profiles", "fp4_mma_peak.json")
+    if not os.path.exists(path):
+        return None
+    with open(path) as f:
+        return float(json.load(f)["pair_tflops"])
+
+
 def _kernel_rows(layers, per_kernel, steps, peaks, sm_mhz, n_sm):
     """Each kernel's achieved rate against the roofline that bounds it: its
     algorithmic bytes or flops per step (defined below, per kernel) over its
@@ -317,8 +327,11 @@ def _kernel_rows(layers, per_kernel, steps, peaks, sm_mhz, n_sm):
                 bound, unit, peak, algo = "alu", "TFLOP/s", alu_peak, alu_flops / 1e12
             else:
                 bound, unit, peak, algo = "hbm", "GB/s", peaks["hbm_gbs"], byts / 1e9
+            loop = _mma_loop_peak()
             extra = {"fp4_tflops": round(flops / t / 1e12, 1) if t > 0 else 0.0,
                      "frac_of_9pf_datasheet": round(flops / t / 9e15, 4) if t > 0 else 0.0,
+                     "frac_of_mma_loop": (round(flops / t / 1e12 / loop, 4)
+                                          if t > 0 and loop else None),
                      "compensation_tflops": round(alu_flops / t / 1e12, 2) if t > 0 else 0.0,
                      "ceilings_ms": {"tensor": round(1e3 * t_tensor, 4),
                                      "alu": round(1e3 * t_alu, 4), "hbm": round(1e3 * t_hbm, 4)},
