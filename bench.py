@@ -161,8 +161,8 @@ class Layer:
         self.Y = torch.empty((M, N), dtype=torch.float32, device=device)
         self.ws_cols = qg.Workspace(qg.QG_OP_QUANTIZE_COLS, 1, K, N, dt, device=device)
         self.ws_act = qg.Workspace(qg.QG_OP_QUANTIZE_ACT, M, K, 1, dt, a_size, device=device)
-        self.ws_gemm = qg.Workspace(qg.QG_OP_FP4_GEMM_COMPENSATED, M, K, N, qg.QG_F32,
-                                    device=device)
+        self.ws_spmm = qg.Workspace(qg.QG_OP_SPMM, M, K, N, dt, device=device)
+        self.ws_gemm = qg.Workspace(qg.QG_OP_FP4_GEMM, M, K, N, qg.QG_F32, device=device)
         self.ws_lin = None          # allocated by the e2e arm
         self.dt = dt
         self.flops = 2 * M * N * K
@@ -170,18 +170,19 @@ class Layer:
         self.w_bytes = K * N * self.W.element_size()
 
     def workspaces(self):
-        return tuple(w for w in (self.ws_cols, self.ws_act, self.ws_gemm, self.ws_lin)
+        return tuple(w for w in (self.ws_cols, self.ws_act, self.ws_spmm, self.ws_gemm, self.ws_lin)
                      if w is not None)
 
 
-KERNELS = ("quantize_cols", "quantize_act", "fp4_gemm_compensated")
+KERNELS = ("quantize_cols", "quantize_act", "spmm", "fp4_gemm")
 
 
 def run_step(qg, layers, ev=None):
-    """One pass of the hot path over every layer: the weight quantizer, the
-    fused activation quantizer (threshold, clamp, dA, codes) and the FP4 GEMM
-    whose kernel also computes dA . W.  With `ev`, record events around each
-    of the three calls of each layer (same stream)."""
+    """One pass of the hot path over every layer, the calls qg_fp4_linear
+    makes for fp32 Y: the weight quantizer, the fused activation quantizer
+    (threshold, clamp, dA, codes), the compensation dA . W written into Y, and
+    the FP4 GEMM adding the scaled product to Y in place.  With `ev`, record
+    events around each of the four calls of each layer (same stream)."""
     def _chk(st, where):
         if st != qg.QG_OK:
             raise qg.QGError(st, where)
@@ -194,10 +195,13 @@ def run_step(qg, layers, ev=None):
         _chk(qg.qg_quantize_act(L.A, L.alpha, L.codes, L.s, L.csr, L.T, L.ws_act), "quantize_act")
         if ev is not None:
             ev[i][2].record()
-        _chk(qg.qg_fp4_gemm_compensated(L.codes, L.s, L.codesT, L.t, L.M, L.N, L.K, L.csr, L.W,
-                                        L.Y, L.ws_gemm), "fp4_gemm_compensated")
+        _chk(qg.qg_spmm_correction(L.csr, L.M, L.W, L.Y, L.ws_spmm), "spmm")
         if ev is not None:
             ev[i][3].record()
+        _chk(qg.qg_fp4_gemm(L.codes, L.s, L.codesT, L.t, L.M, L.N, L.K, L.Y, L.Y, None,
+                            L.ws_gemm), "fp4_gemm")
+        if ev is not None:
+            ev[i][4].record()
 
 
 def capture_step(qg, layers):
@@ -307,7 +311,33 @@ def _kernel_rows(layers, per_kernel, steps, peaks, sm_mhz, n_sm):
     for k in KERNELS:
         kms = sum(per_kernel[k]) / steps
         t = kms * 1e-3
-        if k == "fp4_gemm_compensated":
+        if k == "fp4_gemm":
+            # the GEMM moves the FP4 codes, the scales, the fp32 compensation
+            # (read from Y) and Y (fp32, written in place); its bound is
+            # whichever of the tensor-core time and the HBM time is longer
+            flops = sum(L.flops for L in layers)
+            byts = sum(L.M * L.K / 2 + L.N * L.K / 2 + 4 * (L.M + L.N) + 8 * L.M * L.N
+                       for L in layers)
+            t_tensor = flops / (fp4_peak * 1e12)
+            t_hbm = byts / (peaks["hbm_gbs"] * 1e9)
+            if t_tensor >= t_hbm:
+                bound, unit, peak, algo = "tensor", "TFLOP/s", fp4_peak, flops / 1e12
+            else:
+                bound, unit, peak, algo = "hbm", "GB/s", peaks["hbm_gbs"], byts / 1e9
+            loop = _mma_loop_peak()
+            extra = {"tflops": round(flops / t / 1e12, 1) if t > 0 else 0.0,
+                     "frac_of_9pf_datasheet": round(flops / t / 9e15, 4) if t > 0 else 0.0,
+                     "frac_of_mma_loop": (round(flops / t / 1e12 / loop, 4)
+                                          if t > 0 and loop else None),
+                     "ceilings_ms": {"tensor": round(1e3 * t_tensor, 4), "hbm": round(1e3 * t_hbm, 4)}}
+        elif k == "spmm":
+            # 2 nnz N fp32 FMA flops; every entry gathers its W row segment
+            # (nnz N elements) from L2, and C is written (4 M N bytes)
+            algo = sum(2 * int(L.csr.nnz.item()) * L.N for L in layers) / 1e12
+            bound, unit, peak = "alu", "TFLOP/s", alu_peak
+            extra = {"w_row_gather_bytes": sum(int(L.csr.nnz.item()) * L.N * L.W.element_size()
+                                               for L in layers)}
+        elif k == "fp4_gemm_compensated":
             # three ceilings: the FP4 MMAs on the tensor cores (2 M N K), the
             # compensation's fp32 FMAs on the CUDA cores (2 nnz N), and the
             # HBM bytes (codes, scales, the CSR, W read once, Y written); the
@@ -894,6 +924,61 @@ def mx_sweep(device, workload, reps=20, warm=5):
         torch.cuda.empty_cache()
 
 
+def compensated_sweep(device, workload, alpha=None, reps=10, warm=3):
+    """The compensated GEMM (dA . W computed inside the GEMM kernel) beside the
+    two-kernel form the layer uses for fp32 Y (the SpMM writing the
+    compensation into Y, then the GEMM adding the product in place), on every
+    linear of a workload; median of `reps` CUDA-event timings, L2 flushed
+    before each.  One JSON line per linear."""
+    import quantize_gemm_b200 as qg
+    from workloads import WORKLOADS, make_layer_inputs
+    wl = WORKLOADS[workload]
+    alpha = wl.alphas[0] if alpha is None else alpha
+    flush = torch.empty(L2_FLUSH_BYTES, dtype=torch.uint8, device=device)
+
+    def timed(fn):
+        for _ in range(warm):
+            fn()
+        ts = []
+        for _ in range(reps):
+            flush.fill_(1)
+            a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            ts.append(a.elapsed_time(b))
+        ts.sort()
+        return ts[len(ts) // 2]
+
+    for li, layer in enumerate(wl.layers):
+        A, W = make_layer_inputs(wl, li, device=device)
+        M, K = A.shape
+        N = W.shape[1]
+        codes, s, csr, _ = qg.quantize_act(A, alpha)
+        codesT, t = qg.quantize_cols(W)
+        Y = torch.empty((M, N), dtype=torch.float32, device=device)
+        ws_c = qg.Workspace(qg.QG_OP_FP4_GEMM_COMPENSATED, M, K, N, qg.QG_F32, device=device)
+        ws_s = qg.Workspace(qg.QG_OP_SPMM, M, K, N, qg._dt(W), device=device)
+        ws_g = qg.Workspace(qg.QG_OP_FP4_GEMM, M, K, N, qg.QG_F32, device=device)
+        t_comp = timed(lambda: qg.qg_fp4_gemm_compensated(codes, s, codesT, t, M, N, K, csr, W, Y,
+                                                          ws_c))
+        t_spmm = timed(lambda: qg.qg_spmm_correction(csr, M, W, Y, ws_s))
+        t_gemm = timed(lambda: qg.qg_fp4_gemm(codes, s, codesT, t, M, N, K, Y, Y, None, ws_g))
+        for ws in (ws_c, ws_s, ws_g):
+            qg.check_status(ws, "compensated sweep")
+        nnz = int(csr.nnz.item())
+        print(json.dumps({"sweep": "compensated", "workload": wl.name, "layer": layer.name,
+                          "M": M, "K": K, "N": N, "alpha": alpha, "nnz": nnz,
+                          "compensated_gemm_ms": round(t_comp, 4),
+                          "spmm_ms": round(t_spmm, 4), "gemm_in_place_ms": round(t_gemm, 4),
+                          "two_kernel_ms": round(t_spmm + t_gemm, 4),
+                          "compensation_tflops_fused": round(2 * nnz * N / (t_comp * 1e-3) / 1e12, 2),
+                          "l2": "flushed before each rep", "reps": reps}), flush=True)
+        del A, W, codes, codesT, Y, ws_c, ws_s, ws_g
+        torch.cuda.empty_cache()
+
+
 def fp4_peak_sweep(device, reps=10, warm=3, iters=1 << 16):
     """The tensor pipe's E2M1 rate from the library's MMA-only loop
     (qg_fp4_mma_loop: operands in shared memory, the GEMM's MMA shape, no
@@ -965,6 +1050,10 @@ def main():
     ap.add_argument("--fp4-peak", action="store_true",
                     help="time the library's MMA-only tensor-pipe loop (E2M1 rate of the tensor "
                          "cores, solo and 2-SM pairs) instead of the layer stream")
+    ap.add_argument("--compensated", action="store_true",
+                    help="time the compensated GEMM (dA . W inside the GEMM kernel) beside the "
+                         "SpMM + in-place GEMM pair on each linear of --workload (one JSON line "
+                         "per linear) instead of the layer stream")
     ap.add_argument("--grads", action="store_true",
                     help="time forward, dgrad and wgrad of each linear of --workload (one JSON "
                          "line per linear) instead of the layer stream")
@@ -992,10 +1081,12 @@ def main():
     import __graft_entry__
     if rank == 0:
         __graft_entry__.build()
-    if args.quantizer_sweep or args.grads or args.mx or args.fp4_peak:
+    if args.quantizer_sweep or args.grads or args.mx or args.fp4_peak or args.compensated:
         if rank == 0:
             if args.quantizer_sweep:
                 quantizer_sweep(device)
+            elif args.compensated:
+                compensated_sweep(device, args.workload, args.alpha)
             elif args.fp4_peak:
                 fp4_peak_sweep(device)
             elif args.mx:

@@ -205,7 +205,9 @@ qg_status qg_spmm_correction(const qg_csr* dA, int64_t M, const void* W, qg_dtyp
  * e2m1(codesWT_jk) accumulated in fp32 (exact for K <= 16384), then
  * Y_ij = acc_ij * sA_i * sW_j (+ C_ij when C != NULL), stored as fp32 or bf16
  * (round to nearest even).  raw_acc (nullable, M x N fp32) receives acc itself.
- * Y may be NULL when only raw_acc is wanted. */
+ * Y may be NULL when only raw_acc is wanted.  C may be the same memory as an
+ * fp32 Y (Y += the scaled product, in place): every element of C is read
+ * before the same element of Y is written. */
 qg_status qg_fp4_gemm(const uint8_t* codesA, const float* sA, const uint8_t* codesWT,
                       const float* sW, int64_t M, int64_t N, int64_t K, const float* C,
                       void* Y, qg_dtype y_dtype, float* raw_acc, void* ws, size_t ws_bytes,
@@ -233,14 +235,20 @@ qg_status qg_fp4_gemm_compensated(const uint8_t* codesA, const float* sA, const 
                                   void* Y, qg_dtype y_dtype, void* ws, size_t ws_bytes,
                                   cudaStream_t stream);
 
-/* The whole layer: qg_quantize_act(A) -> qg_fp4_gemm_compensated(codes, dA,
- * W) into Y (M x N, fp32 or bf16).  codesWT / sW come from
- * qg_quantize_cols(W); W is the unquantized weight used by the compensation,
- * K x N row-major and contiguous, stored in the SAME dtype as A (`dtype`
- * describes both; the call has no separate weight dtype, so a weight in the
- * other dtype is read wrongly without an error).  The activation codes, dA
- * and the GEMM's scratch slots live in the workspace
- * (qg_workspace_size(QG_OP_FP4_LINEAR, ...)); no M x N intermediate exists. */
+/* The whole layer into Y (M x N, fp32 or bf16): qg_quantize_act(A), then
+ *   fp32 Y: qg_spmm_correction(dA, W) written into Y itself, then
+ *           qg_fp4_gemm(..., C = Y, Y) adding the scaled FP4 product to it in
+ *           place (the epilogue reads every sub-tile of C before it writes
+ *           that sub-tile of Y);
+ *   bf16 Y: qg_fp4_gemm_compensated (the compensation inside the GEMM).
+ * Both give Y_ij = fp32(acc_ij * sA_i * sW_j) + C_ij with C the fp32 FMA chain
+ * of row i's entries (rounded to bf16 last for bf16 Y).  codesWT / sW come
+ * from qg_quantize_cols(W); W is the unquantized weight used by the
+ * compensation, K x N row-major and contiguous, stored in the SAME dtype as A
+ * (`dtype` describes both; the call has no separate weight dtype, so a weight
+ * in the other dtype is read wrongly without an error).  The activation
+ * codes, dA and the compensated GEMM's scratch slots live in the workspace
+ * (qg_workspace_size(QG_OP_FP4_LINEAR, ...)); no M x N buffer besides Y. */
 qg_status qg_fp4_linear(const void* A, qg_dtype dtype, int64_t M, int64_t K,
                         const uint8_t* codesWT, const float* sW, const void* W, int64_t N,
                         double alpha, void* Y, qg_dtype y_dtype, void* ws, size_t ws_bytes,

@@ -316,12 +316,26 @@ qg_status qg_fp4_linear(const void* A, qg_dtype dtype, int64_t M, int64_t K,
     uint8_t* codes = at<uint8_t>(ws, L.act_codes);
     float* scales = at<float>(ws, L.act_scales);
     const int64_t rank = qg_quantile_rank(alpha, M * K);
+    uint32_t* status = at<uint32_t>(ws, L.status);
     cudaError_t e = run_quantize_act(A, dtype, M, K, K, rank, act_buffers(ws, L), codes, scales, &csr,
                                      at<float>(ws, L.thr), stream);
     if (e != cudaSuccess) return QG_ERR_CUDA;
+    if (y_dtype == QG_F32) {
+        // fp32 Y: the compensation dA . W is written into Y's own memory, and
+        // the GEMM's epilogue adds the scaled FP4 product to it in place (it
+        // reads each 32 x 32 sub-tile before it overwrites it; sub-tiles are
+        // disjoint), so no M x N buffer is needed besides Y
+        launch_spmm(&csr, M, W, dtype, N, N, static_cast<float*>(Y), status, stream);
+        if ((e = cudaGetLastError()) != cudaSuccess) return QG_ERR_CUDA;
+        return cuda_status(launch_fp4_gemm(codes, scales, codesWT, sW, M, N, K,
+                                           static_cast<const float*>(Y), Y, QG_F32, nullptr,
+                                           status, stream));
+    }
+    // bf16 Y has no room for the fp32 compensation: the compensated GEMM
+    // computes it inside the kernel instead
     return cuda_status(launch_fp4_gemm_corr(codes, scales, codesWT, sW, M, N, K, &csr, W, dtype, N,
-                                            at<float>(ws, L.corr_scratch), Y, y_dtype,
-                                            at<uint32_t>(ws, L.status), stream));
+                                            at<float>(ws, L.corr_scratch), Y, y_dtype, status,
+                                            stream));
 }
 
 qg_status qg_fp4_gemm_compensated(const uint8_t* codesA, const float* sA, const uint8_t* codesWT,

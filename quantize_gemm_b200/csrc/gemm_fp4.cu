@@ -115,11 +115,26 @@ constexpr int kEpiBufs = QG_GEMM_EPI_BUFS;   // sub-tile buffers per epilogue wa
 constexpr long long kWaitLimit = 2000000000LL;  // SM clocks (~1-2 s)
 constexpr int kStageABytes = BM * BK_BYTES;
 
-template <int BN, bool PAIR, bool MX = false>
+#ifndef QG_CORR_D
+#define QG_CORR_D 4              // W-row entries in flight per quarter-warp (bf16 W, fused path)
+#endif
+// Shared-memory ring of one correction warp: QG_CORR_D steps x 4 quarters x
+// 448 bytes (a 224-column bf16 W row segment per quarter).
+constexpr int kCorrRingBytes = QG_CORR_D * 4 * 448;
+
+// Shared-memory plan.  With the fused correction (CORR) the operand ring is
+// one stage shorter (pairs) or two (single CTAs) and the pair's epilogue has
+// three sub-tile buffers per warp, which frees room for the correction
+// warps' W-row rings.
+template <int BN, bool PAIR, bool MX = false, bool CORR = false>
 struct Cfg {
     static_assert(BN % 32 == 0 && BN <= 224, "two accumulators + scales must fit in TMEM");
     static_assert(!MX || (!PAIR && BN == 128), "MX tiles: one CTA, 128 x 128");
-    static constexpr int kStages = MX ? QG_GEMM_MX_STAGES : PAIR ? QG_GEMM_PAIR_STAGES : QG_GEMM_SOLO_STAGES;
+    static constexpr int kStages = MX ? QG_GEMM_MX_STAGES
+                                      : CORR ? (PAIR ? QG_GEMM_PAIR_STAGES - 1 : QG_GEMM_SOLO_STAGES - 1)
+                                             : (PAIR ? QG_GEMM_PAIR_STAGES : QG_GEMM_SOLO_STAGES);
+    static constexpr int kEpiB = (CORR && PAIR) ? 3 : kEpiBufs;   // sub-tile buffers per epilogue warp
+    static_assert(kEpiB >= 2 && kStages >= 2, "double buffering at least");
     static_assert(!MX || kMxSfCol + 16 * kStages <= kSfaCol, "MX scale slots below the constant scales");
     static constexpr int kBRows = PAIR ? BN / 2 : BN;   // rows of W^T loaded by one CTA
     static constexpr int kStageBBytes = kBRows * BK_BYTES;
@@ -129,17 +144,18 @@ struct Cfg {
     static constexpr size_t kOffB = (size_t)kStages * kStageABytes;
     static constexpr size_t kOffSf = kOffB + (size_t)kStages * kStageBBytes;
     static constexpr size_t kOffEpi = kOffSf + (size_t)kStages * kStageSfBytes;
-    static constexpr size_t kOffSw = kOffEpi + (size_t)kEpiWarps * kEpiBufs * kEpiBuf;
-    static constexpr size_t kOffBar = kOffSw + (size_t)kEpiWarps * ((BN / 32 + kEpiSplit - 1) / kEpiSplit) * 32 * 4;
+    static constexpr size_t kOffSw = kOffEpi + (size_t)kEpiWarps * kEpiB * kEpiBuf;
+    static constexpr size_t kOffRing = kOffSw + (size_t)kEpiWarps * ((BN / 32 + kEpiSplit - 1) / kEpiSplit) * 32 * 4;
+    static constexpr size_t kOffBar = kOffRing + (CORR ? (size_t)kCorrWarps * kCorrRingBytes : 0);
 };
 
-template <int S>
+template <int S, int EB>
 struct alignas(8) Barriers {
     uint64_t full[S];
     uint64_t empty[S];
     uint64_t acc_full[kAccStages];
     uint64_t acc_empty[kAccStages];
-    uint64_t cbar[kEpiWarps][kEpiBufs];
+    uint64_t cbar[kEpiWarps][EB];
     uint64_t corr_full[kCorrSlots];    // a tile's correction rows are in its scratch slot
     uint64_t corr_empty[kCorrSlots];   // the epilogue has loaded them: the slot is free
     uint64_t mma_done;
@@ -147,12 +163,15 @@ struct alignas(8) Barriers {
     int abort;
 };
 
-template <int BN, bool PAIR, bool MX = false>
+template <int BN, bool PAIR, bool MX = false, bool CORR = false>
 constexpr size_t smem_bytes() {
-    return 1024 + Cfg<BN, PAIR, MX>::kOffBar + sizeof(Barriers<Cfg<BN, PAIR, MX>::kStages>);
+    using CF = Cfg<BN, PAIR, MX, CORR>;
+    return 1024 + CF::kOffBar + sizeof(Barriers<CF::kStages, CF::kEpiB>);
 }
 static_assert(smem_bytes<224, true>() <= 232448 && smem_bytes<224, false>() <= 232448 &&
-                  smem_bytes<128, false, true>() <= 232448,
+                  smem_bytes<128, false, true>() <= 232448 &&
+                  smem_bytes<224, true, false, true>() <= 232448 &&
+                  smem_bytes<224, false, false, true>() <= 232448,
               "pipeline stages and epilogue buffers must fit in 227 KB of shared memory");
 
 // ------------------------------------------------------------------ PTX wraps
@@ -455,23 +474,47 @@ __device__ __forceinline__ void fma2_f32(uint64_t& acc, uint64_t vv, uint32_t a,
         : "l"(vv), "r"(a), "r"(b));
 }
 
+#ifndef QG_CORR_LDG
+#define QG_CORR_LDG 0
+#endif
+// A 16-byte W segment load (read-only data)
+__device__ __forceinline__ uint4 ld_w16(const void* p) {
+#if QG_CORR_LDG == 1
+    uint4 v;
+    asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p));
+    return v;
+#elif QG_CORR_LDG == 2
+    return __ldcg(reinterpret_cast<const uint4*>(p));
+#else
+    return __ldg(reinterpret_cast<const uint4*>(p));
+#endif
+}
+
 // The compensation rows r_begin .. r_end - 1 (at most 31 rows) of dA . W,
 // 8 columns per lane starting at c0: for each row, the fp32 FMA chain over the
 // row's CSR entries in order, value (fp32 of the stored double) times the W
 // row segment.  The warp's entries form one contiguous CSR range, consumed as
-// a stream with D W-row segments in flight (the ring position is a
-// compile-time index: the loop over entries is unrolled by D); lane l holds
-// entry values and the columns of the entries D ahead, batch by batch of 32.
-// Row r's 8 sums go to dst + (r - r_begin) * dst_ld (lanes with lane_on).
-// vec: the 8 columns are inside W and 16-byte aligned (else element loads,
-// zero past N).
-template <bool WBF16, int D>
+// a stream in groups of G entries; NG groups of W-row segments (16 bytes per
+// lane per entry) are in flight.  A group's G loads are issued together and
+// its G entries consumed together, so a group needs one load scoreboard and
+// the wait for the oldest group never waits for a newer one.  Ring positions
+// are compile-time indices (the loop is unrolled by NG groups).  Lane l holds
+// entry values and the columns of the entries NG * G ahead, batch by batch
+// of 32.  Row r's 8 sums go to dst + (r - r_begin) * dst_ld (lanes with
+// lane_on).  fast: every W row segment the warp reads is 16-byte aligned and
+// inside W for the lanes that are on (the caller checks N and ldw); lanes
+// that are off then read the warp's first segment (column c_safe) instead,
+// so the loads are not divergent.  Otherwise element loads, zero past N.
+template <bool WBF16, int NG, int G>
 __device__ __forceinline__ void corr_rows(const int32_t* __restrict__ row_ptr,
                                           const int32_t* __restrict__ col,
                                           const double* __restrict__ val,
                                           const void* __restrict__ W, int64_t ldw, int r_begin,
-                                          int r_end, int N, int c0, bool lane_on, bool vec,
-                                          float* __restrict__ dst, int dst_ld) {
+                                          int r_end, int N, int c0, int c_safe, bool lane_on,
+                                          bool fast, float* __restrict__ dst, int dst_ld) {
+    constexpr int D = NG * G;                   // entries in flight
     static_assert(32 % D == 0, "entry batches of 32 hold whole ring turns");
     constexpr int SEG = WBF16 ? 1 : 2;          // 16-byte words per lane per W row segment
     const int lane = threadIdx.x & 31;
@@ -488,39 +531,40 @@ __device__ __forceinline__ void corr_rows(const int32_t* __restrict__ row_ptr,
         const int b = __shfl_sync(0xFFFFFFFFu, kn, (lane + D) & 31);
         ks = (lane + D < 32) ? a : b;
     }
+    const int cl = lane_on ? c0 : c_safe;       // this lane's load column
     auto fetch = [&](uint4 (&d)[SEG], int k) {
-#pragma unroll
-        for (int s = 0; s < SEG; ++s) d[s] = make_uint4(0u, 0u, 0u, 0u);
-        if (!lane_on) return;
         if constexpr (WBF16) {
-            const uint16_t* src = static_cast<const uint16_t*>(W) + (int64_t)k * ldw + c0;
-            if (vec) {
-                d[0] = __ldg(reinterpret_cast<const uint4*>(src));
+            const uint16_t* src = static_cast<const uint16_t*>(W) + (int64_t)k * ldw + cl;
+            if (fast) {
+                d[0] = ld_w16(src);
             } else {
                 uint32_t w[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
                 for (int e = 0; e < 8; ++e)
-                    if (c0 + e < N) w[e >> 1] |= (uint32_t)__ldg(src + e) << (16 * (e & 1));
+                    if (lane_on && c0 + e < N) w[e >> 1] |= (uint32_t)__ldg(src + e) << (16 * (e & 1));
                 d[0] = make_uint4(w[0], w[1], w[2], w[3]);
             }
         } else {
-            const float* src = static_cast<const float*>(W) + (int64_t)k * ldw + c0;
-            if (vec) {
-                d[0] = __ldg(reinterpret_cast<const uint4*>(src));
-                d[1] = __ldg(reinterpret_cast<const uint4*>(src) + 1);
+            const float* src = static_cast<const float*>(W) + (int64_t)k * ldw + cl;
+            if (fast) {
+                d[0] = ld_w16(src);
+                d[1] = ld_w16(src + 4);
             } else {
                 uint32_t w[8];
 #pragma unroll
-                for (int e = 0; e < 8; ++e) w[e] = (c0 + e < N) ? __float_as_uint(__ldg(src + e)) : 0u;
+                for (int e = 0; e < 8; ++e)
+                    w[e] = (lane_on && c0 + e < N) ? __float_as_uint(__ldg(src + e)) : 0u;
                 d[0] = make_uint4(w[0], w[1], w[2], w[3]);
                 d[1] = make_uint4(w[4], w[5], w[6], w[7]);
             }
         }
     };
-    uint4 buf[D][SEG];
+    uint4 buf[NG][G][SEG];
 #pragma unroll
-    for (int u = 0; u < D; ++u)
-        if (u < n) fetch(buf[u], __shfl_sync(0xFFFFFFFFu, kc, u));
+    for (int g = 0; g < NG; ++g)
+#pragma unroll
+        for (int i = 0; i < G; ++i)
+            if (g * G + i < n) fetch(buf[g][i], __shfl_sync(0xFFFFFFFFu, kc, g * G + i));
     uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
     int row = r_begin;
     int rend = __shfl_sync(0xFFFFFFFFu, rp, 1) - P0;   // entries of rows <= row end here
@@ -535,31 +579,38 @@ __device__ __forceinline__ void corr_rows(const int32_t* __restrict__ row_ptr,
     };
     for (int q = 0; q < n; q += D) {
 #pragma unroll
-        for (int u = 0; u < D; ++u) {
-            const int j = q + u;                 // entry index within the warp's range
-            if (j >= n) break;
-            while (j >= rend) {                  // rows that end before entry j
-                store_row(row);
-                ++row;
-                rend = __shfl_sync(0xFFFFFFFFu, rp, row - r_begin + 1) - P0;
+        for (int g = 0; g < NG; ++g) {
+#pragma unroll
+            for (int i = 0; i < G; ++i) {           // consume group g
+                const int j = q + g * G + i;         // entry index within the warp's range
+                if (j < n) {
+                    while (j >= rend) {              // rows that end before entry j
+                        store_row(row);
+                        ++row;
+                        rend = __shfl_sync(0xFFFFFFFFu, rp, row - r_begin + 1) - P0;
+                    }
+                    const float v = __shfl_sync(0xFFFFFFFFu, vc, (q & 31) + g * G + i);
+                    uint64_t vv;
+                    asm("mov.b64 %0, {%1, %1};" : "=l"(vv) : "f"(v));
+                    if constexpr (WBF16) {
+                        fma2_bf16(acc[0], vv, buf[g][i][0].x);
+                        fma2_bf16(acc[1], vv, buf[g][i][0].y);
+                        fma2_bf16(acc[2], vv, buf[g][i][0].z);
+                        fma2_bf16(acc[3], vv, buf[g][i][0].w);
+                    } else {
+                        fma2_f32(acc[0], vv, buf[g][i][0].x, buf[g][i][0].y);
+                        fma2_f32(acc[1], vv, buf[g][i][0].z, buf[g][i][0].w);
+                        fma2_f32(acc[2], vv, buf[g][i][SEG - 1].x, buf[g][i][SEG - 1].y);
+                        fma2_f32(acc[3], vv, buf[g][i][SEG - 1].z, buf[g][i][SEG - 1].w);
+                    }
+                }
             }
-            const int t = (q & 31) + u;          // position in the batch
-            const float v = __shfl_sync(0xFFFFFFFFu, vc, t);
-            const int kf = __shfl_sync(0xFFFFFFFFu, ks, t);
-            uint64_t vv;
-            asm("mov.b64 %0, {%1, %1};" : "=l"(vv) : "f"(v));
-            if constexpr (WBF16) {
-                fma2_bf16(acc[0], vv, buf[u][0].x);
-                fma2_bf16(acc[1], vv, buf[u][0].y);
-                fma2_bf16(acc[2], vv, buf[u][0].z);
-                fma2_bf16(acc[3], vv, buf[u][0].w);
-            } else {
-                fma2_f32(acc[0], vv, buf[u][0].x, buf[u][0].y);
-                fma2_f32(acc[1], vv, buf[u][0].z, buf[u][0].w);
-                fma2_f32(acc[2], vv, buf[u][SEG - 1].x, buf[u][SEG - 1].y);
-                fma2_f32(acc[3], vv, buf[u][SEG - 1].z, buf[u][SEG - 1].w);
+#pragma unroll
+            for (int i = 0; i < G; ++i) {           // refill group g, entries D ahead
+                const int j = q + g * G + i;
+                const int kf = __shfl_sync(0xFFFFFFFFu, ks, (q & 31) + g * G + i);
+                if (j + D < n) fetch(buf[g][i], kf);
             }
-            if (j + D < n) fetch(buf[u], kf);    // refill this ring position
         }
         if ((q & 31) == 32 - D) {                // batch done: load the next one
             const int Bn = q + D;
@@ -572,6 +623,142 @@ __device__ __forceinline__ void corr_rows(const int32_t* __restrict__ row_ptr,
         }
     }
     while (row < r_end) {                        // the last rows (and empty ones)
+        store_row(row);
+        ++row;
+    }
+}
+
+// The compensation rows of a warp for a tile of 224 (or 192) bf16 columns,
+// four row blocks at a time.  Quarter-warp qd (lanes 8 qd .. 8 qd + 7) walks
+// the contiguous CSR range of its rows [rq0, rq1) (at most 7 rows); lane
+// lq < 7 of a quarter owns the four 8-column groups lq, lq + 7, lq + 14,
+// lq + 21 of the tile, so each of a quarter's four 16-byte copies covers 112
+// contiguous bytes of the W row and a lane sums 32 columns per entry.  The W
+// segments in flight live in shared memory, not registers: every lane copies
+// its chunks of an entry with cp.async (L2 -> shared memory), one commit
+// group per ring step, D steps ahead, and waits with cp.async.wait_group for
+// the oldest step before reading it back; each lane reads only what it
+// copied, so no other synchronisation is needed.  Entry values and columns
+// are held by the quarter's lanes, batch by batch of 8, and broadcast with
+// 8-lane shuffles.  Each row is an fp32 FMA chain over its entries in CSR
+// order; its sums go to dst + (r - r_base) * dst_ld at the lane's columns.
+// ring: this warp's D x 4 x 448 bytes of shared memory.  The loop runs until
+// the warp's longest quarter is done; the other quarters idle meanwhile.
+template <int D>
+__device__ __forceinline__ void corr_rows4s(const int32_t* __restrict__ row_ptr,
+                                            const int32_t* __restrict__ col,
+                                            const double* __restrict__ val,
+                                            const uint16_t* __restrict__ W, int64_t ldw, int rq0,
+                                            int rq1, int n0, int N, int r_base,
+                                            float* __restrict__ dst, int dst_ld, int BNr,
+                                            uint8_t* ring) {
+    static_assert(8 % D == 0, "entry batches of 8 hold whole ring turns");
+    const int lane = threadIdx.x & 31;
+    const int lq = lane & 7, qd = lane >> 3;
+    const unsigned FULL = 0xFFFFFFFFu;
+    const int nrows = rq1 - rq0;
+    const int rp = (lq <= nrows) ? __ldg(row_ptr + rq0 + lq) : 0;
+    const int P0 = __shfl_sync(FULL, rp, 0, 8);
+    const int n = __shfl_sync(FULL, rp, nrows, 8) - P0;
+    int nmax = n;
+#pragma unroll
+    for (int d = 8; d < 32; d <<= 1) nmax = max(nmax, __shfl_xor_sync(FULL, nmax, d));
+    bool on[4];
+    int cg[4];
+#pragma unroll
+    for (int h = 0; h < 4; ++h) {
+        cg[h] = 8 * (lq + 7 * h);
+        on[h] = lq < 7 && cg[h] < BNr && n0 + cg[h] < N;
+        if (!on[h]) cg[h] = 0;
+    }
+    int kc = (lq < n) ? __ldg(col + P0 + lq) : 0;
+    float vc = (lq < n) ? (float)__ldg(val + P0 + lq) : 0.0f;
+    int ks;
+    {
+        const int kn = (8 + lq < n) ? __ldg(col + P0 + 8 + lq) : 0;
+        const int a = __shfl_sync(FULL, kc, (lq + D) & 7, 8);
+        const int b = __shfl_sync(FULL, kn, (lq + D) & 7, 8);
+        ks = (lq + D < 8) ? a : b;
+    }
+    const uint16_t* wl = W + n0;
+    // slot u of this lane: 4 chunks, lane-private, conflict-free per quarter
+    // (lane 7 of a quarter owns no columns: it mirrors lane 6's slots, which
+    // keeps its reads inside the quarter's region; it never copies or stores)
+    const uint32_t sbase = (uint32_t)__cvta_generic_to_shared(ring) + (uint32_t)(qd * 448 + min(lq, 6) * 16);
+    auto slot_addr = [&](int u, int h) { return sbase + (uint32_t)(u * 4 * 448 + h * 112); };
+    auto fetch = [&](int u, int k, bool valid) {
+        const uint16_t* src = wl + (int64_t)k * ldw;
+#pragma unroll
+        for (int h = 0; h < 4; ++h)
+            if (valid && on[h])
+                asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(slot_addr(u, h)),
+                             "l"(src + cg[h])
+                             : "memory");
+        asm volatile("cp.async.commit_group;" ::: "memory");
+    };
+#pragma unroll
+    for (int u = 0; u < D; ++u) fetch(u, __shfl_sync(FULL, kc, u, 8), u < n);
+    uint64_t acc[16];
+#pragma unroll
+    for (int e = 0; e < 16; ++e) acc[e] = 0ull;
+    int row = rq0;
+    int rend = __shfl_sync(FULL, rp, 1, 8) - P0;
+    auto store_row = [&](int r) {
+        float* d = dst + (int64_t)(r - r_base) * dst_ld;
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+            if (on[h]) {
+                ulonglong2* p = reinterpret_cast<ulonglong2*>(d + cg[h]);
+                p[0] = make_ulonglong2(acc[4 * h + 0], acc[4 * h + 1]);
+                p[1] = make_ulonglong2(acc[4 * h + 2], acc[4 * h + 3]);
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < 16; ++e) acc[e] = 0ull;
+    };
+    for (int q = 0; q < nmax; q += D) {
+#pragma unroll
+        for (int u = 0; u < D; ++u) {
+            const int j = q + u;
+            const int t = (q & 7) + u;
+            const float v = __shfl_sync(FULL, vc, t, 8);
+            const int kf = __shfl_sync(FULL, ks, t, 8);
+            // the oldest of the D groups in flight is slot u's
+            asm volatile("cp.async.wait_group %0;" ::"n"(D - 1) : "memory");
+            if (j < n) {
+                while (j >= rend) {
+                    store_row(row);
+                    ++row;
+                    rend = __shfl_sync(__activemask(), rp, row - rq0 + 1, 8) - P0;
+                }
+                uint64_t vv;
+                asm("mov.b64 %0, {%1, %1};" : "=l"(vv) : "f"(v));
+#pragma unroll
+                for (int h = 0; h < 4; ++h) {
+                    uint4 w;
+                    asm volatile("ld.shared.v4.u32 {%0, %1, %2, %3}, [%4];"
+                                 : "=r"(w.x), "=r"(w.y), "=r"(w.z), "=r"(w.w)
+                                 : "r"(slot_addr(u, h)));
+                    fma2_bf16(acc[4 * h + 0], vv, w.x);
+                    fma2_bf16(acc[4 * h + 1], vv, w.y);
+                    fma2_bf16(acc[4 * h + 2], vv, w.z);
+                    fma2_bf16(acc[4 * h + 3], vv, w.w);
+                }
+            }
+            fetch(u, kf, j + D < n);             // refill slot u (an empty group if none)
+        }
+        if ((q & 7) == 8 - D) {
+            const int Bn = q + D;
+            kc = (Bn + lq < n) ? __ldg(col + P0 + Bn + lq) : 0;
+            vc = (Bn + lq < n) ? (float)__ldg(val + P0 + Bn + lq) : 0.0f;
+            const int kn = (Bn + 8 + lq < n) ? __ldg(col + P0 + Bn + 8 + lq) : 0;
+            const int a = __shfl_sync(FULL, kc, (lq + D) & 7, 8);
+            const int b = __shfl_sync(FULL, kn, (lq + D) & 7, 8);
+            ks = (lq + D < 8) ? a : b;
+        }
+    }
+    asm volatile("cp.async.wait_group 0;" ::: "memory");
+    while (row < rq1) {
         store_row(row);
         ++row;
     }
@@ -667,8 +854,9 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 const __grid_constant__ CUtensorMap tmap_b,
                 const __grid_constant__ CUtensorMap tmap_y,
                 const __grid_constant__ CUtensorMap tmap_c, const Params p) {
-    using CF = Cfg<BN, PAIR, MX>;
+    using CF = Cfg<BN, PAIR, MX, CORR>;
     constexpr int S = CF::kStages;
+    constexpr int EB = CF::kEpiB;
     static_assert(!(CORR && MX), "the compensated GEMM uses per-row / per-column scales");
     extern __shared__ uint8_t smem_raw[];
     uint8_t* smem = reinterpret_cast<uint8_t*>(
@@ -677,7 +865,7 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
     uint8_t* sb = smem + CF::kOffB;
     uint8_t* ssf = smem + CF::kOffSf;
     uint8_t* sepi = smem + CF::kOffEpi;
-    Barriers<S>* B = reinterpret_cast<Barriers<S>*>(smem + CF::kOffBar);
+    Barriers<S, EB>* B = reinterpret_cast<Barriers<S, EB>*>(smem + CF::kOffBar);
 
     const int warp = threadIdx.x >> 5;
     const int lane = threadIdx.x & 31;
@@ -700,7 +888,7 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             mbar_init(&B->acc_empty[s], (PAIR ? 2 : 1) * kEpiWarps);
         }
         for (int w = 0; w < kEpiWarps; ++w)
-            for (int b = 0; b < kEpiBufs; ++b) mbar_init(&B->cbar[w][b], 1);
+            for (int b = 0; b < EB; ++b) mbar_init(&B->cbar[w][b], 1);
         for (int s = 0; s < kCorrSlots; ++s) {
             mbar_init(&B->corr_full[s], kCorrWarps);
             mbar_init(&B->corr_empty[s], kEpiWarps);
@@ -851,8 +1039,8 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         // Two warps per TMEM lane quarter when kEpiSplit == 2: warp ew takes
         // the chunks c with c % kEpiSplit == ew / 4.  Each warp walks its
         // chunks of all its tiles as one stream: chunk g uses sub-tile buffer
-        // g % kEpiBufs; with a correction C, the C sub-tile of chunk
-        // g + kEpiBufs - 1 is requested once chunk g is stored.  The next
+        // g % EB; with a correction C, the C sub-tile of chunk
+        // g + EB - 1 is requested once chunk g is stored.  The next
         // tile's row and column scales are loaded while this tile is drained.
         constexpr int NC = BN / 32;
         constexpr int SWR = (NC + kEpiSplit - 1) / kEpiSplit;   // this warp's chunks per tile, at most
@@ -861,7 +1049,7 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         const int par = ew / 4;                // chunk residue class of this warp
         const int my_nc = (NC - par + kEpiSplit - 1) / kEpiSplit;   // its chunks per tile
         const uint32_t lane_base = (uint32_t)(32 * q) << 16;
-        uint8_t* bufs = sepi + (size_t)ew * kEpiBufs * kEpiBuf;
+        uint8_t* bufs = sepi + (size_t)ew * EB * kEpiBuf;
         float* sw = reinterpret_cast<float*>(smem + CF::kOffSw) + ew * SWR * 32;
         const bool use_c = TMA_EPI && (CORR || p.C != nullptr);
         const int my_tiles = unit < num_tiles ? (num_tiles - unit + n_units - 1) / n_units : 0;
@@ -875,7 +1063,7 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             const int ti = g / my_nc, c = par + kEpiSplit * (g - ti * my_nc);
             const int tile = unit + ti * n_units;
             const int mb = tile % num_m, nbk = tile / num_m;
-            const int b = g % kEpiBufs;
+            const int b = g % EB;
             int x = nbk * BN + c * 32, y = mb * CF::kTileRows + (int)rank * BM + 32 * q;
             if constexpr (CORR) {
                 if (g == ti * my_nc &&
@@ -894,7 +1082,7 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         };
         bool ok = true;
         if (use_c)
-            for (int g = 0; ok && g < kEpiBufs - 1 && g < total; ++g) ok = c_load(g);
+            for (int g = 0; ok && g < EB - 1 && g < total; ++g) ok = c_load(g);
         // scales of tile ti into registers (consumed one tile later)
         float swr[SWR];
         float srow_next = 0.0f;
@@ -971,7 +1159,7 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     return true;
                 }
                 const int g = ti * my_nc + h;
-                const int b = g % kEpiBufs;
+                const int b = g % EB;
                 uint8_t* buf = bufs + b * kEpiBuf;
                 // y overwrites the accumulator registers (as fp32 bit patterns)
                 const float4* tw = reinterpret_cast<const float4*>(sw + h * 32);
@@ -1003,8 +1191,8 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                         mbar_arrive(&B->corr_empty[ti & 1]);
                     }
                 } else {
-                    // buffer b was last read by the store of chunk g - kEpiBufs
-                    if (lane == 0) bulk_wait_read<kEpiBufs - 1>();
+                    // buffer b was last read by the store of chunk g - EB
+                    if (lane == 0) bulk_wait_read<EB - 1>();
                 }
                 __syncwarp();   // every lane has read its C row before the buffer is overwritten
                 if (p.y_bf16) {
@@ -1031,10 +1219,10 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                     tma_store_2d(&tmap_y, buf, col0, row0);
                     bulk_commit();
                 }
-                if (use_c && g + kEpiBufs - 1 < total) {
+                if (use_c && g + EB - 1 < total) {
                     // that buffer was last read by the store of chunk g - 1
                     if (lane == 0) bulk_wait_read<1>();
-                    if (!c_load(g + kEpiBufs - 1)) return false;
+                    if (!c_load(g + EB - 1)) return false;
                 }
                 return true;
             };
@@ -1064,7 +1252,7 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         if (TMA_EPI && lane == 0) {
             bulk_wait_all();
             // on abort, C loads still in flight land before the CTA exits
-            for (int b = 0; b < kEpiBufs; ++b)
+            for (int b = 0; b < EB; ++b)
                 if ((cpend >> b) & 1u) mbar_drain(&B->cbar[ew][b], (cphase >> b) & 1u);
         }
         __syncwarp();
@@ -1089,15 +1277,26 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             float* dst = p.corr + ((size_t)((int)blockIdx.x * kCorrSlots + slot) * BM + r_lo) * BN +
                          lane * 8;
             const bool on = lane_on && c0 < p.N;
-            if (rb < re) {
+            const int c_safe = n_blk * BN;           // inside W: the tile exists
+            if (p.w_bf16 && (p.N % 8) == 0 && (p.ldw % 8) == 0) {
+                // bf16 W with whole, aligned 8-column groups: the quarter-warp
+                // loop with its shared-memory ring (every lane of the warp
+                // takes part, also when its quarter has no rows)
+                const int span = r_hi - r_lo, qd = lane >> 3;
+                const int q_lo = r_lo + (qd * span) / 4, q_hi = r_lo + ((qd + 1) * span) / 4;
+                corr_rows4s<QG_CORR_D>(p.row_ptr, p.col, p.val, static_cast<const uint16_t*>(p.Wc),
+                                       p.ldw, min(p.M, row0 + q_lo), min(p.M, row0 + q_hi),
+                                       n_blk * BN, p.N, row0,
+                                       p.corr + (size_t)((int)blockIdx.x * kCorrSlots + slot) * BM * BN,
+                                       BN, BN, smem + CF::kOffRing + (size_t)cw * kCorrRingBytes);
+            } else if (rb < re) {
                 if (p.w_bf16) {
-                    const bool vec = c0 + 8 <= p.N && (p.ldw % 8) == 0;
-                    corr_rows<true, 16>(p.row_ptr, p.col, p.val, p.Wc, p.ldw, rb, re, p.N, c0, on,
-                                        vec, dst, BN);
+                    corr_rows<true, 2, 4>(p.row_ptr, p.col, p.val, p.Wc, p.ldw, rb, re, p.N, c0,
+                                          c_safe, on, false, dst, BN);
                 } else {
-                    const bool vec = c0 + 8 <= p.N && (p.ldw % 4) == 0;
-                    corr_rows<false, 8>(p.row_ptr, p.col, p.val, p.Wc, p.ldw, rb, re, p.N, c0, on,
-                                        vec, dst, BN);
+                    const bool fast = (p.N % 8) == 0 && (p.ldw % 4) == 0;
+                    corr_rows<false, 2, 2>(p.row_ptr, p.col, p.val, p.Wc, p.ldw, rb, re, p.N, c0,
+                                           c_safe, on, fast, dst, BN);
                 }
             }
             // the rows are written (generic proxy); the epilogue reads them by
@@ -1194,7 +1393,7 @@ static cudaError_t launch_variant(const CUtensorMap& ta, const uint8_t* codesWT,
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3((unsigned)(units * per_unit));
     cfg.blockDim = dim3(threads_of<CORR>());
-    cfg.dynamicSmemBytes = smem_bytes<BN, PAIR, MX>();
+    cfg.dynamicSmemBytes = smem_bytes<BN, PAIR, MX, CORR>();
     cfg.stream = s;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -1213,11 +1412,11 @@ template <int BN, bool PAIR, bool MX = false, bool CORR = false>
 static cudaError_t set_smem_attr() {
     cudaError_t e = cudaFuncSetAttribute(fp4_gemm_kernel<BN, PAIR, true, MX, CORR>,
                                          cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         (int)smem_bytes<BN, PAIR, MX>());
+                                         (int)smem_bytes<BN, PAIR, MX, CORR>());
     if (e != cudaSuccess) return e;
     return cudaFuncSetAttribute(fp4_gemm_kernel<BN, PAIR, false, MX, CORR>,
                                 cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                (int)smem_bytes<BN, PAIR, MX>());
+                                (int)smem_bytes<BN, PAIR, MX, CORR>());
 }
 
 }  // namespace gemm

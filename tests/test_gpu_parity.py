@@ -376,6 +376,24 @@ def test_fp4_gemm_direct_epilogue(qg, M, N, K):
     assert y_rel_err(_np(Y), Yo) <= 1e-3
 
 
+@pytest.mark.parametrize("M,N,K", [(300, 600, 1024), (129, 257, 288), (513, 5504, 2048)])
+def test_fp4_gemm_accumulates_in_place(qg, M, N, K):
+    """C given as Y itself (fp32): Y += the scaled product, bit for bit what a
+    separate C gives (TMA epilogue for N % 4 == 0, direct stores otherwise)."""
+    g = np.random.default_rng(M + 3 * N)
+    cA, cW = _rand_codes(M, K, 41 + M), _rand_codes(N, K, 42 + N)
+    sA = torch.from_numpy((g.random(M) * 0.1 + 1e-3).astype(np.float32)).cuda()
+    sW = torch.from_numpy((g.random(N) * 0.01 + 1e-4).astype(np.float32)).cuda()
+    C = torch.from_numpy((g.standard_normal((M, N)) * 0.5).astype(np.float32)).cuda()
+    cA, cW = torch.from_numpy(cA).cuda(), torch.from_numpy(cW).cuda()
+    want = qg.fp4_gemm(cA, sA, cW, sW, K, C=C)
+    Y = C.clone()
+    ws = qg.Workspace(qg.QG_OP_FP4_GEMM, M, K, N, qg.QG_F32)
+    assert qg.qg_fp4_gemm(cA, sA, cW, sW, M, N, K, Y, Y, None, ws) == qg.QG_OK
+    qg.check_status(ws)
+    assert torch.equal(Y, want)
+
+
 def test_fp4_gemm_epilogue_bf16(qg):
     M, N, K = 300, 600, 1024
     g = np.random.default_rng(2)
