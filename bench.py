@@ -283,12 +283,16 @@ def _measure(qg, layers, steps, flush, world, device, no_graph):
     del graph
     step_ms = [a.elapsed_time(b) for a, b in ev_step]
     per_kernel = {k: [] for k in KERNELS}
+    per_layer = {k: [0.0] * n_l for k in KERNELS}
     for ev in ev_steps:
         for kn in KERNELS:
             j = KERNELS.index(kn)
-            per_kernel[kn].append(sum(ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(n_l)))
-    return dict(step_ms=step_ms, per_kernel=per_kernel, launches=int(launches), clocks=clocks,
-                graph=used_graph, wall=wall)
+            t = [ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(n_l)]
+            per_kernel[kn].append(sum(t))
+            for i in range(n_l):
+                per_layer[kn][i] += t[i] / steps
+    return dict(step_ms=step_ms, per_kernel=per_kernel, per_layer=per_layer,
+                launches=int(launches), clocks=clocks, graph=used_graph, wall=wall)
 
 
 def _mma_loop_peak():
@@ -413,6 +417,8 @@ def our_arm(args, rank, world, device):
         total_ms = max_over_ranks(sum(m["step_ms"]), world, device)
         sm_mhz = m["clocks"].get("sm_mhz") or peaks["sm_max_mhz"]
         rows, fp4_peak = _kernel_rows(layers, m["per_kernel"], args.steps, peaks, sm_mhz, n_sm)
+        for k in rows:
+            rows[k]["ms_per_layer"] = [round(x, 4) for x in m["per_layer"][k]]
         nnz = [int(L.csr.nnz.item()) for L in layers]
         results.append(dict(alpha=a, m=m, total_ms=total_ms, rows=rows, fp4_peak=fp4_peak,
                             sm_mhz=sm_mhz, nnz=nnz))
