@@ -95,3 +95,17 @@ def test_reference_arm_line_and_bounded_sample(monkeypatch, budget):
         assert "fraction" in sample
     else:
         assert "full tensors" in sample
+
+
+def test_cpu_baseline_is_bounded_and_labelled(monkeypatch):
+    """The GPU arm's cpu_baseline times the oracle on a bounded sample: with a
+    tiny budget it falls back to the smallest slices and says so."""
+    import types
+    wl = WORKLOADS["tiny"]
+    A, W = make_layer_inputs("tiny", 0, device="cpu")
+    L = types.SimpleNamespace(A=A, W=W, alpha=0.99, flops=2 * A.shape[0] * A.shape[1] * W.shape[1])
+    monkeypatch.setattr(bench, "CPU_BASELINE_BUDGET_S", 1e-3)
+    out = bench.cpu_baseline(None, wl, [L])
+    assert out["kind"] == "oracle" and out["cores"] >= 1 and out["value"] > 0
+    assert 0 < out["sample_fraction"] < 1 and "fraction" in out["sample"]
+    assert out["sample_wall_s"] < 60
