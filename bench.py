@@ -177,31 +177,51 @@ class Layer:
 KERNELS = ("quantize_cols", "quantize_act", "spmm", "fp4_gemm")
 
 
+def layer_order(qg, L):
+    """The order of the layer's four calls, as qg_fp4_linear runs them for
+    fp32 Y: with many clamped entries per row the GEMM writes Y and the SpMM
+    adds the compensation into it; otherwise the SpMM writes the compensation
+    into Y and the GEMM adds its product in place."""
+    if qg.linear_adds_into_y(L.M, L.K, L.alpha):
+        return ("quantize_cols", "quantize_act", "fp4_gemm", "spmm")
+    return ("quantize_cols", "quantize_act", "spmm", "fp4_gemm")
+
+
 def run_step(qg, layers, ev=None):
     """One pass of the hot path over every layer, the calls qg_fp4_linear
     makes for fp32 Y: the weight quantizer, the fused activation quantizer
-    (threshold, clamp, dA, codes), the compensation dA . W written into Y, and
-    the FP4 GEMM adding the scaled product to Y in place.  With `ev`, record
-    events around each of the four calls of each layer (same stream)."""
+    (threshold, clamp, dA, codes), then the compensation dA . W and the FP4
+    GEMM into Y in the layer's order (layer_order).  With `ev`, record events
+    around each of the four calls of each layer (same stream)."""
     def _chk(st, where):
         if st != qg.QG_OK:
             raise qg.QGError(st, where)
+
+    def call(L, name):
+        if name == "quantize_cols":
+            _chk(qg.qg_quantize_cols(L.W, L.codesT, L.t, L.ws_cols), name)
+        elif name == "quantize_act":
+            _chk(qg.qg_quantize_act(L.A, L.alpha, L.codes, L.s, L.csr, L.T, L.ws_act), name)
+        elif name == "spmm":
+            if L.adds:
+                _chk(qg.qg_spmm_accumulate(L.csr, L.M, L.W, L.Y, L.ws_spmm), name)
+            else:
+                _chk(qg.qg_spmm_correction(L.csr, L.M, L.W, L.Y, L.ws_spmm), name)
+        else:
+            C = None if L.adds else L.Y
+            _chk(qg.qg_fp4_gemm(L.codes, L.s, L.codesT, L.t, L.M, L.N, L.K, C, L.Y, None,
+                                L.ws_gemm), name)
+
     for i, L in enumerate(layers):
+        order = layer_order(qg, L)
+        L.adds = order[2] == "fp4_gemm"
+        L.order = order
         if ev is not None:
             ev[i][0].record()
-        _chk(qg.qg_quantize_cols(L.W, L.codesT, L.t, L.ws_cols), "quantize_cols")
-        if ev is not None:
-            ev[i][1].record()
-        _chk(qg.qg_quantize_act(L.A, L.alpha, L.codes, L.s, L.csr, L.T, L.ws_act), "quantize_act")
-        if ev is not None:
-            ev[i][2].record()
-        _chk(qg.qg_spmm_correction(L.csr, L.M, L.W, L.Y, L.ws_spmm), "spmm")
-        if ev is not None:
-            ev[i][3].record()
-        _chk(qg.qg_fp4_gemm(L.codes, L.s, L.codesT, L.t, L.M, L.N, L.K, L.Y, L.Y, None,
-                            L.ws_gemm), "fp4_gemm")
-        if ev is not None:
-            ev[i][4].record()
+        for j, name in enumerate(order):
+            call(L, name)
+            if ev is not None:
+                ev[i][j + 1].record()
 
 
 def capture_step(qg, layers):
@@ -286,8 +306,10 @@ def _measure(qg, layers, steps, flush, world, device, no_graph):
     per_layer = {k: [0.0] * n_l for k in KERNELS}
     for ev in ev_steps:
         for kn in KERNELS:
-            j = KERNELS.index(kn)
-            t = [ev[i][j].elapsed_time(ev[i][j + 1]) for i in range(n_l)]
+            t = []
+            for i in range(n_l):
+                j = layers[i].order.index(kn)
+                t.append(ev[i][j].elapsed_time(ev[i][j + 1]))
             per_kernel[kn].append(sum(t))
             for i in range(n_l):
                 per_layer[kn][i] += t[i] / steps
@@ -320,8 +342,10 @@ def _kernel_rows(layers, per_kernel, steps, peaks, sm_mhz, n_sm):
             # (read from Y) and Y (fp32, written in place); its bound is
             # whichever of the tensor-core time and the HBM time is longer
             flops = sum(L.flops for L in layers)
-            byts = sum(L.M * L.K / 2 + L.N * L.K / 2 + 4 * (L.M + L.N) + 8 * L.M * L.N
-                       for L in layers)
+            # in place: the compensation read from Y and Y written; GEMM first:
+            # Y written only
+            byts = sum(L.M * L.K / 2 + L.N * L.K / 2 + 4 * (L.M + L.N)
+                       + (4 if L.adds else 8) * L.M * L.N for L in layers)
             t_tensor = flops / (fp4_peak * 1e12)
             t_hbm = byts / (peaks["hbm_gbs"] * 1e9)
             if t_tensor >= t_hbm:
@@ -336,7 +360,8 @@ def _kernel_rows(layers, per_kernel, steps, peaks, sm_mhz, n_sm):
                      "ceilings_ms": {"tensor": round(1e3 * t_tensor, 4), "hbm": round(1e3 * t_hbm, 4)}}
         elif k == "spmm":
             # 2 nnz N fp32 FMA flops; every entry gathers its W row segment
-            # (nnz N elements) from L2, and C is written (4 M N bytes)
+            # (nnz N elements) from L2; Y is written (4 M N bytes) or, in the
+            # GEMM-first order, read and written by the memory system's adds
             algo = sum(2 * int(L.csr.nnz.item()) * L.N for L in layers) / 1e12
             bound, unit, peak = "alu", "TFLOP/s", alu_peak
             extra = {"w_row_gather_bytes": sum(int(L.csr.nnz.item()) * L.N * L.W.element_size()
@@ -413,6 +438,7 @@ def our_arm(args, rank, world, device):
         for L in layers:
             L.alpha = a
         warm()
+        orders = [list(L.order) for L in layers]
         m = _measure(qg, layers, args.steps, flush, world, device, args.no_graph)
         total_ms = max_over_ranks(sum(m["step_ms"]), world, device)
         sm_mhz = m["clocks"].get("sm_mhz") or peaks["sm_max_mhz"]
@@ -421,12 +447,14 @@ def our_arm(args, rank, world, device):
             rows[k]["ms_per_layer"] = [round(x, 4) for x in m["per_layer"][k]]
         nnz = [int(L.csr.nnz.item()) for L in layers]
         results.append(dict(alpha=a, m=m, total_ms=total_ms, rows=rows, fp4_peak=fp4_peak,
-                            sm_mhz=sm_mhz, nnz=nnz))
+                            sm_mhz=sm_mhz, nnz=nnz, orders=orders))
 
     head = results[0]
     m, rows, total_ms = head["m"], head["rows"], head["total_ms"]
     for L in layers:
         L.alpha = head["alpha"]
+        L.order = tuple(head["orders"][layers.index(L)])
+        L.adds = L.order[2] == "fp4_gemm"
     ms_per_step = total_ms / args.steps
     value = weak_scaling_value(flops_step, args.steps, total_ms, world) / 1e12
     dominant = max(KERNELS, key=lambda k: rows[k]["ms_per_step"])
@@ -458,6 +486,7 @@ def our_arm(args, rank, world, device):
         "gpu_launches": m["launches"],
         "cuda_graph": m["graph"],
         "nnz_per_layer": head["nnz"],
+        "call_order": [list(L.order) for L in layers],
         "breakdown_ms_per_step": round(sum(sum(v) for v in m["per_kernel"].values()) / args.steps, 4),
         "wall_s": round(m["wall"], 3),
     }
@@ -467,6 +496,7 @@ def our_arm(args, rank, world, device):
              "unit": "TFLOP/s", "ms_per_step": round(r["total_ms"] / args.steps, 4),
              "tokens_per_s": round(weak_scaling_value(tokens_step, args.steps, r["total_ms"], world), 1),
              "nnz_per_layer": r["nnz"], "gpu_launches": r["m"]["launches"],
+             "call_order": r["orders"],
              "kernels": {k: {kk: v[kk] for kk in ("ms_per_step", "achieved", "unit", "frac", "bound")}
                          for k, v in r["rows"].items()},
              "clocks": r["m"]["clocks"]}

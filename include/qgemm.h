@@ -201,6 +201,17 @@ qg_status qg_spmm_correction(const qg_csr* dA, int64_t M, const void* W, qg_dtyp
                              int64_t K, int64_t N, int64_t ldw, float* C, void* ws,
                              size_t ws_bytes, cudaStream_t stream);
 
+/* The compensation added into an existing fp32 output: Y += dA . W (M x N,
+ * row pitch N), with each row's sum formed as in qg_spmm_correction (fp32
+ * FMA chain in CSR order) and then added to Y by the memory system
+ * (red.global.add: fp32 round to nearest; a sum that is subnormal is
+ * flushed to zero).  Rows of dA without entries leave Y untouched.  With Y
+ * holding qg_fp4_gemm's output without C, the result is the layer's Y.
+ * Same arguments and errors as qg_spmm_correction. */
+qg_status qg_spmm_accumulate(const qg_csr* dA, int64_t M, const void* W, qg_dtype w_dtype,
+                             int64_t K, int64_t N, int64_t ldw, float* Y, void* ws,
+                             size_t ws_bytes, cudaStream_t stream);
+
 /* FP4 GEMM on tcgen05 tensor cores: acc_ij = sum_k e2m1(codesA_ik) *
  * e2m1(codesWT_jk) accumulated in fp32 (exact for K <= 16384), then
  * Y_ij = acc_ij * sA_i * sW_j (+ C_ij when C != NULL), stored as fp32 or bf16
@@ -239,7 +250,9 @@ qg_status qg_fp4_gemm_compensated(const uint8_t* codesA, const float* sA, const 
  *   fp32 Y: qg_spmm_correction(dA, W) written into Y itself, then
  *           qg_fp4_gemm(..., C = Y, Y) adding the scaled FP4 product to it in
  *           place (the epilogue reads every sub-tile of C before it writes
- *           that sub-tile of Y);
+ *           that sub-tile of Y); or, when alpha leaves at least 16 clamped
+ *           entries per row possible (n - ceil(alpha n) >= 16 M), the other
+ *           order: qg_fp4_gemm(..., C = NULL, Y), then qg_spmm_accumulate;
  *   bf16 Y: qg_fp4_gemm_compensated (the compensation inside the GEMM).
  * Both give Y_ij = fp32(acc_ij * sA_i * sW_j) + C_ij with C the fp32 FMA chain
  * of row i's entries (rounded to bf16 last for bf16 Y).  codesWT / sW come

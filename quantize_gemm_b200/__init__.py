@@ -43,7 +43,7 @@ EXPORTED = (
     "qg_spmm_correction", "qg_fp4_gemm", "qg_fp4_linear", "qg_launch_count",
     "qg_quantize_cols_static", "qg_fp4_dgrad", "qg_fp4_wgrad", "qg_mx_scale_bytes",
     "qg_mx_quantize_rows", "qg_mx_quantize_cols", "qg_mx_gemm", "qg_fp4_mma_loop",
-    "qg_fp4_linear_parts", "qg_fp4_gemm_compensated",
+    "qg_fp4_linear_parts", "qg_fp4_gemm_compensated", "qg_spmm_accumulate",
 )
 
 
@@ -84,6 +84,8 @@ _sig("qg_clamp_compensate", _INT,
 _sig("qg_quantize_act", _INT,
      [_P, _INT, _I64, _I64, _I64, _D, _P, _P, ctypes.POINTER(_Csr), _P, _P, _SZ, _P])
 _sig("qg_spmm_correction", _INT,
+     [ctypes.POINTER(_Csr), _I64, _P, _INT, _I64, _I64, _I64, _P, _P, _SZ, _P])
+_sig("qg_spmm_accumulate", _INT,
      [ctypes.POINTER(_Csr), _I64, _P, _INT, _I64, _I64, _I64, _P, _P, _SZ, _P])
 _sig("qg_fp4_gemm", _INT,
      [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _INT, _P, _P, _SZ, _P])
@@ -258,6 +260,23 @@ def qg_spmm_correction(csr: CSR, M, W, C, ws: Workspace, stream=None) -> int:
     c = csr.c()
     return _lib.qg_spmm_correction(ctypes.byref(c), M, _ptr(W), _dt(W), K, N, W.stride(0),
                                    _ptr(C), ws.ptr, ws.nbytes, _stream(stream))
+
+
+def qg_spmm_accumulate(csr: CSR, M, W, Y, ws: Workspace, stream=None) -> int:
+    K, N = W.shape
+    c = csr.c()
+    return _lib.qg_spmm_accumulate(ctypes.byref(c), M, _ptr(W), _dt(W), K, N, W.stride(0),
+                                   _ptr(Y), ws.ptr, ws.nbytes, _stream(stream))
+
+
+ADD_ORDER_ENTRIES_PER_ROW = 16   # the layer's order switch (see qg_fp4_linear)
+
+
+def linear_adds_into_y(M: int, K: int, alpha: float) -> bool:
+    """Whether qg_fp4_linear (fp32 Y) runs the GEMM first and adds the
+    compensation into Y (True) or writes the compensation first and lets the
+    GEMM add in place (False)."""
+    return qg_nnz_capacity(M * K, alpha) >= ADD_ORDER_ENTRIES_PER_ROW * M
 
 
 def qg_fp4_gemm(codesA, sA, codesWT, sW, M, N, K, C, Y, raw_acc, ws: Workspace,

@@ -270,6 +270,21 @@ qg_status qg_spmm_correction(const qg_csr* dA, int64_t M, const void* W, qg_dtyp
     return cuda_status(cudaGetLastError());
 }
 
+qg_status qg_spmm_accumulate(const qg_csr* dA, int64_t M, const void* W, qg_dtype w_dtype,
+                             int64_t K, int64_t N, int64_t ldw, float* Y, void* ws,
+                             size_t ws_bytes, cudaStream_t stream) {
+    if (!dtype_ok(w_dtype)) return QG_ERR_INVALID_ARG;
+    if (M < 1 || N < 1 || K < 1) return QG_ERR_UNSUPPORTED_SHAPE;
+    if (dA == nullptr || dA->row_ptr == nullptr) return QG_ERR_INVALID_ARG;
+    if (W == nullptr || !aligned16(W) || ldw < N || Y == nullptr || !aligned16(Y)) return QG_ERR_INVALID_ARG;
+    const WsLayout L = ws_layout(QG_OP_SPMM, M, K, N, w_dtype, 1.0);
+    qg_status st = check_ws(ws, ws_bytes, L.total);
+    if (st != QG_OK) return st;
+    if (ensure_device(nullptr) != cudaSuccess) return QG_ERR_CUDA;
+    launch_spmm(dA, M, W, w_dtype, N, ldw, Y, at<uint32_t>(ws, L.status), stream, true);
+    return cuda_status(cudaGetLastError());
+}
+
 qg_status qg_fp4_gemm(const uint8_t* codesA, const float* sA, const uint8_t* codesWT,
                       const float* sW, int64_t M, int64_t N, int64_t K, const float* C, void* Y,
                       qg_dtype y_dtype, float* raw_acc, void* ws, size_t ws_bytes,
@@ -321,15 +336,25 @@ qg_status qg_fp4_linear(const void* A, qg_dtype dtype, int64_t M, int64_t K,
                                      at<float>(ws, L.thr), stream);
     if (e != cudaSuccess) return QG_ERR_CUDA;
     if (y_dtype == QG_F32) {
-        // fp32 Y: the compensation dA . W is written into Y's own memory, and
-        // the GEMM's epilogue adds the scaled FP4 product to it in place (it
-        // reads each 32 x 32 sub-tile before it overwrites it; sub-tiles are
-        // disjoint), so no M x N buffer is needed besides Y
-        launch_spmm(&csr, M, W, dtype, N, N, static_cast<float*>(Y), status, stream);
+        // fp32 Y, no M x N buffer besides Y, in one of two orders with the same
+        // result: with many entries per row (at least kAddOrderEntriesPerRow
+        // possible on average) the GEMM writes the scaled product and the SpMM
+        // adds the compensation into Y, the SpMM's gathers hiding its reads of
+        // Y; otherwise the compensation is written into Y first and the GEMM's
+        // epilogue adds the product to it in place (it reads each 32 x 32
+        // sub-tile before it overwrites it; sub-tiles are disjoint)
+        float* Yf = static_cast<float*>(Y);
+        if (L.cap >= kAddOrderEntriesPerRow * M) {
+            e = launch_fp4_gemm(codes, scales, codesWT, sW, M, N, K, nullptr, Y, QG_F32, nullptr,
+                                status, stream);
+            if (e != cudaSuccess) return QG_ERR_CUDA;
+            launch_spmm(&csr, M, W, dtype, N, N, Yf, status, stream, true);
+            return cuda_status(cudaGetLastError());
+        }
+        launch_spmm(&csr, M, W, dtype, N, N, Yf, status, stream);
         if ((e = cudaGetLastError()) != cudaSuccess) return QG_ERR_CUDA;
-        return cuda_status(launch_fp4_gemm(codes, scales, codesWT, sW, M, N, K,
-                                           static_cast<const float*>(Y), Y, QG_F32, nullptr,
-                                           status, stream));
+        return cuda_status(launch_fp4_gemm(codes, scales, codesWT, sW, M, N, K, Yf, Y, QG_F32,
+                                           nullptr, status, stream));
     }
     // bf16 Y has no room for the fp32 compensation: the compensated GEMM
     // computes it inside the kernel instead

@@ -101,6 +101,9 @@ constexpr int kSfbCol = 480;
 #ifndef QG_GEMM_EPI_BUFS
 #define QG_GEMM_EPI_BUFS 4
 #endif
+#ifndef QG_GEMM_PAIR_EPI_BUFS
+#define QG_GEMM_PAIR_EPI_BUFS QG_GEMM_EPI_BUFS
+#endif
 #ifndef QG_GEMM_FORCE_BN
 #define QG_GEMM_FORCE_BN 0
 #endif
@@ -133,7 +136,8 @@ struct Cfg {
     static constexpr int kStages = MX ? QG_GEMM_MX_STAGES
                                       : CORR ? (PAIR ? QG_GEMM_PAIR_STAGES - 1 : QG_GEMM_SOLO_STAGES - 1)
                                              : (PAIR ? QG_GEMM_PAIR_STAGES : QG_GEMM_SOLO_STAGES);
-    static constexpr int kEpiB = (CORR && PAIR) ? 3 : kEpiBufs;   // sub-tile buffers per epilogue warp
+    // sub-tile buffers per epilogue warp (C loads in flight: kEpiB - 1 per warp)
+    static constexpr int kEpiB = (CORR && PAIR) ? 3 : PAIR ? QG_GEMM_PAIR_EPI_BUFS : kEpiBufs;
     static_assert(kEpiB >= 2 && kStages >= 2, "double buffering at least");
     static_assert(!MX || kMxSfCol + 16 * kStages <= kSfaCol, "MX scale slots below the constant scales");
     static constexpr int kBRows = PAIR ? BN / 2 : BN;   // rows of W^T loaded by one CTA
@@ -779,6 +783,12 @@ struct Params {
     const uint8_t* sfA;  // MX: E8M0 scale atoms of A, [row block][k group]
     const uint8_t* sfB;  // MX: the same for W^T
     int sf_groups;       // MX: 128-deep k groups per row block (even)
+    // Tile order of the persistent grid: m fastest (consecutive tiles share a
+    // column block: W's codes for it stay in L2 while A's codes stream) or n
+    // fastest (consecutive tiles share a row block: A's codes stay in L2).
+    // The host picks the order that keeps the larger code matrix streaming
+    // once and the smaller one resident.
+    int n_fastest;
     // CORR: dA in CSR, the unquantized W (K x N, row pitch ldw elements, bf16
     // or fp32) and the scratch slots (kCorrSlots x 128 x BN fp32 per CTA)
     const int32_t* row_ptr;
@@ -928,7 +938,8 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             uint32_t phase = 0;
             bool ok = true;
             for (int tile = unit; ok && tile < num_tiles; tile += n_units) {
-                const int m_blk = tile % num_m, n_blk = tile / num_m;
+                const int m_blk = p.n_fastest ? tile / num_n : tile % num_m;
+                const int n_blk = p.n_fastest ? tile % num_n : tile / num_m;
                 const int a_row = m_blk * CF::kTileRows + (int)rank * BM;
                 const int b_row = n_blk * BN + (int)rank * CF::kBRows;
                 for (int kb = 0; kb < num_kb; ++kb) {
@@ -1062,7 +1073,8 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         auto c_load = [&](int g) -> bool {
             const int ti = g / my_nc, c = par + kEpiSplit * (g - ti * my_nc);
             const int tile = unit + ti * n_units;
-            const int mb = tile % num_m, nbk = tile / num_m;
+            const int mb = p.n_fastest ? tile / num_n : tile % num_m;
+            const int nbk = p.n_fastest ? tile % num_n : tile / num_m;
             const int b = g % EB;
             int x = nbk * BN + c * 32, y = mb * CF::kTileRows + (int)rank * BM + 32 * q;
             if constexpr (CORR) {
@@ -1088,7 +1100,8 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         float srow_next = 0.0f;
         auto fetch_scales = [&](int ti) {
             const int tile = unit + ti * n_units;
-            const int m_blk = tile % num_m, n_blk = tile / num_m;
+            const int m_blk = p.n_fastest ? tile / num_n : tile % num_m;
+            const int n_blk = p.n_fastest ? tile % num_n : tile / num_m;
 #pragma unroll
             for (int k = 0; k < SWR; ++k) {
                 const int c = par + kEpiSplit * k;           // k-th chunk of this warp
@@ -1106,7 +1119,8 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         uint32_t va[32], vb[32];
         for (int ti = 0; ok && ti < my_tiles; ++ti) {
             const int tile = unit + ti * n_units;
-            const int m_blk = tile % num_m, n_blk = tile / num_m;
+            const int m_blk = p.n_fastest ? tile / num_n : tile % num_m;
+            const int n_blk = p.n_fastest ? tile % num_n : tile / num_m;
             const int row0 = m_blk * CF::kTileRows + (int)rank * BM + 32 * q;
             const int row = row0 + lane;
             // this tile's column scales into the warp's shared-memory copy
@@ -1266,7 +1280,8 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
         const bool lane_on = lane * 8 < BN;
         for (int ti = 0; ti < my_tiles; ++ti) {
             const int tile = unit + ti * n_units;
-            const int m_blk = tile % num_m, n_blk = tile / num_m;
+            const int m_blk = p.n_fastest ? tile / num_n : tile % num_m;
+            const int n_blk = p.n_fastest ? tile % num_n : tile / num_m;
             const int slot = ti & 1;
             if (!mbar_wait_warp(&B->corr_empty[slot], ((uint32_t)(ti >> 1) & 1u) ^ 1u, &B->abort,
                                 p.status))
@@ -1460,6 +1475,7 @@ cudaError_t launch_fp4_gemm(const uint8_t* codesA, const float* sA, const uint8_
     p.sfA = nullptr;
     p.sfB = nullptr;
     p.sf_groups = 0;
+    p.n_fastest = N < M ? 1 : 0;   // re-read the smaller code matrix from L2
     // TMA epilogue: the row pitches of Y and C must be multiples of 16 bytes
     const size_t ysz = (y_dtype == QG_BF16) ? 2 : 4;
 #ifndef QG_GEMM_DIRECT_EPI
@@ -1541,6 +1557,7 @@ cudaError_t launch_fp4_gemm_corr(const uint8_t* codesA, const float* sA, const u
     p.ldw = ldw;
     p.w_bf16 = (w_dtype == QG_BF16) ? 1 : 0;
     p.corr = scratch;
+    p.n_fastest = N < M ? 1 : 0;
     const size_t ysz = (y_dtype == QG_BF16) ? 2 : 4;
     p.tma_epi = (!QG_GEMM_DIRECT_EPI && ((size_t)N * ysz) % 16 == 0) ? 1 : 0;
     const bool pair = M > BM;

@@ -360,6 +360,13 @@ struct ActBuffers {
     int64_t row_slots;
 };
 
+// The layer's fp32 order switch: with at least this many clamped entries per
+// row possible (n - ceil(alpha n) over M), the GEMM writes Y first and the
+// SpMM adds into it (block16k, alpha 0.99: 41 per row, 4 % faster); below it,
+// the SpMM writes Y and the GEMM adds in place (alpha 0.999: 4 per row, the
+// other order is 9 % slower there).
+constexpr int64_t kAddOrderEntriesPerRow = 16;
+
 // Host-side argument checks shared by the C entry points.
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 inline bool dtype_ok(qg_dtype d) { return d == QG_F32 || d == QG_BF16; }
@@ -380,7 +387,7 @@ void launch_quantize_rows(const void* A, qg_dtype dt, int64_t M, int64_t K, int6
 void launch_quantize_cols(const void* W, qg_dtype dt, int64_t K, int64_t N, int64_t ldw,
                           uint8_t* codesT, float* scales, uint32_t* colmax, cudaStream_t s);
 void launch_spmm(const qg_csr* dA, int64_t M, const void* W, qg_dtype dt, int64_t N, int64_t ldw,
-                 float* C, uint32_t* status, cudaStream_t s);
+                 float* C, uint32_t* status, cudaStream_t s, bool add = false);
 void launch_mx_quantize_rows(const void* A, qg_dtype dt, int64_t M, int64_t K, int64_t lda,
                              uint8_t* codes, uint8_t* sf, uint32_t* status, cudaStream_t s);
 void launch_mx_quantize_cols(const void* W, qg_dtype dt, int64_t K, int64_t N, int64_t ldw,

@@ -27,6 +27,19 @@ constexpr int kSpmmWarps = kSpmmThreads / 32;
 constexpr int kSpmmSlice = 256;       // columns per CTA (32 lanes x 8)
 constexpr int kSpmmRowsPerCta = 32;
 
+// Y += v element by element in the memory system (red.global.add: fire and
+// forget, the L2 adds; fp32 round to nearest, with subnormal sums flushed to
+// zero).  Used when the compensation is added into an output that already
+// holds the scaled FP4 product.
+__device__ __forceinline__ void red_add4(float* p, float a, float b, float c, float d) {
+    asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(p), "f"(a), "f"(b), "f"(c),
+                 "f"(d)
+                 : "memory");
+}
+__device__ __forceinline__ void red_add1(float* p, float a) {
+    asm volatile("red.global.add.f32 [%0], %1;" ::"l"(p), "f"(a) : "memory");
+}
+
 template <qg_dtype DT>
 __device__ __forceinline__ void load_w8(const void* W, int64_t idx, bool vec, int n0, int N,
                                         float (&w)[8]) {
@@ -47,7 +60,7 @@ __device__ __forceinline__ void load_w8(const void* W, int64_t idx, bool vec, in
     }
 }
 
-template <qg_dtype DT>
+template <qg_dtype DT, bool ADD>
 __global__ void __launch_bounds__(kSpmmThreads)
 spmm_slice_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col,
                   const double* __restrict__ val, const void* __restrict__ W, int64_t ldw, int M,
@@ -101,8 +114,18 @@ spmm_slice_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restrict
             }
         }
         if (!col_ok) continue;
+        if (ADD && row_ptr[r] == row_ptr[r + 1]) continue;   // nothing to add
         float* crow = C + (int64_t)r * N + n0;
-        if (vec) {
+        if (ADD) {
+            if (vec) {
+                red_add4(crow, acc[0], acc[1], acc[2], acc[3]);
+                red_add4(crow + 4, acc[4], acc[5], acc[6], acc[7]);
+            } else {
+#pragma unroll
+                for (int e = 0; e < 8; ++e)
+                    if (n0 + e < N) red_add1(crow + e, acc[e]);
+            }
+        } else if (vec) {
             float4* d = reinterpret_cast<float4*>(crow);
             d[0] = make_float4(acc[0], acc[1], acc[2], acc[3]);
             d[1] = make_float4(acc[4], acc[5], acc[6], acc[7]);
@@ -168,7 +191,7 @@ __device__ __forceinline__ void fma_bf16x2(uint64_t& acc, uint64_t vv, uint32_t 
 
 // FULL: every quarter of the slice is inside N (all slices but the last when
 // N is not a multiple of the slice width), so loads and stores need no checks.
-template <int RPW, bool FULL>
+template <int RPW, bool FULL, bool ADD>
 __device__ __forceinline__ void spmm_stream_body(const int32_t* __restrict__ row_ptr,
                                                  const int32_t* __restrict__ col,
                                                  const double* __restrict__ val,
@@ -221,12 +244,27 @@ __device__ __forceinline__ void spmm_stream_body(const int32_t* __restrict__ row
     int rend = __shfl_sync(0xFFFFFFFFu, rp, 1) - P0;   // entries of rows <= row end here
     auto store_row = [&](int r) {
         float* crow = C + (int64_t)r * N + nbase;
+        // ADD: a row without entries adds nothing (its accumulators are 0)
+        const bool live = !ADD || __shfl_sync(0xFFFFFFFFu, rp, r - r_begin) !=
+                                      __shfl_sync(0xFFFFFFFFu, rp, r - r_begin + 1);
 #pragma unroll
         for (int h = 0; h < kStreamParts; ++h) {
-            if (okh[h]) {
-                ulonglong2* d = reinterpret_cast<ulonglong2*>(crow + 256 * h);
-                d[0] = make_ulonglong2(acc[4 * h + 0], acc[4 * h + 1]);
-                d[1] = make_ulonglong2(acc[4 * h + 2], acc[4 * h + 3]);
+            if (okh[h] && live) {
+                if constexpr (ADD) {
+                    float* d = crow + 256 * h;
+                    red_add4(d, __uint_as_float((uint32_t)acc[4 * h + 0]),
+                             __uint_as_float((uint32_t)(acc[4 * h + 0] >> 32)),
+                             __uint_as_float((uint32_t)acc[4 * h + 1]),
+                             __uint_as_float((uint32_t)(acc[4 * h + 1] >> 32)));
+                    red_add4(d + 4, __uint_as_float((uint32_t)acc[4 * h + 2]),
+                             __uint_as_float((uint32_t)(acc[4 * h + 2] >> 32)),
+                             __uint_as_float((uint32_t)acc[4 * h + 3]),
+                             __uint_as_float((uint32_t)(acc[4 * h + 3] >> 32)));
+                } else {
+                    ulonglong2* d = reinterpret_cast<ulonglong2*>(crow + 256 * h);
+                    d[0] = make_ulonglong2(acc[4 * h + 0], acc[4 * h + 1]);
+                    d[1] = make_ulonglong2(acc[4 * h + 2], acc[4 * h + 3]);
+                }
             }
         }
 #pragma unroll
@@ -273,22 +311,22 @@ __device__ __forceinline__ void spmm_stream_body(const int32_t* __restrict__ row
     }
 }
 
-template <int RPW>
+template <int RPW, bool ADD>
 __global__ void __launch_bounds__(kStreamWarps * 32, 2)
 spmm_stream_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restrict__ col,
                    const double* __restrict__ val, const uint16_t* __restrict__ W, int64_t ldw,
                    int M, int N, float* __restrict__ C) {
     if ((int)(blockIdx.y + 1) * kStreamSlice <= N)
-        spmm_stream_body<RPW, true>(row_ptr, col, val, W, ldw, M, N, C);
+        spmm_stream_body<RPW, true, ADD>(row_ptr, col, val, W, ldw, M, N, C);
     else
-        spmm_stream_body<RPW, false>(row_ptr, col, val, W, ldw, M, N, C);
+        spmm_stream_body<RPW, false, ADD>(row_ptr, col, val, W, ldw, M, N, C);
 }
 
 cudaError_t spmm_setup() { return cudaSuccess; }
 
-void launch_spmm(const qg_csr* dA, int64_t M, const void* W, qg_dtype dt, int64_t N, int64_t ldw,
-                 float* C, uint32_t* status, cudaStream_t s) {
-    (void)status;   // no device-side waits that could time out
+template <bool ADD>
+static void launch_spmm_as(const qg_csr* dA, int64_t M, const void* W, qg_dtype dt, int64_t N,
+                           int64_t ldw, float* C, cudaStream_t s) {
     if (dt == QG_BF16 && (N % 8) == 0 && (ldw % 8) == 0) {
         const int64_t slices = (N + kStreamSlice - 1) / kStreamSlice;
         const int64_t want = 8 * (int64_t)num_sms();
@@ -297,23 +335,32 @@ void launch_spmm(const qg_csr* dA, int64_t M, const void* W, qg_dtype dt, int64_
         dim3 grid((unsigned)((M + kStreamWarps * rpw - 1) / (kStreamWarps * rpw)), (unsigned)slices);
         const uint16_t* Wb = static_cast<const uint16_t*>(W);
         if (rpw == 4)
-            spmm_stream_kernel<4><<<grid, kStreamWarps * 32, 0, s>>>(dA->row_ptr, dA->col, dA->val, Wb, ldw, (int)M, (int)N, C);
+            spmm_stream_kernel<4, ADD><<<grid, kStreamWarps * 32, 0, s>>>(dA->row_ptr, dA->col, dA->val, Wb, ldw, (int)M, (int)N, C);
         else if (rpw == 2)
-            spmm_stream_kernel<2><<<grid, kStreamWarps * 32, 0, s>>>(dA->row_ptr, dA->col, dA->val, Wb, ldw, (int)M, (int)N, C);
+            spmm_stream_kernel<2, ADD><<<grid, kStreamWarps * 32, 0, s>>>(dA->row_ptr, dA->col, dA->val, Wb, ldw, (int)M, (int)N, C);
         else
-            spmm_stream_kernel<1><<<grid, kStreamWarps * 32, 0, s>>>(dA->row_ptr, dA->col, dA->val, Wb, ldw, (int)M, (int)N, C);
+            spmm_stream_kernel<1, ADD><<<grid, kStreamWarps * 32, 0, s>>>(dA->row_ptr, dA->col, dA->val, Wb, ldw, (int)M, (int)N, C);
         count_launch(1);
         return;
     }
     dim3 grid((unsigned)((M + kSpmmRowsPerCta - 1) / kSpmmRowsPerCta),
               (unsigned)((N + kSpmmSlice - 1) / kSpmmSlice));
     if (dt == QG_BF16)
-        spmm_slice_kernel<QG_BF16><<<grid, kSpmmThreads, 0, s>>>(dA->row_ptr, dA->col, dA->val, W,
-                                                                  ldw, (int)M, (int)N, C);
+        spmm_slice_kernel<QG_BF16, ADD><<<grid, kSpmmThreads, 0, s>>>(dA->row_ptr, dA->col, dA->val, W,
+                                                                       ldw, (int)M, (int)N, C);
     else
-        spmm_slice_kernel<QG_F32><<<grid, kSpmmThreads, 0, s>>>(dA->row_ptr, dA->col, dA->val, W,
-                                                                 ldw, (int)M, (int)N, C);
+        spmm_slice_kernel<QG_F32, ADD><<<grid, kSpmmThreads, 0, s>>>(dA->row_ptr, dA->col, dA->val, W,
+                                                                      ldw, (int)M, (int)N, C);
     count_launch(1);
+}
+
+// C = dA . W (add == false: every element of C written) or C += dA . W
+// (add == true: rows with entries only, added by the memory system).
+void launch_spmm(const qg_csr* dA, int64_t M, const void* W, qg_dtype dt, int64_t N, int64_t ldw,
+                 float* C, uint32_t* status, cudaStream_t s, bool add) {
+    (void)status;   // no device-side waits that could time out
+    if (add) launch_spmm_as<true>(dA, M, W, dt, N, ldw, C, s);
+    else launch_spmm_as<false>(dA, M, W, dt, N, ldw, C, s);
 }
 
 }  // namespace qg

@@ -270,3 +270,21 @@ def test_compensated_gemm_host_checks(qg):
              None)
     assert lib.qg_fp4_gemm_compensated(*bad_k) == qg.QG_ERR_UNSUPPORTED_SHAPE
     assert qg.qg_launch_count() == before
+
+
+def test_layer_order_switch(qg):
+    """The layer's fp32 order depends only on the clamped entries possible per
+    row: GEMM first from 16 per row up."""
+    assert qg.linear_adds_into_y(16384, 4096, 0.99)        # 41 per row
+    assert not qg.linear_adds_into_y(16384, 4096, 0.999)   # 4 per row
+    assert not qg.linear_adds_into_y(256, 512, 0.99)       # 5 per row
+    assert qg.linear_adds_into_y(4096, 2048, 0.99)         # 20 per row
+    lib = qg._lib
+    fake = ctypes.c_void_p(1 << 20)
+    csr = qg._Csr(1 << 20, 1 << 20, 1 << 20, 1000, 1 << 20)
+    assert lib.qg_spmm_accumulate(None, 64, fake, 1, 64, 64, 64, fake, fake, 1 << 30, None) == \
+        qg.QG_ERR_INVALID_ARG
+    assert lib.qg_spmm_accumulate(ctypes.byref(csr), 64, fake, 1, 64, 64, 32, fake, fake, 1 << 30,
+                                  None) == qg.QG_ERR_INVALID_ARG   # ldw < N
+    assert lib.qg_spmm_accumulate(ctypes.byref(csr), 64, fake, 1, 64, 64, 64, fake, fake, 16,
+                                  None) == qg.QG_ERR_WORKSPACE

@@ -312,6 +312,33 @@ def test_spmm_correction(qg, case, N, wdtype):
     assert np.all(np.abs(C - Co) <= bound), float(np.max(np.abs(C - Co) - bound))
 
 
+@pytest.mark.parametrize("case,N,wdtype", [("llama1.3b_attn_m512", 2048, torch.bfloat16),
+                                            ("tiny", 512, torch.float32),
+                                            ("bf16_ragged_k1056", 257, torch.bfloat16),
+                                            ("no_clamp", 600, torch.bfloat16),
+                                            ("clamp_almost_all", 264, torch.bfloat16)])
+def test_spmm_accumulate(qg, case, N, wdtype):
+    """Y += dA . W by the memory system's adds equals Y + (the stored
+    compensation), element by element in fp32; rows without entries are left
+    as they were."""
+    A, alpha = _act_inputs(case)
+    M, K = A.shape
+    W = make_matrix((K, N), seed=13, device="cuda", dtype=wdtype, scale=0.02)
+    _, csr, _ = qg.clamp_compensate(A, alpha, want_clamped=False)
+    Y0 = make_matrix((M, N), seed=14, device="cuda")
+    C = qg.spmm_correction(csr, M, W)
+    Y = Y0.clone()
+    ws = qg.Workspace(qg.QG_OP_SPMM, M, K, N, qg._dt(W))
+    assert qg.qg_spmm_accumulate(csr, M, W, Y, ws) == qg.QG_OK
+    qg.check_status(ws)
+    assert torch.equal(Y, Y0 + C)
+    rp = _np(csr.row_ptr)
+    empty = np.nonzero(np.diff(rp) == 0)[0]
+    if empty.size:
+        idx = torch.from_numpy(empty).cuda()
+        assert torch.equal(Y[idx], Y0[idx])
+
+
 # ------------------------------------------------------------------ FP4 GEMM
 GEMM_SHAPES = [(128, 256, 256), (1, 8, 32), (129, 257, 288), (300, 600, 1024),
                (1024, 1024, 4096), (256, 512, 16384), (4096, 2048, 2048), (513, 5504, 2048)]
