@@ -1362,6 +1362,17 @@ static bool encode_2d(CUtensorMap* map, CUtensorMapDataType dt, const void* base
               CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// Tile order: m fastest re-reads A's codes once per column block, n fastest
+// W's once per row block.  Both code matrices of the block16k qkv and o
+// layers (25-34 MB) stay in L2 beside the output stream either way, and m
+// fastest measured slightly better there; A's codes of the down layer
+// (16384 x 11008: 90 MB) do not, and n fastest cut that GEMM by a quarter.
+// So: n fastest when A's codes exceed 48 MB and W's codes are the smaller.
+static int n_fastest_order(int64_t M, int64_t N, int64_t K) {
+    const int64_t a_codes = M * (K / 2), w_codes = N * (K / 2);
+    return (a_codes > ((int64_t)48 << 20) && w_codes < a_codes) ? 1 : 0;
+}
+
 // Tile width: the persistent grid runs ceil(tiles / units) rounds of tiles
 // whose time grows with BN, so pick the width with the smaller rounds x BN;
 // on a tie, the one that pads N less.
@@ -1475,7 +1486,7 @@ cudaError_t launch_fp4_gemm(const uint8_t* codesA, const float* sA, const uint8_
     p.sfA = nullptr;
     p.sfB = nullptr;
     p.sf_groups = 0;
-    p.n_fastest = N < M ? 1 : 0;   // re-read the smaller code matrix from L2
+    p.n_fastest = n_fastest_order(M, N, K);
     // TMA epilogue: the row pitches of Y and C must be multiples of 16 bytes
     const size_t ysz = (y_dtype == QG_BF16) ? 2 : 4;
 #ifndef QG_GEMM_DIRECT_EPI
@@ -1557,7 +1568,7 @@ cudaError_t launch_fp4_gemm_corr(const uint8_t* codesA, const float* sA, const u
     p.ldw = ldw;
     p.w_bf16 = (w_dtype == QG_BF16) ? 1 : 0;
     p.corr = scratch;
-    p.n_fastest = N < M ? 1 : 0;
+    p.n_fastest = n_fastest_order(M, N, K);
     const size_t ysz = (y_dtype == QG_BF16) ? 2 : 4;
     p.tma_epi = (!QG_GEMM_DIRECT_EPI && ((size_t)N * ysz) % 16 == 0) ? 1 : 0;
     const bool pair = M > BM;
