@@ -462,28 +462,37 @@ __device__ __forceinline__ void band_units(const uint16_t* __restrict__ A, int64
     const int lane = threadIdx.x & 31;
     const int nchunks = K / 8;
     const int steps = (nchunks + 127) / 128;
-    const int64_t units = (int64_t)M * steps;
-    auto load_unit = [&](int64_t u, uint4 (&dst)[4]) {
-        const int64_t r = u / steps;
-        const int st = (int)(u - r * steps);
-        const uint16_t* base = A + r * lda;
+    // unit u = row * steps + step, walked u = gwarp, gwarp + nwarps, ...; the
+    // (row, step) pair is advanced by (dq, dr) = (nwarps / steps, nwarps %
+    // steps) per unit instead of dividing u (a 64-bit division per unit)
+    const int dq = nwarps / steps, dr = nwarps % steps;
+    int r = gwarp / steps, st = gwarp % steps;
+    auto advance = [&](int& rr, int& ss) {
+        rr += dq;
+        ss += dr;
+        if (ss >= steps) {
+            ss -= steps;
+            ++rr;
+        }
+    };
+    auto load_unit = [&](int rr, int ss, uint4 (&dst)[4]) {
+        const uint16_t* base = A + (int64_t)rr * lda;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-            const int c = st * 128 + 32 * j + lane;
+            const int c = ss * 128 + 32 * j + lane;
             dst[j] = (c < nchunks) ? __ldg(reinterpret_cast<const uint4*>(base) + c)
                                    : make_uint4(0u, 0u, 0u, 0u);
         }
     };
-    int64_t u = gwarp;
     uint4 nxt[4];
-    if (u < units) load_unit(u, nxt);
-    while (u < units) {
+    if (r < M) load_unit(r, st, nxt);
+    while (r < M) {
         uint4 cur[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) cur[j] = nxt[j];
-        const int64_t nu = u + nwarps;
-        if (nu < units) load_unit(nu, nxt);
-        const int st = (int)(u % steps);
+        int nr = r, ns = st;
+        advance(nr, ns);
+        if (nr < M) load_unit(nr, ns, nxt);
         uint32_t mx = 0, mx1 = 0, cnt = 0, cnt1 = 0;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -507,10 +516,11 @@ __device__ __forceinline__ void band_units(const uint16_t* __restrict__ A, int64
         mx = max_u16x2(mx, mx1);
         cnt += cnt1;
         const uint32_t km = warp_max_u32(max(mx & 0xFFFFu, mx >> 16));
-        if (lane == 0) rowmax[u] = km;
+        if (lane == 0) rowmax[(int64_t)r * steps + st] = km;
         bad |= (km >= nonfinite_key<QG_BF16>()) ? 1u : 0u;
         n_ge += (cnt & 0xFFFFu) + (cnt >> 16);
-        u = nu;
+        r = nr;
+        st = ns;
     }
 }
 

@@ -150,15 +150,11 @@ spmm_slice_kernel(const int32_t* __restrict__ row_ptr, const int32_t* __restrict
 // A warp owns RPW consecutive rows, whose CSR entries form one contiguous
 // range consumed in order.
 constexpr int kStreamWarps = 8;
-// A warp owns RPW consecutive rows (16, 8, 4, 2 or 1).  The launcher starts
-// from 4 rows, or more when rows are short (few clamped entries per row
-// possible: a warp should have some 64 entries to stream, or its start-up
-// latency -- the row pointers, the first entry batch, the first W segments
-// -- is most of its time), and halves RPW while that leaves fewer than eight
-// CTAs' worth of work per SM, so narrow or short problems get more, smaller
-// CTAs.
-constexpr int kStreamMaxRowsPerWarp = 16;
-constexpr int kStreamEntriesPerWarp = 64;
+// A warp owns RPW consecutive rows (4, 2 or 1): the launcher takes the
+// largest RPW that still gives every SM eight CTAs' worth of work, so narrow
+// or short problems get more, smaller CTAs.  (8 or 16 rows per warp for
+// short rows -- alpha 0.999, ~4 entries per row -- measured no faster.)
+constexpr int kStreamMaxRowsPerWarp = 4;
 #ifndef QG_SPMM_PARTS
 #define QG_SPMM_PARTS 4
 #endif
@@ -335,17 +331,11 @@ static void launch_spmm_as(const qg_csr* dA, int64_t M, const void* W, qg_dtype 
     if (dt == QG_BF16 && (N % 8) == 0 && (ldw % 8) == 0) {
         const int64_t slices = (N + kStreamSlice - 1) / kStreamSlice;
         const int64_t want = 8 * (int64_t)num_sms();
-        const double per_row = (double)dA->nnz_capacity / (double)M;   // entries per row, at most
-        int rpw = 4;
-        while (rpw < kStreamMaxRowsPerWarp && rpw * per_row < kStreamEntriesPerWarp) rpw *= 2;
+        int rpw = kStreamMaxRowsPerWarp;
         while (rpw > 1 && ((M + kStreamWarps * rpw - 1) / (kStreamWarps * rpw)) * slices < want) rpw /= 2;
         dim3 grid((unsigned)((M + kStreamWarps * rpw - 1) / (kStreamWarps * rpw)), (unsigned)slices);
         const uint16_t* Wb = static_cast<const uint16_t*>(W);
-        if (rpw == 16)
-            spmm_stream_kernel<16, ADD><<<grid, kStreamWarps * 32, 0, s>>>(dA->row_ptr, dA->col, dA->val, Wb, ldw, (int)M, (int)N, C);
-        else if (rpw == 8)
-            spmm_stream_kernel<8, ADD><<<grid, kStreamWarps * 32, 0, s>>>(dA->row_ptr, dA->col, dA->val, Wb, ldw, (int)M, (int)N, C);
-        else if (rpw == 4)
+        if (rpw == 4)
             spmm_stream_kernel<4, ADD><<<grid, kStreamWarps * 32, 0, s>>>(dA->row_ptr, dA->col, dA->val, Wb, ldw, (int)M, (int)N, C);
         else if (rpw == 2)
             spmm_stream_kernel<2, ADD><<<grid, kStreamWarps * 32, 0, s>>>(dA->row_ptr, dA->col, dA->val, Wb, ldw, (int)M, (int)N, C);
