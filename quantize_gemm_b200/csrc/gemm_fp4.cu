@@ -110,9 +110,6 @@ constexpr int kSfbCol = 480;
 #ifndef QG_GEMM_MX_STAGES
 #define QG_GEMM_MX_STAGES 4
 #endif
-#ifndef QG_MX_PREFETCH_SCALES
-#define QG_MX_PREFETCH_SCALES 0
-#endif
 constexpr int kMxSfCol = 256;        // MX: per-stage scale slots, 16 columns each
 constexpr int kMxAtom = 512;         // 32 rows x 16 bytes of E8M0 scales (128 rows x 4 blocks)
 constexpr int kMxStageSf = 4 * kMxAtom;   // two atoms of A, two of W^T per 256-deep stage
@@ -999,11 +996,8 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
             uint32_t phase = 0, acc_phase = 0;
             bool ok = true;
             // MX: a stage's four scale atoms go into its TMEM slot with
-            // tcgen05.cp before its MMAs; with QG_MX_PREFETCH_SCALES the
-            // copies of the next stage are issued before this stage's MMAs
-            // when its data has already landed (bit s of `copied`: stage s's
-            // scales are in its slot for the round about to use them)
-            uint32_t copied = 0;
+            // tcgen05.cp right before its MMAs (issuing them one stage early,
+            // when the next stage's data had landed, measured 13 % slower)
             auto copy_scales = [&](int st) {
                 const uint32_t slot = tmem + (uint32_t)(kMxSfCol + 16 * st);
                 const uint32_t s0 = smem_u32(ssf + (size_t)st * kMxStageSf);
@@ -1026,19 +1020,7 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                         // this stage's scales into its TMEM slot: A atoms at +0, +4,
                         // W^T atoms at +8, +12; the copies run before the MMAs
                         const uint32_t slot = tmem + (uint32_t)(kMxSfCol + 16 * stage);
-                        if (!((copied >> stage) & 1u)) copy_scales(stage);
-                        copied &= ~(1u << stage);
-#if QG_MX_PREFETCH_SCALES
-                        {
-                            const int nx = stage + 1 == S ? 0 : stage + 1;
-                            const uint32_t nph = stage + 1 == S ? phase ^ 1u : phase;
-                            if (mbar_try_wait(&B->full[nx], nph)) {
-                                tc_fence_after();
-                                copy_scales(nx);
-                                copied |= 1u << nx;
-                            }
-                        }
-#endif
+                        copy_scales(stage);
 #pragma unroll
                         for (int ks = 0; ks < BK_BYTES / UMMA_K_BYTES; ++ks) {
                             // MMA ks covers 32-blocks 2 ks, 2 ks + 1: atom ks / 2, bytes
