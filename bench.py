@@ -587,8 +587,9 @@ def e2e_arm(qg, args, layers, device, world):
 
 
 def _ncu_traffic(kernel, workload):
-    """DRAM bytes per launch from a committed ncu summary, when it was taken
-    on the current source of that kernel (else None)."""
+    """DRAM bytes of one step (the kernel's launches over the workload's
+    layers, the unit `achieved` is counted in) from a committed ncu summary,
+    when it was taken on the current source of that kernel (else None)."""
     path = os.path.join(ROOT, "profiles", "traffic.json")
     if not os.path.exists(path):
         return None
@@ -603,7 +604,7 @@ def _ncu_traffic(kernel, workload):
         return None
     with open(src, "rb") as f:
         sha = hashlib.sha256(f.read()).hexdigest()[:16]
-    return rec["dram_bytes_per_launch"] if sha == rec["source_sha256_16"] else None
+    return rec.get("dram_bytes_per_step") if sha == rec["source_sha256_16"] else None
 
 
 # ------------------------------------------------------------------ CPU oracle
