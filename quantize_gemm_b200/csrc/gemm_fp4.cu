@@ -50,15 +50,18 @@
 // CORR = true (the layer's compensated GEMM): kCorrWarps more warps compute
 // the compensation dA . W of each output tile on the CUDA cores while the
 // tensor pipe runs the tile's MMAs.  A correction warp owns a contiguous block
-// of the CTA's 128 rows; lane l owns the 8 columns [8 l, 8 l + 8) of the
-// tile; the warp walks its rows' CSR entries as one stream, keeping a ring of
-// W-row segments (16 bytes per lane per entry) in flight, and accumulates
-// each row with fp32 FMAs in the row's CSR order.  Finished rows go to this
-// CTA's slot of a small scratch ring in global memory (2 slots of 128 x BN
-// fp32 per CTA, rewritten every other tile, so it stays in L2), and the
-// epilogue TMA-loads them exactly as it loads a caller's C.  Two barrier
-// pairs (corr_full / corr_empty) hand the slots between the two roles.  The
-// dense M x N fp32 correction never exists.
+// of the CTA's 128 rows, split into four quarter-warp row blocks; a quarter
+// walks its rows' CSR entries as one stream, each of its lanes summing 32 of
+// the tile's columns, with the W-row chunks in flight copied L2 -> shared
+// memory by cp.async into a per-warp ring (corr_rows4s; bf16 W with N and
+// its pitch multiples of 8), or, otherwise, a warp walks its rows with 8
+// columns per lane and a register ring (corr_rows).  Each row is an fp32 FMA
+// chain in CSR order.  Finished rows go to this CTA's slot of a small
+// scratch ring in global memory (2 slots of 128 x BN fp32 per CTA, rewritten
+// every other tile, so it stays in L2), and the epilogue TMA-loads them
+// exactly as it loads a caller's C.  Two barrier pairs (corr_full /
+// corr_empty) hand the slots between the two roles.  The dense M x N fp32
+// correction never exists.
 // Every mbarrier wait is bounded; a wait that gives up sets the timeout bit in
 // the status word, raises a CTA-wide abort flag, waits (bounded) for copies
 // and MMAs in flight, frees TMEM and returns.
