@@ -256,24 +256,20 @@ __device__ void block_select3(const uint32_t* sh, const unsigned long long (&r)[
     __syncthreads();
 }
 
-// One CTA of NT threads: zero the counters and band bins, histogram the keys
-// >> 3 of a sample (windows of 64 rows spread evenly over A) in sh, and put
-// the band around the sample quantile with a margin of six standard
-// deviations of a sample quantile's rank plus 32.  A margin that runs past
-// the sample's largest (smallest) key opens the band upwards (downwards), up
-// to its 4096-key width, so an extreme quantile is not missed for want of
-// sampled keys above it.
+// One CTA of NT threads: histogram the keys >> 3 of a sample (windows of 64
+// rows spread evenly over A) in sh, and put the band around the sample
+// quantile with a margin of six standard deviations of a sample quantile's
+// rank plus 32.  A margin that runs past the sample's largest (smallest) key
+// opens the band upwards (downwards), up to its 4096-key width, so an extreme
+// quantile is not missed for want of sampled keys above it.  Writes nothing
+// but sh: every CTA that runs it on the same A gets the same band.
 template <int NT>
-__device__ void cta_sample_band(const uint16_t* __restrict__ A, int64_t lda, int M, int K,
-                                Counters* __restrict__ ctr, uint32_t* __restrict__ band_bins,
-                                unsigned long long rank, uint32_t* sh) {
+__device__ void cta_band_local(const uint16_t* __restrict__ A, int64_t lda, int M, int K,
+                               unsigned long long rank, uint32_t* sh, uint32_t& lo_out,
+                               uint32_t& hi_out) {
     __shared__ uint32_t s_sel[3];
+    __shared__ uint32_t s_band[2];
     const int t = threadIdx.x;
-    uint32_t* cz = reinterpret_cast<uint32_t*>(ctr);
-    for (int i = t; i < (int)(sizeof(Counters) / 4); i += NT) cz[i] = 0u;
-    for (int i = t; i < kBandBins; i += NT) band_bins[i] = 0u;
-    for (int i = t; i < kSampleBins; i += NT) sh[i] = 0u;
-    __syncthreads();
     // R rows evenly spaced over M (row ri * M / R); from each a window of cpr
     // 16-byte chunks whose start moves from row to row
     const int nch = K / 8;
@@ -283,6 +279,9 @@ __device__ void cta_sample_band(const uint16_t* __restrict__ A, int64_t lda, int
     const int total = R * cpr;
     const int mq = M / R, mr = M % R;
     constexpr int U = (int)((kSampleTarget / 8 + NT - 1) / NT);   // loads per thread per round
+    for (int i = t; i < kSampleBins; i += NT) sh[i] = 0u;
+    if (t < 3) s_sel[t] = 0u;
+    __syncthreads();
     for (int q0 = t; q0 < total; q0 += U * NT) {
         uint4 v[U];
 #pragma unroll
@@ -319,8 +318,6 @@ __device__ void cta_sample_band(const uint16_t* __restrict__ A, int64_t lda, int
         (unsigned long long)fmin(fmax(floor(center - margin), 0.0), top),
         (unsigned long long)fmin(fmax(ceil(center + margin), 0.0), top),
         (unsigned long long)fmin(fmax(center, 0.0), top)};
-    if (t < 3) s_sel[t] = 0u;
-    __syncthreads();
     block_select3<NT>(sh, r, s_sel);
     if (t == 0) {
         uint32_t lo = s_sel[0] << 3, hi = (s_sel[1] << 3) + 7u;
@@ -331,6 +328,27 @@ __device__ void cta_sample_band(const uint16_t* __restrict__ A, int64_t lda, int
             lo = max(lo, mid > (uint32_t)(kBandBins / 2) ? mid - kBandBins / 2 : 0u);
             hi = min(hi, lo + kBandBins - 1);
         }
+        s_band[0] = lo;
+        s_band[1] = hi;
+    }
+    __syncthreads();
+    lo_out = s_band[0];
+    hi_out = s_band[1];
+    __syncthreads();   // sh and s_band may be reused
+}
+
+// The same band, with the counters and band bins zeroed and the band stored
+// in the counters (the one-CTA kernel of the multi-kernel sequence).
+template <int NT>
+__device__ void cta_sample_band(const uint16_t* __restrict__ A, int64_t lda, int M, int K,
+                                Counters* __restrict__ ctr, uint32_t* __restrict__ band_bins,
+                                unsigned long long rank, uint32_t* sh) {
+    uint32_t* cz = reinterpret_cast<uint32_t*>(ctr);
+    for (int i = threadIdx.x; i < (int)(sizeof(Counters) / 4); i += NT) cz[i] = 0u;
+    for (int i = threadIdx.x; i < kBandBins; i += NT) band_bins[i] = 0u;
+    uint32_t lo, hi;
+    cta_band_local<NT>(A, lda, M, K, rank, sh, lo, hi);
+    if (threadIdx.x == 0) {
         ctr->band_lo = lo;
         ctr->band_hi = hi;
     }
@@ -1075,8 +1093,8 @@ csr_scatter_kernel(const Counters* __restrict__ ctr, ActBuffers b, int M,
                     (int64_t)gridDim.x * blockDim.x);
 }
 
-// Exclusive scan of n counts (in[0..n)) into out[0..n) by one CTA of NT
-// threads; the total goes to *total.  Reads and writes this CTA's own data.
+// Exclusive scan of n counts (in[0..n), written by any CTA: read around L1)
+// into out[0..n) by one CTA of NT threads; the total goes to *total.
 template <int NT>
 __device__ void cta_local_scan(const uint32_t* in, int n, uint32_t* out, uint32_t* total) {
     __shared__ uint32_t s_w[NT / 32];
@@ -1084,7 +1102,7 @@ __device__ void cta_local_scan(const uint32_t* in, int n, uint32_t* out, uint32_
     const int per = (n + NT - 1) / NT;
     const int a = min(n, t * per), e = min(n, a + per);
     uint32_t mine = 0;
-    for (int i = a; i < e; ++i) mine += in[i];
+    for (int i = a; i < e; ++i) mine += __ldcg(in + i);
     const uint32_t incl = (uint32_t)warp_inclusive_scan((int)mine);
     if (lane == 31) s_w[w] = incl;
     __syncthreads();
@@ -1094,7 +1112,7 @@ __device__ void cta_local_scan(const uint32_t* in, int n, uint32_t* out, uint32_
         all += s_w[i];
     }
     for (int i = a; i < e; ++i) {
-        const uint32_t c = in[i];
+        const uint32_t c = __ldcg(in + i);
         out[i] = run;
         run += c;
     }
@@ -1138,13 +1156,65 @@ __device__ void cta_scan_offsets(uint32_t* cta_tot, int ncta, const ActBuffers& 
 }
 
 // --------------------------------------------------------------------------
+// Phase 5 of the fused kernel: the staged entries of rows [r0, r1) to their
+// CSR positions rowpre[r] + off.  A warp takes kScatterRows rows at a time and
+// issues the loads of all of them before any store (staged data was written
+// by other SMs: read around L1).
+constexpr int kScatterRows = 4;
+template <int NT>
+__device__ __forceinline__ void scatter_rows(const ActBuffers& b, int r0, int r1, uint32_t off,
+                                             int32_t* __restrict__ col, double* __restrict__ val) {
+    constexpr int RB = kScatterRows;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    const int row_slots = (int)b.row_slots;
+    for (int rb = r0 + warp * RB; rb < r1; rb += (NT / 32) * RB) {
+        int cnt = 0;
+        long long dst = 0;
+        if (lane < RB && rb + lane < r1) {
+            cnt = min((int)__ldcg(b.rowcnt + rb + lane), row_slots);
+            dst = (long long)__ldcg(b.rowpre + rb + lane) + off;
+        }
+        int c4[RB];
+        long long d4[RB];
+        int maxn = 0;
+#pragma unroll
+        for (int q = 0; q < RB; ++q) {
+            c4[q] = __shfl_sync(0xFFFFFFFFu, cnt, q);
+            d4[q] = __shfl_sync(0xFFFFFFFFu, dst, q);
+            maxn = max(maxn, c4[q]);
+        }
+        for (int j = lane; j < maxn; j += 32) {
+            int cv[RB];
+            double vv[RB];
+#pragma unroll
+            for (int q = 0; q < RB; ++q) {
+                cv[q] = 0;
+                vv[q] = 0.0;
+                if (j < c4[q]) {
+                    const int64_t src = (int64_t)(rb + q) * row_slots + j;
+                    cv[q] = __ldcg(b.st_col + src);
+                    vv[q] = __ldcg(b.st_val + src);
+                }
+            }
+#pragma unroll
+            for (int q = 0; q < RB; ++q) {
+                if (j < c4[q]) {
+                    col[d4[q] + j] = cv[q];
+                    val[d4[q] + j] = vv[q];
+                }
+            }
+        }
+    }
+}
+
 // The whole bf16 quantize_act in one cooperative launch (all CTAs resident):
-//   phase 0  CTA 0 samples A and sets the band (the others wait)
+//   phase 0  every CTA puts the band around the quantile of the same sample
+//            of A (so no barrier follows); CTA 0 also zeroes the counters
 //   phase 1  band pass: row maxima, band histogram, count below the band
 //   phase 2  the last CTA to finish phase 1 selects T, then releases the rest
 //   phase 3  clamp / quantize / dA staging
 //   phase 4  the last CTA to finish phase 3 scans the row counts into row_ptr
-//   phase 5  CSR scatter
+//   phase 5  CSR scatter (a warp moves four rows' entries at a time)
 // The grid barriers are a count and a generation word in the workspace
 // (count returns to 0 after every barrier).  Every wait is bounded: a CTA
 // that gives up sets the timeout bit and returns (the workspace barrier words
@@ -1168,26 +1238,40 @@ act_fused_bf16_kernel(const uint16_t* __restrict__ A, int64_t lda, int M, int K,
     const int gwarp = blockIdx.x * wpc + (threadIdx.x >> 5), nwarps = gridDim.x * wpc;
     GridSync* g = b.gsync;
     uint32_t gen0;
+    uint32_t lo, hi;
 
-    // phase 0 (the other CTAs pull their first band row into L2 meanwhile)
+    // phase 0: every CTA puts the band around the quantile of the same sample
+    // of A, so no barrier follows.  CTA 0 also zeroes the counters and band
+    // bins and then publishes zflag = gen + 1 (the generation word cannot
+    // move before every CTA has arrived at the first barrier, so all CTAs
+    // read the same gen here); each CTA checks it before adding into them.
+    __shared__ uint32_t s_gen;
+    if (threadIdx.x == 0) s_gen = ld_relaxed_u32(&g->gen);
     if (blockIdx.x == 0) {
-        cta_sample_band<kFusedThreads>(A, lda, M, K, b.ctr, b.hist1, rank, sh);
-    } else if (gwarp < M) {
-        const char* rowp = reinterpret_cast<const char*>(A + (int64_t)gwarp * lda);
-        for (int c = threadIdx.x & 31; c < K * 2 / 128; c += 32)
-            asm volatile("prefetch.global.L2 [%0];" ::"l"(rowp + (int64_t)c * 128));
+        uint32_t* cz = reinterpret_cast<uint32_t*>(b.ctr);
+        for (int i = threadIdx.x; i < (int)(sizeof(Counters) / 4); i += kFusedThreads) cz[i] = 0u;
+        for (int i = threadIdx.x; i < kBandBins; i += kFusedThreads) b.hist1[i] = 0u;
     }
-    if (grid_arrive(g, gen0)) grid_release(g);
-    else if (!grid_wait(g, gen0, b.status)) return;
+    cta_band_local<kFusedThreads>(A, lda, M, K, rank, sh, lo, hi);
+    const uint32_t zwant = s_gen + 1u;
+    if (blockIdx.x == 0) {
+        if (threadIdx.x == 0) {
+            b.ctr->band_lo = lo;
+            b.ctr->band_hi = hi;
+        }
+        __threadfence();
+        flag_publish(&g->zflag, zwant);
+    }
 
     // phase 1
     for (int i = threadIdx.x; i < kBandBins; i += kFusedThreads) sh[i] = 0u;
     __syncthreads();
     {
-        const uint32_t lo = __ldcg(&b.ctr->band_lo), hi = __ldcg(&b.ctr->band_hi);
         unsigned long long n_ge = 0;
         uint32_t bad = 0;
         band_units(A, lda, M, K, lo, hi, sh, b.rowmax, gwarp, nwarps, n_ge, bad);
+        // the counters and bins that CTA 0 zeroed (published before its band pass)
+        if (!flag_wait(&g->zflag, zwant, b.status)) return;
         band_flush<kFusedThreads>(sh, b.hist1, n_ge, bad, b.ctr);
     }
     // phase 2
@@ -1219,19 +1303,10 @@ act_fused_bf16_kernel(const uint16_t* __restrict__ A, int64_t lda, int M, int K,
     // the overflow list
     const uint32_t off = __ldcg(cta_off + blockIdx.x);
     for (int r = r0 + (int)threadIdx.x; r < r1; r += kFusedThreads)
-        row_ptr[r] = (int32_t)(b.rowpre[r] + off);
+        row_ptr[r] = (int32_t)(__ldcg(b.rowpre + r) + off);
+    scatter_rows<kFusedThreads>(b, r0, r1, off, col, val);
     {
-        const int lane = threadIdx.x & 31;
         const int row_slots = (int)b.row_slots;
-        for (int r = r0 + (int)(threadIdx.x >> 5); r < r1; r += wpc) {
-            const int n = min((int)b.rowcnt[r], row_slots);
-            const int64_t dst = (int64_t)b.rowpre[r] + off;
-            const int64_t src = (int64_t)r * row_slots;
-            for (int jj = lane; jj < n; jj += 32) {
-                col[dst + jj] = __ldcg(b.st_col + src + jj);
-                val[dst + jj] = __ldcg(b.st_val + src + jj);
-            }
-        }
         const unsigned long long n_over = min(__ldcg(&b.ctr->nnz), (unsigned long long)b.cap);
         const int64_t base = (int64_t)M * row_slots;
         for (unsigned long long e = blockIdx.x * (unsigned long long)kFusedThreads + threadIdx.x;

@@ -62,13 +62,17 @@ constexpr int kHist2Bins = 1 << 16;   // fp32 refine: low 16 bits of |x|
 
 inline size_t align_up(size_t x) { return (x + kAlign - 1) / kAlign * kAlign; }
 
-// Grid barrier of the cooperative activation kernel (inside the status block,
-// so qg_workspace_init zeroes it; the count is back to 0 after every barrier).
+// Grid barrier of the cooperative kernels (inside the status block, so
+// qg_workspace_init zeroes it; the count is back to 0 after every barrier),
+// and the fused activation kernel's flag: gen + 1 once CTA 0 has zeroed that
+// call's counters.
 struct GridSync {
     uint32_t count;
     uint32_t gen;
+    uint32_t zflag;
 };
 constexpr size_t kGridSyncOffset = 16;   // bytes from the workspace base
+static_assert(kGridSyncOffset + sizeof(GridSync) <= 2 * kAlign, "inside the zeroed header");
 
 // Scratch of the compensated GEMM: two slots of 128 rows x 224 fp32 columns
 // per CTA, for up to 160 CTAs (36.7 MB; it stays in L2).
@@ -97,7 +101,7 @@ inline WsLayout ws_layout(qg_op op, int64_t M, int64_t K, int64_t N, qg_dtype dt
         off = align_up(off + (bytes ? bytes : 1));
         return at;
     };
-    L.status = take(32);   // status word at +0, GridSync at +16
+    L.status = take(kGridSyncOffset + sizeof(GridSync));   // status word at +0, GridSync at +16
     L.gsync = L.status + kGridSyncOffset;
     L.counters = take(sizeof(Counters));
     bool act = (op == QG_OP_CLAMP_COMPENSATE || op == QG_OP_QUANTIZE_ACT ||
@@ -340,6 +344,33 @@ __device__ __forceinline__ bool grid_wait(GridSync* g, uint32_t gen0, uint32_t* 
     }
     __syncthreads();
     return s_ok != 0;
+}
+
+
+// Publish a flag value (thread 0, after every thread of the CTA is done with
+// the writes it orders) and wait for it (thread 0 polls with a bound; every
+// thread returns false when the wait gave up, after the timeout bit is set).
+__device__ __forceinline__ void flag_publish(uint32_t* flag, uint32_t value) {
+    __syncthreads();
+    if (threadIdx.x == 0)
+        asm volatile("st.release.gpu.global.u32 [%0], %1;" ::"l"(flag), "r"(value) : "memory");
+}
+__device__ __forceinline__ bool flag_wait(const uint32_t* flag, uint32_t want, uint32_t* status) {
+    __shared__ int s_fok;
+    if (threadIdx.x == 0) {
+        int ok = 1;
+        const long long t0 = clock64();
+        while (ld_acquire_u32(flag) != want) {
+            if (clock64() - t0 > kGridWaitLimit) {
+                ok = 0;
+                flag_status(status, kStatusTimeout);
+                break;
+            }
+        }
+        s_fok = ok;
+    }
+    __syncthreads();
+    return s_fok != 0;
 }
 
 #endif  // __CUDACC__
