@@ -852,6 +852,7 @@ clamp_quant_kernel(const void* __restrict__ A, int64_t lda, int M, int K,
 // this step's work.  Warps walk rows grid-stride; a step covers 1024 columns
 // of one row.
 constexpr int kQ3Threads = 256;
+constexpr int kStepListCap = 512;   // outliers per 1024-column step held in a warp's list
 #ifndef QG_CLAMP_MIN_BLOCKS
 #define QG_CLAMP_MIN_BLOCKS 3
 #endif
@@ -868,7 +869,7 @@ __device__ __forceinline__ void clamp_rows_bf16(const uint16_t* __restrict__ A, 
                                                 uint8_t* __restrict__ codes,
                                                 float* __restrict__ scales, const ActBuffers& b,
                                                 int first, int stride, int row_end,
-                                                int nparts = 1) {
+                                                int nparts, uint16_t* olist) {
     // (an unselected threshold reads as the largest finite-or-not key)
     const uint32_t Tk = min(T_key, 0x7FFFu);
     const uint32_t cT = (0x7FFFu - Tk) * 0x10001u;   // SWAR: key > T sets bit 15
@@ -953,19 +954,17 @@ __device__ __forceinline__ void clamp_rows_bf16(const uint16_t* __restrict__ A, 
             const uint32_t t01 = __shfl_sync(0xFFFFFFFFu, i01, 31);
             const uint32_t t23 = __shfl_sync(0xFFFFFFFFu, i23, 31);
             const uint32_t e01 = i01 - c01, e23 = i23 - c23;
-            // first rank of this lane's outliers in chunk j
-            const int b0 = row_rank + (int)(e01 & 0xFFFF);
-            const int b1 = row_rank + (int)(t01 & 0xFFFF) + (int)(e01 >> 16);
-            const int b2 = row_rank + (int)(t01 & 0xFFFF) + (int)(t01 >> 16) + (int)(e23 & 0xFFFF);
-            const int b3 = row_rank + (int)(t01 & 0xFFFF) + (int)(t01 >> 16) + (int)(t23 & 0xFFFF) +
-                           (int)(e23 >> 16);
+            // first rank within the step of this lane's outliers in chunk j
+            const int b0 = (int)(e01 & 0xFFFF);
+            const int b1 = (int)(t01 & 0xFFFF) + (int)(e01 >> 16);
+            const int b2 = (int)(t01 & 0xFFFF) + (int)(t01 >> 16) + (int)(e23 & 0xFFFF);
+            const int b3 = (int)(t01 & 0xFFFF) + (int)(t01 >> 16) + (int)(t23 & 0xFFFF) + (int)(e23 >> 16);
+            const int n_step = b3 - (int)(e23 >> 16) + (int)(t23 >> 16);
             const uint16_t* arow = A + (int64_t)row * lda;
-            for (uint32_t mm = ob; mm != 0; mm &= mm - 1) {
-                const int bit = __ffs(mm) - 1;
-                const int j = bit >> 3;
-                const int col = (step * 128 + 32 * j + lane) * 8 + (bit & 7);
-                const int idx = (j == 0 ? b0 : j == 1 ? b1 : j == 2 ? b2 : b3) +
-                                __popc(ob & ((1u << bit) - 1u) & (0xFFu << (8 * j)));
+            // entry of rank row_rank + q (step column c): dA value and staging
+            auto emit = [&](int q, int c) {
+                const int col = step * 1024 + c;
+                const int idx = row_rank + q;
                 const float a = __uint_as_float((uint32_t)__ldg(arow + col) << 16);
                 const double d = (double)a - (double)copysignf(T, a);
                 if (idx < row_slots) {
@@ -983,8 +982,31 @@ __device__ __forceinline__ void clamp_rows_bf16(const uint16_t* __restrict__ A, 
                         flag_status(b.status, kStatusOverflow);
                     }
                 }
+            };
+            if (n_step <= kStepListCap) {
+                // each lane drops its outliers' step columns into the warp's
+                // list at their ranks (dense: 0 .. n_step - 1), then the
+                // warp emits the step's entries together, a lane each
+                for (uint32_t mm = ob; mm != 0; mm &= mm - 1) {
+                    const int bit = __ffs(mm) - 1;
+                    const int j = bit >> 3;
+                    const int q = (j == 0 ? b0 : j == 1 ? b1 : j == 2 ? b2 : b3) +
+                                  __popc(ob & ((1u << bit) - 1u) & (0xFFu << (8 * j)));
+                    olist[q] = (uint16_t)((32 * j + lane) * 8 + (bit & 7));
+                }
+                __syncwarp();
+                for (int q = lane; q < n_step; q += 32) emit(q, olist[q]);
+                __syncwarp();   // the list is rewritten by the next step
+            } else {
+                for (uint32_t mm = ob; mm != 0; mm &= mm - 1) {
+                    const int bit = __ffs(mm) - 1;
+                    const int j = bit >> 3;
+                    const int q = (j == 0 ? b0 : j == 1 ? b1 : j == 2 ? b2 : b3) +
+                                  __popc(ob & ((1u << bit) - 1u) & (0xFFu << (8 * j)));
+                    emit(q, (32 * j + lane) * 8 + (bit & 7));
+                }
             }
-            row_rank += (int)(t01 & 0xFFFF) + (int)(t01 >> 16) + (int)(t23 & 0xFFFF) + (int)(t23 >> 16);
+            row_rank += n_step;
         }
         // codes of the clamped row: an outlier x (|x| > T, so amax = T) has
         // |x r| >= |T r|, and T r is 6 within an ulp, so the saturating
@@ -1050,8 +1072,10 @@ clamp_quant_bf16_kernel(const uint16_t* __restrict__ A, int64_t lda, int M, int 
                         uint8_t* __restrict__ codes, float* __restrict__ scales, ActBuffers b,
                         int32_t* __restrict__ row_ptr, int64_t* __restrict__ nnz_out) {
     const int wpc = kQ3Threads / 32;
+    __shared__ uint16_t s_list[kQ3Threads / 32][kStepListCap];
     clamp_rows_bf16(A, lda, M, K, __ldcg(&ctr->T_key), rowmax, ctr, codes, scales, b,
-                    blockIdx.x * wpc + (threadIdx.x >> 5), gridDim.x * wpc, M);
+                    blockIdx.x * wpc + (threadIdx.x >> 5), gridDim.x * wpc, M, 1,
+                    s_list[threadIdx.x >> 5]);
     if (last_block_done(&ctr->done_clamp)) cta_scan_rowcnt<kQ3Threads>(b, M, row_ptr, nnz_out);
 }
 
@@ -1286,8 +1310,11 @@ act_fused_bf16_kernel(const uint16_t* __restrict__ A, int64_t lda, int M, int K,
     // rows' counts locally into rowpre
     const int rpc = (M + (int)gridDim.x - 1) / (int)gridDim.x;
     const int r0 = min(M, (int)blockIdx.x * rpc), r1 = min(M, r0 + rpc);
+    // (the band histogram's shared memory holds the warps' outlier lists now)
+    static_assert(kBandBins * 2 >= (kFusedThreads / 32) * kStepListCap, "lists fit in sh");
     clamp_rows_bf16(A, lda, M, K, __ldcg(&b.ctr->T_key), b.rowmax, b.ctr, codes, scales, b,
-                    r0 + (int)(threadIdx.x >> 5), wpc, r1, (K / 8 + 127) / 128);
+                    r0 + (int)(threadIdx.x >> 5), wpc, r1, (K / 8 + 127) / 128,
+                    reinterpret_cast<uint16_t*>(sh) + (threadIdx.x >> 5) * kStepListCap);
     uint32_t* cta_off = b.hist1 + kCtaTotOffset;   // per-CTA totals, then offsets
     __syncthreads();
     cta_local_scan<kFusedThreads>(b.rowcnt + r0, r1 - r0, b.rowpre + r0, cta_off + blockIdx.x);
