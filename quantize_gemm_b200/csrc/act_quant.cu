@@ -846,11 +846,11 @@ clamp_quant_kernel(const void* __restrict__ A, int64_t lda, int M, int K,
 // The same pass for bf16 A with codes out, written for instruction count: the
 // bf16 pairs stay packed until they are scaled.  Per 32-bit word (two bf16):
 // the outlier test is a SWAR compare of the two magnitudes with T (one add,
-// one and), the clamp is a bit select (only in warps that hold an outlier),
-// the scale one packed fp32x2 multiply (IEEE round to nearest, as
-// __fmul_rn), the encode one cvt.  The next step's loads are issued before
-// this step's work.  Warps walk rows grid-stride; a step covers 1024 columns
-// of one row.
+// one and), the scale one packed fp32x2 multiply (IEEE round to nearest, as
+// __fmul_rn), the encode one cvt; the clamp itself costs nothing, because the
+// saturating conversion already maps an outlier to the code of +-T (see the
+// encode below).  The next step's loads are issued before this step's work.
+// Warps walk rows grid-stride; a step covers 1024 columns of one row.
 constexpr int kQ3Threads = 256;
 constexpr int kStepListCap = 512;   // outliers per 1024-column step held in a warp's list
 #ifndef QG_CLAMP_MIN_BLOCKS
@@ -861,7 +861,9 @@ constexpr int kQ3MinBlocks = QG_CLAMP_MIN_BLOCKS;   // resident CTAs per SM (reg
 
 // The clamp / quantize pass over rows first, first + stride, ... (< row_end)
 // of this warp; M is the matrix height (the overflow slots follow M row
-// regions).
+// regions).  olist: this warp's kStepListCap-entry list in shared memory, in
+// which a step's outliers are placed at their ranks before the warp writes
+// their entries together.
 __device__ __forceinline__ void clamp_rows_bf16(const uint16_t* __restrict__ A, int64_t lda, int M,
                                                 int K, uint32_t T_key,
                                                 const uint32_t* __restrict__ rowmax,
