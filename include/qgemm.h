@@ -168,7 +168,8 @@ qg_status qg_quantize_cols(const void* W, qg_dtype dtype, int64_t K, int64_t N, 
  *     it is stale, so do not call this entry point again after a reset.
  *   - For either dtype it runs the two-pass kernels (column maxima, then the
  *     codes) rather than the single cooperative bf16 kernel of
- *     qg_quantize_cols: same results, somewhat slower on bf16 weights.
+ *     qg_quantize_cols: same results, 12-22 % slower on bf16 weights
+ *     (measured on a B200 from 2048 x 5504 to 4096 x 22016).
  *   - Every call on a GPU uses that GPU's one array and zeroes what it needs
  *     at the start; it keeps the last call's contents in between.  Calls
  *     whose executions overlap on the same GPU (for example on two streams)
