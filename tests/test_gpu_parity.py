@@ -187,6 +187,12 @@ def _act_inputs(name):
     if name == "bf16_ragged_k1056":
         return make_matrix((300, 1056), ("student_t", 4), seed=11, device="cuda",
                            dtype=torch.bfloat16), 0.99
+    if name == "many_outliers_k2048":
+        # alpha 0.3: about 70 % of the entries are clamped, so a 1024-column
+        # step holds more outliers than a warp's list (512) and the clamp
+        # pass stages them from its per-lane loop instead
+        return make_matrix((64, 2048), ("student_t", 4), seed=13, device="cuda",
+                           dtype=torch.bfloat16), 0.3
     if name in ("band_miss_low", "band_miss_high"):
         # M=512, K=256: the bf16 threshold pass samples rows 0, 8, 16, ...
         # only.  Here those rows are all zeros (every other row zero), or
@@ -204,7 +210,8 @@ def _act_inputs(name):
 
 ACT_CASES = ["tiny", "llama1.3b_attn_m512", "llama7b_down_m256", "llama13b_qkv_m128",
              "ragged_k1056_fp32", "no_clamp", "clamp_almost_all", "ties_at_T", "single_row",
-             "fp32_heavy_tail", "bf16_ragged_k1056", "band_miss_low", "band_miss_high"]
+             "fp32_heavy_tail", "bf16_ragged_k1056", "band_miss_low", "band_miss_high",
+             "many_outliers_k2048"]
 
 
 def _check_act(qg, A, alpha, codes, scales, csr, T, exp):
