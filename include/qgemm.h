@@ -46,6 +46,10 @@
  *     bounded wait that timed out, an internal capacity overflow) set bits in
  *     the status word; qg_sync_status() synchronises the stream, returns the
  *     condition and clears it.
+ *   - Environment: QGEMM_NO_COOPERATIVE=1 (read when the library first sets up
+ *     a device) makes it use the multi-kernel sequences of the bf16 activation
+ *     and column quantizers instead of their single cooperative kernels: the
+ *     same results, slower; meant for testing those paths.
  *   - Inputs must be finite.  Calls that scan all of A for the threshold
  *     (quantize_act, clamp_compensate, fp4_linear) report NaN/Inf as
  *     QG_ERR_NONFINITE; the other calls give unspecified codes for them.

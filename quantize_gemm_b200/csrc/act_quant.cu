@@ -1414,6 +1414,7 @@ cudaError_t act_setup() {
     if (e != cudaSuccess) return e;
     e = cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev);
     if (e != cudaSuccess) return e;
+    if (cooperative_disabled()) coop = 0;
     if (coop) {
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, act_fused_bf16_kernel, kFusedThreads, 0);
         if (e != cudaSuccess) return e;

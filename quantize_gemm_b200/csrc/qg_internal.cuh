@@ -7,6 +7,8 @@
 #include <math.h>
 #include <stdint.h>
 
+#include <stdlib.h>
+
 #include <algorithm>
 
 #include "../../include/qgemm.h"
@@ -397,6 +399,15 @@ struct ActBuffers {
 // the SpMM writes Y and the GEMM adds in place (alpha 0.999: 4 per row, the
 // other order is 9 % slower there).
 constexpr int64_t kAddOrderEntriesPerRow = 16;
+
+// QGEMM_NO_COOPERATIVE=1 in the environment (read when a device is first set
+// up) makes the library treat the device as having no cooperative launch, so
+// the bf16 activation and column quantizers take their multi-kernel
+// sequences: the same results by other kernels, for testing those paths.
+inline bool cooperative_disabled() {
+    const char* v = getenv("QGEMM_NO_COOPERATIVE");
+    return v != nullptr && v[0] == '1';
+}
 
 // Host-side argument checks shared by the C entry points.
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }

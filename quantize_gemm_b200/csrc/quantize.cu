@@ -456,6 +456,7 @@ cudaError_t cols_setup() {
     if (e != cudaSuccess) return e;
     e = cudaDeviceGetAttribute(&coop, cudaDevAttrCooperativeLaunch, dev);
     if (e != cudaSuccess) return e;
+    if (cooperative_disabled()) coop = 0;
     if (coop) {
         e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, quantize_cols_fused_bf16_kernel,
                                                           kColsFusedThreads, 0);
