@@ -306,13 +306,17 @@ quantize_cols_kernel(const void* __restrict__ W, int64_t ldw, int K, int N,
 //   phase 1  unit (split s, 256-column block): the max key of each column over
 //            the split's rows -> colpart[s][n] (no atomics, nothing to zero)
 //   barrier
-//   phase 2  tiles of 32 rows x 256 columns, a CTA's tiles consecutive in
-//            (column block, row tile) order: the column scales from the
-//            partial maxima (once per column block), the tile through shared
-//            memory (W is read a second time, mostly from L2), one thread
-//            per column encodes 32 values into 16 output bytes.
+//   phase 2  tiles of 32 rows x 64 columns, one warp each and a warp's tiles
+//            consecutive in (column group, row tile) order: the column scales
+//            from the partial maxima (once per column group), the tile
+//            through the warp's own shared memory (W is read a second time,
+//            partly from L2; only __syncwarp, so warps never wait for one
+//            another), each lane encodes two adjacent columns (32 values
+//            each into 16 output bytes); the next tile's loads are in flight
+//            while the current one is encoded.
 constexpr int kColsFusedThreads = 256;
 constexpr int kColsMaxSplits = 32;
+constexpr int kColsWarpTileN = 64;      // columns of a phase-2 warp tile
 
 __global__ void __launch_bounds__(kColsFusedThreads)
 quantize_cols_fused_bf16_kernel(const uint16_t* __restrict__ W, int64_t ldw, int K, int N,
@@ -320,8 +324,7 @@ quantize_cols_fused_bf16_kernel(const uint16_t* __restrict__ W, int64_t ldw, int
                                 uint8_t* __restrict__ codesT, float* __restrict__ scales,
                                 GridSync* __restrict__ gsync, uint32_t* __restrict__ status) {
     __shared__ uint32_t red[8][256];
-    __shared__ __align__(16) uint16_t tile[kColTileK][kColTileN];
-    __shared__ float s_r[kColTileN];
+    __shared__ __align__(16) uint16_t wtile[kColsFusedThreads / 32][kColTileK][kColsWarpTileN];
     const int t = threadIdx.x, lane = t & 31, warp = t >> 5;
     const int cblocks = (N + 255) / 256;
     const bool ld_vec = (ldw & 7) == 0;
@@ -384,66 +387,82 @@ quantize_cols_fused_bf16_kernel(const uint16_t* __restrict__ W, int64_t ldw, int
 
     // phase 2
     const int ktiles = K / kColTileK;
-    const int total = cblocks * ktiles;
-    const int per = (total + gridDim.x - 1) / gridDim.x;
-    const int t0 = blockIdx.x * per, t1 = min(total, t0 + per);
-    int cur_cb = -1;
-    // this thread's part of a tile: rows warp + 8 u (u < 4), columns lane * 8 .. + 7
-    auto load_tile = [&](int ti, uint4 (&v)[4]) {
-        const int cb = ti / ktiles, kt = ti - cb * ktiles;
-        const int nc = cb * kColTileN + lane * 8;
+    const int cgroups = (N + kColsWarpTileN - 1) / kColsWarpTileN;
+    const int total = cgroups * ktiles;                 // units (column group, row tile)
+    const int gw = blockIdx.x * (kColsFusedThreads / 32) + warp;
+    const int nw = gridDim.x * (kColsFusedThreads / 32);
+    const int per = (total + nw - 1) / nw;
+    const int u0 = min(total, gw * per), u1 = min(total, u0 + per);
+    uint16_t (*tl)[kColsWarpTileN] = wtile[warp];
+    // this lane's part of a unit: rows lane / 8 + 4 i (i < 8), columns
+    // 8 (lane % 8) .. + 7 of the group
+    auto load_unit = [&](int u, uint4 (&v)[8]) {
+        const int cg = u / ktiles, kt = u - cg * ktiles;
+        const int nc = cg * kColsWarpTileN + (lane & 7) * 8;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-            const int k = kt * kColTileK + warp + 8 * u;
-            v[u] = make_uint4(0u, 0u, 0u, 0u);
+        for (int i = 0; i < 8; ++i) {
+            const int k = kt * kColTileK + (lane >> 3) + 4 * i;
+            v[i] = make_uint4(0u, 0u, 0u, 0u);
             if (ld_vec && nc + 8 <= N) {
-                v[u] = __ldg(reinterpret_cast<const uint4*>(W + (int64_t)k * ldw + nc));
+                v[i] = __ldg(reinterpret_cast<const uint4*>(W + (int64_t)k * ldw + nc));
             } else if (nc < N) {
                 uint16_t h[8];
 #pragma unroll
                 for (int e = 0; e < 8; ++e) h[e] = (nc + e < N) ? W[(int64_t)k * ldw + nc + e] : (uint16_t)0;
-                v[u] = make_uint4(h[0] | ((uint32_t)h[1] << 16), h[2] | ((uint32_t)h[3] << 16),
+                v[i] = make_uint4(h[0] | ((uint32_t)h[1] << 16), h[2] | ((uint32_t)h[3] << 16),
                                   h[4] | ((uint32_t)h[5] << 16), h[6] | ((uint32_t)h[7] << 16));
             }
         }
     };
-    uint4 nxt[4];
-    if (t0 < t1) load_tile(t0, nxt);
-    for (int ti = t0; ti < t1; ++ti) {
-        const int cb = ti / ktiles, kt = ti - cb * ktiles;
-        const int n_base = cb * kColTileN, k_base = kt * kColTileK;
-        __syncthreads();   // the previous tile's reads of tile / s_r are done
-        if (cb != cur_cb) {
-            const int n = n_base + t;
-            float r = 0.0f, sc = 0.0f;
-            if (n < N) {
-                uint32_t key = 0;
-                for (int sp = 0; sp < splits; ++sp) key = max(key, __ldcg(colpart + (int64_t)sp * N + n));
-                scale_factors(__uint_as_float(key << 16), r, sc);
-                if (kt == 0) scales[n] = sc;
+    uint4 nxt[8];
+    if (u0 < u1) load_unit(u0, nxt);
+    int cur_cg = -1;
+    float r0 = 0.0f, r1 = 0.0f;
+    for (int u = u0; u < u1; ++u) {
+        const int cg = u / ktiles, kt = u - cg * ktiles;
+        __syncwarp();   // the previous unit's reads of the tile are done
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+            *reinterpret_cast<uint4*>(&tl[(lane >> 3) + 4 * i][(lane & 7) * 8]) = nxt[i];
+        __syncwarp();
+        if (u + 1 < u1) load_unit(u + 1, nxt);   // in flight while this unit is encoded
+        const int n0 = cg * kColsWarpTileN + 2 * lane;   // this lane's columns n0, n0 + 1
+        if (cg != cur_cg) {
+            uint32_t key0 = 0, key1 = 0;
+            for (int sp = 0; sp < splits; ++sp) {
+                if (n0 < N) key0 = max(key0, __ldcg(colpart + (int64_t)sp * N + n0));
+                if (n0 + 1 < N) key1 = max(key1, __ldcg(colpart + (int64_t)sp * N + n0 + 1));
             }
-            s_r[t] = r;
-            cur_cb = cb;
-        }
-#pragma unroll
-        for (int u = 0; u < 4; ++u) *reinterpret_cast<uint4*>(&tile[warp + 8 * u][lane * 8]) = nxt[u];
-        __syncthreads();
-        if (ti + 1 < t1) load_tile(ti + 1, nxt);   // in flight while this tile is encoded
-        const int n = n_base + t;
-        if (n < N) {
-            const float r = s_r[t];
-            uint32_t packed[4];
-#pragma unroll
-            for (int q = 0; q < 4; ++q) {
-                float y[8];
-#pragma unroll
-                for (int e = 0; e < 8; ++e)
-                    y[e] = __fmul_rn(__uint_as_float((uint32_t)tile[q * 8 + e][t] << 16), r);
-                packed[q] = e2m1x8(y);
+            float sc0, sc1;
+            scale_factors(__uint_as_float(key0 << 16), r0, sc0);
+            scale_factors(__uint_as_float(key1 << 16), r1, sc1);
+            if (kt == 0) {
+                if (n0 < N) scales[n0] = sc0;
+                if (n0 + 1 < N) scales[n0 + 1] = sc1;
             }
-            uint4* dst = reinterpret_cast<uint4*>(codesT + (int64_t)n * (K / 2) + k_base / 2);
-            *dst = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+            cur_cg = cg;
         }
+        // column n0 is the low bf16 of each 32-bit word of the lane's pair, n0 + 1 the high one
+        const uint32_t* tw = reinterpret_cast<const uint32_t*>(&tl[0][0]) + lane;
+        uint32_t p0[4], p1[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+            float y0[8], y1[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const uint32_t w = tw[(q * 8 + e) * (kColsWarpTileN / 2)];
+                y0[e] = __fmul_rn(__uint_as_float(w << 16), r0);
+                y1[e] = __fmul_rn(__uint_as_float(w & 0xFFFF0000u), r1);
+            }
+            p0[q] = e2m1x8(y0);
+            p1[q] = e2m1x8(y1);
+        }
+        if (n0 < N)
+            *reinterpret_cast<uint4*>(codesT + (int64_t)n0 * (K / 2) + kt * (kColTileK / 2)) =
+                make_uint4(p0[0], p0[1], p0[2], p0[3]);
+        if (n0 + 1 < N)
+            *reinterpret_cast<uint4*>(codesT + (int64_t)(n0 + 1) * (K / 2) + kt * (kColTileK / 2)) =
+                make_uint4(p1[0], p1[1], p1[2], p1[3]);
     }
 }
 
