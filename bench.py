@@ -406,6 +406,9 @@ def _kernel_rows(layers, per_kernel, steps, peaks, sm_mhz, n_sm):
             bound, unit, peak = "hbm", "GB/s", peaks["hbm_gbs"]
             extra = {}
         achieved = algo / t if kms > 0 else 0.0
+        if bound == "hbm" and k != "fp4_gemm":
+            # the quantizers' stated target is a fraction of the nominal 8 TB/s
+            extra["frac_of_8tbs_nominal"] = round(achieved / 8000.0, 4)
         rows[k] = {"bound": bound, "achieved": round(achieved, 2), "peak": round(peak, 1),
                    "unit": unit, "frac": round(achieved / peak, 4), "ms_per_step": round(kms, 4),
                    **extra}
