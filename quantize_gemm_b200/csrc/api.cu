@@ -356,11 +356,26 @@ qg_status qg_fp4_linear(const void* A, qg_dtype dtype, int64_t M, int64_t K,
         return cuda_status(launch_fp4_gemm(codes, scales, codesWT, sW, M, N, K, Yf, Y, QG_F32,
                                            nullptr, status, stream));
     }
-    // bf16 Y has no room for the fp32 compensation: the compensated GEMM
-    // computes it inside the kernel instead
-    return cuda_status(launch_fp4_gemm_corr(codes, scales, codesWT, sW, M, N, K, &csr, W, dtype, N,
-                                            at<float>(ws, L.corr_scratch), Y, y_dtype, status,
-                                            stream));
+    // bf16 Y has no room for the fp32 compensation, so the rows go in chunks
+    // of R: the SpMM writes a chunk's dA . W into an fp32 scratch of R x N (at
+    // most kLinearScratchMaxBytes, much of it still in L2 when it is read) and
+    // the GEMM reads it as C while it writes the chunk's Y.  Every element is
+    // bf16(acc s_i t_j + c_ij) with c_ij its row's fp32 FMA chain, as when the
+    // compensated GEMM computes c inside the kernel (qg_fp4_gemm_compensated),
+    // which is 1.3-3.8x slower at the 7B block's shapes.
+    const int64_t R = linear_chunk_rows(M, N);
+    float* scratch = at<float>(ws, L.linear_scratch);
+    for (int64_t r0 = 0; r0 < M; r0 += R) {
+        const int64_t rows = std::min<int64_t>(R, M - r0);
+        qg_csr chunk = csr;
+        chunk.row_ptr = csr.row_ptr + r0;   // entries are indexed absolutely
+        launch_spmm(&chunk, rows, W, dtype, N, N, scratch, status, stream);
+        if ((e = cudaGetLastError()) != cudaSuccess) return QG_ERR_CUDA;
+        e = launch_fp4_gemm(codes + r0 * (K / 2), scales + r0, codesWT, sW, rows, N, K, scratch,
+                            static_cast<uint16_t*>(Y) + r0 * N, y_dtype, nullptr, status, stream);
+        if (e != cudaSuccess) return QG_ERR_CUDA;
+    }
+    return QG_OK;
 }
 
 qg_status qg_fp4_gemm_compensated(const uint8_t* codesA, const float* sA, const uint8_t* codesWT,

@@ -80,6 +80,17 @@ static_assert(kGridSyncOffset + sizeof(GridSync) <= 2 * kAlign, "inside the zero
 // per CTA, for up to 160 CTAs (36.7 MB; it stays in L2).
 constexpr size_t kCorrScratchBytes = (size_t)160 * 2 * 128 * 224 * 4;
 
+// The layer with bf16 Y goes through its rows in chunks: the compensation of
+// a chunk is written into an fp32 scratch of R rows x N (at most this many
+// bytes, R a multiple of the GEMM's 256-row pair tile, at least 256 rows or
+// all of M) and the GEMM reads it back while it writes that chunk of Y.
+constexpr size_t kLinearScratchMaxBytes = (size_t)128 << 20;
+inline int64_t linear_chunk_rows(int64_t M, int64_t N) {
+    int64_t r = (int64_t)(kLinearScratchMaxBytes / ((size_t)N * 4)) / 256 * 256;
+    if (r < 256) r = 256;
+    return r < M ? r : M;
+}
+
 struct WsLayout {
     size_t gsync = 0;
     size_t rowpre = 0;
@@ -87,7 +98,7 @@ struct WsLayout {
     size_t status = 0, counters = 0, hist1 = 0, hist2 = 0, rowmax = 0, rowcnt = 0;
     size_t st_row = 0, st_rank = 0, st_col = 0, st_val = 0, colmax = 0;
     size_t act_codes = 0, act_scales = 0, csr_row_ptr = 0, csr_col = 0, csr_val = 0,
-           csr_nnz = 0, thr = 0, corr_scratch = 0;
+           csr_nnz = 0, thr = 0, corr_scratch = 0, linear_scratch = 0;
     size_t total = 0;
     int64_t cap = 0;
     int64_t row_slots = 0;
@@ -160,9 +171,11 @@ inline WsLayout ws_layout(qg_op op, int64_t M, int64_t K, int64_t N, qg_dtype dt
         L.csr_nnz = take(sizeof(int64_t));
         L.thr = take(sizeof(float));
     }
-    // the compensated GEMM's scratch slots (the layer call and the GEMM alone)
-    if (op == QG_OP_FP4_LINEAR || op == QG_OP_FP4_GEMM_COMPENSATED)
-        L.corr_scratch = take(kCorrScratchBytes);
+    // the compensated GEMM's scratch slots
+    if (op == QG_OP_FP4_GEMM_COMPENSATED) L.corr_scratch = take(kCorrScratchBytes);
+    // the layer's chunk of fp32 compensation rows (bf16 Y)
+    if (op == QG_OP_FP4_LINEAR)
+        L.linear_scratch = take((size_t)linear_chunk_rows(M, N) * (size_t)N * sizeof(float));
     L.total = off;
     return L;
 }

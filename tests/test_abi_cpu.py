@@ -57,19 +57,33 @@ def test_workspace_sizes(qg):
                                  (4096, 2048, 5504, 1, 0.99), (16384, 11008, 4096, 1, 0.999)):
             s = qg.qg_workspace_size(op, M, K, N, dt, a)
             assert s >= 256 and s % 256 == 0
-    # the layer's workspace holds the activation codes, the CSR and the fixed
-    # scratch slots of the compensated GEMM, but no M x N correction: it does
-    # not grow with N
-    M, K, N = 4096, 2048, 5504
-    s = qg.qg_workspace_size(qg.QG_OP_FP4_LINEAR, M, K, N, qg.QG_BF16, 0.99)
-    cap = qg.qg_nnz_capacity(M * K, 0.99)
+    # the layer's workspace holds the activation codes, the CSR and one chunk
+    # of fp32 compensation rows for bf16 Y: R rows x N with R a multiple of
+    # 256 and R x N x 4 at most 128 MiB (or all of M when fewer rows), so it
+    # never grows past that bound with M or N
+    cap_bytes = 128 << 20
+
+    def chunk_rows(M, N):
+        r = max(256, cap_bytes // (4 * N) // 256 * 256)
+        return min(r, M)
+
+    for (M, K, N) in ((4096, 2048, 5504), (16384, 4096, 12288), (16384, 4096, 22016),
+                      (16384, 11008, 4096), (65536, 4096, 4096), (300, 512, 1000)):
+        cap = qg.qg_nnz_capacity(M * K, 0.99)
+        s = qg.qg_workspace_size(qg.QG_OP_FP4_LINEAR, M, K, N, qg.QG_BF16, 0.99)
+        R = chunk_rows(M, N)
+        assert R == M or (R % 256 == 0 and R * N * 4 <= cap_bytes)
+        assert s >= 4 * R * N + 12 * cap + M * K // 2
+        # every other part is the same as without the chunk
+        assert s - 4 * R * N < qg.qg_workspace_size(qg.QG_OP_QUANTIZE_ACT, M, K, 1, qg.QG_BF16, 0.99) \
+            + M * K // 2 + 4 * M + 4 * (M + 1) + 12 * cap + 8192
+    # at the 7B block's size the chunk is a fraction of M x N
+    assert chunk_rows(16384, 12288) * 4 <= 16384
     scratch = 160 * 2 * 128 * 224 * 4
-    assert s >= scratch + 12 * cap + M * K // 2
-    assert s == qg.qg_workspace_size(qg.QG_OP_FP4_LINEAR, M, K, 4 * N, qg.QG_BF16, 0.99)
-    assert s < 4 * M * N
-    g = qg.qg_workspace_size(qg.QG_OP_FP4_GEMM_COMPENSATED, M, K, N, qg.QG_F32, 1.0)
+    g = qg.qg_workspace_size(qg.QG_OP_FP4_GEMM_COMPENSATED, 4096, 2048, 5504, qg.QG_F32, 1.0)
     assert scratch <= g < scratch + 4096
     # staging grows as alpha falls
+    M, K = 4096, 2048
     a = qg.qg_workspace_size(qg.QG_OP_QUANTIZE_ACT, M, K, 1, qg.QG_BF16, 0.999)
     b = qg.qg_workspace_size(qg.QG_OP_QUANTIZE_ACT, M, K, 1, qg.QG_BF16, 0.99)
     assert b > a

@@ -492,6 +492,44 @@ def test_fp4_gemm_compensated(qg, case, N, wdtype, ydtype):
         assert np.all(np.abs(_np(Y.float()).astype(np.float64) - Yo) <= bf16_ulp(Yo) + 1e-6 * rms)
 
 
+@pytest.mark.parametrize("M,K,N,alpha", [(700, 256, 65536, 0.99), (1000, 512, 40000, 0.999),
+                                         (300, 1056, 8192, 0.99)])
+def test_fp4_linear_bf16_chunks(qg, M, K, N, alpha):
+    """The layer with bf16 Y goes through its rows in chunks (the SpMM writes a
+    chunk's compensation into an fp32 scratch, the GEMM reads it while writing
+    the chunk's Y).  With N this wide the chunks are 512, 768 or all rows, the
+    last one ragged: Y equals, bit for bit, the compensated GEMM's single
+    kernel on the same codes and CSR, and the oracle within a bf16 ulp on
+    sampled rows."""
+    A = make_matrix((M, K), ("student_t", 3), seed=M + K, device="cuda", dtype=torch.bfloat16)
+    W = make_matrix((K, N), seed=N, device="cuda", dtype=torch.bfloat16, scale=0.02)
+    codesT, t = qg.quantize_cols(W)
+    ws = qg.Workspace(qg.QG_OP_FP4_LINEAR, M, K, N, qg.QG_BF16, alpha)
+    Y = qg.fp4_linear(A, codesT, t, W, alpha, out_dtype=torch.bfloat16, ws=ws)
+    qg.check_status(ws, "layer")
+    # the layer's own codes and CSR, from its workspace
+    st, off = qg.qg_fp4_linear_parts(M, K, N, qg.QG_BF16, alpha)
+    assert st == qg.QG_OK
+    buf = ws.buf
+    codes = buf[off[0]:off[0] + M * (K // 2)].view(M, K // 2)
+    scales = buf[off[1]:off[1] + 4 * M].view(torch.float32)
+    cap = max(qg.qg_nnz_capacity(M * K, alpha), 1)
+    csr = qg.CSR(buf[off[2]:off[2] + 4 * (M + 1)].view(torch.int32),
+                 buf[off[3]:off[3] + 4 * cap].view(torch.int32),
+                 buf[off[4]:off[4] + 8 * cap].view(torch.float64),
+                 buf[off[5]:off[5] + 8].view(torch.int64), cap)
+    wsc = qg.Workspace(qg.QG_OP_FP4_GEMM_COMPENSATED, M, K, N, qg.QG_F32)
+    Y2 = qg.fp4_gemm_compensated(codes, scales, codesT, t, K, csr, W, out_dtype=torch.bfloat16,
+                                 ws=wsc)
+    qg.check_status(wsc, "compensated")
+    assert torch.equal(Y, Y2)
+    rows = np.arange(0, M, 97)
+    Yo, _ = _linear_oracle(A, W, alpha, rows=rows)
+    rms = np.sqrt(np.mean(Yo ** 2))
+    got = _np(Y.float())[rows].astype(np.float64)
+    assert np.all(np.abs(got - Yo) <= bf16_ulp(Yo) + 1e-6 * rms)
+
+
 # ------------------------------------------------------------------ the layer
 def _linear_oracle(A, W, alpha, rows=None):
     act = oracle.quantize_act(A.cpu(), alpha)
