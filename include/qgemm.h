@@ -258,15 +258,21 @@ qg_status qg_fp4_gemm_compensated(const uint8_t* codesA, const float* sA, const 
  *           that sub-tile of Y); or, when alpha leaves at least 16 clamped
  *           entries per row possible (n - ceil(alpha n) >= 16 M), the other
  *           order: qg_fp4_gemm(..., C = NULL, Y), then qg_spmm_accumulate;
- *   bf16 Y: qg_fp4_gemm_compensated (the compensation inside the GEMM).
- * Both give Y_ij = fp32(acc_ij * sA_i * sW_j) + C_ij with C the fp32 FMA chain
+ *   bf16 Y: the rows in chunks of R (a multiple of 256, R x N x 4 <= 128
+ *           MiB, or all of M): qg_spmm_correction of the chunk into an fp32
+ *           scratch of R x N in the workspace, then qg_fp4_gemm(..., C =
+ *           scratch, the chunk of Y) -- the same bytes as
+ *           qg_fp4_gemm_compensated, which computes the compensation inside
+ *           the GEMM kernel but runs 1.3-3.8x slower at the 7B block's shapes.
+ * All give Y_ij = fp32(acc_ij * sA_i * sW_j) + C_ij with C the fp32 FMA chain
  * of row i's entries (rounded to bf16 last for bf16 Y).  codesWT / sW come
  * from qg_quantize_cols(W); W is the unquantized weight used by the
  * compensation, K x N row-major and contiguous, stored in the SAME dtype as A
  * (`dtype` describes both; the call has no separate weight dtype, so a weight
  * in the other dtype is read wrongly without an error).  The activation
- * codes, dA and the compensated GEMM's scratch slots live in the workspace
- * (qg_workspace_size(QG_OP_FP4_LINEAR, ...)); no M x N buffer besides Y. */
+ * codes, dA and the bf16 chunk scratch live in the workspace
+ * (qg_workspace_size(QG_OP_FP4_LINEAR, ...)); besides Y, no buffer grows past
+ * the chunk's 128 MiB with M. */
 qg_status qg_fp4_linear(const void* A, qg_dtype dtype, int64_t M, int64_t K,
                         const uint8_t* codesWT, const float* sW, const void* W, int64_t N,
                         double alpha, void* Y, qg_dtype y_dtype, void* ws, size_t ws_bytes,
