@@ -966,10 +966,12 @@ def mx_sweep(device, workload, reps=20, warm=5):
 
 def compensated_sweep(device, workload, alpha=None, reps=10, warm=3):
     """The compensated GEMM (dA . W computed inside the GEMM kernel) beside the
-    two-kernel form the layer uses for fp32 Y (the SpMM writing the
-    compensation into Y, then the GEMM adding the product in place), on every
-    linear of a workload; median of `reps` CUDA-event timings, L2 flushed
-    before each.  One JSON line per linear."""
+    two-kernel form (the SpMM writing the compensation into Y, then the GEMM
+    adding the product in place), and the whole layer call (qg_fp4_linear,
+    activation quantizer included) with fp32 Y and with bf16 Y (row chunks
+    through the layer's fp32 scratch), on every linear of a workload; median
+    of `reps` CUDA-event timings, L2 flushed before each.  One JSON line per
+    linear."""
     import quantize_gemm_b200 as qg
     from workloads import WORKLOADS, make_layer_inputs
     wl = WORKLOADS[workload]
@@ -1005,17 +1007,27 @@ def compensated_sweep(device, workload, alpha=None, reps=10, warm=3):
                                                           ws_c))
         t_spmm = timed(lambda: qg.qg_spmm_correction(csr, M, W, Y, ws_s))
         t_gemm = timed(lambda: qg.qg_fp4_gemm(codes, s, codesT, t, M, N, K, Y, Y, None, ws_g))
-        for ws in (ws_c, ws_s, ws_g):
+        Yb = torch.empty((M, N), dtype=torch.bfloat16, device=device)
+        ws_l = qg.Workspace(qg.QG_OP_FP4_LINEAR, M, K, N, qg._dt(A), alpha, device=device)
+        ws_a = qg.Workspace(qg.QG_OP_QUANTIZE_ACT, M, K, 1, qg._dt(A), alpha, device=device)
+        t_lf = timed(lambda: qg.qg_fp4_linear(A, codesT, t, W, alpha, Y, ws_l))
+        t_lb = timed(lambda: qg.qg_fp4_linear(A, codesT, t, W, alpha, Yb, ws_l))
+        t_act = timed(lambda: qg.quantize_act(A, alpha, ws=ws_a))
+        for ws in (ws_c, ws_s, ws_g, ws_l, ws_a):
             qg.check_status(ws, "compensated sweep")
         nnz = int(csr.nnz.item())
+        chunk = max(256, (128 << 20) // (4 * N) // 256 * 256)
         print(json.dumps({"sweep": "compensated", "workload": wl.name, "layer": layer.name,
                           "M": M, "K": K, "N": N, "alpha": alpha, "nnz": nnz,
                           "compensated_gemm_ms": round(t_comp, 4),
                           "spmm_ms": round(t_spmm, 4), "gemm_in_place_ms": round(t_gemm, 4),
                           "two_kernel_ms": round(t_spmm + t_gemm, 4),
                           "compensation_tflops_fused": round(2 * nnz * N / (t_comp * 1e-3) / 1e12, 2),
+                          "layer_fp32_y_ms": round(t_lf, 4), "layer_bf16_y_ms": round(t_lb, 4),
+                          "act_quantizer_ms": round(t_act, 4),
+                          "bf16_y_chunk_rows": min(chunk, M),
                           "l2": "flushed before each rep", "reps": reps}), flush=True)
-        del A, W, codes, codesT, Y, ws_c, ws_s, ws_g
+        del A, W, codes, codesT, Y, Yb, ws_c, ws_s, ws_g, ws_l, ws_a
         torch.cuda.empty_cache()
 
 
