@@ -181,7 +181,8 @@ def layer_order(qg, L):
     """The order of the layer's four calls, as qg_fp4_linear runs them for
     fp32 Y: with many clamped entries per row the GEMM writes Y and the SpMM
     adds the compensation into it; otherwise the SpMM writes the compensation
-    into Y and the GEMM adds its product in place."""
+    into Y and the GEMM adds its product into it (qg_fp4_gemm_accumulate; in
+    place through C = Y when N is not a multiple of 4)."""
     if qg.linear_adds_into_y(L.M, L.K, L.alpha):
         return ("quantize_cols", "quantize_act", "fp4_gemm", "spmm")
     return ("quantize_cols", "quantize_act", "spmm", "fp4_gemm")
@@ -207,9 +208,14 @@ def run_step(qg, layers, ev=None):
                 _chk(qg.qg_spmm_accumulate(L.csr, L.M, L.W, L.Y, L.ws_spmm), name)
             else:
                 _chk(qg.qg_spmm_correction(L.csr, L.M, L.W, L.Y, L.ws_spmm), name)
+        elif L.adds:
+            _chk(qg.qg_fp4_gemm(L.codes, L.s, L.codesT, L.t, L.M, L.N, L.K, None, L.Y, None,
+                                L.ws_gemm), name)
+        elif L.N % 4 == 0:
+            _chk(qg.qg_fp4_gemm_accumulate(L.codes, L.s, L.codesT, L.t, L.M, L.N, L.K, L.Y,
+                                           L.ws_gemm), name)
         else:
-            C = None if L.adds else L.Y
-            _chk(qg.qg_fp4_gemm(L.codes, L.s, L.codesT, L.t, L.M, L.N, L.K, C, L.Y, None,
+            _chk(qg.qg_fp4_gemm(L.codes, L.s, L.codesT, L.t, L.M, L.N, L.K, L.Y, L.Y, None,
                                 L.ws_gemm), name)
 
     for i, L in enumerate(layers):

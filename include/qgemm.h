@@ -229,6 +229,17 @@ qg_status qg_fp4_gemm(const uint8_t* codesA, const float* sA, const uint8_t* cod
                       void* Y, qg_dtype y_dtype, float* raw_acc, void* ws, size_t ws_bytes,
                       cudaStream_t stream);
 
+/* The FP4 GEMM's scaled product added into an existing fp32 output:
+ * Y_ij += acc_ij * sA_i * sW_j (the product rounded to fp32 as in qg_fp4_gemm,
+ * then added by the memory system's bulk reduction, fp32 round to nearest).
+ * Y: M x N fp32, contiguous, N a multiple of 4 (else
+ * QG_ERR_UNSUPPORTED_SHAPE).  With Y holding qg_spmm_correction's output,
+ * the result is the layer's Y.  Workspace and other arguments as
+ * qg_fp4_gemm. */
+qg_status qg_fp4_gemm_accumulate(const uint8_t* codesA, const float* sA, const uint8_t* codesWT,
+                                 const float* sW, int64_t M, int64_t N, int64_t K, float* Y,
+                                 void* ws, size_t ws_bytes, cudaStream_t stream);
+
 /* The compensated FP4 GEMM, the layer's product in one kernel:
  *   Y_ij = acc_ij * sA_i * sW_j + sum over the entries (i, k) of dA of
  *          dA_ik * W_kj
@@ -253,11 +264,12 @@ qg_status qg_fp4_gemm_compensated(const uint8_t* codesA, const float* sA, const 
 
 /* The whole layer into Y (M x N, fp32 or bf16): qg_quantize_act(A), then
  *   fp32 Y: qg_spmm_correction(dA, W) written into Y itself, then
- *           qg_fp4_gemm(..., C = Y, Y) adding the scaled FP4 product to it in
- *           place (the epilogue reads every sub-tile of C before it writes
- *           that sub-tile of Y); or, when alpha leaves at least 16 clamped
- *           entries per row possible (n - ceil(alpha n) >= 16 M), the other
- *           order: qg_fp4_gemm(..., C = NULL, Y), then qg_spmm_accumulate;
+ *           qg_fp4_gemm_accumulate adding the scaled FP4 product into it (for
+ *           N not a multiple of 4: qg_fp4_gemm(..., C = Y, Y) in place, the
+ *           epilogue reading every sub-tile of C before it writes that
+ *           sub-tile of Y); or, when alpha leaves at least 16 clamped entries
+ *           per row possible (n - ceil(alpha n) >= 16 M), the other order:
+ *           qg_fp4_gemm(..., C = NULL, Y), then qg_spmm_accumulate;
  *   bf16 Y: the rows in chunks of R (a multiple of 256, R x N x 4 <= 128
  *           MiB, or all of M): qg_spmm_correction of the chunk into an fp32
  *           scratch of R x N in the workspace, then qg_fp4_gemm(..., C =

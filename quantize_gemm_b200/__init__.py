@@ -44,6 +44,7 @@ EXPORTED = (
     "qg_quantize_cols_static", "qg_fp4_dgrad", "qg_fp4_wgrad", "qg_mx_scale_bytes",
     "qg_mx_quantize_rows", "qg_mx_quantize_cols", "qg_mx_gemm", "qg_fp4_mma_loop",
     "qg_fp4_linear_parts", "qg_fp4_gemm_compensated", "qg_spmm_accumulate",
+    "qg_fp4_gemm_accumulate",
 )
 
 
@@ -89,6 +90,7 @@ _sig("qg_spmm_accumulate", _INT,
      [ctypes.POINTER(_Csr), _I64, _P, _INT, _I64, _I64, _I64, _P, _P, _SZ, _P])
 _sig("qg_fp4_gemm", _INT,
      [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _INT, _P, _P, _SZ, _P])
+_sig("qg_fp4_gemm_accumulate", _INT, [_P, _P, _P, _P, _I64, _I64, _I64, _P, _P, _SZ, _P])
 _sig("qg_fp4_gemm_compensated", _INT,
      [_P, _P, _P, _P, _I64, _I64, _I64, ctypes.POINTER(_Csr), _P, _INT, _I64, _P, _INT, _P, _SZ,
       _P])
@@ -293,6 +295,12 @@ def qg_fp4_gemm_compensated(codesA, sA, codesWT, sW, M, N, K, csr: CSR, W, Y, ws
                                         ctypes.byref(c), _ptr(W), _dt(W),
                                         W.stride(0) if ldw is None else ldw, _ptr(Y), _dt(Y),
                                         ws.ptr, ws.nbytes, _stream(stream))
+
+
+def qg_fp4_gemm_accumulate(codesA, sA, codesWT, sW, M, N, K, Y, ws: Workspace,
+                           stream=None) -> int:
+    return _lib.qg_fp4_gemm_accumulate(_ptr(codesA), _ptr(sA), _ptr(codesWT), _ptr(sW), M, N, K,
+                                       _ptr(Y), ws.ptr, ws.nbytes, _stream(stream))
 
 
 def qg_fp4_linear(A, codesWT, sW, W, alpha, Y, ws: Workspace, stream=None) -> int:

@@ -306,6 +306,23 @@ qg_status qg_fp4_gemm(const uint8_t* codesA, const float* sA, const uint8_t* cod
                                        at<uint32_t>(ws, L.status), stream));
 }
 
+qg_status qg_fp4_gemm_accumulate(const uint8_t* codesA, const float* sA, const uint8_t* codesWT,
+                                 const float* sW, int64_t M, int64_t N, int64_t K, float* Y,
+                                 void* ws, size_t ws_bytes, cudaStream_t stream) {
+    qg_status st = check_mk(M, K);
+    if (st != QG_OK) return st;
+    if ((st = check_mk(N, K)) != QG_OK) return st;
+    if (!codesA || !codesWT || !sA || !sW || !Y || !aligned16(codesA) || !aligned16(codesWT) ||
+        !aligned16(sW) || !aligned16(Y))
+        return QG_ERR_INVALID_ARG;
+    if (N % 4 != 0) return QG_ERR_UNSUPPORTED_SHAPE;   // Y rows in whole 16-byte units for TMA
+    const WsLayout L = ws_layout(QG_OP_FP4_GEMM, M, K, N, QG_F32, 1.0);
+    if ((st = check_ws(ws, ws_bytes, L.total)) != QG_OK) return st;
+    if (ensure_device(nullptr) != cudaSuccess) return QG_ERR_CUDA;
+    return cuda_status(launch_fp4_gemm(codesA, sA, codesWT, sW, M, N, K, nullptr, Y, QG_F32,
+                                       nullptr, at<uint32_t>(ws, L.status), stream, true));
+}
+
 qg_status qg_fp4_linear(const void* A, qg_dtype dtype, int64_t M, int64_t K,
                         const uint8_t* codesWT, const float* sW, const void* W, int64_t N,
                         double alpha, void* Y, qg_dtype y_dtype, void* ws, size_t ws_bytes,
@@ -340,9 +357,10 @@ qg_status qg_fp4_linear(const void* A, qg_dtype dtype, int64_t M, int64_t K,
         // result: with many entries per row (at least kAddOrderEntriesPerRow
         // possible on average) the GEMM writes the scaled product and the SpMM
         // adds the compensation into Y, the SpMM's gathers hiding its reads of
-        // Y; otherwise the compensation is written into Y first and the GEMM's
-        // epilogue adds the product to it in place (it reads each 32 x 32
-        // sub-tile before it overwrites it; sub-tiles are disjoint)
+        // Y; otherwise the compensation is written into Y first and the GEMM
+        // adds its product into it through the memory system's bulk reduction
+        // (or, where the TMA epilogue cannot describe Y, reads each 32 x 32
+        // sub-tile of Y as C before it overwrites it in place)
         float* Yf = static_cast<float*>(Y);
         if (L.cap >= kAddOrderEntriesPerRow * M) {
             e = launch_fp4_gemm(codes, scales, codesWT, sW, M, N, K, nullptr, Y, QG_F32, nullptr,
@@ -353,6 +371,10 @@ qg_status qg_fp4_linear(const void* A, qg_dtype dtype, int64_t M, int64_t K,
         }
         launch_spmm(&csr, M, W, dtype, N, N, Yf, status, stream);
         if ((e = cudaGetLastError()) != cudaSuccess) return QG_ERR_CUDA;
+        e = launch_fp4_gemm(codes, scales, codesWT, sW, M, N, K, nullptr, Y, QG_F32, nullptr,
+                            status, stream, true);
+        if (e != cudaErrorInvalidValue) return cuda_status(e);
+        (void)cudaGetLastError();   // nothing was launched: add in place instead
         return cuda_status(launch_fp4_gemm(codes, scales, codesWT, sW, M, N, K, Yf, Y, QG_F32,
                                            nullptr, status, stream));
     }

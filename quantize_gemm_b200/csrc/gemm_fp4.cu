@@ -291,6 +291,17 @@ __device__ __forceinline__ void tma_store_2d(const CUtensorMap* map, const void*
                  "r"(x), "r"(y), "r"(smem_u32(src))
                  : "memory");
 }
+// The same box added into global memory: the memory system reads the
+// destination, adds the shared-memory tile element by element and writes it
+// back (fp32, round to nearest).
+__device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* map, const void* src, int x,
+                                                  int y) {
+    asm volatile(
+        "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%1, %2}], [%3];" ::"l"(
+            reinterpret_cast<uint64_t>(map)),
+        "r"(x), "r"(y), "r"(smem_u32(src))
+        : "memory");
+}
 // Plain bulk copy global -> this CTA's shared memory (16-byte aligned, size a
 // multiple of 16), completing on a barrier of this CTA.
 __device__ __forceinline__ void bulk_load(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
@@ -795,6 +806,7 @@ struct Params {
     int M, N, K;
     int y_bf16;
     int tma_epi;         // Y (and C) through TMA
+    int y_add;           // TMA epilogue, fp32 Y, no C: add the product into Y instead of storing it
     int unit_scales;     // MX: no row / column scales in the epilogue
     const uint8_t* sfA;  // MX: E8M0 scale atoms of A, [row block][k group]
     const uint8_t* sfB;  // MX: the same for W^T
@@ -1253,7 +1265,8 @@ fp4_gemm_kernel(const __grid_constant__ CUtensorMap tmap_a,
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) {
-                    tma_store_2d(&tmap_y, buf, col0, row0);
+                    if (p.y_add) tma_reduce_add_2d(&tmap_y, buf, col0, row0);
+                    else tma_store_2d(&tmap_y, buf, col0, row0);
                     bulk_commit();
                 }
                 if (use_c && g + EB - 1 < total) {
@@ -1498,7 +1511,7 @@ static_assert(kCorrScratchBytes ==
 cudaError_t launch_fp4_gemm(const uint8_t* codesA, const float* sA, const uint8_t* codesWT,
                             const float* sW, int64_t M, int64_t N, int64_t K, const float* C,
                             void* Y, qg_dtype y_dtype, float* raw_acc, uint32_t* status,
-                            cudaStream_t s) {
+                            cudaStream_t s, bool y_add) {
     using namespace gemm;
     Params p{};
     p.sA = sA;
@@ -1525,6 +1538,9 @@ cudaError_t launch_fp4_gemm(const uint8_t* codesA, const float* sA, const uint8_
                  ((size_t)N * ysz) % 16 == 0 && ((size_t)N * 4) % 16 == 0)
                     ? 1
                     : 0;
+    // adding into Y: through the TMA epilogue only, fp32 Y, no C
+    if (y_add && (!p.tma_epi || y_dtype != QG_F32 || C != nullptr)) return cudaErrorInvalidValue;
+    p.y_add = y_add ? 1 : 0;
     CUtensorMap ta, ty, tc;
     if (!encode_2d(&ta, CU_TENSOR_MAP_DATA_TYPE_UINT8, codesA, K / 2, M, K / 2, BK_BYTES, BM,
                    CU_TENSOR_MAP_SWIZZLE_128B))

@@ -454,7 +454,7 @@ cudaError_t launch_fp4_gemm_mx(const uint8_t* codesA, const uint8_t* sfA, const 
 cudaError_t launch_fp4_gemm(const uint8_t* codesA, const float* sA, const uint8_t* codesWT,
                             const float* sW, int64_t M, int64_t N, int64_t K, const float* C,
                             void* Y, qg_dtype y_dtype, float* raw_acc, uint32_t* status,
-                            cudaStream_t s);
+                            cudaStream_t s, bool y_add = false);
 cudaError_t launch_fp4_gemm_corr(const uint8_t* codesA, const float* sA, const uint8_t* codesWT,
                                  const float* sW, int64_t M, int64_t N, int64_t K,
                                  const qg_csr* dA, const void* W, qg_dtype w_dtype, int64_t ldw,

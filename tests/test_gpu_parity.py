@@ -428,6 +428,30 @@ def test_fp4_gemm_accumulates_in_place(qg, M, N, K):
     assert torch.equal(Y, want)
 
 
+@pytest.mark.parametrize("M,N,K", [(128, 256, 512), (300, 1000, 1024), (1024, 4096, 2048),
+                                   (2048, 12288, 4096)])
+def test_fp4_gemm_accumulate(qg, M, N, K):
+    """qg_fp4_gemm_accumulate: Y += the scaled product by the memory system's
+    bulk reduction, bit for bit the fp32 sum of Y and qg_fp4_gemm's own output
+    (single-CTA and pair tiles, ragged tiles); N not a multiple of 4 is
+    rejected before anything is enqueued."""
+    g = np.random.default_rng(M + 5 * N)
+    cA, cW = _rand_codes(M, K, 61 + M), _rand_codes(N, K, 62 + N)
+    sA = torch.from_numpy((g.random(M) * 0.1 + 1e-3).astype(np.float32)).cuda()
+    sW = torch.from_numpy((g.random(N) * 0.01 + 1e-4).astype(np.float32)).cuda()
+    Y0 = torch.from_numpy((g.standard_normal((M, N)) * 0.5).astype(np.float32)).cuda()
+    cA, cW = torch.from_numpy(cA).cuda(), torch.from_numpy(cW).cuda()
+    G = qg.fp4_gemm(cA, sA, cW, sW, K)
+    Y = Y0.clone()
+    ws = qg.Workspace(qg.QG_OP_FP4_GEMM, M, K, N, qg.QG_F32)
+    assert qg.qg_fp4_gemm_accumulate(cA, sA, cW, sW, M, N, K, Y, ws) == qg.QG_OK
+    qg.check_status(ws)
+    assert torch.equal(Y, Y0 + G)
+    bad = torch.zeros((M, N - 2), dtype=torch.float32, device="cuda")
+    assert qg.qg_fp4_gemm_accumulate(cA, sA, cW, sW, M, N - 2, K, bad, ws) == \
+        qg.QG_ERR_UNSUPPORTED_SHAPE
+
+
 def test_fp4_gemm_epilogue_bf16(qg):
     M, N, K = 300, 600, 1024
     g = np.random.default_rng(2)
