@@ -344,12 +344,11 @@ def _kernel_rows(layers, per_kernel, steps, peaks, sm_mhz, n_sm):
         kms = sum(per_kernel[k]) / steps
         t = kms * 1e-3
         if k == "fp4_gemm":
-            # the GEMM moves the FP4 codes, the scales, the fp32 compensation
-            # (read from Y) and Y (fp32, written in place); its bound is
+            # the GEMM moves the FP4 codes, the scales and Y: written only
+            # when it runs first, read and written (by the memory system's
+            # reduction, or in place) when the SpMM wrote Y first; its bound is
             # whichever of the tensor-core time and the HBM time is longer
             flops = sum(L.flops for L in layers)
-            # in place: the compensation read from Y and Y written; GEMM first:
-            # Y written only
             byts = sum(L.M * L.K / 2 + L.N * L.K / 2 + 4 * (L.M + L.N)
                        + (4 if L.adds else 8) * L.M * L.N for L in layers)
             t_tensor = flops / (fp4_peak * 1e12)
