@@ -267,8 +267,8 @@ qg_status qg_fp4_gemm_compensated(const uint8_t* codesA, const float* sA, const 
  *           qg_fp4_gemm_accumulate adding the scaled FP4 product into it (for
  *           N not a multiple of 4: qg_fp4_gemm(..., C = Y, Y) in place, the
  *           epilogue reading every sub-tile of C before it writes that
- *           sub-tile of Y); or, when alpha leaves at least 16 clamped entries
- *           per row possible (n - ceil(alpha n) >= 16 M), the other order:
+ *           sub-tile of Y); or, when alpha leaves at least 10 clamped entries
+ *           per row possible (n - ceil(alpha n) >= 10 M), the other order:
  *           qg_fp4_gemm(..., C = NULL, Y), then qg_spmm_accumulate;
  *   bf16 Y: the rows in chunks of R (a multiple of 256, R x N x 4 <= 128
  *           MiB, or all of M): qg_spmm_correction of the chunk into an fp32

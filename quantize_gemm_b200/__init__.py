@@ -271,7 +271,7 @@ def qg_spmm_accumulate(csr: CSR, M, W, Y, ws: Workspace, stream=None) -> int:
                                    _ptr(Y), ws.ptr, ws.nbytes, _stream(stream))
 
 
-ADD_ORDER_ENTRIES_PER_ROW = 16   # the layer's order switch (see qg_fp4_linear)
+ADD_ORDER_ENTRIES_PER_ROW = 10   # the layer's order switch (see qg_fp4_linear)
 
 
 def linear_adds_into_y(M: int, K: int, alpha: float) -> bool:

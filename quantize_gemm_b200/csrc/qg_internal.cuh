@@ -408,10 +408,11 @@ struct ActBuffers {
 
 // The layer's fp32 order switch: with at least this many clamped entries per
 // row possible (n - ceil(alpha n) over M), the GEMM writes Y first and the
-// SpMM adds into it (block16k, alpha 0.99: 41 per row, 4 % faster); below it,
-// the SpMM writes Y and the GEMM adds in place (alpha 0.999: 4 per row, the
-// other order is 9 % slower there).
-constexpr int64_t kAddOrderEntriesPerRow = 16;
+// SpMM adds into it; below it, the SpMM writes Y and the GEMM adds its
+// product into it.  Measured on the 7B block's K = 4096 layers at M = 16384:
+// GEMM first is 5-11 % faster at 20 entries per row and 2-6 % at 12, the two
+// are within a few per cent at 8, and SpMM first is 5-11 % faster at 4.
+constexpr int64_t kAddOrderEntriesPerRow = 10;
 
 // QGEMM_NO_COOPERATIVE=1 in the environment (read when a device is first set
 // up) makes the library treat the device as having no cooperative launch, so
