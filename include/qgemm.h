@@ -268,7 +268,8 @@ qg_status qg_fp4_gemm_compensated(const uint8_t* codesA, const float* sA, const 
  *           N not a multiple of 4: qg_fp4_gemm(..., C = Y, Y) in place, the
  *           epilogue reading every sub-tile of C before it writes that
  *           sub-tile of Y); or, when alpha leaves at least 10 clamped entries
- *           per row possible (n - ceil(alpha n) >= 10 M), the other order:
+ *           per row possible for every 4096 of K (n - ceil(alpha n) >=
+ *           10 M K / 4096), the other order:
  *           qg_fp4_gemm(..., C = NULL, Y), then qg_spmm_accumulate;
  *   bf16 Y: the rows in chunks of R (a multiple of 256, R x N x 4 <= 128
  *           MiB, or all of M): qg_spmm_correction of the chunk into an fp32

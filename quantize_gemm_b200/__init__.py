@@ -271,14 +271,14 @@ def qg_spmm_accumulate(csr: CSR, M, W, Y, ws: Workspace, stream=None) -> int:
                                    _ptr(Y), ws.ptr, ws.nbytes, _stream(stream))
 
 
-ADD_ORDER_ENTRIES_PER_ROW = 10   # the layer's order switch (see qg_fp4_linear)
+ADD_ORDER_ENTRIES_PER_4096_K = 10   # the layer's order switch (see qg_fp4_linear)
 
 
 def linear_adds_into_y(M: int, K: int, alpha: float) -> bool:
     """Whether qg_fp4_linear (fp32 Y) runs the GEMM first and adds the
     compensation into Y (True) or writes the compensation first and lets the
     GEMM add in place (False)."""
-    return qg_nnz_capacity(M * K, alpha) >= ADD_ORDER_ENTRIES_PER_ROW * M
+    return qg_nnz_capacity(M * K, alpha) * 4096 >= ADD_ORDER_ENTRIES_PER_4096_K * M * K
 
 
 def qg_fp4_gemm(codesA, sA, codesWT, sW, M, N, K, C, Y, raw_acc, ws: Workspace,

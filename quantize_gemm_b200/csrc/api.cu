@@ -354,15 +354,15 @@ qg_status qg_fp4_linear(const void* A, qg_dtype dtype, int64_t M, int64_t K,
     if (e != cudaSuccess) return QG_ERR_CUDA;
     if (y_dtype == QG_F32) {
         // fp32 Y, no M x N buffer besides Y, in one of two orders with the same
-        // result: with many entries per row (at least kAddOrderEntriesPerRow
-        // possible on average) the GEMM writes the scaled product and the SpMM
+        // result: with many entries per row (linear_gemm_first: at least
+        // kAddOrderEntriesPer4096K possible per 4096 of K) the GEMM writes the scaled product and the SpMM
         // adds the compensation into Y, the SpMM's gathers hiding its reads of
         // Y; otherwise the compensation is written into Y first and the GEMM
         // adds its product into it through the memory system's bulk reduction
         // (or, where the TMA epilogue cannot describe Y, reads each 32 x 32
         // sub-tile of Y as C before it overwrites it in place)
         float* Yf = static_cast<float*>(Y);
-        if (L.cap >= kAddOrderEntriesPerRow * M) {
+        if (linear_gemm_first(L.cap, M, K)) {
             e = launch_fp4_gemm(codes, scales, codesWT, sW, M, N, K, nullptr, Y, QG_F32, nullptr,
                                 status, stream);
             if (e != cudaSuccess) return QG_ERR_CUDA;

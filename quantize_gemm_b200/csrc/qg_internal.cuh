@@ -407,12 +407,20 @@ struct ActBuffers {
 };
 
 // The layer's fp32 order switch: with at least this many clamped entries per
-// row possible (n - ceil(alpha n) over M), the GEMM writes Y first and the
-// SpMM adds into it; below it, the SpMM writes Y and the GEMM adds its
-// product into it.  Measured on the 7B block's K = 4096 layers at M = 16384:
-// GEMM first is 5-11 % faster at 20 entries per row and 2-6 % at 12, the two
-// are within a few per cent at 8, and SpMM first is 5-11 % faster at 4.
-constexpr int64_t kAddOrderEntriesPerRow = 10;
+// row possible for every 4096 of K (n - ceil(alpha n) >= 10 M K / 4096), the
+// GEMM writes Y first and the SpMM adds into it; below it, the SpMM writes Y
+// and the GEMM adds its product into it.  Measured on the 7B block at
+// M = 16384: on the K = 4096 layers GEMM first is 5-11 % faster at 20 entries
+// per row and 2-6 % at 12, the two are within a few per cent at 8, and SpMM
+// first is 5-11 % faster at 4; the K = 11008 layer favours SpMM first up to
+// ~33 per row (the rule puts its switch at 27).  The crossover grows with K
+// because the adding GEMM hides its reads of Y under more MMA work per tile.
+constexpr int64_t kAddOrderEntriesPer4096K = 10;
+
+inline bool linear_gemm_first(int64_t cap, int64_t M, int64_t K)
+{
+    return cap * 4096 >= kAddOrderEntriesPer4096K * M * K;
+}
 
 // QGEMM_NO_COOPERATIVE=1 in the environment (read when a device is first set
 // up) makes the library treat the device as having no cooperative launch, so

@@ -288,13 +288,16 @@ def test_compensated_gemm_host_checks(qg):
 
 def test_layer_order_switch(qg):
     """The layer's fp32 order depends only on the clamped entries possible per
-    row: GEMM first from 10 per row up."""
-    assert qg.linear_adds_into_y(16384, 4096, 0.99)        # 41 per row
-    assert not qg.linear_adds_into_y(16384, 4096, 0.999)   # 4 per row
-    assert not qg.linear_adds_into_y(256, 512, 0.99)       # 5 per row
-    assert qg.linear_adds_into_y(4096, 2048, 0.99)         # 20 per row
-    assert qg.linear_adds_into_y(16384, 4096, 0.997)       # 12 per row
-    assert not qg.linear_adds_into_y(16384, 4096, 0.998)   # 8 per row
+    row against K: GEMM first from 10 per row for every 4096 of K up."""
+    assert qg.linear_adds_into_y(16384, 4096, 0.99)         # 41 per row, switch at 10
+    assert not qg.linear_adds_into_y(16384, 4096, 0.999)    # 4 per row
+    assert qg.linear_adds_into_y(16384, 4096, 0.997)        # 12 per row
+    assert not qg.linear_adds_into_y(16384, 4096, 0.998)    # 8 per row
+    assert not qg.linear_adds_into_y(16384, 11008, 0.999)   # 11 per row, switch at 27
+    assert qg.linear_adds_into_y(16384, 11008, 0.997)       # 33 per row
+    assert qg.linear_adds_into_y(4096, 2048, 0.99)          # 20 per row, switch at 5
+    assert qg.linear_adds_into_y(256, 512, 0.99)            # 5 per row, switch at 1.25
+    assert not qg.linear_adds_into_y(256, 512, 0.999)       # 0.5 per row
     lib = qg._lib
     fake = ctypes.c_void_p(1 << 20)
     csr = qg._Csr(1 << 20, 1 << 20, 1 << 20, 1000, 1 << 20)
