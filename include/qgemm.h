@@ -206,7 +206,8 @@ qg_status qg_spmm_correction(const qg_csr* dA, int64_t M, const void* W, qg_dtyp
                              int64_t K, int64_t N, int64_t ldw, float* C, void* ws,
                              size_t ws_bytes, cudaStream_t stream);
 
-/* The compensation added into an existing fp32 output: Y += dA . W (M x N,
+/* The compensation added into an existing fp32 output ([FP4-writeup],
+ * outlier clamping and compensation paragraph): Y += dA . W (M x N,
  * row pitch N), with each row's sum formed as in qg_spmm_correction (fp32
  * FMA chain in CSR order) and then added to Y by the memory system
  * (red.global.add: fp32 round to nearest; a sum that is subnormal is
@@ -217,7 +218,9 @@ qg_status qg_spmm_accumulate(const qg_csr* dA, int64_t M, const void* W, qg_dtyp
                              int64_t K, int64_t N, int64_t ldw, float* Y, void* ws,
                              size_t ws_bytes, cudaStream_t stream);
 
-/* FP4 GEMM on tcgen05 tensor cores: acc_ij = sum_k e2m1(codesA_ik) *
+/* FP4 GEMM on tcgen05 tensor cores ([FP4-writeup], FP4 GEMM paragraph, with
+ * the row and column scales of the granularity paragraph applied after the
+ * contraction): acc_ij = sum_k e2m1(codesA_ik) *
  * e2m1(codesWT_jk) accumulated in fp32 (exact for K <= 16384), then
  * Y_ij = acc_ij * sA_i * sW_j (+ C_ij when C != NULL), stored as fp32 or bf16
  * (round to nearest even).  raw_acc (nullable, M x N fp32) receives acc itself.
@@ -229,8 +232,9 @@ qg_status qg_fp4_gemm(const uint8_t* codesA, const float* sA, const uint8_t* cod
                       void* Y, qg_dtype y_dtype, float* raw_acc, void* ws, size_t ws_bytes,
                       cudaStream_t stream);
 
-/* The FP4 GEMM's scaled product added into an existing fp32 output:
- * Y_ij += acc_ij * sA_i * sW_j (the product rounded to fp32 as in qg_fp4_gemm,
+/* The FP4 GEMM's scaled product added into an existing fp32 output
+ * ([FP4-writeup], FP4 GEMM paragraph; the sum with the compensation of the
+ * outlier paragraph): Y_ij += acc_ij * sA_i * sW_j (the product rounded to fp32 as in qg_fp4_gemm,
  * then added by the memory system's bulk reduction, fp32 round to nearest).
  * Y: M x N fp32, contiguous, N a multiple of 4 (else
  * QG_ERR_UNSUPPORTED_SHAPE).  With Y holding qg_spmm_correction's output,
@@ -262,7 +266,9 @@ qg_status qg_fp4_gemm_compensated(const uint8_t* codesA, const float* sA, const 
                                   void* Y, qg_dtype y_dtype, void* ws, size_t ws_bytes,
                                   cudaStream_t stream);
 
-/* The whole layer into Y (M x N, fp32 or bf16): qg_quantize_act(A), then
+/* The whole layer into Y (M x N, fp32 or bf16), Y = dequant(Q(A_clamped)
+ * Q(W)) + dA . W ([FP4-writeup], outlier clamping and compensation, FP4
+ * GEMM and granularity paragraphs): qg_quantize_act(A), then
  *   fp32 Y: qg_spmm_correction(dA, W) written into Y itself, then
  *           qg_fp4_gemm_accumulate adding the scaled FP4 product into it (for
  *           N not a multiple of 4: qg_fp4_gemm(..., C = Y, Y) in place, the
@@ -285,7 +291,11 @@ qg_status qg_fp4_gemm_compensated(const uint8_t* codesA, const float* sA, const 
  * in the other dtype is read wrongly without an error).  The activation
  * codes, dA and the bf16 chunk scratch live in the workspace
  * (qg_workspace_size(QG_OP_FP4_LINEAR, ...)); besides Y, no buffer grows past
- * the chunk's 128 MiB with M. */
+ * the chunk's 128 MiB with M.  Errors: QG_ERR_INVALID_ARG (bad dtype or
+ * alpha, a NULL or misaligned pointer), the shape and workspace errors of
+ * qg_quantize_act and qg_fp4_gemm, QG_ERR_UNSUPPORTED_SHAPE when the dA
+ * capacity exceeds INT32_MAX entries, QG_ERR_CUDA; device conditions (NaN or
+ * Inf in A, a bounded wait that ran out) go to the workspace's status word. */
 qg_status qg_fp4_linear(const void* A, qg_dtype dtype, int64_t M, int64_t K,
                         const uint8_t* codesWT, const float* sW, const void* W, int64_t N,
                         double alpha, void* Y, qg_dtype y_dtype, void* ws, size_t ws_bytes,
