@@ -555,6 +555,38 @@ def test_fp4_linear_bf16_chunks(qg, M, K, N, alpha):
 
 
 # ------------------------------------------------------------------ the layer
+@pytest.mark.parametrize("M,K,N,dtype,alpha,gemm_first", [
+    (300, 1024, 1002, torch.bfloat16, 0.99, True),     # N % 4 = 2: direct epilogue, 1-wide adds
+    (300, 1024, 1002, torch.bfloat16, 0.999, False),   # N % 4 = 2: GEMM in place through C = Y
+    (260, 512, 1000, torch.float32, 0.999, False),     # reducing GEMM, fp32 W (slice SpMM)
+    (130, 2048, 516, torch.bfloat16, 0.995, True),     # N % 8 = 4: slice SpMM adding
+    (520, 4096, 2048, torch.bfloat16, 0.998, False),   # 8 per row, switch at 10
+    (520, 4096, 2048, torch.bfloat16, 0.997, True),    # 12 per row
+])
+def test_fp4_linear_fp32_orders(qg, M, K, N, dtype, alpha, gemm_first):
+    """fp32 Y in the order the layer picks for the clamped entries per row
+    against K, with widths that force each epilogue and SpMM form: Y equals
+    bit for bit the separate calls on the layer's own codes and CSR (SpMM into
+    a fresh C, then the GEMM reading C), and the oracle within 1e-3 on every
+    fifth row."""
+    assert qg.linear_adds_into_y(M, K, alpha) == gemm_first
+    A = make_matrix((M, K), ("student_t", 3), seed=M + 7 * K, device="cuda", dtype=dtype)
+    W = make_matrix((K, N), seed=N + 1, device="cuda", dtype=dtype, scale=0.02)
+    codesT, t = qg.quantize_cols(W)
+    dt = qg._dt(A)
+    ws = qg.Workspace(qg.QG_OP_FP4_LINEAR, M, K, N, dt, alpha)
+    Y = qg.fp4_linear(A, codesT, t, W, alpha, ws=ws)
+    qg.check_status(ws, "layer")
+    parts = qg.linear_parts(ws, M, K, N, dt, alpha)
+    C = qg.spmm_correction(parts["csr"], M, W)
+    Y2 = qg.fp4_gemm(parts["codes"], parts["scales"], codesT, t, K, C=C)
+    torch.cuda.synchronize()
+    assert torch.equal(Y, Y2)
+    rows = np.arange(0, M, 5)
+    Yo, _ = _linear_oracle(A, W, alpha, rows=rows)
+    assert y_rel_err(_np(Y)[rows], Yo) <= 1e-3
+
+
 def _linear_oracle(A, W, alpha, rows=None):
     act = oracle.quantize_act(A.cpu(), alpha)
     oT, ot = oracle.quantize_cols(W.cpu())
