@@ -277,8 +277,10 @@ qg_status qg_fp4_gemm_compensated(const uint8_t* codesA, const float* sA, const 
  *           per row possible for every 4096 of K (n - ceil(alpha n) >=
  *           10 M K / 4096), the other order:
  *           qg_fp4_gemm(..., C = NULL, Y), then qg_spmm_accumulate;
- *   bf16 Y: the rows in chunks of R (a multiple of 256, R x N x 4 <= 128
- *           MiB, or all of M): qg_spmm_correction of the chunk into an fp32
+ *   bf16 Y: the rows in chunks of R (the largest multiple of 256 with
+ *           R x N x 4 <= 128 MiB, but at least 256 -- more bytes only when
+ *           N > 131072 -- and at most M): qg_spmm_correction of the chunk
+ *           into an fp32
  *           scratch of R x N in the workspace, then qg_fp4_gemm(..., C =
  *           scratch, the chunk of Y) -- the same bytes as
  *           qg_fp4_gemm_compensated, which computes the compensation inside
@@ -290,8 +292,8 @@ qg_status qg_fp4_gemm_compensated(const uint8_t* codesA, const float* sA, const 
  * (`dtype` describes both; the call has no separate weight dtype, so a weight
  * in the other dtype is read wrongly without an error).  The activation
  * codes, dA and the bf16 chunk scratch live in the workspace
- * (qg_workspace_size(QG_OP_FP4_LINEAR, ...)); besides Y, no buffer grows past
- * the chunk's 128 MiB with M.  Errors: QG_ERR_INVALID_ARG (bad dtype or
+ * (qg_workspace_size(QG_OP_FP4_LINEAR, ...)); besides Y, the activation codes
+ * and dA, no buffer grows with M: the chunk stays at its R rows.  Errors: QG_ERR_INVALID_ARG (bad dtype or
  * alpha, a NULL or misaligned pointer), the shape and workspace errors of
  * qg_quantize_act and qg_fp4_gemm, QG_ERR_UNSUPPORTED_SHAPE when the dA
  * capacity exceeds INT32_MAX entries, QG_ERR_CUDA; device conditions (NaN or
