@@ -109,3 +109,21 @@ def test_cpu_baseline_is_bounded_and_labelled(monkeypatch):
     assert out["kind"] == "oracle" and out["cores"] >= 1 and out["value"] > 0
     assert 0 < out["sample_fraction"] < 1 and "fraction" in out["sample"]
     assert out["sample_wall_s"] < 60
+
+
+def test_layer_order_follows_the_library_switch():
+    """The bench times each layer's two kernels in the order qg_fp4_linear
+    picks: at the 7B block's size, GEMM first at alpha 0.99 (41 and 110
+    clamped entries per row possible) and SpMM first at 0.999 (4 and 11, below
+    the switch of 10 per 4096 of K) on every layer."""
+    from types import SimpleNamespace
+    import quantize_gemm_b200 as qg
+    wl = WORKLOADS["block16k"]
+    for a in wl.alphas:
+        for lay in wl.layers:
+            L = SimpleNamespace(M=wl.M, K=lay.K, N=lay.N, alpha=a)
+            order = bench.layer_order(qg, L)
+            assert order[:2] == ("quantize_cols", "quantize_act")
+            assert sorted(order[2:]) == ["fp4_gemm", "spmm"]
+            assert (order[2] == "fp4_gemm") == qg.linear_adds_into_y(wl.M, lay.K, a)
+            assert (order[2] == "fp4_gemm") == (a == 0.99)
