@@ -480,12 +480,9 @@ def our_arm(args, rank, world, device):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_per_step, 4),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "e2m1",
         "data": "synthetic",
-        "config": {"workload": wl.name if args.layer is None else f"{wl.name}:{layers[0].name}",
-                   "description": wl.description, "M": wl.M,
-                   "layers": [[L.name, L.K, L.N] for L in layers], "alpha": head["alpha"],
-                   "input_dtype": wl.dtype, "y_dtype": "f32",
-                   "l2": "flushed (256 MiB write between timed steps)",
-                   "parallelism": f"replicas x{world}"},
+        "config": dict(workload_config(wl, layers, head["alpha"], args.layer is not None),
+                       l2="flushed (256 MiB write between timed steps)",
+                       parallelism=f"replicas x{world}"),
         "tokens_per_s": round(weak_scaling_value(tokens_step, args.steps, total_ms, world), 1),
         "quantizer_gbs": rows["quantize_act"]["achieved"],
         "kernels": rows,
@@ -703,6 +700,15 @@ def cpu_baseline(args, wl, layers):
             "seconds_per_step_estimate": round(t_est, 3)}
 
 
+def workload_config(wl, layers, alpha, one_layer=False):
+    """The `config` keys both arms share: the workload, its shapes, alpha and
+    the input and output dtypes."""
+    return {"workload": f"{wl.name}:{layers[0].name}" if one_layer else wl.name,
+            "description": wl.description, "M": wl.M,
+            "layers": [[L.name, L.K, L.N] for L in layers], "alpha": alpha,
+            "input_dtype": wl.dtype, "y_dtype": "f32"}
+
+
 REFERENCE_BUDGET_S = 150.0   # wall time the reference arm's warm-up + timed steps aim for
 
 
@@ -754,9 +760,10 @@ def reference_arm(args, rank, world):
                              if frac < 1 else "measured quantizers; Y rows sampled and scaled"),
         "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": wl.name if args.layer is None else f"{wl.name}:{wl.layers[idx[0]].name}",
-                   "M": wl.M, "layers": [[wl.layers[i].name, wl.layers[i].K, wl.layers[i].N] for i in idx],
-                   "alpha": wl.alphas[0] if args.alpha is None else args.alpha},
+        "config": dict(workload_config(wl, [wl.layers[i] for i in idx],
+                                       wl.alphas[0] if args.alpha is None else args.alpha,
+                                       args.layer is not None),
+                       parallelism="rank 0 only, on the host cores"),
         "cpu_baseline": {"kind": "oracle", "cores": cores, "sample": sample,
                          "value": round(value, 6), "unit": "TFLOP/s"},
         "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0,

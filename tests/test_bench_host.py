@@ -90,6 +90,11 @@ def test_reference_arm_line_and_bounded_sample(monkeypatch, budget):
     assert line["value"] > 0 and line["e2e"]["value"] == line["value"]
     assert line["e2e"]["h2d_bytes_per_step"] == 0 and line["e2e"]["d2h_bytes_per_step"] == 0
     assert line["cpu_baseline"]["kind"] == "oracle" and line["cpu_baseline"]["cores"] >= 1
+    # the same workload description as the GPU arm's line
+    args = _ref_args(steps=4, warmup=3)
+    wl = WORKLOADS[args.workload]
+    shared = bench.workload_config(wl, list(wl.layers), wl.alphas[0])
+    assert {k: line["config"][k] for k in shared} == shared
     sample = line["cpu_baseline"]["sample"]
     if budget < 1:
         assert "fraction" in sample
